@@ -1,0 +1,401 @@
+/*
+ * gnf4_oracle.c -- CPU oracle for the grouped 4-bit MoE expert GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, obviously
+ * correct statement of what the GPU library computes.  Only the test suite,
+ * the smoke check and the benchmark's CPU-baseline leg may load it.  It
+ * shares no code, header, table or constant generator with the CUDA path.
+ *
+ * Precision: quantise / dequantise in fp32 exactly as the formats define
+ * them; every sum (GEMM, combine) is accumulated in fp64.
+ *
+ * Sources (page title, section):
+ *   [README]   grouped-nf4-gemm 0.33.1 on PyPI, opening paragraphs ("LUT decode
+ *              to fp32 in registers, blockwise scaling, fp32 accumulation, bf16
+ *              epilogue") and "Try it on CPU right now", examples 1 and 2
+ *              (NF4 [N,K] -> [N,K/2] u8 + [N,K/64] fp32; MXFP4 [..,K] ->
+ *              [..,K/32,16] u8 + [..,K/32] u8 e8m0).
+ *   [PATCH]    grouped-nf4-gemm releases, v0.2.6 "The patch point" (argsort of
+ *              the top-k ids, gather x[idxs // k], tokens_per_expert = sizes;
+ *              weighting and unsorting stay with the caller).
+ *   [ARENA]    grouped-nf4-gemm releases, v0.2.5 "arena -> kernel" (expert
+ *              stacks [E,N,K//2] blocks + [E,N,K//32] e8m0 scales).
+ *   [QLORA]    The NF4 codebook itself is not printed on the pages; the values
+ *              are the NormalFloat-4 table of Dettmers et al., "QLoRA", 2023,
+ *              appendix (reading C1).
+ *   [OCP-MX]   OCP Microscaling Formats (MX) v1.0: e2m1 element, e8m0 scale,
+ *              shared exponent floor(log2(amax)) - emax_elem (reading C8).
+ *
+ * Readings of points the pages leave open are listed in the design doc under
+ * "Readings"; each function below names the ones it depends on.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ */
+/* Threads                                                             */
+/* ------------------------------------------------------------------ */
+static int g_threads = 1;
+
+void orc_set_threads(int n) { g_threads = n < 1 ? 1 : n; }
+int orc_get_threads(void) { return g_threads; }
+
+/* ------------------------------------------------------------------ */
+/* Tables                                                              */
+/* ------------------------------------------------------------------ */
+
+/* NF4: 16 NormalFloat values, index 0 = -1, index 7 = exact zero,
+ * index 15 = +1 [QLORA]. */
+static const float NF4_VALUES[16] = {
+    -1.0f,
+    -0.6961928009986877f,
+    -0.5250730514526367f,
+    -0.39491748809814453f,
+    -0.28444138169288635f,
+    -0.18477343022823334f,
+    -0.09105003625154495f,
+    0.0f,
+    0.07958029955625534f,
+    0.16093020141124725f,
+    0.24611230194568634f,
+    0.33791524171829224f,
+    0.44070982933044434f,
+    0.5626170039176941f,
+    0.7229568362236023f,
+    1.0f,
+};
+
+/* e2m1 magnitudes for the three low bits; bit 3 is the sign [OCP-MX]. */
+static const float E2M1_MAGNITUDE[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+void orc_nf4_values(float out[16]) { memcpy(out, NF4_VALUES, sizeof(NF4_VALUES)); }
+
+/* Value of a 4-bit e2m1 code: sign = bit 3, magnitude = bits 2..0.  Code 8
+ * is negative zero (reading C6). */
+static float e2m1_value(unsigned code)
+{
+    float m = E2M1_MAGNITUDE[code & 7u];
+    return (code & 8u) ? -m : m;
+}
+
+void orc_e2m1_values(float out[16])
+{
+    for (unsigned c = 0; c < 16; ++c) out[c] = e2m1_value(c);
+}
+
+/* e8m0 scale 2^(e-127); e = 255 is NaN; e = 0 gives the fp32 subnormal
+ * 2^-127 (reading C7). */
+static float e8m0_value(unsigned e)
+{
+    if (e == 255u) return NAN;
+    return ldexpf(1.0f, (int)e - 127);
+}
+
+float orc_e8m0_value(int e) { return e8m0_value((unsigned)e & 255u); }
+
+/* bf16 bit pattern -> float (exact: bf16 is the top half of an fp32). */
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* ------------------------------------------------------------------ */
+/* NF4 (bitsandbytes gemm_4bit layout) [README example 1]              */
+/* ------------------------------------------------------------------ */
+
+/* Index of the codebook value nearest to x; an exact tie goes to the lower
+ * index (reading C4). */
+static unsigned nf4_nearest(float x)
+{
+    unsigned best = 0;
+    float bestd = fabsf(x - NF4_VALUES[0]);
+    for (unsigned i = 1; i < 16; ++i) {
+        float d = fabsf(x - NF4_VALUES[i]);
+        if (d < bestd) {
+            bestd = d;
+            best = i;
+        }
+    }
+    return best;
+}
+
+/* Quantise rows x K fp32 weights (row-major) into packed [rows, K/2] bytes
+ * and absmax [rows, K/64] fp32.  Blocks are 64 consecutive elements of a row
+ * (reading C3).  Within a byte, element 2i sits in the high nibble and
+ * element 2i+1 in the low nibble (reading C2).  Requires K % 64 == 0. */
+void orc_quant_nf4(const float *w, int64_t rows, int64_t K, uint8_t *packed, float *absmax)
+{
+    const int64_t nb = K / 64;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const float *blk = w + r * K + b * 64;
+            float amax = 0.0f;
+            for (int i = 0; i < 64; ++i) {
+                float a = fabsf(blk[i]);
+                if (a > amax) amax = a;
+            }
+            absmax[r * nb + b] = amax;
+            uint8_t *dst = packed + r * (K / 2) + b * 32;
+            for (int i = 0; i < 32; ++i) {
+                unsigned c0, c1;
+                if (amax == 0.0f) {
+                    c0 = c1 = 7u; /* the exact zero of the codebook */
+                } else {
+                    c0 = nf4_nearest(blk[2 * i] / amax);
+                    c1 = nf4_nearest(blk[2 * i + 1] / amax);
+                }
+                dst[i] = (uint8_t)((c0 << 4) | c1);
+            }
+        }
+    }
+}
+
+/* Decode: value = NF4_VALUES[code] * absmax, one fp32 multiply. */
+void orc_dequant_nf4(const uint8_t *packed, const float *absmax, int64_t rows, int64_t K, float *out)
+{
+    const int64_t nb = K / 64;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = packed[r * (K / 2) + k / 2];
+            unsigned code = (k % 2 == 0) ? (byte >> 4) : (byte & 15u);
+            out[r * K + k] = NF4_VALUES[code] * absmax[r * nb + k / 64];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* MXFP4 (OCP e2m1 + e8m0 per 32) [README example 2], [ARENA]          */
+/* ------------------------------------------------------------------ */
+
+/* Round a non-negative magnitude (already divided by the block scale) to
+ * the nearest e2m1 magnitude index; ties go to the even index (round to
+ * nearest even on the e2m1 mantissa); values above 6 saturate [OCP-MX]. */
+static unsigned e2m1_round_magnitude(float m)
+{
+    if (!(m < 6.0f)) return 7u;
+    unsigned best = 0;
+    float bestd = fabsf(m - E2M1_MAGNITUDE[0]);
+    for (unsigned i = 1; i < 8; ++i) {
+        float d = fabsf(m - E2M1_MAGNITUDE[i]);
+        if (d < bestd || (d == bestd && (i % 2u) == 0u)) {
+            bestd = d;
+            best = i;
+        }
+    }
+    return best;
+}
+
+/* Quantise rows x K fp32 into blocks [rows, K/2] (element 2i in the LOW
+ * nibble, reading C5) and scales [rows, K/32] e8m0.  Shared exponent of a
+ * block = floor(log2(amax)) - 2 (e2m1's largest exponent is 2), clamped to
+ * the e8m0 range; an all-zero block gets scale byte 0 and zero codes
+ * (reading C8).  Requires K % 32 == 0. */
+void orc_quant_mxfp4(const float *w, int64_t rows, int64_t K, uint8_t *blocks, uint8_t *scales)
+{
+    const int64_t nb = K / 32;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const float *blk = w + r * K + b * 32;
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float a = fabsf(blk[i]);
+                if (a > amax) amax = a;
+            }
+            int sexp;
+            if (amax == 0.0f) {
+                sexp = -127;
+            } else {
+                int ex;
+                frexpf(amax, &ex); /* amax = m * 2^ex, m in [0.5, 1) */
+                sexp = (ex - 1) - 2;
+                if (sexp < -127) sexp = -127;
+                if (sexp > 127) sexp = 127;
+            }
+            scales[r * nb + b] = (uint8_t)(sexp + 127);
+            float s = ldexpf(1.0f, sexp);
+            uint8_t *dst = blocks + r * (K / 2) + b * 16;
+            for (int i = 0; i < 16; ++i) {
+                unsigned code[2];
+                for (int h = 0; h < 2; ++h) {
+                    float x = blk[2 * i + h];
+                    unsigned mag = (amax == 0.0f) ? 0u : e2m1_round_magnitude(fabsf(x) / s);
+                    code[h] = mag | (signbit(x) ? 8u : 0u);
+                }
+                dst[i] = (uint8_t)(code[0] | (code[1] << 4));
+            }
+        }
+    }
+}
+
+/* Decode: value = e2m1(code) * 2^(e-127), one fp32 multiply. */
+void orc_dequant_mxfp4(const uint8_t *blocks, const uint8_t *scales, int64_t rows, int64_t K, float *out)
+{
+    const int64_t nb = K / 32;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = blocks[r * (K / 2) + k / 2];
+            unsigned code = (k % 2 == 0) ? (byte & 15u) : (byte >> 4);
+            out[r * K + k] = e2m1_value(code) * e8m0_value(scales[r * nb + k / 32]);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Routing [PATCH]                                                     */
+/* ------------------------------------------------------------------ */
+
+/* Stable counting sort of the M = T*k (token, slot) pairs by expert id.
+ * Pair f = t*k + j.  Outputs:
+ *   offsets[E+1]      offsets[e] = first sorted row of expert e,
+ *                     offsets[E] = number of valid pairs;
+ *   sorted_to_flat[M] pair index of each sorted row, -1 past offsets[E];
+ *   flat_to_sorted[M] sorted row of each pair, -1 for a dropped pair.
+ * Within an expert, pairs keep ascending f (reading C11).  Ids outside
+ * [0, E) are counted into *bad and dropped (reading C16).
+ * Returns 0. */
+int orc_route(const int32_t *topk_ids, int64_t T, int64_t k, int64_t E, int32_t *offsets,
+              int32_t *sorted_to_flat, int32_t *flat_to_sorted, int64_t *bad)
+{
+    const int64_t M = T * k;
+    int64_t *count = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    int64_t *cursor = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    int64_t nbad = 0;
+    for (int64_t f = 0; f < M; ++f) {
+        int32_t e = topk_ids[f];
+        if (e >= 0 && e < E)
+            count[e] += 1;
+        else
+            nbad += 1;
+    }
+    offsets[0] = 0;
+    for (int64_t e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + (int32_t)count[e];
+    for (int64_t e = 0; e < E; ++e) cursor[e] = offsets[e];
+    for (int64_t f = 0; f < M; ++f) {
+        int32_t e = topk_ids[f];
+        if (e >= 0 && e < E) {
+            int64_t p = cursor[e]++;
+            sorted_to_flat[p] = (int32_t)f;
+            flat_to_sorted[f] = (int32_t)p;
+        } else {
+            flat_to_sorted[f] = -1;
+        }
+    }
+    for (int64_t p = offsets[E]; p < M; ++p) sorted_to_flat[p] = -1;
+    *bad = nbad;
+    free(count);
+    free(cursor);
+    return 0;
+}
+
+/* x_sorted[p] = x[sorted_to_flat[p] / k] for p < offsets[E]; later rows are
+ * zero.  Rows are K bf16 values moved as raw 16-bit patterns. */
+void orc_gather(const uint16_t *x, int64_t K, int64_t k, const int32_t *sorted_to_flat, int64_t M,
+                int64_t n_valid, uint16_t *x_sorted)
+{
+    for (int64_t p = 0; p < M; ++p) {
+        if (p < n_valid) {
+            int64_t t = sorted_to_flat[p] / k;
+            memcpy(x_sorted + p * K, x + t * K, (size_t)K * 2);
+        } else {
+            memset(x_sorted + p * K, 0, (size_t)K * 2);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Grouped GEMM [README], [ARENA]                                      */
+/* ------------------------------------------------------------------ */
+
+/* For every requested sorted row r (rows[i], i < n_rows) of expert e, where
+ * offsets[e] <= r < offsets[e+1]:
+ *     y[i, n] = sum_k A[r, k] * W_e[n, k]        (fp64 accumulation)
+ * with W_e the fp32 dequantised weights of expert e, stored [N, K] (both
+ * operands K-major, reading C9).  fmt 0 = NF4 (scales = absmax fp32
+ * [E,N,K/64]), fmt 1 = MXFP4 (scales = e8m0 bytes [E,N,K/32]).  Rows outside
+ * [0, offsets[E]) give NaN.  Each expert is dequantised only if one of its
+ * rows is requested. */
+static void grouped_gemm(int fmt, const uint16_t *a, const uint8_t *w, const void *scales,
+                         const int32_t *offsets, int64_t E, int64_t N, int64_t K, const int64_t *rows,
+                         int64_t n_rows, double *y)
+{
+    float *wd = (float *)malloc((size_t)(N * K) * sizeof(float));
+    int64_t *owner = (int64_t *)malloc((size_t)(n_rows > 0 ? n_rows : 1) * sizeof(int64_t));
+    for (int64_t i = 0; i < n_rows; ++i) {
+        owner[i] = -1;
+        for (int64_t e = 0; e < E; ++e)
+            if (rows[i] >= offsets[e] && rows[i] < offsets[e + 1]) owner[i] = e;
+        if (owner[i] < 0)
+            for (int64_t n = 0; n < N; ++n) y[i * N + n] = NAN;
+    }
+    for (int64_t e = 0; e < E; ++e) {
+        int used = 0;
+        for (int64_t i = 0; i < n_rows; ++i)
+            if (owner[i] == e) used = 1;
+        if (!used) continue;
+        if (fmt == 0)
+            orc_dequant_nf4(w + e * N * (K / 2), (const float *)scales + e * N * (K / 64), N, K, wd);
+        else
+            orc_dequant_mxfp4(w + e * N * (K / 2), (const uint8_t *)scales + e * N * (K / 32), N, K, wd);
+        for (int64_t i = 0; i < n_rows; ++i) {
+            if (owner[i] != e) continue;
+            const uint16_t *arow = a + rows[i] * K;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+            for (int64_t n = 0; n < N; ++n) {
+                const float *wrow = wd + n * K;
+                double acc = 0.0;
+                for (int64_t kk = 0; kk < K; ++kk) acc += (double)bf16_to_float(arow[kk]) * (double)wrow[kk];
+                y[i * N + n] = acc;
+            }
+        }
+    }
+    free(owner);
+    free(wd);
+}
+
+void orc_grouped_gemm_nf4(const uint16_t *a, const uint8_t *w, const float *absmax, const int32_t *offsets,
+                          int64_t E, int64_t N, int64_t K, const int64_t *rows, int64_t n_rows, double *y)
+{
+    grouped_gemm(0, a, w, absmax, offsets, E, N, K, rows, n_rows, y);
+}
+
+void orc_grouped_gemm_mxfp4(const uint16_t *a, const uint8_t *w, const uint8_t *scales, const int32_t *offsets,
+                            int64_t E, int64_t N, int64_t K, const int64_t *rows, int64_t n_rows, double *y)
+{
+    grouped_gemm(1, a, w, scales, offsets, E, N, K, rows, n_rows, y);
+}
+
+/* ------------------------------------------------------------------ */
+/* Top-k combine (the caller's "weighting, unsorting") [PATCH]         */
+/* ------------------------------------------------------------------ */
+
+/* out[t, n] = sum_{j<k} weights[t, j] * Y[flat_to_sorted[t*k + j], n] in
+ * fp64, j ascending; pairs with flat_to_sorted = -1 contribute nothing.
+ * Y holds bf16 patterns. */
+void orc_combine(const uint16_t *y, const int32_t *flat_to_sorted, const float *weights, int64_t T, int64_t k,
+                 int64_t N, double *out)
+{
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < k; ++j) {
+                int32_t p = flat_to_sorted[t * k + j];
+                if (p < 0) continue;
+                acc += (double)weights[t * k + j] * (double)bf16_to_float(y[(int64_t)p * N + n]);
+            }
+            out[t * N + n] = acc;
+        }
+    }
+}

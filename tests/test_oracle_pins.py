@@ -1,0 +1,369 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics
+fix, never against the oracle's own formulas retyped.
+
+Each check is chosen so that a plausible slip in the oracle fails it: a wrong
+codebook entry or nibble order (byte examples, quantile construction, pack
+identity), a wrong scale (e8m0 closed form), a dropped or misplaced term in
+the GEMM (closed forms, one-hot weights, numpy's matmul on E=1, brute force),
+a wrong expert index (per-expert power-of-two weights), an unstable or lossy
+routing sort (brute force by Python's sorted), and a wrong combine weight or
+index (one-hot weights, brute force with math.fsum).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from bit_grouped_moe_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- formats
+
+
+def test_nf4_codebook_structure():
+    v = oracle.nf4_values().astype(np.float64)
+    assert v.shape == (16,)
+    assert np.all(np.diff(v) > 0), "codebook must be strictly increasing"
+    assert v[0] == -1.0 and v[15] == 1.0
+    assert v[7] == 0.0 and np.count_nonzero(v == 0.0) == 1
+    assert np.count_nonzero(v < 0) == 7 and np.count_nonzero(v > 0) == 8
+
+
+def test_nf4_codebook_matches_quantile_construction():
+    """Rebuild the NormalFloat table from N(0,1) quantiles (QLoRA's
+    construction) with scipy and compare to the stored constants."""
+    from scipy.stats import norm
+
+    g = _golden("formats.json")
+    off = g["nf4_quantile_offset"]
+    pos = norm.ppf(np.linspace(off, 0.5, 9)[:-1])
+    neg = -norm.ppf(np.linspace(off, 0.5, 8)[:-1])
+    v = np.sort(np.concatenate([pos, [0.0], neg]))
+    v = v / np.abs(v).max()
+    got = oracle.nf4_values().astype(np.float64)
+    assert np.max(np.abs(got - v)) <= g["nf4_quantile_tolerance"]
+
+
+def test_e2m1_table():
+    g = _golden("formats.json")
+    t = oracle.e2m1_values()
+    mags = np.array(g["e2m1_magnitudes"], np.float32)
+    assert np.array_equal(np.abs(t[:8]), mags) and np.all(np.signbit(t[:8]) == False)  # noqa: E712
+    assert np.array_equal(np.abs(t[8:]), mags) and np.all(np.signbit(t[8:]))
+    assert t[8] == 0.0 and np.signbit(t[8]), "code 8 is negative zero"
+
+
+def test_e8m0_closed_form():
+    for e in range(1, 255):
+        assert oracle.e8m0_value(e) == math.ldexp(1.0, e - 127)
+    assert oracle.e8m0_value(0) == math.ldexp(1.0, -127) > 0.0  # fp32 subnormal, not flushed
+    assert math.isnan(oracle.e8m0_value(255))
+
+
+def test_byte_examples_pin_nibble_order():
+    g = _golden("formats.json")
+    for ex in g["nf4_byte_examples"]:
+        packed = np.array([[ex["byte"]] * 32], np.uint8)
+        absmax = np.array([[ex["absmax"]]], np.float32)
+        out = oracle.dequant_nf4(packed, absmax)
+        assert out[0, 0] == ex["values"][0] and out[0, 1] == ex["values"][1]
+    for ex in g["mxfp4_byte_examples"]:
+        blocks = np.array([[ex["byte"]] * 16], np.uint8)
+        scales = np.array([[ex["scale"]]], np.uint8)
+        out = oracle.dequant_mxfp4(blocks, scales)
+        assert out[0, 0] == ex["values"][0] and out[0, 1] == ex["values"][1]
+
+
+def _codes_from_values(vals, table):
+    """Map decoded values back to code indices by exact match (bit pattern)."""
+    tb = table.view(np.uint32)
+    vb = vals.astype(np.float32).view(np.uint32)
+    idx = np.full(vals.shape, -1, np.int64)
+    for i, b in enumerate(tb):
+        idx[vb == b] = i
+    return idx
+
+
+def test_pack_unpack_identity_nf4():
+    g = inputs.rng(1)
+    packed = g.integers(0, 256, size=(7, 64), dtype=np.uint8)  # K = 128
+    absmax = np.ones((7, 2), np.float32)
+    vals = oracle.dequant_nf4(packed, absmax)
+    codes = _codes_from_values(vals, oracle.nf4_values())
+    assert np.all(codes >= 0)
+    hi = (packed >> 4).astype(np.int64)
+    lo = (packed & 15).astype(np.int64)
+    assert np.array_equal(codes[:, 0::2], hi) and np.array_equal(codes[:, 1::2], lo)
+    # and quantising the decoded values gives the same bytes back
+    p2, a2 = oracle.quant_nf4(vals)
+    # blocks that lack a +-1 code renormalise; compare only blocks holding one
+    full = np.array([[np.any((c == 0) | (c == 15)) for c in np.split(row, 2)] for row in codes])
+    for r in range(7):
+        for b in range(2):
+            if full[r, b] and a2[r, b] == 1.0:
+                assert np.array_equal(p2[r, 32 * b:32 * b + 32], packed[r, 32 * b:32 * b + 32])
+
+
+def test_pack_unpack_identity_mxfp4():
+    g = inputs.rng(2)
+    blocks = g.integers(0, 256, size=(5, 48), dtype=np.uint8)  # K = 96
+    scales = np.full((5, 3), 127, np.uint8)
+    vals = oracle.dequant_mxfp4(blocks, scales)
+    codes = _codes_from_values(vals, oracle.e2m1_values())
+    assert np.all(codes >= 0)
+    assert np.array_equal(codes[:, 0::2], blocks & 15) and np.array_equal(codes[:, 1::2], blocks >> 4)
+
+
+def test_pages_roundtrip_nf4():
+    g = _golden("pages_roundtrip.json")["nf4"]
+    w = inputs.rng(0).standard_normal(g["weight_shape"], dtype=np.float32)
+    packed, absmax = oracle.quant_nf4(w)
+    assert list(packed.shape) == g["packed_shape"] and packed.dtype == np.uint8
+    assert list(absmax.shape) == g["absmax_shape"] and absmax.dtype == np.float32
+    wq = oracle.dequant_nf4(packed, absmax)
+    rel = np.linalg.norm(wq - w) / np.linalg.norm(w)
+    lo, hi = g["rel_err_band"]
+    assert lo <= rel <= hi, rel
+    p2, a2 = oracle.quant_nf4(wq)
+    assert np.array_equal(p2, packed) == g["repack_idempotent"]
+    assert np.array_equal(a2, absmax)
+
+
+def test_pages_roundtrip_mxfp4():
+    g = _golden("pages_roundtrip.json")["mxfp4"]
+    w = inputs.rng(0).standard_normal(g["weight_shape"], dtype=np.float32)
+    blocks, scales = oracle.quant_mxfp4(w)
+    assert blocks.size == int(np.prod(g["blocks_shape_pages"]))
+    assert blocks.reshape(g["blocks_shape_pages"]).shape == tuple(g["blocks_shape_pages"])
+    assert list(scales.shape) == g["scales_shape"]
+    wq = oracle.dequant_mxfp4(blocks, scales)
+    rel = np.linalg.norm(wq - w) / np.linalg.norm(w)
+    lo, hi = g["rel_err_band"]
+    assert lo <= rel <= hi, rel
+
+
+def test_mxfp4_quantiser_is_ocp_rounding():
+    """Values exactly on the e2m1 grid survive; midpoints round to even codes;
+    values beyond 6*scale saturate."""
+    row = np.zeros(32, np.float32)
+    row[:8] = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    row[8:14] = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5]
+    row[14] = 5.0
+    row[15] = -7.0  # amax 7 -> shared exponent floor(log2 7) - 2 = 0 -> saturates to -6
+    b, s = oracle.quant_mxfp4(row[None, :])
+    assert s[0, 0] == 127
+    out = oracle.dequant_mxfp4(b, s)[0]
+    assert np.array_equal(out[:8], row[:8])
+    assert np.array_equal(out[8:14], np.array([0.0, 1.0, 1.0, 2.0, 2.0, 4.0], np.float32))
+    assert out[14] == 4.0 and out[15] == -6.0
+
+
+# ---------------------------------------------------------------- routing
+
+
+def _brute_route(ids, E):
+    pairs = [(int(e), f) for f, e in enumerate(ids.reshape(-1)) if 0 <= e < E]
+    pairs.sort()
+    offsets = [0] * (E + 1)
+    for e, _ in pairs:
+        offsets[e + 1] += 1
+    for e in range(E):
+        offsets[e + 1] += offsets[e]
+    return np.array(offsets, np.int32), np.array([f for _, f in pairs], np.int32)
+
+
+@pytest.mark.parametrize("T,k,E", [(16, 2, 8), (37, 4, 128), (5, 8, 64), (1, 1, 1), (0, 2, 4)])
+def test_route_matches_brute_force(T, k, E):
+    g = inputs.rng(T * 31 + k)
+    ids = g.integers(0, E, size=(T, k)).astype(np.int32)
+    offsets, s2f, f2s, bad = oracle.route(ids, E)
+    bo, bs = _brute_route(ids, E)
+    assert bad == 0
+    assert np.array_equal(offsets, bo)
+    assert np.array_equal(s2f, bs)
+    M = T * k
+    assert np.array_equal(np.sort(s2f), np.arange(M))  # bijection
+    assert np.array_equal(s2f[f2s], np.arange(M))
+    assert np.array_equal(np.diff(offsets), np.bincount(ids.reshape(-1), minlength=E))
+
+
+def test_route_drops_bad_ids_near_boundary():
+    E = 16
+    ids = np.array([[15, 16], [-1, 14], [15, 0], [2**30, 15]], np.int32)
+    offsets, s2f, f2s, bad = oracle.route(ids, E)
+    assert bad == 3
+    assert offsets[E] == 5
+    assert list(f2s[[1, 2, 6]]) == [-1, -1, -1]
+    # expert 15 rows keep ascending flat order 0, 4, 7
+    assert list(s2f[offsets[15]:offsets[16]]) == [0, 4, 7]
+    assert list(s2f[offsets[E]:]) == [-1, -1, -1]
+
+
+def test_gather_rows():
+    g = inputs.rng(3)
+    T, k, E, K = 9, 3, 5, 24
+    ids = inputs.route_uniform(g, T, k, E)[0]
+    x = inputs.bf16_normal(g, (T, K))
+    offsets, s2f, f2s, bad = oracle.route(ids, E)
+    xs = oracle.gather(x, k, s2f, int(offsets[E]))
+    for p in range(T * k):
+        assert np.array_equal(xs[p], x[s2f[p] // k])
+
+
+# ---------------------------------------------------------------- GEMM
+
+
+def _af(bits):
+    return inputs.bf16_bits_to_float(bits).astype(np.float64)
+
+
+def test_gemm_closed_form_row_sums_mxfp4():
+    """All codes 0b0010 (= 1.0) and scale 127: Y[r, n] = sum_k A[r, k]."""
+    g = inputs.rng(4)
+    E, N, K, M = 3, 8, 96, 10
+    a = inputs.bf16_normal(g, (M, K))
+    w = np.full((E, N, K // 2), 0x22, np.uint8)
+    s = np.full((E, N, K // 32), 127, np.uint8)
+    offsets = np.array([0, 4, 4, M], np.int32)
+    y = oracle.grouped_gemm_mxfp4(a, w, s, offsets)
+    for r in range(M):
+        assert np.all(y[r] == math.fsum(_af(a[r])))
+
+
+def test_gemm_selects_expert_by_offsets():
+    """Expert e's weights are 2^e: a wrong group index changes the power."""
+    g = inputs.rng(5)
+    E, N, K = 4, 16, 64
+    counts = [3, 0, 5, 2]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    M = int(offsets[-1])
+    a = inputs.bf16_normal(g, (M, K))
+    w = np.full((E, N, K // 2), 0x22, np.uint8)
+    s = np.stack([np.full((N, K // 32), 127 + e, np.uint8) for e in range(E)])
+    y = oracle.grouped_gemm_mxfp4(a, w, s, offsets)
+    for e in range(E):
+        for r in range(offsets[e], offsets[e + 1]):
+            assert np.all(y[r] == (2.0 ** e) * math.fsum(_af(a[r])))
+
+
+def test_gemm_one_hot_weights_nf4():
+    """Codes all 7 (zero) except one +1 per row at column pi(n): Y = A[:, pi]."""
+    g = inputs.rng(6)
+    E, N, K, M = 2, 32, 128, 7
+    pi = g.integers(0, K, size=(E, N))
+    codes = np.full((E, N, K), 7, np.uint8)
+    for e in range(E):
+        codes[e, np.arange(N), pi[e]] = 15
+    packed = ((codes[..., 0::2] << 4) | codes[..., 1::2]).astype(np.uint8)
+    absmax = np.ones((E, N, K // 64), np.float32)
+    a = inputs.bf16_normal(g, (M, K))
+    offsets = np.array([0, 3, M], np.int32)
+    y = oracle.grouped_gemm_nf4(a, packed, absmax, offsets)
+    af = _af(a)
+    for r in range(M):
+        e = 0 if r < 3 else 1
+        assert np.array_equal(y[r], af[r, pi[e]])
+
+
+@pytest.mark.parametrize("fmt", ["nf4", "mxfp4"])
+def test_gemm_single_expert_is_numpy_matmul(fmt):
+    """E = 1 reduces to a plain GEMM Y = A W^T (N != K catches a transpose)."""
+    g = inputs.rng(7)
+    N, K, M = 48, 192, 13
+    a = inputs.bf16_normal(g, (M, K))
+    offsets = np.array([0, M], np.int32)
+    if fmt == "nf4":
+        w, sc = oracle.quant_nf4(inputs.normal_weights(g, (1, N, K)))
+        wd = oracle.dequant_nf4(w, sc)[0].astype(np.float64)
+        y = oracle.grouped_gemm_nf4(a, w, sc, offsets)
+    else:
+        w, sc = inputs.mxfp4_random(g, 1, N, K)
+        wd = oracle.dequant_mxfp4(w, sc)[0].astype(np.float64)
+        y = oracle.grouped_gemm_mxfp4(a, w, sc, offsets)
+    ref = _af(a) @ wd.T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_gemm_brute_force_tiny():
+    g = inputs.rng(8)
+    E, N, K, T, k = 3, 8, 64, 5, 2
+    ids, _ = inputs.route_uniform(g, T, k, E)
+    offsets, s2f, _, _ = oracle.route(ids, E)
+    w, sc = oracle.quant_nf4(inputs.normal_weights(g, (E, N, K)))
+    wd = oracle.dequant_nf4(w, sc).astype(np.float64)
+    a = inputs.bf16_normal(g, (T * k, K))
+    af = _af(a)
+    y = oracle.grouped_gemm_nf4(a, w, sc, offsets)
+    for e in range(E):
+        for r in range(offsets[e], offsets[e + 1]):
+            for n in range(N):
+                ref = math.fsum(af[r, kk] * wd[e, n, kk] for kk in range(K))
+                assert abs(y[r, n] - ref) <= 1e-14 * max(1.0, abs(ref))
+
+
+def test_gemm_requested_rows_subset():
+    g = inputs.rng(9)
+    E, N, K, M = 4, 16, 64, 20
+    offsets = np.array([0, 5, 5, 12, M], np.int32)
+    w, sc = inputs.mxfp4_random(g, E, N, K)
+    a = inputs.bf16_normal(g, (M, K))
+    full = oracle.grouped_gemm_mxfp4(a, w, sc, offsets)
+    rows = np.array([19, 0, 7, 11], np.int64)
+    part = oracle.grouped_gemm_mxfp4(a, w, sc, offsets, rows=rows)
+    assert np.array_equal(part, full[rows])
+
+
+# ---------------------------------------------------------------- combine
+
+
+def test_combine_one_hot_is_gather():
+    g = inputs.rng(10)
+    T, k, E, N = 6, 3, 4, 40
+    ids, _ = inputs.route_uniform(g, T, k, E)
+    offsets, s2f, f2s, _ = oracle.route(ids, E)
+    y = inputs.bf16_normal(g, (T * k, N))
+    w = np.zeros((T, k), np.float32)
+    pick = g.integers(0, k, size=T)
+    w[np.arange(T), pick] = 1.0
+    out = oracle.combine(y, f2s, w)
+    for t in range(T):
+        assert np.array_equal(out[t], _af(y[f2s[t * k + pick[t]]]))
+
+
+def test_combine_brute_force_and_dropped_pairs():
+    g = inputs.rng(11)
+    T, k, E, N = 7, 4, 6, 16
+    ids, wts = inputs.route_uniform(g, T, k, E)
+    ids[2, 1] = E  # dropped pair
+    offsets, s2f, f2s, bad = oracle.route(ids, E)
+    assert bad == 1
+    y = inputs.bf16_normal(g, (T * k, N))
+    out = oracle.combine(y, f2s, wts)
+    yf = _af(y)
+    for t in range(T):
+        for n in range(N):
+            terms = [float(wts[t, j]) * yf[f2s[t * k + j], n] for j in range(k) if f2s[t * k + j] >= 0]
+            assert abs(out[t, n] - math.fsum(terms)) <= 1e-14 * max(1.0, sum(abs(x) for x in terms))
+
+
+def test_combine_weights_summing_to_one_reproduce_a_shared_row():
+    g = inputs.rng(12)
+    T, k, E, N = 4, 4, 8, 32
+    ids, wts = inputs.route_uniform(g, T, k, E)
+    offsets, s2f, f2s, _ = oracle.route(ids, E)
+    row = inputs.bf16_normal(g, (1, N))
+    y = np.repeat(row, T * k, axis=0)
+    out = oracle.combine(y, f2s, wts)
+    wsum = wts.astype(np.float64).sum(axis=1)
+    assert np.allclose(out, wsum[:, None] * _af(row), rtol=1e-15, atol=0)
+    assert np.allclose(wsum, 1.0, atol=1e-6)
