@@ -1,0 +1,346 @@
+// api.cu -- the extern "C" boundary of libgnf4 (declared in include/gnf4.h).
+//
+// Each entry point validates pointers and shapes on the host, encodes the
+// TMA descriptors it needs, and enqueues its kernels on the caller's stream.
+// Nothing here allocates device memory, synchronises the host, or falls back
+// to the CPU.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "gnf4.h"
+#include "internal.h"
+
+namespace gnf4 {
+
+// Device error word: one per device (each device holds its own copy of this
+// module-scope variable).  Kernels receive its device address as a plain
+// pointer; the host reads it only through gnf4_device_errors().
+static __device__ unsigned g_device_errors;
+
+namespace {
+
+thread_local char t_last_error[512] = "";
+
+gnf4_status fail(gnf4_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+gnf4_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(GNF4_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+struct DeviceState {
+  bool ready = false;
+  int num_sms = 0;
+  int cc_major = 0, cc_minor = 0;
+  unsigned* err = nullptr;  // device address of g_device_errors
+};
+
+constexpr int kMaxDevices = 64;
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Per-device set-up on first use: SM count, compute capability and the
+// device address of the error word.  Touches no stream.
+gnf4_status device_state(DeviceState** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(GNF4_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+    cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_device_errors)) != cudaSuccess)
+      return cuda_fail(e, "cudaGetSymbolAddress(device error word)");
+    d.err = static_cast<unsigned*>(p);
+    d.ready = true;
+  }
+  if (d.cc_major != 10) return fail(GNF4_ERR_CUDA, "libgnf4 is built for sm_100a; device is sm_%d%d", d.cc_major, d.cc_minor);
+  *out = &d;
+  return GNF4_OK;
+}
+
+// A pointer the GPU can read as device memory: device or managed allocations.
+bool is_device_pointer(const void* p) {
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+gnf4_status check_ptr(const void* p, const char* name, size_t align, bool required = true) {
+  if (p == nullptr) {
+    if (required) return fail(GNF4_ERR_INVALID_ARG, "%s is NULL", name);
+    return GNF4_OK;
+  }
+  if (reinterpret_cast<uintptr_t>(p) % align != 0)
+    return fail(GNF4_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+  if (!is_device_pointer(p))
+    return fail(GNF4_ERR_INVALID_ARG,
+                "%s is not device memory: libgnf4 runs on the GPU only and never falls back to the CPU", name);
+  return GNF4_OK;
+}
+
+#define GNF4_TRY(x)                  \
+  do {                               \
+    gnf4_status _s = (x);            \
+    if (_s != GNF4_OK) return _s;    \
+  } while (0)
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// A [M, K] bf16 row-major: 64 x 32 boxes (128-byte rows), 128B swizzle, zero fill.
+gnf4_status encode_act_map(CUtensorMap* m, const void* a, int M, int K) {
+  auto fn = encode_fn();
+  if (!fn) return fail(GNF4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GNF4_ERR_CUDA, "activation tensor map encode failed (CUresult %d)", (int)r);
+  return GNF4_OK;
+}
+
+// W [E, N, K/2] u8: 32-byte x 128-row x 1 boxes, no swizzle, zero fill.
+gnf4_status encode_weight_map(CUtensorMap* m, const void* w, int E, int N, int K) {
+  auto fn = encode_fn();
+  if (!fn) return fail(GNF4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)N, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N * (cuuint64_t)(K / 2)};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(w), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GNF4_ERR_CUDA, "weight tensor map encode failed (CUresult %d)", (int)r);
+  return GNF4_OK;
+}
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Shared validation of the grouped GEMM / GEMV arguments.
+gnf4_status check_grouped(int fmt, const void* a, const uint8_t* w, const void* scales, const int32_t* offsets,
+                          const int32_t* counts, int E, int N, int K, int M, const void* y) {
+  if (E < 1 || E > kMaxExperts) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "E=%d outside [1, %d]", E, kMaxExperts);
+  if (N < 1 || N % 8 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N=%d must be a positive multiple of 8", N);
+  const int kq = fmt == 0 ? 64 : 32;
+  if (K < kq || K % kq != 0 || K > 65536)
+    return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K=%d must be a multiple of %d in [%d, 65536] for %s", K, kq, kq,
+                fmt == 0 ? "NF4" : "MXFP4");
+  if (M < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d is negative", M);
+  if ((offsets == nullptr) == (counts == nullptr))
+    return fail(GNF4_ERR_INVALID_ARG, "pass exactly one of offsets [E+1] and counts [E]");
+  if (M == 0) return GNF4_OK;
+  GNF4_TRY(check_ptr(a, "a", 16));
+  GNF4_TRY(check_ptr(w, "w", 16));
+  GNF4_TRY(check_ptr(scales, fmt == 0 ? "absmax" : "scales", fmt == 0 ? 4 : 1));
+  GNF4_TRY(check_ptr(offsets, "offsets", 4, false));
+  GNF4_TRY(check_ptr(counts, "counts", 4, false));
+  GNF4_TRY(check_ptr(y, "y", 16));
+  return GNF4_OK;
+}
+
+gnf4_status grouped_gemm(int fmt, const void* a, const uint8_t* w, const void* scales, const int32_t* offsets,
+                         const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
+  GNF4_TRY(check_grouped(fmt, a, w, scales, offsets, counts, E, N, K, M, y));
+  if (M == 0) return GNF4_OK;
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  CUtensorMap tm_a, tm_w;
+  GNF4_TRY(encode_act_map(&tm_a, a, M, K));
+  GNF4_TRY(encode_weight_map(&tm_w, w, E, N, K));
+  GroupedArgs p{static_cast<const __nv_bfloat16*>(a), w, scales, offsets, counts,
+                static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
+  // upper bound on work units: every group adds at most one partial chunk
+  const long long nwt = (N + gemm_tc_weight_rows_per_unit() - 1) / gemm_tc_weight_rows_per_unit();
+  const long long rpu = gemm_tc_rows_per_unit();
+  const long long chunks = (M + rpu - 1) / rpu + (E < M ? E : M);
+  const long long units = chunks * nwt;
+  if (units >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d, N=%d give too many work units", M, N);
+  const int grid = (int)(units < d->num_sms ? units : d->num_sms);
+  cudaError_t e = launch_gemm_tc(fmt, tm_a, tm_w, p, grid, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "grouped GEMM launch");
+  return GNF4_OK;
+}
+
+gnf4_status grouped_gemv(int fmt, const void* a, const uint8_t* w, const void* scales, const int32_t* offsets,
+                         const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
+  GNF4_TRY(check_grouped(fmt, a, w, scales, offsets, counts, E, N, K, M, y));
+  if (M == 0) return GNF4_OK;
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  GroupedArgs p{static_cast<const __nv_bfloat16*>(a), w, scales, offsets, counts,
+                static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
+  const long long hit = E < M ? E : M;  // groups with rows
+  const long long warps = hit * ((N + gemv_rows_per_warp() - 1) / gemv_rows_per_warp());
+  const long long blocks = (warps + gemv_warps_per_block() - 1) / gemv_warps_per_block();
+  const long long cap = 2LL * d->num_sms;
+  const int grid = (int)(blocks < cap ? blocks : cap);
+  cudaError_t e = launch_gemv(fmt, p, grid, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "grouped GEMV launch");
+  return GNF4_OK;
+}
+
+}  // namespace
+}  // namespace gnf4
+
+using namespace gnf4;
+
+extern "C" {
+
+const char* gnf4_last_error(void) { return t_last_error; }
+
+const char* gnf4_version(void) { return "libgnf4 0.1.0 (sm_100a)"; }
+
+gnf4_status gnf4_device_errors(uint32_t* flags, int clear) {
+  if (flags == nullptr) return fail(GNF4_ERR_INVALID_ARG, "flags is NULL");
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  unsigned v = 0;
+  cudaError_t e = cudaMemcpy(&v, d->err, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (clear) {
+    const unsigned zero = 0;
+    e = cudaMemcpy(d->err, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  }
+  *flags = v;
+  return GNF4_OK;
+}
+
+size_t gnf4_route_workspace_bytes(int T, int k, int E) {
+  if (T < 0 || k < 1 || E < 1) return 0;
+  return route_workspace_bytes(T, k, E);
+}
+
+gnf4_status gnf4_route_permute(const int32_t* topk_ids, const void* x, int T, int k, int E, int K,
+                               int32_t* offsets, int32_t* sorted_to_flat, int32_t* flat_to_sorted, void* x_sorted,
+                               void* workspace, size_t workspace_bytes, int32_t* bad_id_count, void* stream) {
+  if (T < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T=%d is negative", T);
+  if (E < 1 || E > 4096) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "E=%d outside [1, 4096]", E);
+  if (k < 1 || k > E) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, E=%d]", k, E);
+  if (K < 8 || K % 8 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K=%d must be a positive multiple of 8", K);
+  if ((long long)T * k > (1LL << 30)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T*k too large");
+  GNF4_TRY(check_ptr(offsets, "offsets", 4));
+  GNF4_TRY(check_ptr(bad_id_count, "bad_id_count", 4, false));
+  if (T > 0) {
+    GNF4_TRY(check_ptr(topk_ids, "topk_ids", 4));
+    GNF4_TRY(check_ptr(x, "x", 16));
+    GNF4_TRY(check_ptr(sorted_to_flat, "sorted_to_flat", 4));
+    GNF4_TRY(check_ptr(flat_to_sorted, "flat_to_sorted", 4));
+    GNF4_TRY(check_ptr(x_sorted, "x_sorted", 16));
+  }
+  const size_t need = route_workspace_bytes(T, k, E);
+  if (need > 0) {
+    if (workspace_bytes < need)
+      return fail(GNF4_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu bytes needed",
+                  workspace_bytes, need);
+    GNF4_TRY(check_ptr(workspace, "workspace", 16));
+  }
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  cudaError_t e = launch_route(topk_ids, static_cast<const __nv_bfloat16*>(x), T, k, E, K, offsets,
+                               sorted_to_flat, flat_to_sorted, static_cast<__nv_bfloat16*>(x_sorted), workspace,
+                               bad_id_count, d->num_sms, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "route_permute launch");
+  return GNF4_OK;
+}
+
+gnf4_status gnf4_grouped_gemm_nf4(const void* a, const uint8_t* w, const float* absmax, const int32_t* offsets,
+                                  const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
+  return grouped_gemm(0, a, w, absmax, offsets, counts, E, N, K, M, y, stream);
+}
+
+gnf4_status gnf4_grouped_gemm_mxfp4(const void* a, const uint8_t* w, const uint8_t* scales, const int32_t* offsets,
+                                    const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
+  return grouped_gemm(1, a, w, scales, offsets, counts, E, N, K, M, y, stream);
+}
+
+gnf4_status gnf4_grouped_gemv_nf4(const void* a, const uint8_t* w, const float* absmax, const int32_t* offsets,
+                                  const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
+  return grouped_gemv(0, a, w, absmax, offsets, counts, E, N, K, M, y, stream);
+}
+
+gnf4_status gnf4_grouped_gemv_mxfp4(const void* a, const uint8_t* w, const uint8_t* scales, const int32_t* offsets,
+                                    const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
+  return grouped_gemv(1, a, w, scales, offsets, counts, E, N, K, M, y, stream);
+}
+
+gnf4_status gnf4_combine(const void* y, const int32_t* flat_to_sorted, const float* weights, int T, int k, int N,
+                         void* out, void* stream) {
+  if (T < 0 || k < 1) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T=%d / k=%d invalid", T, k);
+  if (N < 8 || N % 8 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N=%d must be a positive multiple of 8", N);
+  if (T == 0) return GNF4_OK;
+  GNF4_TRY(check_ptr(y, "y", 16));
+  GNF4_TRY(check_ptr(flat_to_sorted, "flat_to_sorted", 4));
+  GNF4_TRY(check_ptr(weights, "weights", 4));
+  GNF4_TRY(check_ptr(out, "out", 16));
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  cudaError_t e = launch_combine(static_cast<const __nv_bfloat16*>(y), flat_to_sorted, weights, T, k, N,
+                                 static_cast<__nv_bfloat16*>(out), d->num_sms, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  return GNF4_OK;
+}
+
+static gnf4_status dequant(int fmt, const uint8_t* w, const void* scales, int64_t rows, int K, float* out,
+                           void* stream) {
+  const int kq = fmt == 0 ? 64 : 32;
+  if (rows < 0 || K < kq || K % kq != 0)
+    return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "rows=%lld / K=%d invalid (K %% %d == 0 required)", (long long)rows, K,
+                kq);
+  if (rows == 0) return GNF4_OK;
+  GNF4_TRY(check_ptr(w, "w", 1));
+  GNF4_TRY(check_ptr(scales, fmt == 0 ? "absmax" : "scales", fmt == 0 ? 4 : 1));
+  GNF4_TRY(check_ptr(out, "out", 8));
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  cudaError_t e = launch_dequant(fmt, w, scales, rows, K, out, d->num_sms, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
+  return GNF4_OK;
+}
+
+gnf4_status gnf4_dequant_nf4_f32(const uint8_t* w, const float* absmax, int64_t rows, int K, float* out,
+                                 void* stream) {
+  return dequant(0, w, absmax, rows, K, out, stream);
+}
+
+gnf4_status gnf4_dequant_mxfp4_f32(const uint8_t* w, const uint8_t* scales, int64_t rows, int K, float* out,
+                                   void* stream) {
+  return dequant(1, w, scales, rows, K, out, stream);
+}
+
+}  // extern "C"

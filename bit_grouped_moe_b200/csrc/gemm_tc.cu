@@ -1,0 +1,304 @@
+// gemm_tc.cu -- grouped 4-bit expert GEMM on tcgen05 tensor cores (sm_100a).
+//
+// Y[r, n] = sum_k A[r, k] * W_e[n, k] for the rows r of every expert e, in
+// one launch for all experts (grouped-nf4-gemm 0.33.1 on PyPI, opening
+// paragraphs: decode in registers, blockwise scaling, fp32 accumulation,
+// bf16 epilogue; no bf16 copy of a weight ever reaches global memory).
+//
+// Design (B200):
+//  * The MMA is computed transposed: D^T[n, r] = W_e[n, :] . A[r, :].  The
+//    decoded weight tile (128 weight rows x 64 k, bf16) is the MMA's A
+//    operand and lives in TMEM; the activation rows of the group are the B
+//    operand, loaded by TMA into 128B-swizzled shared memory.  The token
+//    dimension is the MMA's N, so a group of r rows costs an MMA with
+//    N = round_up(r, 16) instead of a padded 128-row tile.
+//  * Work unit = (expert e, 128-row weight tile j, chunk of <= 128 of the
+//    expert's rows).  Units are listed expert-major, then weight tile, then
+//    chunk, so CTAs running at the same time share weight tiles in L2.  The
+//    list is derived on the device from the group offsets (no host sync, no
+//    tile list in global memory); a persistent grid strides over it.
+//  * Warp roles (16 warps): 0 = TMA producer, 1 = TMEM owner + MMA issuer,
+//    4..11 = decode (two groups of four, alternating k-stages; warp w owns
+//    TMEM lanes 32*(w%4)..+31, i.e. weight rows), 12..15 = epilogue.
+//  * Decode: each thread owns one weight row; per 64-k stage it reads 32
+//    packed bytes from shared memory, looks every byte up in a lane-private
+//    copy of the pair table (two bf16 codes per byte), multiplies by the
+//    block scale in bf16x2 and stores 32 columns to TMEM with tcgen05.st.
+//  * Pipeline: S shared/TMEM stages (full: TMA landed; afull: decoded tile
+//    in TMEM; sdone: MMA finished reading the stage), two TMEM accumulators
+//    so the epilogue of one unit overlaps the main loop of the next.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace gnf4 {
+namespace {
+
+constexpr int kBT = 128;        // activation rows (tokens) per unit = max MMA N
+constexpr int kBW = 128;        // weight rows per unit = MMA M
+constexpr int kBK = 64;         // k per stage
+constexpr int kStages = 4;
+constexpr int kThreads = 512;
+constexpr int kAccCols = 2 * kBT;                   // two fp32 accumulators
+constexpr int kACol0 = kAccCols;                    // decoded-weight ring
+constexpr int kTmemCols = 512;
+constexpr int kActStageBytes = kBT * kBK * 2;       // 16 KB
+constexpr int kWStageBytes = kBW * kBK / 2;         // 4 KB
+constexpr int kActBox = 32;                         // activation rows per TMA box
+
+struct Smem {
+  uint8_t act[kStages][kActStageBytes];  // 1024-aligned (offset 0)
+  uint8_t wq[kStages][kWStageBytes];
+  uint32_t lut[kLutWords];
+  int off[kMaxExperts + 1];
+  int upre[kMaxExperts + 1];
+  int scratch[kMaxExperts];
+  uint64_t full[kStages], afull[kStages], sdone[kStages];
+  uint64_t accf[2], acce[2];
+  uint64_t mdone;  // abort path only: every issued MMA has retired
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
+static_assert(kStages % 2 == 0, "stage parity must match decode group");
+
+struct Unit {
+  int e, j, row0, rows;
+};
+
+__device__ __forceinline__ Unit unit_of(const Smem& s, int E, int nwt, int u) {
+  Unit x;
+  x.e = find_group(s.upre, E, u);
+  const int local = u - s.upre[x.e];
+  const int rows_e = s.off[x.e + 1] - s.off[x.e];
+  const int nch = (rows_e + kBT - 1) / kBT;
+  x.j = local / nch;
+  const int c = local - x.j * nch;
+  x.row0 = s.off[x.e] + c * kBT;
+  x.rows = min(kBT, s.off[x.e + 1] - x.row0);
+  return x;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
+                   GroupedArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  unsigned* err = p.err;
+  volatile int* abort = &s.abort;
+
+  if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, err)) return;
+  const int nwt = (p.N + kBW - 1) / kBW;
+  block_exclusive_scan(p.E, s.upre, s.scratch,
+                       [&](int e) { return ((s.off[e + 1] - s.off[e] + kBT - 1) / kBT) * nwt; });
+  const int U = s.upre[p.E];
+  if ((int)blockIdx.x >= U) return;  // uniform over the block
+  const int nk = (p.K + kBK - 1) / kBK;
+
+  build_pair_lut<FMT>(s.lut, tid, kThreads);
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.afull[i], 4);
+      mbar_init(&s.sdone[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.accf[i], 1);
+      mbar_init(&s.acce[i], 4);
+    }
+    mbar_init(&s.mdone, 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+        const Unit x = unit_of(s, p.E, nwt, u);
+        const int nbox = (x.rows + kActBox - 1) / kActBox;
+        for (int kt = 0; kt < nk && ok; ++kt, ++it) {
+          const int st = it % kStages, use = it / kStages;
+          if (it >= kStages && !(ok = mbar_wait(&s.sdone[st], (use - 1) & 1, err, abort))) break;
+          mbar_arrive_expect_tx(&s.full[st], kWStageBytes + nbox * kActBox * 128);
+          tma_load_3d(s.wq[st], &tm_w, &s.full[st], kt * (kBK / 2), x.j * kBW, x.e);
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(s.act[st] + b * kActBox * 128, &tm_a, &s.full[st], kt * kBK, x.row0 + b * kActBox);
+        }
+      }
+      if (!ok) {
+        // drain the loads still in flight before the CTA's shared memory goes away
+        for (int i = max(0, it - kStages); i < it; ++i) mbar_drain(&s.full[i % kStages], (i / kStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, uc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
+        const Unit x = unit_of(s, p.E, nwt, u);
+        const int ab = uc & 1;
+        if (uc >= 2 && !(ok = mbar_wait(&s.acce[ab], ((uc >> 1) - 1) & 1, err, abort))) break;
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16_m128((uint32_t)((x.rows + 15) & ~15));
+        const uint32_t d_tmem = tmem + (uint32_t)(ab * kBT);
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          const int st = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!(ok = mbar_wait(&s.full[st], ph, err, abort))) break;
+          if (!(ok = mbar_wait(&s.afull[st], ph, err, abort))) break;
+          tc_fence_after();
+          const uint32_t a_col = tmem + (uint32_t)(kACol0 + st * (kBK / 2));
+          const uint32_t b_addr = smem_u32(s.act[st]);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            tc_mma_ts(d_tmem, a_col + kk * 8, sdesc_k_sw128(b_addr + kk * 32), idesc, (kt | kk) != 0);
+          tc_commit(&s.sdone[st]);
+        }
+        if (!ok) break;
+        tc_commit(&s.accf[ab]);
+      }
+      if (!ok) {
+        // abort: let every MMA already issued retire before TMEM is released
+        tc_commit(&s.mdone);
+        mbar_drain(&s.mdone, 0);
+      }
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ decode
+    const int grp = (warp - 4) >> 2, q = warp & 3;
+    const int nl = q * 32 + lane;
+    const uint32_t lut_lane = smem_u32(s.lut) + (uint32_t)lane * 4u;
+    const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+      const Unit x = unit_of(s, p.E, nwt, u);
+      const int n = x.j * kBW + nl;
+      const bool nvalid = n < p.N;
+      const size_t srow = (size_t)x.e * p.N + (size_t)n;
+      for (int kt = 0; kt < nk; ++kt, ++it) {
+        if ((it & 1) != grp) continue;
+        const int st = it % kStages, use = it / kStages;
+        if (!(ok = mbar_wait(&s.full[st], use & 1, err, abort))) break;
+        if (it >= kStages && !(ok = mbar_wait(&s.sdone[st], (use - 1) & 1, err, abort))) break;
+        uint32_t sc0 = 0, sc1 = 0;
+        if (nvalid) {
+          if (FMT == 0) {
+            const float am = __ldg(reinterpret_cast<const float*>(p.scales) + srow * (size_t)(p.K / 64) + kt);
+            const __nv_bfloat162 b2 = __float2bfloat162_rn(am);
+            sc0 = sc1 = *reinterpret_cast<const uint32_t*>(&b2);
+          } else {
+            const uint8_t* sp = reinterpret_cast<const uint8_t*>(p.scales) + srow * (size_t)(p.K / 32) + 2 * kt;
+            sc0 = e8m0_to_bf16x2(__ldg(sp));
+            sc1 = (2 * kt + 1 < p.K / 32) ? e8m0_to_bf16x2(__ldg(sp + 1)) : 0u;
+          }
+        }
+        const uint32_t wrow = smem_u32(s.wq[st]) + (uint32_t)nl * 32u;
+        const uint4 c0 = lds_u128(wrow), c1 = lds_u128(wrow + 16);
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        uint32_t v[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t wv = words[i];
+          const uint32_t sc = (i < 4) ? sc0 : sc1;
+          v[4 * i + 0] = bf16x2_mul(lds_u32(lut_lane + ((wv << 7) & 0x7F80u)), sc);
+          v[4 * i + 1] = bf16x2_mul(lds_u32(lut_lane + ((wv >> 1) & 0x7F80u)), sc);
+          v[4 * i + 2] = bf16x2_mul(lds_u32(lut_lane + ((wv >> 9) & 0x7F80u)), sc);
+          v[4 * i + 3] = bf16x2_mul(lds_u32(lut_lane + ((wv >> 17) & 0x7F80u)), sc);
+        }
+        tmem_st_32x32b_x32(t_lane + (uint32_t)(kACol0 + st * (kBK / 2)), v);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.afull[st]);
+      }
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+    int uc = 0;
+    for (int u = blockIdx.x; u < U; u += gridDim.x, ++uc) {
+      const Unit x = unit_of(s, p.E, nwt, u);
+      const int ab = uc & 1;
+      if (!mbar_wait(&s.accf[ab], (uc >> 1) & 1, err, abort)) break;
+      tc_fence_after();
+      const int n = x.j * kBW + q * 32 + lane;
+      __nv_bfloat16* ycol = p.y + (size_t)x.row0 * p.N + n;
+      for (int c = 0; c * 32 < x.rows; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBT + c * 32), v);
+        tmem_wait_ld();
+        if (n < p.N) {
+          const int lim = min(32, x.rows - c * 32);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < lim) ycol[(size_t)(c * 32 + i) * p.N] = __float2bfloat16_rn(__uint_as_float(v[i]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.acce[ab]);
+    }
+  }
+
+  // Normal path: the epilogue has consumed every accumulator, so every MMA
+  // and TMEM load has completed here.
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+size_t gemm_tc_smem_bytes() { return sizeof(Smem) + 1024; }
+
+template <int FMT>
+cudaError_t launch_gemm_tc_t(const CUtensorMap& tm_a, const CUtensorMap& tm_w, const GroupedArgs& p, int grid,
+                             cudaStream_t stream) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)gemm_tc_smem_bytes());
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  gemm_tc_kernel<FMT><<<grid, kThreads, gemm_tc_smem_bytes(), stream>>>(tm_a, tm_w, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& tm_w, const GroupedArgs& p,
+                           int grid, cudaStream_t stream) {
+  return fmt == 0 ? launch_gemm_tc_t<0>(tm_a, tm_w, p, grid, stream)
+                  : launch_gemm_tc_t<1>(tm_a, tm_w, p, grid, stream);
+}
+
+int gemm_tc_rows_per_unit() { return kBT; }
+int gemm_tc_weight_rows_per_unit() { return kBW; }
+
+}  // namespace gnf4

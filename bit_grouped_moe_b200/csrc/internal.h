@@ -1,0 +1,52 @@
+// internal.h -- launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_bf16.h>
+
+namespace gnf4 {
+
+// Arguments of the grouped GEMM / GEMV kernels (device pointers).
+struct GroupedArgs {
+  const __nv_bfloat16* a;  // [M, K]
+  const uint8_t* w;        // [E, N, K/2]
+  const void* scales;      // absmax fp32 [E, N, K/64] or e8m0 [E, N, K/32]
+  const int* offsets;      // [E+1] or null
+  const int* counts;       // [E] or null
+  __nv_bfloat16* y;        // [M, N]
+  unsigned* err;           // device error word
+  int E, N, K, M;
+};
+
+// gemm_tc.cu
+size_t gemm_tc_smem_bytes();
+int gemm_tc_rows_per_unit();
+int gemm_tc_weight_rows_per_unit();
+cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& tm_w, const GroupedArgs& p,
+                           int grid, cudaStream_t stream);
+
+// gemv.cu
+cudaError_t launch_gemv(int fmt, const GroupedArgs& p, int grid, cudaStream_t stream);
+int gemv_warps_per_block();
+int gemv_rows_per_warp();
+
+// route.cu
+size_t route_workspace_bytes(int T, int k, int E);
+cudaError_t launch_route(const int32_t* topk_ids, const __nv_bfloat16* x, int T, int k, int E, int K,
+                         int32_t* offsets, int32_t* sorted_to_flat, int32_t* flat_to_sorted,
+                         __nv_bfloat16* x_sorted, void* workspace, int32_t* bad_id_count, int num_sms,
+                         cudaStream_t stream);
+
+// combine.cu
+cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* flat_to_sorted, const float* weights, int T,
+                           int k, int N, __nv_bfloat16* out, int num_sms, cudaStream_t stream);
+
+// dequant.cu
+cudaError_t launch_dequant(int fmt, const uint8_t* w, const void* scales, int64_t rows, int K, float* out,
+                           int num_sms, cudaStream_t stream);
+
+}  // namespace gnf4

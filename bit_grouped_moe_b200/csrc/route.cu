@@ -1,0 +1,193 @@
+// route.cu -- sort (token, slot) pairs into per-expert row groups and gather
+// the activations (grouped-nf4-gemm releases, v0.2.6 "The patch point": the
+// argsort of the top-k ids, the gather x[idxs // k] and tokens_per_expert).
+//
+// A stable counting sort in four short launches, with no host sync and no
+// atomics on global memory:
+//   1. hist:    each 256-pair chunk counts its pairs per expert (shared
+//               memory) and writes the counts row hist[chunk][0..E);
+//   2. scan:    one block turns hist into each chunk's first output row per
+//               expert and writes offsets[0..E] and the dropped-id count;
+//   3. scatter: each chunk ranks its pairs within an expert in flat order
+//               (warp match + running per-expert counters, warps in order),
+//               giving sorted_to_flat / flat_to_sorted;
+//   4. gather:  x_sorted[r] = x[sorted_to_flat[r] / k] with 16-byte copies;
+//               rows past offsets[E] are zeroed.
+// Ids outside [0, E) are counted and dropped, never used as an index
+// (releases v0.3.0, "Also": model-global ids read out of bounds silently).
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace gnf4 {
+namespace {
+
+constexpr int kChunk = 256;  // pairs per histogram chunk
+constexpr int kMaxRouteExperts = 4096;
+
+__global__ void __launch_bounds__(kChunk) route_hist_kernel(const int32_t* ids, int M, int E, int32_t* hist,
+                                                            int32_t* badc) {
+  __shared__ int cnt[kMaxRouteExperts];
+  __shared__ int nbad;
+  const int tid = threadIdx.x, c = blockIdx.x;
+  for (int i = tid; i < E; i += kChunk) cnt[i] = 0;
+  if (tid == 0) nbad = 0;
+  __syncthreads();
+  const int f = c * kChunk + tid;
+  if (f < M) {
+    const int e = ids[f];
+    if (e >= 0 && e < E)
+      atomicAdd(&cnt[e], 1);
+    else
+      atomicAdd(&nbad, 1);
+  }
+  __syncthreads();
+  for (int i = tid; i < E; i += kChunk) hist[(size_t)c * E + i] = cnt[i];
+  if (tid == 0) badc[c] = nbad;
+}
+
+__global__ void __launch_bounds__(1024) route_scan_kernel(int32_t* hist, const int32_t* badc, int nchunk, int E,
+                                                          int32_t* offsets, int32_t* bad_out) {
+  __shared__ int tot[kMaxRouteExperts];
+  __shared__ int wsum[32];
+  const int tid = threadIdx.x;
+  // per expert: running count over chunks (coalesced across experts)
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < nchunk; ++c) {
+      const int v = hist[(size_t)c * E + e];
+      hist[(size_t)c * E + e] = run;
+      run += v;
+    }
+    tot[e] = run;
+  }
+  __syncthreads();
+  // exclusive scan of tot over experts: each thread takes a contiguous slice
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int lo = min(E, tid * per), hi = min(E, lo + per);
+  int mine = 0;
+  for (int e = lo; e < hi; ++e) mine += tot[e];
+  // block-wide exclusive scan of `mine`
+  const int lane = tid & 31, wid = tid >> 5;
+  int incl = mine;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) wsum[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    int w = (lane < (int)(blockDim.x >> 5)) ? wsum[lane] : 0;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, d);
+      if (lane >= d) w += v;
+    }
+    wsum[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  int base = incl - mine + (wid > 0 ? wsum[wid - 1] : 0);
+  for (int e = lo; e < hi; ++e) {
+    const int t = tot[e];
+    tot[e] = base;  // now the exclusive prefix
+    base += t;
+  }
+  // the owner of the last expert ends with the number of valid pairs
+  if (lo < hi && hi == E) offsets[E] = base;
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) offsets[e] = tot[e];
+  if (tid == 0 && bad_out != nullptr) {
+    int bad = 0;
+    for (int c = 0; c < nchunk; ++c) bad += badc[c];
+    *bad_out = bad;
+  }
+  // chunk bases: hist[c][e] += offsets[e]
+  for (size_t i = tid; i < (size_t)nchunk * E; i += blockDim.x) hist[i] += tot[i % E];
+}
+
+__global__ void __launch_bounds__(kChunk) route_scatter_kernel(const int32_t* ids, int M, int E,
+                                                               const int32_t* hist, int32_t* s2f,
+                                                               int32_t* f2s) {
+  __shared__ int run[kMaxRouteExperts];
+  const int tid = threadIdx.x, c = blockIdx.x, lane = tid & 31, wid = tid >> 5;
+  for (int i = tid; i < E; i += kChunk) run[i] = 0;
+  __syncthreads();
+  const int f = c * kChunk + tid;
+  const int e = (f < M) ? ids[f] : -1;
+  const bool valid = (f < M) && e >= 0 && e < E;
+  const unsigned lt = (1u << lane) - 1u;
+  int pos = -1;
+  for (int w = 0; w < kChunk / 32; ++w) {
+    if (wid == w) {
+      const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+      const int before = valid ? run[e] : 0;
+      __syncwarp();
+      if (valid) {
+        pos = hist[(size_t)c * E + e] + before + __popc(peers & lt);
+        if ((peers & lt) == 0u) run[e] = before + __popc(peers);  // lowest lane of the peer set
+      }
+    }
+    __syncthreads();
+  }
+  if (f < M) {
+    f2s[f] = valid ? pos : -1;
+    if (valid) s2f[pos] = f;
+  }
+}
+
+__global__ void route_gather_kernel(const uint4* x, int K8, int k, const int32_t* offsets, int E, int M,
+                                    int32_t* s2f, uint4* xs) {
+  const int nvalid = offsets[E];
+  const size_t total = (size_t)M * K8;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / K8);
+    const int v = (int)(i - (size_t)r * K8);
+    if (r < nvalid) {
+      const int f = s2f[r];
+      // a pair index outside [0, M) would mean a broken permutation: never
+      // dereference it, write zeros instead
+      xs[i] = (f >= 0 && f < M) ? x[(size_t)(f / k) * K8 + v] : make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      xs[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (v == 0) s2f[r] = -1;
+    }
+  }
+}
+
+}  // namespace
+
+size_t route_workspace_bytes(int T, int k, int E) {
+  const size_t M = (size_t)T * (size_t)k;
+  const size_t nchunk = (M + kChunk - 1) / kChunk;
+  size_t b = nchunk * (size_t)E * 4 + nchunk * 4;
+  return (b + 255) & ~(size_t)255;
+}
+
+cudaError_t launch_route(const int32_t* topk_ids, const __nv_bfloat16* x, int T, int k, int E, int K,
+                         int32_t* offsets, int32_t* sorted_to_flat, int32_t* flat_to_sorted,
+                         __nv_bfloat16* x_sorted, void* workspace, int32_t* bad_id_count, int num_sms,
+                         cudaStream_t stream) {
+  const int M = T * k;
+  const int nchunk = (M + kChunk - 1) / kChunk;
+  int32_t* hist = reinterpret_cast<int32_t*>(workspace);
+  int32_t* badc = hist + (size_t)nchunk * E;
+  if (M > 0) {
+    route_hist_kernel<<<nchunk, kChunk, 0, stream>>>(topk_ids, M, E, hist, badc);
+  }
+  route_scan_kernel<<<1, 1024, 0, stream>>>(hist, badc, nchunk, E, offsets, bad_id_count);
+  if (M > 0) {
+    route_scatter_kernel<<<nchunk, kChunk, 0, stream>>>(topk_ids, M, E, hist, sorted_to_flat, flat_to_sorted);
+    const int K8 = K / 8;
+    const size_t total = (size_t)M * K8;
+    const int threads = 256;
+    const size_t want = (total + threads - 1) / threads;
+    const int grid = (int)(want < (size_t)num_sms * 16 ? want : (size_t)num_sms * 16);
+    route_gather_kernel<<<grid, threads, 0, stream>>>(reinterpret_cast<const uint4*>(x), K8, k, offsets, E, M,
+                                                      sorted_to_flat, reinterpret_cast<uint4*>(x_sorted));
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace gnf4

@@ -1,0 +1,190 @@
+"""Thin ctypes binding of libgnf4 (the C ABI in include/gnf4.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (device memory and streams are the
+only things torch provides); the library refuses host memory, so there is no
+CPU fallback anywhere.  Importing this module loads ``libgnf4.so`` and fails
+loudly if it has not been built (``python -m bit_grouped_moe_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgnf4.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "gnf4.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m bit_grouped_moe_b200.build` "
+        "(libgnf4 has no CPU implementation to fall back to)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+DEVERR_TIMEOUT, DEVERR_BAD_OFFSETS, DEVERR_GEMV_ROWS = 0x1, 0x2, 0x4
+MAX_GEMV_ROWS = 8
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+_lib.gnf4_last_error.restype = ctypes.c_char_p
+_lib.gnf4_version.restype = ctypes.c_char_p
+_lib.gnf4_device_errors.argtypes = [_P, _I]
+_lib.gnf4_route_workspace_bytes.argtypes = [_I, _I, _I]
+_lib.gnf4_route_workspace_bytes.restype = _SZ
+_lib.gnf4_route_permute.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P, _P]
+for _name in ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_gemv_nf4", "gnf4_grouped_gemv_mxfp4"):
+    getattr(_lib, _name).argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+_lib.gnf4_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
+_lib.gnf4_dequant_nf4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
+_lib.gnf4_dequant_mxfp4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
+for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4",
+              "gnf4_grouped_gemv_nf4", "gnf4_grouped_gemv_mxfp4", "gnf4_combine", "gnf4_dequant_nf4_f32",
+              "gnf4_dequant_mxfp4_f32"):
+    getattr(_lib, _name).restype = _I
+
+
+class Gnf4Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"libgnf4 status {status}: {message}")
+        self.status = status
+
+
+def declared_symbols() -> list[str]:
+    """Names of the entry points declared in include/gnf4.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^[A-Za-z_][\w \*]*?\b(gnf4_\w+)\s*\(", text, flags=re.M)))
+
+
+def version() -> str:
+    return _lib.gnf4_version().decode()
+
+
+def last_error() -> str:
+    return _lib.gnf4_last_error().decode()
+
+
+def _check(status: int) -> None:
+    if status != OK:
+        raise Gnf4Error(status, last_error())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def device_errors(clear: bool = True) -> int:
+    """Device error word (synchronising; diagnostics only)."""
+    v = ctypes.c_uint32(0)
+    _check(_lib.gnf4_device_errors(ctypes.cast(ctypes.pointer(v), ctypes.c_void_p), int(clear)))
+    return int(v.value)
+
+
+def route_workspace_bytes(T: int, k: int, E: int) -> int:
+    return int(_lib.gnf4_route_workspace_bytes(T, k, E))
+
+
+def route_permute(topk_ids, x, E, offsets, sorted_to_flat, flat_to_sorted, x_sorted, workspace,
+                  bad_id_count=None, stream=None) -> None:
+    """Stable sort of (token, slot) pairs by expert + activation gather (all outputs preallocated)."""
+    T, k = topk_ids.shape
+    K = x.shape[1]
+    _check(_lib.gnf4_route_permute(_ptr(topk_ids), _ptr(x), T, k, E, K, _ptr(offsets), _ptr(sorted_to_flat),
+                                   _ptr(flat_to_sorted), _ptr(x_sorted), _ptr(workspace),
+                                   0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                   _ptr(bad_id_count), _stream(stream)))
+
+
+def _grouped(fn, a, w, scales, y, offsets=None, counts=None, stream=None):
+    E, N, K2 = w.shape
+    M = a.shape[0]
+    _check(fn(_ptr(a), _ptr(w), _ptr(scales), _ptr(offsets), _ptr(counts), E, N, 2 * K2, M, _ptr(y),
+              _stream(stream)))
+
+
+def grouped_gemm_nf4(a, w, absmax, y, offsets=None, counts=None, stream=None):
+    _grouped(_lib.gnf4_grouped_gemm_nf4, a, w, absmax, y, offsets, counts, stream)
+
+
+def grouped_gemm_mxfp4(a, w, scales, y, offsets=None, counts=None, stream=None):
+    _grouped(_lib.gnf4_grouped_gemm_mxfp4, a, w, scales, y, offsets, counts, stream)
+
+
+def grouped_gemv_nf4(a, w, absmax, y, offsets=None, counts=None, stream=None):
+    _grouped(_lib.gnf4_grouped_gemv_nf4, a, w, absmax, y, offsets, counts, stream)
+
+
+def grouped_gemv_mxfp4(a, w, scales, y, offsets=None, counts=None, stream=None):
+    _grouped(_lib.gnf4_grouped_gemv_mxfp4, a, w, scales, y, offsets, counts, stream)
+
+
+def combine(y, flat_to_sorted, weights, out, stream=None):
+    T, k = weights.shape
+    N = y.shape[1]
+    _check(_lib.gnf4_combine(_ptr(y), _ptr(flat_to_sorted), _ptr(weights), T, k, N, _ptr(out), _stream(stream)))
+
+
+def dequant_nf4_f32(w, absmax, out, stream=None):
+    K = w.shape[-1] * 2
+    rows = w.numel() // (K // 2)
+    _check(_lib.gnf4_dequant_nf4_f32(_ptr(w), _ptr(absmax), rows, K, _ptr(out), _stream(stream)))
+
+
+def dequant_mxfp4_f32(w, scales, out, stream=None):
+    K = w.shape[-1] * 2
+    rows = w.numel() // (K // 2)
+    _check(_lib.gnf4_dequant_mxfp4_f32(_ptr(w), _ptr(scales), rows, K, _ptr(out), _stream(stream)))
+
+
+# ---------------------------------------------------------------- convenience
+
+
+def moe_step(fmt, x, topk_ids, weights, w1, s1, w2, s2, h=None, ws=None, stream=None, decode=None):
+    """One pass of the path: route -> GEMM (proj 1) -> GEMM (proj 2) -> combine.
+
+    The activation between the two projections is not part of the path (no
+    GLU here): ``h`` [T*k, K2] bf16 is the second projection's input; if None,
+    the first projection's output columns [:K2] are used.  ``decode`` forces
+    the GEMV (True) or the tiled GEMM (False); by default the GEMV is used when
+    T <= 8 (at most 8 rows per group, host-known with no sync).
+    Returns (out [T, N2] bf16, offsets).
+    """
+    T, k = topk_ids.shape
+    E = w1.shape[0]
+    K1 = x.shape[1]
+    M = T * k
+    dev = x.device
+    N1 = w1.shape[1]
+    N2, K2 = w2.shape[1], w2.shape[2] * 2
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    s2f = torch.empty(M, dtype=torch.int32, device=dev)
+    f2s = torch.empty(M, dtype=torch.int32, device=dev)
+    xs = torch.empty(M, K1, dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = torch.empty(max(route_workspace_bytes(T, k, E), 16), dtype=torch.uint8, device=dev)
+    route_permute(topk_ids, x, E, offsets, s2f, f2s, xs, ws, stream=stream)
+    use_gemv = (T <= MAX_GEMV_ROWS) if decode is None else decode
+    y1 = torch.empty(M, N1, dtype=torch.bfloat16, device=dev)
+    fn1 = {("nf4", True): grouped_gemv_nf4, ("nf4", False): grouped_gemm_nf4,
+           ("mxfp4", True): grouped_gemv_mxfp4, ("mxfp4", False): grouped_gemm_mxfp4}[(fmt, use_gemv)]
+    fn1(xs, w1, s1, y1, offsets=offsets, stream=stream)
+    a2 = h if h is not None else y1[:, :K2].contiguous()
+    y2 = torch.empty(M, N2, dtype=torch.bfloat16, device=dev)
+    fn1(a2, w2, s2, y2, offsets=offsets, stream=stream)
+    out = torch.empty(T, N2, dtype=torch.bfloat16, device=dev)
+    combine(y2, f2s, weights, out, stream=stream)
+    return out, offsets

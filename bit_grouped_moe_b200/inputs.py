@@ -151,3 +151,31 @@ def routing_for(w: Workload, g: np.random.Generator, T: int | None = None):
     if w.routing == "zipf":
         return route_topk(g, T, w.k, w.E, zipf_s=w.zipf_s)
     return route_topk(g, T, w.k, w.E)
+
+
+def device_random_bytes(seed: int, shape, device="cuda", lo: int = 0, hi: int = 256):
+    """uint8 tensor drawn uniformly in [lo, hi) directly on the device with a
+    seeded torch generator (for expert stacks of several GB)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return torch.randint(lo, hi, tuple(shape), generator=gen, device=device, dtype=torch.int16).to(torch.uint8)
+
+
+def device_bf16_normal(seed: int, shape, device="cuda"):
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return torch.randn(tuple(shape), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def device_absmax(seed: int, shape, device="cuda", std: float = 0.02):
+    """Block absmax values with the statistics of 64 N(0, std^2) draws."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    out = torch.empty(tuple(shape), dtype=torch.float32, device=device)
+    flat = out.view(-1)
+    step = 1 << 22
+    for i in range(0, flat.numel(), step):
+        n = min(step, flat.numel() - i)
+        z = torch.randn((n, 64), generator=gen, device=device, dtype=torch.float32).abs().amax(dim=1)
+        flat[i:i + n] = z * std
+    return out

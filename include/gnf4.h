@@ -1,0 +1,196 @@
+/*
+ * gnf4.h -- C ABI of libgnf4: the grouped Mixture-of-Experts expert GEMM
+ * computed directly on 4-bit-packed weights, on one NVIDIA B200 (sm_100a).
+ *
+ * The operation (grouped-nf4-gemm 0.33.1 on PyPI, opening paragraphs): one
+ * launch runs the expert GEMM for every routed expert, decoding the packed
+ * weights in registers with their block scale, accumulating in fp32 and
+ * writing bf16.  No bf16 copy of any expert is ever written to memory.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All array pointers are DEVICE pointers, allocated and owned by the
+ *    caller.  libgnf4 allocates nothing, frees nothing and keeps no pointer
+ *    after a call returns.  A host pointer is refused (GNF4_ERR_INVALID_ARG)
+ *    before any launch: nothing ever falls back to the CPU (grouped-nf4-gemm
+ *    index.json, "non_goals": no silent fallbacks).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Calls only enqueue work on it; none synchronises the host.
+ *  - Inputs are never written (grouped-nf4-gemm releases, v0.2.5 "Fix:
+ *    build_group_tiles mutated its sizes argument").
+ *  - Shapes and alignment are checked on the host before launch and refused
+ *    with GNF4_ERR_UNSUPPORTED_SHAPE (grouped-nf4-gemm status page, "#324's
+ *    pre-launch shape refusal").  Byte offsets into the expert stacks are
+ *    64-bit (same page, "#87 ... int32 offset overflow").
+ *  - Errors that only the device can see (offsets that are not monotone or
+ *    exceed M, a GEMV group with more than 8 rows, a pipeline wait that ran
+ *    out) set bits in a device-side error word; read it with
+ *    gnf4_device_errors().
+ *  - gnf4_last_error() returns the text of the calling thread's last failure.
+ *
+ * Layouts
+ * -------
+ *  bf16 activations A / x / y / out are row-major, rows contiguous.
+ *  NF4 stack (bitsandbytes gemm_4bit layout; grouped-nf4-gemm 0.33.1 on
+ *    PyPI, "Try it on CPU right now", example 1):
+ *      w      uint8 [E, N, K/2]  two codes per byte, element 2i in the HIGH
+ *                                nibble, element 2i+1 in the LOW nibble;
+ *      absmax fp32  [E, N, K/64] one scale per 64 consecutive elements of a
+ *                                row; value = NF4[code] * absmax.
+ *  MXFP4 stack (OCP e2m1 + e8m0; same page, example 2, and grouped-nf4-gemm
+ *    releases, v0.2.5 "arena -> kernel"):
+ *      w      uint8 [E, N, K/2]  element 2i in the LOW nibble, 2i+1 in the
+ *                                HIGH nibble; bit 3 of a nibble is the sign;
+ *      scales uint8 [E, N, K/32] e8m0: value = e2m1[code] * 2^(scale-127).
+ *  Group description: `offsets` int32 [E+1] (rows of expert e are
+ *    offsets[e] .. offsets[e+1]-1 of the group-sorted A and Y, offsets[0] = 0,
+ *    offsets[E] <= M) or `counts` int32 [E] (per-group row count, the
+ *    pages' `sizes`: grouped-nf4-gemm releases, v0.3.1 "sizes is a per-group
+ *    token count").  Exactly one of the two is non-NULL.
+ *  Y[r, n] = sum_k A[r, k] * W_e[n, k] for offsets[e] <= r < offsets[e+1]
+ *    (both operands K-major).  Rows r >= offsets[E] of Y are not written.
+ */
+#ifndef GNF4_H
+#define GNF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GNF4_OK = 0,
+    GNF4_ERR_INVALID_ARG = 1,       /* NULL / host / misaligned pointer, bad count */
+    GNF4_ERR_UNSUPPORTED_SHAPE = 2, /* a shape rule below is broken */
+    GNF4_ERR_CUDA = 3,              /* a CUDA runtime call or launch failed */
+    GNF4_ERR_TIMEOUT = 4            /* reported through gnf4_device_errors() */
+} gnf4_status;
+
+/* Bits of the device error word (gnf4_device_errors). */
+#define GNF4_DEVERR_TIMEOUT 0x1u      /* a bounded pipeline wait gave up; outputs incomplete */
+#define GNF4_DEVERR_BAD_OFFSETS 0x2u  /* offsets not monotone, offsets[0] != 0 or offsets[E] > M */
+#define GNF4_DEVERR_GEMV_ROWS 0x4u    /* a GEMV group held more than 8 rows; that group was skipped */
+
+/* Text of the calling thread's last failure ("" if none). */
+const char *gnf4_last_error(void);
+
+/* Library version string. */
+const char *gnf4_version(void);
+
+/* Reads (and if `clear` != 0, resets) the device error word of the current
+ * device into *flags.  Synchronises the device: diagnostics only, never on
+ * the hot path. */
+gnf4_status gnf4_device_errors(uint32_t *flags, int clear);
+
+/* ------------------------------------------------------------------ */
+/* Routing: sort (token, slot) pairs into per-expert row groups         */
+/* ------------------------------------------------------------------ */
+
+/* Workspace bytes gnf4_route_permute needs for T tokens, top-k, E experts. */
+size_t gnf4_route_workspace_bytes(int T, int k, int E);
+
+/* Stable counting sort of the M = T*k (token, slot) pairs by expert id and
+ * gather of the activations into group-sorted order (grouped-nf4-gemm
+ * releases, v0.2.6 "The patch point": argsort of the top-k ids, the gather
+ * x[idxs // k], and tokens_per_expert as the group sizes).
+ *   topk_ids       int32 [T, k]   expert of pair f = t*k + j;
+ *   x              bf16  [T, K]   token activations;
+ *   offsets        int32 [E+1]    OUT: group row offsets, offsets[E] = valid pairs;
+ *   sorted_to_flat int32 [M]      OUT: pair of each sorted row, -1 past offsets[E];
+ *   flat_to_sorted int32 [M]      OUT: sorted row of each pair, -1 if dropped;
+ *   x_sorted       bf16  [M, K]   OUT: x_sorted[r] = x[sorted_to_flat[r] / k];
+ *                                 rows past offsets[E] are zero;
+ *   workspace      device bytes, at least gnf4_route_workspace_bytes(T, k, E),
+ *                  16-byte aligned; its contents on entry do not matter;
+ *   bad_id_count   int32 [1] OUT (may be NULL): pairs whose id is outside
+ *                  [0, E).  Such pairs are dropped, never used as an index
+ *                  (grouped-nf4-gemm releases, v0.3.0 "Also": model-global
+ *                  expert ids read out of bounds silently).
+ * Within an expert, pairs keep ascending flat index (a stable sort).
+ * Rules: T >= 0, 1 <= k <= E <= 4096, K % 8 == 0, x and x_sorted 16-byte
+ * aligned.  T == 0 writes offsets only. */
+gnf4_status gnf4_route_permute(const int32_t *topk_ids, const void *x, int T, int k, int E, int K,
+                               int32_t *offsets, int32_t *sorted_to_flat, int32_t *flat_to_sorted,
+                               void *x_sorted, void *workspace, size_t workspace_bytes,
+                               int32_t *bad_id_count, void *stream);
+
+/* ------------------------------------------------------------------ */
+/* Grouped GEMM (prefill: any number of rows per group)                */
+/* ------------------------------------------------------------------ */
+
+/* NF4 grouped GEMM on tcgen05 tensor cores (grouped-nf4-gemm 0.33.1 on PyPI,
+ * opening paragraphs; grouped-nf4-gemm index.json, problems_solved[0]).
+ *   a      bf16 [M, K] group-sorted activations (16-byte aligned);
+ *   w, absmax: the NF4 stack above (w 16-byte aligned);
+ *   offsets / counts: the group description above;
+ *   y      bf16 [M, N] OUT.
+ * Rules: 1 <= E <= 1024, N >= 1, N % 8 == 0, K % 64 == 0, 64 <= K <= 65536,
+ * M >= 0 (M == 0 launches nothing).  Decoded weights are rounded to bf16 for
+ * the tensor-core multiply; sums are fp32; the output is rounded to bf16. */
+gnf4_status gnf4_grouped_gemm_nf4(const void *a, const uint8_t *w, const float *absmax, const int32_t *offsets,
+                                  const int32_t *counts, int E, int N, int K, int M, void *y, void *stream);
+
+/* MXFP4 grouped GEMM (grouped-nf4-gemm releases, v0.2.0 "the MXFP4
+ * native-byte lane": the e2m1 codebook is a table swap of the NF4 mainloop;
+ * v0.3.1: gemm_mxfp4_grouped's sizes is a per-group token count).
+ * Same arguments with `scales` (e8m0 [E, N, K/32]) for absmax.
+ * Rules: as NF4 but K % 32 == 0, 32 <= K <= 65536.  e2m1 times a power of two
+ * is exact in bf16, so the tensor cores see the exact decoded weights. */
+gnf4_status gnf4_grouped_gemm_mxfp4(const void *a, const uint8_t *w, const uint8_t *scales, const int32_t *offsets,
+                                    const int32_t *counts, int E, int N, int K, int M, void *y, void *stream);
+
+/* ------------------------------------------------------------------ */
+/* Grouped GEMV (decode: at most 8 rows per group)                     */
+/* ------------------------------------------------------------------ */
+
+/* Decode variant for a handful of rows per expert (grouped-nf4-gemm
+ * index.json, limitations: gemv_mxfp4_b32 "re-streams weights per row: it is
+ * a decode lever for a handful of rows").  Here every weight byte is read
+ * once for all of its group's rows.  Same arguments and rules as the GEMM
+ * calls; additionally every group must hold at most 8 rows (a caller with
+ * T <= 8 tokens and distinct experts per token always satisfies this).  A
+ * larger group is skipped and flagged with GNF4_DEVERR_GEMV_ROWS. */
+gnf4_status gnf4_grouped_gemv_nf4(const void *a, const uint8_t *w, const float *absmax, const int32_t *offsets,
+                                  const int32_t *counts, int E, int N, int K, int M, void *y, void *stream);
+gnf4_status gnf4_grouped_gemv_mxfp4(const void *a, const uint8_t *w, const uint8_t *scales, const int32_t *offsets,
+                                    const int32_t *counts, int E, int N, int K, int M, void *y, void *stream);
+
+/* ------------------------------------------------------------------ */
+/* Top-k combine                                                       */
+/* ------------------------------------------------------------------ */
+
+/* Weighted scatter of expert outputs back to tokens (grouped-nf4-gemm
+ * index.json, problems_solved[5] "top-k combine"; releases v0.2.6: the
+ * caller's "weighting, unsorting"):
+ *   out[t, n] = sum_{j<k} weights[t, j] * y[flat_to_sorted[t*k + j], n],
+ * summed in fp32 in order j = 0..k-1, rounded to bf16; pairs whose
+ * flat_to_sorted is -1 (or not below T*k) contribute nothing.
+ *   y bf16 [T*k, N] (group-sorted expert outputs); flat_to_sorted int32 [T*k];
+ *   weights fp32 [T, k]; out bf16 [T, N] OUT.
+ * Rules: T >= 0, k >= 1, N % 8 == 0, y and out 16-byte aligned. */
+gnf4_status gnf4_combine(const void *y, const int32_t *flat_to_sorted, const float *weights, int T, int k, int N,
+                         void *out, void *stream);
+
+/* ------------------------------------------------------------------ */
+/* Decode checks (test support)                                        */
+/* ------------------------------------------------------------------ */
+
+/* fp32 decode of `rows` packed rows of K elements: out[r, k] = NF4[code] *
+ * absmax[r, k/64] (one fp32 multiply, round to nearest, no flush to zero).
+ * This is the reference decode the pages call dequant_ref (grouped-nf4-gemm
+ * 0.33.1 on PyPI, example 1).  Rules: K % 64 == 0, rows >= 0. */
+gnf4_status gnf4_dequant_nf4_f32(const uint8_t *w, const float *absmax, int64_t rows, int K, float *out,
+                                 void *stream);
+
+/* fp32 decode of MXFP4 rows: out[r, k] = e2m1[code] * 2^(scale-127), with
+ * scale 255 decoding to NaN (same page, example 2).  Rules: K % 32 == 0. */
+gnf4_status gnf4_dequant_mxfp4_f32(const uint8_t *w, const uint8_t *scales, int64_t rows, int K, float *out,
+                                   void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GNF4_H */

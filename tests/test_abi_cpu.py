@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point the header declares, and refuses bad shapes and host
+pointers before it would touch the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from bit_grouped_moe_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib_path():
+    return build.build()
+
+
+@pytest.fixture(scope="module")
+def g(lib_path):
+    from bit_grouped_moe_b200 import gnf4
+    return gnf4
+
+
+def test_header_symbols_exported(lib_path, g):
+    names = g.declared_symbols()
+    assert len(names) >= 12, names
+    for required in ("gnf4_route_permute", "gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4",
+                     "gnf4_grouped_gemv_nf4", "gnf4_grouped_gemv_mxfp4", "gnf4_combine"):
+        assert required in names
+    lib = ctypes.CDLL(lib_path)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/gnf4.h but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", lib_path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (gnf4_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_version(g):
+    assert "sm_100a" in g.version()
+
+
+def test_route_workspace_size(g):
+    assert g.route_workspace_bytes(16, 2, 8) >= (8 + 1) * 4
+    assert g.route_workspace_bytes(4096, 8, 384) >= 128 * 384 * 4
+    assert g.route_workspace_bytes(0, 2, 8) == 0
+    assert g.route_workspace_bytes(4, 0, 8) == 0
+
+
+def _raw(g, name, *args):
+    return getattr(g._lib, name)(*args)
+
+
+@pytest.mark.parametrize("E,N,K,fmt,expect", [
+    (0, 64, 64, "nf4", 2), (1025, 64, 64, "nf4", 2), (4, 60, 64, "nf4", 2),
+    (4, 64, 96, "nf4", 2), (4, 64, 48, "mxfp4", 2), (4, 64, 0, "mxfp4", 2),
+])
+def test_gemm_shape_refusals(g, E, N, K, fmt, expect):
+    fn = g._lib.gnf4_grouped_gemm_nf4 if fmt == "nf4" else g._lib.gnf4_grouped_gemm_mxfp4
+    st = fn(None, None, None, ctypes.c_void_p(16), None, E, N, K, 8, None, None)
+    assert st == expect, g.last_error()
+    assert g.last_error()
+
+
+def test_exactly_one_group_description(g):
+    for fn in (g._lib.gnf4_grouped_gemm_nf4, g._lib.gnf4_grouped_gemv_mxfp4):
+        assert fn(None, None, None, None, None, 4, 64, 64, 8, None, None) == g.ERR_INVALID_ARG
+        assert fn(None, None, None, ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 64, 64, 8, None, None) \
+            == g.ERR_INVALID_ARG
+
+
+def test_empty_gemm_is_a_no_op(g):
+    # M == 0 launches nothing and needs no device pointers
+    assert g._lib.gnf4_grouped_gemm_nf4(None, None, None, ctypes.c_void_p(16), None, 4, 64, 64, 0, None, None) == 0
+
+
+def test_host_pointers_refused(g):
+    """A CPU buffer is never computed on: the call refuses it (no CPU fallback)."""
+    a = np.zeros((8, 64), np.uint16)
+    w = np.zeros((4, 64, 32), np.uint8)
+    am = np.ones((4, 64, 1), np.float32)
+    off = np.array([0, 2, 4, 6, 8], np.int32)
+    y = np.zeros((8, 64), np.uint16)
+    p = lambda x: x.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    st = g._lib.gnf4_grouped_gemm_nf4(p(a), p(w), p(am), p(off), None, 4, 64, 64, 8, p(y), None)
+    assert st in (g.ERR_INVALID_ARG, g.ERR_CUDA)
+    assert "device" in g.last_error() or "CUDA" in g.last_error() or "aligned" in g.last_error()
+
+
+def test_route_refusals(g):
+    f = g._lib.gnf4_route_permute
+    assert f(None, None, 4, 0, 8, 64, None, None, None, None, None, 0, None, None) == g.ERR_UNSUPPORTED_SHAPE
+    assert f(None, None, 4, 9, 8, 64, None, None, None, None, None, 0, None, None) == g.ERR_UNSUPPORTED_SHAPE
+    assert f(None, None, 4, 2, 8, 60, None, None, None, None, None, 0, None, None) == g.ERR_UNSUPPORTED_SHAPE
+    assert f(None, None, -1, 2, 8, 64, None, None, None, None, None, 0, None, None) == g.ERR_UNSUPPORTED_SHAPE
+
+
+def test_combine_refusals(g):
+    f = g._lib.gnf4_combine
+    assert f(None, None, None, 4, 2, 12, None, None) == g.ERR_UNSUPPORTED_SHAPE
+    assert f(None, None, None, 4, 0, 16, None, None) == g.ERR_UNSUPPORTED_SHAPE
+    assert f(None, None, None, 0, 2, 16, None, None) == g.OK
+
+
+def test_product_path_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "bit_grouped_moe_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), fn
+                assert "gnf4_oracle" not in text and "liboracle" not in text, fn
