@@ -1,0 +1,595 @@
+#!/usr/bin/env python
+"""Benchmark of the grouped 4-bit MoE expert path on B200.
+
+One step = one pass of the whole path over one batch of synthetic tokens:
+route_permute -> projection 1 (gate_up) -> projection 2 (down) -> combine.
+Decode workloads (T <= 8 tokens) run the grouped GEMV; prefill workloads the
+tcgen05 grouped GEMM.  The activation between the projections (a GLU) is not
+part of the path: projection 2 reads a resident synthetic [T*k, K2] input.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl libgnf4|reference]
+
+Prints ONE JSON line (rank 0).  For N > 1 (torchrun) every rank runs its own
+replica of the workload (no data-path collective; weak scaling) and the time
+is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_grouped_moe_b200 import inputs  # noqa: E402
+
+METRIC = "grouped 4-bit GEMM TFLOP/s (prefill) & weight GB/s (decode) vs B200 roofline"
+DEFAULT_WORKLOAD = "olmoe-decode-t8"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+N_WEIGHT_COPIES = 4
+N_BATCHES = 8
+
+
+# ------------------------------------------------------------------ helpers
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "bit_grouped_moe_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel_key, sha):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the kernel source as it stands now."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(kernel_key)
+    if not e or e.get("source_sha") != sha:
+        return None
+    return e.get("dram_bytes_per_launch_full_size")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled in the background."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        rows = [s for (t, s) in self.samples if t0 - 0.15 <= t <= t1 + 0.15]
+        if not rows and self.samples:
+            rows = [min(self.samples, key=lambda ts: min(abs(ts[0] - t0), abs(ts[0] - t1)))[1]]
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            parts = [p.strip() for p in r.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                mhz.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------ workload
+
+
+class Workload:
+    """Device-resident inputs of one workload: rotating weight copies larger
+    than L2, a set of token batches, and the step's output buffers."""
+
+    def __init__(self, name, device, seed, build_host_copy):
+        import torch
+
+        from bit_grouped_moe_b200 import gnf4
+
+        self.g = gnf4
+        self.torch = torch
+        self.wl = inputs.WORKLOADS[name]
+        wl = self.wl
+        self.name = name
+        self.dev = device
+        self.T, self.k, self.E = wl.T, wl.k, wl.E
+        self.M = self.T * self.k
+        self.decode = self.T <= gnf4.MAX_GEMV_ROWS
+        self.p1, self.p2 = wl.projections[0], wl.projections[-1]
+        rng = inputs.rng(seed)
+        # token batches (ids, router weights, x) resident on the device; host copies kept for e2e
+        self.batches = []
+        for _ in range(N_BATCHES):
+            ids, wts = inputs.routing_for(wl, rng)
+            x = inputs.bf16_normal(rng, (self.T, self.p1.K))
+            self.batches.append((ids, wts, x))
+        self.d_batches = [(torch.from_numpy(i).to(device), torch.from_numpy(w).to(device),
+                           torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device))
+                          for (i, w, x) in self.batches]
+        # weight stacks: N_WEIGHT_COPIES rotating copies of both projections
+        self.host_stacks = None
+        self.stacks = []
+        for c in range(N_WEIGHT_COPIES):
+            st = []
+            for j, p in enumerate((self.p1, self.p2)):
+                st.append(self._stack(wl.fmt, p, seed * 100 + c * 10 + j, keep_host=(c == 0 and build_host_copy)))
+            self.stacks.append(st)
+        self.h = torch.from_numpy(inputs.bf16_normal(rng, (self.M, self.p2.K)).view(np.int16)).view(
+            torch.bfloat16).to(device)
+        # outputs and scratch
+        E, M = self.E, self.M
+        self.off = torch.empty(E + 1, dtype=torch.int32, device=device)
+        self.s2f = torch.empty(M, dtype=torch.int32, device=device)
+        self.f2s = torch.empty(M, dtype=torch.int32, device=device)
+        self.xs = torch.empty(M, self.p1.K, dtype=torch.bfloat16, device=device)
+        self.ws = torch.empty(max(gnf4.route_workspace_bytes(self.T, self.k, E), 16), dtype=torch.uint8,
+                              device=device)
+        self.y1 = torch.empty(M, self.p1.N, dtype=torch.bfloat16, device=device)
+        self.y2 = torch.empty(M, self.p2.N, dtype=torch.bfloat16, device=device)
+        self.out = torch.empty(self.T, self.p2.N, dtype=torch.bfloat16, device=device)
+        # host routing of every batch: number of experts hit (algorithmic bytes)
+        self.hit = [int(np.count_nonzero(np.bincount(b[0].reshape(-1), minlength=E))) for b in self.batches]
+        f = gnf4
+        self.fn = {("nf4", True): f.grouped_gemv_nf4, ("nf4", False): f.grouped_gemm_nf4,
+                   ("mxfp4", True): f.grouped_gemv_mxfp4, ("mxfp4", False): f.grouped_gemm_mxfp4}[
+            (wl.fmt, self.decode)]
+
+    def _stack(self, fmt, p, seed, keep_host):
+        torch = self.torch
+        E = self.E
+        if keep_host:  # the copy the CPU baseline also reads is drawn on the host
+            rng = inputs.rng(seed)
+            if fmt == "nf4":
+                w, s = inputs.nf4_direct(rng, E, p.N, p.K)
+            else:
+                w, s = inputs.mxfp4_random(rng, E, p.N, p.K)
+            if keep_host:
+                if self.host_stacks is None:
+                    self.host_stacks = []
+                self.host_stacks.append((w, s))
+            return torch.from_numpy(w).to(self.dev), torch.from_numpy(s).to(self.dev)
+        w = inputs.device_random_bytes(seed, (E, p.N, p.K // 2), device=self.dev)
+        if fmt == "nf4":
+            s = inputs.device_absmax(seed + 1, (E, p.N, p.K // 64), device=self.dev)
+        else:
+            s = inputs.device_random_bytes(seed + 1, (E, p.N, p.K // 32), device=self.dev, lo=118, hi=131)
+        return w, s
+
+    # bytes / flops -----------------------------------------------------
+    def weight_bytes(self, p, hit):
+        per_elem_scale = 4 / 64 if self.wl.fmt == "nf4" else 1 / 32
+        return int(hit * p.N * (p.K // 2 + p.K * per_elem_scale))
+
+    def proj_bytes(self, p, hit):
+        """Algorithmic bytes of one projection launch: weights + scales of the
+        experts hit, activations read, outputs written."""
+        return self.weight_bytes(p, hit) + self.M * p.K * 2 + self.M * p.N * 2
+
+    def step_weight_bytes(self, i):
+        h = self.hit[i % N_BATCHES]
+        return self.weight_bytes(self.p1, h) + self.weight_bytes(self.p2, h)
+
+    def step_flops(self):
+        return 2 * self.M * (self.p1.N * self.p1.K + self.p2.N * self.p2.K)
+
+    # one step ------------------------------------------------------------
+    def step(self, i, ev=None):
+        g = self.g
+        ids, wts, x = self.d_batches[i % N_BATCHES]
+        (w1, s1), (w2, s2) = self.stacks[i % N_WEIGHT_COPIES]
+        g.route_permute(ids, x, self.E, self.off, self.s2f, self.f2s, self.xs, self.ws)
+        if ev is not None:
+            ev[0].record()
+        self.fn(self.xs, w1, s1, self.y1, offsets=self.off)
+        if ev is not None:
+            ev[1].record()
+        self.fn(self.h, w2, s2, self.y2, offsets=self.off)
+        g.combine(self.y2, self.f2s, wts, self.out)
+
+    def launches_per_step(self):
+        return 4 + 2 + 1  # route (hist, scan, scatter, gather) + 2 projections + combine
+
+
+# ------------------------------------------------------------------ distributed
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU (oracle) legs
+
+
+def oracle_step(wl_obj, batch_i, n_slice=None):
+    """The same step computed by the oracle on the host (fp64): route, gather,
+    both projections (optionally on their first n_slice weight rows) and the
+    combine.  Returns (weight bytes, flops) of the work done."""
+    import torch
+
+    import oracle
+
+    ids, wts, x = wl_obj.batches[batch_i % N_BATCHES]
+    E, k = wl_obj.E, wl_obj.k
+    off, s2f, f2s, _ = oracle.route(ids, E)
+    xs = oracle.gather(x, k, s2f, int(off[E]))
+    (w1, s1), (w2, s2) = wl_obj.host_stacks
+    n1 = wl_obj.p1.N if n_slice is None else min(n_slice, wl_obj.p1.N)
+    n2 = wl_obj.p2.N if n_slice is None else min(n_slice, wl_obj.p2.N)
+    gemm = oracle.grouped_gemm_nf4 if wl_obj.wl.fmt == "nf4" else oracle.grouped_gemm_mxfp4
+    gemm(xs, np.ascontiguousarray(w1[:, :n1]), np.ascontiguousarray(s1[:, :n1]), off)
+    y2 = gemm(wl_obj.h_host, np.ascontiguousarray(w2[:, :n2]), np.ascontiguousarray(s2[:, :n2]), off)
+    y2_bits = np.zeros((wl_obj.M, n2), np.uint16)
+    y2_bits[:y2.shape[0]] = torch.from_numpy(y2).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    oracle.combine(y2_bits, f2s, wts)
+    hit = wl_obj.hit[batch_i % N_BATCHES]
+    scale = 4 / 64 if wl_obj.wl.fmt == "nf4" else 1 / 32
+    wbytes = hit * (n1 * wl_obj.p1.K + n2 * wl_obj.p2.K) * (0.5 + scale)
+    return int(wbytes), 2 * wl_obj.M * (n1 * wl_obj.p1.K + n2 * wl_obj.p2.K)
+
+
+def cpu_baseline(wl_obj, budget_s=15.0):
+    """Oracle timed on the host cores on a bounded sample of the workload."""
+    import oracle
+
+    cores = os.cpu_count() or 1
+    oracle.set_threads(cores)
+    # calibrate the weight-row slice so that one step costs ~budget/6
+    t0 = time.perf_counter()
+    oracle_step(wl_obj, 0, n_slice=64)
+    t_unit = max(time.perf_counter() - t0, 1e-3)
+    n_slice = int(min(max(64, 64 * (budget_s / 6) / t_unit), max(wl_obj.p1.N, wl_obj.p2.N)))
+    n_slice -= n_slice % 8
+    tot_b, tot_f, steps = 0, 0, 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s and steps < 6:
+        b, f = oracle_step(wl_obj, steps, n_slice=n_slice)
+        tot_b += b
+        tot_f += f
+        steps += 1
+    dt = time.perf_counter() - t0
+    return {"bytes": tot_b, "flops": tot_f, "seconds": dt, "cores": cores, "steps": steps, "n_slice": n_slice}
+
+
+# ------------------------------------------------------------------ main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--impl", default="libgnf4", choices=["libgnf4", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    wl_def = inputs.WORKLOADS[args.workload]
+    decode = wl_def.T <= 8
+    steps = args.steps if args.steps is not None else (20000 if decode else 200)
+    warmup = args.warmup if args.warmup is not None else (100 if decode else 10)
+    warmup = max(warmup, 3)
+
+    world, rank, local = (1, 0, 0)
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        return run_reference(args, steps, warmup, world)
+    world, rank, local = dist_setup(args.gpus)
+    return run_gpu(args, steps, warmup, world, rank, local, decode)
+
+
+def _unit(decode):
+    return ("GB/s", "weight GB/s") if decode else ("TFLOP/s", "TFLOP/s")
+
+
+def _config(wl_obj_or_def, world):
+    wl = wl_obj_or_def
+    return {
+        "workload": f"{wl.name}: {wl.fmt.upper()} grouped MoE experts, E={wl.E}, top-{wl.k}, T={wl.T} tokens",
+        "experts": wl.E, "top_k": wl.k, "tokens_per_step": wl.T,
+        "projections": [{"name": p.name, "K": p.K, "N": p.N} for p in wl.projections],
+        "format": wl.fmt,
+        "l2": f"{N_WEIGHT_COPIES} rotating copies of every weight stack (inputs larger than L2), {N_BATCHES} token batches",
+        "parallelism": f"{world} independent replica(s)",
+    }
+
+
+def run_gpu(args, steps, warmup, world, rank, local, decode):
+    import torch
+
+    dev = f"cuda:{local}"
+    torch.cuda.set_device(local)
+    wl = Workload(args.workload, dev, seed=1234 + rank, build_host_copy=(rank == 0 and world == 1))
+    wl.h_host = wl.h.cpu().view(torch.int16).numpy().view(np.uint16)
+    stream = torch.cuda.current_stream()
+
+    # warm-up
+    for i in range(warmup):
+        wl.step(i)
+    torch.cuda.synchronize()
+    assert wl.g.device_errors() == 0, "device error word set during warm-up"
+
+    # timed region (inputs resident): K steps, events around the dominant kernel
+    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record(stream)
+    for i in range(steps):
+        wl.step(i, ev_pairs[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    time.sleep(0.2)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    ms_local = start.elapsed_time(stop)
+    ms = max_over_ranks(ms_local, world)
+    dom_ms = sum(a.elapsed_time(b) for a, b in ev_pairs) / steps
+    assert wl.g.device_errors() == 0, "device error word set during the timed steps"
+
+    # e2e through the public API with host buffers (pinned), copies in the timed region
+    host_in = []
+    for (ids, wts, x) in wl.batches:
+        host_in.append((torch.from_numpy(ids).pin_memory(), torch.from_numpy(wts).pin_memory(),
+                        torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()))
+    host_out = torch.empty(wl.T, wl.p2.N, dtype=torch.bfloat16).pin_memory()
+    d_ids = torch.empty_like(wl.d_batches[0][0])
+    d_w = torch.empty_like(wl.d_batches[0][1])
+    d_x = torch.empty_like(wl.d_batches[0][2])
+    e2e_steps = max(1, min(steps, 2000 if decode else steps))
+
+    def e2e_step(i):
+        hi, hw, hx = host_in[i % N_BATCHES]
+        d_ids.copy_(hi, non_blocking=True)
+        d_w.copy_(hw, non_blocking=True)
+        d_x.copy_(hx, non_blocking=True)
+        (w1, s1), (w2, s2) = wl.stacks[i % N_WEIGHT_COPIES]
+        g = wl.g
+        g.route_permute(d_ids, d_x, wl.E, wl.off, wl.s2f, wl.f2s, wl.xs, wl.ws)
+        wl.fn(wl.xs, w1, s1, wl.y1, offsets=wl.off)
+        wl.fn(wl.h, w2, s2, wl.y2, offsets=wl.off)
+        g.combine(wl.y2, wl.f2s, d_w, wl.out)
+        host_out.copy_(wl.out, non_blocking=True)
+
+    for i in range(warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = int(wl.batches[0][0].nbytes + wl.batches[0][1].nbytes + wl.batches[0][2].nbytes)
+    d2h = int(host_out.numel() * 2)
+
+    unit, _ = _unit(decode)
+    if decode:
+        per_rank = sum(wl.step_weight_bytes(i) for i in range(steps))
+        value = world * per_rank / (ms / 1e3) / 1e9
+        e2e_val = world * sum(wl.step_weight_bytes(i) for i in range(e2e_steps)) / (e2e_ms / 1e3) / 1e9
+    else:
+        value = world * steps * wl.step_flops() / (ms / 1e3) / 1e12
+        e2e_val = world * e2e_steps * wl.step_flops() / (e2e_ms / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    kern_file = "gemv.cu" if decode else "gemm_tc.cu"
+    kern_key = f"{'gemv' if decode else 'gemm_tc'}_{wl.wl.fmt}:{args.workload}:{wl.p1.name}"
+    sha = kernel_source_sha([kern_file, "common.cuh"])
+    if decode:
+        mean_hit = sum(wl.hit[i % N_BATCHES] for i in range(steps)) / steps
+        alg = wl.proj_bytes(wl.p1, mean_hit)
+        achieved = alg / (dom_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": committed_traffic(kern_key, sha),
+                "kernel": f"gemv_kernel<{wl.wl.fmt}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})",
+                "algorithmic_bytes_per_launch": int(alg), "avg_launch_us": round(dom_ms * 1e3, 3),
+                "peak_source": f"hbm_gbs of {peak_src}"}
+    else:
+        flops = 2 * wl.M * wl.p1.N * wl.p1.K
+        achieved = flops / (dom_ms / 1e3) / 1e12
+        pk = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk, "unit": "TFLOP/s",
+                "frac": round(achieved / pk, 4), "traffic": committed_traffic(kern_key, sha),
+                "kernel": f"gemm_tc_kernel<{wl.wl.fmt}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})",
+                "algorithmic_flops_per_launch": int(flops), "avg_launch_us": round(dom_ms * 1e3, 3),
+                "peak_source": f"bf16_tflops_sustained of {peak_src} (kind::f16 MMA on decoded bf16 tiles)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(wl)
+        v = cb["bytes"] / cb["seconds"] / 1e9 if decode else cb["flops"] / cb["seconds"] / 1e12
+        cpu = {"value": round(v, 6), "unit": unit, "cores": cb["cores"], "kind": "oracle",
+               "sample": f"{cb['steps']} steps of the same workload on the first {cb['n_slice']} weight rows of "
+                         f"each projection (route + fp64 grouped GEMM x2 + combine), {cb['seconds']:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": steps,
+            "warmup": warmup, "ms_per_step": round(ms / steps, 6), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(wl.wl, world),
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "gpu_launches": steps * wl.launches_per_step(), "clocks": clocks, "impl": "libgnf4",
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference(args, steps, warmup, world):
+    """The oracle arm: the same metric computed by the CPU oracle on the box's
+    host cores, each step a bounded sample of the workload."""
+    import oracle
+
+    wl_def = inputs.WORKLOADS[args.workload]
+    decode = wl_def.T <= 8
+    unit, _ = _unit(decode)
+
+    class HostWL:
+        pass
+
+    h = HostWL()
+    h.wl = wl_def
+    h.E, h.k, h.T = wl_def.E, wl_def.k, wl_def.T
+    h.M = h.T * h.k
+    h.p1, h.p2 = wl_def.projections[0], wl_def.projections[-1]
+    rng = inputs.rng(1234)
+    h.batches = []
+    for _ in range(N_BATCHES):
+        ids, wts = inputs.routing_for(wl_def, rng)
+        x = inputs.bf16_normal(rng, (h.T, h.p1.K))
+        h.batches.append((ids, wts, x))
+    h.hit = [int(np.count_nonzero(np.bincount(b[0].reshape(-1), minlength=h.E))) for b in h.batches]
+    # only the weight rows the sample touches are drawn
+    cores = os.cpu_count() or 1
+    oracle.set_threads(cores)
+    budget = 90.0 / (steps + warmup)
+    n_slice = 64
+    srng = inputs.rng(99)
+    mk = inputs.nf4_direct if wl_def.fmt == "nf4" else inputs.mxfp4_random
+
+    def stacks(ns):
+        return [mk(srng, h.E, min(ns, p.N), p.K) for p in (h.p1, h.p2)]
+
+    h.host_stacks = stacks(n_slice)
+    h.h_host = inputs.bf16_normal(rng, (h.M, h.p2.K))
+    t0 = time.perf_counter()
+    oracle_step(h, 0, n_slice=n_slice)
+    t1 = max(time.perf_counter() - t0, 1e-4)
+    n_slice = int(max(8, min(max(h.p1.N, h.p2.N), n_slice * budget / t1)))
+    n_slice -= n_slice % 8
+    n_slice = max(n_slice, 8)
+    h.host_stacks = stacks(n_slice)
+    for i in range(warmup):
+        oracle_step(h, i, n_slice=n_slice)
+    tb, tf = 0, 0
+    t0 = time.perf_counter()
+    for i in range(steps):
+        b, f = oracle_step(h, i, n_slice=n_slice)
+        tb += b
+        tf += f
+    dt = time.perf_counter() - t0
+    value = tb / dt / 1e9 if decode else tf / dt / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": world, "steps": steps, "warmup": warmup,
+        "ms_per_step": round(dt * 1e3 / steps, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config(wl_def, world),
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: the full route + combine and the fp64 grouped GEMM of both "
+                                   f"projections on the first {n_slice} weight rows"},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
