@@ -36,7 +36,7 @@ from bit_grouped_moe_b200 import inputs  # noqa: E402
 METRIC = "grouped 4-bit GEMM TFLOP/s (prefill) & weight GB/s (decode) vs B200 roofline"
 DEFAULT_WORKLOAD = "olmoe-decode-t8"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-N_WEIGHT_COPIES = 4
+N_WEIGHT_COPIES = 4  # default; --weight-copies changes it (profiling uses 1)
 N_BATCHES = 8
 
 
@@ -353,7 +353,10 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--impl", default="libgnf4", choices=["libgnf4", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--weight-copies", type=int, default=N_WEIGHT_COPIES,
+                    help="rotating copies of every weight stack (4 keeps the rotation larger than L2)")
     args = ap.parse_args()
+    globals()["N_WEIGHT_COPIES"] = max(1, args.weight_copies)
 
     wl_def = inputs.WORKLOADS[args.workload]
     decode = wl_def.T <= 8

@@ -205,8 +205,7 @@ gnf4_status grouped_gemv(int fmt, const void* a, const uint8_t* w, const void* s
   GroupedArgs p{static_cast<const __nv_bfloat16*>(a), w, scales, offsets, counts,
                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
   const long long hit = E < M ? E : M;  // groups with rows
-  const long long warps = hit * ((N + gemv_rows_per_warp() - 1) / gemv_rows_per_warp());
-  const long long blocks = (warps + gemv_warps_per_block() - 1) / gemv_warps_per_block();
+  const long long blocks = hit * ((N + gemv_rows_per_block() - 1) / gemv_rows_per_block());
   const long long cap = 2LL * d->num_sms;
   const int grid = (int)(blocks < cap ? blocks : cap);
   cudaError_t e = launch_gemv(fmt, p, grid, as_stream(stream));

@@ -75,6 +75,36 @@ __device__ __forceinline__ void build_pair_lut(uint32_t* lut, int tid, int nthre
   }
 }
 
+// Same pair table with a 256-byte entry stride (entry b, lane l at byte
+// b*256 + 4*l; the upper 128 bytes of every entry are unused).  The address
+// of a lookup is then one PRMT: byte 0 = 4*lane, byte 1 = the packed byte,
+// bytes 2..3 = 0 -- one integer instruction and one shared load per byte.
+constexpr int kLut256Words = 256 * 64;
+constexpr int kLut256Bytes = kLut256Words * 4;
+
+template <int FMT>
+__device__ __forceinline__ void build_pair_lut256(uint32_t* lut, int tid, int nthreads) {
+  for (int i = tid; i < 256 * 32; i += nthreads) {
+    const uint32_t b = (uint32_t)i >> 5, l = (uint32_t)i & 31u;
+    float lo, hi;
+    if (FMT == 0) {
+      lo = kNf4Code[b >> 4];
+      hi = kNf4Code[b & 15u];
+    } else {
+      lo = e2m1_value(b & 15u);
+      hi = e2m1_value(b >> 4);
+    }
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    lut[b * 64u + l] = *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
   __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
   __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
@@ -107,12 +137,37 @@ __device__ __forceinline__ uint2 ldg_nc_u64(const void* p) {
   return v;
 }
 
+__device__ __forceinline__ uint4 ldg_nc_u128(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ uint4 ldg_u128(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
+}
+
+// Decodes the 16 packed bytes of `w` (byte i = elements 2i, 2i+1 of 32
+// codes) into 16 bf16x2 pairs multiplied by the bf16x2 scale `sc`.
+// `lane4` = 4 * lane; the table is the 256-byte-stride pair table.
+__device__ __forceinline__ uint32_t lut256_get(const uint8_t* lut, uint32_t word, uint32_t lane4, uint32_t j) {
+  return *reinterpret_cast<const uint32_t*>(lut + prmt_b32(word, lane4, 0x5504u | (j << 4)));
+}
+
+__device__ __forceinline__ void decode16_lut256(const uint8_t* lut, uint32_t lane4, uint4 w, uint32_t sc,
+                                                uint32_t (&out)[16]) {
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out[4 * i + j] = bf16x2_mul(lut256_get(lut, words[i], lane4, (uint32_t)j), sc);
+  }
 }
 
 // ---------------------------------------------------------------- mbarrier
@@ -281,7 +336,7 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // D (16x8 fp32) += A (16x16 bf16, row) x B (16x8 bf16, col).
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])

@@ -17,16 +17,20 @@
 //    chunk, so CTAs running at the same time share weight tiles in L2.  The
 //    list is derived on the device from the group offsets (no host sync, no
 //    tile list in global memory); a persistent grid strides over it.
-//  * Warp roles (16 warps): 0 = TMA producer, 1 = TMEM owner + MMA issuer,
-//    4..11 = decode (two groups of four, alternating k-stages; warp w owns
-//    TMEM lanes 32*(w%4)..+31, i.e. weight rows), 12..15 = epilogue.
-//  * Decode: each thread owns one weight row; per 64-k stage it reads 32
-//    packed bytes from shared memory, looks every byte up in a lane-private
-//    copy of the pair table (two bf16 codes per byte), multiplies by the
-//    block scale in bf16x2 and stores 32 columns to TMEM with tcgen05.st.
-//  * Pipeline: S shared/TMEM stages (full: TMA landed; afull: decoded tile
-//    in TMEM; sdone: MMA finished reading the stage), two TMEM accumulators
-//    so the epilogue of one unit overlaps the main loop of the next.
+//  * Three decoupled rings keep enough bytes in flight: packed weights (12
+//    stages x 4 KB, its own TMA thread), activation tiles (6 stages x 16 KB,
+//    its own TMA thread) and decoded weights in TMEM (8 stages x 32 columns),
+//    plus two TMEM accumulators so the epilogue of one unit overlaps the
+//    main loop of the next.
+//  * Warp roles (18 warps): 0 = weight TMA, 1 = TMEM owner + MMA issuer,
+//    2 = activation TMA, 4..15 = decode (three groups of four taking k-stages
+//    in turn; warp w owns TMEM lanes 32*(w%4)..+31, i.e. weight rows),
+//    16..19 = epilogue.
+//  * Decode: a thread owns one weight row; per 64-k stage it reads its 32
+//    packed bytes from shared memory, and for every byte builds the address
+//    of a lane-private pair-table entry with one PRMT, loads the two bf16
+//    codes, multiplies them by the block scale in bf16x2 and finally stores
+//    32 columns to TMEM with tcgen05.st.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -36,39 +40,46 @@
 namespace gnf4 {
 namespace {
 
-constexpr int kBT = 128;        // activation rows (tokens) per unit = max MMA N
-constexpr int kBW = 128;        // weight rows per unit = MMA M
-constexpr int kBK = 64;         // k per stage
-constexpr int kStages = 4;
-constexpr int kThreads = 512;
-constexpr int kAccCols = 2 * kBT;                   // two fp32 accumulators
-constexpr int kACol0 = kAccCols;                    // decoded-weight ring
+constexpr int kBT = 128;   // activation rows (tokens) per unit = max MMA N
+constexpr int kBW = 128;   // weight rows per unit = MMA M
+constexpr int kBK = 64;    // k per stage
+constexpr int kWStages = 12;
+constexpr int kAStages = 6;
+constexpr int kTStages = 8;
+constexpr int kDecGroups = 3;
+constexpr int kDecWarp0 = 4;
+constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;  // 16
+constexpr int kThreads = (kEpiWarp0 + 4) * 32;        // 640
+constexpr int kAccCols = 2 * kBT;                      // two fp32 accumulators
+constexpr int kACol0 = kAccCols;                       // decoded-weight ring
 constexpr int kTmemCols = 512;
-constexpr int kActStageBytes = kBT * kBK * 2;       // 16 KB
-constexpr int kWStageBytes = kBW * kBK / 2;         // 4 KB
-constexpr int kActBox = 32;                         // activation rows per TMA box
+constexpr int kActStageBytes = kBT * kBK * 2;          // 16 KB
+constexpr int kWStageBytes = kBW * kBK / 2;            // 4 KB
+constexpr int kActBox = 32;                            // activation rows per TMA box
+static_assert(kACol0 + kTStages * (kBK / 2) <= kTmemCols, "TMEM budget");
 
 struct Smem {
-  uint8_t act[kStages][kActStageBytes];  // 1024-aligned (offset 0)
-  uint8_t wq[kStages][kWStageBytes];
-  uint32_t lut[kLutWords];
+  uint8_t act[kAStages][kActStageBytes];  // 1024-aligned (offset 0)
+  uint32_t lut[kLut256Words];             // 64 KB
+  uint8_t wq[kWStages][kWStageBytes];
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
-  uint64_t full[kStages], afull[kStages], sdone[kStages];
+  uint64_t wfull[kWStages], wempty[kWStages];
+  uint64_t afull[kAStages], aempty[kAStages];
+  uint64_t tfull[kTStages], tempty[kTStages];
   uint64_t accf[2], acce[2];
   uint64_t mdone;  // abort path only: every issued MMA has retired
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
-static_assert(kStages % 2 == 0, "stage parity must match decode group");
 
 struct Unit {
   int e, j, row0, rows;
 };
 
-__device__ __forceinline__ Unit unit_of(const Smem& s, int E, int nwt, int u) {
+__device__ __forceinline__ Unit unit_of(const Smem& s, int E, int u) {
   Unit x;
   x.e = find_group(s.upre, E, u);
   const int local = u - s.upre[x.e];
@@ -99,12 +110,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if ((int)blockIdx.x >= U) return;  // uniform over the block
   const int nk = (p.K + kBK - 1) / kBK;
 
-  build_pair_lut<FMT>(s.lut, tid, kThreads);
+  build_pair_lut256<FMT>(s.lut, tid, kThreads);
   if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.afull[i], 4);
-      mbar_init(&s.sdone[i], 1);
+    for (int i = 0; i < kWStages; ++i) {
+      mbar_init(&s.wfull[i], 1);
+      mbar_init(&s.wempty[i], 4);
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&s.afull[i], 1);
+      mbar_init(&s.aempty[i], 1);
+    }
+    for (int i = 0; i < kTStages; ++i) {
+      mbar_init(&s.tfull[i], 4);
+      mbar_init(&s.tempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.accf[i], 1);
@@ -128,26 +146,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ weight TMA
     if (lane == 0) {
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-        const Unit x = unit_of(s, p.E, nwt, u);
-        const int nbox = (x.rows + kActBox - 1) / kActBox;
-        for (int kt = 0; kt < nk && ok; ++kt, ++it) {
-          const int st = it % kStages, use = it / kStages;
-          if (it >= kStages && !(ok = mbar_wait(&s.sdone[st], (use - 1) & 1, err, abort))) break;
-          mbar_arrive_expect_tx(&s.full[st], kWStageBytes + nbox * kActBox * 128);
-          tma_load_3d(s.wq[st], &tm_w, &s.full[st], kt * (kBK / 2), x.j * kBW, x.e);
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d(s.act[st] + b * kActBox * 128, &tm_a, &s.full[st], kt * kBK, x.row0 + b * kActBox);
+        const Unit x = unit_of(s, p.E, u);
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          const int st = it % kWStages, use = it / kWStages;
+          if (it >= kWStages && !(ok = mbar_wait(&s.wempty[st], (use - 1) & 1, err, abort))) break;
+          mbar_arrive_expect_tx(&s.wfull[st], kWStageBytes);
+          tma_load_3d(s.wq[st], &tm_w, &s.wfull[st], kt * (kBK / 2), x.j * kBW, x.e);
         }
       }
-      if (!ok) {
-        // drain the loads still in flight before the CTA's shared memory goes away
-        for (int i = max(0, it - kStages); i < it; ++i) mbar_drain(&s.full[i % kStages], (i / kStages) & 1);
+      if (!ok)  // drain loads still in flight before shared memory goes away
+        for (int i = max(0, it - kWStages); i < it; ++i) mbar_drain(&s.wfull[i % kWStages], (i / kWStages) & 1);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ activation TMA
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+        const Unit x = unit_of(s, p.E, u);
+        const int nbox = (x.rows + kActBox - 1) / kActBox;
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          const int st = it % kAStages, use = it / kAStages;
+          if (it >= kAStages && !(ok = mbar_wait(&s.aempty[st], (use - 1) & 1, err, abort))) break;
+          mbar_arrive_expect_tx(&s.afull[st], nbox * kActBox * 128);
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(s.act[st] + b * kActBox * 128, &tm_a, &s.afull[st], kt * kBK, x.row0 + b * kActBox);
+        }
       }
+      if (!ok)
+        for (int i = max(0, it - kAStages); i < it; ++i) mbar_drain(&s.afull[i % kAStages], (i / kAStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -155,24 +187,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0, uc = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
-        const Unit x = unit_of(s, p.E, nwt, u);
+        const Unit x = unit_of(s, p.E, u);
         const int ab = uc & 1;
         if (uc >= 2 && !(ok = mbar_wait(&s.acce[ab], ((uc >> 1) - 1) & 1, err, abort))) break;
         tc_fence_after();
         const uint32_t idesc = idesc_bf16_m128((uint32_t)((x.rows + 15) & ~15));
         const uint32_t d_tmem = tmem + (uint32_t)(ab * kBT);
         for (int kt = 0; kt < nk; ++kt, ++it) {
-          const int st = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!(ok = mbar_wait(&s.full[st], ph, err, abort))) break;
-          if (!(ok = mbar_wait(&s.afull[st], ph, err, abort))) break;
+          const int sa = it % kAStages, sT = it % kTStages;
+          if (!(ok = mbar_wait(&s.afull[sa], (it / kAStages) & 1, err, abort))) break;
+          if (!(ok = mbar_wait(&s.tfull[sT], (it / kTStages) & 1, err, abort))) break;
           tc_fence_after();
-          const uint32_t a_col = tmem + (uint32_t)(kACol0 + st * (kBK / 2));
-          const uint32_t b_addr = smem_u32(s.act[st]);
+          const uint32_t a_col = tmem + (uint32_t)(kACol0 + sT * (kBK / 2));
+          const uint32_t b_addr = smem_u32(s.act[sa]);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
             tc_mma_ts(d_tmem, a_col + kk * 8, sdesc_k_sw128(b_addr + kk * 32), idesc, (kt | kk) != 0);
-          tc_commit(&s.sdone[st]);
+          tc_commit(&s.aempty[sa]);
+          tc_commit(&s.tempty[sT]);
         }
         if (!ok) break;
         tc_commit(&s.accf[ab]);
@@ -183,24 +215,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_drain(&s.mdone, 0);
       }
     }
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp >= kDecWarp0 && warp < kEpiWarp0) {
     // ------------------------------------------------------------ decode
-    const int grp = (warp - 4) >> 2, q = warp & 3;
+    const int grp = (warp - kDecWarp0) >> 2, q = warp & 3;
     const int nl = q * 32 + lane;
-    const uint32_t lut_lane = smem_u32(s.lut) + (uint32_t)lane * 4u;
+    const uint8_t* lut = reinterpret_cast<const uint8_t*>(s.lut);
+    const uint32_t lane4 = (uint32_t)lane * 4u;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-      const Unit x = unit_of(s, p.E, nwt, u);
+      const Unit x = unit_of(s, p.E, u);
       const int n = x.j * kBW + nl;
       const bool nvalid = n < p.N;
-      const size_t srow = (size_t)x.e * p.N + (size_t)n;
+      const size_t srow = (size_t)x.e * p.N + (size_t)(nvalid ? n : 0);
       for (int kt = 0; kt < nk; ++kt, ++it) {
-        if ((it & 1) != grp) continue;
-        const int st = it % kStages, use = it / kStages;
-        if (!(ok = mbar_wait(&s.full[st], use & 1, err, abort))) break;
-        if (it >= kStages && !(ok = mbar_wait(&s.sdone[st], (use - 1) & 1, err, abort))) break;
+        if (it % kDecGroups != grp) continue;
+        const int sw = it % kWStages, sT = it % kTStages;
+        if (!(ok = mbar_wait(&s.wfull[sw], (it / kWStages) & 1, err, abort))) break;
+        if (it >= kTStages && !(ok = mbar_wait(&s.tempty[sT], ((it / kTStages) - 1) & 1, err, abort))) break;
         uint32_t sc0 = 0, sc1 = 0;
         if (nvalid) {
           if (FMT == 0) {
@@ -213,33 +246,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             sc1 = (2 * kt + 1 < p.K / 32) ? e8m0_to_bf16x2(__ldg(sp + 1)) : 0u;
           }
         }
-        const uint32_t wrow = smem_u32(s.wq[st]) + (uint32_t)nl * 32u;
-        const uint4 c0 = lds_u128(wrow), c1 = lds_u128(wrow + 16);
-        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        uint32_t v[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t wv = words[i];
-          const uint32_t sc = (i < 4) ? sc0 : sc1;
-          v[4 * i + 0] = bf16x2_mul(lds_u32(lut_lane + ((wv << 7) & 0x7F80u)), sc);
-          v[4 * i + 1] = bf16x2_mul(lds_u32(lut_lane + ((wv >> 1) & 0x7F80u)), sc);
-          v[4 * i + 2] = bf16x2_mul(lds_u32(lut_lane + ((wv >> 9) & 0x7F80u)), sc);
-          v[4 * i + 3] = bf16x2_mul(lds_u32(lut_lane + ((wv >> 17) & 0x7F80u)), sc);
+        // two 16-byte reads of this row's 32 bytes, ordered so a quarter warp
+        // touches 8 distinct 16-byte bank groups
+        const uint32_t wrow = smem_u32(s.wq[sw]) + (uint32_t)nl * 32u;
+        const uint32_t c_first = ((uint32_t)nl >> 2) & 1u;
+        uint4 c0 = lds_u128(wrow + 16u * c_first), c1 = lds_u128(wrow + 16u * (c_first ^ 1u));
+        if (c_first) {
+          const uint4 tmp = c0;
+          c0 = c1;
+          c1 = tmp;
         }
-        tmem_st_32x32b_x32(t_lane + (uint32_t)(kACol0 + st * (kBK / 2)), v);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.wempty[sw]);  // packed bytes are in registers now
+        uint32_t v[32];
+        {
+          uint32_t h0[16], h1[16];
+          decode16_lut256(lut, lane4, c0, sc0, h0);
+          decode16_lut256(lut, lane4, c1, sc1, h1);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            v[i] = h0[i];
+            v[16 + i] = h1[i];
+          }
+        }
+        tmem_st_32x32b_x32(t_lane + (uint32_t)(kACol0 + sT * (kBK / 2)), v);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s.afull[st]);
+        if (lane == 0) mbar_arrive(&s.tfull[sT]);
       }
     }
-  } else if (warp >= 12) {
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     int uc = 0;
     for (int u = blockIdx.x; u < U; u += gridDim.x, ++uc) {
-      const Unit x = unit_of(s, p.E, nwt, u);
+      const Unit x = unit_of(s, p.E, u);
       const int ab = uc & 1;
       if (!mbar_wait(&s.accf[ab], (uc >> 1) & 1, err, abort)) break;
       tc_fence_after();
@@ -263,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // Normal path: the epilogue has consumed every accumulator, so every MMA
-  // and TMEM load has completed here.
+  // and TMEM access has completed here.
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

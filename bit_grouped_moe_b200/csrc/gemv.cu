@@ -6,21 +6,24 @@
 // row (same page, limitations); here every weight byte is read once and used
 // for all of its group's rows.
 //
-// Work unit = one warp x (expert e, 16 consecutive weight rows, all of K).
-// The warp streams its 16 rows with 8-byte loads (each 32-byte sector of a
-// row is fully used by 4 lanes), decodes every packed byte with a lookup in
-// a lane-private copy of the pair table (two bf16 codes per byte), and feeds
-// the bf16 codes straight into m16n8k16 warp MMAs whose 8 columns are the
-// group's (<= 8) activation rows.  The MMA does the k-reduction that a
-// CUDA-core GEMV would do with warp shuffles.
-//   * NF4: codes enter the MMA unscaled; each 64-k block is accumulated on
-//     its own and folded in with its fp32 absmax (exact fp32 scaling).
-//   * MXFP4: codes are scaled by their power of two in bf16 before the MMA
-//     (exact), so the whole K accumulates in one fragment.
-// Lane (g, t) = (lane / 4, lane % 4) owns weight rows g and g+8 of the warp's
-// 16 and, within every 64-k chunk, the 16 consecutive k in [16t, 16t+16).
-// The MMA's k index is a permutation of these physical k; the activation
-// fragment uses the same permutation, so the contraction is unchanged.
+// Work unit = one CTA x (expert e, 64 consecutive weight rows).  The 8 warps
+// split K: warp w takes a contiguous range of 128-k "double chunks" and
+// computes the partial sums of all 64 rows (four m16 tiles) for the group's
+// <= 8 rows (the MMA's 8 columns); a fixed-order shared-memory reduction over
+// the warps finishes the unit.  Per double chunk a lane loads 16 bytes (32
+// codes) of each of its 8 weight rows with one 16-byte load each, decodes
+// every byte with one PRMT (which builds the table address) and one shared
+// load from a lane-private copy of the pair table, multiplies the bf16 pair
+// by the row's block scale, and feeds the pairs to m16n8k16 warp MMAs.  The
+// MMA does the k reduction that a CUDA-core GEMV would do with shuffles.
+//
+// Lane (g, t) = (lane / 4, lane % 4) owns rows g and g+8 of every tile and,
+// in every double chunk, the 32 consecutive k in [32t, 32t+32) (one NF4
+// block, one MXFP4 block).  The MMA's k index is a permutation of these
+// physical k; the activation fragment uses the same permutation.
+//   * MXFP4: e2m1 x 2^(e-127) is exact in bf16.
+//   * NF4: the code is rounded to bf16, then multiplied by bf16(absmax) and
+//     rounded again (relative error <= ~3 * 2^-9 per weight); sums are fp32.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -31,12 +34,13 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kRowsPerWarp = 16;
-constexpr int kMaxRows = 8;
-constexpr int kUnroll = 4;  // 64-k chunks whose loads are issued together
+constexpr int kRows = 64;        // weight rows per unit (4 m16 tiles)
+constexpr int kMaxTokens = 8;    // rows of a group = MMA columns
+constexpr int kDK = 128;         // k per double chunk
 
 struct GemvSmem {
-  uint32_t lut[kLutWords];
+  uint32_t lut[kLut256Words];                 // 64 KB pair table, 256-byte entry stride
+  float red[kWarps][4][32][4];                // 16 KB cross-warp partial sums
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
@@ -44,124 +48,107 @@ struct GemvSmem {
 
 template <int FMT>
 __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(GroupedArgs p) {
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   GemvSmem& s = *reinterpret_cast<GemvSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
 
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, p.err)) return;
-  const int nsl = (p.N + kRowsPerWarp - 1) / kRowsPerWarp;
-  block_exclusive_scan(p.E, s.upre, s.scratch, [&](int e) { return (s.off[e + 1] > s.off[e]) ? nsl : 0; });
+  const int nblk = (p.N + kRows - 1) / kRows;
+  block_exclusive_scan(p.E, s.upre, s.scratch, [&](int e) { return (s.off[e + 1] > s.off[e]) ? nblk : 0; });
   const int U = s.upre[p.E];
-  if ((int)blockIdx.x * kWarps >= U) return;
-  build_pair_lut<FMT>(s.lut, tid, kThreads);
+  if ((int)blockIdx.x >= U) return;
+  build_pair_lut256<FMT>(s.lut, tid, kThreads);
   __syncthreads();
 
-  const uint32_t lut_lane = smem_u32(s.lut) + (uint32_t)lane * 4u;
+  const uint8_t* lut = reinterpret_cast<const uint8_t*>(s.lut);
+  const uint32_t lane4 = (uint32_t)lane * 4u;
   const int K = p.K;
-  const int nchunk = (K + 63) / 64;
+  const int ndk = (K + kDK - 1) / kDK;
+  const int d_lo = (warp * ndk) / kWarps, d_hi = ((warp + 1) * ndk) / kWarps;
   const size_t row_bytes = (size_t)K / 2;
+  const int nsc = FMT == 0 ? K / 64 : K / 32;  // scales per weight row
 
-  for (int u = blockIdx.x * kWarps + warp; u < U; u += gridDim.x * kWarps) {
+  for (int u = blockIdx.x; u < U; u += gridDim.x) {
     const int e = find_group(s.upre, p.E, u);
-    const int sl = u - s.upre[e];
+    const int jb = u - s.upre[e];
     const int r0 = s.off[e], rows = s.off[e + 1] - r0;
-    if (rows > kMaxRows) {
-      if (lane == 0 && sl == 0) atomicOr(p.err, GNF4_DEVERR_GEMV_ROWS);
+    if (rows > kMaxTokens) {  // uniform over the CTA
+      if (tid == 0 && jb == 0) atomicOr(p.err, GNF4_DEVERR_GEMV_ROWS);
       continue;
     }
-    const int nA = sl * kRowsPerWarp + g, nB = nA + 8;
-    const bool vA = nA < p.N, vB = nB < p.N, vT = g < rows;
-    const uint8_t* wA = p.w + ((size_t)e * p.N + (vA ? nA : 0)) * row_bytes + 8 * t;
-    const uint8_t* wB = p.w + ((size_t)e * p.N + (vB ? nB : 0)) * row_bytes + 8 * t;
-    const __nv_bfloat16* xr = p.a + (size_t)(r0 + (vT ? g : 0)) * K + 16 * t;
-    const size_t sA = ((size_t)e * p.N + (vA ? nA : 0)), sB = ((size_t)e * p.N + (vB ? nB : 0));
+    // this lane's 8 weight rows: q = 2*tile + half -> row jb*64 + g + 8q
+    const int n0 = jb * kRows + g;
+    const size_t rr0 = (size_t)e * p.N + (size_t)n0;
+    const uint8_t* wbase = p.w + rr0 * row_bytes;
+    const size_t sbase = rr0 * (size_t)nsc;
+    const int nvalid_q = (p.N - n0 + 7) / 8;  // rows n0 + 8q < N  <=>  q < nvalid_q
+    const bool tv = g < rows;
+    const __nv_bfloat16* xrow = p.a + (size_t)(r0 + (tv ? g : 0)) * K;
 
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int c0 = 0; c0 < nchunk; c0 += kUnroll) {
-      uint2 qa[kUnroll], qb[kUnroll];
-      uint4 xa[kUnroll], xb[kUnroll];
-      uint32_t sa[kUnroll], sb[kUnroll];
+    float acc[4][4];
 #pragma unroll
-      for (int d = 0; d < kUnroll; ++d) {
-        const int c = c0 + d;
-        const bool inK = (c < nchunk) && (c * 64 + 16 * t < K);
-        qa[d] = (inK && vA) ? ldg_nc_u64(wA + (size_t)c * 32) : make_uint2(0u, 0u);
-        qb[d] = (inK && vB) ? ldg_nc_u64(wB + (size_t)c * 32) : make_uint2(0u, 0u);
-        if (inK && vT) {
-          xa[d] = ldg_u128(xr + (size_t)c * 64);
-          xb[d] = ldg_u128(xr + (size_t)c * 64 + 8);
-        } else {
-          xa[d] = make_uint4(0u, 0u, 0u, 0u);
-          xb[d] = make_uint4(0u, 0u, 0u, 0u);
-        }
+    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+    for (int d = d_lo; d < d_hi; ++d) {
+      const int k0 = d * kDK + 32 * t;
+      const bool inK = k0 < K;
+      uint4 wq[8];
+      uint32_t sc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const bool ok = inK && q < nvalid_q;
+        const size_t roff = (size_t)(8 * q);
+        wq[q] = ok ? ldg_nc_u128(wbase + roff * row_bytes + (k0 >> 1)) : make_uint4(0u, 0u, 0u, 0u);
         if (FMT == 0) {
-          const float* am = reinterpret_cast<const float*>(p.scales);
-          sa[d] = (inK && vA) ? __float_as_uint(__ldg(am + sA * (size_t)(K / 64) + c)) : 0u;
-          sb[d] = (inK && vB) ? __float_as_uint(__ldg(am + sB * (size_t)(K / 64) + c)) : 0u;
+          const float am =
+              ok ? __ldg(reinterpret_cast<const float*>(p.scales) + sbase + roff * (size_t)nsc + (k0 >> 6)) : 0.f;
+          const __nv_bfloat162 b2 = __float2bfloat162_rn(am);
+          sc[q] = *reinterpret_cast<const uint32_t*>(&b2);
         } else {
-          const uint8_t* sc = reinterpret_cast<const uint8_t*>(p.scales);
-          const int blk = 2 * c + (t >> 1);
-          sa[d] = (inK && vA) ? e8m0_to_bf16x2(__ldg(sc + sA * (size_t)(K / 32) + blk)) : 0u;
-          sb[d] = (inK && vB) ? e8m0_to_bf16x2(__ldg(sc + sB * (size_t)(K / 32) + blk)) : 0u;
+          sc[q] = ok ? e8m0_to_bf16x2(
+                           __ldg(reinterpret_cast<const uint8_t*>(p.scales) + sbase + roff * (size_t)nsc + (k0 >> 5)))
+                     : 0u;
         }
       }
+      uint4 xa[4];
 #pragma unroll
-      for (int d = 0; d < kUnroll; ++d) {
-        if (c0 + d >= nchunk) break;
-        uint32_t pa[8], pb[8];
-        const uint32_t wa[2] = {qa[d].x, qa[d].y}, wb[2] = {qb[d].x, qb[d].y};
+      for (int v = 0; v < 4; ++v)
+        xa[v] = (tv && inK) ? ldg_u128(xrow + k0 + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t xp[16] = {xa[0].x, xa[0].y, xa[0].z, xa[0].w, xa[1].x, xa[1].y, xa[1].z, xa[1].w,
+                               xa[2].x, xa[2].y, xa[2].z, xa[2].w, xa[3].x, xa[3].y, xa[3].z, xa[3].w};
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          pa[4 * i + 0] = lds_u32(lut_lane + ((wa[i] << 7) & 0x7F80u));
-          pa[4 * i + 1] = lds_u32(lut_lane + ((wa[i] >> 1) & 0x7F80u));
-          pa[4 * i + 2] = lds_u32(lut_lane + ((wa[i] >> 9) & 0x7F80u));
-          pa[4 * i + 3] = lds_u32(lut_lane + ((wa[i] >> 17) & 0x7F80u));
-          pb[4 * i + 0] = lds_u32(lut_lane + ((wb[i] << 7) & 0x7F80u));
-          pb[4 * i + 1] = lds_u32(lut_lane + ((wb[i] >> 1) & 0x7F80u));
-          pb[4 * i + 2] = lds_u32(lut_lane + ((wb[i] >> 9) & 0x7F80u));
-          pb[4 * i + 3] = lds_u32(lut_lane + ((wb[i] >> 17) & 0x7F80u));
-        }
-        const uint32_t xv[8] = {xa[d].x, xa[d].y, xa[d].z, xa[d].w, xb[d].x, xb[d].y, xb[d].z, xb[d].w};
-        if (FMT == 0) {
-          float blk[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i = 0; i < 4; ++i) {
+        uint32_t pa[16], pb[16];
+        decode16_lut256(lut, lane4, wq[2 * i], sc[2 * i], pa);
+        decode16_lut256(lut, lane4, wq[2 * i + 1], sc[2 * i + 1], pb);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            mma_bf16_16816(blk, pa[2 * j], pb[2 * j], pa[2 * j + 1], pb[2 * j + 1], xv[2 * j], xv[2 * j + 1]);
-          const float amA = __uint_as_float(sa[d]), amB = __uint_as_float(sb[d]);
-          acc[0] = fmaf(blk[0], amA, acc[0]);
-          acc[1] = fmaf(blk[1], amA, acc[1]);
-          acc[2] = fmaf(blk[2], amB, acc[2]);
-          acc[3] = fmaf(blk[3], amB, acc[3]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            pa[i] = bf16x2_mul(pa[i], sa[d]);
-            pb[i] = bf16x2_mul(pb[i], sb[d]);
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            mma_bf16_16816(acc, pa[2 * j], pb[2 * j], pa[2 * j + 1], pb[2 * j + 1], xv[2 * j], xv[2 * j + 1]);
-        }
+        for (int j = 0; j < 8; ++j)
+          mma_bf16_16816(acc[i], pa[2 * j], pb[2 * j], pa[2 * j + 1], pb[2 * j + 1], xp[2 * j], xp[2 * j + 1]);
       }
     }
-    // acc[0..1]: weight row nA, tokens 2t, 2t+1; acc[2..3]: row nB.
-    const int t0 = 2 * t, t1 = 2 * t + 1;
-    if (vA) {
-      if (t0 < rows) p.y[(size_t)(r0 + t0) * p.N + nA] = __float2bfloat16_rn(acc[0]);
-      if (t1 < rows) p.y[(size_t)(r0 + t1) * p.N + nA] = __float2bfloat16_rn(acc[1]);
+    // fixed-order reduction over the warps
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s.red[warp][i][lane][j] = acc[i][j];
+    __syncthreads();
+    for (int o = tid; o < 4 * 32 * 4; o += kThreads) {
+      const int i = o >> 7, l = (o >> 2) & 31, j = o & 3;
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) v += s.red[w][i][l][j];
+      const int n = jb * kRows + 16 * i + (l >> 2) + 8 * (j >> 1);
+      const int tok = 2 * (l & 3) + (j & 1);
+      if (n < p.N && tok < rows) p.y[(size_t)(r0 + tok) * p.N + n] = __float2bfloat16_rn(v);
     }
-    if (vB) {
-      if (t0 < rows) p.y[(size_t)(r0 + t0) * p.N + nB] = __float2bfloat16_rn(acc[2]);
-      if (t1 < rows) p.y[(size_t)(r0 + t1) * p.N + nB] = __float2bfloat16_rn(acc[3]);
-    }
+    __syncthreads();
   }
 }
 
 }  // namespace
 
-int gemv_warps_per_block() { return kWarps; }
-int gemv_rows_per_warp() { return kRowsPerWarp; }
+int gemv_rows_per_block() { return kRows; }
 
 template <int FMT>
 static cudaError_t launch_gemv_t(const GroupedArgs& p, int grid, cudaStream_t stream) {

@@ -31,8 +31,7 @@ cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& 
 
 // gemv.cu
 cudaError_t launch_gemv(int fmt, const GroupedArgs& p, int grid, cudaStream_t stream);
-int gemv_warps_per_block();
-int gemv_rows_per_warp();
+int gemv_rows_per_block();
 
 // route.cu
 size_t route_workspace_bytes(int T, int k, int E);
