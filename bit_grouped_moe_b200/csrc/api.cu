@@ -214,6 +214,9 @@ gnf4_status grouped_gemv(int fmt, const void* a, const uint8_t* w, const void* s
 }
 
 }  // namespace
+
+void set_last_error(const char* msg) { snprintf(t_last_error, sizeof(t_last_error), "%s", msg); }
+
 }  // namespace gnf4
 
 using namespace gnf4;

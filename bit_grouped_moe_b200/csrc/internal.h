@@ -44,6 +44,9 @@ cudaError_t launch_route(const int32_t* topk_ids, const __nv_bfloat16* x, int T,
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* flat_to_sorted, const float* weights, int T,
                            int k, int N, __nv_bfloat16* out, int num_sms, cudaStream_t stream);
 
+// api.cu: sets the text gnf4_last_error() returns on this thread
+void set_last_error(const char* msg);
+
 // dequant.cu
 cudaError_t launch_dequant(int fmt, const uint8_t* w, const void* scales, int64_t rows, int K, float* out,
                            int num_sms, cudaStream_t stream);

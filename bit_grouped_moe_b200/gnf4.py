@@ -40,12 +40,13 @@ _lib.gnf4_device_errors.argtypes = [_P, _I]
 _lib.gnf4_route_workspace_bytes.argtypes = [_I, _I, _I]
 _lib.gnf4_route_workspace_bytes.restype = _SZ
 _lib.gnf4_route_permute.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P, _P]
+_lib.gnf4_route_permute_static.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]
 for _name in ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_gemv_nf4", "gnf4_grouped_gemv_mxfp4"):
     getattr(_lib, _name).argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
 _lib.gnf4_dequant_nf4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 _lib.gnf4_dequant_mxfp4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
-for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4",
+for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", "gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4",
               "gnf4_grouped_gemv_nf4", "gnf4_grouped_gemv_mxfp4", "gnf4_combine", "gnf4_dequant_nf4_f32",
               "gnf4_dequant_mxfp4_f32"):
     getattr(_lib, _name).restype = _I
@@ -107,6 +108,23 @@ def route_permute(topk_ids, x, E, offsets, sorted_to_flat, flat_to_sorted, x_sor
                                    _ptr(flat_to_sorted), _ptr(x_sorted), _ptr(workspace),
                                    0 if workspace is None else workspace.numel() * workspace.element_size(),
                                    _ptr(bad_id_count), _stream(stream)))
+
+
+ROUTE_STATIC_SCRATCH_BYTES = 1 << 20  # GNF4_ROUTE_STATIC_SCRATCH_BYTES in include/gnf4.h
+
+
+def route_permute_static(topk_ids, x, E, offsets, sorted_to_flat, flat_to_sorted, x_sorted, bad_id_count=None,
+                         stream=None) -> None:
+    """route_permute without a workspace argument, for callers that cannot
+    allocate device memory: the scratch is a fixed array inside libgnf4 (one
+    per device, ROUTE_STATIC_SCRATCH_BYTES).  Calls that overlap on the GPU
+    share that array and must be ordered; the first call on a device does a
+    one-time address lookup and should come before any stream capture."""
+    T, k = topk_ids.shape
+    K = x.shape[1]
+    _check(_lib.gnf4_route_permute_static(_ptr(topk_ids), _ptr(x), T, k, E, K, _ptr(offsets),
+                                          _ptr(sorted_to_flat), _ptr(flat_to_sorted), _ptr(x_sorted),
+                                          _ptr(bad_id_count), _stream(stream)))
 
 
 def _grouped(fn, a, w, scales, y, offsets=None, counts=None, stream=None):

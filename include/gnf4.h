@@ -116,6 +116,31 @@ gnf4_status gnf4_route_permute(const int32_t *topk_ids, const void *x, int T, in
                                void *x_sorted, void *workspace, size_t workspace_bytes,
                                int32_t *bad_id_count, void *stream);
 
+/* Allocation-free variant of gnf4_route_permute.  The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate
+ * device memory -- e.g. a plugin inside an inference engine whose device
+ * memory is budgeted and owned by the host process, or latency-critical code
+ * that must not pay for cudaMalloc's implicit synchronisation.  It computes
+ * exactly what gnf4_route_permute computes, with the same arguments minus
+ * the workspace: its scratch is a fixed array of
+ * GNF4_ROUTE_STATIC_SCRATCH_BYTES bytes compiled into the library, one copy
+ * on every GPU that loads libgnf4, held until the process exits.
+ *  - Shapes whose scratch (gnf4_route_workspace_bytes(T, k, E)) exceeds the
+ *    array are refused with GNF4_ERR_UNSUPPORTED_SHAPE; use
+ *    gnf4_route_permute with your own workspace for those.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture begins.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; nothing in it needs to start at zero.  Calls whose executions
+ *    overlap on the GPU (different streams, no ordering between them) race
+ *    on the array: order them.
+ *  - It never calls cudaMalloc, cudaFree or any allocating routine. */
+#define GNF4_ROUTE_STATIC_SCRATCH_BYTES ((size_t)1 << 20)
+gnf4_status gnf4_route_permute_static(const int32_t *topk_ids, const void *x, int T, int k, int E, int K,
+                                      int32_t *offsets, int32_t *sorted_to_flat, int32_t *flat_to_sorted,
+                                      void *x_sorted, int32_t *bad_id_count, void *stream);
+
 /* ------------------------------------------------------------------ */
 /* Grouped GEMM (prefill: any number of rows per group)                */
 /* ------------------------------------------------------------------ */
