@@ -119,13 +119,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// A [M, K] bf16 row-major: 64 x 32 boxes (128-byte rows), 128B swizzle, zero fill.
-gnf4_status encode_act_map(CUtensorMap* m, const void* a, int M, int K) {
+// A [M, K] bf16 row-major: 64 x box_rows boxes (128-byte rows), 128B swizzle, zero fill.
+gnf4_status encode_act_map(CUtensorMap* m, const void* a, int M, int K, int box_rows = 32) {
   auto fn = encode_fn();
   if (!fn) return fail(GNF4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
   cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  cuuint32_t box[2] = {64, 32};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -179,8 +179,9 @@ gnf4_status grouped_gemm(int fmt, const void* a, const uint8_t* w, const void* s
   if (M == 0) return GNF4_OK;
   DeviceState* d = nullptr;
   GNF4_TRY(device_state(&d));
-  CUtensorMap tm_a, tm_w;
-  GNF4_TRY(encode_act_map(&tm_a, a, M, K));
+  CUtensorMap tm_a, tm_a_big, tm_w;
+  GNF4_TRY(encode_act_map(&tm_a, a, M, K, 32));
+  GNF4_TRY(encode_act_map(&tm_a_big, a, M, K, 128));
   GNF4_TRY(encode_weight_map(&tm_w, w, E, N, K));
   GroupedArgs p{static_cast<const __nv_bfloat16*>(a), w, scales, offsets, counts,
                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
@@ -191,7 +192,7 @@ gnf4_status grouped_gemm(int fmt, const void* a, const uint8_t* w, const void* s
   const long long units = chunks * nwt;
   if (units >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d, N=%d give too many work units", M, N);
   const int grid = (int)(units < d->num_sms ? units : d->num_sms);
-  cudaError_t e = launch_gemm_tc(fmt, tm_a, tm_w, p, grid, as_stream(stream));
+  cudaError_t e = launch_gemm_tc(fmt, tm_a, tm_a_big, tm_w, p, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMM launch");
   return GNF4_OK;
 }

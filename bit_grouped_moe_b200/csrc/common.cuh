@@ -99,6 +99,17 @@ __device__ __forceinline__ void build_pair_lut256(uint32_t* lut, int tid, int nt
   }
 }
 
+// fp32 -> bf16 round-to-nearest-even on the integer pipe, duplicated in both
+// halves (the hardware conversion runs on the narrow XU pipe, which a decode
+// loop would saturate).  Exact RNE for every finite input and +-Inf; a NaN
+// stays a NaN.
+__device__ __forceinline__ uint32_t f32_to_bf16x2_rn(float f) {
+  const uint32_t u = __float_as_uint(f);
+  uint32_t h = (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) h = (u >> 16) | 0x0040u;  // NaN: keep it quiet
+  return h | (h << 16);
+}
+
 __device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -156,11 +167,17 @@ __device__ __forceinline__ uint4 ldg_u128(const void* p) {
 // Decodes the 16 packed bytes of `w` (byte i = elements 2i, 2i+1 of 32
 // codes) into 16 bf16x2 pairs multiplied by the bf16x2 scale `sc`.
 // `lane4` = 4 * lane; the table is the 256-byte-stride pair table.
-__device__ __forceinline__ uint32_t lut256_get(const uint8_t* lut, uint32_t word, uint32_t lane4, uint32_t j) {
-  return *reinterpret_cast<const uint32_t*>(lut + prmt_b32(word, lane4, 0x5504u | (j << 4)));
+// Table lookup with 32-bit shared-memory addressing: the PRMT result is the
+// byte offset inside the table and `lut` its shared-window address, so the
+// lookup is one PRMT and one shared load.  (Not volatile: the table is
+// read-only once built, so the compiler may schedule the loads freely.)
+__device__ __forceinline__ uint32_t lut256_get(uint32_t lut, uint32_t word, uint32_t lane4, uint32_t j) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(lut + prmt_b32(word, lane4, 0x5504u | (j << 4))));
+  return v;
 }
 
-__device__ __forceinline__ void decode16_lut256(const uint8_t* lut, uint32_t lane4, uint4 w, uint32_t sc,
+__device__ __forceinline__ void decode16_lut256(uint32_t lut, uint32_t lane4, uint4 w, uint32_t sc,
                                                 uint32_t (&out)[16]) {
   const uint32_t words[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -240,6 +257,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "[%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+
+// 4-byte asynchronous global -> shared copy (both addresses 4-byte aligned).
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// Arrives on `bar` once every cp.async this thread issued so far has landed
+// (the barrier's expected count must include this arrival).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Orders this thread's earlier generic-proxy shared-memory accesses before

@@ -17,15 +17,18 @@
 //    chunk, so CTAs running at the same time share weight tiles in L2.  The
 //    list is derived on the device from the group offsets (no host sync, no
 //    tile list in global memory); a persistent grid strides over it.
-//  * Three decoupled rings keep enough bytes in flight: packed weights (12
-//    stages x 4 KB, its own TMA thread), activation tiles (6 stages x 16 KB,
+//  * Decoupled rings keep enough bytes in flight: packed weights (10
+//    stages x 4 KB, its own TMA thread), activation tiles (5 stages x 16 KB,
 //    its own TMA thread) and decoded weights in TMEM (8 stages x 32 columns),
 //    plus two TMEM accumulators so the epilogue of one unit overlaps the
 //    main loop of the next.
-//  * Warp roles (18 warps): 0 = weight TMA, 1 = TMEM owner + MMA issuer,
-//    2 = activation TMA, 4..15 = decode (three groups of four taking k-stages
-//    in turn; warp w owns TMEM lanes 32*(w%4)..+31, i.e. weight rows),
-//    16..19 = epilogue.
+//  * Warp roles (22 warps): 0 and 20 = weight TMA (alternate stages), 1 =
+//    TMEM owner + MMA issuer, 2 and 21 = activation TMA (alternate stages; a
+//    group of more than 32 rows comes as one 128-row box), 3 = scale loader (raw block scales copied into a
+//    shared-memory ring with cp.async, 8 k-stages per chunk, 3 chunks ahead,
+//    so decode never waits on a global load), 4..15 = decode (three groups of
+//    four taking k-stages in turn; warp w owns TMEM lanes 32*(w%4)..+31, i.e.
+//    weight rows), 16..19 = epilogue.
 //  * Decode: a thread owns one weight row; per 64-k stage it reads its 32
 //    packed bytes from shared memory, and for every byte builds the address
 //    of a lane-private pair-table entry with one PRMT, loads the two bf16
@@ -43,13 +46,19 @@ namespace {
 constexpr int kBT = 128;   // activation rows (tokens) per unit = max MMA N
 constexpr int kBW = 128;   // weight rows per unit = MMA M
 constexpr int kBK = 64;    // k per stage
-constexpr int kWStages = 12;
-constexpr int kAStages = 6;
+constexpr int kWStages = 10;
+constexpr int kAStages = 5;
 constexpr int kTStages = 8;
+constexpr int kSChunk = 8;       // k-stages per scale chunk
+constexpr int kSStages = 3;      // scale chunks in flight
+constexpr int kSRowWords = 9;    // raw scale words per row per chunk (NF4 8, MXFP4 5), padded
 constexpr int kDecGroups = 3;
 constexpr int kDecWarp0 = 4;
 constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;  // 16
-constexpr int kThreads = (kEpiWarp0 + 4) * 32;        // 640
+constexpr int kWProd2 = kEpiWarp0 + 4;                 // 20: second weight producer
+constexpr int kAProd2 = kWProd2 + 1;                   // 21: second activation producer
+constexpr int kThreads = (kAProd2 + 1) * 32;           // 704
+constexpr int kBigBox = 128;                           // activation rows per TMA box for large groups
 constexpr int kAccCols = 2 * kBT;                      // two fp32 accumulators
 constexpr int kACol0 = kAccCols;                       // decoded-weight ring
 constexpr int kTmemCols = 512;
@@ -62,12 +71,14 @@ struct Smem {
   uint8_t act[kAStages][kActStageBytes];  // 1024-aligned (offset 0)
   uint32_t lut[kLut256Words];             // 64 KB
   uint8_t wq[kWStages][kWStageBytes];
+  uint32_t sring[kSStages][kBW][kSRowWords];  // raw block scales of kSChunk k-stages per row
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
   uint64_t wfull[kWStages], wempty[kWStages];
   uint64_t afull[kAStages], aempty[kAStages];
   uint64_t tfull[kTStages], tempty[kTStages];
+  uint64_t sfull[kSStages], sempty[kSStages];
   uint64_t accf[2], acce[2];
   uint64_t mdone;  // abort path only: every issued MMA has retired
   uint32_t tmem_base;
@@ -94,8 +105,8 @@ __device__ __forceinline__ Unit unit_of(const Smem& s, int E, int u) {
 
 template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
-                   GroupedArgs p) {
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_big,
+                   const __grid_constant__ CUtensorMap tm_w, GroupedArgs p) {
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -124,6 +135,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.tfull[i], 4);
       mbar_init(&s.tempty[i], 1);
     }
+    for (int i = 0; i < kSStages; ++i) {
+      mbar_init(&s.sfull[i], 32);
+      mbar_init(&s.sempty[i], 4 * kDecGroups);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.accf[i], 1);
       mbar_init(&s.acce[i], 4);
@@ -134,6 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_a_big);
     prefetch_tmap(&tm_w);
   }
   if (warp == 1) {
@@ -145,14 +161,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == kWProd2) {
     // ------------------------------------------------------------ weight TMA
+    // Two producer threads take the k-stages in turn: an SM completes about
+    // one box per issuing thread per memory latency, so one producer alone
+    // would cap the weight stream (measured on B200).
+    const int pi = warp == 0 ? 0 : 1;
     if (lane == 0) {
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const Unit x = unit_of(s, p.E, u);
         for (int kt = 0; kt < nk; ++kt, ++it) {
+          if ((it & 1) != pi) continue;
           const int st = it % kWStages, use = it / kWStages;
           if (it >= kWStages && !(ok = mbar_wait(&s.wempty[st], (use - 1) & 1, err, abort))) break;
           mbar_arrive_expect_tx(&s.wfull[st], kWStageBytes);
@@ -160,26 +181,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok)  // drain loads still in flight before shared memory goes away
-        for (int i = max(0, it - kWStages); i < it; ++i) mbar_drain(&s.wfull[i % kWStages], (i / kWStages) & 1);
+        for (int i = max(0, it - kWStages); i < it; ++i)
+          if ((i & 1) == pi) mbar_drain(&s.wfull[i % kWStages], (i / kWStages) & 1);
     }
-  } else if (warp == 2) {
+  } else if (warp == 2 || warp == kAProd2) {
     // ------------------------------------------------------------ activation TMA
+    // Two producer threads alternate stages; a group of more than 32 rows is
+    // loaded as one 128-row box, a smaller one as one 32-row box.
+    const int pi = warp == 2 ? 0 : 1;
     if (lane == 0) {
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const Unit x = unit_of(s, p.E, u);
-        const int nbox = (x.rows + kActBox - 1) / kActBox;
+        const bool big = x.rows > kActBox;
         for (int kt = 0; kt < nk; ++kt, ++it) {
+          if ((it & 1) != pi) continue;
           const int st = it % kAStages, use = it / kAStages;
           if (it >= kAStages && !(ok = mbar_wait(&s.aempty[st], (use - 1) & 1, err, abort))) break;
-          mbar_arrive_expect_tx(&s.afull[st], nbox * kActBox * 128);
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d(s.act[st] + b * kActBox * 128, &tm_a, &s.afull[st], kt * kBK, x.row0 + b * kActBox);
+          if (big) {
+            mbar_arrive_expect_tx(&s.afull[st], kBigBox * 128);
+            tma_load_2d(s.act[st], &tm_a_big, &s.afull[st], kt * kBK, x.row0);
+          } else {
+            mbar_arrive_expect_tx(&s.afull[st], kActBox * 128);
+            tma_load_2d(s.act[st], &tm_a, &s.afull[st], kt * kBK, x.row0);
+          }
         }
       }
       if (!ok)
-        for (int i = max(0, it - kAStages); i < it; ++i) mbar_drain(&s.afull[i % kAStages], (i / kAStages) & 1);
+        for (int i = max(0, it - kAStages); i < it; ++i)
+          if ((i & 1) == pi) mbar_drain(&s.afull[i % kAStages], (i / kAStages) & 1);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ scale loader
+    // Copies the raw block scales of the next kSChunk k-stages of every
+    // weight row into a shared-memory ring with 4-byte cp.async, three
+    // chunks ahead, so decode never waits on a global load.  NF4: the 8
+    // absmax floats of the chunk; MXFP4: the 5 aligned words that cover the
+    // chunk's 16 scale bytes.  Lane l serves rows l, l+32, l+64, l+96.
+    const int nsc = FMT == 0 ? p.K / 64 : p.K / 32;
+    int ci = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+      const Unit x = unit_of(s, p.E, u);
+      for (int kt0 = 0; kt0 < nk; kt0 += kSChunk, ++ci) {
+        const int slot = ci % kSStages;
+        if (ci >= kSStages && !(ok = mbar_wait(&s.sempty[slot], ((ci / kSStages) - 1) & 1, err, abort))) break;
+#pragma unroll
+        for (int m = 0; m < kBW / 32; ++m) {
+          const int r = lane + 32 * m;
+          const int n = x.j * kBW + r;
+          if (n >= p.N) continue;
+          const size_t rowsc = ((size_t)x.e * p.N + (size_t)n) * (size_t)nsc;
+          if (FMT == 0) {
+            const float* src = reinterpret_cast<const float*>(p.scales) + rowsc + kt0;
+            const int cnt = min(kSChunk, nk - kt0);
+            for (int q = 0; q < cnt; ++q) cp_async_4(&s.sring[slot][r][q], src + q);
+          } else {
+            const uint8_t* base = reinterpret_cast<const uint8_t*>(p.scales);
+            const size_t b0 = rowsc + 2 * (size_t)kt0;               // first scale byte of the chunk
+            const size_t b1 = min(rowsc + (size_t)nsc, b0 + 2 * kSChunk);  // one past the last
+            const size_t w0 = b0 & ~(size_t)3;
+            for (size_t wq = w0, q = 0; wq < b1; wq += 4, ++q) cp_async_4(&s.sring[slot][r][q], base + wq);
+          }
+        }
+        cp_async_arrive_noinc(&s.sfull[slot]);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -219,61 +286,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ decode
     const int grp = (warp - kDecWarp0) >> 2, q = warp & 3;
     const int nl = q * 32 + lane;
-    const uint8_t* lut = reinterpret_cast<const uint8_t*>(s.lut);
+    const uint32_t lut = smem_u32(s.lut);
     const uint32_t lane4 = (uint32_t)lane * 4u;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
-    int it = 0;
+    int it = 0, ci = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-      const Unit x = unit_of(s, p.E, u);
-      const int n = x.j * kBW + nl;
-      const bool nvalid = n < p.N;
-      const size_t srow = (size_t)x.e * p.N + (size_t)(nvalid ? n : 0);
+      const Unit xu = unit_of(s, p.E, u);
       for (int kt = 0; kt < nk; ++kt, ++it) {
-        if (it % kDecGroups != grp) continue;
-        const int sw = it % kWStages, sT = it % kTStages;
-        if (!(ok = mbar_wait(&s.wfull[sw], (it / kWStages) & 1, err, abort))) break;
-        if (it >= kTStages && !(ok = mbar_wait(&s.tempty[sT], ((it / kTStages) - 1) & 1, err, abort))) break;
-        uint32_t sc0 = 0, sc1 = 0;
-        if (nvalid) {
+        const int q8 = kt % kSChunk, slot = ci % kSStages;
+        if (q8 == 0 && !(ok = mbar_wait(&s.sfull[slot], (ci / kSStages) & 1, err, abort))) break;
+        if (it % kDecGroups == grp) {
+          const int sw = it % kWStages, sT = it % kTStages;
+          if (!(ok = mbar_wait(&s.wfull[sw], (it / kWStages) & 1, err, abort))) break;
+          if (it >= kTStages && !(ok = mbar_wait(&s.tempty[sT], ((it / kTStages) - 1) & 1, err, abort))) break;
+          uint32_t sc0, sc1;
           if (FMT == 0) {
-            const float am = __ldg(reinterpret_cast<const float*>(p.scales) + srow * (size_t)(p.K / 64) + kt);
-            const __nv_bfloat162 b2 = __float2bfloat162_rn(am);
-            sc0 = sc1 = *reinterpret_cast<const uint32_t*>(&b2);
+            sc0 = sc1 = f32_to_bf16x2_rn(__uint_as_float(s.sring[slot][nl][q8]));
           } else {
-            const uint8_t* sp = reinterpret_cast<const uint8_t*>(p.scales) + srow * (size_t)(p.K / 32) + 2 * kt;
-            sc0 = e8m0_to_bf16x2(__ldg(sp));
-            sc1 = (2 * kt + 1 < p.K / 32) ? e8m0_to_bf16x2(__ldg(sp + 1)) : 0u;
+            // bytes of the chunk start at (row offset & 3) inside the copied words
+            const size_t rowsc = ((size_t)xu.e * p.N + (size_t)(xu.j * kBW + nl)) * (size_t)(p.K / 32);
+            const uint32_t b = (uint32_t)(rowsc & 3u) + 2u * (uint32_t)q8;
+            const uint8_t* bytes = reinterpret_cast<const uint8_t*>(s.sring[slot][nl]);
+            sc0 = e8m0_to_bf16x2(bytes[b]);
+            sc1 = (2 * kt + 1 < p.K / 32) ? e8m0_to_bf16x2(bytes[b + 1]) : 0u;
           }
-        }
-        // two 16-byte reads of this row's 32 bytes, ordered so a quarter warp
-        // touches 8 distinct 16-byte bank groups
-        const uint32_t wrow = smem_u32(s.wq[sw]) + (uint32_t)nl * 32u;
-        const uint32_t c_first = ((uint32_t)nl >> 2) & 1u;
-        uint4 c0 = lds_u128(wrow + 16u * c_first), c1 = lds_u128(wrow + 16u * (c_first ^ 1u));
-        if (c_first) {
-          const uint4 tmp = c0;
-          c0 = c1;
-          c1 = tmp;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.wempty[sw]);  // packed bytes are in registers now
-        uint32_t v[32];
-        {
-          uint32_t h0[16], h1[16];
-          decode16_lut256(lut, lane4, c0, sc0, h0);
-          decode16_lut256(lut, lane4, c1, sc1, h1);
+          // two 16-byte reads of this row's 32 bytes, ordered so a quarter warp
+          // touches 8 distinct 16-byte bank groups
+          const uint32_t wrow = smem_u32(s.wq[sw]) + (uint32_t)nl * 32u;
+          const uint32_t c_first = ((uint32_t)nl >> 2) & 1u;
+          uint4 c0 = lds_u128(wrow + 16u * c_first), c1 = lds_u128(wrow + 16u * (c_first ^ 1u));
+          if (c_first) {
+            const uint4 tmp = c0;
+            c0 = c1;
+            c1 = tmp;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.wempty[sw]);  // packed bytes are in registers now
+          uint32_t v[32];
+          {
+            uint32_t h0[16], h1[16];
+            decode16_lut256(lut, lane4, c0, sc0, h0);
+            decode16_lut256(lut, lane4, c1, sc1, h1);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            v[i] = h0[i];
-            v[16 + i] = h1[i];
+            for (int i = 0; i < 16; ++i) {
+              v[i] = h0[i];
+              v[16 + i] = h1[i];
+            }
           }
+          tmem_st_32x32b_x32(t_lane + (uint32_t)(kACol0 + sT * (kBK / 2)), v);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.tfull[sT]);
         }
-        tmem_st_32x32b_x32(t_lane + (uint32_t)(kACol0 + sT * (kBK / 2)), v);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.tfull[sT]);
+        if (q8 == kSChunk - 1 || kt == nk - 1) {  // this warp is done with the chunk
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.sempty[slot]);
+          ++ci;
+        }
       }
     }
   } else if (warp >= kEpiWarp0) {
@@ -320,8 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 size_t gemm_tc_smem_bytes() { return sizeof(Smem) + 1024; }
 
 template <int FMT>
-cudaError_t launch_gemm_tc_t(const CUtensorMap& tm_a, const CUtensorMap& tm_w, const GroupedArgs& p, int grid,
-                             cudaStream_t stream) {
+cudaError_t launch_gemm_tc_t(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
+                             const GroupedArgs& p, int grid, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -331,14 +402,14 @@ cudaError_t launch_gemm_tc_t(const CUtensorMap& tm_a, const CUtensorMap& tm_w, c
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  gemm_tc_kernel<FMT><<<grid, kThreads, gemm_tc_smem_bytes(), stream>>>(tm_a, tm_w, p);
+  gemm_tc_kernel<FMT><<<grid, kThreads, gemm_tc_smem_bytes(), stream>>>(tm_a, tm_a_big, tm_w, p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& tm_w, const GroupedArgs& p,
-                           int grid, cudaStream_t stream) {
-  return fmt == 0 ? launch_gemm_tc_t<0>(tm_a, tm_w, p, grid, stream)
-                  : launch_gemm_tc_t<1>(tm_a, tm_w, p, grid, stream);
+cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
+                           const GroupedArgs& p, int grid, cudaStream_t stream) {
+  return fmt == 0 ? launch_gemm_tc_t<0>(tm_a, tm_a_big, tm_w, p, grid, stream)
+                  : launch_gemm_tc_t<1>(tm_a, tm_a_big, tm_w, p, grid, stream);
 }
 
 int gemm_tc_rows_per_unit() { return kBT; }

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(GroupedArgs p) {
   build_pair_lut256<FMT>(s.lut, tid, kThreads);
   __syncthreads();
 
-  const uint8_t* lut = reinterpret_cast<const uint8_t*>(s.lut);
+  const uint32_t lut = smem_u32(s.lut);
   const uint32_t lane4 = (uint32_t)lane * 4u;
   const int K = p.K;
   const int ndk = (K + kDK - 1) / kDK;
@@ -103,8 +103,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(GroupedArgs p) {
         if (FMT == 0) {
           const float am =
               ok ? __ldg(reinterpret_cast<const float*>(p.scales) + sbase + roff * (size_t)nsc + (k0 >> 6)) : 0.f;
-          const __nv_bfloat162 b2 = __float2bfloat162_rn(am);
-          sc[q] = *reinterpret_cast<const uint32_t*>(&b2);
+          sc[q] = f32_to_bf16x2_rn(am);
         } else {
           sc[q] = ok ? e8m0_to_bf16x2(
                            __ldg(reinterpret_cast<const uint8_t*>(p.scales) + sbase + roff * (size_t)nsc + (k0 >> 5)))

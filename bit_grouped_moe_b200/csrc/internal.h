@@ -26,8 +26,8 @@ struct GroupedArgs {
 size_t gemm_tc_smem_bytes();
 int gemm_tc_rows_per_unit();
 int gemm_tc_weight_rows_per_unit();
-cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& tm_w, const GroupedArgs& p,
-                           int grid, cudaStream_t stream);
+cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
+                           const GroupedArgs& p, int grid, cudaStream_t stream);
 
 // gemv.cu
 cudaError_t launch_gemv(int fmt, const GroupedArgs& p, int grid, cudaStream_t stream);
