@@ -207,8 +207,7 @@ gnf4_status grouped_gemv(int fmt, const void* a, const uint8_t* w, const void* s
                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
   const long long hit = E < M ? E : M;  // groups with rows
   const long long blocks = hit * ((N + gemv_rows_per_block() - 1) / gemv_rows_per_block());
-  const long long cap = 2LL * d->num_sms;
-  const int grid = (int)(blocks < cap ? blocks : cap);
+  const int grid = gemv_grid(blocks, d->num_sms);
   cudaError_t e = launch_gemv(fmt, p, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMV launch");
   return GNF4_OK;

@@ -6,21 +6,32 @@
 // row (same page, limitations); here every weight byte is read once and used
 // for all of its group's rows.
 //
-// Work unit = one CTA x (expert e, 64 consecutive weight rows).  The 8 warps
-// split K: warp w takes a contiguous range of 128-k "double chunks" and
+// Work unit = (expert e, 64 consecutive weight rows).  A CTA (one per SM,
+// 16 warps) runs two units at a time, one per half of 8 warps; the 8 warps of
+// a half split K: warp s takes a contiguous range of 128-k "items" and
 // computes the partial sums of all 64 rows (four m16 tiles) for the group's
 // <= 8 rows (the MMA's 8 columns); a fixed-order shared-memory reduction over
-// the warps finishes the unit.  Per double chunk a lane loads 16 bytes (32
-// codes) of each of its 8 weight rows with one 16-byte load each, decodes
-// every byte with one PRMT (which builds the table address) and one shared
-// load from a lane-private copy of the pair table, multiplies the bf16 pair
-// by the row's block scale, and feeds the pairs to m16n8k16 warp MMAs.  The
-// MMA does the k reduction that a CUDA-core GEMV would do with shuffles.
+// the 8 warps finishes the unit.  Per item a lane holds 16 bytes (32 codes)
+// of each of its 8 weight rows, decodes every byte with one PRMT, which
+// builds the shared-memory address of a lane-private pair-table entry, and
+// one shared load, multiplies the bf16 pair by the row's block scale, and
+// feeds the pairs to m16n8k16 warp MMAs.  The MMA does the k reduction that
+// a CUDA-core GEMV would do with shuffles.
+//
+// Latency hiding: a warp's items form one stream across unit boundaries, and
+// the loads of the next item are issued tile by tile while the current item
+// is decoded (each tile's registers are refilled as soon as they have been
+// decoded), so every warp always has about one item (4 KB) in flight without
+// a second register set.
+//
+// The pair table sits at shared-window address 0x10000 (one copy per SM, 64
+// KB): the PRMT that extracts a byte also inserts the table's base, so a
+// lookup is exactly one PRMT and one shared load.
 //
 // Lane (g, t) = (lane / 4, lane % 4) owns rows g and g+8 of every tile and,
-// in every double chunk, the 32 consecutive k in [32t, 32t+32) (one NF4
-// block, one MXFP4 block).  The MMA's k index is a permutation of these
-// physical k; the activation fragment uses the same permutation.
+// in every item, the 32 consecutive k in [32t, 32t+32) (one NF4 half-block,
+// one MXFP4 block).  The MMA's k index is a permutation of these physical k;
+// the activation fragment uses the same permutation.
 //   * MXFP4: e2m1 x 2^(e-127) is exact in bf16.
 //   * NF4: the code is rounded to bf16, then multiplied by bf16(absmax) and
 //     rounded again (relative error <= ~3 * 2^-9 per weight); sums are fp32.
@@ -32,140 +43,242 @@
 namespace gnf4 {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kRows = 64;        // weight rows per unit (4 m16 tiles)
-constexpr int kMaxTokens = 8;    // rows of a group = MMA columns
-constexpr int kDK = 128;         // k per double chunk
+constexpr int kSplit = 8;                 // warps per half = K-splits of a unit
+constexpr int kRows = 64;                 // weight rows per unit (4 m16 tiles)
+constexpr int kMaxTokens = 8;             // rows of a group = MMA columns
+constexpr int kDK = 128;                  // k per item
+constexpr uint32_t kLutWindow = 0x10000u;  // shared-window address of the pair table
+constexpr int kSmemBytes = 0x20000;        // dynamic shared memory per CTA
 
-struct GemvSmem {
-  uint32_t lut[kLut256Words];                 // 64 KB pair table, 256-byte entry stride
-  float red[kWarps][4][32][4];                // 16 KB cross-warp partial sums
+// Everything but the pair table; lives below kLutWindow.
+struct GemvLow {
+  float red[2][kSplit][4][32][4];  // 32 KB: partial sums per half and K-split
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
 };
 
+// f32 -> bf16 (round to nearest even, NaN kept quiet), duplicated in both halves.
+__device__ __forceinline__ uint32_t cvt_bf16x2_dup(float f) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(d) : "f"(f));
+  return d;
+}
+
+// One pair-table lookup: byte j of `word` selects the entry; `lanesel` holds
+// 4*lane in byte 0 and the table base's byte 2 (0x01) in byte 2.
+__device__ __forceinline__ uint32_t lut_lookup(uint32_t word, uint32_t lanesel, uint32_t j) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(prmt_b32(word, lanesel, 0x7604u | (j << 4))));
+  return v;
+}
+
+__device__ __forceinline__ void half_barrier(int h) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + h), "r"(kThreads / 2) : "memory");
+}
+
+// Per-lane view of one unit: where this lane's rows, scales and activation row start.
+struct UnitView {
+  const uint8_t* w;            // weight row n0 (q = 0), byte 0
+  const uint8_t* sc;           // first scale of row n0 (bytes)
+  const __nv_bfloat16* x;      // activation row of token g (row 0 if g >= rows), k = 32t
+  int qv;                      // rows n0 + 8q < N  <=>  q < qv
+  bool tv;                     // token g exists
+};
+
 template <int FMT>
-__global__ void __launch_bounds__(kThreads, 2) gemv_kernel(GroupedArgs p) {
+__device__ __forceinline__ UnitView unit_view(const GemvLow& s, const GroupedArgs& p, int u, int g, int t) {
+  const int e = find_group(s.upre, p.E, u);
+  const int jb = u - s.upre[e];
+  const int r0 = s.off[e], rows = s.off[e + 1] - r0;
+  const int n0 = jb * kRows + g;
+  const size_t row = (size_t)e * p.N + (size_t)n0;
+  const int nsc = FMT == 0 ? p.K / 64 : p.K / 32;
+  UnitView v;
+  v.w = p.w + row * (size_t)(p.K / 2);
+  v.sc = reinterpret_cast<const uint8_t*>(p.scales) + row * (size_t)nsc * (FMT == 0 ? 4u : 1u);
+  v.tv = g < rows;
+  v.x = p.a + (size_t)(r0 + (v.tv ? g : 0)) * p.K + 32 * t;
+  v.qv = (p.N - n0 + 7) / 8;
+  return v;
+}
+
+// Loads of one item for tile i (rows q = 2i, 2i+1): packed weights and raw scales.
+template <int FMT, bool FULLN>
+__device__ __forceinline__ void load_tile(const UnitView& v, int d, int t, int K, size_t rs8, size_t ss8, int i,
+                                          uint4 (&wq)[8], uint32_t (&sr)[8]) {
+  const bool inK = d * kDK + 32 * t < K;
+  const size_t kb = inK ? (size_t)(d * (kDK / 2) + 16 * t) : 0;  // outside K: any valid address
+  const size_t si = inK ? (size_t)(FMT == 0 ? 2 * d + (t >> 1) : 4 * d + t) : 0;
+#pragma unroll
+  for (int hq = 0; hq < 2; ++hq) {
+    const int q = 2 * i + hq;
+    const int qe = FULLN ? q : min(q, v.qv - 1);
+    wq[q] = ldg_nc_u128(v.w + (size_t)qe * rs8 + kb);
+    if (FMT == 0)
+      sr[q] = __ldg(reinterpret_cast<const unsigned int*>(v.sc + ((size_t)qe * ss8 + si) * 4u));
+    else
+      sr[q] = __ldg(v.sc + (size_t)qe * ss8 + si);
+  }
+}
+
+__device__ __forceinline__ void load_acts(const UnitView& v, int d, int t, int K, uint4 (&xa)[4]) {
+  const bool ok = v.tv && (d * kDK + 32 * t < K);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) xa[c] = ok ? ldg_u128(v.x + d * kDK + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+}
+
+template <int FMT>
+__device__ __forceinline__ uint32_t scale_pair(uint32_t raw) {
+  return FMT == 0 ? cvt_bf16x2_dup(__uint_as_float(raw)) : e8m0_to_bf16x2(raw);
+}
+
+template <int FMT, bool FULLN>
+__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  GemvSmem& s = *reinterpret_cast<GemvSmem*>(smem_raw);
+  GemvLow& s = *reinterpret_cast<GemvLow*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
+  const int h = warp / kSplit, ks = warp % kSplit;
 
+  // The table must occupy [kLutWindow, kLutWindow + 64 KB) of this CTA's
+  // shared window, with GemvLow below it.
+  const uint32_t base = smem_u32(smem_raw);
+  if (base + (uint32_t)sizeof(GemvLow) > kLutWindow ||
+      base + (uint32_t)kSmemBytes < kLutWindow + (uint32_t)kLut256Bytes) {
+    if (tid == 0) atomicOr(p.err, GNF4_DEVERR_INTERNAL);
+    return;
+  }
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, p.err)) return;
   const int nblk = (p.N + kRows - 1) / kRows;
   block_exclusive_scan(p.E, s.upre, s.scratch, [&](int e) { return (s.off[e + 1] > s.off[e]) ? nblk : 0; });
   const int U = s.upre[p.E];
-  if ((int)blockIdx.x >= U) return;
-  build_pair_lut256<FMT>(s.lut, tid, kThreads);
-  __syncthreads();
+  if (2 * (int)blockIdx.x >= U) return;  // uniform over the CTA
 
-  const uint32_t lut = smem_u32(s.lut);
-  const uint32_t lane4 = (uint32_t)lane * 4u;
   const int K = p.K;
   const int ndk = (K + kDK - 1) / kDK;
-  const int d_lo = (warp * ndk) / kWarps, d_hi = ((warp + 1) * ndk) / kWarps;
-  const size_t row_bytes = (size_t)K / 2;
-  const int nsc = FMT == 0 ? K / 64 : K / 32;  // scales per weight row
+  const int d_lo = (ks * ndk) / kSplit, d_hi = ((ks + 1) * ndk) / kSplit;
+  const size_t rs8 = (size_t)8 * (size_t)(K / 2);                 // bytes between rows q and q+1
+  const size_t ss8 = (size_t)8 * (size_t)(FMT == 0 ? K / 64 : K / 32);  // scales between rows q and q+1
+  const int ustride = 2 * (int)gridDim.x;
+  int u = 2 * (int)blockIdx.x + h;
 
-  for (int u = blockIdx.x; u < U; u += gridDim.x) {
-    const int e = find_group(s.upre, p.E, u);
-    const int jb = u - s.upre[e];
-    const int r0 = s.off[e], rows = s.off[e + 1] - r0;
-    if (rows > kMaxTokens) {  // uniform over the CTA
-      if (tid == 0 && jb == 0) atomicOr(p.err, GNF4_DEVERR_GEMV_ROWS);
-      continue;
+  // first item of this warp's stream, issued before the table is built
+  uint4 wq[8], xa[4];
+  uint32_t sr[8];
+  UnitView cur{};
+  if (u < U) {
+    cur = unit_view<FMT>(s, p, u, g, t);
+    if (d_lo < d_hi) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) load_tile<FMT, FULLN>(cur, d_lo, t, K, rs8, ss8, i, wq, sr);
+      load_acts(cur, d_lo, t, K, xa);
     }
-    // this lane's 8 weight rows: q = 2*tile + half -> row jb*64 + g + 8q
-    const int n0 = jb * kRows + g;
-    const size_t rr0 = (size_t)e * p.N + (size_t)n0;
-    const uint8_t* wbase = p.w + rr0 * row_bytes;
-    const size_t sbase = rr0 * (size_t)nsc;
-    const int nvalid_q = (p.N - n0 + 7) / 8;  // rows n0 + 8q < N  <=>  q < nvalid_q
-    const bool tv = g < rows;
-    const __nv_bfloat16* xrow = p.a + (size_t)(r0 + (tv ? g : 0)) * K;
+  }
+  build_pair_lut256<FMT>(reinterpret_cast<uint32_t*>(smem_raw + (kLutWindow - base)), tid, kThreads);
+  __syncthreads();
 
+  const uint32_t lanesel = (uint32_t)lane * 4u | (kLutWindow & 0x00FF0000u);
+
+  for (; u < U; u += ustride) {  // uniform over the half
     float acc[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 
     for (int d = d_lo; d < d_hi; ++d) {
-      const int k0 = d * kDK + 32 * t;
-      const bool inK = k0 < K;
-      uint4 wq[8];
-      uint32_t sc[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const bool ok = inK && q < nvalid_q;
-        const size_t roff = (size_t)(8 * q);
-        wq[q] = ok ? ldg_nc_u128(wbase + roff * row_bytes + (k0 >> 1)) : make_uint4(0u, 0u, 0u, 0u);
-        if (FMT == 0) {
-          const float am =
-              ok ? __ldg(reinterpret_cast<const float*>(p.scales) + sbase + roff * (size_t)nsc + (k0 >> 6)) : 0.f;
-          sc[q] = f32_to_bf16x2_rn(am);
-        } else {
-          sc[q] = ok ? e8m0_to_bf16x2(
-                           __ldg(reinterpret_cast<const uint8_t*>(p.scales) + sbase + roff * (size_t)nsc + (k0 >> 5)))
-                     : 0u;
-        }
-      }
-      uint4 xa[4];
-#pragma unroll
-      for (int v = 0; v < 4; ++v)
-        xa[v] = (tv && inK) ? ldg_u128(xrow + k0 + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+      // The next item of this warp's stream is (u, d+1), or the first item of
+      // the next unit.  The current item's loads were issued one iteration
+      // ago, so `cur` can already describe the unit of the next item.
+      const bool last = d + 1 == d_hi;
+      const int dn = last ? d_lo : d + 1;
+      const bool has_next = !last || u + ustride < U;
+      if (last && has_next) cur = unit_view<FMT>(s, p, u + ustride, g, t);
+      uint4 xn[4];
+      if (has_next) load_acts(cur, dn, t, K, xn);
+
       const uint32_t xp[16] = {xa[0].x, xa[0].y, xa[0].z, xa[0].w, xa[1].x, xa[1].y, xa[1].z, xa[1].w,
                                xa[2].x, xa[2].y, xa[2].z, xa[2].w, xa[3].x, xa[3].y, xa[3].z, xa[3].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        uint32_t pa[16], pb[16];
-        decode16_lut256(lut, lane4, wq[2 * i], sc[2 * i], pa);
-        decode16_lut256(lut, lane4, wq[2 * i + 1], sc[2 * i + 1], pb);
+        const uint32_t s0 = scale_pair<FMT>(sr[2 * i]), s1 = scale_pair<FMT>(sr[2 * i + 1]);
+        const uint32_t w0[4] = {wq[2 * i].x, wq[2 * i].y, wq[2 * i].z, wq[2 * i].w};
+        const uint32_t w1[4] = {wq[2 * i + 1].x, wq[2 * i + 1].y, wq[2 * i + 1].z, wq[2 * i + 1].w};
+        // MMA step j takes bytes 2j, 2j+1 of both rows (word j/2, bytes 2(j%2) and 2(j%2)+1)
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          mma_bf16_16816(acc[i], pa[2 * j], pb[2 * j], pa[2 * j + 1], pb[2 * j + 1], xp[2 * j], xp[2 * j + 1]);
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t b0 = 2u * (uint32_t)(j & 1);
+          const uint32_t a0 = bf16x2_mul(lut_lookup(w0[j >> 1], lanesel, b0), s0);
+          const uint32_t a1 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0), s1);
+          const uint32_t a2 = bf16x2_mul(lut_lookup(w0[j >> 1], lanesel, b0 + 1u), s0);
+          const uint32_t a3 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0 + 1u), s1);
+          mma_bf16_16816(acc[i], a0, a1, a2, a3, xp[2 * j], xp[2 * j + 1]);
+        }
+        if (has_next) load_tile<FMT, FULLN>(cur, dn, t, K, rs8, ss8, i, wq, sr);
+      }
+      if (has_next) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) xa[c] = xn[c];
       }
     }
-    // fixed-order reduction over the warps
+
+    // fixed-order reduction over the half's 8 warps
 #pragma unroll
     for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4*>(&s.red[h][ks][i][lane][0]) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    half_barrier(h);
+    {
+      const int e = find_group(s.upre, p.E, u);
+      const int jb = u - s.upre[e];
+      const int r0 = s.off[e], rows = s.off[e + 1] - r0;
+      const int ht = tid & (kThreads / 2 - 1);
+      if (rows > kMaxTokens) {
+        if (ht == 0 && jb == 0) atomicOr(p.err, GNF4_DEVERR_GEMV_ROWS);
+      } else {
+        for (int o = ht; o < 4 * 32 * 4; o += kThreads / 2) {
+          const int i = o >> 7, l = (o >> 2) & 31, j = o & 3;
+          float v = 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) s.red[warp][i][lane][j] = acc[i][j];
-    __syncthreads();
-    for (int o = tid; o < 4 * 32 * 4; o += kThreads) {
-      const int i = o >> 7, l = (o >> 2) & 31, j = o & 3;
-      float v = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) v += s.red[w][i][l][j];
-      const int n = jb * kRows + 16 * i + (l >> 2) + 8 * (j >> 1);
-      const int tok = 2 * (l & 3) + (j & 1);
-      if (n < p.N && tok < rows) p.y[(size_t)(r0 + tok) * p.N + n] = __float2bfloat16_rn(v);
+          for (int w = 0; w < kSplit; ++w) v += s.red[h][w][i][l][j];
+          const int n = jb * kRows + 16 * i + (l >> 2) + 8 * (j >> 1);
+          const int tok = 2 * (l & 3) + (j & 1);
+          if (n < p.N && tok < rows) p.y[(size_t)(r0 + tok) * p.N + n] = __float2bfloat16_rn(v);
+        }
+      }
     }
-    __syncthreads();
+    half_barrier(h);
   }
 }
 
 }  // namespace
 
-int gemv_rows_per_block() { return kRows; }
+int gemv_grid(long long units, int num_sms) {
+  const long long ctas = (units + 1) / 2;  // two units at a time per CTA
+  return (int)(ctas < num_sms ? ctas : num_sms);
+}
 
-template <int FMT>
+template <int FMT, bool FULLN>
 static cudaError_t launch_gemv_t(const GroupedArgs& p, int grid, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(GemvSmem));
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, FULLN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  gemv_kernel<FMT><<<grid, kThreads, sizeof(GemvSmem), stream>>>(p);
+  gemv_kernel<FMT, FULLN><<<grid, kThreads, kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemv(int fmt, const GroupedArgs& p, int grid, cudaStream_t stream) {
-  return fmt == 0 ? launch_gemv_t<0>(p, grid, stream) : launch_gemv_t<1>(p, grid, stream);
+  const bool full = p.N % kRows == 0;
+  if (fmt == 0) return full ? launch_gemv_t<0, true>(p, grid, stream) : launch_gemv_t<0, false>(p, grid, stream);
+  return full ? launch_gemv_t<1, true>(p, grid, stream) : launch_gemv_t<1, false>(p, grid, stream);
 }
+
+int gemv_rows_per_block() { return kRows; }
 
 }  // namespace gnf4

@@ -32,6 +32,8 @@ cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& 
 // gemv.cu
 cudaError_t launch_gemv(int fmt, const GroupedArgs& p, int grid, cudaStream_t stream);
 int gemv_rows_per_block();
+// CTAs for a GEMV launch over `units` (expert, 64-row) units.
+int gemv_grid(long long units, int num_sms);
 
 // route.cu
 size_t route_workspace_bytes(int T, int k, int E);

@@ -26,7 +26,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
-DEVERR_TIMEOUT, DEVERR_BAD_OFFSETS, DEVERR_GEMV_ROWS = 0x1, 0x2, 0x4
+DEVERR_TIMEOUT, DEVERR_BAD_OFFSETS, DEVERR_GEMV_ROWS, DEVERR_INTERNAL = 0x1, 0x2, 0x4, 0x8
 MAX_GEMV_ROWS = 8
 
 _P = ctypes.c_void_p

@@ -72,6 +72,7 @@ typedef enum {
 #define GNF4_DEVERR_TIMEOUT 0x1u      /* a bounded pipeline wait gave up; outputs incomplete */
 #define GNF4_DEVERR_BAD_OFFSETS 0x2u  /* offsets not monotone, offsets[0] != 0 or offsets[E] > M */
 #define GNF4_DEVERR_GEMV_ROWS 0x4u    /* a GEMV group held more than 8 rows; that group was skipped */
+#define GNF4_DEVERR_INTERNAL 0x8u     /* a kernel's shared-memory layout check failed; no output written */
 
 /* Text of the calling thread's last failure ("" if none). */
 const char *gnf4_last_error(void);
