@@ -90,6 +90,10 @@ struct Unit {
   int e, j, row0, rows;
 };
 
+// Partial accumulators per unit: groups of at most 32 (64) rows split the
+// 128 accumulator columns into 4 (2) independent sums of 32 (64) columns.
+__device__ __forceinline__ int acc_split(int rows) { return rows <= 32 ? 4 : (rows <= 64 ? 2 : 1); }
+
 __device__ __forceinline__ Unit unit_of(const Smem& s, int E, int u) {
   Unit x;
   x.e = find_group(s.upre, E, u);
@@ -260,16 +264,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t idesc = idesc_bf16_m128((uint32_t)((x.rows + 15) & ~15));
         const uint32_t d_tmem = tmem + (uint32_t)(ab * kBT);
+        // Small groups: the k-steps of a stage go to independent partial
+        // accumulators, so consecutive MMAs do not wait for each other.
+        const int nsplit = acc_split(x.rows);
+        const uint32_t sub_w = (uint32_t)(kBT / nsplit);
         for (int kt = 0; kt < nk; ++kt, ++it) {
           const int sa = it % kAStages, sT = it % kTStages;
-          if (!(ok = mbar_wait(&s.afull[sa], (it / kAStages) & 1, err, abort))) break;
-          if (!(ok = mbar_wait(&s.tfull[sT], (it / kTStages) & 1, err, abort))) break;
+          // poll both barriers before looking at either result
+          const bool ra = mbar_try_wait(&s.afull[sa], (it / kAStages) & 1);
+          const bool rt = mbar_try_wait(&s.tfull[sT], (it / kTStages) & 1);
+          if (!(ra && rt)) {
+            if (!(ok = mbar_wait(&s.afull[sa], (it / kAStages) & 1, err, abort))) break;
+            if (!(ok = mbar_wait(&s.tfull[sT], (it / kTStages) & 1, err, abort))) break;
+          }
           tc_fence_after();
           const uint32_t a_col = tmem + (uint32_t)(kACol0 + sT * (kBK / 2));
           const uint32_t b_addr = smem_u32(s.act[sa]);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            tc_mma_ts(d_tmem, a_col + kk * 8, sdesc_k_sw128(b_addr + kk * 32), idesc, (kt | kk) != 0);
+            tc_mma_ts(d_tmem + (uint32_t)(kk % nsplit) * sub_w, a_col + kk * 8, sdesc_k_sw128(b_addr + kk * 32), idesc,
+                      kt != 0 || kk >= nsplit);
           tc_commit(&s.aempty[sa]);
           tc_commit(&s.tempty[sT]);
         }
@@ -359,10 +373,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int n = x.j * kBW + q * 32 + lane;
       __nv_bfloat16* ycol = p.y + (size_t)x.row0 * p.N + n;
+      const int nsplit = acc_split(x.rows);
       for (int c = 0; c * 32 < x.rows; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBT + c * 32), v);
         tmem_wait_ld();
+        for (int j = 1; j < nsplit; ++j) {  // partial accumulators, summed in a fixed order
+          uint32_t w2[32];
+          tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBT + j * (kBT / nsplit) + c * 32), w2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w2[i]));
+        }
         if (n < p.N) {
           const int lim = min(32, x.rows - c * 32);
 #pragma unroll
