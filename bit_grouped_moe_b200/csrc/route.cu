@@ -15,6 +15,10 @@
 //               rows past offsets[E] are zeroed.
 // Ids outside [0, E) are counted and dropped, never used as an index
 // (releases v0.3.0, "Also": model-global ids read out of bounds silently).
+//
+// Decode-sized calls (at most 256 pairs) take a single launch instead: every
+// block repeats the whole (tiny) sort in shared memory, block 0 writes the
+// routing outputs and all blocks share the gather.  Same results, bit for bit.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -156,6 +160,91 @@ __global__ void route_gather_kernel(const uint4* x, int K8, int k, const int32_t
   }
 }
 
+
+// Single-launch routing for M <= kChunk pairs: each block sorts all pairs in
+// shared memory (same counting sort, same ranks), block 0 writes offsets and
+// permutations, and block b gathers rows b, b + gridDim.x, ...
+__global__ void __launch_bounds__(kChunk) route_small_kernel(const int32_t* ids, int M, int E, const uint4* x,
+                                                             int K8, int k, int32_t* offsets, int32_t* s2f,
+                                                             int32_t* f2s, int32_t* bad_out, uint4* xs) {
+  __shared__ int cnt[kMaxRouteExperts];
+  __shared__ int s2f_sm[kChunk];
+  __shared__ int wsum[kChunk / 32];
+  __shared__ int nbad, nvalid_sm;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  for (int i = tid; i < E; i += kChunk) cnt[i] = 0;
+  if (tid == 0) nbad = 0;
+  __syncthreads();
+  const int e = (tid < M) ? ids[tid] : -1;
+  const bool valid = tid < M && e >= 0 && e < E;
+  if (valid) atomicAdd(&cnt[e], 1);
+  else if (tid < M) atomicAdd(&nbad, 1);
+  __syncthreads();
+  // exclusive scan of cnt over experts: each thread a contiguous slice
+  const int per = (E + kChunk - 1) / kChunk;
+  const int lo = min(E, tid * per), hi = min(E, lo + per);
+  int mine = 0;
+  for (int i = lo; i < hi; ++i) mine += cnt[i];
+  int incl = mine;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) wsum[wid] = incl;
+  __syncthreads();
+  int base = incl - mine;
+  for (int w = 0; w < wid; ++w) base += wsum[w];
+  __syncthreads();  // every thread has read its slice of cnt
+  for (int i = lo; i < hi; ++i) {
+    const int c = cnt[i];
+    cnt[i] = base;  // exclusive prefix = first row of expert i
+    base += c;
+  }
+  if (lo < hi && hi == E) nvalid_sm = base;
+  if (E == 0 && tid == 0) nvalid_sm = 0;
+  __syncthreads();
+  // stable rank within the expert: warps in order, lanes by match
+  const unsigned lt = (1u << lane) - 1u;
+  int pos = -1;
+  for (int w = 0; w < kChunk / 32; ++w) {
+    if (wid == w) {
+      const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+      const int before = valid ? cnt[e] : 0;
+      __syncwarp();
+      if (valid) {
+        pos = before + __popc(peers & lt);
+        if ((peers & lt) == 0u) cnt[e] = before + __popc(peers);
+      }
+    }
+    __syncthreads();
+  }
+  if (valid) s2f_sm[pos] = tid;
+  __syncthreads();
+  const int nvalid = nvalid_sm;
+  if (blockIdx.x == 0) {
+    if (tid < M) {
+      f2s[tid] = valid ? pos : -1;
+      s2f[tid] = tid < nvalid ? s2f_sm[tid] : -1;
+    }
+    // offsets: cnt now holds each expert's end row = the next expert's start
+    for (int i = tid; i < E; i += kChunk) offsets[i + 1] = cnt[i];
+    if (tid == 0) {
+      offsets[0] = 0;
+      if (bad_out != nullptr) *bad_out = nbad;
+    }
+  }
+  for (int r = blockIdx.x; r < M; r += gridDim.x) {
+    uint4* dst = xs + (size_t)r * K8;
+    if (r < nvalid) {
+      const uint4* src = x + (size_t)(s2f_sm[r] / k) * K8;
+      for (int v = tid; v < K8; v += kChunk) dst[v] = src[v];
+    } else {
+      for (int v = tid; v < K8; v += kChunk) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
 }  // namespace
 
 size_t route_workspace_bytes(int T, int k, int E) {
@@ -170,6 +259,13 @@ cudaError_t launch_route(const int32_t* topk_ids, const __nv_bfloat16* x, int T,
                          __nv_bfloat16* x_sorted, void* workspace, int32_t* bad_id_count, int num_sms,
                          cudaStream_t stream) {
   const int M = T * k;
+  if (M > 0 && M <= kChunk) {
+    const int grid = M < 2 * num_sms ? M : 2 * num_sms;
+    route_small_kernel<<<grid, kChunk, 0, stream>>>(topk_ids, M, E, reinterpret_cast<const uint4*>(x), K / 8, k,
+                                                   offsets, sorted_to_flat, flat_to_sorted, bad_id_count,
+                                                   reinterpret_cast<uint4*>(x_sorted));
+    return cudaGetLastError();
+  }
   const int nchunk = (M + kChunk - 1) / kChunk;
   int32_t* hist = reinterpret_cast<int32_t*>(workspace);
   int32_t* badc = hist + (size_t)nchunk * E;
