@@ -14,6 +14,8 @@ namespace {
 
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* y, const int32_t* f2s, const float* w, int T,
                                                       int k, int N8, uint4* out) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int rows_y = T * k;
   const size_t total = (size_t)T * N8;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
@@ -52,9 +54,8 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* flat_to_sorted
   const int threads = 256;
   const size_t want = (total + threads - 1) / threads;
   const int grid = (int)(want < (size_t)num_sms * 16 ? want : (size_t)num_sms * 16);
-  combine_kernel<<<grid, threads, 0, stream>>>(reinterpret_cast<const uint4*>(y), flat_to_sorted, weights, T, k, N8,
-                                               reinterpret_cast<uint4*>(out));
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(grid), dim3(threads), 0, stream, reinterpret_cast<const uint4*>(y),
+                    flat_to_sorted, weights, T, k, N8, reinterpret_cast<uint4*>(out));
 }
 
 }  // namespace gnf4

@@ -117,6 +117,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned* err = p.err;
   volatile int* abort = &s.abort;
 
+  griddep_launch_dependents();
+  griddep_wait();
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, err)) return;
   const int nwt = (p.N + kBW - 1) / kBW;
   block_exclusive_scan(p.E, s.upre, s.scratch,
@@ -424,8 +426,8 @@ cudaError_t launch_gemm_tc_t(const CUtensorMap& tm_a, const CUtensorMap& tm_a_bi
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  gemm_tc_kernel<FMT><<<grid, kThreads, gemm_tc_smem_bytes(), stream>>>(tm_a, tm_a_big, tm_w, p);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<FMT>, dim3(grid), dim3(kThreads), gemm_tc_smem_bytes(), stream, tm_a, tm_a_big,
+                    tm_w, p);
 }
 
 cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,

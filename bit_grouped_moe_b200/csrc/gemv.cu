@@ -151,6 +151,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
     if (tid == 0) atomicOr(p.err, GNF4_DEVERR_INTERNAL);
     return;
   }
+  griddep_launch_dependents();
+  // the pair table depends on nothing earlier in the stream: build it while
+  // the previous kernel finishes (made visible by the barriers below)
+  build_pair_lut256<FMT>(reinterpret_cast<uint32_t*>(smem_raw + (kLutWindow - base)), tid, kThreads);
+  griddep_wait();
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, p.err)) return;
   const int nblk = (p.N + kRows - 1) / kRows;
   block_exclusive_scan(p.E, s.upre, s.scratch, [&](int e) { return (s.off[e + 1] > s.off[e]) ? nblk : 0; });
@@ -165,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
   const int ustride = 2 * (int)gridDim.x;
   int u = 2 * (int)blockIdx.x + h;
 
-  // first item of this warp's stream, issued before the table is built
+  // first item of this warp's stream
   uint4 wq[8], xa[4];
   uint32_t sr[8];
   UnitView cur{};
@@ -177,7 +182,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
       load_acts(cur, d_lo, t, K, xa);
     }
   }
-  build_pair_lut256<FMT>(reinterpret_cast<uint32_t*>(smem_raw + (kLutWindow - base)), tid, kThreads);
   __syncthreads();
 
   const uint32_t lanesel = (uint32_t)lane * 4u | (kLutWindow & 0x00FF0000u);
@@ -269,8 +273,7 @@ static cudaError_t launch_gemv_t(const GroupedArgs& p, int grid, cudaStream_t st
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  gemv_kernel<FMT, FULLN><<<grid, kThreads, kSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(gemv_kernel<FMT, FULLN>, dim3(grid), dim3(kThreads), (size_t)kSmemBytes, stream, p);
 }
 
 cudaError_t launch_gemv(int fmt, const GroupedArgs& p, int grid, cudaStream_t stream) {

@@ -8,7 +8,29 @@
 
 #include <cuda_bf16.h>
 
+#include <utility>
+
 namespace gnf4 {
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel of the stream is still finishing.  Every kernel
+// launched this way executes griddep_wait() (common.cuh) before it reads or
+// writes any global memory that earlier work in the stream uses.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Arguments of the grouped GEMM / GEMV kernels (device pointers).
 struct GroupedArgs {

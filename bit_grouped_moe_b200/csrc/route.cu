@@ -32,6 +32,8 @@ constexpr int kMaxRouteExperts = 4096;
 
 __global__ void __launch_bounds__(kChunk) route_hist_kernel(const int32_t* ids, int M, int E, int32_t* hist,
                                                             int32_t* badc) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ int cnt[kMaxRouteExperts];
   __shared__ int nbad;
   const int tid = threadIdx.x, c = blockIdx.x;
@@ -53,6 +55,8 @@ __global__ void __launch_bounds__(kChunk) route_hist_kernel(const int32_t* ids, 
 
 __global__ void __launch_bounds__(1024) route_scan_kernel(int32_t* hist, const int32_t* badc, int nchunk, int E,
                                                           int32_t* offsets, int32_t* bad_out) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ int tot[kMaxRouteExperts];
   __shared__ int wsum[32];
   const int tid = threadIdx.x;
@@ -114,6 +118,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int32_t* hist, const i
 __global__ void __launch_bounds__(kChunk) route_scatter_kernel(const int32_t* ids, int M, int E,
                                                                const int32_t* hist, int32_t* s2f,
                                                                int32_t* f2s) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ int run[kMaxRouteExperts];
   const int tid = threadIdx.x, c = blockIdx.x, lane = tid & 31, wid = tid >> 5;
   for (int i = tid; i < E; i += kChunk) run[i] = 0;
@@ -143,6 +149,8 @@ __global__ void __launch_bounds__(kChunk) route_scatter_kernel(const int32_t* id
 
 __global__ void route_gather_kernel(const uint4* x, int K8, int k, const int32_t* offsets, int E, int M,
                                     int32_t* s2f, uint4* xs) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int nvalid = offsets[E];
   const size_t total = (size_t)M * K8;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
@@ -167,6 +175,8 @@ __global__ void route_gather_kernel(const uint4* x, int K8, int k, const int32_t
 __global__ void __launch_bounds__(kChunk) route_small_kernel(const int32_t* ids, int M, int E, const uint4* x,
                                                              int K8, int k, int32_t* offsets, int32_t* s2f,
                                                              int32_t* f2s, int32_t* bad_out, uint4* xs) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ int cnt[kMaxRouteExperts];
   __shared__ int s2f_sm[kChunk];
   __shared__ int wsum[kChunk / 32];
@@ -261,27 +271,34 @@ cudaError_t launch_route(const int32_t* topk_ids, const __nv_bfloat16* x, int T,
   const int M = T * k;
   if (M > 0 && M <= kChunk) {
     const int grid = M < 2 * num_sms ? M : 2 * num_sms;
-    route_small_kernel<<<grid, kChunk, 0, stream>>>(topk_ids, M, E, reinterpret_cast<const uint4*>(x), K / 8, k,
-                                                   offsets, sorted_to_flat, flat_to_sorted, bad_id_count,
-                                                   reinterpret_cast<uint4*>(x_sorted));
-    return cudaGetLastError();
+    return launch_pdl(route_small_kernel, dim3(grid), dim3(kChunk), 0, stream, topk_ids, M, E,
+                      reinterpret_cast<const uint4*>(x), K / 8, k, offsets, sorted_to_flat, flat_to_sorted,
+                      bad_id_count, reinterpret_cast<uint4*>(x_sorted));
   }
   const int nchunk = (M + kChunk - 1) / kChunk;
   int32_t* hist = reinterpret_cast<int32_t*>(workspace);
   int32_t* badc = hist + (size_t)nchunk * E;
   if (M > 0) {
-    route_hist_kernel<<<nchunk, kChunk, 0, stream>>>(topk_ids, M, E, hist, badc);
+    cudaError_t e = launch_pdl(route_hist_kernel, dim3(nchunk), dim3(kChunk), 0, stream, topk_ids, M, E, hist, badc);
+    if (e != cudaSuccess) return e;
   }
-  route_scan_kernel<<<1, 1024, 0, stream>>>(hist, badc, nchunk, E, offsets, bad_id_count);
+  {
+    cudaError_t e = launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, hist, badc, nchunk, E, offsets,
+                               bad_id_count);
+    if (e != cudaSuccess) return e;
+  }
   if (M > 0) {
-    route_scatter_kernel<<<nchunk, kChunk, 0, stream>>>(topk_ids, M, E, hist, sorted_to_flat, flat_to_sorted);
+    cudaError_t e = launch_pdl(route_scatter_kernel, dim3(nchunk), dim3(kChunk), 0, stream, topk_ids, M, E,
+                               (const int32_t*)hist, sorted_to_flat, flat_to_sorted);
+    if (e != cudaSuccess) return e;
     const int K8 = K / 8;
     const size_t total = (size_t)M * K8;
     const int threads = 256;
     const size_t want = (total + threads - 1) / threads;
     const int grid = (int)(want < (size_t)num_sms * 16 ? want : (size_t)num_sms * 16);
-    route_gather_kernel<<<grid, threads, 0, stream>>>(reinterpret_cast<const uint4*>(x), K8, k, offsets, E, M,
-                                                      sorted_to_flat, reinterpret_cast<uint4*>(x_sorted));
+    e = launch_pdl(route_gather_kernel, dim3(grid), dim3(threads), 0, stream, reinterpret_cast<const uint4*>(x), K8,
+                   k, (const int32_t*)offsets, E, M, sorted_to_flat, reinterpret_cast<uint4*>(x_sorted));
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
