@@ -56,6 +56,7 @@ def _load():
     lib.orc_grouped_gemm_nf4.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
     lib.orc_grouped_gemm_mxfp4.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
     lib.orc_combine.argtypes = [P, P, P, I64, I64, I64, P]
+    lib.orc_swiglu.argtypes = [P, I64, I64, P]
     _lib = lib
     return lib
 
@@ -202,3 +203,20 @@ def combine(y_bits: np.ndarray, flat_to_sorted: np.ndarray, weights: np.ndarray)
     out = np.empty((T, N), np.float64)
     _load().orc_combine(_p(y_bits), _p(f2s), _p(w), T, k, N, _p(out))
     return out
+
+
+def swiglu(gate_up: np.ndarray) -> np.ndarray:
+    """fp64 h [R, I] = silu(gate_up[:, :I]) * gate_up[:, I:] (gate half first)."""
+    gu = _c(gate_up, np.float64)
+    R, I2 = gu.shape
+    I = I2 // 2
+    h = np.empty((R, I), np.float64)
+    _load().orc_swiglu(_p(gu), R, I, _p(h))
+    return h
+
+
+def grouped_gemm_swiglu(fmt: str, a_bits, w, scales, offsets, rows=None):
+    """fp64 fused gate_up projection + SwiGLU: the plain GEMM over the [E, 2I, K]
+    stack followed by swiglu()."""
+    fn = grouped_gemm_nf4 if fmt == "nf4" else grouped_gemm_mxfp4
+    return swiglu(fn(a_bits, w, scales, offsets, rows=rows))

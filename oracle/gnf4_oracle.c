@@ -18,6 +18,9 @@
  *   [PATCH]    grouped-nf4-gemm releases, v0.2.6 "The patch point" (argsort of
  *              the top-k ids, gather x[idxs // k], tokens_per_expert = sizes;
  *              weighting and unsorting stay with the caller).
+ *   [MOE]      grouped-nf4-gemm 0.33.1 on PyPI, "API": moe_layer_forward runs
+ *              gate_up -> GLU -> down; swiglu_rows is listed with the glue
+ *              helpers (reading C17 for the row order and the activation).
  *   [ARENA]    grouped-nf4-gemm releases, v0.2.5 "arena -> kernel" (expert
  *              stacks [E,N,K//2] blocks + [E,N,K//32] e8m0 scales).
  *   [QLORA]    The NF4 codebook itself is not printed on the pages; the values
@@ -396,6 +399,27 @@ void orc_combine(const uint16_t *y, const int32_t *flat_to_sorted, const float *
                 acc += (double)weights[t * k + j] * (double)bf16_to_float(y[(int64_t)p * N + n]);
             }
             out[t * N + n] = acc;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Gated activation between the two projections [MOE]                  */
+/* ------------------------------------------------------------------ */
+
+/* SwiGLU over a gate_up projection output (reading C17): row r of gu holds
+ * 2I values, the gate half first, then the up half;
+ *     h[r, i] = silu(gu[r, i]) * gu[r, I + i],   silu(x) = x / (1 + exp(-x)),
+ * all in fp64.  Applied to the fp64 output of orc_grouped_gemm_* this is the
+ * plain definition of the fused gate_up + SwiGLU projection. */
+void orc_swiglu(const double *gu, int64_t rows, int64_t I, double *h)
+{
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t i = 0; i < I; ++i) {
+            const double g = gu[r * 2 * I + i];
+            const double u = gu[r * 2 * I + I + i];
+            h[r * I + i] = g / (1.0 + exp(-g)) * u;
         }
     }
 }

@@ -367,3 +367,46 @@ def test_combine_weights_summing_to_one_reproduce_a_shared_row():
     wsum = wts.astype(np.float64).sum(axis=1)
     assert np.allclose(out, wsum[:, None] * _af(row), rtol=1e-15, atol=0)
     assert np.allclose(wsum, 1.0, atol=1e-6)
+
+
+# ------------------------------------------------------------------ SwiGLU (reading C17)
+
+
+def test_silu_closed_forms():
+    """sigmoid(ln 3) = 3/4, so silu(ln 3) = 0.75 ln 3 and silu(-ln 3) = -0.25 ln 3;
+    silu(0) = 0; an up value of 0 zeroes the product."""
+    L = math.log(3.0)
+    gu = np.array([[L, -L, 0.0, 5.0, 1.0, 1.0, 1.0, 0.0]], np.float64)  # gate | up, I = 4
+    h = oracle.swiglu(gu)[0]
+    assert abs(h[0] - 0.75 * L) <= 1e-15
+    assert abs(h[1] + 0.25 * L) <= 1e-15
+    assert h[2] == 0.0
+    assert h[3] == 0.0
+
+
+def test_silu_odd_part_is_identity():
+    """x*sigmoid(x) - (-x)*sigmoid(-x) = x (since sigmoid(x) + sigmoid(-x) = 1)."""
+    g = inputs.rng(50).standard_normal(64) * 4
+    gu = np.stack([np.concatenate([g, np.ones(64)]), np.concatenate([-g, np.ones(64)])])
+    h = oracle.swiglu(gu)
+    np.testing.assert_allclose(h[0] - h[1], g, rtol=0, atol=1e-13)
+
+
+def test_swiglu_takes_the_gate_half_first():
+    """MXFP4 codes all 1.0: the gate half with scale 127 gives the row sum s,
+    the up half with scale 126 gives s/2, so h = silu(s) * s/2; swapping the
+    halves would give silu(s/2) * s."""
+    g = inputs.rng(51)
+    E, I, K, M = 2, 8, 64, 5
+    a = inputs.bf16_normal(g, (M, K))
+    w = np.full((E, 2 * I, K // 2), 0x22, np.uint8)
+    s = np.full((E, 2 * I, K // 32), 127, np.uint8)
+    s[:, I:, :] = 126
+    offsets = np.array([0, 2, M], np.int32)
+    h = oracle.grouped_gemm_swiglu("mxfp4", a, w, s, offsets)
+    for r in range(M):
+        rs = math.fsum(_af(a[r]))
+        ref = oracle.swiglu(np.array([[rs, rs / 2.0]]))[0, 0]
+        swapped = oracle.swiglu(np.array([[rs / 2.0, rs]]))[0, 0]
+        assert np.all(h[r] == ref)
+        assert rs == 0.0 or ref != swapped
