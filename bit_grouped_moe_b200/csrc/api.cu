@@ -134,13 +134,13 @@ gnf4_status encode_act_map(CUtensorMap* m, const void* a, int M, int K, int box_
   return GNF4_OK;
 }
 
-// W [E, N, K/2] u8: 32-byte x 128-row x 1 boxes, no swizzle, zero fill.
-gnf4_status encode_weight_map(CUtensorMap* m, const void* w, int E, int N, int K) {
+// W [E, N, K/2] u8: box_bytes x box_rows x 1 boxes, no swizzle, zero fill.
+gnf4_status encode_weight_map(CUtensorMap* m, const void* w, int E, int N, int K, int box_bytes, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return fail(GNF4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)N, (cuuint64_t)E};
   cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N * (cuuint64_t)(K / 2)};
-  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t box[3] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(w), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -173,8 +173,10 @@ gnf4_status check_grouped(int fmt, const void* a, const uint8_t* w, const void* 
   return GNF4_OK;
 }
 
-gnf4_status grouped_gemm(int fmt, const void* a, const uint8_t* w, const void* scales, const int32_t* offsets,
-                         const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
+// swiglu: w is a gate_up stack [E, N = 2I, K/2] and y the [M, I] output h.
+gnf4_status grouped_gemm(int fmt, bool swiglu, const void* a, const uint8_t* w, const void* scales,
+                         const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M, void* y,
+                         void* stream) {
   GNF4_TRY(check_grouped(fmt, a, w, scales, offsets, counts, E, N, K, M, y));
   if (M == 0) return GNF4_OK;
   DeviceState* d = nullptr;
@@ -182,23 +184,25 @@ gnf4_status grouped_gemm(int fmt, const void* a, const uint8_t* w, const void* s
   CUtensorMap tm_a, tm_a_big, tm_w;
   GNF4_TRY(encode_act_map(&tm_a, a, M, K, 32));
   GNF4_TRY(encode_act_map(&tm_a_big, a, M, K, 128));
-  GNF4_TRY(encode_weight_map(&tm_w, w, E, N, K));
+  const int wrows = gemm_tc_weight_rows_per_unit();
+  GNF4_TRY(encode_weight_map(&tm_w, w, E, N, K, 32, swiglu ? wrows / 2 : wrows));
   GroupedArgs p{static_cast<const __nv_bfloat16*>(a), w, scales, offsets, counts,
                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
   // upper bound on work units: every group adds at most one partial chunk
-  const long long nwt = (N + gemm_tc_weight_rows_per_unit() - 1) / gemm_tc_weight_rows_per_unit();
+  const long long nwt = (N + wrows - 1) / wrows;  // SwiGLU: (2I / 128) tiles of 64 gate + 64 up rows
   const long long rpu = gemm_tc_rows_per_unit();
   const long long chunks = (M + rpu - 1) / rpu + (E < M ? E : M);
   const long long units = chunks * nwt;
   if (units >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d, N=%d give too many work units", M, N);
   const int grid = (int)(units < d->num_sms ? units : d->num_sms);
-  cudaError_t e = launch_gemm_tc(fmt, tm_a, tm_a_big, tm_w, p, grid, as_stream(stream));
+  cudaError_t e = launch_gemm_tc(fmt, swiglu, tm_a, tm_a_big, tm_w, p, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMM launch");
   return GNF4_OK;
 }
 
-gnf4_status grouped_gemv(int fmt, const void* a, const uint8_t* w, const void* scales, const int32_t* offsets,
-                         const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
+gnf4_status grouped_gemv(int fmt, bool swiglu, const void* a, const uint8_t* w, const void* scales,
+                         const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M, void* y,
+                         void* stream) {
   GNF4_TRY(check_grouped(fmt, a, w, scales, offsets, counts, E, N, K, M, y));
   if (M == 0) return GNF4_OK;
   DeviceState* d = nullptr;
@@ -206,10 +210,18 @@ gnf4_status grouped_gemv(int fmt, const void* a, const uint8_t* w, const void* s
   GroupedArgs p{static_cast<const __nv_bfloat16*>(a), w, scales, offsets, counts,
                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
   const long long hit = E < M ? E : M;  // groups with rows
-  const long long blocks = hit * ((N + gemv_rows_per_block() - 1) / gemv_rows_per_block());
-  const int grid = gemv_grid(blocks, d->num_sms);
-  cudaError_t e = launch_gemv(fmt, p, grid, as_stream(stream));
+  const long long per = swiglu ? (N / 2) / gemv_swiglu_cols_per_block()
+                               : (N + gemv_rows_per_block() - 1) / gemv_rows_per_block();
+  const int grid = gemv_grid(hit * per, d->num_sms);
+  cudaError_t e = launch_gemv(fmt, swiglu, p, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMV launch");
+  return GNF4_OK;
+}
+
+// The fused gate_up + SwiGLU calls take I (the output width); the stack has 2I rows.
+gnf4_status check_swiglu_width(int I) {
+  if (I < 64 || I % 64 != 0 || I > (1 << 29))
+    return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "I=%d must be a positive multiple of 64 (gate_up stack of 2I rows)", I);
   return GNF4_OK;
 }
 
@@ -283,22 +295,22 @@ gnf4_status gnf4_route_permute(const int32_t* topk_ids, const void* x, int T, in
 
 gnf4_status gnf4_grouped_gemm_nf4(const void* a, const uint8_t* w, const float* absmax, const int32_t* offsets,
                                   const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
-  return grouped_gemm(0, a, w, absmax, offsets, counts, E, N, K, M, y, stream);
+  return grouped_gemm(0, false, a, w, absmax, offsets, counts, E, N, K, M, y, stream);
 }
 
 gnf4_status gnf4_grouped_gemm_mxfp4(const void* a, const uint8_t* w, const uint8_t* scales, const int32_t* offsets,
                                     const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
-  return grouped_gemm(1, a, w, scales, offsets, counts, E, N, K, M, y, stream);
+  return grouped_gemm(1, false, a, w, scales, offsets, counts, E, N, K, M, y, stream);
 }
 
 gnf4_status gnf4_grouped_gemv_nf4(const void* a, const uint8_t* w, const float* absmax, const int32_t* offsets,
                                   const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
-  return grouped_gemv(0, a, w, absmax, offsets, counts, E, N, K, M, y, stream);
+  return grouped_gemv(0, false, a, w, absmax, offsets, counts, E, N, K, M, y, stream);
 }
 
 gnf4_status gnf4_grouped_gemv_mxfp4(const void* a, const uint8_t* w, const uint8_t* scales, const int32_t* offsets,
                                     const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
-  return grouped_gemv(1, a, w, scales, offsets, counts, E, N, K, M, y, stream);
+  return grouped_gemv(1, false, a, w, scales, offsets, counts, E, N, K, M, y, stream);
 }
 
 gnf4_status gnf4_combine(const void* y, const int32_t* flat_to_sorted, const float* weights, int T, int k, int N,
@@ -343,6 +355,38 @@ gnf4_status gnf4_dequant_nf4_f32(const uint8_t* w, const float* absmax, int64_t 
 gnf4_status gnf4_dequant_mxfp4_f32(const uint8_t* w, const uint8_t* scales, int64_t rows, int K, float* out,
                                    void* stream) {
   return dequant(1, w, scales, rows, K, out, stream);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+gnf4_status gnf4_grouped_gemm_nf4_swiglu(const void* a, const uint8_t* w_gate_up, const float* absmax,
+                                         const int32_t* offsets, const int32_t* counts, int E, int I, int K, int M,
+                                         void* h, void* stream) {
+  GNF4_TRY(check_swiglu_width(I));
+  return grouped_gemm(0, true, a, w_gate_up, absmax, offsets, counts, E, 2 * I, K, M, h, stream);
+}
+
+gnf4_status gnf4_grouped_gemm_mxfp4_swiglu(const void* a, const uint8_t* w_gate_up, const uint8_t* scales,
+                                           const int32_t* offsets, const int32_t* counts, int E, int I, int K, int M,
+                                           void* h, void* stream) {
+  GNF4_TRY(check_swiglu_width(I));
+  return grouped_gemm(1, true, a, w_gate_up, scales, offsets, counts, E, 2 * I, K, M, h, stream);
+}
+
+gnf4_status gnf4_grouped_gemv_nf4_swiglu(const void* a, const uint8_t* w_gate_up, const float* absmax,
+                                         const int32_t* offsets, const int32_t* counts, int E, int I, int K, int M,
+                                         void* h, void* stream) {
+  GNF4_TRY(check_swiglu_width(I));
+  return grouped_gemv(0, true, a, w_gate_up, absmax, offsets, counts, E, 2 * I, K, M, h, stream);
+}
+
+gnf4_status gnf4_grouped_gemv_mxfp4_swiglu(const void* a, const uint8_t* w_gate_up, const uint8_t* scales,
+                                           const int32_t* offsets, const int32_t* counts, int E, int I, int K, int M,
+                                           void* h, void* stream) {
+  GNF4_TRY(check_swiglu_width(I));
+  return grouped_gemv(1, true, a, w_gate_up, scales, offsets, counts, E, 2 * I, K, M, h, stream);
 }
 
 }  // extern "C"

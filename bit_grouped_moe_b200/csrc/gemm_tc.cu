@@ -94,6 +94,26 @@ struct Unit {
 // 128 accumulator columns into 4 (2) independent sums of 32 (64) columns.
 __device__ __forceinline__ int acc_split(int rows) { return rows <= 32 ? 4 : (rows <= 64 ? 2 : 1); }
 
+// Weight row (within the expert) held by TMEM lane nl of weight tile j.
+// SwiGLU tiles take 64 gate rows and the matching 64 up rows of a gate_up
+// stack [E, 2I, K]; inside every 32-lane quarter q, lanes 0..15 are gate rows
+// 64j + 16q + x and lanes 16..31 the up rows I + 64j + 16q + x, so the
+// epilogue pairs them with one shuffle.
+template <bool SWI>
+__device__ __forceinline__ int tile_row(int j, int nl, int I) {
+  if (!SWI) return j * kBW + nl;
+  const int q = nl >> 5, x = nl & 31;
+  return (x < 16 ? 0 : I) + 64 * j + 16 * q + (x & 15);
+}
+// Row of lane nl's packed bytes inside a weight stage (SwiGLU stages hold the
+// gate box in rows 0..63 and the up box in rows 64..127).
+template <bool SWI>
+__device__ __forceinline__ int stage_row(int nl) {
+  if (!SWI) return nl;
+  const int q = nl >> 5, x = nl & 31;
+  return (x < 16 ? 0 : 64) + 16 * q + (x & 15);
+}
+
 __device__ __forceinline__ Unit unit_of(const Smem& s, int E, int u) {
   Unit x;
   x.e = find_group(s.upre, E, u);
@@ -107,7 +127,7 @@ __device__ __forceinline__ Unit unit_of(const Smem& s, int E, int u) {
   return x;
 }
 
-template <int FMT>
+template <int FMT, bool SWI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_big,
                    const __grid_constant__ CUtensorMap tm_w, GroupedArgs p) {
@@ -120,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_launch_dependents();
   griddep_wait();
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, err)) return;
-  const int nwt = (p.N + kBW - 1) / kBW;
+  const int I = p.N / 2;  // SwiGLU: output columns
+  const int nwt = SWI ? I / (kBW / 2) : (p.N + kBW - 1) / kBW;
   block_exclusive_scan(p.E, s.upre, s.scratch,
                        [&](int e) { return ((s.off[e + 1] - s.off[e] + kBT - 1) / kBT) * nwt; });
   const int U = s.upre[p.E];
@@ -183,7 +204,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = it % kWStages, use = it / kWStages;
           if (it >= kWStages && !(ok = mbar_wait(&s.wempty[st], (use - 1) & 1, err, abort))) break;
           mbar_arrive_expect_tx(&s.wfull[st], kWStageBytes);
-          tma_load_3d(s.wq[st], &tm_w, &s.wfull[st], kt * (kBK / 2), x.j * kBW, x.e);
+          if (SWI) {  // two 64-row boxes: gate rows, then the matching up rows
+            tma_load_3d(s.wq[st], &tm_w, &s.wfull[st], kt * (kBK / 2), x.j * (kBW / 2), x.e);
+            tma_load_3d(s.wq[st] + kWStageBytes / 2, &tm_w, &s.wfull[st], kt * (kBK / 2), I + x.j * (kBW / 2), x.e);
+          } else {
+            tma_load_3d(s.wq[st], &tm_w, &s.wfull[st], kt * (kBK / 2), x.j * kBW, x.e);
+          }
         }
       }
       if (!ok)  // drain loads still in flight before shared memory goes away
@@ -236,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int m = 0; m < kBW / 32; ++m) {
           const int r = lane + 32 * m;
-          const int n = x.j * kBW + r;
+          const int n = tile_row<SWI>(x.j, r, I);
           if (n >= p.N) continue;
           const size_t rowsc = ((size_t)x.e * p.N + (size_t)n) * (size_t)nsc;
           if (FMT == 0) {
@@ -321,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             sc0 = sc1 = f32_to_bf16x2_rn(__uint_as_float(s.sring[slot][nl][q8]));
           } else {
             // bytes of the chunk start at (row offset & 3) inside the copied words
-            const size_t rowsc = ((size_t)xu.e * p.N + (size_t)(xu.j * kBW + nl)) * (size_t)(p.K / 32);
+            const size_t rowsc = ((size_t)xu.e * p.N + (size_t)tile_row<SWI>(xu.j, nl, I)) * (size_t)(p.K / 32);
             const uint32_t b = (uint32_t)(rowsc & 3u) + 2u * (uint32_t)q8;
             const uint8_t* bytes = reinterpret_cast<const uint8_t*>(s.sring[slot][nl]);
             sc0 = e8m0_to_bf16x2(bytes[b]);
@@ -329,8 +355,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // two 16-byte reads of this row's 32 bytes, ordered so a quarter warp
           // touches 8 distinct 16-byte bank groups
-          const uint32_t wrow = smem_u32(s.wq[sw]) + (uint32_t)nl * 32u;
-          const uint32_t c_first = ((uint32_t)nl >> 2) & 1u;
+          const uint32_t srow = (uint32_t)stage_row<SWI>(nl);
+          const uint32_t wrow = smem_u32(s.wq[sw]) + srow * 32u;
+          const uint32_t c_first = (srow >> 2) & 1u;
           uint4 c0 = lds_u128(wrow + 16u * c_first), c1 = lds_u128(wrow + 16u * (c_first ^ 1u));
           if (c_first) {
             const uint4 tmp = c0;
@@ -387,8 +414,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w2[i]));
         }
-        if (n < p.N) {
-          const int lim = min(32, x.rows - c * 32);
+        const int lim = min(32, x.rows - c * 32);
+        if (SWI) {
+          // lane x < 16 holds gate(col), lane x + 16 up(col): exchange, then the
+          // low lanes store even rows and the high lanes odd rows
+          const bool up_lane = lane >= 16;
+          const int col = x.j * (kBW / 2) + q * 16 + (lane & 15);
+          __nv_bfloat16* hcol = p.y + (size_t)x.row0 * I + col;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float mine = __uint_as_float(v[i]);
+            const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
+            const float g = up_lane ? other : mine, uu = up_lane ? mine : other;
+            if (i < lim && (i & 1) == (int)up_lane)
+              hcol[(size_t)(c * 32 + i) * I] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * uu);
+          }
+        } else if (n < p.N) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (i < lim) ycol[(size_t)(c * 32 + i) * p.N] = __float2bfloat16_rn(__uint_as_float(v[i]));
@@ -414,26 +455,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t gemm_tc_smem_bytes() { return sizeof(Smem) + 1024; }
 
-template <int FMT>
+template <int FMT, bool SWI>
 cudaError_t launch_gemm_tc_t(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
                              const GroupedArgs& p, int grid, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<FMT, SWI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)gemm_tc_smem_bytes());
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  return launch_pdl(gemm_tc_kernel<FMT>, dim3(grid), dim3(kThreads), gemm_tc_smem_bytes(), stream, tm_a, tm_a_big,
-                    tm_w, p);
+  return launch_pdl(gemm_tc_kernel<FMT, SWI>, dim3(grid), dim3(kThreads), gemm_tc_smem_bytes(), stream, tm_a,
+                    tm_a_big, tm_w, p);
 }
 
-cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
-                           const GroupedArgs& p, int grid, cudaStream_t stream) {
-  return fmt == 0 ? launch_gemm_tc_t<0>(tm_a, tm_a_big, tm_w, p, grid, stream)
-                  : launch_gemm_tc_t<1>(tm_a, tm_a_big, tm_w, p, grid, stream);
+cudaError_t launch_gemm_tc(int fmt, bool swiglu, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big,
+                           const CUtensorMap& tm_w, const GroupedArgs& p, int grid, cudaStream_t stream) {
+  if (fmt == 0)
+    return swiglu ? launch_gemm_tc_t<0, true>(tm_a, tm_a_big, tm_w, p, grid, stream)
+                  : launch_gemm_tc_t<0, false>(tm_a, tm_a_big, tm_w, p, grid, stream);
+  return swiglu ? launch_gemm_tc_t<1, true>(tm_a, tm_a_big, tm_w, p, grid, stream)
+                : launch_gemm_tc_t<1, false>(tm_a, tm_a_big, tm_w, p, grid, stream);
 }
 
 int gemm_tc_rows_per_unit() { return kBT; }

@@ -75,6 +75,9 @@ __device__ __forceinline__ uint32_t lut_lookup(uint32_t word, uint32_t lanesel, 
   return v;
 }
 
+// silu(g) * u = g / (1 + e^-g) * u in fp32.
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
 __device__ __forceinline__ void half_barrier(int h) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + h), "r"(kThreads / 2) : "memory");
 }
@@ -88,12 +91,19 @@ struct UnitView {
   bool tv;                     // token g exists
 };
 
-template <int FMT>
+// Row layouts of a unit's 8 rows per lane (q = 0..7):
+//   kModeClamp  rows n0 + 8q of a [E, N, K] stack, N % 8 == 0 (rows past N read row N-1, never stored)
+//   kModeFull   rows n0 + 8q, N % 64 == 0
+//   kModeSwiglu gate_up stack [E, 2I, K]: q < 4 are gate rows n0 + 8q, q >= 4 the matching up rows
+//               I + n0 + 8(q-4), with n0 = 32 jb + g; the unit writes h columns [32 jb, 32 jb + 32)
+constexpr int kModeClamp = 0, kModeFull = 1, kModeSwiglu = 2;
+
+template <int FMT, int MODE>
 __device__ __forceinline__ UnitView unit_view(const GemvLow& s, const GroupedArgs& p, int u, int g, int t) {
   const int e = find_group(s.upre, p.E, u);
   const int jb = u - s.upre[e];
   const int r0 = s.off[e], rows = s.off[e + 1] - r0;
-  const int n0 = jb * kRows + g;
+  const int n0 = jb * (MODE == kModeSwiglu ? kRows / 2 : kRows) + g;
   const size_t row = (size_t)e * p.N + (size_t)n0;
   const int nsc = FMT == 0 ? p.K / 64 : p.K / 32;
   UnitView v;
@@ -106,21 +116,23 @@ __device__ __forceinline__ UnitView unit_view(const GemvLow& s, const GroupedArg
 }
 
 // Loads of one item for tile i (rows q = 2i, 2i+1): packed weights and raw scales.
-template <int FMT, bool FULLN>
-__device__ __forceinline__ void load_tile(const UnitView& v, int d, int t, int K, size_t rs8, size_t ss8, int i,
-                                          uint4 (&wq)[8], uint32_t (&sr)[8]) {
+// `rb` = packed bytes per weight row, `nsr` = scales per weight row, `gap` =
+// I - 32 (kModeSwiglu: rows from the unit's last gate row block to its up rows).
+template <int FMT, int MODE>
+__device__ __forceinline__ void load_tile(const UnitView& v, int d, int t, int K, size_t rb, size_t nsr, int gap,
+                                          int i, uint4 (&wq)[8], uint32_t (&sr)[8]) {
   const bool inK = d * kDK + 32 * t < K;
   const size_t kb = inK ? (size_t)(d * (kDK / 2) + 16 * t) : 0;  // outside K: any valid address
   const size_t si = inK ? (size_t)(FMT == 0 ? 2 * d + (t >> 1) : 4 * d + t) : 0;
 #pragma unroll
   for (int hq = 0; hq < 2; ++hq) {
     const int q = 2 * i + hq;
-    const int qe = FULLN ? q : min(q, v.qv - 1);
-    wq[q] = ldg_nc_u128(v.w + (size_t)qe * rs8 + kb);
+    const int roff = MODE == kModeClamp ? 8 * min(q, v.qv - 1) : (MODE == kModeSwiglu && q >= 4 ? 8 * q + gap : 8 * q);
+    wq[q] = ldg_nc_u128(v.w + (size_t)roff * rb + kb);
     if (FMT == 0)
-      sr[q] = __ldg(reinterpret_cast<const unsigned int*>(v.sc + ((size_t)qe * ss8 + si) * 4u));
+      sr[q] = __ldg(reinterpret_cast<const unsigned int*>(v.sc + ((size_t)roff * nsr + si) * 4u));
     else
-      sr[q] = __ldg(v.sc + (size_t)qe * ss8 + si);
+      sr[q] = __ldg(v.sc + (size_t)roff * nsr + si);
   }
 }
 
@@ -135,7 +147,7 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t raw) {
   return FMT == 0 ? cvt_bf16x2_dup(__uint_as_float(raw)) : e8m0_to_bf16x2(raw);
 }
 
-template <int FMT, bool FULLN>
+template <int FMT, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   GemvLow& s = *reinterpret_cast<GemvLow*>(smem_raw);
@@ -157,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
   build_pair_lut256<FMT>(reinterpret_cast<uint32_t*>(smem_raw + (kLutWindow - base)), tid, kThreads);
   griddep_wait();
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, p.err)) return;
-  const int nblk = (p.N + kRows - 1) / kRows;
+  const int nblk = MODE == kModeSwiglu ? (p.N / 2) / (kRows / 2) : (p.N + kRows - 1) / kRows;
   block_exclusive_scan(p.E, s.upre, s.scratch, [&](int e) { return (s.off[e + 1] > s.off[e]) ? nblk : 0; });
   const int U = s.upre[p.E];
   if (2 * (int)blockIdx.x >= U) return;  // uniform over the CTA
@@ -165,8 +177,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
   const int K = p.K;
   const int ndk = (K + kDK - 1) / kDK;
   const int d_lo = (ks * ndk) / kSplit, d_hi = ((ks + 1) * ndk) / kSplit;
-  const size_t rs8 = (size_t)8 * (size_t)(K / 2);                 // bytes between rows q and q+1
-  const size_t ss8 = (size_t)8 * (size_t)(FMT == 0 ? K / 64 : K / 32);  // scales between rows q and q+1
+  const size_t rb = (size_t)(K / 2);                              // packed bytes per weight row
+  const size_t nsr = (size_t)(FMT == 0 ? K / 64 : K / 32);         // scales per weight row
+  const int gap = p.N / 2 - kRows / 2;                             // kModeSwiglu only
   const int ustride = 2 * (int)gridDim.x;
   int u = 2 * (int)blockIdx.x + h;
 
@@ -175,10 +188,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
   uint32_t sr[8];
   UnitView cur{};
   if (u < U) {
-    cur = unit_view<FMT>(s, p, u, g, t);
+    cur = unit_view<FMT, MODE>(s, p, u, g, t);
     if (d_lo < d_hi) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) load_tile<FMT, FULLN>(cur, d_lo, t, K, rs8, ss8, i, wq, sr);
+      for (int i = 0; i < 4; ++i) load_tile<FMT, MODE>(cur, d_lo, t, K, rb, nsr, gap, i, wq, sr);
       load_acts(cur, d_lo, t, K, xa);
     }
   }
@@ -198,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
       const bool last = d + 1 == d_hi;
       const int dn = last ? d_lo : d + 1;
       const bool has_next = !last || u + ustride < U;
-      if (last && has_next) cur = unit_view<FMT>(s, p, u + ustride, g, t);
+      if (last && has_next) cur = unit_view<FMT, MODE>(s, p, u + ustride, g, t);
       uint4 xn[4];
       if (has_next) load_acts(cur, dn, t, K, xn);
 
@@ -219,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
           const uint32_t a3 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0 + 1u), s1);
           mma_bf16_16816(acc[i], a0, a1, a2, a3, xp[2 * j], xp[2 * j + 1]);
         }
-        if (has_next) load_tile<FMT, FULLN>(cur, dn, t, K, rs8, ss8, i, wq, sr);
+        if (has_next) load_tile<FMT, MODE>(cur, dn, t, K, rb, nsr, gap, i, wq, sr);
       }
       if (has_next) {
 #pragma unroll
@@ -239,6 +252,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
       const int ht = tid & (kThreads / 2 - 1);
       if (rows > kMaxTokens) {
         if (ht == 0 && jb == 0) atomicOr(p.err, GNF4_DEVERR_GEMV_ROWS);
+      } else if (MODE == kModeSwiglu) {
+        // tiles 0, 1 hold gate rows, tiles 2, 3 the matching up rows
+        const int I = p.N / 2;
+        for (int o = ht; o < 2 * 32 * 4; o += kThreads / 2) {
+          const int i = o >> 7, l = (o >> 2) & 31, j = o & 3;
+          float vg = 0.f, vu = 0.f;
+#pragma unroll
+          for (int w = 0; w < kSplit; ++w) {
+            vg += s.red[h][w][i][l][j];
+            vu += s.red[h][w][i + 2][l][j];
+          }
+          const int col = jb * (kRows / 2) + 16 * i + (l >> 2) + 8 * (j >> 1);
+          const int tok = 2 * (l & 3) + (j & 1);
+          if (tok < rows) p.y[(size_t)(r0 + tok) * I + col] = __float2bfloat16_rn(silu_mul(vg, vu));
+        }
       } else {
         for (int o = ht; o < 4 * 32 * 4; o += kThreads / 2) {
           const int i = o >> 7, l = (o >> 2) & 31, j = o & 3;
@@ -262,26 +290,32 @@ int gemv_grid(long long units, int num_sms) {
   return (int)(ctas < num_sms ? ctas : num_sms);
 }
 
-template <int FMT, bool FULLN>
+template <int FMT, int MODE>
 static cudaError_t launch_gemv_t(const GroupedArgs& p, int grid, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, FULLN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  return launch_pdl(gemv_kernel<FMT, FULLN>, dim3(grid), dim3(kThreads), (size_t)kSmemBytes, stream, p);
+  return launch_pdl(gemv_kernel<FMT, MODE>, dim3(grid), dim3(kThreads), (size_t)kSmemBytes, stream, p);
 }
 
-cudaError_t launch_gemv(int fmt, const GroupedArgs& p, int grid, cudaStream_t stream) {
-  const bool full = p.N % kRows == 0;
-  if (fmt == 0) return full ? launch_gemv_t<0, true>(p, grid, stream) : launch_gemv_t<0, false>(p, grid, stream);
-  return full ? launch_gemv_t<1, true>(p, grid, stream) : launch_gemv_t<1, false>(p, grid, stream);
+template <int FMT>
+static cudaError_t launch_gemv_f(bool swiglu, const GroupedArgs& p, int grid, cudaStream_t stream) {
+  if (swiglu) return launch_gemv_t<FMT, kModeSwiglu>(p, grid, stream);
+  return p.N % kRows == 0 ? launch_gemv_t<FMT, kModeFull>(p, grid, stream)
+                          : launch_gemv_t<FMT, kModeClamp>(p, grid, stream);
+}
+
+cudaError_t launch_gemv(int fmt, bool swiglu, const GroupedArgs& p, int grid, cudaStream_t stream) {
+  return fmt == 0 ? launch_gemv_f<0>(swiglu, p, grid, stream) : launch_gemv_f<1>(swiglu, p, grid, stream);
 }
 
 int gemv_rows_per_block() { return kRows; }
+int gemv_swiglu_cols_per_block() { return kRows / 2; }
 
 }  // namespace gnf4

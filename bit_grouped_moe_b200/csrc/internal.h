@@ -48,12 +48,15 @@ struct GroupedArgs {
 size_t gemm_tc_smem_bytes();
 int gemm_tc_rows_per_unit();
 int gemm_tc_weight_rows_per_unit();
-cudaError_t launch_gemm_tc(int fmt, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
-                           const GroupedArgs& p, int grid, cudaStream_t stream);
+// swiglu: p.w is a gate_up stack [E, N = 2I, K/2] (tm_w with 64-row boxes) and p.y the [M, I] output h.
+cudaError_t launch_gemm_tc(int fmt, bool swiglu, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big,
+                           const CUtensorMap& tm_w, const GroupedArgs& p, int grid, cudaStream_t stream);
 
 // gemv.cu
-cudaError_t launch_gemv(int fmt, const GroupedArgs& p, int grid, cudaStream_t stream);
+// swiglu: p.w is a gate_up stack [E, N = 2I, K/2] and p.y the [M, I] output h.
+cudaError_t launch_gemv(int fmt, bool swiglu, const GroupedArgs& p, int grid, cudaStream_t stream);
 int gemv_rows_per_block();
+int gemv_swiglu_cols_per_block();
 // CTAs for a GEMV launch over `units` (expert, 64-row) units.
 int gemv_grid(long long units, int num_sms);
 

@@ -41,14 +41,16 @@ _lib.gnf4_route_workspace_bytes.argtypes = [_I, _I, _I]
 _lib.gnf4_route_workspace_bytes.restype = _SZ
 _lib.gnf4_route_permute.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P, _P]
 _lib.gnf4_route_permute_static.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]
-for _name in ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_gemv_nf4", "gnf4_grouped_gemv_mxfp4"):
+_GROUPED = ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_gemv_nf4", "gnf4_grouped_gemv_mxfp4",
+            "gnf4_grouped_gemm_nf4_swiglu", "gnf4_grouped_gemm_mxfp4_swiglu", "gnf4_grouped_gemv_nf4_swiglu",
+            "gnf4_grouped_gemv_mxfp4_swiglu")
+for _name in _GROUPED:
     getattr(_lib, _name).argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
 _lib.gnf4_dequant_nf4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 _lib.gnf4_dequant_mxfp4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
-for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", "gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4",
-              "gnf4_grouped_gemv_nf4", "gnf4_grouped_gemv_mxfp4", "gnf4_combine", "gnf4_dequant_nf4_f32",
-              "gnf4_dequant_mxfp4_f32"):
+for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", *_GROUPED, "gnf4_combine",
+              "gnf4_dequant_nf4_f32", "gnf4_dequant_mxfp4_f32"):
     getattr(_lib, _name).restype = _I
 
 
@@ -148,6 +150,30 @@ def grouped_gemv_nf4(a, w, absmax, y, offsets=None, counts=None, stream=None):
 
 def grouped_gemv_mxfp4(a, w, scales, y, offsets=None, counts=None, stream=None):
     _grouped(_lib.gnf4_grouped_gemv_mxfp4, a, w, scales, y, offsets, counts, stream)
+
+
+def _grouped_swiglu(fn, a, w_gate_up, scales, h, offsets=None, counts=None, stream=None):
+    E, N2, K2 = w_gate_up.shape
+    M = a.shape[0]
+    _check(fn(_ptr(a), _ptr(w_gate_up), _ptr(scales), _ptr(offsets), _ptr(counts), E, N2 // 2, 2 * K2, M, _ptr(h),
+              _stream(stream)))
+
+
+def grouped_gemm_nf4_swiglu(a, w_gate_up, absmax, h, offsets=None, counts=None, stream=None):
+    """h [M, I] = silu(gate) * up of the gate_up stack [E, 2I, K/2] (gate rows first)."""
+    _grouped_swiglu(_lib.gnf4_grouped_gemm_nf4_swiglu, a, w_gate_up, absmax, h, offsets, counts, stream)
+
+
+def grouped_gemm_mxfp4_swiglu(a, w_gate_up, scales, h, offsets=None, counts=None, stream=None):
+    _grouped_swiglu(_lib.gnf4_grouped_gemm_mxfp4_swiglu, a, w_gate_up, scales, h, offsets, counts, stream)
+
+
+def grouped_gemv_nf4_swiglu(a, w_gate_up, absmax, h, offsets=None, counts=None, stream=None):
+    _grouped_swiglu(_lib.gnf4_grouped_gemv_nf4_swiglu, a, w_gate_up, absmax, h, offsets, counts, stream)
+
+
+def grouped_gemv_mxfp4_swiglu(a, w_gate_up, scales, h, offsets=None, counts=None, stream=None):
+    _grouped_swiglu(_lib.gnf4_grouped_gemv_mxfp4_swiglu, a, w_gate_up, scales, h, offsets, counts, stream)
 
 
 def combine(y, flat_to_sorted, weights, out, stream=None):

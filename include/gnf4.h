@@ -184,6 +184,40 @@ gnf4_status gnf4_grouped_gemv_mxfp4(const void *a, const uint8_t *w, const uint8
                                     const int32_t *counts, int E, int N, int K, int M, void *y, void *stream);
 
 /* ------------------------------------------------------------------ */
+/* Fused gate_up projection + SwiGLU                                   */
+/* ------------------------------------------------------------------ */
+
+/* The first projection of the expert MLP with its gated activation in the
+ * epilogue (grouped-nf4-gemm releases, v0.2.5 "arena -> kernel":
+ * moe_layer_forward runs gate -> GLU -> down; index.json, system_manifest:
+ * swiglu is one of the decode glue kernels).  The pages print neither the
+ * activation nor the row order; the reading used here: w_gate_up is one
+ * stack [E, 2I, K/2] (scales [E, 2I, K/64] fp32 for NF4, [E, 2I, K/32] e8m0
+ * for MXFP4) whose rows [0, I) are the gate rows and rows [I, 2I) the up
+ * rows, and for every sorted row r of expert e
+ *     h[r, i] = silu(g) * u,  g = sum_k a[r,k] W_e[i,k],  u = sum_k a[r,k] W_e[I+i,k],
+ *     silu(x) = x / (1 + exp(-x)),
+ * with g and u accumulated in fp32 and h rounded once to bf16 [M, I].  The
+ * [M, 2I] projection output never reaches global memory.
+ *
+ * Arguments as the grouped GEMM / GEMV calls, with I (the output width) in
+ * place of N: I must be a positive multiple of 64.  The GEMV forms keep the
+ * rule of at most 8 rows per group (larger groups are skipped and flagged
+ * with GNF4_DEVERR_GEMV_ROWS). */
+gnf4_status gnf4_grouped_gemm_nf4_swiglu(const void *a, const uint8_t *w_gate_up, const float *absmax,
+                                         const int32_t *offsets, const int32_t *counts, int E, int I, int K, int M,
+                                         void *h, void *stream);
+gnf4_status gnf4_grouped_gemm_mxfp4_swiglu(const void *a, const uint8_t *w_gate_up, const uint8_t *scales,
+                                           const int32_t *offsets, const int32_t *counts, int E, int I, int K, int M,
+                                           void *h, void *stream);
+gnf4_status gnf4_grouped_gemv_nf4_swiglu(const void *a, const uint8_t *w_gate_up, const float *absmax,
+                                         const int32_t *offsets, const int32_t *counts, int E, int I, int K, int M,
+                                         void *h, void *stream);
+gnf4_status gnf4_grouped_gemv_mxfp4_swiglu(const void *a, const uint8_t *w_gate_up, const uint8_t *scales,
+                                           const int32_t *offsets, const int32_t *counts, int E, int I, int K, int M,
+                                           void *h, void *stream);
+
+/* ------------------------------------------------------------------ */
 /* Top-k combine                                                       */
 /* ------------------------------------------------------------------ */
 

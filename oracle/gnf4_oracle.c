@@ -18,9 +18,10 @@
  *   [PATCH]    grouped-nf4-gemm releases, v0.2.6 "The patch point" (argsort of
  *              the top-k ids, gather x[idxs // k], tokens_per_expert = sizes;
  *              weighting and unsorting stay with the caller).
- *   [MOE]      grouped-nf4-gemm 0.33.1 on PyPI, "API": moe_layer_forward runs
- *              gate_up -> GLU -> down; swiglu_rows is listed with the glue
- *              helpers (reading C17 for the row order and the activation).
+ *   [MOE]      grouped-nf4-gemm releases, v0.2.5 "arena -> kernel"
+ *              (moe_layer_forward runs gate -> GLU -> down), and index.json,
+ *              system_manifest.owns / entrypoints (swiglu among the decode
+ *              glue kernels); reading C17 for the row order and activation.
  *   [ARENA]    grouped-nf4-gemm releases, v0.2.5 "arena -> kernel" (expert
  *              stacks [E,N,K//2] blocks + [E,N,K//32] e8m0 scales).
  *   [QLORA]    The NF4 codebook itself is not printed on the pages; the values
