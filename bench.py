@@ -143,7 +143,7 @@ class Workload:
     """Device-resident inputs of one workload: rotating weight copies larger
     than L2, a set of token batches, and the step's output buffers."""
 
-    def __init__(self, name, device, seed, build_host_copy):
+    def __init__(self, name, device, seed, build_host_copy, swiglu=False):
         import torch
 
         from bit_grouped_moe_b200 import gnf4
@@ -195,6 +195,14 @@ class Workload:
         self.fn = {("nf4", True): f.grouped_gemv_nf4, ("nf4", False): f.grouped_gemm_nf4,
                    ("mxfp4", True): f.grouped_gemv_mxfp4, ("mxfp4", False): f.grouped_gemm_mxfp4}[
             (wl.fmt, self.decode)]
+        # optional fused gate_up + SwiGLU first projection: h [M, N1/2] feeds the second
+        self.swiglu = swiglu
+        if swiglu:
+            assert self.p1.N // 2 == self.p2.K, "SwiGLU needs the second projection's K = first projection's N / 2"
+            self.fn1 = {("nf4", True): f.grouped_gemv_nf4_swiglu, ("nf4", False): f.grouped_gemm_nf4_swiglu,
+                        ("mxfp4", True): f.grouped_gemv_mxfp4_swiglu, ("mxfp4", False): f.grouped_gemm_mxfp4_swiglu}[
+                (wl.fmt, self.decode)]
+            self.hs = torch.empty(M, self.p1.N // 2, dtype=torch.bfloat16, device=device)
 
     def _stack(self, fmt, p, seed, keep_host):
         torch = self.torch
@@ -224,8 +232,10 @@ class Workload:
 
     def proj_bytes(self, p, hit):
         """Algorithmic bytes of one projection launch: weights + scales of the
-        experts hit, activations read, outputs written."""
-        return self.weight_bytes(p, hit) + self.M * p.K * 2 + self.M * p.N * 2
+        experts hit, activations read, outputs written (N/2 columns for the
+        fused gate_up + SwiGLU first projection)."""
+        n_out = p.N // 2 if (self.swiglu and p is self.p1) else p.N
+        return self.weight_bytes(p, hit) + self.M * p.K * 2 + self.M * n_out * 2
 
     def step_weight_bytes(self, i):
         h = self.hit[i % N_BATCHES]
@@ -242,14 +252,22 @@ class Workload:
         g.route_permute(ids, x, self.E, self.off, self.s2f, self.f2s, self.xs, self.ws)
         if ev is not None:
             ev[0].record()
-        self.fn(self.xs, w1, s1, self.y1, offsets=self.off)
-        if ev is not None:
-            ev[1].record()
-        self.fn(self.h, w2, s2, self.y2, offsets=self.off)
+        self.project(w1, s1, w2, s2, ev)
         g.combine(self.y2, self.f2s, wts, self.out)
 
+    def project(self, w1, s1, w2, s2, ev=None):
+        if self.swiglu:
+            self.fn1(self.xs, w1, s1, self.hs, offsets=self.off)
+        else:
+            self.fn(self.xs, w1, s1, self.y1, offsets=self.off)
+        if ev is not None:
+            ev[1].record()
+        self.fn(self.hs if self.swiglu else self.h, w2, s2, self.y2, offsets=self.off)
+
     def launches_per_step(self):
-        return 4 + 2 + 1  # route (hist, scan, scatter, gather) + 2 projections + combine
+        # route (one launch for at most 256 pairs, else hist + scan + scatter + gather) + 2 projections + combine
+        route = 1 if 0 < self.M <= 256 else 4
+        return route + 2 + 1
 
 
 # ------------------------------------------------------------------ distributed
@@ -353,6 +371,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--impl", default="libgnf4", choices=["libgnf4", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--swiglu", action="store_true",
+                    help="first projection = fused gate_up + SwiGLU (gate rows first); the second reads its output")
     ap.add_argument("--weight-copies", type=int, default=N_WEIGHT_COPIES,
                     help="rotating copies of every weight stack (4 keeps the rotation larger than L2)")
     args = ap.parse_args()
@@ -396,7 +416,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
 
     dev = f"cuda:{local}"
     torch.cuda.set_device(local)
-    wl = Workload(args.workload, dev, seed=1234 + rank, build_host_copy=(rank == 0 and world == 1))
+    wl = Workload(args.workload, dev, seed=1234 + rank, build_host_copy=(rank == 0 and world == 1),
+                  swiglu=args.swiglu)
     wl.h_host = wl.h.cpu().view(torch.int16).numpy().view(np.uint16)
     stream = torch.cuda.current_stream()
 
@@ -449,8 +470,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         (w1, s1), (w2, s2) = wl.stacks[i % N_WEIGHT_COPIES]
         g = wl.g
         g.route_permute(d_ids, d_x, wl.E, wl.off, wl.s2f, wl.f2s, wl.xs, wl.ws)
-        wl.fn(wl.xs, w1, s1, wl.y1, offsets=wl.off)
-        wl.fn(wl.h, w2, s2, wl.y2, offsets=wl.off)
+        wl.project(w1, s1, w2, s2)
         g.combine(wl.y2, wl.f2s, d_w, wl.out)
         host_out.copy_(wl.out, non_blocking=True)
 
@@ -479,7 +499,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
 
     peaks, peak_src = load_peaks()
     kern_file = "gemv.cu" if decode else "gemm_tc.cu"
-    kern_key = f"{'gemv' if decode else 'gemm_tc'}_{wl.wl.fmt}:{args.workload}:{wl.p1.name}"
+    kern_key = f"{'gemv' if decode else 'gemm_tc'}_{wl.wl.fmt}{'_swiglu' if wl.swiglu else ''}:{args.workload}:{wl.p1.name}"
     sha = kernel_source_sha([kern_file, "common.cuh"])
     if decode:
         mean_hit = sum(wl.hit[i % N_BATCHES] for i in range(steps)) / steps
@@ -487,7 +507,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         achieved = alg / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": committed_traffic(kern_key, sha),
-                "kernel": f"gemv_kernel<{wl.wl.fmt}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})",
+                "kernel": f"gemv_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})",
                 "algorithmic_bytes_per_launch": int(alg), "avg_launch_us": round(dom_ms * 1e3, 3),
                 "peak_source": f"hbm_gbs of {peak_src}"}
     else:
@@ -496,7 +516,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         pk = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk, "unit": "TFLOP/s",
                 "frac": round(achieved / pk, 4), "traffic": committed_traffic(kern_key, sha),
-                "kernel": f"gemm_tc_kernel<{wl.wl.fmt}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})",
+                "kernel": f"gemm_tc_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})",
                 "algorithmic_flops_per_launch": int(flops), "avg_launch_us": round(dom_ms * 1e3, 3),
                 "peak_source": f"bf16_tflops_sustained of {peak_src} (kind::f16 MMA on decoded bf16 tiles)"}
 
@@ -512,7 +532,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": steps,
             "warmup": warmup, "ms_per_step": round(ms / steps, 6), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(wl.wl, world),
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(_config(wl.wl, world), **({"first_projection": "fused gate_up + SwiGLU"} if wl.swiglu else {})),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},

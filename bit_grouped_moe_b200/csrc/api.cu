@@ -149,6 +149,23 @@ gnf4_status encode_weight_map(CUtensorMap* m, const void* w, int E, int N, int K
   return GNF4_OK;
 }
 
+// gate_up stack W [E, 2I, K/2] u8 viewed as [E][I/64][2][64][K/2]: one box =
+// 32 bytes of 64 gate rows followed by the same 32 bytes of the matching 64 up rows.
+gnf4_status encode_swiglu_weight_map(CUtensorMap* m, const void* w, int E, int I, int K) {
+  auto fn = encode_fn();
+  if (!fn) return fail(GNF4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t rb = (cuuint64_t)(K / 2);
+  cuuint64_t dims[5] = {rb, 64, 2, (cuuint64_t)(I / 64), (cuuint64_t)E};
+  cuuint64_t strides[4] = {rb, (cuuint64_t)I * rb, 64 * rb, 2 * (cuuint64_t)I * rb};
+  cuuint32_t box[5] = {32, 64, 2, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(w), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GNF4_ERR_CUDA, "gate_up tensor map encode failed (CUresult %d)", (int)r);
+  return GNF4_OK;
+}
+
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 // Shared validation of the grouped GEMM / GEMV arguments.
@@ -185,7 +202,10 @@ gnf4_status grouped_gemm(int fmt, bool swiglu, const void* a, const uint8_t* w, 
   GNF4_TRY(encode_act_map(&tm_a, a, M, K, 32));
   GNF4_TRY(encode_act_map(&tm_a_big, a, M, K, 128));
   const int wrows = gemm_tc_weight_rows_per_unit();
-  GNF4_TRY(encode_weight_map(&tm_w, w, E, N, K, 32, swiglu ? wrows / 2 : wrows));
+  if (swiglu)
+    GNF4_TRY(encode_swiglu_weight_map(&tm_w, w, E, N / 2, K));
+  else
+    GNF4_TRY(encode_weight_map(&tm_w, w, E, N, K, 32, wrows));
   GroupedArgs p{static_cast<const __nv_bfloat16*>(a), w, scales, offsets, counts,
                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
   // upper bound on work units: every group adds at most one partial chunk

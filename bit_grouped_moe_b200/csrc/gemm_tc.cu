@@ -204,9 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = it % kWStages, use = it / kWStages;
           if (it >= kWStages && !(ok = mbar_wait(&s.wempty[st], (use - 1) & 1, err, abort))) break;
           mbar_arrive_expect_tx(&s.wfull[st], kWStageBytes);
-          if (SWI) {  // two 64-row boxes: gate rows, then the matching up rows
-            tma_load_3d(s.wq[st], &tm_w, &s.wfull[st], kt * (kBK / 2), x.j * (kBW / 2), x.e);
-            tma_load_3d(s.wq[st] + kWStageBytes / 2, &tm_w, &s.wfull[st], kt * (kBK / 2), I + x.j * (kBW / 2), x.e);
+          if (SWI) {  // one box of 64 gate rows followed by the matching 64 up rows
+            tma_load_5d(s.wq[st], &tm_w, &s.wfull[st], kt * (kBK / 2), 0, 0, x.j, x.e);
           } else {
             tma_load_3d(s.wq[st], &tm_w, &s.wfull[st], kt * (kBK / 2), x.j * kBW, x.e);
           }
@@ -416,18 +415,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int lim = min(32, x.rows - c * 32);
         if (SWI) {
-          // lane x < 16 holds gate(col), lane x + 16 up(col): exchange, then the
-          // low lanes store even rows and the high lanes odd rows
+          // lane x < 16 holds gate(col), lane x + 16 up(col).  Per pair of rows
+          // (2m, 2m+1) the low lane finishes row 2m and the high lane row 2m+1:
+          // each sends its partner the value the partner lacks.
           const bool up_lane = lane >= 16;
           const int col = x.j * (kBW / 2) + q * 16 + (lane & 15);
           __nv_bfloat16* hcol = p.y + (size_t)x.row0 * I + col;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float mine = __uint_as_float(v[i]);
-            const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
-            const float g = up_lane ? other : mine, uu = up_lane ? mine : other;
-            if (i < lim && (i & 1) == (int)up_lane)
-              hcol[(size_t)(c * 32 + i) * I] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * uu);
+          for (int m = 0; m < 16; ++m) {
+            const float keep = __uint_as_float(v[2 * m + (up_lane ? 1 : 0)]);
+            const float send = __uint_as_float(v[2 * m + (up_lane ? 0 : 1)]);
+            const float got = __shfl_xor_sync(0xffffffffu, send, 16);
+            const int i = 2 * m + (up_lane ? 1 : 0);
+            // low lane: gate = keep (row 2m), up = got; high lane: up = keep (row 2m+1), gate = got
+            const float g = up_lane ? got : keep, uu = up_lane ? keep : got;
+            if (i < lim) hcol[(size_t)(c * 32 + i) * I] = __float2bfloat16_rn(silu_mul(g, uu));
           }
         } else if (n < p.N) {
 #pragma unroll

@@ -75,9 +75,6 @@ __device__ __forceinline__ uint32_t lut_lookup(uint32_t word, uint32_t lanesel, 
   return v;
 }
 
-// silu(g) * u = g / (1 + e^-g) * u in fp32.
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
-
 __device__ __forceinline__ void half_barrier(int h) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + h), "r"(kThreads / 2) : "memory");
 }
