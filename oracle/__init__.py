@@ -57,6 +57,7 @@ def _load():
     lib.orc_grouped_gemm_mxfp4.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
     lib.orc_combine.argtypes = [P, P, P, I64, I64, I64, P]
     lib.orc_swiglu.argtypes = [P, I64, I64, P]
+    lib.orc_router_topk.argtypes = [P, P, I64, I64, I64, P, P]
     _lib = lib
     return lib
 
@@ -220,3 +221,15 @@ def grouped_gemm_swiglu(fmt: str, a_bits, w, scales, offsets, rows=None):
     stack followed by swiglu()."""
     fn = grouped_gemm_nf4 if fmt == "nf4" else grouped_gemm_mxfp4
     return swiglu(fn(a_bits, w, scales, offsets, rows=rows))
+
+
+def router_topk(logits: np.ndarray, k: int, bias: np.ndarray | None = None):
+    """(ids int32 [T, k], weights fp64 [T, k]): top-k of logits + bias (fp32),
+    softmax over the selected raw logits."""
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    b = None if bias is None else _c(bias, np.float32)
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    _load().orc_router_topk(_p(lg), None if b is None else _p(b), T, E, k, _p(ids), _p(w))
+    return ids, w

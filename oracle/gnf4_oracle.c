@@ -22,6 +22,10 @@
  *              (moe_layer_forward runs gate -> GLU -> down), and index.json,
  *              system_manifest.owns / entrypoints (swiglu among the decode
  *              glue kernels); reading C17 for the row order and activation.
+ *   [ROUTER]   grouped-nf4-gemm index.json, problems_solved[5] ("router softmax
+ *              and top-k" among the decode tail folded into one launch) and
+ *              entrypoints (int4_b32:router_epilogue); reading C18 for ties,
+ *              the optional bias and the softmax over the selected logits.
  *   [ARENA]    grouped-nf4-gemm releases, v0.2.5 "arena -> kernel" (expert
  *              stacks [E,N,K//2] blocks + [E,N,K//32] e8m0 scales).
  *   [QLORA]    The NF4 codebook itself is not printed on the pages; the values
@@ -422,5 +426,58 @@ void orc_swiglu(const double *gu, int64_t rows, int64_t I, double *h)
             const double u = gu[r * 2 * I + I + i];
             h[r * I + i] = g / (1.0 + exp(-g)) * u;
         }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Router epilogue: top-k selection and softmax weights [ROUTER]       */
+/* ------------------------------------------------------------------ */
+
+/* Rank of a score in the selection order: NaN below every number. */
+static int score_before(float a, int64_t ia, float b, int64_t ib)
+{
+    const int na = isnan(a), nb = isnan(b);
+    if (na != nb) return nb; /* the non-NaN one comes first */
+    if (!na && a != b) return a > b;
+    return ia < ib; /* equal (or both NaN): lower expert index first */
+}
+
+/* For every token t (reading C18):
+ *   score[e] = logits[t, e] + bias[e]  (one fp32 addition, bias may be NULL),
+ *   ids[t, 0..k) = the k distinct experts with the largest scores, in
+ *                  descending score order, ties to the lower expert index,
+ *                  NaN scores ranked below every number;
+ *   weights[t, j] = exp(l_j - m) / sum_i exp(l_i - m) over the RAW logits l of
+ *                   the k selected experts, m = their maximum (fp64 here).
+ * The selection is taken in fp32, the precision of the scores. */
+void orc_router_topk(const float *logits, const float *bias, int64_t T, int64_t E, int64_t k, int32_t *ids,
+                     double *weights)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        const float *row = logits + t * E;
+        for (int64_t j = 0; j < k; ++j) {
+            int64_t best = -1;
+            float bs = 0.0f;
+            for (int64_t e = 0; e < E; ++e) {
+                int taken = 0;
+                for (int64_t i = 0; i < j; ++i)
+                    if (ids[t * k + i] == (int32_t)e) taken = 1;
+                if (taken) continue;
+                const float s = bias != NULL ? row[e] + bias[e] : row[e];
+                if (best < 0 || score_before(s, e, bs, best)) {
+                    best = e;
+                    bs = s;
+                }
+            }
+            ids[t * k + j] = (int32_t)best;
+        }
+        double m = -INFINITY;
+        for (int64_t j = 0; j < k; ++j) {
+            const double l = (double)row[ids[t * k + j]];
+            if (l > m || isnan(l)) m = l;
+        }
+        double sum = 0.0;
+        for (int64_t j = 0; j < k; ++j) sum += exp((double)row[ids[t * k + j]] - m);
+        for (int64_t j = 0; j < k; ++j) weights[t * k + j] = exp((double)row[ids[t * k + j]] - m) / sum;
     }
 }

@@ -410,3 +410,51 @@ def test_swiglu_takes_the_gate_half_first():
         swapped = oracle.swiglu(np.array([[rs / 2.0, rs]]))[0, 0]
         assert np.all(h[r] == ref)
         assert rs == 0.0 or ref != swapped
+
+
+# ------------------------------------------------------------------ router epilogue (reading C18)
+
+
+def test_router_selection_is_a_stable_descending_sort():
+    """numpy's stable argsort of the negated fp32 scores (ties to the lower index)."""
+    g = inputs.rng(60)
+    T, E, k = 40, 24, 6
+    logits = (np.round(g.standard_normal((T, E)) * 2) / 2).astype(np.float32)  # coarse grid: many ties
+    bias = (np.round(g.standard_normal(E)) / 4).astype(np.float32)
+    ids, _ = oracle.router_topk(logits, k, bias)
+    score = (logits + bias[None, :]).astype(np.float32)
+    ref = np.argsort(-score, axis=1, kind="stable")[:, :k]
+    assert np.array_equal(ids, ref)
+    ids0, _ = oracle.router_topk(logits, k)
+    assert np.array_equal(ids0, np.argsort(-logits, axis=1, kind="stable")[:, :k])
+
+
+def test_router_weights_closed_forms():
+    """softmax(0, ln 3) = (1/4, 3/4); one expert gets weight 1; equal logits share 1/k."""
+    L = math.log(3.0)
+    logits = np.array([[0.0, -5.0, np.float32(L), -7.0],
+                       [1.0, 1.0, 1.0, 1.0]], np.float32)
+    ids, w = oracle.router_topk(logits, 2)
+    assert list(ids[0]) == [2, 0]
+    assert abs(w[0, 0] - 0.75) < 1e-7 and abs(w[0, 1] - 0.25) < 1e-7  # L rounded to fp32
+    assert list(ids[1]) == [0, 1] and np.all(w[1] == 0.5)
+    _, w1 = oracle.router_topk(logits, 1)
+    assert np.all(w1 == 1.0)
+    _, w4 = oracle.router_topk(logits[1:], 4)
+    assert np.all(w4 == 0.25)
+
+
+def test_router_bias_moves_selection_not_weights():
+    """A bias picks experts 3 and 1, whose raw logits ln 3 and 0 set the weights."""
+    L = np.float32(math.log(3.0))
+    logits = np.array([[5.0, 0.0, 4.0, L]], np.float32)
+    bias = np.array([-100.0, 50.0, -100.0, 60.0], np.float32)
+    ids, w = oracle.router_topk(logits, 2, bias)
+    assert list(ids[0]) == [3, 1]
+    assert abs(w[0, 0] - 0.75) < 1e-7 and abs(w[0, 1] - 0.25) < 1e-7
+
+
+def test_router_ranks_nan_scores_last():
+    logits = np.array([[np.nan, -1e30, 2.0, np.nan]], np.float32)
+    ids, _ = oracle.router_topk(logits, 4)
+    assert list(ids[0]) == [2, 1, 0, 3]
