@@ -313,6 +313,44 @@ gnf4_status gnf4_route_permute(const int32_t* topk_ids, const void* x, int T, in
   return GNF4_OK;
 }
 
+gnf4_status gnf4_route_topk_permute(const float* logits, const float* bias, int T, int E, int k, const void* x, int K,
+                                    int32_t* topk_ids, float* topk_weights, int32_t* offsets,
+                                    int32_t* sorted_to_flat, int32_t* flat_to_sorted, void* x_sorted,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T=%d is negative", T);
+  if (E < 1 || E > 4096) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "E=%d outside [1, 4096]", E);
+  if (k < 1 || k > E || k > kMaxRouterTopK)
+    return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, min(E=%d, %d)]", k, E, kMaxRouterTopK);
+  if (K < 8 || K % 8 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K=%d must be a positive multiple of 8", K);
+  if ((long long)T * k > (1LL << 30)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T*k too large");
+  GNF4_TRY(check_ptr(offsets, "offsets", 4));
+  GNF4_TRY(check_ptr(bias, "bias", 4, false));
+  if (T > 0) {
+    GNF4_TRY(check_ptr(logits, "logits", 4));
+    GNF4_TRY(check_ptr(x, "x", 16));
+    GNF4_TRY(check_ptr(topk_ids, "topk_ids", 4));
+    GNF4_TRY(check_ptr(topk_weights, "topk_weights", 4));
+    GNF4_TRY(check_ptr(sorted_to_flat, "sorted_to_flat", 4));
+    GNF4_TRY(check_ptr(flat_to_sorted, "flat_to_sorted", 4));
+    GNF4_TRY(check_ptr(x_sorted, "x_sorted", 16));
+  }
+  const size_t need = route_workspace_bytes(T, k, E);
+  if (need > 0) {
+    if (workspace_bytes < need)
+      return fail(GNF4_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu bytes needed",
+                  workspace_bytes, need);
+    GNF4_TRY(check_ptr(workspace, "workspace", 16));
+  }
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  cudaError_t e = launch_route_topk(logits, bias, T, E, k, static_cast<const __nv_bfloat16*>(x), K, topk_ids,
+                                    topk_weights, offsets, sorted_to_flat, flat_to_sorted,
+                                    static_cast<__nv_bfloat16*>(x_sorted), workspace, d->num_sms,
+                                    as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "route_topk_permute launch");
+  return GNF4_OK;
+}
+
 gnf4_status gnf4_grouped_gemm_nf4(const void* a, const uint8_t* w, const float* absmax, const int32_t* offsets,
                                   const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
   return grouped_gemm(0, false, a, w, absmax, offsets, counts, E, N, K, M, y, stream);

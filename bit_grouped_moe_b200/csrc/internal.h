@@ -67,6 +67,13 @@ cudaError_t launch_route(const int32_t* topk_ids, const __nv_bfloat16* x, int T,
                          __nv_bfloat16* x_sorted, void* workspace, int32_t* bad_id_count, int num_sms,
                          cudaStream_t stream);
 
+// Router epilogue (top-k of logits + bias, softmax weights) followed by the routing above.
+cudaError_t launch_route_topk(const float* logits, const float* bias, int T, int E, int k, const __nv_bfloat16* x,
+                              int K, int32_t* topk_ids, float* topk_weights, int32_t* offsets,
+                              int32_t* sorted_to_flat, int32_t* flat_to_sorted, __nv_bfloat16* x_sorted,
+                              void* workspace, int num_sms, cudaStream_t stream);
+constexpr int kMaxRouterTopK = 32;
+
 // combine.cu
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* flat_to_sorted, const float* weights, int T,
                            int k, int N, __nv_bfloat16* out, int num_sms, cudaStream_t stream);

@@ -169,23 +169,129 @@ __global__ void route_gather_kernel(const uint4* x, int K8, int k, const int32_t
 }
 
 
+// ---------------------------------------------------------------- router epilogue
+// Top-k of score = logit + bias (fp32) per token and the softmax of the
+// selected raw logits (grouped-nf4-gemm index.json, problems_solved[5]:
+// router softmax and top-k among the decode tail folded into one launch).
+constexpr int kMaxRouterK = 32;
+
+// Selection order: NaN scores after every number, larger scores first, ties
+// to the lower expert index; an index < 0 is "no candidate".
+__device__ __forceinline__ bool sel_before(float a, int ia, float b, int ib) {
+  if (ib < 0) return ia >= 0;
+  if (ia < 0) return false;
+  const bool na = a != a, nb = b != b;
+  if (na != nb) return nb;
+  if (!na && a != b) return a > b;
+  return ia < ib;
+}
+
+// One warp, one token: lane j < k ends with the j-th selected expert in
+// *id and its weight in *w.  Lane l scans experts l, l+32, ...; the experts
+// it has lost to the selection are bits of four words (E <= 4096).
+__device__ __forceinline__ void router_warp(const float* row, const float* bias, int E, int k, int lane, int* id,
+                                            float* w) {
+  uint32_t tk0 = 0u, tk1 = 0u, tk2 = 0u, tk3 = 0u;
+  int mine = -1;
+  for (int j = 0; j < k; ++j) {
+    float bv = 0.f;
+    int bi = -1;
+    for (int c = 0, e = lane; e < E; ++c, e += 32) {
+      const uint32_t word = c < 32 ? tk0 : (c < 64 ? tk1 : (c < 96 ? tk2 : tk3));
+      if ((word >> (c & 31)) & 1u) continue;
+      const float sc = bias != nullptr ? row[e] + bias[e] : row[e];
+      if (sel_before(sc, e, bv, bi)) {
+        bv = sc;
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, d);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, d);
+      if (sel_before(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (bi >= 0 && (bi & 31) == lane) {
+      const int c = bi >> 5;
+      const uint32_t bit = 1u << (c & 31);
+      if (c < 32) tk0 |= bit;
+      else if (c < 64) tk1 |= bit;
+      else if (c < 96) tk2 |= bit;
+      else tk3 |= bit;
+    }
+    if (lane == j) mine = bi;
+  }
+  // softmax over the selected raw logits (a NaN logit makes every weight NaN)
+  const float l = lane < k ? row[mine] : -INFINITY;
+  float m = l;
+#pragma unroll
+  for (int d = 16; d >= 1; d >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, m, d);
+    if (m == m && (o != o || o > m)) m = o;
+  }
+  const float ex = lane < k ? expf(l - m) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int d = 16; d >= 1; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
+  *id = mine;
+  *w = ex / sum;
+}
+
+__global__ void __launch_bounds__(256) router_kernel(const float* logits, const float* bias, int T, int E, int k,
+                                                     int32_t* ids, float* weights) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (t >= T) return;  // uniform over the warp
+  int id;
+  float w;
+  router_warp(logits + (size_t)t * E, bias, E, k, lane, &id, &w);
+  if (lane < k) {
+    ids[(size_t)t * k + lane] = id;
+    weights[(size_t)t * k + lane] = w;
+  }
+}
+
 // Single-launch routing for M <= kChunk pairs: each block sorts all pairs in
 // shared memory (same counting sort, same ranks), block 0 writes offsets and
 // permutations, and block b gathers rows b, b + gridDim.x, ...
+// With logits != nullptr the block first runs the router epilogue for all
+// T = M / k tokens (ids into shared memory; block 0 also writes ids and
+// weights out) and sorts those ids.
 __global__ void __launch_bounds__(kChunk) route_small_kernel(const int32_t* ids, int M, int E, const uint4* x,
                                                              int K8, int k, int32_t* offsets, int32_t* s2f,
-                                                             int32_t* f2s, int32_t* bad_out, uint4* xs) {
+                                                             int32_t* f2s, int32_t* bad_out, uint4* xs,
+                                                             const float* logits, const float* bias,
+                                                             int32_t* ids_out, float* w_out) {
   griddep_launch_dependents();
   griddep_wait();
   __shared__ int cnt[kMaxRouteExperts];
   __shared__ int s2f_sm[kChunk];
+  __shared__ int ids_sm[kChunk];
   __shared__ int wsum[kChunk / 32];
   __shared__ int nbad, nvalid_sm;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   for (int i = tid; i < E; i += kChunk) cnt[i] = 0;
   if (tid == 0) nbad = 0;
+  if (logits != nullptr) {
+    for (int t = wid; t * k < M; t += kChunk / 32) {  // uniform over the warp
+      int id;
+      float w;
+      router_warp(logits + (size_t)t * E, bias, E, k, lane, &id, &w);
+      if (lane < k) {
+        ids_sm[t * k + lane] = id;
+        if (blockIdx.x == 0) {
+          ids_out[t * k + lane] = id;
+          w_out[t * k + lane] = w;
+        }
+      }
+    }
+  }
   __syncthreads();
-  const int e = (tid < M) ? ids[tid] : -1;
+  const int e = (tid < M) ? (logits != nullptr ? ids_sm[tid] : ids[tid]) : -1;
   const bool valid = tid < M && e >= 0 && e < E;
   if (valid) atomicAdd(&cnt[e], 1);
   else if (tid < M) atomicAdd(&nbad, 1);
@@ -273,7 +379,8 @@ cudaError_t launch_route(const int32_t* topk_ids, const __nv_bfloat16* x, int T,
     const int grid = M < 2 * num_sms ? M : 2 * num_sms;
     return launch_pdl(route_small_kernel, dim3(grid), dim3(kChunk), 0, stream, topk_ids, M, E,
                       reinterpret_cast<const uint4*>(x), K / 8, k, offsets, sorted_to_flat, flat_to_sorted,
-                      bad_id_count, reinterpret_cast<uint4*>(x_sorted));
+                      bad_id_count, reinterpret_cast<uint4*>(x_sorted), (const float*)nullptr,
+                      (const float*)nullptr, (int32_t*)nullptr, (float*)nullptr);
   }
   const int nchunk = (M + kChunk - 1) / kChunk;
   int32_t* hist = reinterpret_cast<int32_t*>(workspace);
@@ -301,6 +408,26 @@ cudaError_t launch_route(const int32_t* topk_ids, const __nv_bfloat16* x, int T,
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_route_topk(const float* logits, const float* bias, int T, int E, int k, const __nv_bfloat16* x,
+                              int K, int32_t* topk_ids, float* topk_weights, int32_t* offsets,
+                              int32_t* sorted_to_flat, int32_t* flat_to_sorted, __nv_bfloat16* x_sorted,
+                              void* workspace, int num_sms, cudaStream_t stream) {
+  const int M = T * k;
+  if (M > 0 && M <= kChunk) {
+    const int grid = M < 2 * num_sms ? M : 2 * num_sms;
+    return launch_pdl(route_small_kernel, dim3(grid), dim3(kChunk), 0, stream, (const int32_t*)topk_ids, M, E,
+                      reinterpret_cast<const uint4*>(x), K / 8, k, offsets, sorted_to_flat, flat_to_sorted,
+                      (int32_t*)nullptr, reinterpret_cast<uint4*>(x_sorted), logits, bias, topk_ids, topk_weights);
+  }
+  if (M > 0) {
+    cudaError_t e = launch_pdl(router_kernel, dim3((T + 7) / 8), dim3(256), 0, stream, logits, bias, T, E, k,
+                               topk_ids, topk_weights);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_route(topk_ids, x, T, k, E, K, offsets, sorted_to_flat, flat_to_sorted, x_sorted, workspace,
+                      nullptr, num_sms, stream);
 }
 
 }  // namespace gnf4

@@ -41,6 +41,7 @@ _lib.gnf4_route_workspace_bytes.argtypes = [_I, _I, _I]
 _lib.gnf4_route_workspace_bytes.restype = _SZ
 _lib.gnf4_route_permute.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P, _P]
 _lib.gnf4_route_permute_static.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]
+_lib.gnf4_route_topk_permute.argtypes = [_P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
 _GROUPED = ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_gemv_nf4", "gnf4_grouped_gemv_mxfp4",
             "gnf4_grouped_gemm_nf4_swiglu", "gnf4_grouped_gemm_mxfp4_swiglu", "gnf4_grouped_gemv_nf4_swiglu",
             "gnf4_grouped_gemv_mxfp4_swiglu")
@@ -49,7 +50,8 @@ for _name in _GROUPED:
 _lib.gnf4_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
 _lib.gnf4_dequant_nf4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 _lib.gnf4_dequant_mxfp4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
-for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", *_GROUPED, "gnf4_combine",
+for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", "gnf4_route_topk_permute",
+              *_GROUPED, "gnf4_combine",
               "gnf4_dequant_nf4_f32", "gnf4_dequant_mxfp4_f32"):
     getattr(_lib, _name).restype = _I
 
@@ -110,6 +112,19 @@ def route_permute(topk_ids, x, E, offsets, sorted_to_flat, flat_to_sorted, x_sor
                                    _ptr(flat_to_sorted), _ptr(x_sorted), _ptr(workspace),
                                    0 if workspace is None else workspace.numel() * workspace.element_size(),
                                    _ptr(bad_id_count), _stream(stream)))
+
+
+def route_topk_permute(logits, x, k, topk_ids, topk_weights, offsets, sorted_to_flat, flat_to_sorted, x_sorted,
+                       workspace, bias=None, stream=None) -> None:
+    """Router epilogue (top-k of logits + bias, softmax over the selected logits)
+    followed by route_permute on the selected ids; all outputs preallocated."""
+    T, E = logits.shape
+    K = x.shape[1]
+    _check(_lib.gnf4_route_topk_permute(_ptr(logits), _ptr(bias), T, E, k, _ptr(x), K, _ptr(topk_ids),
+                                        _ptr(topk_weights), _ptr(offsets), _ptr(sorted_to_flat),
+                                        _ptr(flat_to_sorted), _ptr(x_sorted), _ptr(workspace),
+                                        0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                        _stream(stream)))
 
 
 ROUTE_STATIC_SCRATCH_BYTES = 1 << 20  # GNF4_ROUTE_STATIC_SCRATCH_BYTES in include/gnf4.h

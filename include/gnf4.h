@@ -143,6 +143,34 @@ gnf4_status gnf4_route_permute_static(const int32_t *topk_ids, const void *x, in
                                       void *x_sorted, int32_t *bad_id_count, void *stream);
 
 /* ------------------------------------------------------------------ */
+/* Router epilogue + routing                                           */
+/* ------------------------------------------------------------------ */
+
+/* The router's softmax and top-k fused with the routing above
+ * (grouped-nf4-gemm index.json, problems_solved[5]: router softmax and
+ * top-k among the decode tail folded into one launch; entrypoints:
+ * int4_b32:router_epilogue).  For every token t, with score[e] =
+ * logits[t, e] + bias[e] computed in fp32 (bias NULL = no bias):
+ *   topk_ids[t, 0..k)     the k distinct experts with the largest scores,
+ *                         descending; ties go to the lower expert index;
+ *                         NaN scores rank below every number;
+ *   topk_weights[t, j]    softmax over the k selected RAW logits (the bias
+ *                         moves the selection only), fp32;
+ * then offsets, sorted_to_flat, flat_to_sorted and x_sorted exactly as
+ * gnf4_route_permute computes them from topk_ids.
+ *
+ * logits: device fp32 [T, E] (4-byte aligned); bias: device fp32 [E] or
+ * NULL; x: bf16 [T, K]; outputs as gnf4_route_permute plus topk_ids int32
+ * [T, k] and topk_weights fp32 [T, k].  1 <= k <= min(E, 32), E <= 4096;
+ * workspace as gnf4_route_workspace_bytes(T, k, E).  T*k <= 256 runs as one
+ * launch.  The pages fix no tie rule or weight convention: this is a
+ * reading. */
+gnf4_status gnf4_route_topk_permute(const float *logits, const float *bias, int T, int E, int k, const void *x, int K,
+                                    int32_t *topk_ids, float *topk_weights, int32_t *offsets,
+                                    int32_t *sorted_to_flat, int32_t *flat_to_sorted, void *x_sorted,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------ */
 /* Grouped GEMM (prefill: any number of rows per group)                */
 /* ------------------------------------------------------------------ */
 
