@@ -38,6 +38,8 @@ DEFAULT_WORKLOAD = "olmoe-decode-t8"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 N_WEIGHT_COPIES = 4  # default; --weight-copies changes it (profiling uses 1)
 N_BATCHES = 8
+GRAPH_STEPS = 20  # steps captured per CUDA graph (decode timing only)
+EVENT_EVERY = 7  # the dominant kernel is event-timed on every 7th timed step (7 is coprime with the batch and copy rotations)
 
 
 # ------------------------------------------------------------------ helpers
@@ -371,6 +373,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--impl", default="libgnf4", choices=["libgnf4", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help=f"decode: also time the steps replayed from one CUDA graph of {20} steps")
     ap.add_argument("--swiglu", action="store_true",
                     help="first projection = fused gate_up + SwiGLU (gate rows first); the second reads its output")
     ap.add_argument("--weight-copies", type=int, default=N_WEIGHT_COPIES,
@@ -428,7 +432,10 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     assert wl.g.device_errors() == 0, "device error word set during warm-up"
 
     # timed region (inputs resident): K steps, events around the dominant kernel
-    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    # The dominant kernel is timed with events on every EVENT_EVERY-th step: an
+    # event between two launches ends the programmatic overlap of the pair.
+    sampled = [i for i in range(steps) if i % EVENT_EVERY == 0]
+    ev_pairs = {i: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for i in sampled}
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     sampler.start()
@@ -438,7 +445,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     t_wall0 = time.time()
     start.record(stream)
     for i in range(steps):
-        wl.step(i, ev_pairs[i])
+        wl.step(i, ev_pairs.get(i))
     stop.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
@@ -448,7 +455,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     clocks = sampler.summary(t_wall0, t_wall1)
     ms_local = start.elapsed_time(stop)
     ms = max_over_ranks(ms_local, world)
-    dom_ms = sum(a.elapsed_time(b) for a, b in ev_pairs) / steps
+    dom_ms = sum(a.elapsed_time(b) for a, b in ev_pairs.values()) / len(ev_pairs)
     assert wl.g.device_errors() == 0, "device error word set during the timed steps"
 
     # e2e through the public API with host buffers (pinned), copies in the timed region
@@ -488,6 +495,37 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     h2d = int(wl.batches[0][0].nbytes + wl.batches[0][1].nbytes + wl.batches[0][2].nbytes)
     d2h = int(host_out.numel() * 2)
 
+    # decode: the same steps replayed from one CUDA graph of GRAPH_STEPS steps
+    graph = None
+    if decode and args.graph:
+        gs = torch.cuda.Stream()
+        gs.wait_stream(stream)
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(gs):
+            for i in range(2):
+                wl.step(i)
+            gs.synchronize()
+            with torch.cuda.graph(cg, stream=gs):
+                for i in range(GRAPH_STEPS):
+                    wl.step(i)
+        torch.cuda.synchronize()
+        reps = max(1, steps // GRAPH_STEPS)
+        for _ in range(3):
+            cg.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(reps):
+            cg.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        g_ms = max_over_ranks(g0.elapsed_time(g1), world) / (reps * GRAPH_STEPS)
+        gbytes = sum(wl.step_weight_bytes(i) for i in range(GRAPH_STEPS)) / GRAPH_STEPS
+        graph = {"ms_per_step": round(g_ms, 6), "value": round(world * gbytes / (g_ms / 1e3) / 1e9, 3),
+                 "unit": "GB/s", "steps_per_graph": GRAPH_STEPS, "replays": reps}
+        del cg
+        assert wl.g.device_errors() == 0, "device error word set during the graph replays"
+
     unit, _ = _unit(decode)
     if decode:
         per_rank = sum(wl.step_weight_bytes(i) for i in range(steps))
@@ -502,7 +540,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     kern_key = f"{'gemv' if decode else 'gemm_tc'}_{wl.wl.fmt}{'_swiglu' if wl.swiglu else ''}:{args.workload}:{wl.p1.name}"
     sha = kernel_source_sha([kern_file, "common.cuh"])
     if decode:
-        mean_hit = sum(wl.hit[i % N_BATCHES] for i in range(steps)) / steps
+        mean_hit = sum(wl.hit[i % N_BATCHES] for i in sampled) / len(sampled)
         alg = wl.proj_bytes(wl.p1, mean_hit)
         achieved = alg / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -538,6 +576,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
             "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
             "gpu_launches": steps * wl.launches_per_step(), "clocks": clocks, "impl": "libgnf4",
+            **({"cuda_graph": graph} if graph is not None else {}),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
