@@ -353,7 +353,7 @@ def cpu_baseline(wl_obj, budget_s=15.0):
     n_slice -= n_slice % 8
     tot_b, tot_f, steps = 0, 0, 0
     t0 = time.perf_counter()
-    while time.perf_counter() - t0 < budget_s and steps < 6:
+    while time.perf_counter() - t0 < budget_s and steps < 400:
         b, f = oracle_step(wl_obj, steps, n_slice=n_slice)
         tot_b += b
         tot_f += f
