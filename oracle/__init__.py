@@ -58,6 +58,8 @@ def _load():
     lib.orc_combine.argtypes = [P, P, P, I64, I64, I64, P]
     lib.orc_swiglu.argtypes = [P, I64, I64, P]
     lib.orc_router_topk.argtypes = [P, P, I64, I64, I64, P, P]
+    lib.orc_grouped_dgrad_nf4.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
+    lib.orc_grouped_dgrad_mxfp4.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
     _lib = lib
     return lib
 
@@ -233,3 +235,20 @@ def router_topk(logits: np.ndarray, k: int, bias: np.ndarray | None = None):
     w = np.empty((T, k), np.float64)
     _load().orc_router_topk(_p(lg), None if b is None else _p(b), T, E, k, _p(ids), _p(w))
     return ids, w
+
+
+def grouped_dgrad(fmt: str, dy_bits, w, scales, offsets, rows=None):
+    """fp64 dX[rows, K] = dY[rows, :] . W_e for each row's expert (dY [M, N] bf16 patterns)."""
+    dy_bits = _c(dy_bits, np.uint16)
+    w = _c(w, np.uint8)
+    scales = _c(scales, np.float32 if fmt == "nf4" else np.uint8)
+    offsets = _c(offsets, np.int32)
+    E, N, K2 = w.shape
+    K = 2 * K2
+    if rows is None:
+        rows = np.arange(int(offsets[-1]), dtype=np.int64)
+    rows = _c(rows, np.int64)
+    dx = np.empty((rows.shape[0], K), np.float64)
+    fn = _load().orc_grouped_dgrad_nf4 if fmt == "nf4" else _load().orc_grouped_dgrad_mxfp4
+    fn(_p(dy_bits), _p(w), _p(scales), _p(offsets), E, N, K, _p(rows), rows.shape[0], _p(dx))
+    return dx

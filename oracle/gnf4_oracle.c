@@ -26,6 +26,9 @@
  *              and top-k" among the decode tail folded into one launch) and
  *              entrypoints (int4_b32:router_epilogue); reading C18 for ties,
  *              the optional bias and the softmax over the selected logits.
+ *   [DGRAD]    grouped-nf4-gemm index.json, system_manifest.owns ("grouped packed
+ *              GEMM (NF4 and native MXFP4) and its dgrad") and entrypoints
+ *              (nf4_grouped:dgrad_4bit_grouped): dX = dY . W on the same stacks.
  *   [ARENA]    grouped-nf4-gemm releases, v0.2.5 "arena -> kernel" (expert
  *              stacks [E,N,K//2] blocks + [E,N,K//32] e8m0 scales).
  *   [QLORA]    The NF4 codebook itself is not printed on the pages; the values
@@ -480,4 +483,60 @@ void orc_router_topk(const float *logits, const float *bias, int64_t T, int64_t 
         for (int64_t j = 0; j < k; ++j) sum += exp((double)row[ids[t * k + j]] - m);
         for (int64_t j = 0; j < k; ++j) weights[t * k + j] = exp((double)row[ids[t * k + j]] - m) / sum;
     }
+}
+
+/* ------------------------------------------------------------------ */
+/* Data gradient of the grouped projection [DGRAD]                     */
+/* ------------------------------------------------------------------ */
+
+/* For every requested sorted row r (rows[i], i < n_rows) of expert e:
+ *     dx[i, k] = sum_n dy[r, n] * W_e[n, k]        (fp64 accumulation)
+ * with W_e the fp32 dequantised weights [N, K] of expert e (the same stack
+ * the forward call reads) and dy [M, N] bf16 patterns.  fmt 0 = NF4, 1 =
+ * MXFP4.  Rows outside [0, offsets[E]) give NaN. */
+static void grouped_dgrad(int fmt, const uint16_t *dy, const uint8_t *w, const void *scales,
+                          const int32_t *offsets, int64_t E, int64_t N, int64_t K, const int64_t *rows,
+                          int64_t n_rows, double *dx)
+{
+    float *wd = (float *)malloc((size_t)(N * K) * sizeof(float));
+    for (int64_t i = 0; i < n_rows; ++i) {
+        int64_t owner = -1;
+        for (int64_t e = 0; e < E; ++e)
+            if (rows[i] >= offsets[e] && rows[i] < offsets[e + 1]) owner = e;
+        if (owner < 0)
+            for (int64_t kk = 0; kk < K; ++kk) dx[i * K + kk] = NAN;
+    }
+    for (int64_t e = 0; e < E; ++e) {
+        int used = 0;
+        for (int64_t i = 0; i < n_rows; ++i)
+            if (rows[i] >= offsets[e] && rows[i] < offsets[e + 1]) used = 1;
+        if (!used) continue;
+        if (fmt == 0)
+            orc_dequant_nf4(w + e * N * (K / 2), (const float *)scales + e * N * (K / 64), N, K, wd);
+        else
+            orc_dequant_mxfp4(w + e * N * (K / 2), (const uint8_t *)scales + e * N * (K / 32), N, K, wd);
+        for (int64_t i = 0; i < n_rows; ++i) {
+            if (!(rows[i] >= offsets[e] && rows[i] < offsets[e + 1])) continue;
+            const uint16_t *grow = dy + rows[i] * N;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+            for (int64_t kk = 0; kk < K; ++kk) {
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) acc += (double)bf16_to_float(grow[n]) * (double)wd[n * K + kk];
+                dx[i * K + kk] = acc;
+            }
+        }
+    }
+    free(wd);
+}
+
+void orc_grouped_dgrad_nf4(const uint16_t *dy, const uint8_t *w, const float *absmax, const int32_t *offsets,
+                           int64_t E, int64_t N, int64_t K, const int64_t *rows, int64_t n_rows, double *dx)
+{
+    grouped_dgrad(0, dy, w, absmax, offsets, E, N, K, rows, n_rows, dx);
+}
+
+void orc_grouped_dgrad_mxfp4(const uint16_t *dy, const uint8_t *w, const uint8_t *scales, const int32_t *offsets,
+                             int64_t E, int64_t N, int64_t K, const int64_t *rows, int64_t n_rows, double *dx)
+{
+    grouped_dgrad(1, dy, w, scales, offsets, E, N, K, rows, n_rows, dx);
 }

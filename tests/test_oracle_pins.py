@@ -458,3 +458,56 @@ def test_router_ranks_nan_scores_last():
     logits = np.array([[np.nan, -1e30, 2.0, np.nan]], np.float32)
     ids, _ = oracle.router_topk(logits, 4)
     assert list(ids[0]) == [2, 1, 0, 3]
+
+
+# ------------------------------------------------------------------ dgrad
+
+
+@pytest.mark.parametrize("fmt", ["nf4", "mxfp4"])
+def test_dgrad_single_expert_is_numpy_matmul(fmt):
+    """E = 1: dX = dY @ dequant(W) (numpy matmul in fp64 on the dequantised stack)."""
+    g = inputs.rng(70)
+    N, K, M = 48, 128, 7
+    if fmt == "nf4":
+        w, s = oracle.quant_nf4(inputs.normal_weights(g, (1, N, K)))
+        wd = oracle.dequant_nf4(w[0], s[0])
+    else:
+        w, s = inputs.mxfp4_random(g, 1, N, K)
+        wd = oracle.dequant_mxfp4(w[0], s[0])
+    dy = inputs.bf16_normal(g, (M, N))
+    dx = oracle.grouped_dgrad(fmt, dy, w, s, np.array([0, M], np.int32))
+    ref = _af(dy) @ wd.astype(np.float64)
+    np.testing.assert_allclose(dx, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_dgrad_closed_form_column_sums_mxfp4():
+    """All codes 1.0, scale 127 + e for expert e: dX[r, k] = 2^e * sum_n dY[r, n]."""
+    g = inputs.rng(71)
+    E, N, K = 3, 40, 64
+    counts = [2, 0, 3]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    M = int(offsets[-1])
+    dy = inputs.bf16_normal(g, (M, N))
+    w = np.full((E, N, K // 2), 0x22, np.uint8)
+    s = np.stack([np.full((N, K // 32), 127 + e, np.uint8) for e in range(E)])
+    dx = oracle.grouped_dgrad("mxfp4", dy, w, s, offsets)
+    for e in range(E):
+        for r in range(offsets[e], offsets[e + 1]):
+            assert np.all(dx[r] == (2.0 ** e) * math.fsum(_af(dy[r])))
+
+
+def test_dgrad_is_the_transpose_of_the_forward_gemm():
+    """<dY, X W^T> = <dY W, X>: the forward GEMM and dgrad are adjoint on the same stack."""
+    g = inputs.rng(72)
+    E, N, K = 2, 24, 128
+    counts = [3, 4]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    M = int(offsets[-1])
+    w, s = oracle.quant_nf4(inputs.normal_weights(g, (E, N, K)))
+    x = inputs.bf16_normal(g, (M, K))
+    dy = inputs.bf16_normal(g, (M, N))
+    y = oracle.grouped_gemm_nf4(x, w, s, offsets)
+    dx = oracle.grouped_dgrad("nf4", dy, w, s, offsets)
+    lhs = math.fsum((_af(dy) * y).ravel())
+    rhs = math.fsum((dx * _af(x)).ravel())
+    assert abs(lhs - rhs) <= 1e-9 * (abs(lhs) + 1.0)
