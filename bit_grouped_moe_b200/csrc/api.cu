@@ -238,6 +238,27 @@ gnf4_status grouped_gemv(int fmt, bool swiglu, const void* a, const uint8_t* w, 
   return GNF4_OK;
 }
 
+// dY [M, N] bf16 and the [E, N, K/2] stack -> dX [M, K] bf16.
+gnf4_status grouped_dgrad(int fmt, const void* dy, const uint8_t* w, const void* scales, const int32_t* offsets,
+                          const int32_t* counts, int E, int N, int K, int M, void* dx, void* stream) {
+  GNF4_TRY(check_grouped(fmt, dy, w, scales, offsets, counts, E, N, K, M, dx));
+  if (M == 0) return GNF4_OK;
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  CUtensorMap tm_y, tm_w;
+  GNF4_TRY(encode_act_map(&tm_y, dy, M, N, dgrad_tc_rows_per_unit()));
+  GNF4_TRY(encode_weight_map(&tm_w, w, E, N, K, dgrad_tc_k_per_unit() / 2, dgrad_tc_n_per_stage()));
+  GroupedArgs p{static_cast<const __nv_bfloat16*>(dy), w, scales, offsets, counts,
+                static_cast<__nv_bfloat16*>(dx), d->err, E, N, K, M};
+  const long long rpu = dgrad_tc_rows_per_unit(), kpu = dgrad_tc_k_per_unit();
+  const long long units = ((M + rpu - 1) / rpu + (E < M ? E : M)) * ((K + kpu - 1) / kpu);
+  if (units >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d, K=%d give too many work units", M, K);
+  const int grid = (int)(units < d->num_sms ? units : d->num_sms);
+  cudaError_t e = launch_dgrad_tc(fmt, tm_y, tm_w, p, grid, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "grouped dgrad launch");
+  return GNF4_OK;
+}
+
 // The fused gate_up + SwiGLU calls take I (the output width); the stack has 2I rows.
 gnf4_status check_swiglu_width(int I) {
   if (I < 64 || I % 64 != 0 || I > (1 << 29))
@@ -418,6 +439,16 @@ gnf4_status gnf4_dequant_mxfp4_f32(const uint8_t* w, const uint8_t* scales, int6
 }  // extern "C"
 
 extern "C" {
+
+gnf4_status gnf4_grouped_dgrad_nf4(const void* dy, const uint8_t* w, const float* absmax, const int32_t* offsets,
+                                   const int32_t* counts, int E, int N, int K, int M, void* dx, void* stream) {
+  return grouped_dgrad(0, dy, w, absmax, offsets, counts, E, N, K, M, dx, stream);
+}
+
+gnf4_status gnf4_grouped_dgrad_mxfp4(const void* dy, const uint8_t* w, const uint8_t* scales, const int32_t* offsets,
+                                     const int32_t* counts, int E, int N, int K, int M, void* dx, void* stream) {
+  return grouped_dgrad(1, dy, w, scales, offsets, counts, E, N, K, M, dx, stream);
+}
 
 gnf4_status gnf4_grouped_gemm_nf4_swiglu(const void* a, const uint8_t* w_gate_up, const float* absmax,
                                          const int32_t* offsets, const int32_t* counts, int E, int I, int K, int M,

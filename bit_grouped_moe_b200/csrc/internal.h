@@ -60,6 +60,14 @@ int gemv_swiglu_cols_per_block();
 // CTAs for a GEMV launch over `units` (expert, 64-row) units.
 int gemv_grid(long long units, int num_sms);
 
+// dgrad.cu: p.w is the [E, N, K/2] stack, p.a = dY [M, N], p.y = dX [M, K]
+cudaError_t launch_dgrad_tc(int fmt, const CUtensorMap& tm_y, const CUtensorMap& tm_w, const GroupedArgs& p,
+                            int grid, cudaStream_t stream);
+size_t dgrad_tc_smem_bytes();
+int dgrad_tc_rows_per_unit();
+int dgrad_tc_k_per_unit();
+int dgrad_tc_n_per_stage();
+
 // route.cu
 size_t route_workspace_bytes(int T, int k, int E);
 cudaError_t launch_route(const int32_t* topk_ids, const __nv_bfloat16* x, int T, int k, int E, int K,

@@ -173,7 +173,6 @@ __global__ void route_gather_kernel(const uint4* x, int K8, int k, const int32_t
 // Top-k of score = logit + bias (fp32) per token and the softmax of the
 // selected raw logits (grouped-nf4-gemm index.json, problems_solved[5]:
 // router softmax and top-k among the decode tail folded into one launch).
-constexpr int kMaxRouterK = 32;
 
 // Selection order: NaN scores after every number, larger scores first, ties
 // to the lower expert index; an index < 0 is "no candidate".

@@ -44,7 +44,7 @@ _lib.gnf4_route_permute_static.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _
 _lib.gnf4_route_topk_permute.argtypes = [_P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
 _GROUPED = ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_gemv_nf4", "gnf4_grouped_gemv_mxfp4",
             "gnf4_grouped_gemm_nf4_swiglu", "gnf4_grouped_gemm_mxfp4_swiglu", "gnf4_grouped_gemv_nf4_swiglu",
-            "gnf4_grouped_gemv_mxfp4_swiglu")
+            "gnf4_grouped_gemv_mxfp4_swiglu", "gnf4_grouped_dgrad_nf4", "gnf4_grouped_dgrad_mxfp4")
 for _name in _GROUPED:
     getattr(_lib, _name).argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
@@ -165,6 +165,15 @@ def grouped_gemv_nf4(a, w, absmax, y, offsets=None, counts=None, stream=None):
 
 def grouped_gemv_mxfp4(a, w, scales, y, offsets=None, counts=None, stream=None):
     _grouped(_lib.gnf4_grouped_gemv_mxfp4, a, w, scales, y, offsets, counts, stream)
+
+
+def grouped_dgrad_nf4(dy, w, absmax, dx, offsets=None, counts=None, stream=None):
+    """dX [M, K] = dY [M, N] . W_e for each row's expert (the forward stack [E, N, K/2])."""
+    _grouped(_lib.gnf4_grouped_dgrad_nf4, dy, w, absmax, dx, offsets, counts, stream)
+
+
+def grouped_dgrad_mxfp4(dy, w, scales, dx, offsets=None, counts=None, stream=None):
+    _grouped(_lib.gnf4_grouped_dgrad_mxfp4, dy, w, scales, dx, offsets, counts, stream)
 
 
 def _grouped_swiglu(fn, a, w_gate_up, scales, h, offsets=None, counts=None, stream=None):

@@ -212,6 +212,23 @@ gnf4_status gnf4_grouped_gemv_mxfp4(const void *a, const uint8_t *w, const uint8
                                     const int32_t *counts, int E, int N, int K, int M, void *y, void *stream);
 
 /* ------------------------------------------------------------------ */
+/* Data gradient of the grouped projection                             */
+/* ------------------------------------------------------------------ */
+
+/* dX = dY . W on the same packed stacks the forward call reads
+ * (grouped-nf4-gemm index.json, system_manifest.owns: "grouped packed GEMM
+ * (NF4 and native MXFP4) and its dgrad"; entrypoints:
+ * nf4_grouped:dgrad_4bit_grouped).  For every sorted row r of expert e:
+ *     dx[r, k] = sum_n dy[r, n] * dq(W_e)[n, k],
+ * fp32 accumulation, bf16 output [M, K].  dy is bf16 [M, N] (the gradient of
+ * the forward output), w / scales / offsets / counts exactly as the grouped
+ * GEMM calls (same shape rules).  Rows past offsets[E] are not written. */
+gnf4_status gnf4_grouped_dgrad_nf4(const void *dy, const uint8_t *w, const float *absmax, const int32_t *offsets,
+                                   const int32_t *counts, int E, int N, int K, int M, void *dx, void *stream);
+gnf4_status gnf4_grouped_dgrad_mxfp4(const void *dy, const uint8_t *w, const uint8_t *scales, const int32_t *offsets,
+                                     const int32_t *counts, int E, int N, int K, int M, void *dx, void *stream);
+
+/* ------------------------------------------------------------------ */
 /* Fused gate_up projection + SwiGLU                                   */
 /* ------------------------------------------------------------------ */
 
