@@ -145,7 +145,7 @@ class Workload:
     """Device-resident inputs of one workload: rotating weight copies larger
     than L2, a set of token batches, and the step's output buffers."""
 
-    def __init__(self, name, device, seed, build_host_copy, swiglu=False):
+    def __init__(self, name, device, seed, build_host_copy, swiglu=False, dgrad=False):
         import torch
 
         from bit_grouped_moe_b200 import gnf4
@@ -197,6 +197,17 @@ class Workload:
         self.fn = {("nf4", True): f.grouped_gemv_nf4, ("nf4", False): f.grouped_gemm_nf4,
                    ("mxfp4", True): f.grouped_gemv_mxfp4, ("mxfp4", False): f.grouped_gemm_mxfp4}[
             (wl.fmt, self.decode)]
+        # optional backward step: the data gradients of both projections
+        self.dgrad = dgrad
+        if dgrad:
+            self.decode = False  # the dgrad call has no decode variant
+            self.dy1 = torch.from_numpy(inputs.bf16_normal(rng, (M, self.p1.N)).view(np.int16)).view(
+                torch.bfloat16).to(device)
+            self.dy2 = torch.from_numpy(inputs.bf16_normal(rng, (M, self.p2.N)).view(np.int16)).view(
+                torch.bfloat16).to(device)
+            self.dx1 = torch.empty(M, self.p1.K, dtype=torch.bfloat16, device=device)
+            self.dh = torch.empty(M, self.p2.K, dtype=torch.bfloat16, device=device)
+            self.dfn = f.grouped_dgrad_nf4 if wl.fmt == "nf4" else f.grouped_dgrad_mxfp4
         # optional fused gate_up + SwiGLU first projection: h [M, N1/2] feeds the second
         self.swiglu = swiglu
         if swiglu:
@@ -252,6 +263,14 @@ class Workload:
         ids, wts, x = self.d_batches[i % N_BATCHES]
         (w1, s1), (w2, s2) = self.stacks[i % N_WEIGHT_COPIES]
         g.route_permute(ids, x, self.E, self.off, self.s2f, self.f2s, self.xs, self.ws)
+        if self.dgrad:  # backward through both projections: dH = dY2 . W2, dX = dY1 . W1
+            self.dfn(self.dy2, w2, s2, self.dh, offsets=self.off)
+            if ev is not None:
+                ev[0].record()
+            self.dfn(self.dy1, w1, s1, self.dx1, offsets=self.off)
+            if ev is not None:
+                ev[1].record()
+            return
         if ev is not None:
             ev[0].record()
         self.project(w1, s1, w2, s2, ev)
@@ -269,7 +288,7 @@ class Workload:
     def launches_per_step(self):
         # route (one launch for at most 256 pairs, else hist + scan + scatter + gather) + 2 projections + combine
         route = 1 if 0 < self.M <= 256 else 4
-        return route + 2 + 1
+        return route + 2 + (0 if self.dgrad else 1)
 
 
 # ------------------------------------------------------------------ distributed
@@ -373,6 +392,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--impl", default="libgnf4", choices=["libgnf4", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dgrad", action="store_true",
+                    help="time the backward step instead: route + the dgrad of both projections (TFLOP/s)")
     ap.add_argument("--graph", action="store_true",
                     help=f"decode: also time the steps replayed from one CUDA graph of {20} steps")
     ap.add_argument("--swiglu", action="store_true",
@@ -383,7 +404,7 @@ def main():
     globals()["N_WEIGHT_COPIES"] = max(1, args.weight_copies)
 
     wl_def = inputs.WORKLOADS[args.workload]
-    decode = wl_def.T <= 8
+    decode = wl_def.T <= 8 and not args.dgrad
     steps = args.steps if args.steps is not None else (20000 if decode else 200)
     warmup = args.warmup if args.warmup is not None else (100 if decode else 10)
     warmup = max(warmup, 3)
@@ -421,7 +442,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     dev = f"cuda:{local}"
     torch.cuda.set_device(local)
     wl = Workload(args.workload, dev, seed=1234 + rank, build_host_copy=(rank == 0 and world == 1),
-                  swiglu=args.swiglu)
+                  swiglu=args.swiglu, dgrad=args.dgrad)
+    decode = wl.decode
     wl.h_host = wl.h.cpu().view(torch.int16).numpy().view(np.uint16)
     stream = torch.cuda.current_stream()
 
@@ -463,7 +485,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     for (ids, wts, x) in wl.batches:
         host_in.append((torch.from_numpy(ids).pin_memory(), torch.from_numpy(wts).pin_memory(),
                         torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()))
-    host_out = torch.empty(wl.T, wl.p2.N, dtype=torch.bfloat16).pin_memory()
+    out_dev = wl.dx1 if wl.dgrad else wl.out
+    host_out = torch.empty(tuple(out_dev.shape), dtype=torch.bfloat16).pin_memory()
     d_ids = torch.empty_like(wl.d_batches[0][0])
     d_w = torch.empty_like(wl.d_batches[0][1])
     d_x = torch.empty_like(wl.d_batches[0][2])
@@ -477,9 +500,13 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         (w1, s1), (w2, s2) = wl.stacks[i % N_WEIGHT_COPIES]
         g = wl.g
         g.route_permute(d_ids, d_x, wl.E, wl.off, wl.s2f, wl.f2s, wl.xs, wl.ws)
-        wl.project(w1, s1, w2, s2)
-        g.combine(wl.y2, wl.f2s, d_w, wl.out)
-        host_out.copy_(wl.out, non_blocking=True)
+        if wl.dgrad:
+            wl.dfn(wl.dy2, w2, s2, wl.dh, offsets=wl.off)
+            wl.dfn(wl.dy1, w1, s1, wl.dx1, offsets=wl.off)
+        else:
+            wl.project(w1, s1, w2, s2)
+            g.combine(wl.y2, wl.f2s, d_w, wl.out)
+        host_out.copy_(out_dev, non_blocking=True)
 
     for i in range(warmup):
         e2e_step(i)
@@ -536,8 +563,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         e2e_val = world * e2e_steps * wl.step_flops() / (e2e_ms / 1e3) / 1e12
 
     peaks, peak_src = load_peaks()
-    kern_file = "gemv.cu" if decode else "gemm_tc.cu"
-    kern_key = f"{'gemv' if decode else 'gemm_tc'}_{wl.wl.fmt}{'_swiglu' if wl.swiglu else ''}:{args.workload}:{wl.p1.name}"
+    kern_file = "gemv.cu" if decode else ("dgrad.cu" if wl.dgrad else "gemm_tc.cu")
+    kern_key = f"{'gemv' if decode else ('dgrad_tc' if wl.dgrad else 'gemm_tc')}_{wl.wl.fmt}{'_swiglu' if wl.swiglu else ''}:{args.workload}:{wl.p1.name}"
     sha = kernel_source_sha([kern_file, "common.cuh"])
     if decode:
         mean_hit = sum(wl.hit[i % N_BATCHES] for i in sampled) / len(sampled)
@@ -554,7 +581,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         pk = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk, "unit": "TFLOP/s",
                 "frac": round(achieved / pk, 4), "traffic": committed_traffic(kern_key, sha),
-                "kernel": f"gemm_tc_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})",
+                "kernel": (f"dgrad_tc_kernel<{wl.wl.fmt}> (dX of {wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.dgrad else
+                           f"gemm_tc_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})"),
                 "algorithmic_flops_per_launch": int(flops), "avg_launch_us": round(dom_ms * 1e3, 3),
                 "peak_source": f"bf16_tflops_sustained of {peak_src} (kind::f16 MMA on decoded bf16 tiles)"}
 
@@ -571,7 +599,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
             "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": steps,
             "warmup": warmup, "ms_per_step": round(ms / steps, 6), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(_config(wl.wl, world), **({"first_projection": "fused gate_up + SwiGLU"} if wl.swiglu else {})),
+            "config": dict(_config(wl.wl, world), **({"first_projection": "fused gate_up + SwiGLU"} if wl.swiglu else {}),
+                           **({"step": "backward: route + dgrad of both projections"} if wl.dgrad else {})),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
