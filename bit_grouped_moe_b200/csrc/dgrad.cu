@@ -13,10 +13,11 @@
 //    B operand), so both operands use the plain K-major descriptor.
 // D[r, k] accumulates in TMEM (lane = row r, column = k).  Work unit = (expert
 // e, chunk of <= 128 of its rows, 128-wide k tile); a persistent grid strides
-// over the units.  Pipeline: packed weights and dY tiles in a 4-deep TMA ring
-// issued three stages ahead, block scales staged in shared memory one stage
-// ahead, the decoded W^T double-buffered, so the copies and the MMAs of
-// earlier stages overlap the decode of the current one.
+// over the units.  Warp roles: 8 decode warps, a TMA producer, an MMA issuer
+// and 4 epilogue warps.  Packed weights and dY tiles stream through a 4-deep
+// TMA ring, block scales are staged in shared memory by the decode warps two
+// stages ahead, the decoded W^T is double-buffered and the accumulator too,
+// so copies, MMAs, decode and the epilogue of the previous unit overlap.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -26,7 +27,10 @@
 namespace gnf4 {
 namespace {
 
-constexpr int kThreads = 256;                  // 8 warps: all decode, all read the accumulator
+constexpr int kDecWarps = 8;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kProdWarp = 8, kMmaWarp = 9, kEpiWarp0 = 10;
+constexpr int kThreads = (kEpiWarp0 + 4) * 32;  // 448
 constexpr int kRing = 4;                       // dY / packed-weight stages in flight
 constexpr int kBR = 128;                   // rows per unit (MMA M)
 constexpr int kBKt = 128;                  // k per unit (MMA N)
@@ -34,7 +38,7 @@ constexpr int kBN = 64;                    // n per stage (four k-steps of 16)
 constexpr int kYBytes = kBR * kBN * 2;     // 16 KB
 constexpr int kTBytes = kBKt * kBN * 2;    // 16 KB
 constexpr int kWBytes = kBN * kBKt / 2;    // 4 KB
-constexpr int kTmemCols = kBKt;
+constexpr int kTmemCols = 2 * kBKt;  // two accumulators
 
 struct DSmem {
   uint8_t y[kRing][kYBytes];  // dY tiles (1024-aligned for the 128-byte swizzle)
@@ -45,7 +49,7 @@ struct DSmem {
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
-  uint64_t full[kRing], mdone[kRing], accf, drain;
+  uint64_t full[kRing], mdone[kRing], decoded[2], accf[2], acce[2], drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -119,14 +123,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.full[i], 1);
       mbar_init(&s.mdone[i], 1);
     }
-    mbar_init(&s.accf, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.decoded[i], kDecThreads);
+      mbar_init(&s.accf[i], 1);
+      mbar_init(&s.acce[i], 128);
+    }
     mbar_init(&s.drain, 1);
     s.abort = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_y);
     prefetch_tmap(&tm_w);
   }
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&s.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -134,10 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  const uint32_t lut = smem_u32(s.lut);
-  const uint32_t lane4 = (uint32_t)lane * 4u;
-  const uint32_t idesc = idesc_bf16_m128((uint32_t)kBKt);
-  const int nsc = FMT == 0 ? K / 64 : K / 32;    // scales per weight row
+  const int nsc = FMT == 0 ? K / 64 : K / 32;        // scales per weight row
   const int spk = FMT == 0 ? kBKt / 64 : kBKt / 32;  // scale blocks of a row in one k tile
 
   // The CTA's stage stream: stage g = (unit u, n block sb), units strided by the grid.
@@ -151,161 +156,184 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     return q;
   };
-  // thread 0: the tiles of stage gi (at position q) into ring slot gi % kRing
-  int issued = 0;
-  auto issue = [&](Pos q, int gi) {
-    const DUnit x = dunit_of(s, p.E, nkt, q.u);
-    const int b = gi % kRing;
-    mbar_arrive_expect_tx(&s.full[b], kYBytes + kWBytes);
-    tma_load_2d(s.y[b], &tm_y, &s.full[b], q.sb * kBN, x.row0);
-    tma_load_3d(s.w[b], &tm_w, &s.full[b], x.kt * (kBKt / 2), q.sb * kBN, x.e);
-    ++issued;
-  };
-  // one raw block scale of stage position q per thread (rows past N: none)
-  auto scale_raw = [&](Pos q, bool& valid) -> uint32_t {
-    valid = false;
-    if (q.u >= U || tid >= kBN * spk) return 0u;
-    const DUnit x = dunit_of(s, p.E, nkt, q.u);
-    const int rr = tid / spk, bb = tid - rr * spk;
-    const int n = q.sb * kBN + rr;
-    if (n >= N) return 0u;
-    const int blk = min(x.kt * spk + bb, nsc - 1);  // past K: any valid scale, never stored
-    const size_t idx = ((size_t)x.e * N + (size_t)n) * (size_t)nsc + (size_t)blk;
-    valid = true;
-    return FMT == 0 ? __float_as_uint(__ldg(reinterpret_cast<const float*>(p.scales) + idx))
-                    : (uint32_t)__ldg(reinterpret_cast<const uint8_t*>(p.scales) + idx);
-  };
-  // bf16x2 scale pair (0 for rows past N) into sc[buf]
-  auto scale_store = [&](int buf, uint32_t raw, bool valid) {
-    if (tid >= kBN * spk) return;
-    const int rr = tid / spk, bb = tid - rr * spk;
-    s.sc[buf][rr][bb] = !valid ? 0u : (FMT == 0 ? f32_to_bf16x2_rn(__uint_as_float(raw)) : e8m0_to_bf16x2(raw));
-  };
 
-  Pos cur{(int)blockIdx.x, 0};
-  Pos pf = cur;  // next stage to issue (thread 0)
-  if (tid == 0)
-    for (int i = 0; i < kRing - 1 && pf.u < U; ++i) {
-      issue(pf, i);
-      pf = next(pf);
+  if (warp == kProdWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int g = 0;
+      for (Pos q{(int)blockIdx.x, 0}; q.u < U && !*abort; q = next(q), ++g) {
+        const int b = g % kRing;
+        if (g >= kRing && !mbar_wait(&s.mdone[b], (uint32_t)((g - kRing) / kRing) & 1u, err, abort)) break;
+        const DUnit x = dunit_of(s, p.E, nkt, q.u);
+        mbar_arrive_expect_tx(&s.full[b], kYBytes + kWBytes);
+        tma_load_2d(s.y[b], &tm_y, &s.full[b], q.sb * kBN, x.row0);
+        tma_load_3d(s.w[b], &tm_w, &s.full[b], x.kt * (kBKt / 2), q.sb * kBN, x.e);
+      }
+      if (*abort)  // let the last copies land before shared memory goes away
+        for (int i = max(0, g - kRing); i < g; ++i) mbar_drain(&s.full[i % kRing], (uint32_t)(i / kRing) & 1u);
     }
-  {
-    bool v;
-    const uint32_t raw = scale_raw(cur, v);
-    scale_store(0, raw, v);
-  }
-  __syncthreads();
-  // Block scales travel two stages ahead: loaded into a register during stage
-  // g for stage g+2, stored into sc at the end of stage g+1.
-  Pos sp = next(cur);
-  bool sv_a;
-  uint32_t sraw_a = scale_raw(sp, sv_a);  // stage 1
-  sp = next(sp);                          // stage 2
-
-  int g = 0, uc = 0;  // stages consumed, units finished by this CTA
-  bool ok = true;
-  for (int u = blockIdx.x; u < U; u += gridDim.x, ++uc) {
-    const DUnit x = dunit_of(s, p.E, nkt, u);
-    const int k0 = x.kt * kBKt;
-    for (int sb = 0; sb < ns; ++sb, ++g) {
-      const int b = g % kRing, tb = g & 1;
-      // producer: stage g + kRing - 1 into slot (g - 1) % kRing once the MMAs of stage g-1 are done with it
-      if (tid == 0 && !*abort && pf.u < U) {
-        if (g >= 1) ok = mbar_wait(&s.mdone[(g - 1) % kRing], (uint32_t)((g - 1) / kRing) & 1u, err, abort);
-        if (ok) issue(pf, g + kRing - 1);
-        pf = next(pf);
-      }
-      // scales of stage g+2: loaded now, staged at the end of stage g+1
-      bool sv_b;
-      const uint32_t sraw_b = scale_raw(sp, sv_b);
-      sp = next(sp);
-      // this stage's tiles have landed, and the MMAs of stage g-2 no longer read t[tb]
-      if (!*abort) mbar_wait(&s.full[b], (uint32_t)(g / kRing) & 1u, err, abort);
-      if (g >= 2 && !*abort) mbar_wait(&s.mdone[(g - 2) % kRing], (uint32_t)((g - 2) / kRing) & 1u, err, abort);
-
-      // decode: item (kp, nb) = k pair kp (k = 2kp, 2kp+1 of the tile), n rows nb*8 .. nb*8+7
-      const uint32_t wbase = smem_u32(s.w[b]);
-      const uint32_t tbase = smem_u32(s.t[tb]);
-#pragma unroll
-      for (int j = 0; j < (kBKt / 2) * (kBN / 8) / kThreads; ++j) {
-        const int item = tid + kThreads * j;
-        const int kp = item & 63, nb = item >> 6;
-        const int bb = FMT == 0 ? (2 * kp) / 64 : (2 * kp) / 32;
-        uint32_t pr[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t byte = lds_u8(wbase + (uint32_t)((nb * 8 + i) * (kBKt / 2) + kp));
-          pr[i] = bf16x2_mul(lut256_get(lut, byte, lane4, 0u), s.sc[tb][nb * 8 + i][bb]);
-        }
-        // row 2kp of W^T takes the low halves (even k), row 2kp+1 the high halves
-        sts_u128(tbase + sw128_chunk(2 * kp, nb), prmt_b32(pr[0], pr[1], 0x5410u), prmt_b32(pr[2], pr[3], 0x5410u),
-                 prmt_b32(pr[4], pr[5], 0x5410u), prmt_b32(pr[6], pr[7], 0x5410u));
-        sts_u128(tbase + sw128_chunk(2 * kp + 1, nb), prmt_b32(pr[0], pr[1], 0x7632u),
-                 prmt_b32(pr[2], pr[3], 0x7632u), prmt_b32(pr[4], pr[5], 0x7632u), prmt_b32(pr[6], pr[7], 0x7632u));
-      }
-      scale_store(tb ^ 1, sraw_a, sv_a);  // stage g+1
-      sraw_a = sraw_b;
-      sv_a = sv_b;
-      fence_proxy_async_smem();  // generic-proxy writes of t[tb] before the MMA reads them
-      __syncthreads();
-      if (tid == 0 && !*abort) {
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_m128((uint32_t)kBKt);
+      int g = 0, uc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
+        const int ab = uc & 1;
+        if (uc >= 2 && !(ok = mbar_wait(&s.acce[ab], (uint32_t)((uc >> 1) - 1) & 1u, err, abort))) break;
         tc_fence_after();
-        const uint32_t ya = smem_u32(s.y[b]), ta = smem_u32(s.t[tb]);
+        const uint32_t d_tmem = tmem + (uint32_t)(ab * kBKt);
+        for (int sb = 0; sb < ns; ++sb, ++g) {
+          const int b = g % kRing, tb = g & 1;
+          if (!(ok = mbar_wait(&s.full[b], (uint32_t)(g / kRing) & 1u, err, abort))) break;
+          if (!(ok = mbar_wait(&s.decoded[tb], (uint32_t)(g >> 1) & 1u, err, abort))) break;
+          tc_fence_after();
+          const uint32_t ya = smem_u32(s.y[b]), ta = smem_u32(s.t[tb]);
 #pragma unroll
-        for (int q = 0; q < kBN / 16; ++q)
-          tc_mma_ss(tmem, sdesc_k_sw128(ya + q * 32), sdesc_k_sw128(ta + q * 32), idesc, (sb | q) != 0);
-        tc_commit(&s.mdone[b]);
+          for (int q = 0; q < kBN / 16; ++q)
+            tc_mma_ss(d_tmem, sdesc_k_sw128(ya + q * 32), sdesc_k_sw128(ta + q * 32), idesc, (sb | q) != 0);
+          tc_commit(&s.mdone[b]);
+        }
+        if (!ok) break;
+        tc_commit(&s.accf[ab]);
+      }
+      if (!ok) {  // let every issued MMA retire before TMEM is released
+        tc_commit(&s.drain);
+        mbar_drain(&s.drain, 0);
       }
     }
-    // epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (rows), columns 64 (w / 4) .. +63
-    if (tid == 0 && !*abort) tc_commit(&s.accf);
-    if (!*abort) mbar_wait(&s.accf, (uint32_t)uc & 1u, err, abort);
-    tc_fence_after();
-    const int r = (warp & 3) * 32 + lane;
-    const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    for (int c = 2 * (warp >> 2); c < 2 * (warp >> 2) + 2; ++c) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(t_lane + (uint32_t)(c * 32), v);
-      tmem_wait_ld();
-      const int kc = k0 + c * 32;
-      if (r < x.rows && kc < K && !*abort) {
-        __nv_bfloat16* dst = p.y + (size_t)(x.row0 + r) * K + kc;
-        if (kc + 32 <= K) {
+  } else if (warp < kDecWarps) {
+    // ------------------------------------------------------------ decode
+    const uint32_t lut = smem_u32(s.lut);
+    const uint32_t lane4 = (uint32_t)lane * 4u;
+    // one raw block scale of the stage at position q per thread (rows past N: none)
+    auto scale_raw = [&](Pos q, bool& valid) -> uint32_t {
+      valid = false;
+      if (q.u >= U || tid >= kBN * spk) return 0u;
+      const DUnit x = dunit_of(s, p.E, nkt, q.u);
+      const int rr = tid / spk, bb = tid - rr * spk;
+      const int n = q.sb * kBN + rr;
+      if (n >= N) return 0u;
+      const int blk = min(x.kt * spk + bb, nsc - 1);  // past K: any valid scale, never stored
+      const size_t idx = ((size_t)x.e * N + (size_t)n) * (size_t)nsc + (size_t)blk;
+      valid = true;
+      return FMT == 0 ? __float_as_uint(__ldg(reinterpret_cast<const float*>(p.scales) + idx))
+                      : (uint32_t)__ldg(reinterpret_cast<const uint8_t*>(p.scales) + idx);
+    };
+    // bf16x2 scale pair (0 for rows past N) into sc[buf]
+    auto scale_store = [&](int buf, uint32_t raw, bool valid) {
+      if (tid >= kBN * spk) return;
+      const int rr = tid / spk, bb = tid - rr * spk;
+      s.sc[buf][rr][bb] = !valid ? 0u : (FMT == 0 ? f32_to_bf16x2_rn(__uint_as_float(raw)) : e8m0_to_bf16x2(raw));
+    };
+    auto dec_barrier = [&]() { asm volatile("bar.sync 1, %0;" ::"r"(kDecThreads) : "memory"); };
+
+    Pos sp{(int)blockIdx.x, 0};
+    {
+      bool v;
+      const uint32_t raw = scale_raw(sp, v);
+      scale_store(0, raw, v);
+    }
+    // block scales travel two stages ahead: loaded during stage g for stage g+2,
+    // stored at the end of stage g+1
+    sp = next(sp);
+    bool sv_a;
+    uint32_t sraw_a = scale_raw(sp, sv_a);
+    sp = next(sp);
+    dec_barrier();
+    // After an abort the loop still runs to its end (no waits, garbage
+    // results), so every decode warp reaches every named barrier.
+    int g = 0;
+    for (int u = blockIdx.x; u < U; u += gridDim.x) {
+      for (int sb = 0; sb < ns; ++sb, ++g) {
+        const int b = g % kRing, tb = g & 1;
+        bool sv_b;
+        const uint32_t sraw_b = scale_raw(sp, sv_b);
+        sp = next(sp);
+        // this stage's packed weights have landed, and the MMAs of stage g-2 no longer read t[tb]
+        if (!*abort) mbar_wait(&s.full[b], (uint32_t)(g / kRing) & 1u, err, abort);
+        if (g >= 2 && !*abort) mbar_wait(&s.mdone[(g - 2) % kRing], (uint32_t)((g - 2) / kRing) & 1u, err, abort);
+        // item (kp, nb) = k pair kp (k = 2kp, 2kp+1 of the tile), n rows nb*8 .. nb*8+7
+        const uint32_t wbase = smem_u32(s.w[b]);
+        const uint32_t tbase = smem_u32(s.t[tb]);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-            __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-            uint4 o;
-            o.x = *reinterpret_cast<uint32_t*>(&h0);
-            o.y = *reinterpret_cast<uint32_t*>(&h1);
-            o.z = *reinterpret_cast<uint32_t*>(&h2);
-            o.w = *reinterpret_cast<uint32_t*>(&h3);
-            reinterpret_cast<uint4*>(dst)[q] = o;
+        for (int j = 0; j < (kBKt / 2) * (kBN / 8) / kDecThreads; ++j) {
+          const int item = tid + kDecThreads * j;
+          const int kp = item & 63, nb = item >> 6;
+          const int bb = FMT == 0 ? (2 * kp) / 64 : (2 * kp) / 32;
+          uint32_t pr[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t byte = lds_u8(wbase + (uint32_t)((nb * 8 + i) * (kBKt / 2) + kp));
+            pr[i] = bf16x2_mul(lut256_get(lut, byte, lane4, 0u), s.sc[tb][nb * 8 + i][bb]);
           }
-        } else {
-          for (int i = 0; i < 32 && kc + i < K; ++i) dst[i] = __float2bfloat16_rn(__uint_as_float(v[i]));
+          // row 2kp of W^T takes the low halves (even k), row 2kp+1 the high halves
+          sts_u128(tbase + sw128_chunk(2 * kp, nb), prmt_b32(pr[0], pr[1], 0x5410u),
+                   prmt_b32(pr[2], pr[3], 0x5410u), prmt_b32(pr[4], pr[5], 0x5410u),
+                   prmt_b32(pr[6], pr[7], 0x5410u));
+          sts_u128(tbase + sw128_chunk(2 * kp + 1, nb), prmt_b32(pr[0], pr[1], 0x7632u),
+                   prmt_b32(pr[2], pr[3], 0x7632u), prmt_b32(pr[4], pr[5], 0x7632u),
+                   prmt_b32(pr[6], pr[7], 0x7632u));
+        }
+        fence_proxy_async_smem();  // generic-proxy writes of t[tb] before the MMA reads them
+        mbar_arrive(&s.decoded[tb]);
+        scale_store(tb ^ 1, sraw_a, sv_a);  // stage g+1
+        sraw_a = sraw_b;
+        sv_a = sv_b;
+        dec_barrier();  // sc[tb ^ 1] written, sc[tb] no longer read
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // a warp reaches TMEM lanes 32 (warp % 4) .. +31: these rows
+    const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+    const int r = q * 32 + lane;
+    int uc = 0;
+    for (int u = blockIdx.x; u < U; u += gridDim.x, ++uc) {
+      const DUnit x = dunit_of(s, p.E, nkt, u);
+      const int ab = uc & 1;
+      if (!mbar_wait(&s.accf[ab], (uint32_t)(uc >> 1) & 1u, err, abort)) break;
+      tc_fence_after();
+      const int k0 = x.kt * kBKt;
+      for (int c = 0; c < kBKt / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBKt + c * 32), v);
+        tmem_wait_ld();
+        const int kc = k0 + c * 32;
+        if (r < x.rows && kc < K) {
+          __nv_bfloat16* dst = p.y + (size_t)(x.row0 + r) * K + kc;
+          if (kc + 32 <= K) {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[8 * qq + 0]), __uint_as_float(v[8 * qq + 1]));
+              __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[8 * qq + 2]), __uint_as_float(v[8 * qq + 3]));
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[8 * qq + 4]), __uint_as_float(v[8 * qq + 5]));
+              __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[8 * qq + 6]), __uint_as_float(v[8 * qq + 7]));
+              uint4 o;
+              o.x = *reinterpret_cast<uint32_t*>(&h0);
+              o.y = *reinterpret_cast<uint32_t*>(&h1);
+              o.z = *reinterpret_cast<uint32_t*>(&h2);
+              o.w = *reinterpret_cast<uint32_t*>(&h3);
+              reinterpret_cast<uint4*>(dst)[qq] = o;
+            }
+          } else {
+            for (int i = 0; i < 32 && kc + i < K; ++i) dst[i] = __float2bfloat16_rn(__uint_as_float(v[i]));
+          }
         }
       }
+      tc_fence_before();
+      mbar_arrive(&s.acce[ab]);
     }
-    tc_fence_before();
-    __syncthreads();  // the accumulator is read before the next unit's first MMA
   }
-  if (*abort && tid == 0) {
-    // let issued MMAs retire and landing copies complete before the memory goes away
-    tc_commit(&s.drain);
-    mbar_drain(&s.drain, 0);
-    for (int i = max(0, issued - kRing); i < issued; ++i)
-      mbar_drain(&s.full[i % kRing], (uint32_t)(i / kRing) & 1u);
-  }
+
+  // Normal path: the epilogue has read every accumulator, so every MMA and
+  // TMEM access has completed.
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  (void)ok;
 }
 
 }  // namespace
