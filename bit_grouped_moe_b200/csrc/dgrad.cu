@@ -160,11 +160,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProdWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int g = 0;
+      int g = 0, xu = -1;
+      DUnit x{};
       for (Pos q{(int)blockIdx.x, 0}; q.u < U && !*abort; q = next(q), ++g) {
         const int b = g % kRing;
         if (g >= kRing && !mbar_wait(&s.mdone[b], (uint32_t)((g - kRing) / kRing) & 1u, err, abort)) break;
-        const DUnit x = dunit_of(s, p.E, nkt, q.u);
+        if (q.u != xu) {
+          x = dunit_of(s, p.E, nkt, q.u);
+          xu = q.u;
+        }
         mbar_arrive_expect_tx(&s.full[b], kYBytes + kWBytes);
         tma_load_2d(s.y[b], &tm_y, &s.full[b], q.sb * kBN, x.row0);
         tma_load_3d(s.w[b], &tm_w, &s.full[b], x.kt * (kBKt / 2), q.sb * kBN, x.e);
@@ -206,11 +210,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ decode
     const uint32_t lut = smem_u32(s.lut);
     const uint32_t lane4 = (uint32_t)lane * 4u;
-    // one raw block scale of the stage at position q per thread (rows past N: none)
+    // one raw block scale of the stage at position q per thread (rows past N:
+    // none); the unit's view is recomputed only when q moves to another unit
+    int xs_u = -1;
+    DUnit xs{};
     auto scale_raw = [&](Pos q, bool& valid) -> uint32_t {
       valid = false;
       if (q.u >= U || tid >= kBN * spk) return 0u;
-      const DUnit x = dunit_of(s, p.E, nkt, q.u);
+      if (q.u != xs_u) {
+        xs = dunit_of(s, p.E, nkt, q.u);
+        xs_u = q.u;
+      }
+      const DUnit& x = xs;
       const int rr = tid / spk, bb = tid - rr * spk;
       const int n = q.sb * kBN + rr;
       if (n >= N) return 0u;
