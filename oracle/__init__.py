@@ -60,6 +60,10 @@ def _load():
     lib.orc_router_topk.argtypes = [P, P, I64, I64, I64, P, P]
     lib.orc_grouped_dgrad_nf4.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
     lib.orc_grouped_dgrad_mxfp4.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
+    lib.orc_e4m3_values.argtypes = [P]
+    lib.orc_quant_mxfp8.argtypes = [P, I64, I64, P, P]
+    lib.orc_dequant_mxfp8.argtypes = [P, P, I64, I64, P]
+    lib.orc_grouped_gemm_w4a8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P]
     _lib = lib
     return lib
 
@@ -252,3 +256,51 @@ def grouped_dgrad(fmt: str, dy_bits, w, scales, offsets, rows=None):
     fn = _load().orc_grouped_dgrad_nf4 if fmt == "nf4" else _load().orc_grouped_dgrad_mxfp4
     fn(_p(dy_bits), _p(w), _p(scales), _p(offsets), E, N, K, _p(rows), rows.shape[0], _p(dx))
     return dx
+
+
+def e4m3_values() -> np.ndarray:
+    """fp64 value of every e4m3 code 0..255 (NaN for 0x7F and 0xFF)."""
+    out = np.empty(256, np.float64)
+    _load().orc_e4m3_values(_p(out))
+    return out
+
+
+def quant_mxfp8(x_bits: np.ndarray):
+    """[..., K] bf16 patterns (uint16) -> (codes [..., K] u8 e4m3, scales [..., K/32] u8 e8m0)."""
+    x_bits = _c(x_bits, np.uint16)
+    K = x_bits.shape[-1]
+    if K % 32:
+        raise ValueError("MXFP8 needs K % 32 == 0")
+    rows = x_bits.size // K if K else 0
+    codes = np.empty(x_bits.shape, np.uint8)
+    scales = np.empty(x_bits.shape[:-1] + (K // 32,), np.uint8)
+    _load().orc_quant_mxfp8(_p(x_bits), rows, K, _p(codes), _p(scales))
+    return codes, scales
+
+
+def dequant_mxfp8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint8)
+    K = codes.shape[-1]
+    rows = codes.size // K if K else 0
+    out = np.empty(codes.shape, np.float64)
+    _load().orc_dequant_mxfp8(_p(codes), _p(scales), rows, K, _p(out))
+    return out
+
+
+def grouped_gemm_w4a8(codes, a_scales, w, w_scales, offsets, rows=None):
+    """fp64 Y[rows, N] of the native W4A8 mode: MXFP8 activations x MXFP4 weights."""
+    codes = _c(codes, np.uint8)
+    a_scales = _c(a_scales, np.uint8)
+    w = _c(w, np.uint8)
+    w_scales = _c(w_scales, np.uint8)
+    offsets = _c(offsets, np.int32)
+    E, N, K2 = w.shape
+    K = 2 * K2
+    if rows is None:
+        rows = np.arange(int(offsets[-1]), dtype=np.int64)
+    rows = _c(rows, np.int64)
+    y = np.empty((rows.shape[0], N), np.float64)
+    _load().orc_grouped_gemm_w4a8(_p(codes), _p(a_scales), _p(w), _p(w_scales), _p(offsets), E, N, K, _p(rows),
+                                  rows.shape[0], _p(y))
+    return y

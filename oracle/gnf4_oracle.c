@@ -29,6 +29,12 @@
  *   [DGRAD]    grouped-nf4-gemm index.json, system_manifest.owns ("grouped packed
  *              GEMM (NF4 and native MXFP4) and its dgrad") and entrypoints
  *              (nf4_grouped:dgrad_4bit_grouped): dX = dY . W on the same stacks.
+ *   [W4A8]     bw24 v0.9.0 release notes, Features ("f8f4 tile piece 1":
+ *              e4m3 activation quantisation; "mixed e4m3xe2m1 mxf8f6f4 probe")
+ *              and Documentation ("prefill arc design": W4A8-FP8, native e2m1
+ *              weights times e4m3 activations in one block-scaled MMA), with
+ *              grouped-nf4-gemm index.json, system_manifest.owns ("native
+ *              MXFP4"); reading C19 for the activation scale rule.
  *   [ARENA]    grouped-nf4-gemm releases, v0.2.5 "arena -> kernel" (expert
  *              stacks [E,N,K//2] blocks + [E,N,K//32] e8m0 scales).
  *   [QLORA]    The NF4 codebook itself is not printed on the pages; the values
@@ -539,4 +545,130 @@ void orc_grouped_dgrad_mxfp4(const uint16_t *dy, const uint8_t *w, const uint8_t
                              int64_t E, int64_t N, int64_t K, const int64_t *rows, int64_t n_rows, double *dx)
 {
     grouped_dgrad(1, dy, w, scales, offsets, E, N, K, rows, n_rows, dx);
+}
+
+/* ------------------------------------------------------------------ */
+/* Native W4A8: MXFP8 activations x MXFP4 weights [W4A8] [OCP-MX]      */
+/* ------------------------------------------------------------------ */
+
+/* Value of an e4m3 code (OCP "E4M3": no infinities): sign = bit 7,
+ * exponent = bits 6..3 with bias 7, mantissa = bits 2..0; exponent 0 is
+ * subnormal (m/8 * 2^-6); S.1111.111 is NaN; the largest finite magnitude
+ * is 448 (code 0x7E). */
+static double e4m3_value(unsigned code)
+{
+    const unsigned e = (code >> 3) & 15u, m = code & 7u;
+    double v;
+    if (e == 15u && m == 7u) return NAN;
+    if (e == 0u)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, (int)e - 7);
+    return (code & 0x80u) ? -v : v;
+}
+
+void orc_e4m3_values(double out[256])
+{
+    for (unsigned c = 0; c < 256; ++c) out[c] = e4m3_value(c);
+}
+
+/* Nearest finite e4m3 magnitude code (0x00 .. 0x7E) to a non-negative m,
+ * found by comparing against every candidate; an exact tie goes to the even
+ * code (round to nearest even on the mantissa).  Everything above 448 ends
+ * at 448, the largest candidate (saturation, reading C19). */
+static unsigned e4m3_round_magnitude(double m)
+{
+    unsigned best = 0u;
+    double bestd = m; /* distance to code 0 (= 0.0) */
+    for (unsigned c = 1u; c <= 0x7Eu; ++c) {
+        const double d = fabs(m - e4m3_value(c));
+        if (d < bestd || (d == bestd && (c % 2u) == 0u)) {
+            bestd = d;
+            best = c;
+        }
+    }
+    return best;
+}
+
+/* Quantise rows x K bf16 activations to MXFP8: codes [rows, K] e4m3 and
+ * scales [rows, K/32] e8m0.  Per block of 32: X = floor(log2(amax)) - 8 (8
+ * is e4m3's largest exponent), clamped to [-127, 127]; code = the nearest
+ * e4m3 value to x / 2^X (saturating at 448), with x's sign; an all-zero
+ * block gets scale byte 0 and zero codes (reading C19).  x / 2^X is exact
+ * in fp64.  Requires K % 32 == 0 and finite inputs. */
+void orc_quant_mxfp8(const uint16_t *x, int64_t rows, int64_t K, uint8_t *codes, uint8_t *scales)
+{
+    const int64_t nb = K / 32;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const uint16_t *blk = x + r * K + b * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                const double a = fabs((double)bf16_to_float(blk[i]));
+                if (a > amax) amax = a;
+            }
+            int sexp;
+            if (amax == 0.0) {
+                sexp = -127;
+            } else {
+                int ex;
+                frexp(amax, &ex); /* amax = f * 2^ex, f in [0.5, 1) */
+                sexp = (ex - 1) - 8;
+                if (sexp < -127) sexp = -127;
+                if (sexp > 127) sexp = 127;
+            }
+            scales[r * nb + b] = (uint8_t)(sexp + 127);
+            for (int i = 0; i < 32; ++i) {
+                const double v = (double)bf16_to_float(blk[i]);
+                const unsigned mag = e4m3_round_magnitude(ldexp(fabs(v), -sexp));
+                codes[r * K + b * 32 + i] = (uint8_t)(mag | (signbit(v) ? 0x80u : 0u));
+            }
+        }
+    }
+}
+
+/* Decode MXFP8: value = e4m3(code) * 2^(s-127), in fp64. */
+void orc_dequant_mxfp8(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K, double *out)
+{
+    const int64_t nb = K / 32;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            out[r * K + k] = e4m3_value(codes[r * K + k]) * ldexp(1.0, (int)scales[r * nb + k / 32] - 127);
+}
+
+/* Native W4A8 grouped GEMM: y[i, n] = sum_k A[r, k] * W_e[n, k] for the
+ * sorted rows r = rows[i] of expert e, with A the MXFP8 activations
+ * (e4m3 x 2^(sa-127)) and W the MXFP4 weights (e2m1 x 2^(sw-127)); every
+ * product and sum in fp64 [W4A8].  Rows outside [0, offsets[E]) give NaN. */
+void orc_grouped_gemm_w4a8(const uint8_t *qa, const uint8_t *sa, const uint8_t *w, const uint8_t *sw,
+                           const int32_t *offsets, int64_t E, int64_t N, int64_t K, const int64_t *rows,
+                           int64_t n_rows, double *y)
+{
+    float *wd = (float *)malloc((size_t)(N * K) * sizeof(float));
+    double *ad = (double *)malloc((size_t)K * sizeof(double));
+    for (int64_t e = 0; e < E; ++e) {
+        int used = 0;
+        for (int64_t i = 0; i < n_rows; ++i)
+            if (rows[i] >= offsets[e] && rows[i] < offsets[e + 1]) used = 1;
+        if (!used) continue;
+        orc_dequant_mxfp4(w + e * N * (K / 2), sw + e * N * (K / 32), N, K, wd);
+        for (int64_t i = 0; i < n_rows; ++i) {
+            if (!(rows[i] >= offsets[e] && rows[i] < offsets[e + 1])) continue;
+            orc_dequant_mxfp8(qa + rows[i] * K, sa + rows[i] * (K / 32), 1, K, ad);
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+            for (int64_t n = 0; n < N; ++n) {
+                const float *wrow = wd + n * K;
+                double acc = 0.0;
+                for (int64_t kk = 0; kk < K; ++kk) acc += ad[kk] * (double)wrow[kk];
+                y[i * N + n] = acc;
+            }
+        }
+    }
+    for (int64_t i = 0; i < n_rows; ++i)
+        if (!(rows[i] >= 0 && rows[i] < offsets[E]))
+            for (int64_t n = 0; n < N; ++n) y[i * N + n] = NAN;
+    free(ad);
+    free(wd);
 }

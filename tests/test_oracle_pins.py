@@ -511,3 +511,165 @@ def test_dgrad_is_the_transpose_of_the_forward_gemm():
     lhs = math.fsum((_af(dy) * y).ravel())
     rhs = math.fsum((dx * _af(x)).ravel())
     assert abs(lhs - rhs) <= 1e-9 * (abs(lhs) + 1.0)
+
+
+# ---------------------------------------------------------------- native W4A8 (MXFP8 activations)
+
+
+def _bf16_bits(vals):
+    return (np.asarray(vals, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_e4m3_table_matches_torch_float8():
+    """Every e4m3 code decodes as torch's float8_e4m3fn does (an independent
+    implementation of the OCP E4M3 format), NaN at the same two codes."""
+    torch = pytest.importorskip("torch")
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.e4m3_values()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.flatnonzero(np.isnan(got)).tolist() == [0x7F, 0xFF]
+
+
+def test_e4m3_codes_from_the_specification():
+    g = _golden("mxfp8.json")
+    v = oracle.e4m3_values()
+    for c in g["e4m3_codes"]:
+        assert v[c["code"]] == c["value"], c
+
+
+def test_mxfp8_worked_block():
+    """The hand-worked block: scale byte, every code (ties to even, subnormals,
+    negative zero)."""
+    g = _golden("mxfp8.json")
+    x = np.zeros(32, np.float32)
+    for i, e in enumerate(g["block"]):
+        x[i] = e["x"]
+    codes, scales = oracle.quant_mxfp8(_bf16_bits(x)[None, :])
+    assert scales[0, 0] == g["block_scale_byte"]
+    for i, e in enumerate(g["block"]):
+        assert codes[0, i] == e["code"], (e, codes[0, i])
+    assert np.all(codes[0, len(g["block"]):] == 0)
+
+
+def test_mxfp8_saturates_above_448():
+    g = _golden("mxfp8.json")["saturation"]
+    x = np.zeros(32, np.float32)
+    x[3] = g["amax"]
+    x[4] = -g["amax"]
+    codes, scales = oracle.quant_mxfp8(_bf16_bits(x)[None, :])
+    assert scales[0, 0] == g["scale_byte"]
+    assert codes[0, 3] == g["code"] and codes[0, 4] == (g["code"] | 0x80)
+
+
+def test_mxfp8_rounding_matches_torch_float8_conversion():
+    """Inside each block the codes are torch's round-to-nearest-even fp32 ->
+    float8_e4m3fn conversion of x / 2^X, wherever that conversion is finite
+    (|x / 2^X| < 464); beyond it the oracle saturates to 448."""
+    torch = pytest.importorskip("torch")
+    rng = inputs.rng(71)
+    rows, K = 64, 256
+    x = rng.standard_normal((rows, K)).astype(np.float32)
+    x *= np.exp2(rng.integers(-20, 20, size=(rows, K // 32, 1))).repeat(32, axis=2).reshape(rows, K)
+    x[5, 32:64] = 0.0  # an all-zero block
+    bits = _bf16_bits(x)
+    xf = (bits.astype(np.uint32) << 16).view(np.float32)
+    codes, scales = oracle.quant_mxfp8(bits)
+    inv = np.exp2(127.0 - scales.astype(np.float64)).repeat(32, axis=1)
+    scaled = (xf.astype(np.float64) * inv).astype(np.float32)  # exact: power-of-two scaling of a bf16
+    ref = torch.from_numpy(scaled).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    fin = np.abs(scaled) < 464
+    assert np.array_equal(codes[fin], ref[fin])
+    assert np.all((codes[~fin] & 0x7F) == 0x7E)
+    assert scales[5, 1] == 0 and np.all(codes[5, 32:64] == 0)
+
+
+def test_mxfp8_shared_exponent_is_the_smallest_without_overflow():
+    """X is the OCP choice: the block's largest element lands in [256, 512)
+    after division by 2^X (so one exponent lower would leave e4m3's range and
+    one higher would waste the top binade)."""
+    rng = inputs.rng(72)
+    x = rng.standard_normal((200, 64)).astype(np.float32) * np.exp2(rng.integers(-30, 30, (200, 1))).astype(np.float32)
+    bits = _bf16_bits(x)
+    xf = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    _, scales = oracle.quant_mxfp8(bits)
+    amax = np.abs(xf.reshape(200, 2, 32)).max(axis=2)
+    lead = amax / np.exp2(scales.astype(np.float64) - 127.0)
+    assert np.all((lead >= 256) & (lead < 512))
+
+
+def test_mxfp8_dequant_error_bounds():
+    """|x - dequant| <= 2^-4 |x| for normal e4m3 results (half an ulp of a
+    3-bit mantissa), <= 2^-10 * 2^X for subnormal ones, < 64 * 2^X when
+    saturated."""
+    rng = inputs.rng(73)
+    x = rng.standard_normal((128, 128)).astype(np.float32)
+    x[:, ::7] *= 1e-3
+    bits = _bf16_bits(x)
+    xf = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    codes, scales = oracle.quant_mxfp8(bits)
+    deq = oracle.dequant_mxfp8(codes, scales)
+    s = np.exp2(scales.astype(np.float64) - 127.0).repeat(32, axis=1)
+    v = np.abs(xf) / s
+    err = np.abs(deq - xf)
+    normal = (v >= 2.0 ** -6) & (v < 448)
+    sub = v < 2.0 ** -6
+    sat = v >= 448
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(xf[normal]))
+    assert np.all(err[sub] <= 2.0 ** -10 * s[sub])
+    assert np.all(err[sat] < 64 * s[sat])
+
+
+def test_w4a8_gemm_is_numpy_matmul_of_the_dequantised_operands():
+    rng = inputs.rng(74)
+    E, N, K = 3, 24, 192
+    counts = [5, 0, 7]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    M = int(offsets[-1])
+    w, sw = inputs.mxfp4_random(rng, E, N, K)
+    codes, sa = oracle.quant_mxfp8(inputs.bf16_normal(rng, (M, K)))
+    y = oracle.grouped_gemm_w4a8(codes, sa, w, sw, offsets)
+    ad = oracle.dequant_mxfp8(codes, sa)
+    for e in range(E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        if r1 == r0:
+            continue
+        wd = oracle.dequant_mxfp4(w[e], sw[e]).astype(np.float64)
+        assert np.allclose(y[r0:r1], ad[r0:r1] @ wd.T, rtol=1e-13, atol=1e-13)
+
+
+def test_w4a8_gemm_closed_form():
+    """Codes 0x38 (= 1.0) with activation scale byte 127 + s and weights all
+    e2m1 1.0 with scale byte 127 + t: every output is K * 2^(s + t)."""
+    E, N, K = 2, 8, 128
+    offsets = np.array([0, 3, 4], np.int32)
+    codes = np.full((4, K), 0x38, np.uint8)
+    sa = np.full((4, K // 32), 127, np.uint8)
+    sa[3] = 129
+    w = np.full((E, N, K // 2), 0x22, np.uint8)
+    sw = np.full((E, N, K // 32), 127, np.uint8)
+    sw[1] = 124
+    y = oracle.grouped_gemm_w4a8(codes, sa, w, sw, offsets)
+    assert np.all(y[:3] == K) and np.all(y[3] == K * 2.0 ** (2 - 3))
+
+
+def test_w4a8_stays_within_the_e4m3_bound_of_the_bf16_activation_result():
+    """Quantising the activations moves each product by at most 1/8 of its
+    size (2^-4 when not saturated), so |Y_w4a8 - Y_bf16| <= sum |a w| / 8."""
+    rng = inputs.rng(75)
+    E, N, K = 2, 16, 256
+    offsets = np.array([0, 6, 9], np.int32)
+    w, sw = inputs.mxfp4_random(rng, E, N, K)
+    a = inputs.bf16_normal(rng, (9, K))
+    codes, sa = oracle.quant_mxfp8(a)
+    y8 = oracle.grouped_gemm_w4a8(codes, sa, w, sw, offsets)
+    y16 = oracle.grouped_gemm_mxfp4(a, w, sw, offsets)
+    af = np.abs(_af(a))
+    for e in range(E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        wd = np.abs(oracle.dequant_mxfp4(w[e], sw[e]).astype(np.float64))
+        bound = af[r0:r1] @ wd.T / 8
+        assert np.all(np.abs(y8[r0:r1] - y16[r0:r1]) <= bound)
+    rel = np.linalg.norm(y8 - y16) / np.linalg.norm(y16)
+    assert rel < 0.04, rel
