@@ -1,0 +1,413 @@
+// mx.cu -- native W4A8 mode: MXFP8 activations times MXFP4 weights on the
+// block-scaled tcgen05 tensor cores (kind::mxf8f6f4), and the MXFP8
+// activation quantiser that feeds it.
+//
+// bw24 v0.9.0 release notes (Features, "f8f4 tile piece 1"; Documentation,
+// "prefill arc design"): W4A8-FP8 multiplies native e2m1 weights by e4m3
+// activations in one block-scaled MMA.  grouped-nf4-gemm index.json,
+// system_manifest.owns: the grouped GEMM runs on native MXFP4.
+//
+// Quantiser (OCP MX v1.0, MXFP8 E4M3): the 32 consecutive k of one row share
+// an e8m0 scale 2^X with X = floor(log2(amax)) - 8 clamped to [-127, 127];
+// each element is x * 2^-X rounded to the nearest e4m3 value, ties to even,
+// saturating at +-448 (cvt.rn.satfinite).  An all-zero block gets scale 0.
+//
+// GEMM design (B200):
+//  * D^T[n, r] = W_e[n, :] . A[r, :]: the 128 weight rows of a tile are the
+//    MMA's M, the rows (tokens) of the group its N, as in the bf16 path.
+//  * Both operands go straight from global memory into 128B-swizzled shared
+//    memory by TMA.  The packed e2m1 weights are expanded by the TMA unit
+//    itself into the layout the MMA reads (16 codes in 8 bytes followed by 8
+//    bytes of padding, so 128 codes fill one 128-byte row); the e4m3
+//    activations are plain bytes.  The SM decodes nothing: no lookup table
+//    and no bf16 copy of a weight exist anywhere.
+//  * Block scales: a loader warp copies, per 128-k stage, the e8m0 scales of
+//    the tile's 128 weight rows and of the group's rows into shared memory
+//    in the layout tcgen05.cp reads (row m at byte 16*(m%32) + 4*(m/32), one
+//    byte per 32-k block); the MMA thread copies both to TMEM with
+//    tcgen05.cp.32x128b.warpx4 just before the stage's four K=32 MMAs, whose
+//    scale-factor ids select the byte of the block.
+//  * K % 128 == 64 (e.g. 2880): the last stage reads [K-128, K) and issues
+//    only its upper two K=32 steps, so no box reads past the end of a row.
+//  * Warp roles (8 warps): 0 = TMA producer, 1 = TMEM owner + MMA issuer,
+//    2 = scale loader, 4..7 = epilogue (warp w reads TMEM lanes
+//    32*(w%4)..+31, i.e. weight rows).  Two TMEM accumulators let the
+//    epilogue of one unit overlap the main loop of the next.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace gnf4 {
+namespace {
+
+// ------------------------------------------------------------------ quantiser
+
+constexpr int kQThreads = 256;
+
+// One thread quantises 8 consecutive k (16 bytes of bf16); the 4 threads of
+// a 32-k block agree on its amax with two shuffles.
+__global__ void __launch_bounds__(kQThreads) quant_mxfp8_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                long long octets, uint8_t* __restrict__ codes,
+                                                                uint8_t* __restrict__ scales) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const long long o = (long long)blockIdx.x * kQThreads + threadIdx.x;
+  const bool ok = o < octets;
+  const uint4 v = ok ? ldg_nc_u128(x + o * 8) : make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  // |bf16| compares like its bit pattern with the sign cleared
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  // floor(log2(amax)) is the bf16 exponent field - 127; zero and subnormal
+  // amax clamp to the smallest scale
+  const int ef = (int)(m >> 7);
+  const int X = ef == 0 ? -127 : max(ef - 127 - 8, -127);
+  const float inv = __uint_as_float((uint32_t)(127 - X) << 23);  // 2^-X, a normal float for every X here
+  uint32_t out[2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __fmul_rn(__uint_as_float(w[i] << 16), inv);
+    const float hi = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv);
+    uint16_t pr;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(hi), "f"(lo));
+    if (i & 1)
+      out[i >> 1] |= (uint32_t)pr << 16;
+    else
+      out[i >> 1] = pr;
+  }
+  if (ok) {
+    *reinterpret_cast<uint2*>(codes + o * 8) = make_uint2(out[0], out[1]);
+    if ((threadIdx.x & 3) == 0) scales[o >> 2] = (uint8_t)(X + 127);
+  }
+}
+
+// ------------------------------------------------------------------ GEMM
+
+constexpr int kBT = 128;  // rows (tokens) per unit = max MMA N
+constexpr int kBW = 128;  // weight rows per unit = MMA M
+constexpr int kBK = 128;  // k per stage
+constexpr int kStages = 6;
+constexpr int kSmallBox = 32;  // activation rows per TMA box for groups of <= 32 rows
+constexpr int kEpiWarp0 = 4;
+constexpr int kThreads = 8 * 32;
+constexpr int kWStageBytes = kBW * kBK;    // padded e2m1 in shared memory: one byte per code
+constexpr int kWStageTx = kBW * kBK / 2;   // bytes the TMA reads: two codes per byte
+constexpr int kAStageBytes = kBT * kBK;    // e4m3
+constexpr int kTmemCols = 512;
+constexpr int kSfwCol = 2 * kBT;           // 4 columns of weight scales
+constexpr int kSfaCol = kSfwCol + 4;       // 4 columns of activation scales
+static_assert(kSfaCol + 4 <= kTmemCols, "TMEM budget");
+
+struct MxSmem {
+  uint8_t w[kStages][kWStageBytes];  // 1024-aligned (offset 0)
+  uint8_t a[kStages][kAStageBytes];
+  uint32_t sfw[kStages][kBW];        // weight scales of the stage, tcgen05.cp layout
+  uint32_t sfa[kStages][kBT];        // activation scales of the stage
+  int off[kMaxExperts + 1];
+  int upre[kMaxExperts + 1];
+  int scratch[kMaxExperts];
+  uint64_t full[kStages], sfull[kStages], empty[kStages];
+  uint64_t accf[2], acce[2];
+  uint64_t mdone;  // abort path only: every issued MMA has retired
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(MxSmem) + 1024 <= 227 * 1024, "shared memory budget");
+
+struct MxArgs {
+  const uint8_t* sa;   // activation scales e8m0 [M, K/32] (the codes come by TMA)
+  const uint8_t* sw;   // e8m0 [E, N, K/32]
+  const int* offsets;  // [E+1] or null
+  const int* counts;   // [E] or null
+  __nv_bfloat16* y;    // [M, N]
+  unsigned* err;
+  int E, N, K, M;
+};
+
+struct Unit {
+  int e, j, row0, rows;
+};
+
+__device__ __forceinline__ Unit unit_of(const MxSmem& s, int E, int u) {
+  Unit x;
+  x.e = find_group(s.upre, E, u);
+  const int local = u - s.upre[x.e];
+  const int rows_e = s.off[x.e + 1] - s.off[x.e];
+  const int nch = (rows_e + kBT - 1) / kBT;
+  x.j = local / nch;
+  const int c = local - x.j * nch;
+  x.row0 = s.off[x.e] + c * kBT;
+  x.rows = min(kBT, s.off[x.e + 1] - x.row0);
+  return x;
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte scale block (no swizzle;
+// 8-row core matrices 128 bytes apart; one 16-byte column, so the leading
+// byte offset is unused).
+__device__ __forceinline__ uint64_t sdesc_scales(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(128u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  return d;
+}
+
+// 32 lanes x 128 bits from shared memory into TMEM, replicated to all four
+// 32-lane quarters.
+__device__ __forceinline__ void tc_copy_scales(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Instruction descriptor: kind::mxf8f6f4, A = e2m1, B = e4m3, e8m0 scales,
+// both K-major, M = 128, N = n (multiple of 16), K = 32; scale-factor ids
+// (the byte of the scale column) j for both operands.
+__device__ __forceinline__ uint32_t idesc_w4a8(uint32_t n, uint32_t j) {
+  return (j << 4) | (5u << 7) | (0u << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) | (j << 29);
+}
+
+__device__ __forceinline__ void tc_mma_w4a8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// 4 scale bytes starting at an even byte address (two 2-byte loads).
+__device__ __forceinline__ uint32_t ld_scales4(const uint8_t* p) {
+  const uint16_t* q = reinterpret_cast<const uint16_t*>(p);
+  return (uint32_t)__ldg(q) | ((uint32_t)__ldg(q + 1) << 16);
+}
+
+__device__ __forceinline__ void sts_u128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_w4a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_big,
+                     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_w_tail,
+                     MxArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  MxSmem& s = *reinterpret_cast<MxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  unsigned* err = p.err;
+  volatile int* abort = &s.abort;
+
+  griddep_launch_dependents();
+  griddep_wait();
+  if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, err)) return;
+  const int nwt = (p.N + kBW - 1) / kBW;
+  block_exclusive_scan(p.E, s.upre, s.scratch,
+                       [&](int e) { return ((s.off[e + 1] - s.off[e] + kBT - 1) / kBT) * nwt; });
+  const int U = s.upre[p.E];
+  if ((int)blockIdx.x >= U) return;  // uniform over the block
+  const int K = p.K;
+  const int nk = (K + kBK - 1) / kBK;
+  const bool tail = (K % kBK) != 0;  // K % 128 == 64
+
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.sfull[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.accf[i], 1);
+      mbar_init(&s.acce[i], 4);
+    }
+    mbar_init(&s.mdone, 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_a_big);
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_w_tail);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+        const Unit x = unit_of(s, p.E, u);
+        const bool big = x.rows > kSmallBox;
+        const int wrow = x.e * p.N + x.j * kBW;
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          const int st = it % kStages, use = it / kStages;
+          if (it >= kStages && !(ok = mbar_wait(&s.empty[st], (use - 1) & 1, err, abort))) break;
+          const bool last_tail = tail && kt == nk - 1;
+          const int k0 = last_tail ? K - kBK : kt * kBK;
+          mbar_arrive_expect_tx(&s.full[st], kWStageTx + (big ? kBT : kSmallBox) * kBK);
+          if (last_tail)
+            tma_load_2d(s.w[st], &tm_w_tail, &s.full[st], 0, wrow);
+          else
+            tma_load_3d(s.w[st], &tm_w, &s.full[st], 0, kt, wrow);
+          tma_load_2d(s.a[st], big ? &tm_a_big : &tm_a, &s.full[st], k0, x.row0);
+        }
+      }
+      if (!ok)  // drain loads still in flight before shared memory goes away
+        for (int i = max(0, it - kStages); i < it; ++i) mbar_drain(&s.full[i % kStages], (i / kStages) & 1);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale loader
+    // Lane l serves rows l, l+32, l+64, l+96 of the tile and of the group
+    // chunk; rows outside them get scale 2^0 (their products are never stored).
+    const int nsb = K / 32;
+    const uint8_t* swb = p.sw;
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+      const Unit x = unit_of(s, p.E, u);
+      for (int kt = 0; kt < nk; ++kt, ++it) {
+        const int st = it % kStages, use = it / kStages;
+        if (it >= kStages && !(ok = mbar_wait(&s.empty[st], (use - 1) & 1, err, abort))) break;
+        const int b0 = ((tail && kt == nk - 1) ? K - kBK : kt * kBK) / 32;  // even: K % 64 == 0
+        uint32_t wv[4], av[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int m = lane + 32 * c;
+          const int n = x.j * kBW + m;
+          wv[c] = n < p.N ? ld_scales4(swb + ((size_t)x.e * p.N + (size_t)n) * (size_t)nsb + b0) : 0x7F7F7F7Fu;
+          av[c] = m < x.rows ? ld_scales4(p.sa + (size_t)(x.row0 + m) * (size_t)nsb + b0) : 0x7F7F7F7Fu;
+        }
+        sts_u128(smem_u32(&s.sfw[st][lane * 4]), wv[0], wv[1], wv[2], wv[3]);
+        sts_u128(smem_u32(&s.sfa[st][lane * 4]), av[0], av[1], av[2], av[3]);
+        fence_proxy_async_smem();  // the tensor core reads these through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.sfull[st]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, uc = 0;
+      bool ok = true;
+      const uint32_t t_sfw = tmem + (uint32_t)kSfwCol, t_sfa = tmem + (uint32_t)kSfaCol;
+      for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
+        const Unit x = unit_of(s, p.E, u);
+        const int ab = uc & 1;
+        if (uc >= 2 && !(ok = mbar_wait(&s.acce[ab], ((uc >> 1) - 1) & 1, err, abort))) break;
+        tc_fence_after();
+        const uint32_t n_mma = (uint32_t)((x.rows + 15) & ~15);
+        const uint32_t d_tmem = tmem + (uint32_t)(ab * kBT);
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          const int st = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          const bool rf = mbar_try_wait(&s.full[st], ph);
+          const bool rs = mbar_try_wait(&s.sfull[st], ph);
+          if (!(rf && rs)) {
+            if (!(ok = mbar_wait(&s.full[st], ph, err, abort))) break;
+            if (!(ok = mbar_wait(&s.sfull[st], ph, err, abort))) break;
+          }
+          tc_fence_after();
+          tc_copy_scales(t_sfw, sdesc_scales(smem_u32(s.sfw[st])));
+          tc_copy_scales(t_sfa, sdesc_scales(smem_u32(s.sfa[st])));
+          const uint32_t w_addr = smem_u32(s.w[st]), a_addr = smem_u32(s.a[st]);
+          const int j0 = (tail && kt == nk - 1) ? 2 : 0;
+          for (int j = j0; j < kBK / 32; ++j)
+            tc_mma_w4a8(d_tmem, sdesc_k_sw128(w_addr + 32 * j), sdesc_k_sw128(a_addr + 32 * j),
+                        idesc_w4a8(n_mma, (uint32_t)j), t_sfw | ((uint32_t)j << 30), t_sfa | ((uint32_t)j << 30),
+                        kt != 0 || j > j0);
+          tc_commit(&s.empty[st]);
+        }
+        if (!ok) break;
+        tc_commit(&s.accf[ab]);
+      }
+      if (!ok) {
+        // abort: let every MMA already issued retire before TMEM is released
+        tc_commit(&s.mdone);
+        mbar_drain(&s.mdone, 0);
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+    int uc = 0;
+    for (int u = blockIdx.x; u < U; u += gridDim.x, ++uc) {
+      const Unit x = unit_of(s, p.E, u);
+      const int ab = uc & 1;
+      if (!mbar_wait(&s.accf[ab], (uc >> 1) & 1, err, abort)) break;
+      tc_fence_after();
+      const int n = x.j * kBW + q * 32 + lane;
+      __nv_bfloat16* ycol = p.y + (size_t)x.row0 * p.N + n;
+      for (int c = 0; c * 32 < x.rows; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBT + c * 32), v);
+        tmem_wait_ld();
+        const int lim = min(32, x.rows - c * 32);
+        if (n < p.N) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < lim) ycol[(size_t)(c * 32 + i) * p.N] = __float2bfloat16_rn(__uint_as_float(v[i]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.acce[ab]);
+    }
+  }
+
+  // Normal path: the epilogue has consumed every accumulator, so every MMA
+  // and TMEM access has completed here.
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quant_mxfp8(const __nv_bfloat16* x, long long elems, uint8_t* codes, uint8_t* scales,
+                               cudaStream_t stream) {
+  const long long octets = elems / 8;
+  if (octets == 0) return cudaSuccess;
+  const long long blocks = (octets + kQThreads - 1) / kQThreads;
+  return launch_pdl(quant_mxfp8_kernel, dim3((unsigned)blocks), dim3(kQThreads), 0, stream, x, octets, codes,
+                    scales);
+}
+
+size_t gemm_w4a8_smem_bytes() { return sizeof(MxSmem) + 1024; }
+int gemm_w4a8_rows_per_unit() { return kBT; }
+int gemm_w4a8_weight_rows_per_unit() { return kBW; }
+int gemm_w4a8_small_box_rows() { return kSmallBox; }
+
+cudaError_t launch_gemm_w4a8(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
+                             const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* w_scales,
+                             const int* offsets, const int* counts, __nv_bfloat16* y, unsigned* err, int E, int N,
+                             int K, int M, int grid, cudaStream_t stream) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_w4a8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)gemm_w4a8_smem_bytes());
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  MxArgs p{a_scales, w_scales, offsets, counts, y, err, E, N, K, M};
+  return launch_pdl(gemm_w4a8_kernel, dim3(grid), dim3(kThreads), gemm_w4a8_smem_bytes(), stream, tm_a, tm_a_big,
+                    tm_w, tm_w_tail, p);
+}
+
+}  // namespace gnf4

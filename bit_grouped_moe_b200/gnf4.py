@@ -47,11 +47,13 @@ _GROUPED = ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_ge
             "gnf4_grouped_gemv_mxfp4_swiglu", "gnf4_grouped_dgrad_nf4", "gnf4_grouped_dgrad_mxfp4")
 for _name in _GROUPED:
     getattr(_lib, _name).argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+_lib.gnf4_quantize_mxfp8.argtypes = [_P, _I, _I, _P, _P, _P]
+_lib.gnf4_grouped_gemm_w4a8.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
 _lib.gnf4_dequant_nf4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 _lib.gnf4_dequant_mxfp4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", "gnf4_route_topk_permute",
-              *_GROUPED, "gnf4_combine",
+              *_GROUPED, "gnf4_combine", "gnf4_quantize_mxfp8", "gnf4_grouped_gemm_w4a8",
               "gnf4_dequant_nf4_f32", "gnf4_dequant_mxfp4_f32"):
     getattr(_lib, _name).restype = _I
 
@@ -256,3 +258,17 @@ def moe_step(fmt, x, topk_ids, weights, w1, s1, w2, s2, h=None, ws=None, stream=
     out = torch.empty(T, N2, dtype=torch.bfloat16, device=dev)
     combine(y2, f2s, weights, out, stream=stream)
     return out, offsets
+
+
+def quantize_mxfp8(x, codes, scales, stream=None):
+    """x bf16 [M, K] -> codes uint8 [M, K] (e4m3) and scales uint8 [M, K/32] (e8m0), preallocated."""
+    M, K = x.shape
+    _check(_lib.gnf4_quantize_mxfp8(_ptr(x), M, K, _ptr(codes), _ptr(scales), _stream(stream)))
+
+
+def grouped_gemm_w4a8(a_codes, a_scales, w, w_scales, y, offsets=None, counts=None, stream=None):
+    """Native W4A8: y [M, N] = MXFP8 activations (codes, scales) x the MXFP4 stack [E, N, K/2] per group."""
+    E, N, K2 = w.shape
+    M = a_codes.shape[0]
+    _check(_lib.gnf4_grouped_gemm_w4a8(_ptr(a_codes), _ptr(a_scales), _ptr(w), _ptr(w_scales), _ptr(offsets),
+                                       _ptr(counts), E, N, 2 * K2, M, _ptr(y), _stream(stream)))

@@ -263,6 +263,42 @@ gnf4_status gnf4_grouped_gemv_mxfp4_swiglu(const void *a, const uint8_t *w_gate_
                                            void *h, void *stream);
 
 /* ------------------------------------------------------------------ */
+/* Native W4A8 mode: MXFP8 activations x MXFP4 weights                 */
+/* ------------------------------------------------------------------ */
+
+/* The block-scaled tensor-core form of the MXFP4 projection (bw24 v0.9.0
+ * release notes, Documentation "prefill arc design": W4A8-FP8, e4m3
+ * activations times native e2m1 weights in one block-scaled MMA; Features
+ * "f8f4 tile piece 1": e4m3 activation quantisation; grouped-nf4-gemm
+ * index.json, system_manifest.owns: native MXFP4).  The activations are
+ * first quantised to MXFP8; the weights are the MXFP4 stack unchanged.
+ *
+ * gnf4_quantize_mxfp8: x bf16 [M, K] -> codes e4m3 [M, K] (u8) and scales
+ * e8m0 [M, K/32] (u8).  Per block of 32 consecutive k of one row:
+ *     X = floor(log2(max |x|)) - 8, clamped to [-127, 127] (X = -127 for an
+ *         all-zero block); scale byte = X + 127;
+ *     code = x * 2^-X rounded to the nearest e4m3 value, ties to even,
+ *            saturating at +-448, sign kept on zero results
+ * (OCP MX v1.0 MXFP8; the pages give no rule, this is the reading used).
+ * Bit-exact: the same inputs give the same bytes on every run.  K must be a
+ * positive multiple of 32; inputs must be finite.  x, codes: 16-byte
+ * aligned device memory; scales: device memory.
+ *
+ * gnf4_grouped_gemm_w4a8: for every sorted row r of expert e
+ *     y[r, n] = sum_k A[r, k] * W_e[n, k],
+ *     A[r, k] = e4m3(codes[r, k]) * 2^(a_scales[r, k/32] - 127),
+ *     W_e[n, k] = e2m1(w[e, n, k]) * 2^(w_scales[e, n, k/32] - 127),
+ * products exact, fp32 accumulation, bf16 output y [M, N].  w, w_scales,
+ * offsets, counts, E, N and M as the MXFP4 grouped GEMM; a_codes / a_scales
+ * as written by gnf4_quantize_mxfp8 for the group-sorted rows.  K must be a
+ * multiple of 64 in [128, 65536].  Alignment: a_codes 16 bytes, w 32 bytes,
+ * y 16 bytes.  Rows past offsets[E] are not written. */
+gnf4_status gnf4_quantize_mxfp8(const void *x, int M, int K, uint8_t *codes, uint8_t *scales, void *stream);
+gnf4_status gnf4_grouped_gemm_w4a8(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *w,
+                                   const uint8_t *w_scales, const int32_t *offsets, const int32_t *counts, int E,
+                                   int N, int K, int M, void *y, void *stream);
+
+/* ------------------------------------------------------------------ */
 /* Top-k combine                                                       */
 /* ------------------------------------------------------------------ */
 
