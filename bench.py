@@ -145,7 +145,7 @@ class Workload:
     """Device-resident inputs of one workload: rotating weight copies larger
     than L2, a set of token batches, and the step's output buffers."""
 
-    def __init__(self, name, device, seed, build_host_copy, swiglu=False, dgrad=False):
+    def __init__(self, name, device, seed, build_host_copy, swiglu=False, dgrad=False, w4a8=False):
         import torch
 
         from bit_grouped_moe_b200 import gnf4
@@ -208,6 +208,16 @@ class Workload:
             self.dx1 = torch.empty(M, self.p1.K, dtype=torch.bfloat16, device=device)
             self.dh = torch.empty(M, self.p2.K, dtype=torch.bfloat16, device=device)
             self.dfn = f.grouped_dgrad_nf4 if wl.fmt == "nf4" else f.grouped_dgrad_mxfp4
+        # optional native W4A8 mode (MXFP4 stacks): both projections' activations are
+        # quantised to MXFP8 every step and the block-scaled GEMM runs on the codes
+        self.w4a8 = w4a8
+        if w4a8:
+            assert wl.fmt == "mxfp4", "the W4A8 mode runs on MXFP4 weight stacks"
+            self.decode = False  # one GEMM path for every group size
+            self.qa1 = torch.empty(M, self.p1.K, dtype=torch.uint8, device=device)
+            self.sa1 = torch.empty(M, self.p1.K // 32, dtype=torch.uint8, device=device)
+            self.qa2 = torch.empty(M, self.p2.K, dtype=torch.uint8, device=device)
+            self.sa2 = torch.empty(M, self.p2.K // 32, dtype=torch.uint8, device=device)
         # optional fused gate_up + SwiGLU first projection: h [M, N1/2] feeds the second
         self.swiglu = swiglu
         if swiglu:
@@ -271,12 +281,24 @@ class Workload:
             if ev is not None:
                 ev[1].record()
             return
+        if self.w4a8:
+            g.quantize_mxfp8(self.xs, self.qa1, self.sa1)
         if ev is not None:
             ev[0].record()
         self.project(w1, s1, w2, s2, ev)
         g.combine(self.y2, self.f2s, wts, self.out)
 
-    def project(self, w1, s1, w2, s2, ev=None):
+    def project(self, w1, s1, w2, s2, ev=None, quantize_first=False):
+        if self.w4a8:
+            g = self.g
+            if quantize_first:
+                g.quantize_mxfp8(self.xs, self.qa1, self.sa1)
+            g.grouped_gemm_w4a8(self.qa1, self.sa1, w1, s1, self.y1, offsets=self.off)
+            if ev is not None:
+                ev[1].record()
+            g.quantize_mxfp8(self.h, self.qa2, self.sa2)
+            g.grouped_gemm_w4a8(self.qa2, self.sa2, w2, s2, self.y2, offsets=self.off)
+            return
         if self.swiglu:
             self.fn1(self.xs, w1, s1, self.hs, offsets=self.off)
         else:
@@ -288,7 +310,7 @@ class Workload:
     def launches_per_step(self):
         # route (one launch for at most 256 pairs, else hist + scan + scatter + gather) + 2 projections + combine
         route = 1 if 0 < self.M <= 256 else 4
-        return route + 2 + (0 if self.dgrad else 1)
+        return route + 2 + (0 if self.dgrad else 1) + (2 if self.w4a8 else 0)
 
 
 # ------------------------------------------------------------------ distributed
@@ -346,7 +368,12 @@ def oracle_step(wl_obj, batch_i, n_slice=None):
     (w1, s1), (w2, s2) = wl_obj.host_stacks
     n1 = wl_obj.p1.N if n_slice is None else min(n_slice, wl_obj.p1.N)
     n2 = wl_obj.p2.N if n_slice is None else min(n_slice, wl_obj.p2.N)
-    gemm = oracle.grouped_gemm_nf4 if wl_obj.wl.fmt == "nf4" else oracle.grouped_gemm_mxfp4
+    if getattr(wl_obj, "w4a8", False):
+        def gemm(a_bits, w, s, off):
+            qa, sa = oracle.quant_mxfp8(a_bits)
+            return oracle.grouped_gemm_w4a8(qa, sa, w, s, off)
+    else:
+        gemm = oracle.grouped_gemm_nf4 if wl_obj.wl.fmt == "nf4" else oracle.grouped_gemm_mxfp4
     gemm(xs, np.ascontiguousarray(w1[:, :n1]), np.ascontiguousarray(s1[:, :n1]), off)
     y2 = gemm(wl_obj.h_host, np.ascontiguousarray(w2[:, :n2]), np.ascontiguousarray(s2[:, :n2]), off)
     y2_bits = np.zeros((wl_obj.M, n2), np.uint16)
@@ -396,6 +423,8 @@ def main():
                     help="time the backward step instead: route + the dgrad of both projections (TFLOP/s)")
     ap.add_argument("--graph", action="store_true",
                     help=f"decode: also time the steps replayed from one CUDA graph of {20} steps")
+    ap.add_argument("--w4a8", action="store_true",
+                    help="MXFP4 workloads: native W4A8 mode (MXFP8 activations, block-scaled tcgen05 GEMM)")
     ap.add_argument("--swiglu", action="store_true",
                     help="first projection = fused gate_up + SwiGLU (gate rows first); the second reads its output")
     ap.add_argument("--weight-copies", type=int, default=N_WEIGHT_COPIES,
@@ -404,7 +433,7 @@ def main():
     globals()["N_WEIGHT_COPIES"] = max(1, args.weight_copies)
 
     wl_def = inputs.WORKLOADS[args.workload]
-    decode = wl_def.T <= 8 and not args.dgrad
+    decode = wl_def.T <= 8 and not args.dgrad and not args.w4a8
     steps = args.steps if args.steps is not None else (20000 if decode else 200)
     warmup = args.warmup if args.warmup is not None else (100 if decode else 10)
     warmup = max(warmup, 3)
@@ -442,7 +471,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     dev = f"cuda:{local}"
     torch.cuda.set_device(local)
     wl = Workload(args.workload, dev, seed=1234 + rank, build_host_copy=(rank == 0 and world == 1),
-                  swiglu=args.swiglu, dgrad=args.dgrad)
+                  swiglu=args.swiglu, dgrad=args.dgrad, w4a8=args.w4a8)
     decode = wl.decode
     wl.h_host = wl.h.cpu().view(torch.int16).numpy().view(np.uint16)
     stream = torch.cuda.current_stream()
@@ -504,7 +533,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
             wl.dfn(wl.dy2, w2, s2, wl.dh, offsets=wl.off)
             wl.dfn(wl.dy1, w1, s1, wl.dx1, offsets=wl.off)
         else:
-            wl.project(w1, s1, w2, s2)
+            wl.project(w1, s1, w2, s2, quantize_first=True)
             g.combine(wl.y2, wl.f2s, d_w, wl.out)
         host_out.copy_(out_dev, non_blocking=True)
 
@@ -563,8 +592,9 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         e2e_val = world * e2e_steps * wl.step_flops() / (e2e_ms / 1e3) / 1e12
 
     peaks, peak_src = load_peaks()
-    kern_file = "gemv.cu" if decode else ("dgrad.cu" if wl.dgrad else "gemm_tc.cu")
-    kern_key = f"{'gemv' if decode else ('dgrad_tc' if wl.dgrad else 'gemm_tc')}_{wl.wl.fmt}{'_swiglu' if wl.swiglu else ''}:{args.workload}:{wl.p1.name}"
+    kern_file = "gemv.cu" if decode else ("dgrad.cu" if wl.dgrad else ("mx.cu" if wl.w4a8 else "gemm_tc.cu"))
+    kern_base = "gemv" if decode else ("dgrad_tc" if wl.dgrad else ("gemm_w4a8" if wl.w4a8 else "gemm_tc"))
+    kern_key = f"{kern_base}_{wl.wl.fmt}{'_swiglu' if wl.swiglu else ''}:{args.workload}:{wl.p1.name}"
     sha = kernel_source_sha([kern_file, "common.cuh"])
     if decode:
         mean_hit = sum(wl.hit[i % N_BATCHES] for i in sampled) / len(sampled)
@@ -579,12 +609,17 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         flops = 2 * wl.M * wl.p1.N * wl.p1.K
         achieved = flops / (dom_ms / 1e3) / 1e12
         pk = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        pk_src = f"bf16_tflops_sustained of {peak_src} (kind::f16 MMA on decoded bf16 tiles)"
+        if wl.w4a8:  # 8-bit-rate MMA: the measured bf16 peak x the nominal dense fp8 / bf16 ratio (4.5 / 2.25)
+            pk = round(2 * pk, 1)
+            pk_src = f"2 x bf16_tflops_sustained of {peak_src} (kind::mxf8f6f4 runs at the fp8 rate)"
+        kname = (f"dgrad_tc_kernel<{wl.wl.fmt}> (dX of {wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.dgrad else
+                 f"gemm_w4a8_kernel ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.w4a8 else
+                 f"gemm_tc_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})")
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk, "unit": "TFLOP/s",
-                "frac": round(achieved / pk, 4), "traffic": committed_traffic(kern_key, sha),
-                "kernel": (f"dgrad_tc_kernel<{wl.wl.fmt}> (dX of {wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.dgrad else
-                           f"gemm_tc_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})"),
+                "frac": round(achieved / pk, 4), "traffic": committed_traffic(kern_key, sha), "kernel": kname,
                 "algorithmic_flops_per_launch": int(flops), "avg_launch_us": round(dom_ms * 1e3, 3),
-                "peak_source": f"bf16_tflops_sustained of {peak_src} (kind::f16 MMA on decoded bf16 tiles)"}
+                "peak_source": pk_src}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -598,8 +633,9 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": steps,
             "warmup": warmup, "ms_per_step": round(ms / steps, 6), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "e4m3 x e2m1 (fp32 accumulate)" if wl.w4a8 else "bf16", "data": "synthetic",
             "config": dict(_config(wl.wl, world), **({"first_projection": "fused gate_up + SwiGLU"} if wl.swiglu else {}),
+                           **({"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if wl.w4a8 else {}),
                            **({"step": "backward: route + dgrad of both projections"} if wl.dgrad else {})),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -621,7 +657,7 @@ def run_reference(args, steps, warmup, world):
     import oracle
 
     wl_def = inputs.WORKLOADS[args.workload]
-    decode = wl_def.T <= 8
+    decode = wl_def.T <= 8 and not args.w4a8
     unit, _ = _unit(decode)
 
     class HostWL:
@@ -629,6 +665,7 @@ def run_reference(args, steps, warmup, world):
 
     h = HostWL()
     h.wl = wl_def
+    h.w4a8 = args.w4a8
     h.E, h.k, h.T = wl_def.E, wl_def.k, wl_def.T
     h.M = h.T * h.k
     h.p1, h.p2 = wl_def.projections[0], wl_def.projections[-1]
@@ -672,7 +709,9 @@ def run_reference(args, steps, warmup, world):
     line = {
         "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": world, "steps": steps, "warmup": warmup,
         "ms_per_step": round(dt * 1e3 / steps, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config(wl_def, world),
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(_config(wl_def, world),
+                       **({"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if args.w4a8 else {})),
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle",
                          "sample": f"each step: the full route + combine and the fp64 grouped GEMM of both "

@@ -29,10 +29,11 @@
 //    scale-factor ids select the byte of the block.
 //  * K % 128 == 64 (e.g. 2880): the last stage reads [K-128, K) and issues
 //    only its upper two K=32 steps, so no box reads past the end of a row.
-//  * Warp roles (8 warps): 0 = TMA producer, 1 = TMEM owner + MMA issuer,
-//    2 = scale loader, 4..7 = epilogue (warp w reads TMEM lanes
-//    32*(w%4)..+31, i.e. weight rows).  Two TMEM accumulators let the
-//    epilogue of one unit overlap the main loop of the next.
+//  * Warp roles (12 warps): 0 = TMA producer, 1 = TMEM owner + MMA issuer,
+//    4..7 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31, i.e. weight
+//    rows), 2, 3 and 8..11 = scale loaders, one per ring slot, so the global
+//    loads of six stages are in flight at once.  Two TMEM accumulators let
+//    the epilogue of one unit overlap the main loop of the next.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -94,7 +95,11 @@ constexpr int kBK = 128;  // k per stage
 constexpr int kStages = 6;
 constexpr int kSmallBox = 32;  // activation rows per TMA box for groups of <= 32 rows
 constexpr int kEpiWarp0 = 4;
-constexpr int kThreads = 8 * 32;
+constexpr int kThreads = 12 * 32;
+// scale-loader index of a warp (its ring slot), or -1
+__device__ __forceinline__ int loader_index(int warp) {
+  return warp == 2 || warp == 3 ? warp - 2 : (warp >= 8 && warp < 8 + kStages - 2 ? warp - 6 : -1);
+}
 constexpr int kWStageBytes = kBW * kBK;    // padded e2m1 in shared memory: one byte per code
 constexpr int kWStageTx = kBW * kBK / 2;   // bytes the TMA reads: two codes per byte
 constexpr int kAStageBytes = kBT * kBK;    // e4m3
@@ -102,6 +107,7 @@ constexpr int kTmemCols = 512;
 constexpr int kSfwCol = 2 * kBT;           // 4 columns of weight scales
 constexpr int kSfaCol = kSfwCol + 4;       // 4 columns of activation scales
 static_assert(kSfaCol + 4 <= kTmemCols, "TMEM budget");
+static_assert(kStages == 6, "one scale-loader warp per ring slot: warps 2, 3, 8..11");
 
 struct MxSmem {
   uint8_t w[kStages][kWStageBytes];  // 1024-aligned (offset 0)
@@ -266,10 +272,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok)  // drain loads still in flight before shared memory goes away
         for (int i = max(0, it - kStages); i < it; ++i) mbar_drain(&s.full[i % kStages], (i / kStages) & 1);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ scale loader
-    // Lane l serves rows l, l+32, l+64, l+96 of the tile and of the group
-    // chunk; rows outside them get scale 2^0 (their products are never stored).
+  } else if (loader_index(warp) >= 0) {
+    // ------------------------------------------------------------ scale loaders
+    // Loader i fills ring slot i only.  Lane l serves rows l, l+32, l+64, l+96
+    // of the tile and of the group chunk; rows outside them get scale 2^0
+    // (their products are never stored).
+    const int li = loader_index(warp);
     const int nsb = K / 32;
     const uint8_t* swb = p.sw;
     int it = 0;
@@ -278,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit x = unit_of(s, p.E, u);
       for (int kt = 0; kt < nk; ++kt, ++it) {
         const int st = it % kStages, use = it / kStages;
+        if (st != li) continue;
         if (it >= kStages && !(ok = mbar_wait(&s.empty[st], (use - 1) & 1, err, abort))) break;
         const int b0 = ((tail && kt == nk - 1) ? K - kBK : kt * kBK) / 32;  // even: K % 64 == 0
         uint32_t wv[4], av[4];
