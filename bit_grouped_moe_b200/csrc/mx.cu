@@ -21,15 +21,18 @@
 //    bytes of padding, so 128 codes fill one 128-byte row); the e4m3
 //    activations are plain bytes.  The SM decodes nothing: no lookup table
 //    and no bf16 copy of a weight exist anywhere.
-//  * Block scales: a loader warp copies, per 128-k stage, the e8m0 scales of
+//  * Block scales: per 128-k stage a loader warp copies the e8m0 scales of
 //    the tile's 128 weight rows and of the group's rows into shared memory
 //    in the layout tcgen05.cp reads (row m at byte 16*(m%32) + 4*(m/32), one
-//    byte per 32-k block); the MMA thread copies both to TMEM with
-//    tcgen05.cp.32x128b.warpx4 just before the stage's four K=32 MMAs, whose
-//    scale-factor ids select the byte of the block.
+//    byte per 32-k block), moves both to the stage's own TMEM columns with
+//    tcgen05.cp.32x128b.warpx4 and commits the copies to the stage's full
+//    barrier; the four K=32 MMAs of the stage select the byte of their block
+//    with their scale-factor ids.  The MMA thread only waits, issues four
+//    MMAs and commits: it is the one serial thread of the pipeline.
 //  * K % 128 == 64 (e.g. 2880): the last stage reads [K-128, K) and issues
 //    only its upper two K=32 steps, so no box reads past the end of a row.
-//  * Warp roles (12 warps): 0 = TMA producer, 1 = TMEM owner + MMA issuer,
+//  * Warp roles (13 warps): 0 and 12 = TMA producers (alternate stages: one
+//    issuing thread alone caps the stream), 1 = TMEM owner + MMA issuer,
 //    4..7 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31, i.e. weight
 //    rows), 2, 3 and 8..11 = scale loaders, one per ring slot, so the global
 //    loads of six stages are in flight at once.  Two TMEM accumulators let
@@ -95,7 +98,8 @@ constexpr int kBK = 128;  // k per stage
 constexpr int kStages = 6;
 constexpr int kSmallBox = 32;  // activation rows per TMA box for groups of <= 32 rows
 constexpr int kEpiWarp0 = 4;
-constexpr int kThreads = 12 * 32;
+constexpr int kProd2 = 12;  // second TMA producer warp
+constexpr int kThreads = 13 * 32;
 // scale-loader index of a warp (its ring slot), or -1
 __device__ __forceinline__ int loader_index(int warp) {
   return warp == 2 || warp == 3 ? warp - 2 : (warp >= 8 && warp < 8 + kStages - 2 ? warp - 6 : -1);
@@ -104,9 +108,8 @@ constexpr int kWStageBytes = kBW * kBK;    // padded e2m1 in shared memory: one 
 constexpr int kWStageTx = kBW * kBK / 2;   // bytes the TMA reads: two codes per byte
 constexpr int kAStageBytes = kBT * kBK;    // e4m3
 constexpr int kTmemCols = 512;
-constexpr int kSfwCol = 2 * kBT;           // 4 columns of weight scales
-constexpr int kSfaCol = kSfwCol + 4;       // 4 columns of activation scales
-static_assert(kSfaCol + 4 <= kTmemCols, "TMEM budget");
+constexpr int kSfCol0 = 2 * kBT;           // per stage: 4 columns of weight scales, then 4 of activation scales
+static_assert(kSfCol0 + 8 * kStages <= kTmemCols, "TMEM budget");
 static_assert(kStages == 6, "one scale-loader warp per ring slot: warps 2, 3, 8..11");
 
 struct MxSmem {
@@ -117,7 +120,8 @@ struct MxSmem {
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
-  uint64_t full[kStages], sfull[kStages], empty[kStages];
+  uint64_t full[kStages], empty[kStages];  // full: TMA bytes + the producer's arrival + the scale copies' commit
+  uint64_t ldone[kStages];                 // abort path only: a loader's scale copies have retired
   uint64_t accf[2], acce[2];
   uint64_t mdone;  // abort path only: every issued MMA has retired
   uint32_t tmem_base;
@@ -138,6 +142,12 @@ struct MxArgs {
 struct Unit {
   int e, j, row0, rows;
 };
+
+// Partial accumulators per unit: the K=32 steps of a unit of at most 32 (64)
+// rows rotate over 4 (2) accumulators of 32 (64) columns, so consecutive
+// block-scaled MMAs do not wait for each other; the epilogue adds them in a
+// fixed order.
+__device__ __forceinline__ int acc_split(int rows) { return rows <= 32 ? 4 : (rows <= 64 ? 2 : 1); }
 
 __device__ __forceinline__ Unit unit_of(const MxSmem& s, int E, int u) {
   Unit x;
@@ -220,9 +230,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.sfull[i], 1);
+      mbar_init(&s.full[i], 2);
       mbar_init(&s.empty[i], 1);
+      mbar_init(&s.ldone[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.accf[i], 1);
@@ -247,8 +257,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == kProd2) {
+    // ------------------------------------------------------------ TMA producers
+    const int pi = warp == 0 ? 0 : 1;
     if (lane == 0) {
       int it = 0;
       bool ok = true;
@@ -257,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool big = x.rows > kSmallBox;
         const int wrow = x.e * p.N + x.j * kBW;
         for (int kt = 0; kt < nk; ++kt, ++it) {
+          if ((it & 1) != pi) continue;
           const int st = it % kStages, use = it / kStages;
           if (it >= kStages && !(ok = mbar_wait(&s.empty[st], (use - 1) & 1, err, abort))) break;
           const bool last_tail = tail && kt == nk - 1;
@@ -270,7 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok)  // drain loads still in flight before shared memory goes away
-        for (int i = max(0, it - kStages); i < it; ++i) mbar_drain(&s.full[i % kStages], (i / kStages) & 1);
+        for (int i = max(0, it - kStages); i < it; ++i)
+          if ((i & 1) == pi) mbar_drain(&s.full[i % kStages], (i / kStages) & 1);
     }
   } else if (loader_index(warp) >= 0) {
     // ------------------------------------------------------------ scale loaders
@@ -301,15 +314,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         sts_u128(smem_u32(&s.sfa[st][lane * 4]), av[0], av[1], av[2], av[3]);
         fence_proxy_async_smem();  // the tensor core reads these through the async proxy
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s.sfull[st]);
+        if (lane == 0) {
+          const uint32_t col = tmem + (uint32_t)(kSfCol0 + 8 * st);
+          tc_copy_scales(col, sdesc_scales(smem_u32(s.sfw[st])));
+          tc_copy_scales(col + 4, sdesc_scales(smem_u32(s.sfa[st])));
+          tc_commit(&s.full[st]);
+        }
       }
+    }
+    if (!ok && lane == 0) {  // abort: the copies already issued retire before TMEM is released
+      tc_commit(&s.ldone[li]);
+      mbar_drain(&s.ldone[li], 0);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int it = 0, uc = 0;
-      bool ok = true;
-      const uint32_t t_sfw = tmem + (uint32_t)kSfwCol, t_sfa = tmem + (uint32_t)kSfaCol;
+      bool ok = true, ready = false;  // ready: the full barrier of stage `it` was seen complete in advance
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
         const Unit x = unit_of(s, p.E, u);
         const int ab = uc & 1;
@@ -317,24 +338,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t n_mma = (uint32_t)((x.rows + 15) & ~15);
         const uint32_t d_tmem = tmem + (uint32_t)(ab * kBT);
+        const int nsplit = acc_split(x.rows);
+        const uint32_t sub_w = (uint32_t)(kBT / nsplit);
         for (int kt = 0; kt < nk; ++kt, ++it) {
           const int st = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-          const bool rf = mbar_try_wait(&s.full[st], ph);
-          const bool rs = mbar_try_wait(&s.sfull[st], ph);
-          if (!(rf && rs)) {
-            if (!(ok = mbar_wait(&s.full[st], ph, err, abort))) break;
-            if (!(ok = mbar_wait(&s.sfull[st], ph, err, abort))) break;
-          }
+          if (!ready && !(ok = mbar_wait(&s.full[st], ph, err, abort))) break;
           tc_fence_after();
-          tc_copy_scales(t_sfw, sdesc_scales(smem_u32(s.sfw[st])));
-          tc_copy_scales(t_sfa, sdesc_scales(smem_u32(s.sfa[st])));
+          // test the next stage's barrier now: its latency overlaps this stage's issue
+          ready = mbar_try_wait(&s.full[(it + 1) % kStages], (uint32_t)((it + 1) / kStages) & 1u);
+          const uint32_t t_sfw = tmem + (uint32_t)(kSfCol0 + 8 * st), t_sfa = t_sfw + 4u;
           const uint32_t w_addr = smem_u32(s.w[st]), a_addr = smem_u32(s.a[st]);
           const int j0 = (tail && kt == nk - 1) ? 2 : 0;
-          for (int j = j0; j < kBK / 32; ++j)
-            tc_mma_w4a8(d_tmem, sdesc_k_sw128(w_addr + 32 * j), sdesc_k_sw128(a_addr + 32 * j),
-                        idesc_w4a8(n_mma, (uint32_t)j), t_sfw | ((uint32_t)j << 30), t_sfa | ((uint32_t)j << 30),
-                        kt != 0 || j > j0);
+          for (int j = j0; j < kBK / 32; ++j) {
+            const int q = kt * (kBK / 32) + j;  // K=32 step of the unit (every unit has at least 4)
+            tc_mma_w4a8(d_tmem + (uint32_t)(q % nsplit) * sub_w, sdesc_k_sw128(w_addr + 32 * j),
+                        sdesc_k_sw128(a_addr + 32 * j), idesc_w4a8(n_mma, (uint32_t)j), t_sfw | ((uint32_t)j << 30),
+                        t_sfa | ((uint32_t)j << 30), q >= nsplit);
+          }
           tc_commit(&s.empty[st]);
         }
         if (!ok) break;
@@ -346,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_drain(&s.mdone, 0);
       }
     }
-  } else if (warp >= kEpiWarp0) {
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
@@ -358,10 +379,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int n = x.j * kBW + q * 32 + lane;
       __nv_bfloat16* ycol = p.y + (size_t)x.row0 * p.N + n;
+      const int nsplit = acc_split(x.rows);
       for (int c = 0; c * 32 < x.rows; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBT + c * 32), v);
         tmem_wait_ld();
+        for (int j = 1; j < nsplit; ++j) {  // partial accumulators, summed in a fixed order
+          uint32_t w2[32];
+          tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBT + j * (kBT / nsplit) + c * 32), w2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w2[i]));
+        }
         const int lim = min(32, x.rows - c * 32);
         if (n < p.N) {
 #pragma unroll
