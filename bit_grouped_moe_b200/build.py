@@ -13,7 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgnf4.so")
-SOURCES = ["api.cu", "gemm_tc.cu", "gemv.cu", "dgrad.cu", "mx.cu", "route.cu", "route_static.cu", "combine.cu", "dequant.cu"]
+SOURCES = ["api.cu", "gemm_tc.cu", "gemv.cu", "dgrad.cu", "mx.cu", "route.cu", "route_static.cu", "combine.cu", "dequant.cu", "selftest.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 
 NVCC_FLAGS = [

@@ -370,6 +370,16 @@ gnf4_status gnf4_device_errors(uint32_t* flags, int clear) {
   return GNF4_OK;
 }
 
+gnf4_status gnf4_selftest_bounded_wait(unsigned long long limit_cycles, void* stream) {
+  if (limit_cycles < 1 || limit_cycles > (1ull << 32))
+    return fail(GNF4_ERR_INVALID_ARG, "limit_cycles=%llu outside [1, 2^32]", limit_cycles);
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  cudaError_t e = launch_bounded_wait_probe(d->err, (long long)limit_cycles, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bounded-wait probe launch");
+  return GNF4_OK;
+}
+
 size_t gnf4_route_workspace_bytes(int T, int k, int E) {
   if (T < 0 || k < 1 || E < 1) return 0;
   return route_workspace_bytes(T, k, E);

@@ -232,21 +232,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0u;
 }
 
-// Waits for the phase with the given parity to complete.  Gives up after the
-// spin limit, or as soon as another role of the CTA has raised *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
-                                          volatile int* abort) {
+// Waits for the phase with the given parity to complete.  Gives up after
+// `limit` cycles (raising GNF4_DEVERR_TIMEOUT and *abort), or as soon as
+// another role of the CTA has raised *abort.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned* err, volatile int* abort,
+                                              long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kSpinLimitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(err, GNF4_DEVERR_TIMEOUT);
       *abort = 1;
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
+                                          volatile int* abort) {
+  return mbar_wait_for(bar, parity, err, abort, kSpinLimitCycles);
 }
 
 // Short bounded wait used while draining after an abort (no error raised).

@@ -100,6 +100,9 @@ constexpr int kMaxRouterTopK = 32;
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* flat_to_sorted, const float* weights, int T,
                            int k, int N, __nv_bfloat16* out, int num_sms, cudaStream_t stream);
 
+// selftest.cu: one bounded wait on a barrier nothing arrives on
+cudaError_t launch_bounded_wait_probe(unsigned* err, long long limit_cycles, cudaStream_t stream);
+
 // api.cu: sets the text gnf4_last_error() returns on this thread
 void set_last_error(const char* msg);
 

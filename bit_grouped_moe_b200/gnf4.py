@@ -47,13 +47,14 @@ _GROUPED = ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_ge
             "gnf4_grouped_gemv_mxfp4_swiglu", "gnf4_grouped_dgrad_nf4", "gnf4_grouped_dgrad_mxfp4")
 for _name in _GROUPED:
     getattr(_lib, _name).argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+_lib.gnf4_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, _P]
 _lib.gnf4_quantize_mxfp8.argtypes = [_P, _I, _I, _P, _P, _P]
 _lib.gnf4_grouped_gemm_w4a8.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
 _lib.gnf4_dequant_nf4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 _lib.gnf4_dequant_mxfp4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", "gnf4_route_topk_permute",
-              *_GROUPED, "gnf4_combine", "gnf4_quantize_mxfp8", "gnf4_grouped_gemm_w4a8",
+              *_GROUPED, "gnf4_combine", "gnf4_quantize_mxfp8", "gnf4_grouped_gemm_w4a8", "gnf4_selftest_bounded_wait",
               "gnf4_dequant_nf4_f32", "gnf4_dequant_mxfp4_f32"):
     getattr(_lib, _name).restype = _I
 
@@ -272,3 +273,8 @@ def grouped_gemm_w4a8(a_codes, a_scales, w, w_scales, y, offsets=None, counts=No
     M = a_codes.shape[0]
     _check(_lib.gnf4_grouped_gemm_w4a8(_ptr(a_codes), _ptr(a_scales), _ptr(w), _ptr(w_scales), _ptr(offsets),
                                        _ptr(counts), E, N, 2 * K2, M, _ptr(y), _stream(stream)))
+
+
+def selftest_bounded_wait(limit_cycles: int, stream=None) -> None:
+    """One bounded pipeline wait on a barrier nothing arrives on (gives up after limit_cycles)."""
+    _check(_lib.gnf4_selftest_bounded_wait(int(limit_cycles), _stream(stream)))

@@ -85,6 +85,13 @@ const char *gnf4_version(void);
  * the hot path. */
 gnf4_status gnf4_device_errors(uint32_t *flags, int clear);
 
+/* Failure-detection self-test: enqueues one kernel whose single thread runs
+ * the pipelines' bounded mbarrier wait on a barrier that nothing ever
+ * arrives on, giving up after limit_cycles SM clock cycles (1 .. 2^32).  On
+ * return of the kernel the device error word holds GNF4_DEVERR_TIMEOUT and
+ * the context stays usable.  No fault, trap or unbounded spin is involved. */
+gnf4_status gnf4_selftest_bounded_wait(unsigned long long limit_cycles, void *stream);
+
 /* ------------------------------------------------------------------ */
 /* Routing: sort (token, slot) pairs into per-expert row groups         */
 /* ------------------------------------------------------------------ */

@@ -235,6 +235,31 @@ def test_bad_offsets_flagged_not_computed(g, kind):
     assert torch.all(y == 2.0)
 
 
+def test_bounded_wait_times_out_and_the_context_stays_usable(g):
+    """The pipelines' bounded wait, run on a barrier nothing arrives on with a
+    ~0.5 ms limit, raises GNF4_DEVERR_TIMEOUT and returns; the next grouped
+    GEMM on the same context is still correct."""
+    g.device_errors(clear=True)
+    g.selftest_bounded_wait(1 << 20)
+    torch.cuda.synchronize()
+    assert g.device_errors(clear=True) == g.DEVERR_TIMEOUT
+    E, N, K = 2, 64, 128
+    offsets = np.array([0, 3, 5], np.int32)
+    w, sc = _make_stack("mxfp4", E, N, K, seed=430)
+    a = inputs.bf16_normal(inputs.rng(431), (5, K))
+    y = torch.empty((5, N), dtype=torch.bfloat16, device="cuda")
+    _gpu_call(g, "mxfp4", "gemm", to_dev_bf16(a), to_dev(w), to_dev(sc), y, off_d=to_dev(offsets))
+    torch.cuda.synchronize()
+    assert g.device_errors() == 0
+    assert_within_tolerance(bf16_to_f64(y), _oracle_gemm("mxfp4", a, w, sc, offsets), "after the timeout")
+
+
+def test_bounded_wait_rejects_a_zero_limit(g):
+    with pytest.raises(g.Gnf4Error) as ei:
+        g.selftest_bounded_wait(0)
+    assert ei.value.status == g.ERR_INVALID_ARG
+
+
 # ------------------------------------------------------------------ combine
 
 
