@@ -238,6 +238,36 @@ gnf4_status grouped_gemv(int fmt, bool swiglu, const void* a, const uint8_t* w, 
   return GNF4_OK;
 }
 
+// GEMV with the top-k combine in its epilogue.
+gnf4_status grouped_gemv_combine(int fmt, const void* a, const uint8_t* w, const void* scales,
+                                 const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M, void* y,
+                                 const int32_t* sorted_to_flat, const int32_t* flat_to_sorted, const float* weights,
+                                 int T, int k, void* out, int32_t* counters, void* stream) {
+  GNF4_TRY(check_grouped(fmt, a, w, scales, offsets, counts, E, N, K, M, y));
+  if (T < 0 || k < 1) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T=%d / k=%d invalid", T, k);
+  if ((long long)T * k >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T*k too large");
+  if (T == 0) return GNF4_OK;
+  GNF4_TRY(check_ptr(offsets, "offsets", 4, false));
+  GNF4_TRY(check_ptr(counts, "counts", 4, false));
+  GNF4_TRY(check_ptr(flat_to_sorted, "flat_to_sorted", 4));
+  GNF4_TRY(check_ptr(weights, "weights", 4));
+  GNF4_TRY(check_ptr(out, "out", 16));
+  GNF4_TRY(check_ptr(counters, "counters", 4));
+  if (M > 0) GNF4_TRY(check_ptr(sorted_to_flat, "sorted_to_flat", 4));
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  GroupedArgs p{static_cast<const __nv_bfloat16*>(a), w, scales, offsets, counts,
+                static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
+  CombineArgs c{sorted_to_flat, flat_to_sorted, weights, static_cast<__nv_bfloat16*>(out), counters, T, k};
+  const long long hit = E < M ? E : M;
+  const long long per = (N + gemv_rows_per_block() - 1) / gemv_rows_per_block();
+  // at least one CTA, so tokens without a valid pair still get their zero row
+  const int grid = M > 0 ? gemv_grid(hit * per, d->num_sms) : 1;
+  cudaError_t e = launch_gemv(fmt, false, p, grid, as_stream(stream), &c);
+  if (e != cudaSuccess) return cuda_fail(e, "grouped GEMV + combine launch");
+  return GNF4_OK;
+}
+
 // dY [M, N] bf16 and the [E, N, K/2] stack -> dX [M, K] bf16.
 gnf4_status grouped_dgrad(int fmt, const void* dy, const uint8_t* w, const void* scales, const int32_t* offsets,
                           const int32_t* counts, int E, int N, int K, int M, void* dx, void* stream) {
@@ -539,6 +569,29 @@ gnf4_status gnf4_grouped_gemm_nf4_swiglu(const void* a, const uint8_t* w_gate_up
                                          void* h, void* stream) {
   GNF4_TRY(check_swiglu_width(I));
   return grouped_gemm(0, true, a, w_gate_up, absmax, offsets, counts, E, 2 * I, K, M, h, stream);
+}
+
+size_t gnf4_combine_counters_bytes(int T, int N) {
+  if (T < 0 || N < 1) return 0;
+  return gemv_combine_counter_bytes(T, N);
+}
+
+gnf4_status gnf4_grouped_gemv_nf4_combine(const void* a, const uint8_t* w, const float* absmax,
+                                          const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M,
+                                          void* y, const int32_t* sorted_to_flat, const int32_t* flat_to_sorted,
+                                          const float* weights, int T, int k, void* out, int32_t* counters,
+                                          void* stream) {
+  return grouped_gemv_combine(0, a, w, absmax, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
+                              weights, T, k, out, counters, stream);
+}
+
+gnf4_status gnf4_grouped_gemv_mxfp4_combine(const void* a, const uint8_t* w, const uint8_t* scales,
+                                            const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M,
+                                            void* y, const int32_t* sorted_to_flat, const int32_t* flat_to_sorted,
+                                            const float* weights, int T, int k, void* out, int32_t* counters,
+                                            void* stream) {
+  return grouped_gemv_combine(1, a, w, scales, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
+                              weights, T, k, out, counters, stream);
 }
 
 gnf4_status gnf4_quantize_mxfp8(const void* x, int M, int K, uint8_t* codes, uint8_t* scales, void* stream) {

@@ -18,6 +18,14 @@
 // feeds the pairs to m16n8k16 warp MMAs.  The MMA does the k reduction that
 // a CUDA-core GEMV would do with shuffles.
 //
+// Fused combine (CMB): after a half has stored its unit's rows, each row
+// counts its (token, 64-column block) in; the half that completes a token's
+// last valid pair computes that token's 64 output columns with the same fp32
+// fmaf sequence as the separate combine (pairs in slot order), so the fused
+// output equals the unfused one bit for bit, and resets the counter for the
+// next call.  Stores are published with a fence before the count; the
+// completing half fences again before it reads the other rows through L2.
+//
 // Latency hiding: a warp's items form one stream across unit boundaries, and
 // the loads of the next item are issued tile by tile while the current item
 // is decoded (each tile's registers are refilled as soon as they have been
@@ -55,6 +63,7 @@ constexpr int kSmemBytes = 0x20000;        // dynamic shared memory per CTA
 // Everything but the pair table; lives below kLutWindow.
 struct GemvLow {
   float red[2][kSplit][4][32][4];  // 32 KB: partial sums per half and K-split
+  int done[2][kMaxTokens];         // fused combine: tokens a half's unit completed (-1: none)
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
@@ -144,8 +153,18 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t raw) {
   return FMT == 0 ? cvt_bf16x2_dup(__uint_as_float(raw)) : e8m0_to_bf16x2(raw);
 }
 
-template <int FMT, int MODE>
-__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
+// Sum over the valid pairs of token t (sorted row inside [0, nvalid)).
+__device__ __forceinline__ int valid_pairs(const CombineArgs& c, int t, int nvalid) {
+  int need = 0;
+  for (int j = 0; j < c.k; ++j) {
+    const int r = __ldg(c.f2s + (size_t)t * c.k + j);
+    need += (r >= 0 && r < nvalid) ? 1 : 0;
+  }
+  return need;
+}
+
+template <int FMT, int MODE, bool CMB>
+__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p, CombineArgs cmb) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   GemvLow& s = *reinterpret_cast<GemvLow*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -169,6 +188,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
   const int nblk = MODE == kModeSwiglu ? (p.N / 2) / (kRows / 2) : (p.N + kRows - 1) / kRows;
   block_exclusive_scan(p.E, s.upre, s.scratch, [&](int e) { return (s.off[e + 1] > s.off[e]) ? nblk : 0; });
   const int U = s.upre[p.E];
+  if (CMB && blockIdx.x == 0) {  // tokens without a valid pair get a zero row (no unit ever completes them)
+    const int nvalid = s.off[p.E];
+    for (int t = tid; t < cmb.T; t += kThreads)
+      if (valid_pairs(cmb, t, nvalid) == 0)
+        for (int n = 0; n < p.N; ++n) cmb.out[(size_t)t * p.N + n] = __float2bfloat16_rn(0.f);
+  }
   if (2 * (int)blockIdx.x >= U) return;  // uniform over the CTA
 
   const int K = p.K;
@@ -274,6 +299,41 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p) {
           const int tok = 2 * (l & 3) + (j & 1);
           if (n < p.N && tok < rows) p.y[(size_t)(r0 + tok) * p.N + n] = __float2bfloat16_rn(v);
         }
+        if (CMB) {
+          __threadfence();  // this thread's rows are visible device-wide before they are counted
+          half_barrier(h);
+          const int nvalid = s.off[p.E];
+          if (ht < kMaxTokens) {
+            int t = -1;
+            if (ht < rows) {
+              const int f = __ldg(cmb.s2f + r0 + ht);
+              if (f >= 0 && f < cmb.T * cmb.k) {
+                const int tk = f / cmb.k;
+                int* ctr = cmb.cnt + (size_t)tk * nblk + jb;
+                if (atomicAdd(ctr, 1) == valid_pairs(cmb, tk, nvalid) - 1) {
+                  t = tk;
+                  *ctr = 0;  // every pair of this block is in: ready for the next call
+                }
+              }
+            }
+            s.done[h][ht] = t;
+          }
+          half_barrier(h);
+          __threadfence();  // the other units' rows of these tokens are visible from here on
+          for (int o = ht; o < kMaxTokens * kRows; o += kThreads / 2) {
+            const int t = s.done[h][o / kRows];
+            const int n = jb * kRows + (o % kRows);
+            if (t < 0 || n >= p.N) continue;
+            float acc = 0.f;
+            for (int j = 0; j < cmb.k; ++j) {
+              const int r = __ldg(cmb.f2s + (size_t)t * cmb.k + j);
+              if (r < 0 || r >= nvalid) continue;  // dropped pair
+              const unsigned short yb = __ldcg(reinterpret_cast<const unsigned short*>(p.y) + (size_t)r * p.N + n);
+              acc = fmaf(__ldg(cmb.w + (size_t)t * cmb.k + j), __uint_as_float((uint32_t)yb << 16), acc);
+            }
+            cmb.out[(size_t)t * p.N + n] = __float2bfloat16_rn(acc);
+          }
+        }
       }
     }
     half_barrier(h);
@@ -287,30 +347,39 @@ int gemv_grid(long long units, int num_sms) {
   return (int)(ctas < num_sms ? ctas : num_sms);
 }
 
-template <int FMT, int MODE>
-static cudaError_t launch_gemv_t(const GroupedArgs& p, int grid, cudaStream_t stream) {
+template <int FMT, int MODE, bool CMB>
+static cudaError_t launch_gemv_t(const GroupedArgs& p, const CombineArgs& c, int grid, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, MODE, CMB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  return launch_pdl(gemv_kernel<FMT, MODE>, dim3(grid), dim3(kThreads), (size_t)kSmemBytes, stream, p);
+  return launch_pdl(gemv_kernel<FMT, MODE, CMB>, dim3(grid), dim3(kThreads), (size_t)kSmemBytes, stream, p, c);
 }
 
 template <int FMT>
-static cudaError_t launch_gemv_f(bool swiglu, const GroupedArgs& p, int grid, cudaStream_t stream) {
-  if (swiglu) return launch_gemv_t<FMT, kModeSwiglu>(p, grid, stream);
-  return p.N % kRows == 0 ? launch_gemv_t<FMT, kModeFull>(p, grid, stream)
-                          : launch_gemv_t<FMT, kModeClamp>(p, grid, stream);
+static cudaError_t launch_gemv_f(bool swiglu, const GroupedArgs& p, const CombineArgs* c, int grid,
+                                 cudaStream_t stream) {
+  const CombineArgs none{};
+  if (swiglu) return launch_gemv_t<FMT, kModeSwiglu, false>(p, none, grid, stream);
+  if (c != nullptr)
+    return p.N % kRows == 0 ? launch_gemv_t<FMT, kModeFull, true>(p, *c, grid, stream)
+                            : launch_gemv_t<FMT, kModeClamp, true>(p, *c, grid, stream);
+  return p.N % kRows == 0 ? launch_gemv_t<FMT, kModeFull, false>(p, none, grid, stream)
+                          : launch_gemv_t<FMT, kModeClamp, false>(p, none, grid, stream);
 }
 
-cudaError_t launch_gemv(int fmt, bool swiglu, const GroupedArgs& p, int grid, cudaStream_t stream) {
-  return fmt == 0 ? launch_gemv_f<0>(swiglu, p, grid, stream) : launch_gemv_f<1>(swiglu, p, grid, stream);
+cudaError_t launch_gemv(int fmt, bool swiglu, const GroupedArgs& p, int grid, cudaStream_t stream,
+                        const CombineArgs* combine) {
+  return fmt == 0 ? launch_gemv_f<0>(swiglu, p, combine, grid, stream)
+                  : launch_gemv_f<1>(swiglu, p, combine, grid, stream);
 }
+
+size_t gemv_combine_counter_bytes(int T, int N) { return (size_t)T * (size_t)((N + kRows - 1) / kRows) * 4; }
 
 int gemv_rows_per_block() { return kRows; }
 int gemv_swiglu_cols_per_block() { return kRows / 2; }

@@ -52,9 +52,22 @@ int gemm_tc_weight_rows_per_unit();
 cudaError_t launch_gemm_tc(int fmt, bool swiglu, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big,
                            const CUtensorMap& tm_w, const GroupedArgs& p, int grid, cudaStream_t stream);
 
+// Fused top-k combine in the GEMV epilogue (device pointers).
+struct CombineArgs {
+  const int* s2f;     // sorted_to_flat [M]
+  const int* f2s;     // flat_to_sorted [T*k]
+  const float* w;     // weights [T, k]
+  __nv_bfloat16* out; // [T, N]
+  int* cnt;           // [T, ceil(N/64)] counters, zero before the call and after it
+  int T, k;
+};
+
 // gemv.cu
 // swiglu: p.w is a gate_up stack [E, N = 2I, K/2] and p.y the [M, I] output h.
-cudaError_t launch_gemv(int fmt, bool swiglu, const GroupedArgs& p, int grid, cudaStream_t stream);
+// combine (not with swiglu): also out[t] = sum_j w[t,j] y[f2s[t*k+j]] in the epilogue.
+cudaError_t launch_gemv(int fmt, bool swiglu, const GroupedArgs& p, int grid, cudaStream_t stream,
+                        const CombineArgs* combine = nullptr);
+size_t gemv_combine_counter_bytes(int T, int N);
 int gemv_rows_per_block();
 int gemv_swiglu_cols_per_block();
 // CTAs for a GEMV launch over `units` (expert, 64-row) units.

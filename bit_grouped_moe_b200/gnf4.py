@@ -47,6 +47,10 @@ _GROUPED = ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_ge
             "gnf4_grouped_gemv_mxfp4_swiglu", "gnf4_grouped_dgrad_nf4", "gnf4_grouped_dgrad_mxfp4")
 for _name in _GROUPED:
     getattr(_lib, _name).argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+_lib.gnf4_combine_counters_bytes.argtypes = [_I, _I]
+_lib.gnf4_combine_counters_bytes.restype = _SZ
+for _name in ("gnf4_grouped_gemv_nf4_combine", "gnf4_grouped_gemv_mxfp4_combine"):
+    getattr(_lib, _name).argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P]
 _lib.gnf4_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, _P]
 _lib.gnf4_quantize_mxfp8.argtypes = [_P, _I, _I, _P, _P, _P]
 _lib.gnf4_grouped_gemm_w4a8.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
@@ -55,6 +59,7 @@ _lib.gnf4_dequant_nf4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 _lib.gnf4_dequant_mxfp4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", "gnf4_route_topk_permute",
               *_GROUPED, "gnf4_combine", "gnf4_quantize_mxfp8", "gnf4_grouped_gemm_w4a8", "gnf4_selftest_bounded_wait",
+              "gnf4_grouped_gemv_nf4_combine", "gnf4_grouped_gemv_mxfp4_combine",
               "gnf4_dequant_nf4_f32", "gnf4_dequant_mxfp4_f32"):
     getattr(_lib, _name).restype = _I
 
@@ -278,3 +283,31 @@ def grouped_gemm_w4a8(a_codes, a_scales, w, w_scales, y, offsets=None, counts=No
 def selftest_bounded_wait(limit_cycles: int, stream=None) -> None:
     """One bounded pipeline wait on a barrier nothing arrives on (gives up after limit_cycles)."""
     _check(_lib.gnf4_selftest_bounded_wait(int(limit_cycles), _stream(stream)))
+
+
+def combine_counters_bytes(T: int, N: int) -> int:
+    return int(_lib.gnf4_combine_counters_bytes(T, N))
+
+
+def _gemv_combine(fn, a, w, scales, y, sorted_to_flat, flat_to_sorted, weights, out, counters, offsets=None,
+                  counts=None, stream=None):
+    E, N, K2 = w.shape
+    M = a.shape[0]
+    T, k = weights.shape
+    _check(fn(_ptr(a), _ptr(w), _ptr(scales), _ptr(offsets), _ptr(counts), E, N, 2 * K2, M, _ptr(y),
+              _ptr(sorted_to_flat), _ptr(flat_to_sorted), _ptr(weights), T, k, _ptr(out), _ptr(counters),
+              _stream(stream)))
+
+
+def grouped_gemv_nf4_combine(a, w, absmax, y, sorted_to_flat, flat_to_sorted, weights, out, counters,
+                             offsets=None, counts=None, stream=None):
+    """Decode GEMV (y) with the top-k combine of y into out [T, N] in the same launch.
+    counters: zeroed int32 device buffer of combine_counters_bytes(T, N) bytes (left zero)."""
+    _gemv_combine(_lib.gnf4_grouped_gemv_nf4_combine, a, w, absmax, y, sorted_to_flat, flat_to_sorted, weights,
+                  out, counters, offsets, counts, stream)
+
+
+def grouped_gemv_mxfp4_combine(a, w, scales, y, sorted_to_flat, flat_to_sorted, weights, out, counters,
+                               offsets=None, counts=None, stream=None):
+    _gemv_combine(_lib.gnf4_grouped_gemv_mxfp4_combine, a, w, scales, y, sorted_to_flat, flat_to_sorted, weights,
+                  out, counters, offsets, counts, stream)

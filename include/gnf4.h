@@ -270,6 +270,42 @@ gnf4_status gnf4_grouped_gemv_mxfp4_swiglu(const void *a, const uint8_t *w_gate_
                                            void *h, void *stream);
 
 /* ------------------------------------------------------------------ */
+/* Decode GEMV with the top-k combine in its epilogue                  */
+/* ------------------------------------------------------------------ */
+
+/* The grouped GEMV of the second projection followed, in the same launch,
+ * by the top-k combine (grouped-nf4-gemm index.json, problems_solved[5]:
+ * "top-k combine" among the decode tail folded into fewer launches):
+ *     y[r, n]   = sum_k a[r, k] * W_e[n, k]            (as gnf4_grouped_gemv_*)
+ *     out[t, n] = sum_{j<k} weights[t, j] * y[flat_to_sorted[t*k + j], n]
+ * The combine is the same fp32 fmaf sequence as gnf4_combine (slots in
+ * order j = 0..k-1, one bf16 rounding), so out equals the unfused
+ * GEMV + combine bit for bit.  Pairs whose sorted row is -1 or not below
+ * the number of routed rows (offsets[E]) contribute nothing; a token with no
+ * such pair gets a zero row.
+ *   a, w, scales, offsets, counts, E, N, K, M, y: as gnf4_grouped_gemv_*
+ *     (y is still written: the combine reads it);
+ *   sorted_to_flat int32 [M] and flat_to_sorted int32 [T*k]: as written by
+ *     gnf4_route_permute; weights fp32 [T, k]; out bf16 [T, N];
+ *   counters: int32 device memory of gnf4_combine_counters_bytes(T, N)
+ *     bytes, zero-filled once by the caller before its first use; every call
+ *     that ends without a device error leaves it zero again (so the call is
+ *     safe to capture in a CUDA graph).  After a call that set a device
+ *     error, zero it again.  Calls that overlap on the GPU need separate
+ *     counters. */
+size_t gnf4_combine_counters_bytes(int T, int N);
+gnf4_status gnf4_grouped_gemv_nf4_combine(const void *a, const uint8_t *w, const float *absmax,
+                                          const int32_t *offsets, const int32_t *counts, int E, int N, int K, int M,
+                                          void *y, const int32_t *sorted_to_flat, const int32_t *flat_to_sorted,
+                                          const float *weights, int T, int k, void *out, int32_t *counters,
+                                          void *stream);
+gnf4_status gnf4_grouped_gemv_mxfp4_combine(const void *a, const uint8_t *w, const uint8_t *scales,
+                                            const int32_t *offsets, const int32_t *counts, int E, int N, int K,
+                                            int M, void *y, const int32_t *sorted_to_flat,
+                                            const int32_t *flat_to_sorted, const float *weights, int T, int k,
+                                            void *out, int32_t *counters, void *stream);
+
+/* ------------------------------------------------------------------ */
 /* Native W4A8 mode: MXFP8 activations x MXFP4 weights                 */
 /* ------------------------------------------------------------------ */
 
