@@ -145,7 +145,8 @@ class Workload:
     """Device-resident inputs of one workload: rotating weight copies larger
     than L2, a set of token batches, and the step's output buffers."""
 
-    def __init__(self, name, device, seed, build_host_copy, swiglu=False, dgrad=False, w4a8=False):
+    def __init__(self, name, device, seed, build_host_copy, swiglu=False, dgrad=False, w4a8=False,
+                 fused_combine=False):
         import torch
 
         from bit_grouped_moe_b200 import gnf4
@@ -218,6 +219,12 @@ class Workload:
             self.sa1 = torch.empty(M, self.p1.K // 32, dtype=torch.uint8, device=device)
             self.qa2 = torch.empty(M, self.p2.K, dtype=torch.uint8, device=device)
             self.sa2 = torch.empty(M, self.p2.K // 32, dtype=torch.uint8, device=device)
+        # decode: the second projection's GEMV carries the top-k combine in its epilogue
+        self.fused_combine = fused_combine and self.decode and not dgrad and not w4a8
+        if self.fused_combine:
+            self.fn2c = f.grouped_gemv_nf4_combine if wl.fmt == "nf4" else f.grouped_gemv_mxfp4_combine
+            self.cnt = torch.zeros(max(f.combine_counters_bytes(self.T, self.p2.N) // 4, 1), dtype=torch.int32,
+                                   device=device)
         # optional fused gate_up + SwiGLU first projection: h [M, N1/2] feeds the second
         self.swiglu = swiglu
         if swiglu:
@@ -285,10 +292,11 @@ class Workload:
             g.quantize_mxfp8(self.xs, self.qa1, self.sa1)
         if ev is not None:
             ev[0].record()
-        self.project(w1, s1, w2, s2, ev)
-        g.combine(self.y2, self.f2s, wts, self.out)
+        self.project(w1, s1, w2, s2, ev, wts=wts)
+        if not self.fused_combine:
+            g.combine(self.y2, self.f2s, wts, self.out)
 
-    def project(self, w1, s1, w2, s2, ev=None, quantize_first=False):
+    def project(self, w1, s1, w2, s2, ev=None, quantize_first=False, wts=None):
         if self.w4a8:
             g = self.g
             if quantize_first:
@@ -305,12 +313,17 @@ class Workload:
             self.fn(self.xs, w1, s1, self.y1, offsets=self.off)
         if ev is not None:
             ev[1].record()
-        self.fn(self.hs if self.swiglu else self.h, w2, s2, self.y2, offsets=self.off)
+        a2 = self.hs if self.swiglu else self.h
+        if self.fused_combine:
+            self.fn2c(a2, w2, s2, self.y2, self.s2f, self.f2s, wts, self.out, self.cnt, offsets=self.off)
+        else:
+            self.fn(a2, w2, s2, self.y2, offsets=self.off)
 
     def launches_per_step(self):
         # route (one launch for at most 256 pairs, else hist + scan + scatter + gather) + 2 projections + combine
         route = 1 if 0 < self.M <= 256 else 4
-        return route + 2 + (0 if self.dgrad else 1) + (2 if self.w4a8 else 0)
+        combine = 0 if (self.dgrad or self.fused_combine) else 1
+        return route + 2 + combine + (2 if self.w4a8 else 0)
 
 
 # ------------------------------------------------------------------ distributed
@@ -425,6 +438,9 @@ def main():
                     help=f"decode: also time the steps replayed from one CUDA graph of {20} steps")
     ap.add_argument("--w4a8", action="store_true",
                     help="MXFP4 workloads: native W4A8 mode (MXFP8 activations, block-scaled tcgen05 GEMM)")
+    ap.add_argument("--fused-combine", action="store_true",
+                    help="decode: run the top-k combine in the second GEMV's epilogue instead of as its own launch "
+                         "(measured slower on B200: the epilogue's round trips extend every unit)")
     ap.add_argument("--swiglu", action="store_true",
                     help="first projection = fused gate_up + SwiGLU (gate rows first); the second reads its output")
     ap.add_argument("--weight-copies", type=int, default=N_WEIGHT_COPIES,
@@ -471,7 +487,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     dev = f"cuda:{local}"
     torch.cuda.set_device(local)
     wl = Workload(args.workload, dev, seed=1234 + rank, build_host_copy=(rank == 0 and world == 1),
-                  swiglu=args.swiglu, dgrad=args.dgrad, w4a8=args.w4a8)
+                  swiglu=args.swiglu, dgrad=args.dgrad, w4a8=args.w4a8, fused_combine=args.fused_combine)
     decode = wl.decode
     wl.h_host = wl.h.cpu().view(torch.int16).numpy().view(np.uint16)
     stream = torch.cuda.current_stream()
@@ -533,8 +549,9 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
             wl.dfn(wl.dy2, w2, s2, wl.dh, offsets=wl.off)
             wl.dfn(wl.dy1, w1, s1, wl.dx1, offsets=wl.off)
         else:
-            wl.project(w1, s1, w2, s2, quantize_first=True)
-            g.combine(wl.y2, wl.f2s, d_w, wl.out)
+            wl.project(w1, s1, w2, s2, quantize_first=True, wts=d_w)
+            if not wl.fused_combine:
+                g.combine(wl.y2, wl.f2s, d_w, wl.out)
         host_out.copy_(out_dev, non_blocking=True)
 
     for i in range(warmup):
@@ -636,6 +653,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
             "vs_baseline": None, "dtype": "e4m3 x e2m1 (fp32 accumulate)" if wl.w4a8 else "bf16", "data": "synthetic",
             "config": dict(_config(wl.wl, world), **({"first_projection": "fused gate_up + SwiGLU"} if wl.swiglu else {}),
                            **({"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if wl.w4a8 else {}),
+                           **({"combine": "in the second GEMV's epilogue"} if wl.fused_combine else {}),
                            **({"step": "backward: route + dgrad of both projections"} if wl.dgrad else {})),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

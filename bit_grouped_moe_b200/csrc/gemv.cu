@@ -300,7 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p, Combin
           if (n < p.N && tok < rows) p.y[(size_t)(r0 + tok) * p.N + n] = __float2bfloat16_rn(v);
         }
         if (CMB) {
-          __threadfence();  // this thread's rows are visible device-wide before they are counted
+          // The half's stores happen before the barrier; the counting thread's
+          // fence (cumulative) publishes them at GPU scope before its count.
           half_barrier(h);
           const int nvalid = s.off[p.E];
           if (ht < kMaxTokens) {
@@ -310,7 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p, Combin
               if (f >= 0 && f < cmb.T * cmb.k) {
                 const int tk = f / cmb.k;
                 int* ctr = cmb.cnt + (size_t)tk * nblk + jb;
+                __threadfence();
                 if (atomicAdd(ctr, 1) == valid_pairs(cmb, tk, nvalid) - 1) {
+                  __threadfence();  // the other units' rows of tk are visible to this half from here on
                   t = tk;
                   *ctr = 0;  // every pair of this block is in: ready for the next call
                 }
@@ -319,17 +322,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p, Combin
             s.done[h][ht] = t;
           }
           half_barrier(h);
-          __threadfence();  // the other units' rows of these tokens are visible from here on
           for (int o = ht; o < kMaxTokens * kRows; o += kThreads / 2) {
             const int t = s.done[h][o / kRows];
             const int n = jb * kRows + (o % kRows);
             if (t < 0 || n >= p.N) continue;
             float acc = 0.f;
-            for (int j = 0; j < cmb.k; ++j) {
-              const int r = __ldg(cmb.f2s + (size_t)t * cmb.k + j);
-              if (r < 0 || r >= nvalid) continue;  // dropped pair
-              const unsigned short yb = __ldcg(reinterpret_cast<const unsigned short*>(p.y) + (size_t)r * p.N + n);
-              acc = fmaf(__ldg(cmb.w + (size_t)t * cmb.k + j), __uint_as_float((uint32_t)yb << 16), acc);
+            for (int j0 = 0; j0 < cmb.k; j0 += 8) {  // 8 independent row loads, then the fmaf chain in slot order
+              float yv[8], wv[8];
+              bool okv[8];
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj) {
+                const int j = j0 + jj;
+                const int r = j < cmb.k ? __ldg(cmb.f2s + (size_t)t * cmb.k + j) : -1;
+                const bool ok = r >= 0 && r < nvalid;  // else a dropped pair
+                const unsigned short yb =
+                    ok ? __ldcg(reinterpret_cast<const unsigned short*>(p.y) + (size_t)r * p.N + n) : (unsigned short)0;
+                yv[jj] = __uint_as_float((uint32_t)yb << 16);
+                wv[jj] = ok ? __ldg(cmb.w + (size_t)t * cmb.k + j) : 0.f;
+                okv[jj] = ok;
+              }
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj)
+                if (okv[jj]) acc = fmaf(wv[jj], yv[jj], acc);
             }
             cmb.out[(size_t)t * p.N + n] = __float2bfloat16_rn(acc);
           }
