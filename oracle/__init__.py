@@ -64,6 +64,8 @@ def _load():
     lib.orc_quant_mxfp8.argtypes = [P, I64, I64, P, P]
     lib.orc_dequant_mxfp8.argtypes = [P, P, I64, I64, P]
     lib.orc_grouped_gemm_w4a8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P]
+    lib.orc_quant_mxfp8_split.argtypes = [P, I64, I64, P, P, P, P]
+    lib.orc_grouped_gemm_w4a8x2.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, P, I64, P]
     _lib = lib
     return lib
 
@@ -303,4 +305,37 @@ def grouped_gemm_w4a8(codes, a_scales, w, w_scales, offsets, rows=None):
     y = np.empty((rows.shape[0], N), np.float64)
     _load().orc_grouped_gemm_w4a8(_p(codes), _p(a_scales), _p(w), _p(w_scales), _p(offsets), E, N, K, _p(rows),
                                   rows.shape[0], _p(y))
+    return y
+
+
+def quant_mxfp8_split(x_bits: np.ndarray):
+    """Two-term MXFP8 split of bf16 activations: (hi_codes, hi_scales, lo_codes, lo_scales)."""
+    x_bits = _c(x_bits, np.uint16)
+    K = x_bits.shape[-1]
+    if K % 32:
+        raise ValueError("MXFP8 needs K % 32 == 0")
+    rows = x_bits.size // K if K else 0
+    hc = np.empty(x_bits.shape, np.uint8)
+    lc = np.empty(x_bits.shape, np.uint8)
+    hs = np.empty(x_bits.shape[:-1] + (K // 32,), np.uint8)
+    ls = np.empty(x_bits.shape[:-1] + (K // 32,), np.uint8)
+    _load().orc_quant_mxfp8_split(_p(x_bits), rows, K, _p(hc), _p(hs), _p(lc), _p(ls))
+    return hc, hs, lc, ls
+
+
+def grouped_gemm_w4a8x2(hi_codes, hi_scales, lo_codes, lo_scales, w, w_scales, offsets, rows=None):
+    """fp64 Y[rows, N] of the two-term native mode: (hi + lo) MXFP8 activations x MXFP4 weights."""
+    hc, hs = _c(hi_codes, np.uint8), _c(hi_scales, np.uint8)
+    lc, ls = _c(lo_codes, np.uint8), _c(lo_scales, np.uint8)
+    w = _c(w, np.uint8)
+    w_scales = _c(w_scales, np.uint8)
+    offsets = _c(offsets, np.int32)
+    E, N, K2 = w.shape
+    K = 2 * K2
+    if rows is None:
+        rows = np.arange(int(offsets[-1]), dtype=np.int64)
+    rows = _c(rows, np.int64)
+    y = np.empty((rows.shape[0], N), np.float64)
+    _load().orc_grouped_gemm_w4a8x2(_p(hc), _p(hs), _p(lc), _p(ls), _p(w), _p(w_scales), _p(offsets), E, N, K,
+                                    _p(rows), rows.shape[0], _p(y))
     return y

@@ -590,6 +590,34 @@ static unsigned e4m3_round_magnitude(double m)
     return best;
 }
 
+/* One MXFP8 block: 32 values (exact in fp64) -> 32 e4m3 codes + the e8m0
+ * scale byte.  Shared exponent floor(log2(amax)) - top: top = 8 is the OCP
+ * rule of reading C19 (the largest element lands in [256, 512) and may
+ * saturate at 448); top = 7 leaves one binade of headroom (largest element
+ * in [128, 256), nothing saturates), the rule of the two-term split
+ * (reading C20). */
+static uint8_t mxfp8_block(const double *v, uint8_t *codes, int top)
+{
+    double amax = 0.0;
+    for (int i = 0; i < 32; ++i)
+        if (fabs(v[i]) > amax) amax = fabs(v[i]);
+    int sexp;
+    if (amax == 0.0) {
+        sexp = -127;
+    } else {
+        int ex;
+        frexp(amax, &ex); /* amax = f * 2^ex, f in [0.5, 1) */
+        sexp = (ex - 1) - top;
+        if (sexp < -127) sexp = -127;
+        if (sexp > 127) sexp = 127;
+    }
+    for (int i = 0; i < 32; ++i) {
+        const unsigned mag = e4m3_round_magnitude(ldexp(fabs(v[i]), -sexp));
+        codes[i] = (uint8_t)(mag | (signbit(v[i]) ? 0x80u : 0u));
+    }
+    return (uint8_t)(sexp + 127);
+}
+
 /* Quantise rows x K bf16 activations to MXFP8: codes [rows, K] e4m3 and
  * scales [rows, K/32] e8m0.  Per block of 32: X = floor(log2(amax)) - 8 (8
  * is e4m3's largest exponent), clamped to [-127, 127]; code = the nearest
@@ -602,28 +630,9 @@ void orc_quant_mxfp8(const uint16_t *x, int64_t rows, int64_t K, uint8_t *codes,
 #pragma omp parallel for num_threads(g_threads) schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t b = 0; b < nb; ++b) {
-            const uint16_t *blk = x + r * K + b * 32;
-            double amax = 0.0;
-            for (int i = 0; i < 32; ++i) {
-                const double a = fabs((double)bf16_to_float(blk[i]));
-                if (a > amax) amax = a;
-            }
-            int sexp;
-            if (amax == 0.0) {
-                sexp = -127;
-            } else {
-                int ex;
-                frexp(amax, &ex); /* amax = f * 2^ex, f in [0.5, 1) */
-                sexp = (ex - 1) - 8;
-                if (sexp < -127) sexp = -127;
-                if (sexp > 127) sexp = 127;
-            }
-            scales[r * nb + b] = (uint8_t)(sexp + 127);
-            for (int i = 0; i < 32; ++i) {
-                const double v = (double)bf16_to_float(blk[i]);
-                const unsigned mag = e4m3_round_magnitude(ldexp(fabs(v), -sexp));
-                codes[r * K + b * 32 + i] = (uint8_t)(mag | (signbit(v) ? 0x80u : 0u));
-            }
+            double v[32];
+            for (int i = 0; i < 32; ++i) v[i] = (double)bf16_to_float(x[r * K + b * 32 + i]);
+            scales[r * nb + b] = mxfp8_block(v, codes + r * K + b * 32, 8);
         }
     }
 }
@@ -671,4 +680,40 @@ void orc_grouped_gemm_w4a8(const uint8_t *qa, const uint8_t *sa, const uint8_t *
             for (int64_t n = 0; n < N; ++n) y[i * N + n] = NAN;
     free(ad);
     free(wd);
+}
+
+/* Two-term MXFP8 split of bf16 activations (reading C20): per block of 32,
+ * hi = MXFP8 of x and lo = MXFP8 of the residual r = x - dequant(hi) (exact
+ * in fp64), both with the headroom rule (shared exponent
+ * floor(log2(amax)) - 7, so no element saturates).  x ~ hi + lo with the
+ * error of one e4m3 rounding of the residual. */
+void orc_quant_mxfp8_split(const uint16_t *x, int64_t rows, int64_t K, uint8_t *hi_codes, uint8_t *hi_scales,
+                           uint8_t *lo_codes, uint8_t *lo_scales)
+{
+    const int64_t nb = K / 32;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            double v[32], res[32];
+            for (int i = 0; i < 32; ++i) v[i] = (double)bf16_to_float(x[r * K + b * 32 + i]);
+            uint8_t *hc = hi_codes + r * K + b * 32, *lc = lo_codes + r * K + b * 32;
+            const uint8_t hs = mxfp8_block(v, hc, 7);
+            hi_scales[r * nb + b] = hs;
+            for (int i = 0; i < 32; ++i) res[i] = v[i] - e4m3_value(hc[i]) * ldexp(1.0, (int)hs - 127);
+            lo_scales[r * nb + b] = mxfp8_block(res, lc, 7);
+        }
+    }
+}
+
+/* Two-term native GEMM: y[i, n] = sum_k (hi[r, k] + lo[r, k]) * W_e[n, k] in
+ * fp64, hi and lo the dequantised MXFP8 terms of reading C20 [W4A8]. */
+void orc_grouped_gemm_w4a8x2(const uint8_t *hc, const uint8_t *hs, const uint8_t *lc, const uint8_t *ls,
+                             const uint8_t *w, const uint8_t *sw, const int32_t *offsets, int64_t E, int64_t N,
+                             int64_t K, const int64_t *rows, int64_t n_rows, double *y)
+{
+    double *yl = (double *)malloc((size_t)(n_rows > 0 ? n_rows : 1) * (size_t)N * sizeof(double));
+    orc_grouped_gemm_w4a8(hc, hs, w, sw, offsets, E, N, K, rows, n_rows, y);
+    orc_grouped_gemm_w4a8(lc, ls, w, sw, offsets, E, N, K, rows, n_rows, yl);
+    for (int64_t i = 0; i < n_rows * N; ++i) y[i] += yl[i];
+    free(yl);
 }

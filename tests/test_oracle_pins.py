@@ -673,3 +673,80 @@ def test_w4a8_stays_within_the_e4m3_bound_of_the_bf16_activation_result():
         assert np.all(np.abs(y8[r0:r1] - y16[r0:r1]) <= bound)
     rel = np.linalg.norm(y8 - y16) / np.linalg.norm(y16)
     assert rel < 0.04, rel
+
+
+# ---------------------------------------------------------------- two-term MXFP8 split
+
+
+def test_mxfp8_split_worked_example():
+    """x = 1 + 2^-7 alone in its block, headroom rule (exponent
+    floor(log2 amax) - 7): hi = 129 at scale 2^-7 rounds to 128 (code 0x70,
+    scale byte 120); the residual 2^-7 is exact in lo (128 at scale 2^-14,
+    code 0x70, scale byte 113): hi + lo == x.  A block of 1.9375 (which the
+    single-term rule saturates at 448): 248 at scale 2^-7 is a tie between
+    240 (odd code 0x77) and 256 (even code 0x78) and goes to 256; the
+    residual -1/16 is exact in lo (-128 at scale 2^-11: code 0xF0, scale byte
+    116)."""
+    x = np.zeros(32, np.float32)
+    x[5] = 1.0 + 2.0 ** -7
+    hc, hs, lc, ls = oracle.quant_mxfp8_split(_bf16_bits(x)[None, :])
+    assert hs[0, 0] == 120 and hc[0, 5] == 0x70
+    assert ls[0, 0] == 113 and lc[0, 5] == 0x70
+    assert np.all(np.delete(hc[0], 5) == 0) and np.all(np.delete(lc[0], 5) == 0)
+    x[:] = 1.9375
+    hc, hs, lc, ls = oracle.quant_mxfp8_split(_bf16_bits(x)[None, :])
+    assert hs[0, 0] == 120 and np.all(hc[0] == 0x78)
+    assert ls[0, 0] == 116 and np.all(lc[0] == 0xF0)
+
+
+def test_mxfp8_split_never_saturates():
+    rng = inputs.rng(81)
+    x = rng.standard_normal((32, 256)).astype(np.float32) * np.float32(1.99)
+    hc, hs, lc, ls = oracle.quant_mxfp8_split(_bf16_bits(x))
+    v = oracle.e4m3_values()
+    assert np.abs(v[hc]).max() <= 256 and np.abs(v[lc]).max() <= 256  # far below 448: nothing saturates
+
+
+def test_mxfp8_split_error_bound_and_exact_residuals():
+    """The residual x - hi is computed here with numpy in float64; lo must
+    reproduce it within one e4m3 rounding (half an ulp: 2^-4 relative for
+    normal codes, 2^-10 * 2^X_lo absolute for subnormal ones), so the split
+    error never exceeds 2^-8 of the block's largest |x|; and most residuals
+    (few significant bits) come back exactly."""
+    rng = inputs.rng(82)
+    x = rng.standard_normal((64, 512)).astype(np.float32)
+    x *= np.exp2(rng.integers(-12, 12, size=(64, 16, 1))).repeat(32, axis=2).reshape(64, 512).astype(np.float32)
+    bits = _bf16_bits(x)
+    xf = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    hc, hs, lc, ls = oracle.quant_mxfp8_split(bits)
+    hi = oracle.dequant_mxfp8(hc, hs)
+    lo = oracle.dequant_mxfp8(lc, ls)
+    res = xf - hi
+    sl = np.exp2(ls.astype(np.float64) - 127.0).repeat(32, axis=1)
+    v = np.abs(res) / sl
+    err = np.abs(lo - res)
+    normal = (v >= 2.0 ** -6) & (v < 448)
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(res[normal]))
+    assert np.all(err[v < 2.0 ** -6] <= 2.0 ** -10 * sl[v < 2.0 ** -6])
+    amax = np.abs(xf.reshape(64, 16, 32)).max(axis=2).repeat(32, axis=1)
+    assert np.all(np.abs(xf - hi - lo) <= 2.0 ** -8 * amax)
+    assert np.mean(hi + lo == xf) > 0.9
+
+
+def test_w4a8x2_gemm_meets_the_bf16_activation_tolerance():
+    """With both terms the native mode lands within the path's standard
+    tolerance of the bf16-activation result (1e-2 max|ref| + 2^-7 |ref|)."""
+    rng = inputs.rng(83)
+    E, N, K = 3, 32, 2880
+    offsets = np.array([0, 7, 7, 20], np.int32)
+    w, sw = inputs.mxfp4_random(rng, E, N, K)
+    a = inputs.bf16_normal(rng, (20, K))
+    hc, hs, lc, ls = oracle.quant_mxfp8_split(a)
+    y2 = oracle.grouped_gemm_w4a8x2(hc, hs, lc, ls, w, sw, offsets)
+    y16 = oracle.grouped_gemm_mxfp4(a, w, sw, offsets)
+    bound = 1e-2 * np.abs(y16).max() + 2.0 ** -7 * np.abs(y16)
+    assert np.all(np.abs(y2 - y16) <= bound)
+    # and it is the sum of the two single-term products
+    y_hi = oracle.grouped_gemm_w4a8(hc, hs, w, sw, offsets)
+    y_lo = oracle.grouped_gemm_w4a8(lc, ls, w, sw, offsets)
+    assert np.allclose(y2, y_hi + y_lo, rtol=1e-14, atol=1e-12)
