@@ -292,9 +292,12 @@ gnf4_status grouped_dgrad(int fmt, const void* dy, const uint8_t* w, const void*
 // Native W4A8 GEMM: e4m3 codes [M, K] by TMA (32- and 128-row boxes of 128 codes), the e2m1 stack as
 // [E*N] x (K/128) x 128 codes expanded by the TMA unit into the padded 16-codes-per-16-bytes layout, and
 // for K % 128 == 64 a second view of codes [K-128, K) of every row.
-gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w,
-                              const uint8_t* w_scales, const int32_t* offsets, const int32_t* counts, int E, int N,
-                              int K, int M, void* y, void* stream) {
+// lo_codes / lo_scales non-null: the two-term mode (a_codes / a_scales are the hi term).
+gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* lo_codes,
+                              const uint8_t* lo_scales, const uint8_t* w, const uint8_t* w_scales,
+                              const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M, void* y,
+                              void* stream) {
+  const bool split = lo_codes != nullptr || lo_scales != nullptr;
   if (E < 1 || E > kMaxExperts) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "E=%d outside [1, %d]", E, kMaxExperts);
   if (N < 1 || N % 8 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N=%d must be a positive multiple of 8", N);
   if (K < 128 || K % 64 != 0 || K > 65536)
@@ -304,8 +307,12 @@ gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, c
   if ((offsets == nullptr) == (counts == nullptr))
     return fail(GNF4_ERR_INVALID_ARG, "pass exactly one of offsets [E+1] and counts [E]");
   if (M == 0) return GNF4_OK;
-  GNF4_TRY(check_ptr(a_codes, "a_codes", 16));
-  GNF4_TRY(check_ptr(a_scales, "a_scales", 2));
+  GNF4_TRY(check_ptr(a_codes, split ? "hi_codes" : "a_codes", 16));
+  GNF4_TRY(check_ptr(a_scales, split ? "hi_scales" : "a_scales", 2));
+  if (split) {
+    GNF4_TRY(check_ptr(lo_codes, "lo_codes", 16));
+    GNF4_TRY(check_ptr(lo_scales, "lo_scales", 2));
+  }
   GNF4_TRY(check_ptr(w, "w", 32));
   GNF4_TRY(check_ptr(w_scales, "w_scales", 2));
   GNF4_TRY(check_ptr(offsets, "offsets", 4, false));
@@ -321,8 +328,11 @@ gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, c
     cuuint64_t strides[1] = {(cuuint64_t)K};
     cuuint32_t estr[2] = {1, 1};
     for (int big = 0; big < 2; ++big) {
-      cuuint32_t box[2] = {128, (cuuint32_t)(big ? gemm_w4a8_rows_per_unit() : gemm_w4a8_small_box_rows())};
-      CUresult r = fn(big ? &tm_a_big : &tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a_codes), dims,
+      // single term: 32- and 128-row boxes of the codes; two terms: 32-row boxes of hi and of lo
+      const uint8_t* src = (split && big) ? lo_codes : a_codes;
+      cuuint32_t box[2] = {128, (cuuint32_t)((big && !split) ? gemm_w4a8_rows_per_unit(false)
+                                                             : gemm_w4a8_small_box_rows())};
+      CUresult r = fn(big ? &tm_a_big : &tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(src), dims,
                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
       if (r != CUDA_SUCCESS) return fail(GNF4_ERR_CUDA, "e4m3 tensor map encode failed (CUresult %d)", (int)r);
@@ -353,12 +363,13 @@ gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, c
     tm_w_tail = tm_w;  // never used
   }
   const long long nwt = (N + (long long)wrows - 1) / wrows;
-  const long long rpu = gemm_w4a8_rows_per_unit();
+  const long long rpu = gemm_w4a8_rows_per_unit(split);
   const long long units = ((M + rpu - 1) / rpu + (E < M ? E : M)) * nwt;
   if (units >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d, N=%d give too many work units", M, N);
   const int grid = (int)(units < d->num_sms ? units : d->num_sms);
-  cudaError_t e = launch_gemm_w4a8(tm_a, tm_a_big, tm_w, tm_w_tail, a_scales, w_scales, offsets, counts,
-                                   static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M, grid, as_stream(stream));
+  cudaError_t e = launch_gemm_w4a8(tm_a, tm_a_big, tm_w, tm_w_tail, a_scales, split ? lo_scales : nullptr,
+                                   w_scales, offsets, counts, static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M,
+                                   grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "W4A8 grouped GEMM launch");
   return GNF4_OK;
 }
@@ -603,8 +614,8 @@ gnf4_status gnf4_quantize_mxfp8(const void* x, int M, int K, uint8_t* codes, uin
   GNF4_TRY(check_ptr(scales, "scales", 1));
   DeviceState* d = nullptr;
   GNF4_TRY(device_state(&d));
-  cudaError_t e = launch_quant_mxfp8(static_cast<const __nv_bfloat16*>(x), (long long)M * K, codes, scales,
-                                     as_stream(stream));
+  cudaError_t e = launch_quant_mxfp8(static_cast<const __nv_bfloat16*>(x), (long long)M * K, codes, scales, nullptr,
+                                     nullptr, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "MXFP8 quantiser launch");
   return GNF4_OK;
 }
@@ -612,7 +623,34 @@ gnf4_status gnf4_quantize_mxfp8(const void* x, int M, int K, uint8_t* codes, uin
 gnf4_status gnf4_grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w,
                                    const uint8_t* w_scales, const int32_t* offsets, const int32_t* counts, int E,
                                    int N, int K, int M, void* y, void* stream) {
-  return grouped_gemm_w4a8(a_codes, a_scales, w, w_scales, offsets, counts, E, N, K, M, y, stream);
+  return grouped_gemm_w4a8(a_codes, a_scales, nullptr, nullptr, w, w_scales, offsets, counts, E, N, K, M, y, stream);
+}
+
+gnf4_status gnf4_quantize_mxfp8_split(const void* x, int M, int K, uint8_t* hi_codes, uint8_t* hi_scales,
+                                      uint8_t* lo_codes, uint8_t* lo_scales, void* stream) {
+  if (M < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d is negative", M);
+  if (K < 32 || K % 32 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K=%d must be a positive multiple of 32", K);
+  if (M == 0) return GNF4_OK;
+  GNF4_TRY(check_ptr(x, "x", 16));
+  GNF4_TRY(check_ptr(hi_codes, "hi_codes", 16));
+  GNF4_TRY(check_ptr(hi_scales, "hi_scales", 1));
+  GNF4_TRY(check_ptr(lo_codes, "lo_codes", 16));
+  GNF4_TRY(check_ptr(lo_scales, "lo_scales", 1));
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  cudaError_t e = launch_quant_mxfp8(static_cast<const __nv_bfloat16*>(x), (long long)M * K, hi_codes, hi_scales,
+                                     lo_codes, lo_scales, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "MXFP8 split quantiser launch");
+  return GNF4_OK;
+}
+
+gnf4_status gnf4_grouped_gemm_w4a8x2(const uint8_t* hi_codes, const uint8_t* hi_scales, const uint8_t* lo_codes,
+                                     const uint8_t* lo_scales, const uint8_t* w, const uint8_t* w_scales,
+                                     const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M,
+                                     void* y, void* stream) {
+  if (lo_codes == nullptr || lo_scales == nullptr) return fail(GNF4_ERR_INVALID_ARG, "lo_codes / lo_scales is NULL");
+  return grouped_gemm_w4a8(hi_codes, hi_scales, lo_codes, lo_scales, w, w_scales, offsets, counts, E, N, K, M, y,
+                           stream);
 }
 
 gnf4_status gnf4_grouped_gemm_mxfp4_swiglu(const void* a, const uint8_t* w_gate_up, const uint8_t* scales,

@@ -82,16 +82,18 @@ int dgrad_tc_k_per_unit();
 int dgrad_tc_n_per_stage();
 
 // mx.cu: native W4A8 (MXFP8 activations x MXFP4 weights, kind::mxf8f6f4)
+// lo_codes / lo_scales non-null: the two-term split (hi into codes / scales)
 cudaError_t launch_quant_mxfp8(const __nv_bfloat16* x, long long elems, uint8_t* codes, uint8_t* scales,
-                               cudaStream_t stream);
+                               uint8_t* lo_codes, uint8_t* lo_scales, cudaStream_t stream);
 // tm_a / tm_a_big: e4m3 codes [M, K] in 128 x 32 / 128 x 128 boxes; tm_w: the [E*N] x (K/128) x 128-code
 // view of the e2m1 stack; tm_w_tail: codes [K-128, K) of every row (used when K % 128 == 64).
+// lo_scales non-null: the two-term mode; tm_a = hi codes, tm_a_big = lo codes, both in 128 x 32 boxes.
 cudaError_t launch_gemm_w4a8(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
-                             const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* w_scales,
-                             const int* offsets, const int* counts, __nv_bfloat16* y, unsigned* err, int E, int N,
-                             int K, int M, int grid, cudaStream_t stream);
-size_t gemm_w4a8_smem_bytes();
-int gemm_w4a8_rows_per_unit();
+                             const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* lo_scales,
+                             const uint8_t* w_scales, const int* offsets, const int* counts, __nv_bfloat16* y,
+                             unsigned* err, int E, int N, int K, int M, int grid, cudaStream_t stream);
+size_t gemm_w4a8_smem_bytes(bool split);
+int gemm_w4a8_rows_per_unit(bool split);
 int gemm_w4a8_weight_rows_per_unit();
 int gemm_w4a8_small_box_rows();
 

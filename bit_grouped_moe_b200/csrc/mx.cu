@@ -39,6 +39,7 @@
 //    the epilogue of one unit overlap the main loop of the next.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -50,11 +51,40 @@ namespace {
 
 constexpr int kQThreads = 256;
 
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float hi, float lo) {
+  uint16_t pr;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(hi), "f"(lo));
+  return pr;
+}
+
+// e4m3 pair (low byte = first element) -> two floats, exactly (through f16).
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t pr) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)pr));
+  const __half2 hh = *reinterpret_cast<const __half2*>(&h);
+  return __half22float2(hh);
+}
+
+// Exact power of two 2^e for e in [-126, 127].
+__device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// floor(log2(a)) of a positive float given by its bits (subnormals included).
+__device__ __forceinline__ int ilog2_f32(uint32_t b) {
+  return (b >> 23) != 0 ? (int)(b >> 23) - 127 : (31 - __clz((int)b)) - 149;
+}
+
 // One thread quantises 8 consecutive k (16 bytes of bf16); the 4 threads of
-// a 32-k block agree on its amax with two shuffles.
+// a 32-k block agree on its amax with two shuffles.  TOP = 8: the OCP rule
+// (exponent floor(log2 amax) - 8).  SPLIT: the two-term split with one
+// binade of headroom (exponent floor(log2 amax) - 7 for both terms): hi of
+// x, then lo of the exact residual x - hi.
+template <bool SPLIT>
 __global__ void __launch_bounds__(kQThreads) quant_mxfp8_kernel(const __nv_bfloat16* __restrict__ x,
                                                                 long long octets, uint8_t* __restrict__ codes,
-                                                                uint8_t* __restrict__ scales) {
+                                                                uint8_t* __restrict__ scales,
+                                                                uint8_t* __restrict__ lo_codes,
+                                                                uint8_t* __restrict__ lo_scales) {
+  constexpr int kTop = SPLIT ? 7 : 8;
   griddep_launch_dependents();
   griddep_wait();
   const long long o = (long long)blockIdx.x * kQThreads + threadIdx.x;
@@ -70,17 +100,20 @@ __global__ void __launch_bounds__(kQThreads) quant_mxfp8_kernel(const __nv_bfloa
   // floor(log2(amax)) is the bf16 exponent field - 127; zero and subnormal
   // amax clamp to the smallest scale
   const int ef = (int)(m >> 7);
-  const int X = ef == 0 ? -127 : max(ef - 127 - 8, -127);
+  const int X = ef == 0 ? -127 : max(ef - 127 - kTop, -127);
   const float inv = __uint_as_float((uint32_t)(127 - X) << 23);  // 2^-X, a normal float for every X here
+  float xv[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    xv[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), inv);  // exact: a power-of-two scaling
+    xv[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv);
+  }
   uint32_t out[2];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float lo = __fmul_rn(__uint_as_float(w[i] << 16), inv);
-    const float hi = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv);
-    uint16_t pr;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(hi), "f"(lo));
+    const uint32_t pr = cvt_e4m3x2(xv[2 * i + 1], xv[2 * i]);
     if (i & 1)
-      out[i >> 1] |= (uint32_t)pr << 16;
+      out[i >> 1] |= pr << 16;
     else
       out[i >> 1] = pr;
   }
@@ -88,49 +121,102 @@ __global__ void __launch_bounds__(kQThreads) quant_mxfp8_kernel(const __nv_bfloa
     *reinterpret_cast<uint2*>(codes + o * 8) = make_uint2(out[0], out[1]);
     if ((threadIdx.x & 3) == 0) scales[o >> 2] = (uint8_t)(X + 127);
   }
+  if (SPLIT) {
+    // residual in the scaled domain: exact in fp32 (x has 8 significant bits,
+    // hi is x rounded to 4 of them, or to the 2^-9 grid below 2^-6)
+    float r[8];
+    uint32_t rm = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 h = e4m3x2_to_f32((out[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+      r[2 * i] = __fsub_rn(xv[2 * i], h.x);
+      r[2 * i + 1] = __fsub_rn(xv[2 * i + 1], h.y);
+      rm = max(rm, max(__float_as_uint(r[2 * i]) & 0x7FFFFFFFu, __float_as_uint(r[2 * i + 1]) & 0x7FFFFFFFu));
+    }
+    rm = max(rm, __shfl_xor_sync(0xffffffffu, rm, 1));
+    rm = max(rm, __shfl_xor_sync(0xffffffffu, rm, 2));
+    // lo exponent in absolute terms: floor(log2(max|r| * 2^X)) - 7, clamped
+    const int XL = rm == 0 ? -127 : min(max(ilog2_f32(rm) + X - kTop, -127), 127);
+    const int d = X - XL;  // >= 0: lo value = r * 2^d, split in two exact steps
+    const int d1 = min(d, 126);
+    const float m1 = exp2i(d1), m2 = exp2i(d - d1);
+    uint32_t lo[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float a = __fmul_rn(__fmul_rn(r[2 * i], m1), m2);
+      const float b = __fmul_rn(__fmul_rn(r[2 * i + 1], m1), m2);
+      const uint32_t pr = cvt_e4m3x2(b, a);
+      if (i & 1)
+        lo[i >> 1] |= pr << 16;
+      else
+        lo[i >> 1] = pr;
+    }
+    if (ok) {
+      *reinterpret_cast<uint2*>(lo_codes + o * 8) = make_uint2(lo[0], lo[1]);
+      if ((threadIdx.x & 3) == 0) lo_scales[o >> 2] = (uint8_t)(XL + 127);
+    }
+  }
 }
 
 // ------------------------------------------------------------------ GEMM
 
-constexpr int kBT = 128;  // rows (tokens) per unit = max MMA N
+// Geometry of the two modes.  SPLIT (two-term activations): a unit takes at
+// most 96 rows of a group; its B operand stacks the hi rows of the chunk
+// (nbx = ceil(rows / 32) boxes of 32 rows) over the lo rows (nbx more
+// boxes), so one MMA with N = 64 * nbx multiplies both terms, and the
+// epilogue adds the two halves of the accumulator.
+template <bool SPLIT>
+struct Geo {
+  static constexpr int kBT = SPLIT ? 96 : 128;          // rows (tokens) per unit
+  static constexpr int kStages = SPLIT ? 5 : 6;
+  static constexpr int kAccW = SPLIT ? 192 : 128;       // accumulator columns per buffer
+  static constexpr int kARows = SPLIT ? 192 : 128;      // activation rows per stage in shared memory
+  static constexpr int kSfaWords = SPLIT ? 256 : 128;   // activation scale words per stage
+  static constexpr int kSfCols = SPLIT ? 12 : 8;        // TMEM scale columns per stage
+};
+
 constexpr int kBW = 128;  // weight rows per unit = MMA M
 constexpr int kBK = 128;  // k per stage
-constexpr int kStages = 6;
-constexpr int kSmallBox = 32;  // activation rows per TMA box for groups of <= 32 rows
+constexpr int kBox = 32;  // activation rows per small TMA box
 constexpr int kEpiWarp0 = 4;
 constexpr int kProd2 = 12;  // second TMA producer warp
 constexpr int kThreads = 13 * 32;
-// scale-loader index of a warp (its ring slot), or -1
-__device__ __forceinline__ int loader_index(int warp) {
-  return warp == 2 || warp == 3 ? warp - 2 : (warp >= 8 && warp < 8 + kStages - 2 ? warp - 6 : -1);
-}
-constexpr int kWStageBytes = kBW * kBK;    // padded e2m1 in shared memory: one byte per code
-constexpr int kWStageTx = kBW * kBK / 2;   // bytes the TMA reads: two codes per byte
-constexpr int kAStageBytes = kBT * kBK;    // e4m3
+constexpr int kWStageBytes = kBW * kBK;   // padded e2m1 in shared memory: one byte per code
+constexpr int kWStageTx = kBW * kBK / 2;  // bytes the TMA reads: two codes per byte
 constexpr int kTmemCols = 512;
-constexpr int kSfCol0 = 2 * kBT;           // per stage: 4 columns of weight scales, then 4 of activation scales
-static_assert(kSfCol0 + 8 * kStages <= kTmemCols, "TMEM budget");
-static_assert(kStages == 6, "one scale-loader warp per ring slot: warps 2, 3, 8..11");
 
+// scale-loader index of a warp (its ring slot), or -1: warps 2, 3, 8, 9, ...
+template <bool SPLIT>
+__device__ __forceinline__ int loader_index(int warp) {
+  return warp == 2 || warp == 3 ? warp - 2 : (warp >= 8 && warp < 8 + Geo<SPLIT>::kStages - 2 ? warp - 6 : -1);
+}
+
+template <bool SPLIT>
 struct MxSmem {
-  uint8_t w[kStages][kWStageBytes];  // 1024-aligned (offset 0)
-  uint8_t a[kStages][kAStageBytes];
-  uint32_t sfw[kStages][kBW];        // weight scales of the stage, tcgen05.cp layout
-  uint32_t sfa[kStages][kBT];        // activation scales of the stage
+  using G = Geo<SPLIT>;
+  uint8_t w[G::kStages][kWStageBytes];  // 1024-aligned (offset 0)
+  uint8_t a[G::kStages][G::kARows * kBK];
+  uint32_t sfw[G::kStages][kBW];        // weight scales of the stage, tcgen05.cp layout
+  uint32_t sfa[G::kStages][G::kSfaWords];  // activation scales of the stage (two 128-row blocks in SPLIT)
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
-  uint64_t full[kStages], empty[kStages];  // full: TMA bytes + the producer's arrival + the scale copies' commit
-  uint64_t ldone[kStages];                 // abort path only: a loader's scale copies have retired
+  uint64_t full[G::kStages], empty[G::kStages];  // full: TMA bytes + producer arrival + the scale copies' commit
+  uint64_t ldone[G::kStages];                    // abort path only: a loader's scale copies have retired
   uint64_t accf[2], acce[2];
   uint64_t mdone;  // abort path only: every issued MMA has retired
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(MxSmem) + 1024 <= 227 * 1024, "shared memory budget");
+static_assert(sizeof(MxSmem<false>) + 1024 <= 227 * 1024, "shared memory budget");
+static_assert(sizeof(MxSmem<true>) + 1024 <= 227 * 1024, "shared memory budget");
+static_assert(2 * Geo<false>::kAccW + Geo<false>::kSfCols * Geo<false>::kStages <= kTmemCols, "TMEM budget");
+static_assert(2 * Geo<true>::kAccW + Geo<true>::kSfCols * Geo<true>::kStages <= kTmemCols, "TMEM budget");
+static_assert(Geo<false>::kStages <= 6 && Geo<true>::kStages <= 6, "scale loaders are warps 2, 3, 8..11");
 
 struct MxArgs {
-  const uint8_t* sa;   // activation scales e8m0 [M, K/32] (the codes come by TMA)
+  const uint8_t* sa;   // activation scales e8m0 [M, K/32] (SPLIT: of the hi term; the codes come by TMA)
+  const uint8_t* sl;   // SPLIT: lo-term scales [M, K/32]
   const uint8_t* sw;   // e8m0 [E, N, K/32]
   const int* offsets;  // [E+1] or null
   const int* counts;   // [E] or null
@@ -143,13 +229,14 @@ struct Unit {
   int e, j, row0, rows;
 };
 
-// Partial accumulators per unit: the K=32 steps of a unit of at most 32 (64)
-// rows rotate over 4 (2) accumulators of 32 (64) columns, so consecutive
-// block-scaled MMAs do not wait for each other; the epilogue adds them in a
-// fixed order.
+// Partial accumulators per unit (single-term mode): the K=32 steps of a unit
+// of at most 32 (64) rows rotate over 4 (2) accumulators of 32 (64) columns;
+// the epilogue adds them in a fixed order.
 __device__ __forceinline__ int acc_split(int rows) { return rows <= 32 ? 4 : (rows <= 64 ? 2 : 1); }
 
-__device__ __forceinline__ Unit unit_of(const MxSmem& s, int E, int u) {
+template <bool SPLIT>
+__device__ __forceinline__ Unit unit_of(const MxSmem<SPLIT>& s, int E, int u) {
+  constexpr int kBT = Geo<SPLIT>::kBT;
   Unit x;
   x.e = find_group(s.upre, E, u);
   const int local = u - s.upre[x.e];
@@ -206,12 +293,18 @@ __device__ __forceinline__ void sts_u128(uint32_t addr, uint32_t a, uint32_t b, 
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+// Single-term mode: tm_a / tm_a_big are the e4m3 codes in 32- / 128-row
+// boxes.  SPLIT: tm_a = hi codes, tm_a_big = lo codes, both in 32-row boxes.
+template <bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w4a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_big,
                      const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_w_tail,
                      MxArgs p) {
+  using G = Geo<SPLIT>;
+  constexpr int kStages = G::kStages;
   extern __shared__ uint8_t smem_raw[];
-  MxSmem& s = *reinterpret_cast<MxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  MxSmem<SPLIT>& s =
+      *reinterpret_cast<MxSmem<SPLIT>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   unsigned* err = p.err;
   volatile int* abort = &s.abort;
@@ -221,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, err)) return;
   const int nwt = (p.N + kBW - 1) / kBW;
   block_exclusive_scan(p.E, s.upre, s.scratch,
-                       [&](int e) { return ((s.off[e + 1] - s.off[e] + kBT - 1) / kBT) * nwt; });
+                       [&](int e) { return ((s.off[e + 1] - s.off[e] + G::kBT - 1) / G::kBT) * nwt; });
   const int U = s.upre[p.E];
   if ((int)blockIdx.x >= U) return;  // uniform over the block
   const int K = p.K;
@@ -256,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
+  const int sf_col0 = 2 * G::kAccW;
 
   if (warp == 0 || warp == kProd2) {
     // ------------------------------------------------------------ TMA producers
@@ -264,8 +358,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-        const Unit x = unit_of(s, p.E, u);
-        const bool big = x.rows > kSmallBox;
+        const Unit x = unit_of<SPLIT>(s, p.E, u);
+        const bool big = x.rows > kBox;
+        const int nbx = (x.rows + kBox - 1) / kBox;  // SPLIT: 32-row boxes per term
         const int wrow = x.e * p.N + x.j * kBW;
         for (int kt = 0; kt < nk; ++kt, ++it) {
           if ((it & 1) != pi) continue;
@@ -273,51 +368,74 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (it >= kStages && !(ok = mbar_wait(&s.empty[st], (use - 1) & 1, err, abort))) break;
           const bool last_tail = tail && kt == nk - 1;
           const int k0 = last_tail ? K - kBK : kt * kBK;
-          mbar_arrive_expect_tx(&s.full[st], kWStageTx + (big ? kBT : kSmallBox) * kBK);
+          if (SPLIT)
+            mbar_arrive_expect_tx(&s.full[st], kWStageTx + 2 * nbx * kBox * kBK);
+          else
+            mbar_arrive_expect_tx(&s.full[st], kWStageTx + (big ? G::kBT : kBox) * kBK);
           if (last_tail)
             tma_load_2d(s.w[st], &tm_w_tail, &s.full[st], 0, wrow);
           else
             tma_load_3d(s.w[st], &tm_w, &s.full[st], 0, kt, wrow);
-          tma_load_2d(s.a[st], big ? &tm_a_big : &tm_a, &s.full[st], k0, x.row0);
+          if (SPLIT) {
+            for (int b = 0; b < nbx; ++b) {
+              tma_load_2d(s.a[st] + b * kBox * kBK, &tm_a, &s.full[st], k0, x.row0 + b * kBox);
+              tma_load_2d(s.a[st] + (nbx + b) * kBox * kBK, &tm_a_big, &s.full[st], k0, x.row0 + b * kBox);
+            }
+          } else {
+            tma_load_2d(s.a[st], big ? &tm_a_big : &tm_a, &s.full[st], k0, x.row0);
+          }
         }
       }
       if (!ok)  // drain loads still in flight before shared memory goes away
         for (int i = max(0, it - kStages); i < it; ++i)
           if ((i & 1) == pi) mbar_drain(&s.full[i % kStages], (i / kStages) & 1);
     }
-  } else if (loader_index(warp) >= 0) {
+  } else if (loader_index<SPLIT>(warp) >= 0) {
     // ------------------------------------------------------------ scale loaders
-    // Loader i fills ring slot i only.  Lane l serves rows l, l+32, l+64, l+96
-    // of the tile and of the group chunk; rows outside them get scale 2^0
-    // (their products are never stored).
-    const int li = loader_index(warp);
+    // Loader i fills ring slot i only.  Lane l serves rows l + 32c of the
+    // weight tile (c < 4) and of the activation operand (c < 4, or < 8 for the
+    // stacked hi / lo rows of SPLIT); rows outside the tile or the group get
+    // scale 2^0 (their products are never stored).
+    const int li = loader_index<SPLIT>(warp);
     const int nsb = K / 32;
     const uint8_t* swb = p.sw;
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-      const Unit x = unit_of(s, p.E, u);
+      const Unit x = unit_of<SPLIT>(s, p.E, u);
+      const int hrows = kBox * ((x.rows + kBox - 1) / kBox);  // SPLIT: hi rows of the stacked operand
       for (int kt = 0; kt < nk; ++kt, ++it) {
         const int st = it % kStages, use = it / kStages;
         if (st != li) continue;
         if (it >= kStages && !(ok = mbar_wait(&s.empty[st], (use - 1) & 1, err, abort))) break;
         const int b0 = ((tail && kt == nk - 1) ? K - kBK : kt * kBK) / 32;  // even: K % 64 == 0
-        uint32_t wv[4], av[4];
+        uint32_t wv[4], av[G::kSfaWords / 32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int m = lane + 32 * c;
-          const int n = x.j * kBW + m;
+          const int n = x.j * kBW + lane + 32 * c;
           wv[c] = n < p.N ? ld_scales4(swb + ((size_t)x.e * p.N + (size_t)n) * (size_t)nsb + b0) : 0x7F7F7F7Fu;
-          av[c] = m < x.rows ? ld_scales4(p.sa + (size_t)(x.row0 + m) * (size_t)nsb + b0) : 0x7F7F7F7Fu;
+        }
+#pragma unroll
+        for (int c = 0; c < G::kSfaWords / 32; ++c) {
+          const int m = lane + 32 * c;
+          const bool lo_row = SPLIT && m >= hrows;
+          const int rr = lo_row ? m - hrows : m;
+          const uint8_t* src = lo_row ? p.sl : p.sa;
+          av[c] = rr < x.rows ? ld_scales4(src + (size_t)(x.row0 + rr) * (size_t)nsb + b0) : 0x7F7F7F7Fu;
         }
         sts_u128(smem_u32(&s.sfw[st][lane * 4]), wv[0], wv[1], wv[2], wv[3]);
-        sts_u128(smem_u32(&s.sfa[st][lane * 4]), av[0], av[1], av[2], av[3]);
+#pragma unroll
+        for (int bl = 0; bl < G::kSfaWords / 128; ++bl)
+          sts_u128(smem_u32(&s.sfa[st][bl * 128 + lane * 4]), av[4 * bl], av[4 * bl + 1], av[4 * bl + 2],
+                   av[4 * bl + 3]);
         fence_proxy_async_smem();  // the tensor core reads these through the async proxy
         __syncwarp();
         if (lane == 0) {
-          const uint32_t col = tmem + (uint32_t)(kSfCol0 + 8 * st);
+          const uint32_t col = tmem + (uint32_t)(sf_col0 + G::kSfCols * st);
           tc_copy_scales(col, sdesc_scales(smem_u32(s.sfw[st])));
-          tc_copy_scales(col + 4, sdesc_scales(smem_u32(s.sfa[st])));
+#pragma unroll
+          for (int bl = 0; bl < G::kSfaWords / 128; ++bl)
+            tc_copy_scales(col + 4u + 4u * (uint32_t)bl, sdesc_scales(smem_u32(&s.sfa[st][bl * 128])));
           tc_commit(&s.full[st]);
         }
       }
@@ -332,14 +450,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0, uc = 0;
       bool ok = true, ready = false;  // ready: the full barrier of stage `it` was seen complete in advance
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
-        const Unit x = unit_of(s, p.E, u);
+        const Unit x = unit_of<SPLIT>(s, p.E, u);
         const int ab = uc & 1;
         if (uc >= 2 && !(ok = mbar_wait(&s.acce[ab], ((uc >> 1) - 1) & 1, err, abort))) break;
         tc_fence_after();
-        const uint32_t n_mma = (uint32_t)((x.rows + 15) & ~15);
-        const uint32_t d_tmem = tmem + (uint32_t)(ab * kBT);
-        const int nsplit = acc_split(x.rows);
-        const uint32_t sub_w = (uint32_t)(kBT / nsplit);
+        const uint32_t n_mma =
+            SPLIT ? (uint32_t)(2 * kBox * ((x.rows + kBox - 1) / kBox)) : (uint32_t)((x.rows + 15) & ~15);
+        const uint32_t d_tmem = tmem + (uint32_t)(ab * G::kAccW);
+        const int nsplit = SPLIT ? 1 : acc_split(x.rows);
+        const uint32_t sub_w = (uint32_t)(G::kAccW / nsplit);
         for (int kt = 0; kt < nk; ++kt, ++it) {
           const int st = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -347,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           // test the next stage's barrier now: its latency overlaps this stage's issue
           ready = mbar_try_wait(&s.full[(it + 1) % kStages], (uint32_t)((it + 1) / kStages) & 1u);
-          const uint32_t t_sfw = tmem + (uint32_t)(kSfCol0 + 8 * st), t_sfa = t_sfw + 4u;
+          const uint32_t t_sfw = tmem + (uint32_t)(sf_col0 + G::kSfCols * st), t_sfa = t_sfw + 4u;
           const uint32_t w_addr = smem_u32(s.w[st]), a_addr = smem_u32(s.a[st]);
           const int j0 = (tail && kt == nk - 1) ? 2 : 0;
           for (int j = j0; j < kBK / 32; ++j) {
@@ -373,20 +492,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     int uc = 0;
     for (int u = blockIdx.x; u < U; u += gridDim.x, ++uc) {
-      const Unit x = unit_of(s, p.E, u);
+      const Unit x = unit_of<SPLIT>(s, p.E, u);
       const int ab = uc & 1;
       if (!mbar_wait(&s.accf[ab], (uc >> 1) & 1, err, abort)) break;
       tc_fence_after();
       const int n = x.j * kBW + q * 32 + lane;
       __nv_bfloat16* ycol = p.y + (size_t)x.row0 * p.N + n;
-      const int nsplit = acc_split(x.rows);
+      const int nsplit = SPLIT ? 1 : acc_split(x.rows);
+      // SPLIT: the lo term of row i sits hrows columns after its hi term
+      const int hrows = kBox * ((x.rows + kBox - 1) / kBox);
       for (int c = 0; c * 32 < x.rows; ++c) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBT + c * 32), v);
+        tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * G::kAccW + c * 32), v);
         tmem_wait_ld();
-        for (int j = 1; j < nsplit; ++j) {  // partial accumulators, summed in a fixed order
+        const int nparts = SPLIT ? 2 : nsplit;
+        for (int j = 1; j < nparts; ++j) {  // partial accumulators (or the lo term), summed in a fixed order
           uint32_t w2[32];
-          tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBT + j * (kBT / nsplit) + c * 32), w2);
+          const int off = SPLIT ? hrows : j * (G::kAccW / nsplit);
+          tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * G::kAccW + off + c * 32), w2);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w2[i]));
@@ -417,35 +540,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_quant_mxfp8(const __nv_bfloat16* x, long long elems, uint8_t* codes, uint8_t* scales,
-                               cudaStream_t stream) {
+                               uint8_t* lo_codes, uint8_t* lo_scales, cudaStream_t stream) {
   const long long octets = elems / 8;
   if (octets == 0) return cudaSuccess;
   const long long blocks = (octets + kQThreads - 1) / kQThreads;
-  return launch_pdl(quant_mxfp8_kernel, dim3((unsigned)blocks), dim3(kQThreads), 0, stream, x, octets, codes,
-                    scales);
+  if (lo_codes != nullptr)
+    return launch_pdl(quant_mxfp8_kernel<true>, dim3((unsigned)blocks), dim3(kQThreads), 0, stream, x, octets, codes,
+                      scales, lo_codes, lo_scales);
+  return launch_pdl(quant_mxfp8_kernel<false>, dim3((unsigned)blocks), dim3(kQThreads), 0, stream, x, octets, codes,
+                    scales, lo_codes, lo_scales);
 }
 
-size_t gemm_w4a8_smem_bytes() { return sizeof(MxSmem) + 1024; }
-int gemm_w4a8_rows_per_unit() { return kBT; }
+size_t gemm_w4a8_smem_bytes(bool split) { return (split ? sizeof(MxSmem<true>) : sizeof(MxSmem<false>)) + 1024; }
+int gemm_w4a8_rows_per_unit(bool split) { return split ? Geo<true>::kBT : Geo<false>::kBT; }
 int gemm_w4a8_weight_rows_per_unit() { return kBW; }
-int gemm_w4a8_small_box_rows() { return kSmallBox; }
+int gemm_w4a8_small_box_rows() { return kBox; }
 
-cudaError_t launch_gemm_w4a8(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
-                             const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* w_scales,
-                             const int* offsets, const int* counts, __nv_bfloat16* y, unsigned* err, int E, int N,
-                             int K, int M, int grid, cudaStream_t stream) {
+template <bool SPLIT>
+static cudaError_t launch_gemm_w4a8_t(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
+                                      const CUtensorMap& tm_w_tail, const MxArgs& p, int grid, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_w4a8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)gemm_w4a8_smem_bytes());
+    cudaError_t e = cudaFuncSetAttribute(gemm_w4a8_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)gemm_w4a8_smem_bytes(SPLIT));
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  MxArgs p{a_scales, w_scales, offsets, counts, y, err, E, N, K, M};
-  return launch_pdl(gemm_w4a8_kernel, dim3(grid), dim3(kThreads), gemm_w4a8_smem_bytes(), stream, tm_a, tm_a_big,
-                    tm_w, tm_w_tail, p);
+  return launch_pdl(gemm_w4a8_kernel<SPLIT>, dim3(grid), dim3(kThreads), gemm_w4a8_smem_bytes(SPLIT), stream, tm_a,
+                    tm_a_big, tm_w, tm_w_tail, p);
+}
+
+cudaError_t launch_gemm_w4a8(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
+                             const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* lo_scales,
+                             const uint8_t* w_scales, const int* offsets, const int* counts, __nv_bfloat16* y,
+                             unsigned* err, int E, int N, int K, int M, int grid, cudaStream_t stream) {
+  MxArgs p{a_scales, lo_scales, w_scales, offsets, counts, y, err, E, N, K, M};
+  if (lo_scales != nullptr) return launch_gemm_w4a8_t<true>(tm_a, tm_a_big, tm_w, tm_w_tail, p, grid, stream);
+  return launch_gemm_w4a8_t<false>(tm_a, tm_a_big, tm_w, tm_w_tail, p, grid, stream);
 }
 
 }  // namespace gnf4

@@ -337,6 +337,28 @@ gnf4_status gnf4_grouped_gemv_mxfp4_combine(const void *a, const uint8_t *w, con
  * multiple of 64 in [128, 65536].  Alignment: a_codes 16 bytes, w 32 bytes,
  * y 16 bytes.  Rows past offsets[E] are not written. */
 gnf4_status gnf4_quantize_mxfp8(const void *x, int M, int K, uint8_t *codes, uint8_t *scales, void *stream);
+
+/* Two-term form (the activations as hi + lo, two MXFP8 tensors), which
+ * keeps the bf16-activation accuracy of the MXFP4 GEMM on the native path
+ * (SURVEY reading of the block-scaled MXFP4 operand; the pages give no
+ * rule).  Per block of 32 consecutive k of one row:
+ *     hi = MXFP8 of x, lo = MXFP8 of the exact residual r = x - hi,
+ *     both with X = floor(log2(max |value|)) - 7 (one binade of headroom,
+ *     so no element saturates), e4m3 round to nearest even;
+ * x - (hi + lo) is one e4m3 rounding of r (at most 2^-8 of the block's
+ * largest |x|).  Bit-exact.  Buffers as gnf4_quantize_mxfp8, twice.
+ *
+ * gnf4_grouped_gemm_w4a8x2: y[r, n] = sum_k (hi[r,k] + lo[r,k]) * W_e[n,k],
+ * products exact, fp32 accumulation, bf16 output; the hi and lo rows of a
+ * group are stacked into one operand, so each block-scaled MMA multiplies
+ * both terms.  Arguments and rules as gnf4_grouped_gemm_w4a8, with both
+ * terms' codes (16-byte aligned) and scales. */
+gnf4_status gnf4_quantize_mxfp8_split(const void *x, int M, int K, uint8_t *hi_codes, uint8_t *hi_scales,
+                                      uint8_t *lo_codes, uint8_t *lo_scales, void *stream);
+gnf4_status gnf4_grouped_gemm_w4a8x2(const uint8_t *hi_codes, const uint8_t *hi_scales, const uint8_t *lo_codes,
+                                     const uint8_t *lo_scales, const uint8_t *w, const uint8_t *w_scales,
+                                     const int32_t *offsets, const int32_t *counts, int E, int N, int K, int M,
+                                     void *y, void *stream);
 gnf4_status gnf4_grouped_gemm_w4a8(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *w,
                                    const uint8_t *w_scales, const int32_t *offsets, const int32_t *counts, int E,
                                    int N, int K, int M, void *y, void *stream);

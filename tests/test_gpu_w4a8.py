@@ -143,3 +143,70 @@ def test_w4a8_refuses_k_that_is_not_a_multiple_of_64(g, K):
     with pytest.raises(g.Gnf4Error) as ei:
         g.grouped_gemm_w4a8(codes, sa, w, sw, y, offsets=off)
     assert ei.value.status == g.ERR_UNSUPPORTED_SHAPE
+
+
+# ---------------------------------------------------------------- two-term split (hi + lo)
+
+
+def _check_split(g, bits):
+    M, K = bits.shape
+    t = [torch.empty((M, K), dtype=torch.uint8, device="cuda"), torch.empty((M, K // 32), dtype=torch.uint8, device="cuda"),
+         torch.empty((M, K), dtype=torch.uint8, device="cuda"), torch.empty((M, K // 32), dtype=torch.uint8, device="cuda")]
+    g.quantize_mxfp8_split(to_dev_bf16(bits), *t)
+    torch.cuda.synchronize()
+    ref = oracle.quant_mxfp8_split(bits)
+    for name, got, r in zip(("hi codes", "hi scales", "lo codes", "lo scales"), t, ref):
+        got = got.cpu().numpy()
+        bad = np.argwhere(got != r)
+        assert bad.size == 0, f"{name}: {len(bad)} differ, first {[(tuple(i), int(got[tuple(i)]), int(r[tuple(i)])) for i in bad[:5]]}"
+    return t
+
+
+@pytest.mark.parametrize("M,K", [(37, 2880), (128, 2048), (1, 32), (300, 416)])
+def test_quantize_mxfp8_split_is_bit_exact(g, M, K):
+    _check_split(g, _activations(950 + K + M, M, K))
+
+
+def _run_split(g, counts, N, K, seed, use_counts=False):
+    E = len(counts)
+    offsets = offsets_from_counts(counts)
+    nv = int(offsets[-1])
+    M = nv + 3
+    w, sw = inputs.mxfp4_random(inputs.rng(seed), E, N, K)
+    bits = _activations(seed + 1, M, K)
+    hc, hs, lc, ls = _check_split(g, bits)
+    y = torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    kw = {"counts": to_dev(np.array(counts, np.int32))} if use_counts else {"offsets": to_dev(offsets)}
+    g.grouped_gemm_w4a8x2(hc, hs, lc, ls, to_dev(w), to_dev(sw), y, **kw)
+    torch.cuda.synchronize()
+    assert g.device_errors() == 0
+    got = bf16_to_f64(y)
+    assert np.all(got[nv:] == 7.0), "rows past offsets[E] were written"
+    return got[:nv], (w, sw, bits, offsets)
+
+
+@pytest.mark.parametrize("N,K", [(128, 128), (136, 192), (256, 2880), (384, 448)])
+def test_w4a8x2_gemm_ragged_parity(g, N, K):
+    got, (w, sw, bits, offsets) = _run_split(g, GROUPS, N, K, seed=1600 + K + N)
+    ref = oracle.grouped_gemm_w4a8x2(*oracle.quant_mxfp8_split(bits), w, sw, offsets)
+    amax = float(np.abs(ref).max())
+    err = np.abs(got - ref)
+    bad = np.argwhere(~(err <= W4A8_REL * np.abs(ref) + W4A8_ABS_OF_MAX * amax))
+    assert bad.size == 0, f"{len(bad)} outputs out of tolerance, first {[tuple(i) for i in bad[:5]]}"
+
+
+@pytest.mark.parametrize("N,K", [(256, 2880), (128, 2048)])
+def test_w4a8x2_meets_the_bf16_activation_tolerance(g, N, K):
+    """The two-term native path holds the standard tolerance of the grouped
+    GEMM against the bf16-activation oracle (1e-2 max|ref| + 2^-7 |ref|)."""
+    counts = [3, 60, 0, 130, 9, 1, 33]
+    got, (w, sw, bits, offsets) = _run_split(g, counts, N, K, seed=1700 + K)
+    from tests._util import assert_within_tolerance
+    assert_within_tolerance(got, oracle.grouped_gemm_mxfp4(bits, w, sw, offsets), "w4a8x2 vs bf16 activations")
+
+
+def test_w4a8x2_counts_equal_offsets(g):
+    counts = [40, 0, 129, 1, 7, 96, 97]
+    a, _ = _run_split(g, counts, 128, 256, seed=1800)
+    b, _ = _run_split(g, counts, 128, 256, seed=1800, use_counts=True)
+    assert np.array_equal(a, b)
