@@ -146,7 +146,7 @@ class Workload:
     than L2, a set of token batches, and the step's output buffers."""
 
     def __init__(self, name, device, seed, build_host_copy, swiglu=False, dgrad=False, w4a8=False,
-                 fused_combine=False):
+                 fused_combine=False, w4a8x2=False):
         import torch
 
         from bit_grouped_moe_b200 import gnf4
@@ -211,14 +211,20 @@ class Workload:
             self.dfn = f.grouped_dgrad_nf4 if wl.fmt == "nf4" else f.grouped_dgrad_mxfp4
         # optional native W4A8 mode (MXFP4 stacks): both projections' activations are
         # quantised to MXFP8 every step and the block-scaled GEMM runs on the codes
-        self.w4a8 = w4a8
-        if w4a8:
+        self.w4a8 = w4a8 or w4a8x2
+        self.split = w4a8x2  # two-term activations (hi + lo): the bf16-activation accuracy on the native path
+        if self.w4a8:
             assert wl.fmt == "mxfp4", "the W4A8 mode runs on MXFP4 weight stacks"
             self.decode = False  # one GEMM path for every group size
             self.qa1 = torch.empty(M, self.p1.K, dtype=torch.uint8, device=device)
             self.sa1 = torch.empty(M, self.p1.K // 32, dtype=torch.uint8, device=device)
             self.qa2 = torch.empty(M, self.p2.K, dtype=torch.uint8, device=device)
             self.sa2 = torch.empty(M, self.p2.K // 32, dtype=torch.uint8, device=device)
+            if self.split:
+                self.la1 = torch.empty_like(self.qa1)
+                self.ls1 = torch.empty_like(self.sa1)
+                self.la2 = torch.empty_like(self.qa2)
+                self.ls2 = torch.empty_like(self.sa2)
         # decode: the second projection's GEMV carries the top-k combine in its epilogue
         self.fused_combine = fused_combine and self.decode and not dgrad and not w4a8
         if self.fused_combine:
@@ -289,23 +295,36 @@ class Workload:
                 ev[1].record()
             return
         if self.w4a8:
-            g.quantize_mxfp8(self.xs, self.qa1, self.sa1)
+            self._quant1()
         if ev is not None:
             ev[0].record()
         self.project(w1, s1, w2, s2, ev, wts=wts)
         if not self.fused_combine:
             g.combine(self.y2, self.f2s, wts, self.out)
 
+    def _quant1(self):
+        if self.split:
+            self.g.quantize_mxfp8_split(self.xs, self.qa1, self.sa1, self.la1, self.ls1)
+        else:
+            self.g.quantize_mxfp8(self.xs, self.qa1, self.sa1)
+
     def project(self, w1, s1, w2, s2, ev=None, quantize_first=False, wts=None):
         if self.w4a8:
             g = self.g
             if quantize_first:
-                g.quantize_mxfp8(self.xs, self.qa1, self.sa1)
-            g.grouped_gemm_w4a8(self.qa1, self.sa1, w1, s1, self.y1, offsets=self.off)
+                self._quant1()
+            if self.split:
+                g.grouped_gemm_w4a8x2(self.qa1, self.sa1, self.la1, self.ls1, w1, s1, self.y1, offsets=self.off)
+            else:
+                g.grouped_gemm_w4a8(self.qa1, self.sa1, w1, s1, self.y1, offsets=self.off)
             if ev is not None:
                 ev[1].record()
-            g.quantize_mxfp8(self.h, self.qa2, self.sa2)
-            g.grouped_gemm_w4a8(self.qa2, self.sa2, w2, s2, self.y2, offsets=self.off)
+            if self.split:
+                g.quantize_mxfp8_split(self.h, self.qa2, self.sa2, self.la2, self.ls2)
+                g.grouped_gemm_w4a8x2(self.qa2, self.sa2, self.la2, self.ls2, w2, s2, self.y2, offsets=self.off)
+            else:
+                g.quantize_mxfp8(self.h, self.qa2, self.sa2)
+                g.grouped_gemm_w4a8(self.qa2, self.sa2, w2, s2, self.y2, offsets=self.off)
             return
         if self.swiglu:
             self.fn1(self.xs, w1, s1, self.hs, offsets=self.off)
@@ -381,7 +400,10 @@ def oracle_step(wl_obj, batch_i, n_slice=None):
     (w1, s1), (w2, s2) = wl_obj.host_stacks
     n1 = wl_obj.p1.N if n_slice is None else min(n_slice, wl_obj.p1.N)
     n2 = wl_obj.p2.N if n_slice is None else min(n_slice, wl_obj.p2.N)
-    if getattr(wl_obj, "w4a8", False):
+    if getattr(wl_obj, "split", False):
+        def gemm(a_bits, w, s, off):
+            return oracle.grouped_gemm_w4a8x2(*oracle.quant_mxfp8_split(a_bits), w, s, off)
+    elif getattr(wl_obj, "w4a8", False):
         def gemm(a_bits, w, s, off):
             qa, sa = oracle.quant_mxfp8(a_bits)
             return oracle.grouped_gemm_w4a8(qa, sa, w, s, off)
@@ -438,6 +460,9 @@ def main():
                     help=f"decode: also time the steps replayed from one CUDA graph of {20} steps")
     ap.add_argument("--w4a8", action="store_true",
                     help="MXFP4 workloads: native W4A8 mode (MXFP8 activations, block-scaled tcgen05 GEMM)")
+    ap.add_argument("--w4a8x2", action="store_true",
+                    help="MXFP4 workloads: two-term native mode (hi + lo MXFP8 activations, the bf16-activation "
+                         "accuracy on the block-scaled tcgen05 GEMM)")
     ap.add_argument("--fused-combine", action="store_true",
                     help="decode: run the top-k combine in the second GEMV's epilogue instead of as its own launch "
                          "(measured slower on B200: the epilogue's round trips extend every unit)")
@@ -449,7 +474,7 @@ def main():
     globals()["N_WEIGHT_COPIES"] = max(1, args.weight_copies)
 
     wl_def = inputs.WORKLOADS[args.workload]
-    decode = wl_def.T <= 8 and not args.dgrad and not args.w4a8
+    decode = wl_def.T <= 8 and not args.dgrad and not args.w4a8 and not args.w4a8x2
     steps = args.steps if args.steps is not None else (20000 if decode else 200)
     warmup = args.warmup if args.warmup is not None else (100 if decode else 10)
     warmup = max(warmup, 3)
@@ -487,7 +512,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     dev = f"cuda:{local}"
     torch.cuda.set_device(local)
     wl = Workload(args.workload, dev, seed=1234 + rank, build_host_copy=(rank == 0 and world == 1),
-                  swiglu=args.swiglu, dgrad=args.dgrad, w4a8=args.w4a8, fused_combine=args.fused_combine)
+                  swiglu=args.swiglu, dgrad=args.dgrad, w4a8=args.w4a8, fused_combine=args.fused_combine, w4a8x2=args.w4a8x2)
     decode = wl.decode
     wl.h_host = wl.h.cpu().view(torch.int16).numpy().view(np.uint16)
     stream = torch.cuda.current_stream()
@@ -610,7 +635,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
 
     peaks, peak_src = load_peaks()
     kern_file = "gemv.cu" if decode else ("dgrad.cu" if wl.dgrad else ("mx.cu" if wl.w4a8 else "gemm_tc.cu"))
-    kern_base = "gemv" if decode else ("dgrad_tc" if wl.dgrad else ("gemm_w4a8" if wl.w4a8 else "gemm_tc"))
+    kern_base = "gemv" if decode else ("dgrad_tc" if wl.dgrad else
+                                       ("gemm_w4a8x2" if wl.split else ("gemm_w4a8" if wl.w4a8 else "gemm_tc")))
     kern_key = f"{kern_base}_{wl.wl.fmt}{'_swiglu' if wl.swiglu else ''}:{args.workload}:{wl.p1.name}"
     sha = kernel_source_sha([kern_file, "common.cuh"])
     if decode:
@@ -631,6 +657,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
             pk = round(2 * pk, 1)
             pk_src = f"2 x bf16_tflops_sustained of {peak_src} (kind::mxf8f6f4 runs at the fp8 rate)"
         kname = (f"dgrad_tc_kernel<{wl.wl.fmt}> (dX of {wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.dgrad else
+                 f"gemm_w4a8_kernel<two-term> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.split else
                  f"gemm_w4a8_kernel ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.w4a8 else
                  f"gemm_tc_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})")
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk, "unit": "TFLOP/s",
@@ -650,9 +677,13 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": steps,
             "warmup": warmup, "ms_per_step": round(ms / steps, 6), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "e4m3 x e2m1 (fp32 accumulate)" if wl.w4a8 else "bf16", "data": "synthetic",
+            "vs_baseline": None,
+            "dtype": ("(e4m3 hi + e4m3 lo) x e2m1 (fp32 accumulate)" if wl.split else
+                      "e4m3 x e2m1 (fp32 accumulate)" if wl.w4a8 else "bf16"), "data": "synthetic",
             "config": dict(_config(wl.wl, world), **({"first_projection": "fused gate_up + SwiGLU"} if wl.swiglu else {}),
-                           **({"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if wl.w4a8 else {}),
+                           **({"activations": "two-term MXFP8 hi + lo (quantised every step; bf16-activation accuracy)"}
+                              if wl.split else
+                              {"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if wl.w4a8 else {}),
                            **({"combine": "in the second GEMV's epilogue"} if wl.fused_combine else {}),
                            **({"step": "backward: route + dgrad of both projections"} if wl.dgrad else {})),
             "roofline": roof, "cpu_baseline": cpu,
@@ -675,7 +706,7 @@ def run_reference(args, steps, warmup, world):
     import oracle
 
     wl_def = inputs.WORKLOADS[args.workload]
-    decode = wl_def.T <= 8 and not args.w4a8
+    decode = wl_def.T <= 8 and not args.w4a8 and not args.w4a8x2
     unit, _ = _unit(decode)
 
     class HostWL:
@@ -683,7 +714,8 @@ def run_reference(args, steps, warmup, world):
 
     h = HostWL()
     h.wl = wl_def
-    h.w4a8 = args.w4a8
+    h.w4a8 = args.w4a8 or args.w4a8x2
+    h.split = args.w4a8x2
     h.E, h.k, h.T = wl_def.E, wl_def.k, wl_def.T
     h.M = h.T * h.k
     h.p1, h.p2 = wl_def.projections[0], wl_def.projections[-1]
@@ -729,7 +761,9 @@ def run_reference(args, steps, warmup, world):
         "ms_per_step": round(dt * 1e3 / steps, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(_config(wl_def, world),
-                       **({"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if args.w4a8 else {})),
+                       **({"activations": "two-term MXFP8 hi + lo (quantised every step; bf16-activation accuracy)"}
+                          if args.w4a8x2 else
+                          {"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if args.w4a8 else {})),
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle",
                          "sample": f"each step: the full route + combine and the fp64 grouped GEMM of both "
