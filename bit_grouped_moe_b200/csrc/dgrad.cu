@@ -16,7 +16,7 @@
 // over the units.  Warp roles: 8 decode warps, a TMA producer, an MMA issuer
 // and 4 epilogue warps.  Packed weights and dY tiles stream through a 4-deep
 // TMA ring, block scales are staged in shared memory by the decode warps two
-// stages ahead, the decoded W^T is double-buffered and the accumulator too,
+// stages ahead, four decoded W^T tiles are in flight and two accumulators,
 // so copies, MMAs, decode and the epilogue of the previous unit overlap.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -32,6 +32,8 @@ constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kProdWarp = 8, kMmaWarp = 9, kEpiWarp0 = 10;
 constexpr int kThreads = (kEpiWarp0 + 4) * 32;  // 448
 constexpr int kRing = 4;                       // dY / packed-weight stages in flight
+constexpr int kTBuf = 4;                       // decoded W^T tiles in flight
+static_assert(kTBuf <= kRing, "a decoded tile is released through the ring's MMA-done barriers");
 constexpr int kBR = 128;                   // rows per unit (MMA M)
 constexpr int kBKt = 128;                  // k per unit (MMA N)
 constexpr int kBN = 64;                    // n per stage (four k-steps of 16)
@@ -42,17 +44,19 @@ constexpr int kTmemCols = 2 * kBKt;  // two accumulators
 
 struct DSmem {
   uint8_t y[kRing][kYBytes];  // dY tiles (1024-aligned for the 128-byte swizzle)
-  uint8_t t[2][kTBytes];      // decoded W^T tiles
+  uint8_t t[kTBuf][kTBytes];  // decoded W^T tiles
   uint8_t w[kRing][kWBytes];  // packed weight blocks
   uint32_t lut[kLut256Words];
   uint32_t sc[2][kBN][4];     // raw block scales of a stage: 64 rows x (2 NF4 | 4 MXFP4) blocks of the k tile
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
-  uint64_t full[kRing], mdone[kRing], decoded[2], accf[2], acce[2], drain;
+  uint64_t full[kRing], mdone[kRing], decoded[kTBuf], accf[2], acce[2], drain;
   uint32_t tmem_base;
   int abort;
 };
+
+static_assert(sizeof(DSmem) + 1024 <= 227 * 1024, "shared memory budget");
 
 struct DUnit {
   int e, kt, row0, rows;
@@ -123,8 +127,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.full[i], 1);
       mbar_init(&s.mdone[i], 1);
     }
+    for (int i = 0; i < kTBuf; ++i) mbar_init(&s.decoded[i], kDecThreads);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.decoded[i], kDecThreads);
       mbar_init(&s.accf[i], 1);
       mbar_init(&s.acce[i], 128);
     }
@@ -188,9 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(ab * kBKt);
         for (int sb = 0; sb < ns; ++sb, ++g) {
-          const int b = g % kRing, tb = g & 1;
+          const int b = g % kRing, tb = g % kTBuf;
           if (!(ok = mbar_wait(&s.full[b], (uint32_t)(g / kRing) & 1u, err, abort))) break;
-          if (!(ok = mbar_wait(&s.decoded[tb], (uint32_t)(g >> 1) & 1u, err, abort))) break;
+          if (!(ok = mbar_wait(&s.decoded[tb], (uint32_t)(g / kTBuf) & 1u, err, abort))) break;
           tc_fence_after();
           const uint32_t ya = smem_u32(s.y[b]), ta = smem_u32(s.t[tb]);
 #pragma unroll
@@ -257,13 +261,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g = 0;
     for (int u = blockIdx.x; u < U; u += gridDim.x) {
       for (int sb = 0; sb < ns; ++sb, ++g) {
-        const int b = g % kRing, tb = g & 1;
+        const int b = g % kRing, tb = g % kTBuf, sb2 = g & 1;  // sb2: scale buffer of this stage
         bool sv_b;
         const uint32_t sraw_b = scale_raw(sp, sv_b);
         sp = next(sp);
-        // this stage's packed weights have landed, and the MMAs of stage g-2 no longer read t[tb]
+        // this stage's packed weights have landed, and the MMAs of stage g-kTBuf no longer read t[tb]
         if (!*abort) mbar_wait(&s.full[b], (uint32_t)(g / kRing) & 1u, err, abort);
-        if (g >= 2 && !*abort) mbar_wait(&s.mdone[(g - 2) % kRing], (uint32_t)((g - 2) / kRing) & 1u, err, abort);
+        if (g >= kTBuf && !*abort)
+          mbar_wait(&s.mdone[(g - kTBuf) % kRing], (uint32_t)((g - kTBuf) / kRing) & 1u, err, abort);
         // item (kp, nb) = k pair kp (k = 2kp, 2kp+1 of the tile), n rows nb*8 .. nb*8+7
         const uint32_t wbase = smem_u32(s.w[b]);
         const uint32_t tbase = smem_u32(s.t[tb]);
@@ -276,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const uint32_t byte = lds_u8(wbase + (uint32_t)((nb * 8 + i) * (kBKt / 2) + kp));
-            pr[i] = bf16x2_mul(lut256_get(lut, byte, lane4, 0u), s.sc[tb][nb * 8 + i][bb]);
+            pr[i] = bf16x2_mul(lut256_get(lut, byte, lane4, 0u), s.sc[sb2][nb * 8 + i][bb]);
           }
           // row 2kp of W^T takes the low halves (even k), row 2kp+1 the high halves
           sts_u128(tbase + sw128_chunk(2 * kp, nb), prmt_b32(pr[0], pr[1], 0x5410u),
@@ -288,10 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();  // generic-proxy writes of t[tb] before the MMA reads them
         mbar_arrive(&s.decoded[tb]);
-        scale_store(tb ^ 1, sraw_a, sv_a);  // stage g+1
+        scale_store(sb2 ^ 1, sraw_a, sv_a);  // stage g+1
         sraw_a = sraw_b;
         sv_a = sv_b;
-        dec_barrier();  // sc[tb ^ 1] written, sc[tb] no longer read
+        dec_barrier();  // sc[sb2 ^ 1] written, sc[sb2] no longer read
       }
     }
   } else {
