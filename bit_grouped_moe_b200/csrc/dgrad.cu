@@ -362,15 +362,9 @@ int dgrad_tc_n_per_stage() { return kBN; }
 template <int FMT>
 static cudaError_t launch_dgrad_t(const CUtensorMap& tm_y, const CUtensorMap& tm_w, const GroupedArgs& p, int grid,
                                   cudaStream_t stream) {
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(dgrad_tc_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)dgrad_tc_smem_bytes());
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static std::atomic<bool> configured[64];
+  const cudaError_t e = set_smem_limit_once(dgrad_tc_kernel<FMT>, (int)dgrad_tc_smem_bytes(), configured);
+  if (e != cudaSuccess) return e;
   return launch_pdl(dgrad_tc_kernel<FMT>, dim3(grid), dim3(kThreads), dgrad_tc_smem_bytes(), stream, tm_y, tm_w, p);
 }
 

@@ -460,15 +460,9 @@ size_t gemm_tc_smem_bytes() { return sizeof(Smem) + 1024; }
 template <int FMT, bool SWI>
 cudaError_t launch_gemm_tc_t(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
                              const GroupedArgs& p, int grid, cudaStream_t stream) {
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<FMT, SWI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)gemm_tc_smem_bytes());
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static std::atomic<bool> configured[64];
+  const cudaError_t e = set_smem_limit_once(gemm_tc_kernel<FMT, SWI>, (int)gemm_tc_smem_bytes(), configured);
+  if (e != cudaSuccess) return e;
   return launch_pdl(gemm_tc_kernel<FMT, SWI>, dim3(grid), dim3(kThreads), gemm_tc_smem_bytes(), stream, tm_a,
                     tm_a_big, tm_w, p);
 }

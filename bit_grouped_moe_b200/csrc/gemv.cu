@@ -363,15 +363,9 @@ int gemv_grid(long long units, int num_sms) {
 
 template <int FMT, int MODE, bool CMB>
 static cudaError_t launch_gemv_t(const GroupedArgs& p, const CombineArgs& c, int grid, cudaStream_t stream) {
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, MODE, CMB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static std::atomic<bool> configured[64];
+  const cudaError_t e = set_smem_limit_once(gemv_kernel<FMT, MODE, CMB>, kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
   return launch_pdl(gemv_kernel<FMT, MODE, CMB>, dim3(grid), dim3(kThreads), (size_t)kSmemBytes, stream, p, c);
 }
 

@@ -8,6 +8,7 @@
 
 #include <cuda_bf16.h>
 
+#include <atomic>
 #include <utility>
 
 namespace gnf4 {
@@ -30,6 +31,21 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Raises a kernel's dynamic shared-memory limit to `bytes`, once per device
+// (`done` is the kernel's flag array; a racing second call is harmless, and
+// devices past 64 set the attribute on every call).
+template <typename Kernel>
+cudaError_t set_smem_limit_once(Kernel kernel, int bytes, std::atomic<bool> (&done)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool tracked = dev >= 0 && dev < 64;
+  if (tracked && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && tracked) done[dev].store(true, std::memory_order_release);
+  return e;
 }
 
 // Arguments of the grouped GEMM / GEMV kernels (device pointers).

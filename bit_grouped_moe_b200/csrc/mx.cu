@@ -559,15 +559,10 @@ int gemm_w4a8_small_box_rows() { return kBox; }
 template <bool SPLIT>
 static cudaError_t launch_gemm_w4a8_t(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
                                       const CUtensorMap& tm_w_tail, const MxArgs& p, int grid, cudaStream_t stream) {
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_w4a8_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)gemm_w4a8_smem_bytes(SPLIT));
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static std::atomic<bool> configured[64];
+  const cudaError_t e =
+      set_smem_limit_once(gemm_w4a8_kernel<SPLIT>, (int)gemm_w4a8_smem_bytes(SPLIT), configured);
+  if (e != cudaSuccess) return e;
   return launch_pdl(gemm_w4a8_kernel<SPLIT>, dim3(grid), dim3(kThreads), gemm_w4a8_smem_bytes(SPLIT), stream, tm_a,
                     tm_a_big, tm_w, tm_w_tail, p);
 }
