@@ -57,3 +57,30 @@ def test_reference_arm_nonzero_rank_exits(monkeypatch, capsys):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--steps", "1", "--warmup", "1"])
     assert bench.main() == 0
     assert capsys.readouterr().out == ""
+
+
+@pytest.mark.parametrize("extra", [[], ["--w4a8x2"]])
+def test_reference_arm_prints_one_contract_line(monkeypatch, capsys, extra):
+    """The oracle arm on CPU: one JSON line with the contract's keys, the
+    reference marker and its own cpu_baseline / e2e blocks."""
+    import json
+    import sys
+
+    import bench
+
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    wl = "tiny-nf4" if not extra else "gptoss-t1"
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", wl, "--steps", "1",
+                                      "--warmup", "1", *extra])
+    assert bench.main() == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["config"]["workload"].startswith(wl)
