@@ -65,6 +65,8 @@ def _load():
     lib.orc_dequant_mxfp8.argtypes = [P, P, I64, I64, P]
     lib.orc_grouped_gemm_w4a8.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P]
     lib.orc_quant_mxfp8_split.argtypes = [P, I64, I64, P, P, P, P]
+    lib.orc_quant_mxfp4_act.argtypes = [P, I64, I64, P, P]
+    lib.orc_grouped_gemm_w4a4.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P]
     lib.orc_grouped_gemm_w4a8x2.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, P, I64, P]
     _lib = lib
     return lib
@@ -338,4 +340,33 @@ def grouped_gemm_w4a8x2(hi_codes, hi_scales, lo_codes, lo_scales, w, w_scales, o
     y = np.empty((rows.shape[0], N), np.float64)
     _load().orc_grouped_gemm_w4a8x2(_p(hc), _p(hs), _p(lc), _p(ls), _p(w), _p(w_scales), _p(offsets), E, N, K,
                                     _p(rows), rows.shape[0], _p(y))
+    return y
+
+
+def quant_mxfp4_act(x_bits: np.ndarray):
+    """bf16 activations [..., K] -> MXFP4 (blocks [..., K/2] u8, scales [..., K/32] u8), OCP rule."""
+    x_bits = _c(x_bits, np.uint16)
+    K = x_bits.shape[-1]
+    if K % 32:
+        raise ValueError("MXFP4 needs K % 32 == 0")
+    rows = x_bits.size // K if K else 0
+    blocks = np.empty(x_bits.shape[:-1] + (K // 2,), np.uint8)
+    scales = np.empty(x_bits.shape[:-1] + (K // 32,), np.uint8)
+    _load().orc_quant_mxfp4_act(_p(x_bits), rows, K, _p(blocks), _p(scales))
+    return blocks, scales
+
+
+def grouped_gemm_w4a4(a_blocks, a_scales, w, w_scales, offsets, rows=None):
+    """fp64 Y[rows, N] of the native W4A4 mode: MXFP4 activations x MXFP4 weights."""
+    a_blocks, a_scales = _c(a_blocks, np.uint8), _c(a_scales, np.uint8)
+    w, w_scales = _c(w, np.uint8), _c(w_scales, np.uint8)
+    offsets = _c(offsets, np.int32)
+    E, N, K2 = w.shape
+    K = 2 * K2
+    if rows is None:
+        rows = np.arange(int(offsets[-1]), dtype=np.int64)
+    rows = _c(rows, np.int64)
+    y = np.empty((rows.shape[0], N), np.float64)
+    _load().orc_grouped_gemm_w4a4(_p(a_blocks), _p(a_scales), _p(w), _p(w_scales), _p(offsets), E, N, K, _p(rows),
+                                  rows.shape[0], _p(y))
     return y

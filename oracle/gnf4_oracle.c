@@ -717,3 +717,51 @@ void orc_grouped_gemm_w4a8x2(const uint8_t *hc, const uint8_t *hs, const uint8_t
     for (int64_t i = 0; i < n_rows * N; ++i) y[i] += yl[i];
     free(yl);
 }
+
+/* ------------------------------------------------------------------ */
+/* Native W4A4: MXFP4 activations x MXFP4 weights [W4A8] [OCP-MX]      */
+/* ------------------------------------------------------------------ */
+
+/* Quantise rows x K bf16 activations to MXFP4 (blocks [rows, K/2], element
+ * 2i in the low nibble; scales [rows, K/32] e8m0) by the same OCP rule as
+ * the weights (reading C8, applied to activations: reading C21). */
+void orc_quant_mxfp4_act(const uint16_t *x, int64_t rows, int64_t K, uint8_t *blocks, uint8_t *scales)
+{
+    float *xf = (float *)malloc((size_t)(rows * K > 0 ? rows * K : 1) * sizeof(float));
+    for (int64_t i = 0; i < rows * K; ++i) xf[i] = bf16_to_float(x[i]);
+    orc_quant_mxfp4(xf, rows, K, blocks, scales);
+    free(xf);
+}
+
+/* Native W4A4 grouped GEMM: y[i, n] = sum_k A[r, k] * W_e[n, k] with both
+ * operands MXFP4 (e2m1 x 2^(s-127)); every product and sum in fp64. */
+void orc_grouped_gemm_w4a4(const uint8_t *ab, const uint8_t *as, const uint8_t *w, const uint8_t *sw,
+                           const int32_t *offsets, int64_t E, int64_t N, int64_t K, const int64_t *rows,
+                           int64_t n_rows, double *y)
+{
+    float *wd = (float *)malloc((size_t)(N * K) * sizeof(float));
+    float *ad = (float *)malloc((size_t)K * sizeof(float));
+    for (int64_t e = 0; e < E; ++e) {
+        int used = 0;
+        for (int64_t i = 0; i < n_rows; ++i)
+            if (rows[i] >= offsets[e] && rows[i] < offsets[e + 1]) used = 1;
+        if (!used) continue;
+        orc_dequant_mxfp4(w + e * N * (K / 2), sw + e * N * (K / 32), N, K, wd);
+        for (int64_t i = 0; i < n_rows; ++i) {
+            if (!(rows[i] >= offsets[e] && rows[i] < offsets[e + 1])) continue;
+            orc_dequant_mxfp4(ab + rows[i] * (K / 2), as + rows[i] * (K / 32), 1, K, ad);
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+            for (int64_t n = 0; n < N; ++n) {
+                const float *wrow = wd + n * K;
+                double acc = 0.0;
+                for (int64_t kk = 0; kk < K; ++kk) acc += (double)ad[kk] * (double)wrow[kk];
+                y[i * N + n] = acc;
+            }
+        }
+    }
+    for (int64_t i = 0; i < n_rows; ++i)
+        if (!(rows[i] >= 0 && rows[i] < offsets[E]))
+            for (int64_t n = 0; n < N; ++n) y[i * N + n] = NAN;
+    free(ad);
+    free(wd);
+}

@@ -750,3 +750,72 @@ def test_w4a8x2_gemm_meets_the_bf16_activation_tolerance():
     y_hi = oracle.grouped_gemm_w4a8(hc, hs, w, sw, offsets)
     y_lo = oracle.grouped_gemm_w4a8(lc, ls, w, sw, offsets)
     assert np.allclose(y2, y_hi + y_lo, rtol=1e-14, atol=1e-12)
+
+
+# ---------------------------------------------------------------- native W4A4 (MXFP4 activations)
+
+
+def test_mxfp4_act_quantiser_is_the_weight_quantiser_on_bf16():
+    """The activation quantiser is the pinned MXFP4 weight quantiser applied to
+    the (exact) fp32 value of each bf16."""
+    rng = inputs.rng(91)
+    bits = inputs.bf16_normal(rng, (24, 256))
+    b1, s1 = oracle.quant_mxfp4_act(bits)
+    b2, s2 = oracle.quant_mxfp4(_af(bits).astype(np.float32))
+    assert np.array_equal(b1, b2) and np.array_equal(s1, s2)
+
+
+def test_w4a4_gemm_is_numpy_matmul_of_the_dequantised_operands():
+    rng = inputs.rng(92)
+    E, N, K = 3, 16, 256
+    offsets = np.array([0, 5, 5, 11], np.int32)
+    w, sw = inputs.mxfp4_random(rng, E, N, K)
+    ab, as_ = oracle.quant_mxfp4_act(inputs.bf16_normal(rng, (11, K)))
+    y = oracle.grouped_gemm_w4a4(ab, as_, w, sw, offsets)
+    ad = oracle.dequant_mxfp4(ab, as_).astype(np.float64)
+    for e in range(E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        if r1 == r0:
+            continue
+        wd = oracle.dequant_mxfp4(w[e], sw[e]).astype(np.float64)
+        assert np.allclose(y[r0:r1], ad[r0:r1] @ wd.T, rtol=1e-13, atol=1e-13)
+
+
+def test_w4a4_gemm_closed_form():
+    """Activation codes 0x22 (1.0, 1.0) with scale 2^s and weights 1.0 with
+    scale 2^t: every output is K * 2^(s + t)."""
+    E, N, K = 2, 8, 256
+    offsets = np.array([0, 2, 3], np.int32)
+    ab = np.full((3, K // 2), 0x22, np.uint8)
+    as_ = np.full((3, K // 32), 127, np.uint8)
+    as_[2] = 125
+    w = np.full((E, N, K // 2), 0x22, np.uint8)
+    sw = np.full((E, N, K // 32), 128, np.uint8)
+    y = oracle.grouped_gemm_w4a4(ab, as_, w, sw, offsets)
+    assert np.all(y[:2] == 2 * K) and np.all(y[2] == K * 2.0 ** (1 - 2))
+
+
+def test_w4a4_stays_within_the_e2m1_bound_of_the_bf16_activation_result():
+    """e2m1 rounds to nearest with one mantissa bit.  After division by the
+    block scale 2^X, a value of at least 0.5 moves by at most 1/5 of itself
+    (1/4 when saturated at 6 from below 8), and a smaller one by at most 0.25
+    (it lands on 0 or 0.5).  So |a - q(a)| <= |a|/3 + 2^(X-2) for every
+    activation, which bounds |Y_w4a4 - Y_bf16|.  The rms error is far larger
+    than the e4m3 mode's."""
+    rng = inputs.rng(93)
+    E, N, K = 2, 16, 512
+    offsets = np.array([0, 6, 9], np.int32)
+    w, sw = inputs.mxfp4_random(rng, E, N, K)
+    a = inputs.bf16_normal(rng, (9, K))
+    ab, as_ = oracle.quant_mxfp4_act(a)
+    y4 = oracle.grouped_gemm_w4a4(ab, as_, w, sw, offsets)
+    y16 = oracle.grouped_gemm_mxfp4(a, w, sw, offsets)
+    af = np.abs(_af(a))
+    err_a = af / 3 + np.exp2(as_.astype(np.float64) - 127.0 - 2.0).repeat(32, axis=1)
+    assert np.all(np.abs(oracle.dequant_mxfp4(ab, as_).astype(np.float64) - _af(a)) <= err_a)
+    for e in range(E):
+        r0, r1 = offsets[e], offsets[e + 1]
+        wd = np.abs(oracle.dequant_mxfp4(w[e], sw[e]).astype(np.float64))
+        assert np.all(np.abs(y4[r0:r1] - y16[r0:r1]) <= err_a[r0:r1] @ wd.T)
+    rel = np.linalg.norm(y4 - y16) / np.linalg.norm(y16)
+    assert 0.04 < rel < 0.2, rel
