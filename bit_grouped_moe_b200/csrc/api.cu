@@ -330,8 +330,7 @@ gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, c
     for (int big = 0; big < 2; ++big) {
       // single term: 32- and 128-row boxes of the codes; two terms: 32-row boxes of hi and of lo
       const uint8_t* src = (split && big) ? lo_codes : a_codes;
-      cuuint32_t box[2] = {128, (cuuint32_t)((big && !split) ? gemm_w4a8_rows_per_unit(false)
-                                                             : gemm_w4a8_small_box_rows())};
+      cuuint32_t box[2] = {128, (cuuint32_t)((big && !split) ? gemm_mx_rows_per_unit(0) : gemm_mx_small_box_rows())};
       CUresult r = fn(big ? &tm_a_big : &tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(src), dims,
                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -339,7 +338,7 @@ gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, c
     }
   }
   const cuuint64_t rows = (cuuint64_t)E * (cuuint64_t)N, rb = (cuuint64_t)(K / 2);
-  const cuuint32_t wrows = (cuuint32_t)gemm_w4a8_weight_rows_per_unit();
+  const cuuint32_t wrows = (cuuint32_t)gemm_mx_weight_rows_per_unit();
   {
     cuuint64_t dims[3] = {128, (cuuint64_t)(K / 128), rows};
     cuuint64_t strides[2] = {64, rb};
@@ -363,14 +362,72 @@ gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, c
     tm_w_tail = tm_w;  // never used
   }
   const long long nwt = (N + (long long)wrows - 1) / wrows;
-  const long long rpu = gemm_w4a8_rows_per_unit(split);
+  const long long rpu = gemm_mx_rows_per_unit(split ? 1 : 0);
   const long long units = ((M + rpu - 1) / rpu + (E < M ? E : M)) * nwt;
   if (units >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d, N=%d give too many work units", M, N);
   const int grid = (int)(units < d->num_sms ? units : d->num_sms);
-  cudaError_t e = launch_gemm_w4a8(tm_a, tm_a_big, tm_w, tm_w_tail, a_scales, split ? lo_scales : nullptr,
-                                   w_scales, offsets, counts, static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M,
-                                   grid, as_stream(stream));
+  cudaError_t e = launch_gemm_mx(split ? 1 : 0, tm_a, tm_a_big, tm_w, tm_w_tail, a_scales,
+                                 split ? lo_scales : nullptr, w_scales, offsets, counts,
+                                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "W4A8 grouped GEMM launch");
+  return GNF4_OK;
+}
+
+// Native W4A4 GEMM: both operands packed e2m1 bytes by TMA (128-byte swizzled boxes of 256 codes).
+gnf4_status grouped_gemm_w4a4(const uint8_t* a_blocks, const uint8_t* a_scales, const uint8_t* w,
+                              const uint8_t* w_scales, const int32_t* offsets, const int32_t* counts, int E, int N,
+                              int K, int M, void* y, void* stream) {
+  if (E < 1 || E > kMaxExperts) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "E=%d outside [1, %d]", E, kMaxExperts);
+  if (N < 1 || N % 8 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N=%d must be a positive multiple of 8", N);
+  if (K < 256 || K % 64 != 0 || K > 65536)
+    return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K=%d must be a multiple of 64 in [256, 65536] for W4A4", K);
+  if (M < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d is negative", M);
+  if ((long long)E * N >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "E*N too large");
+  if ((offsets == nullptr) == (counts == nullptr))
+    return fail(GNF4_ERR_INVALID_ARG, "pass exactly one of offsets [E+1] and counts [E]");
+  if (M == 0) return GNF4_OK;
+  GNF4_TRY(check_ptr(a_blocks, "a_blocks", 16));
+  GNF4_TRY(check_ptr(a_scales, "a_scales", 2));
+  GNF4_TRY(check_ptr(w, "w", 16));
+  GNF4_TRY(check_ptr(w_scales, "w_scales", 2));
+  GNF4_TRY(check_ptr(offsets, "offsets", 4, false));
+  GNF4_TRY(check_ptr(counts, "counts", 4, false));
+  GNF4_TRY(check_ptr(y, "y", 16));
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  auto fn = encode_fn();
+  if (!fn) return fail(GNF4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  CUtensorMap tm_a, tm_a_big, tm_w;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t estr[2] = {1, 1};
+    for (int big = 0; big < 2; ++big) {
+      cuuint32_t box[2] = {128, (cuuint32_t)(big ? gemm_mx_rows_per_unit(2) : gemm_mx_small_box_rows())};
+      CUresult r = fn(big ? &tm_a_big : &tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a_blocks), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(GNF4_ERR_CUDA, "e2m1 activation tensor map encode failed (CUresult %d)", (int)r);
+    }
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)N, (cuuint64_t)E};
+    cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)N * (cuuint64_t)(K / 2)};
+    cuuint32_t box[3] = {128, (cuuint32_t)gemm_mx_weight_rows_per_unit(), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(w), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(GNF4_ERR_CUDA, "e2m1 weight tensor map encode failed (CUresult %d)", (int)r);
+  }
+  const long long nwt = (N + (long long)gemm_mx_weight_rows_per_unit() - 1) / gemm_mx_weight_rows_per_unit();
+  const long long rpu = gemm_mx_rows_per_unit(2);
+  const long long units = ((M + rpu - 1) / rpu + (E < M ? E : M)) * nwt;
+  if (units >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d, N=%d give too many work units", M, N);
+  const int grid = (int)(units < d->num_sms ? units : d->num_sms);
+  cudaError_t e = launch_gemm_mx(2, tm_a, tm_a_big, tm_w, tm_w, a_scales, nullptr, w_scales, offsets, counts,
+                                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M, grid, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "W4A4 grouped GEMM launch");
   return GNF4_OK;
 }
 
@@ -624,6 +681,27 @@ gnf4_status gnf4_grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scal
                                    const uint8_t* w_scales, const int32_t* offsets, const int32_t* counts, int E,
                                    int N, int K, int M, void* y, void* stream) {
   return grouped_gemm_w4a8(a_codes, a_scales, nullptr, nullptr, w, w_scales, offsets, counts, E, N, K, M, y, stream);
+}
+
+gnf4_status gnf4_quantize_mxfp4_act(const void* x, int M, int K, uint8_t* blocks, uint8_t* scales, void* stream) {
+  if (M < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d is negative", M);
+  if (K < 32 || K % 32 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K=%d must be a positive multiple of 32", K);
+  if (M == 0) return GNF4_OK;
+  GNF4_TRY(check_ptr(x, "x", 16));
+  GNF4_TRY(check_ptr(blocks, "blocks", 4));
+  GNF4_TRY(check_ptr(scales, "scales", 1));
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  cudaError_t e = launch_quant_mxfp4_act(static_cast<const __nv_bfloat16*>(x), (long long)M * K, blocks, scales,
+                                         as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "MXFP4 activation quantiser launch");
+  return GNF4_OK;
+}
+
+gnf4_status gnf4_grouped_gemm_w4a4(const uint8_t* a_blocks, const uint8_t* a_scales, const uint8_t* w,
+                                   const uint8_t* w_scales, const int32_t* offsets, const int32_t* counts, int E,
+                                   int N, int K, int M, void* y, void* stream) {
+  return grouped_gemm_w4a4(a_blocks, a_scales, w, w_scales, offsets, counts, E, N, K, M, y, stream);
 }
 
 gnf4_status gnf4_quantize_mxfp8_split(const void* x, int M, int K, uint8_t* hi_codes, uint8_t* hi_scales,

@@ -97,21 +97,27 @@ int dgrad_tc_rows_per_unit();
 int dgrad_tc_k_per_unit();
 int dgrad_tc_n_per_stage();
 
-// mx.cu: native W4A8 (MXFP8 activations x MXFP4 weights, kind::mxf8f6f4)
+// mx.cu: native block-scaled MXFP4 modes.  mode 0 = W4A8 (MXFP8 activations,
+// kind::mxf8f6f4), 1 = two-term MXFP8 (hi + lo), 2 = W4A4 (MXFP4 activations,
+// kind::mxf4).
 // lo_codes / lo_scales non-null: the two-term split (hi into codes / scales)
 cudaError_t launch_quant_mxfp8(const __nv_bfloat16* x, long long elems, uint8_t* codes, uint8_t* scales,
                                uint8_t* lo_codes, uint8_t* lo_scales, cudaStream_t stream);
-// tm_a / tm_a_big: e4m3 codes [M, K] in 128 x 32 / 128 x 128 boxes; tm_w: the [E*N] x (K/128) x 128-code
-// view of the e2m1 stack; tm_w_tail: codes [K-128, K) of every row (used when K % 128 == 64).
-// lo_scales non-null: the two-term mode; tm_a = hi codes, tm_a_big = lo codes, both in 128 x 32 boxes.
-cudaError_t launch_gemm_w4a8(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
-                             const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* lo_scales,
-                             const uint8_t* w_scales, const int* offsets, const int* counts, __nv_bfloat16* y,
-                             unsigned* err, int E, int N, int K, int M, int grid, cudaStream_t stream);
-size_t gemm_w4a8_smem_bytes(bool split);
-int gemm_w4a8_rows_per_unit(bool split);
-int gemm_w4a8_weight_rows_per_unit();
-int gemm_w4a8_small_box_rows();
+cudaError_t launch_quant_mxfp4_act(const __nv_bfloat16* x, long long elems, uint8_t* blocks, uint8_t* scales,
+                                   cudaStream_t stream);
+// Modes 0 / 2: tm_a / tm_a_big = the activation codes in 32- / 128-row boxes of 128 bytes; mode 1: tm_a = hi
+// codes, tm_a_big = lo codes, both in 32-row boxes.  tm_w: modes 0 / 1 the [E*N] x (K/128) x 128-code view of
+// the e2m1 stack in 16-byte slots, tm_w_tail its codes [K-128, K) (K % 128 == 64); mode 2 the [E, N, K/2] bytes
+// in 128-byte x 128-row boxes.
+cudaError_t launch_gemm_mx(int mode, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
+                           const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* lo_scales,
+                           const uint8_t* w_scales, const int* offsets, const int* counts, __nv_bfloat16* y,
+                           unsigned* err, int E, int N, int K, int M, int grid, cudaStream_t stream);
+size_t gemm_mx_smem_bytes(int mode);
+int gemm_mx_rows_per_unit(int mode);
+int gemm_mx_k_per_stage(int mode);
+int gemm_mx_weight_rows_per_unit();
+int gemm_mx_small_box_rows();
 
 // route.cu
 size_t route_workspace_bytes(int T, int k, int E);

@@ -158,46 +158,100 @@ __global__ void __launch_bounds__(kQThreads) quant_mxfp8_kernel(const __nv_bfloa
   }
 }
 
+// MXFP4 activations (the W4A4 mode): the OCP rule of the weights, exponent
+// floor(log2(amax)) - 2, e2m1 round to nearest even saturating at +-6,
+// element 2i in the low nibble.  One thread packs 8 k into 4 bytes.
+__global__ void __launch_bounds__(kQThreads) quant_mxfp4_act_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                    long long octets, uint8_t* __restrict__ blocks,
+                                                                    uint8_t* __restrict__ scales) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const long long o = (long long)blockIdx.x * kQThreads + threadIdx.x;
+  const bool ok = o < octets;
+  const uint4 v = ok ? ldg_nc_u128(x + o * 8) : make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  const int ef = (int)(m >> 7);
+  const int X = ef == 0 ? -127 : max(ef - 127 - 2, -127);
+  const float inv = __uint_as_float((uint32_t)(127 - X) << 23);
+  float xv[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    xv[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), inv);
+    xv[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv);
+  }
+  uint32_t packed;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(packed)
+      : "f"(xv[0]), "f"(xv[1]), "f"(xv[2]), "f"(xv[3]), "f"(xv[4]), "f"(xv[5]), "f"(xv[6]), "f"(xv[7]));
+  if (ok) {
+    reinterpret_cast<uint32_t*>(blocks)[o] = packed;
+    if ((threadIdx.x & 3) == 0) scales[o >> 2] = (uint8_t)(X + 127);
+  }
+}
+
 // ------------------------------------------------------------------ GEMM
 
-// Geometry of the two modes.  SPLIT (two-term activations): a unit takes at
-// most 96 rows of a group; its B operand stacks the hi rows of the chunk
-// (nbx = ceil(rows / 32) boxes of 32 rows) over the lo rows (nbx more
-// boxes), so one MMA with N = 64 * nbx multiplies both terms, and the
-// epilogue adds the two halves of the accumulator.
-template <bool SPLIT>
+// Modes of the native kernel:
+//   kW4A8  MXFP8 activations x MXFP4 weights, kind::mxf8f6f4 (K = 32 per MMA)
+//   kSplit two-term MXFP8 activations: a unit takes at most 96 rows of a
+//          group; its B operand stacks the hi rows (nbx = ceil(rows / 32)
+//          boxes of 32 rows) over the lo rows (nbx more boxes), so one MMA
+//          with N = 64 * nbx multiplies both terms and the epilogue adds the
+//          two halves of the accumulator
+//   kW4A4  MXFP4 activations x MXFP4 weights, kind::mxf4 (K = 64 per MMA,
+//          both operands packed two codes per byte; two scale bytes per row
+//          per MMA)
+constexpr int kW4A8 = 0, kSplit = 1, kW4A4 = 2;
+
+template <int MODE>
 struct Geo {
-  static constexpr int kBT = SPLIT ? 96 : 128;          // rows (tokens) per unit
-  static constexpr int kStages = SPLIT ? 5 : 6;
-  static constexpr int kAccW = SPLIT ? 192 : 128;       // accumulator columns per buffer
-  static constexpr int kARows = SPLIT ? 192 : 128;      // activation rows per stage in shared memory
-  static constexpr int kSfaWords = SPLIT ? 256 : 128;   // activation scale words per stage
-  static constexpr int kSfCols = SPLIT ? 12 : 8;        // TMEM scale columns per stage
+  static constexpr int kBT = MODE == kSplit ? 96 : 128;         // rows (tokens) per unit
+  static constexpr int kBK = MODE == kW4A4 ? 256 : 128;         // k per stage (128-byte rows in shared memory)
+  static constexpr int kMmaK = MODE == kW4A4 ? 64 : 32;         // k per MMA
+  static constexpr int kStages = MODE == kSplit ? 5 : 6;
+  static constexpr int kAccW = MODE == kSplit ? 192 : 128;      // accumulator columns per buffer
+  static constexpr int kARows = MODE == kSplit ? 192 : 128;     // activation rows per stage in shared memory
+  static constexpr int kSfBlocks = MODE == kW4A4 ? 2 : 1;       // 4-scale blocks per row per stage
+  static constexpr int kSfwWords = 128 * kSfBlocks;             // weight scale words per stage
+  static constexpr int kSfaWords = MODE == kSplit ? 256 : 128 * kSfBlocks;  // activation scale words per stage
+  static constexpr int kSfCols = 4 * (kSfwWords + kSfaWords) / 128;        // TMEM scale columns per stage
 };
 
 constexpr int kBW = 128;  // weight rows per unit = MMA M
-constexpr int kBK = 128;  // k per stage
 constexpr int kBox = 32;  // activation rows per small TMA box
 constexpr int kEpiWarp0 = 4;
 constexpr int kProd2 = 12;  // second TMA producer warp
 constexpr int kThreads = 13 * 32;
-constexpr int kWStageBytes = kBW * kBK;   // padded e2m1 in shared memory: one byte per code
-constexpr int kWStageTx = kBW * kBK / 2;  // bytes the TMA reads: two codes per byte
+constexpr int kWStageBytes = kBW * 128;  // one 128-byte row per weight row and stage
 constexpr int kTmemCols = 512;
 
+// bytes the TMA delivers for a stage's weights: packed codes, two per byte
+template <int MODE>
+constexpr int w_stage_tx() { return kBW * Geo<MODE>::kBK / 2; }
+
 // scale-loader index of a warp (its ring slot), or -1: warps 2, 3, 8, 9, ...
-template <bool SPLIT>
+template <int MODE>
 __device__ __forceinline__ int loader_index(int warp) {
-  return warp == 2 || warp == 3 ? warp - 2 : (warp >= 8 && warp < 8 + Geo<SPLIT>::kStages - 2 ? warp - 6 : -1);
+  return warp == 2 || warp == 3 ? warp - 2 : (warp >= 8 && warp < 8 + Geo<MODE>::kStages - 2 ? warp - 6 : -1);
 }
 
-template <bool SPLIT>
+template <int MODE>
 struct MxSmem {
-  using G = Geo<SPLIT>;
+  using G = Geo<MODE>;
   uint8_t w[G::kStages][kWStageBytes];  // 1024-aligned (offset 0)
-  uint8_t a[G::kStages][G::kARows * kBK];
-  uint32_t sfw[G::kStages][kBW];        // weight scales of the stage, tcgen05.cp layout
-  uint32_t sfa[G::kStages][G::kSfaWords];  // activation scales of the stage (two 128-row blocks in SPLIT)
+  uint8_t a[G::kStages][G::kARows * 128];
+  uint32_t sfw[G::kStages][G::kSfwWords];  // weight scales of the stage, tcgen05.cp layout
+  uint32_t sfa[G::kStages][G::kSfaWords];  // activation scales of the stage
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
@@ -208,15 +262,18 @@ struct MxSmem {
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(MxSmem<false>) + 1024 <= 227 * 1024, "shared memory budget");
-static_assert(sizeof(MxSmem<true>) + 1024 <= 227 * 1024, "shared memory budget");
-static_assert(2 * Geo<false>::kAccW + Geo<false>::kSfCols * Geo<false>::kStages <= kTmemCols, "TMEM budget");
-static_assert(2 * Geo<true>::kAccW + Geo<true>::kSfCols * Geo<true>::kStages <= kTmemCols, "TMEM budget");
-static_assert(Geo<false>::kStages <= 6 && Geo<true>::kStages <= 6, "scale loaders are warps 2, 3, 8..11");
+#define GNF4_MX_CHECK(M)                                                                               \
+  static_assert(sizeof(MxSmem<M>) + 1024 <= 227 * 1024, "shared memory budget");                       \
+  static_assert(2 * Geo<M>::kAccW + Geo<M>::kSfCols * Geo<M>::kStages <= kTmemCols, "TMEM budget");    \
+  static_assert(Geo<M>::kStages <= 6, "scale loaders are warps 2, 3, 8..11");
+GNF4_MX_CHECK(kW4A8)
+GNF4_MX_CHECK(kSplit)
+GNF4_MX_CHECK(kW4A4)
+#undef GNF4_MX_CHECK
 
 struct MxArgs {
-  const uint8_t* sa;   // activation scales e8m0 [M, K/32] (SPLIT: of the hi term; the codes come by TMA)
-  const uint8_t* sl;   // SPLIT: lo-term scales [M, K/32]
+  const uint8_t* sa;   // activation scales e8m0 [M, K/32] (kSplit: of the hi term; the codes come by TMA)
+  const uint8_t* sl;   // kSplit: lo-term scales [M, K/32]
   const uint8_t* sw;   // e8m0 [E, N, K/32]
   const int* offsets;  // [E+1] or null
   const int* counts;   // [E] or null
@@ -229,14 +286,14 @@ struct Unit {
   int e, j, row0, rows;
 };
 
-// Partial accumulators per unit (single-term mode): the K=32 steps of a unit
-// of at most 32 (64) rows rotate over 4 (2) accumulators of 32 (64) columns;
+// Partial accumulators per unit (single-term modes): the MMAs of a unit of
+// at most 32 (64) rows rotate over 4 (2) accumulators of 32 (64) columns;
 // the epilogue adds them in a fixed order.
 __device__ __forceinline__ int acc_split(int rows) { return rows <= 32 ? 4 : (rows <= 64 ? 2 : 1); }
 
-template <bool SPLIT>
-__device__ __forceinline__ Unit unit_of(const MxSmem<SPLIT>& s, int E, int u) {
-  constexpr int kBT = Geo<SPLIT>::kBT;
+template <int MODE>
+__device__ __forceinline__ Unit unit_of(const MxSmem<MODE>& s, int E, int u) {
+  constexpr int kBT = Geo<MODE>::kBT;
   Unit x;
   x.e = find_group(s.upre, E, u);
   const int local = u - s.upre[x.e];
@@ -266,19 +323,31 @@ __device__ __forceinline__ void tc_copy_scales(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-// Instruction descriptor: kind::mxf8f6f4, A = e2m1, B = e4m3, e8m0 scales,
-// both K-major, M = 128, N = n (multiple of 16), K = 32; scale-factor ids
-// (the byte of the scale column) j for both operands.
-__device__ __forceinline__ uint32_t idesc_w4a8(uint32_t n, uint32_t j) {
-  return (j << 4) | (5u << 7) | (0u << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) | (j << 29);
+// Instruction descriptor of a block-scaled MMA: operand formats fa / fb, e8m0
+// scales, both K-major, M = 128, N = n (multiple of 16); scale-factor ids sf
+// (the first byte of the MMA's scales inside their 32-bit TMEM column).
+__device__ __forceinline__ uint32_t idesc_mx(uint32_t fa, uint32_t fb, uint32_t n, uint32_t sf) {
+  return (sf << 4) | (fa << 7) | (fb << 10) | ((n >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) | (sf << 29);
 }
 
-__device__ __forceinline__ void tc_mma_w4a8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+// A = e2m1 (format 5), B = e4m3 (format 0), K = 32.
+__device__ __forceinline__ void tc_mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// A = B = e2m1 (format 1), packed, K = 64, one e8m0 scale per 32 k.
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
@@ -293,18 +362,22 @@ __device__ __forceinline__ void sts_u128(uint32_t addr, uint32_t a, uint32_t b, 
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// Single-term mode: tm_a / tm_a_big are the e4m3 codes in 32- / 128-row
-// boxes.  SPLIT: tm_a = hi codes, tm_a_big = lo codes, both in 32-row boxes.
-template <bool SPLIT>
+// kW4A8 / kW4A4: tm_a / tm_a_big are the activation codes in 32- / 128-row
+// boxes (kW4A4: packed bytes).  kSplit: tm_a = hi codes, tm_a_big = lo codes,
+// both in 32-row boxes.  tm_w: kW4A8 / kSplit the [E*N] x (K/128) x 128-code
+// view expanded to 16-byte slots (16U4_ALIGN16B), tm_w_tail the codes
+// [K-128, K) of every row; kW4A4 the [E, N, K/2] bytes in 128-byte boxes.
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_w4a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_big,
-                     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_w_tail,
-                     MxArgs p) {
-  using G = Geo<SPLIT>;
+    gemm_mx_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_big,
+                   const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_w_tail,
+                   MxArgs p) {
+  using G = Geo<MODE>;
   constexpr int kStages = G::kStages;
+  constexpr bool SPLIT = MODE == kSplit;
   extern __shared__ uint8_t smem_raw[];
-  MxSmem<SPLIT>& s =
-      *reinterpret_cast<MxSmem<SPLIT>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  MxSmem<MODE>& s =
+      *reinterpret_cast<MxSmem<MODE>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   unsigned* err = p.err;
   volatile int* abort = &s.abort;
@@ -318,8 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int U = s.upre[p.E];
   if ((int)blockIdx.x >= U) return;  // uniform over the block
   const int K = p.K;
-  const int nk = (K + kBK - 1) / kBK;
-  const bool tail = (K % kBK) != 0;  // K % 128 == 64
+  const int nk = (K + G::kBK - 1) / G::kBK;
+  // the last stage reads [K - kBK, K) and skips the MMAs already covered
+  auto stage_k0 = [&](int kt) { return min(kt * G::kBK, K - G::kBK); };
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -358,31 +432,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-        const Unit x = unit_of<SPLIT>(s, p.E, u);
+        const Unit x = unit_of<MODE>(s, p.E, u);
         const bool big = x.rows > kBox;
-        const int nbx = (x.rows + kBox - 1) / kBox;  // SPLIT: 32-row boxes per term
+        const int nbx = (x.rows + kBox - 1) / kBox;  // kSplit: 32-row boxes per term
         const int wrow = x.e * p.N + x.j * kBW;
         for (int kt = 0; kt < nk; ++kt, ++it) {
           if ((it & 1) != pi) continue;
           const int st = it % kStages, use = it / kStages;
           if (it >= kStages && !(ok = mbar_wait(&s.empty[st], (use - 1) & 1, err, abort))) break;
-          const bool last_tail = tail && kt == nk - 1;
-          const int k0 = last_tail ? K - kBK : kt * kBK;
-          if (SPLIT)
-            mbar_arrive_expect_tx(&s.full[st], kWStageTx + 2 * nbx * kBox * kBK);
-          else
-            mbar_arrive_expect_tx(&s.full[st], kWStageTx + (big ? G::kBT : kBox) * kBK);
-          if (last_tail)
+          const int k0 = stage_k0(kt);
+          const int abytes = SPLIT ? 2 * nbx * kBox * 128 : (big ? G::kBT : kBox) * 128;
+          mbar_arrive_expect_tx(&s.full[st], w_stage_tx<MODE>() + abytes);
+          if (MODE == kW4A4)
+            tma_load_3d(s.w[st], &tm_w, &s.full[st], k0 / 2, x.j * kBW, x.e);
+          else if (k0 != kt * G::kBK)
             tma_load_2d(s.w[st], &tm_w_tail, &s.full[st], 0, wrow);
           else
             tma_load_3d(s.w[st], &tm_w, &s.full[st], 0, kt, wrow);
+          const int ax = MODE == kW4A4 ? k0 / 2 : k0;  // activation bytes: packed in kW4A4
           if (SPLIT) {
             for (int b = 0; b < nbx; ++b) {
-              tma_load_2d(s.a[st] + b * kBox * kBK, &tm_a, &s.full[st], k0, x.row0 + b * kBox);
-              tma_load_2d(s.a[st] + (nbx + b) * kBox * kBK, &tm_a_big, &s.full[st], k0, x.row0 + b * kBox);
+              tma_load_2d(s.a[st] + b * kBox * 128, &tm_a, &s.full[st], ax, x.row0 + b * kBox);
+              tma_load_2d(s.a[st] + (nbx + b) * kBox * 128, &tm_a_big, &s.full[st], ax, x.row0 + b * kBox);
             }
           } else {
-            tma_load_2d(s.a[st], big ? &tm_a_big : &tm_a, &s.full[st], k0, x.row0);
+            tma_load_2d(s.a[st], big ? &tm_a_big : &tm_a, &s.full[st], ax, x.row0);
           }
         }
       }
@@ -390,52 +464,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = max(0, it - kStages); i < it; ++i)
           if ((i & 1) == pi) mbar_drain(&s.full[i % kStages], (i / kStages) & 1);
     }
-  } else if (loader_index<SPLIT>(warp) >= 0) {
+  } else if (loader_index<MODE>(warp) >= 0) {
     // ------------------------------------------------------------ scale loaders
     // Loader i fills ring slot i only.  Lane l serves rows l + 32c of the
     // weight tile (c < 4) and of the activation operand (c < 4, or < 8 for the
-    // stacked hi / lo rows of SPLIT); rows outside the tile or the group get
-    // scale 2^0 (their products are never stored).
-    const int li = loader_index<SPLIT>(warp);
+    // stacked hi / lo rows of kSplit); per row it copies 4 scale bytes per
+    // 4-scale block of the stage (kW4A4: two blocks).  Rows outside the tile
+    // or the group get scale 2^0 (their products are never stored).
+    const int li = loader_index<MODE>(warp);
     const int nsb = K / 32;
     const uint8_t* swb = p.sw;
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-      const Unit x = unit_of<SPLIT>(s, p.E, u);
-      const int hrows = kBox * ((x.rows + kBox - 1) / kBox);  // SPLIT: hi rows of the stacked operand
+      const Unit x = unit_of<MODE>(s, p.E, u);
+      const int hrows = kBox * ((x.rows + kBox - 1) / kBox);  // kSplit: hi rows of the stacked operand
       for (int kt = 0; kt < nk; ++kt, ++it) {
         const int st = it % kStages, use = it / kStages;
         if (st != li) continue;
         if (it >= kStages && !(ok = mbar_wait(&s.empty[st], (use - 1) & 1, err, abort))) break;
-        const int b0 = ((tail && kt == nk - 1) ? K - kBK : kt * kBK) / 32;  // even: K % 64 == 0
-        uint32_t wv[4], av[G::kSfaWords / 32];
+        const int b0 = stage_k0(kt) / 32;  // even: K % 64 == 0
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int n = x.j * kBW + lane + 32 * c;
-          wv[c] = n < p.N ? ld_scales4(swb + ((size_t)x.e * p.N + (size_t)n) * (size_t)nsb + b0) : 0x7F7F7F7Fu;
+        for (int bl = 0; bl < G::kSfBlocks; ++bl) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int n = x.j * kBW + lane + 32 * c;
+            wv[c] = n < p.N ? ld_scales4(swb + ((size_t)x.e * p.N + (size_t)n) * (size_t)nsb + b0 + 4 * bl)
+                            : 0x7F7F7F7Fu;
+          }
+          sts_u128(smem_u32(&s.sfw[st][bl * 128 + lane * 4]), wv[0], wv[1], wv[2], wv[3]);
         }
+        constexpr int kARowsSf = SPLIT ? 256 : 128;  // activation rows with a scale block
 #pragma unroll
-        for (int c = 0; c < G::kSfaWords / 32; ++c) {
-          const int m = lane + 32 * c;
-          const bool lo_row = SPLIT && m >= hrows;
-          const int rr = lo_row ? m - hrows : m;
-          const uint8_t* src = lo_row ? p.sl : p.sa;
-          av[c] = rr < x.rows ? ld_scales4(src + (size_t)(x.row0 + rr) * (size_t)nsb + b0) : 0x7F7F7F7Fu;
+        for (int bl = 0; bl < G::kSfaWords / 128; ++bl) {
+          uint32_t av[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            // kSplit: block bl covers stacked rows 128 bl + ..; kW4A4: scale block bl of rows 0..127
+            const int m = (SPLIT ? bl * 128 : 0) + lane + 32 * c;
+            const bool lo_row = SPLIT && m >= hrows;
+            const int rr = lo_row ? m - hrows : m;
+            const uint8_t* src = lo_row ? p.sl : p.sa;
+            const int boff = MODE == kW4A4 ? 4 * bl : 0;
+            av[c] = (rr < x.rows && m < kARowsSf) ? ld_scales4(src + (size_t)(x.row0 + rr) * (size_t)nsb + b0 + boff)
+                                                  : 0x7F7F7F7Fu;
+          }
+          sts_u128(smem_u32(&s.sfa[st][bl * 128 + lane * 4]), av[0], av[1], av[2], av[3]);
         }
-        sts_u128(smem_u32(&s.sfw[st][lane * 4]), wv[0], wv[1], wv[2], wv[3]);
-#pragma unroll
-        for (int bl = 0; bl < G::kSfaWords / 128; ++bl)
-          sts_u128(smem_u32(&s.sfa[st][bl * 128 + lane * 4]), av[4 * bl], av[4 * bl + 1], av[4 * bl + 2],
-                   av[4 * bl + 3]);
         fence_proxy_async_smem();  // the tensor core reads these through the async proxy
         __syncwarp();
         if (lane == 0) {
           const uint32_t col = tmem + (uint32_t)(sf_col0 + G::kSfCols * st);
-          tc_copy_scales(col, sdesc_scales(smem_u32(s.sfw[st])));
+#pragma unroll
+          for (int bl = 0; bl < G::kSfwWords / 128; ++bl)
+            tc_copy_scales(col + 4u * (uint32_t)bl, sdesc_scales(smem_u32(&s.sfw[st][bl * 128])));
 #pragma unroll
           for (int bl = 0; bl < G::kSfaWords / 128; ++bl)
-            tc_copy_scales(col + 4u + 4u * (uint32_t)bl, sdesc_scales(smem_u32(&s.sfa[st][bl * 128])));
+            tc_copy_scales(col + 4u * (uint32_t)(G::kSfwWords / 128 + bl),
+                           sdesc_scales(smem_u32(&s.sfa[st][bl * 128])));
           tc_commit(&s.full[st]);
         }
       }
@@ -450,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0, uc = 0;
       bool ok = true, ready = false;  // ready: the full barrier of stage `it` was seen complete in advance
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
-        const Unit x = unit_of<SPLIT>(s, p.E, u);
+        const Unit x = unit_of<MODE>(s, p.E, u);
         const int ab = uc & 1;
         if (uc >= 2 && !(ok = mbar_wait(&s.acce[ab], ((uc >> 1) - 1) & 1, err, abort))) break;
         tc_fence_after();
@@ -466,14 +553,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           // test the next stage's barrier now: its latency overlaps this stage's issue
           ready = mbar_try_wait(&s.full[(it + 1) % kStages], (uint32_t)((it + 1) / kStages) & 1u);
-          const uint32_t t_sfw = tmem + (uint32_t)(sf_col0 + G::kSfCols * st), t_sfa = t_sfw + 4u;
+          const uint32_t t_sfw = tmem + (uint32_t)(sf_col0 + G::kSfCols * st);
+          const uint32_t t_sfa = t_sfw + 4u * (uint32_t)(G::kSfwWords / 128);
           const uint32_t w_addr = smem_u32(s.w[st]), a_addr = smem_u32(s.a[st]);
-          const int j0 = (tail && kt == nk - 1) ? 2 : 0;
-          for (int j = j0; j < kBK / 32; ++j) {
-            const int q = kt * (kBK / 32) + j;  // K=32 step of the unit (every unit has at least 4)
-            tc_mma_w4a8(d_tmem + (uint32_t)(q % nsplit) * sub_w, sdesc_k_sw128(w_addr + 32 * j),
-                        sdesc_k_sw128(a_addr + 32 * j), idesc_w4a8(n_mma, (uint32_t)j), t_sfw | ((uint32_t)j << 30),
-                        t_sfa | ((uint32_t)j << 30), q >= nsplit);
+          const int j0 = (kt * G::kBK - stage_k0(kt)) / G::kMmaK;
+          constexpr int kSteps = G::kBK / G::kMmaK;  // 4 MMAs per stage, 32 bytes of each row apiece
+          for (int j = j0; j < kSteps; ++j) {
+            const int q = kt * kSteps + j;  // MMA step of the unit (every unit has at least 4)
+            const uint32_t d = d_tmem + (uint32_t)(q % nsplit) * sub_w;
+            const uint64_t da = sdesc_k_sw128(w_addr + 32 * j), db = sdesc_k_sw128(a_addr + 32 * j);
+            const uint32_t acc = q >= nsplit;
+            if (MODE == kW4A4) {
+              // two scales per row per MMA: column set j / 2, bytes 2 (j % 2) and 2 (j % 2) + 1
+              const uint32_t sf = 2u * (uint32_t)(j & 1), cs = 4u * (uint32_t)(j >> 1);
+              tc_mma_mxf4(d, da, db, idesc_mx(1u, 1u, n_mma, sf), (t_sfw + cs) | (sf << 30), (t_sfa + cs) | (sf << 30),
+                          acc);
+            } else {
+              tc_mma_mxf8f6f4(d, da, db, idesc_mx(5u, 0u, n_mma, (uint32_t)j), t_sfw | ((uint32_t)j << 30),
+                              t_sfa | ((uint32_t)j << 30), acc);
+            }
           }
           tc_commit(&s.empty[st]);
         }
@@ -492,14 +590,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     int uc = 0;
     for (int u = blockIdx.x; u < U; u += gridDim.x, ++uc) {
-      const Unit x = unit_of<SPLIT>(s, p.E, u);
+      const Unit x = unit_of<MODE>(s, p.E, u);
       const int ab = uc & 1;
       if (!mbar_wait(&s.accf[ab], (uc >> 1) & 1, err, abort)) break;
       tc_fence_after();
       const int n = x.j * kBW + q * 32 + lane;
       __nv_bfloat16* ycol = p.y + (size_t)x.row0 * p.N + n;
       const int nsplit = SPLIT ? 1 : acc_split(x.rows);
-      // SPLIT: the lo term of row i sits hrows columns after its hi term
+      // kSplit: the lo term of row i sits hrows columns after its hi term
       const int hrows = kBox * ((x.rows + kBox - 1) / kBox);
       for (int c = 0; c * 32 < x.rows; ++c) {
         uint32_t v[32];
@@ -551,29 +649,45 @@ cudaError_t launch_quant_mxfp8(const __nv_bfloat16* x, long long elems, uint8_t*
                     scales, lo_codes, lo_scales);
 }
 
-size_t gemm_w4a8_smem_bytes(bool split) { return (split ? sizeof(MxSmem<true>) : sizeof(MxSmem<false>)) + 1024; }
-int gemm_w4a8_rows_per_unit(bool split) { return split ? Geo<true>::kBT : Geo<false>::kBT; }
-int gemm_w4a8_weight_rows_per_unit() { return kBW; }
-int gemm_w4a8_small_box_rows() { return kBox; }
-
-template <bool SPLIT>
-static cudaError_t launch_gemm_w4a8_t(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
-                                      const CUtensorMap& tm_w_tail, const MxArgs& p, int grid, cudaStream_t stream) {
-  static std::atomic<bool> configured[64];
-  const cudaError_t e =
-      set_smem_limit_once(gemm_w4a8_kernel<SPLIT>, (int)gemm_w4a8_smem_bytes(SPLIT), configured);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(gemm_w4a8_kernel<SPLIT>, dim3(grid), dim3(kThreads), gemm_w4a8_smem_bytes(SPLIT), stream, tm_a,
-                    tm_a_big, tm_w, tm_w_tail, p);
+cudaError_t launch_quant_mxfp4_act(const __nv_bfloat16* x, long long elems, uint8_t* blocks, uint8_t* scales,
+                                   cudaStream_t stream) {
+  const long long octets = elems / 8;
+  if (octets == 0) return cudaSuccess;
+  const long long nb = (octets + kQThreads - 1) / kQThreads;
+  return launch_pdl(quant_mxfp4_act_kernel, dim3((unsigned)nb), dim3(kQThreads), 0, stream, x, octets, blocks, scales);
 }
 
-cudaError_t launch_gemm_w4a8(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
-                             const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* lo_scales,
-                             const uint8_t* w_scales, const int* offsets, const int* counts, __nv_bfloat16* y,
-                             unsigned* err, int E, int N, int K, int M, int grid, cudaStream_t stream) {
+template <int MODE>
+static size_t smem_bytes_t() { return sizeof(MxSmem<MODE>) + 1024; }
+
+size_t gemm_mx_smem_bytes(int mode) {
+  return mode == kW4A4 ? smem_bytes_t<kW4A4>() : (mode == kSplit ? smem_bytes_t<kSplit>() : smem_bytes_t<kW4A8>());
+}
+int gemm_mx_rows_per_unit(int mode) {
+  return mode == kW4A4 ? Geo<kW4A4>::kBT : (mode == kSplit ? Geo<kSplit>::kBT : Geo<kW4A8>::kBT);
+}
+int gemm_mx_k_per_stage(int mode) { return mode == kW4A4 ? Geo<kW4A4>::kBK : Geo<kW4A8>::kBK; }
+int gemm_mx_weight_rows_per_unit() { return kBW; }
+int gemm_mx_small_box_rows() { return kBox; }
+
+template <int MODE>
+static cudaError_t launch_gemm_mx_t(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
+                                    const CUtensorMap& tm_w_tail, const MxArgs& p, int grid, cudaStream_t stream) {
+  static std::atomic<bool> configured[64];
+  const cudaError_t e = set_smem_limit_once(gemm_mx_kernel<MODE>, (int)smem_bytes_t<MODE>(), configured);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(gemm_mx_kernel<MODE>, dim3(grid), dim3(kThreads), smem_bytes_t<MODE>(), stream, tm_a, tm_a_big,
+                    tm_w, tm_w_tail, p);
+}
+
+cudaError_t launch_gemm_mx(int mode, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
+                           const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* lo_scales,
+                           const uint8_t* w_scales, const int* offsets, const int* counts, __nv_bfloat16* y,
+                           unsigned* err, int E, int N, int K, int M, int grid, cudaStream_t stream) {
   MxArgs p{a_scales, lo_scales, w_scales, offsets, counts, y, err, E, N, K, M};
-  if (lo_scales != nullptr) return launch_gemm_w4a8_t<true>(tm_a, tm_a_big, tm_w, tm_w_tail, p, grid, stream);
-  return launch_gemm_w4a8_t<false>(tm_a, tm_a_big, tm_w, tm_w_tail, p, grid, stream);
+  if (mode == kW4A4) return launch_gemm_mx_t<kW4A4>(tm_a, tm_a_big, tm_w, tm_w_tail, p, grid, stream);
+  if (mode == kSplit) return launch_gemm_mx_t<kSplit>(tm_a, tm_a_big, tm_w, tm_w_tail, p, grid, stream);
+  return launch_gemm_mx_t<kW4A8>(tm_a, tm_a_big, tm_w, tm_w_tail, p, grid, stream);
 }
 
 }  // namespace gnf4

@@ -55,13 +55,16 @@ _lib.gnf4_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, _P]
 _lib.gnf4_quantize_mxfp8.argtypes = [_P, _I, _I, _P, _P, _P]
 _lib.gnf4_grouped_gemm_w4a8.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_quantize_mxfp8_split.argtypes = [_P, _I, _I, _P, _P, _P, _P, _P]
+_lib.gnf4_quantize_mxfp4_act.argtypes = [_P, _I, _I, _P, _P, _P]
+_lib.gnf4_grouped_gemm_w4a4.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_grouped_gemm_w4a8x2.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
 _lib.gnf4_dequant_nf4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 _lib.gnf4_dequant_mxfp4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", "gnf4_route_topk_permute",
               *_GROUPED, "gnf4_combine", "gnf4_quantize_mxfp8", "gnf4_grouped_gemm_w4a8",
-              "gnf4_quantize_mxfp8_split", "gnf4_grouped_gemm_w4a8x2", "gnf4_selftest_bounded_wait",
+              "gnf4_quantize_mxfp8_split", "gnf4_grouped_gemm_w4a8x2",
+              "gnf4_quantize_mxfp4_act", "gnf4_grouped_gemm_w4a4", "gnf4_selftest_bounded_wait",
               "gnf4_grouped_gemv_nf4_combine", "gnf4_grouped_gemv_mxfp4_combine",
               "gnf4_dequant_nf4_f32", "gnf4_dequant_mxfp4_f32"):
     getattr(_lib, _name).restype = _I
@@ -331,3 +334,17 @@ def grouped_gemm_w4a8x2(hi_codes, hi_scales, lo_codes, lo_scales, w, w_scales, y
     _check(_lib.gnf4_grouped_gemm_w4a8x2(_ptr(hi_codes), _ptr(hi_scales), _ptr(lo_codes), _ptr(lo_scales), _ptr(w),
                                          _ptr(w_scales), _ptr(offsets), _ptr(counts), E, N, 2 * K2, M, _ptr(y),
                                          _stream(stream)))
+
+
+def quantize_mxfp4_act(x, blocks, scales, stream=None):
+    """x bf16 [M, K] -> MXFP4 blocks uint8 [M, K/2] and scales uint8 [M, K/32], preallocated."""
+    M, K = x.shape
+    _check(_lib.gnf4_quantize_mxfp4_act(_ptr(x), M, K, _ptr(blocks), _ptr(scales), _stream(stream)))
+
+
+def grouped_gemm_w4a4(a_blocks, a_scales, w, w_scales, y, offsets=None, counts=None, stream=None):
+    """Native W4A4: y [M, N] = MXFP4 activations x the MXFP4 stack [E, N, K/2] per group."""
+    E, N, K2 = w.shape
+    M = a_blocks.shape[0]
+    _check(_lib.gnf4_grouped_gemm_w4a4(_ptr(a_blocks), _ptr(a_scales), _ptr(w), _ptr(w_scales), _ptr(offsets),
+                                       _ptr(counts), E, N, 2 * K2, M, _ptr(y), _stream(stream)))

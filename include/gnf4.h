@@ -363,6 +363,27 @@ gnf4_status gnf4_grouped_gemm_w4a8(const uint8_t *a_codes, const uint8_t *a_scal
                                    const uint8_t *w_scales, const int32_t *offsets, const int32_t *counts, int E,
                                    int N, int K, int M, void *y, void *stream);
 
+/* Native W4A4 mode: MXFP4 activations x MXFP4 weights on kind::mxf4
+ * (the "W4A4" MX mode named next to W4A8; the pages give no rule).
+ *
+ * gnf4_quantize_mxfp4_act: x bf16 [M, K] -> blocks [M, K/2] (e2m1, element
+ * 2i in the low nibble) and scales [M, K/32] (e8m0) by the OCP rule of the
+ * weights: X = floor(log2(max |x|)) - 2 clamped to [-127, 127] (-127 for an
+ * all-zero block), code = x * 2^-X rounded to the nearest e2m1 value, ties
+ * to even, saturating at +-6.  Bit-exact.  K % 32 == 0; x 16-byte and
+ * blocks 4-byte aligned.
+ *
+ * gnf4_grouped_gemm_w4a4: y[r, n] = sum_k A[r, k] * W_e[n, k] with A and W
+ * both e2m1 x 2^(scale - 127); products exact, fp32 accumulation, bf16
+ * output.  K must be a multiple of 64 in [256, 65536]; a_blocks and w
+ * 16-byte aligned, y 16-byte aligned; other rules as gnf4_grouped_gemm_w4a8.
+ * The result carries the e2m1 rounding of the activations: against bf16
+ * activations each activation moves by at most |a|/3 + 2^(X-2). */
+gnf4_status gnf4_quantize_mxfp4_act(const void *x, int M, int K, uint8_t *blocks, uint8_t *scales, void *stream);
+gnf4_status gnf4_grouped_gemm_w4a4(const uint8_t *a_blocks, const uint8_t *a_scales, const uint8_t *w,
+                                   const uint8_t *w_scales, const int32_t *offsets, const int32_t *counts, int E,
+                                   int N, int K, int M, void *y, void *stream);
+
 /* ------------------------------------------------------------------ */
 /* Top-k combine                                                       */
 /* ------------------------------------------------------------------ */

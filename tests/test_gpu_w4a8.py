@@ -210,3 +210,74 @@ def test_w4a8x2_counts_equal_offsets(g):
     a, _ = _run_split(g, counts, 128, 256, seed=1800)
     b, _ = _run_split(g, counts, 128, 256, seed=1800, use_counts=True)
     assert np.array_equal(a, b)
+
+
+# ---------------------------------------------------------------- W4A4 (MXFP4 activations, kind::mxf4)
+
+
+def _check_quant4(g, bits):
+    M, K = bits.shape
+    blocks = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((M, K // 32), dtype=torch.uint8, device="cuda")
+    g.quantize_mxfp4_act(to_dev_bf16(bits), blocks, scales)
+    torch.cuda.synchronize()
+    rb, rs = oracle.quant_mxfp4_act(bits)
+    gb, gs = blocks.cpu().numpy(), scales.cpu().numpy()
+    assert np.array_equal(gs, rs), f"scales differ at {np.argwhere(gs != rs)[:5].tolist()}"
+    bad = np.argwhere(gb != rb)
+    assert bad.size == 0, f"{len(bad)} bytes differ, first {[(tuple(i), int(gb[tuple(i)]), int(rb[tuple(i)])) for i in bad[:5]]}"
+    return blocks, scales
+
+
+@pytest.mark.parametrize("M,K", [(37, 2880), (128, 2048), (1, 32), (300, 416)])
+def test_quantize_mxfp4_act_is_bit_exact(g, M, K):
+    _check_quant4(g, _activations(2000 + K + M, M, K))
+
+
+def _run4(g, counts, N, K, seed, use_counts=False):
+    E = len(counts)
+    offsets = offsets_from_counts(counts)
+    nv = int(offsets[-1])
+    M = nv + 3
+    w, sw = inputs.mxfp4_random(inputs.rng(seed), E, N, K)
+    bits = _activations(seed + 1, M, K)
+    ab, as_ = _check_quant4(g, bits)
+    y = torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    kw = {"counts": to_dev(np.array(counts, np.int32))} if use_counts else {"offsets": to_dev(offsets)}
+    g.grouped_gemm_w4a4(ab, as_, to_dev(w), to_dev(sw), y, **kw)
+    torch.cuda.synchronize()
+    assert g.device_errors() == 0
+    got = bf16_to_f64(y)
+    assert np.all(got[nv:] == 7.0), "rows past offsets[E] were written"
+    return got[:nv], (w, sw, bits, offsets)
+
+
+@pytest.mark.parametrize("N,K", [(128, 256), (136, 320), (256, 2880), (384, 512)])
+def test_w4a4_gemm_ragged_parity(g, N, K):
+    got, (w, sw, bits, offsets) = _run4(g, GROUPS, N, K, seed=2100 + K + N)
+    ref = oracle.grouped_gemm_w4a4(*oracle.quant_mxfp4_act(bits), w, sw, offsets)
+    amax = float(np.abs(ref).max())
+    err = np.abs(got - ref)
+    bad = np.argwhere(~(err <= W4A8_REL * np.abs(ref) + W4A8_ABS_OF_MAX * amax))
+    assert bad.size == 0, (f"{len(bad)} outputs out of tolerance (max|ref| {amax:.4g}), first "
+                           + ", ".join(f"{tuple(i)} gpu={got[tuple(i)]:.6g} ref={ref[tuple(i)]:.6g}" for i in bad[:5]))
+
+
+def test_w4a4_counts_equal_offsets(g):
+    counts = [40, 0, 129, 1, 7]
+    a, _ = _run4(g, counts, 128, 512, seed=2200)
+    b, _ = _run4(g, counts, 128, 512, seed=2200, use_counts=True)
+    assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("K", [128, 192, 288])
+def test_w4a4_refuses_short_or_unaligned_k(g, K):
+    w = torch.zeros((1, 128, K // 2), dtype=torch.uint8, device="cuda")
+    sw = torch.full((1, 128, K // 32), 127, dtype=torch.uint8, device="cuda")
+    ab = torch.zeros((4, K // 2), dtype=torch.uint8, device="cuda")
+    sa = torch.full((4, K // 32), 127, dtype=torch.uint8, device="cuda")
+    y = torch.zeros((4, 128), dtype=torch.bfloat16, device="cuda")
+    off = torch.tensor([0, 4], dtype=torch.int32, device="cuda")
+    with pytest.raises(g.Gnf4Error) as ei:
+        g.grouped_gemm_w4a4(ab, sa, w, sw, y, offsets=off)
+    assert ei.value.status == g.ERR_UNSUPPORTED_SHAPE
