@@ -146,7 +146,7 @@ class Workload:
     than L2, a set of token batches, and the step's output buffers."""
 
     def __init__(self, name, device, seed, build_host_copy, swiglu=False, dgrad=False, w4a8=False,
-                 fused_combine=False, w4a8x2=False):
+                 fused_combine=False, w4a8x2=False, w4a4=False):
         import torch
 
         from bit_grouped_moe_b200 import gnf4
@@ -211,14 +211,16 @@ class Workload:
             self.dfn = f.grouped_dgrad_nf4 if wl.fmt == "nf4" else f.grouped_dgrad_mxfp4
         # optional native W4A8 mode (MXFP4 stacks): both projections' activations are
         # quantised to MXFP8 every step and the block-scaled GEMM runs on the codes
-        self.w4a8 = w4a8 or w4a8x2
+        self.w4a8 = w4a8 or w4a8x2 or w4a4
         self.split = w4a8x2  # two-term activations (hi + lo): the bf16-activation accuracy on the native path
+        self.a4 = w4a4       # MXFP4 activations (kind::mxf4)
         if self.w4a8:
             assert wl.fmt == "mxfp4", "the W4A8 mode runs on MXFP4 weight stacks"
             self.decode = False  # one GEMM path for every group size
-            self.qa1 = torch.empty(M, self.p1.K, dtype=torch.uint8, device=device)
+            cw = 2 if w4a4 else 1  # activation codes per byte
+            self.qa1 = torch.empty(M, self.p1.K // cw, dtype=torch.uint8, device=device)
             self.sa1 = torch.empty(M, self.p1.K // 32, dtype=torch.uint8, device=device)
-            self.qa2 = torch.empty(M, self.p2.K, dtype=torch.uint8, device=device)
+            self.qa2 = torch.empty(M, self.p2.K // cw, dtype=torch.uint8, device=device)
             self.sa2 = torch.empty(M, self.p2.K // 32, dtype=torch.uint8, device=device)
             if self.split:
                 self.la1 = torch.empty_like(self.qa1)
@@ -303,7 +305,9 @@ class Workload:
             g.combine(self.y2, self.f2s, wts, self.out)
 
     def _quant1(self):
-        if self.split:
+        if self.a4:
+            self.g.quantize_mxfp4_act(self.xs, self.qa1, self.sa1)
+        elif self.split:
             self.g.quantize_mxfp8_split(self.xs, self.qa1, self.sa1, self.la1, self.ls1)
         else:
             self.g.quantize_mxfp8(self.xs, self.qa1, self.sa1)
@@ -313,13 +317,18 @@ class Workload:
             g = self.g
             if quantize_first:
                 self._quant1()
-            if self.split:
+            if self.a4:
+                g.grouped_gemm_w4a4(self.qa1, self.sa1, w1, s1, self.y1, offsets=self.off)
+            elif self.split:
                 g.grouped_gemm_w4a8x2(self.qa1, self.sa1, self.la1, self.ls1, w1, s1, self.y1, offsets=self.off)
             else:
                 g.grouped_gemm_w4a8(self.qa1, self.sa1, w1, s1, self.y1, offsets=self.off)
             if ev is not None:
                 ev[1].record()
-            if self.split:
+            if self.a4:
+                g.quantize_mxfp4_act(self.h, self.qa2, self.sa2)
+                g.grouped_gemm_w4a4(self.qa2, self.sa2, w2, s2, self.y2, offsets=self.off)
+            elif self.split:
                 g.quantize_mxfp8_split(self.h, self.qa2, self.sa2, self.la2, self.ls2)
                 g.grouped_gemm_w4a8x2(self.qa2, self.sa2, self.la2, self.ls2, w2, s2, self.y2, offsets=self.off)
             else:
@@ -400,7 +409,10 @@ def oracle_step(wl_obj, batch_i, n_slice=None):
     (w1, s1), (w2, s2) = wl_obj.host_stacks
     n1 = wl_obj.p1.N if n_slice is None else min(n_slice, wl_obj.p1.N)
     n2 = wl_obj.p2.N if n_slice is None else min(n_slice, wl_obj.p2.N)
-    if getattr(wl_obj, "split", False):
+    if getattr(wl_obj, "a4", False):
+        def gemm(a_bits, w, s, off):
+            return oracle.grouped_gemm_w4a4(*oracle.quant_mxfp4_act(a_bits), w, s, off)
+    elif getattr(wl_obj, "split", False):
         def gemm(a_bits, w, s, off):
             return oracle.grouped_gemm_w4a8x2(*oracle.quant_mxfp8_split(a_bits), w, s, off)
     elif getattr(wl_obj, "w4a8", False):
@@ -463,6 +475,8 @@ def main():
     ap.add_argument("--w4a8x2", action="store_true",
                     help="MXFP4 workloads: two-term native mode (hi + lo MXFP8 activations, the bf16-activation "
                          "accuracy on the block-scaled tcgen05 GEMM)")
+    ap.add_argument("--w4a4", action="store_true",
+                    help="MXFP4 workloads: native W4A4 mode (MXFP4 activations, kind::mxf4 block-scaled GEMM)")
     ap.add_argument("--fused-combine", action="store_true",
                     help="decode: run the top-k combine in the second GEMV's epilogue instead of as its own launch "
                          "(measured slower on B200: the epilogue's round trips extend every unit)")
@@ -474,7 +488,7 @@ def main():
     globals()["N_WEIGHT_COPIES"] = max(1, args.weight_copies)
 
     wl_def = inputs.WORKLOADS[args.workload]
-    decode = wl_def.T <= 8 and not args.dgrad and not args.w4a8 and not args.w4a8x2
+    decode = wl_def.T <= 8 and not args.dgrad and not args.w4a8 and not args.w4a8x2 and not args.w4a4
     steps = args.steps if args.steps is not None else (20000 if decode else 200)
     warmup = args.warmup if args.warmup is not None else (100 if decode else 10)
     warmup = max(warmup, 3)
@@ -512,7 +526,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     dev = f"cuda:{local}"
     torch.cuda.set_device(local)
     wl = Workload(args.workload, dev, seed=1234 + rank, build_host_copy=(rank == 0 and world == 1),
-                  swiglu=args.swiglu, dgrad=args.dgrad, w4a8=args.w4a8, fused_combine=args.fused_combine, w4a8x2=args.w4a8x2)
+                  swiglu=args.swiglu, dgrad=args.dgrad, w4a8=args.w4a8, fused_combine=args.fused_combine, w4a8x2=args.w4a8x2, w4a4=args.w4a4)
     decode = wl.decode
     wl.h_host = wl.h.cpu().view(torch.int16).numpy().view(np.uint16)
     stream = torch.cuda.current_stream()
@@ -645,7 +659,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     peaks, peak_src = load_peaks()
     kern_file = "gemv.cu" if decode else ("dgrad.cu" if wl.dgrad else ("mx.cu" if wl.w4a8 else "gemm_tc.cu"))
     kern_base = "gemv" if decode else ("dgrad_tc" if wl.dgrad else
-                                       ("gemm_w4a8x2" if wl.split else ("gemm_w4a8" if wl.w4a8 else "gemm_tc")))
+                                       ("gemm_w4a4" if wl.a4 else ("gemm_w4a8x2" if wl.split else
+                                                                  ("gemm_w4a8" if wl.w4a8 else "gemm_tc"))))
     kern_key = f"{kern_base}_{wl.wl.fmt}{'_swiglu' if wl.swiglu else ''}:{args.workload}:{wl.p1.name}"
     sha = kernel_source_sha([kern_file, "common.cuh"])
     if decode:
@@ -662,12 +677,16 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
         achieved = flops / (dom_ms / 1e3) / 1e12
         pk = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         pk_src = f"bf16_tflops_sustained of {peak_src} (kind::f16 MMA on decoded bf16 tiles)"
-        if wl.w4a8:  # 8-bit-rate MMA: the measured bf16 peak x the nominal dense fp8 / bf16 ratio (4.5 / 2.25)
+        if wl.a4:  # fp4-rate MMA: the measured bf16 peak x the nominal dense fp4 / bf16 ratio (9 / 2.25)
+            pk = round(4 * pk, 1)
+            pk_src = f"4 x bf16_tflops_sustained of {peak_src} (kind::mxf4 runs at the fp4 rate)"
+        elif wl.w4a8:  # 8-bit-rate MMA: the measured bf16 peak x the nominal dense fp8 / bf16 ratio (4.5 / 2.25)
             pk = round(2 * pk, 1)
             pk_src = f"2 x bf16_tflops_sustained of {peak_src} (kind::mxf8f6f4 runs at the fp8 rate)"
         kname = (f"dgrad_tc_kernel<{wl.wl.fmt}> (dX of {wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.dgrad else
-                 f"gemm_w4a8_kernel<two-term> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.split else
-                 f"gemm_w4a8_kernel ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.w4a8 else
+                 f"gemm_mx_kernel<W4A4> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.a4 else
+                 f"gemm_mx_kernel<two-term> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.split else
+                 f"gemm_mx_kernel<W4A8> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.w4a8 else
                  f"gemm_tc_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})")
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk, "unit": "TFLOP/s",
                 "frac": round(achieved / pk, 4), "traffic": committed_traffic(kern_key, sha), "kernel": kname,
@@ -687,10 +706,12 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
             "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": steps,
             "warmup": warmup, "ms_per_step": round(ms / steps, 6), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
-            "dtype": ("(e4m3 hi + e4m3 lo) x e2m1 (fp32 accumulate)" if wl.split else
+            "dtype": ("e2m1 x e2m1 (fp32 accumulate)" if wl.a4 else
+                      "(e4m3 hi + e4m3 lo) x e2m1 (fp32 accumulate)" if wl.split else
                       "e4m3 x e2m1 (fp32 accumulate)" if wl.w4a8 else "bf16"), "data": "synthetic",
             "config": dict(_config(wl.wl, world), **({"first_projection": "fused gate_up + SwiGLU"} if wl.swiglu else {}),
-                           **({"activations": "two-term MXFP8 hi + lo (quantised every step; bf16-activation accuracy)"}
+                           **({"activations": "MXFP4 (native W4A4 mode: quantised every step)"} if wl.a4 else
+                              {"activations": "two-term MXFP8 hi + lo (quantised every step; bf16-activation accuracy)"}
                               if wl.split else
                               {"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if wl.w4a8 else {}),
                            **({"combine": "in the second GEMV's epilogue"} if wl.fused_combine else {}),
@@ -715,7 +736,7 @@ def run_reference(args, steps, warmup, world):
     import oracle
 
     wl_def = inputs.WORKLOADS[args.workload]
-    decode = wl_def.T <= 8 and not args.w4a8 and not args.w4a8x2
+    decode = wl_def.T <= 8 and not args.w4a8 and not args.w4a8x2 and not args.w4a4
     unit, _ = _unit(decode)
 
     class HostWL:
@@ -723,8 +744,9 @@ def run_reference(args, steps, warmup, world):
 
     h = HostWL()
     h.wl = wl_def
-    h.w4a8 = args.w4a8 or args.w4a8x2
+    h.w4a8 = args.w4a8 or args.w4a8x2 or args.w4a4
     h.split = args.w4a8x2
+    h.a4 = args.w4a4
     h.E, h.k, h.T = wl_def.E, wl_def.k, wl_def.T
     h.M = h.T * h.k
     h.p1, h.p2 = wl_def.projections[0], wl_def.projections[-1]
@@ -770,7 +792,8 @@ def run_reference(args, steps, warmup, world):
         "ms_per_step": round(dt * 1e3 / steps, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(_config(wl_def, world),
-                       **({"activations": "two-term MXFP8 hi + lo (quantised every step; bf16-activation accuracy)"}
+                       **({"activations": "MXFP4 (native W4A4 mode: quantised every step)"} if args.w4a4 else
+                          {"activations": "two-term MXFP8 hi + lo (quantised every step; bf16-activation accuracy)"}
                           if args.w4a8x2 else
                           {"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if args.w4a8 else {})),
         "impl": "reference",
