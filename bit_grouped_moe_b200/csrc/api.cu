@@ -243,9 +243,10 @@ gnf4_status grouped_gemv_combine(int fmt, const void* a, const uint8_t* w, const
                                  const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M, void* y,
                                  const int32_t* sorted_to_flat, const int32_t* flat_to_sorted, const float* weights,
                                  int T, int k, void* out, int32_t* counters, void* stream) {
-  GNF4_TRY(check_grouped(fmt, a, w, scales, offsets, counts, E, N, K, M, y));
+  // every shape rule before any pointer
   if (T < 0 || k < 1) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T=%d / k=%d invalid", T, k);
   if ((long long)T * k >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T*k too large");
+  GNF4_TRY(check_grouped(fmt, a, w, scales, offsets, counts, E, N, K, M, y));
   if (T == 0) return GNF4_OK;
   GNF4_TRY(check_ptr(offsets, "offsets", 4, false));
   GNF4_TRY(check_ptr(counts, "counts", 4, false));

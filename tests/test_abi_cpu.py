@@ -113,3 +113,49 @@ def test_product_path_never_imports_the_oracle():
                 text = open(os.path.join(dirpath, fn)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), fn
                 assert "gnf4_oracle" not in text and "liboracle" not in text, fn
+
+
+@pytest.mark.parametrize("name,K", [("gnf4_grouped_gemm_w4a8", 96), ("gnf4_grouped_gemm_w4a8", 64),
+                                    ("gnf4_grouped_gemm_w4a8", 2848), ("gnf4_grouped_gemm_w4a4", 192),
+                                    ("gnf4_grouped_gemm_w4a4", 320 + 32)])
+def test_native_gemm_shape_refusals(g, name, K):
+    """K rules of the native modes are checked before any pointer: W4A8 needs a
+    multiple of 64 of at least 128, W4A4 a multiple of 64 of at least 256."""
+    st = getattr(g._lib, name)(None, None, None, None, ctypes.c_void_p(16), None, 4, 64, K, 8, None, None)
+    assert st == g.ERR_UNSUPPORTED_SHAPE, g.last_error()
+
+
+def test_two_term_gemm_needs_both_terms(g):
+    f = g._lib.gnf4_grouped_gemm_w4a8x2
+    st = f(None, None, None, None, None, None, ctypes.c_void_p(16), None, 4, 64, 128, 8, None, None)
+    assert st == g.ERR_INVALID_ARG and "lo_" in g.last_error()
+
+
+@pytest.mark.parametrize("name", ["gnf4_quantize_mxfp8", "gnf4_quantize_mxfp4_act"])
+def test_quantiser_refusals(g, name):
+    f = getattr(g._lib, name)
+    assert f(None, 4, 48, None, None, None) == g.ERR_UNSUPPORTED_SHAPE
+    assert f(None, -1, 64, None, None, None) == g.ERR_UNSUPPORTED_SHAPE
+    assert f(None, 0, 64, None, None, None) == g.OK  # nothing to do
+
+
+def test_split_quantiser_refusals(g):
+    f = g._lib.gnf4_quantize_mxfp8_split
+    assert f(None, 4, 16, None, None, None, None, None) == g.ERR_UNSUPPORTED_SHAPE
+    assert f(None, 0, 64, None, None, None, None, None) == g.OK
+
+
+def test_fused_combine_gemv_refusals(g):
+    f = g._lib.gnf4_grouped_gemv_nf4_combine
+    off = ctypes.c_void_p(16)
+    assert f(None, None, None, off, None, 4, 60, 64, 8, None, None, None, None, 2, 4, None, None, None) \
+        == g.ERR_UNSUPPORTED_SHAPE  # N % 8
+    assert f(None, None, None, off, None, 4, 64, 64, 8, None, None, None, None, 2, 0, None, None, None) \
+        == g.ERR_UNSUPPORTED_SHAPE  # k < 1
+    assert g.combine_counters_bytes(8, 2048) == 8 * 32 * 4
+    assert g.combine_counters_bytes(8, 136) == 8 * 3 * 4
+
+
+def test_selftest_limit_refusal(g):
+    assert g._lib.gnf4_selftest_bounded_wait(0, None) == g.ERR_INVALID_ARG
+    assert g._lib.gnf4_selftest_bounded_wait((1 << 32) + 1, None) == g.ERR_INVALID_ARG
