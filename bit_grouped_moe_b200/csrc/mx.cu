@@ -1,42 +1,52 @@
-// mx.cu -- native W4A8 mode: MXFP8 activations times MXFP4 weights on the
-// block-scaled tcgen05 tensor cores (kind::mxf8f6f4), and the MXFP8
-// activation quantiser that feeds it.
+// mx.cu -- the native block-scaled MXFP4 modes on tcgen05, and the
+// activation quantisers that feed them:
+//   W4A8     MXFP8 activations x MXFP4 weights   (kind::mxf8f6f4, K = 32 per MMA)
+//   two-term hi + lo MXFP8 activations x MXFP4     (same MMA; both terms stacked
+//            in one B operand): the accuracy of bf16 activations
+//   W4A4     MXFP4 activations x MXFP4 weights   (kind::mxf4, K = 64 per MMA)
 //
 // bw24 v0.9.0 release notes (Features, "f8f4 tile piece 1"; Documentation,
 // "prefill arc design"): W4A8-FP8 multiplies native e2m1 weights by e4m3
 // activations in one block-scaled MMA.  grouped-nf4-gemm index.json,
 // system_manifest.owns: the grouped GEMM runs on native MXFP4.
 //
-// Quantiser (OCP MX v1.0, MXFP8 E4M3): the 32 consecutive k of one row share
-// an e8m0 scale 2^X with X = floor(log2(amax)) - 8 clamped to [-127, 127];
-// each element is x * 2^-X rounded to the nearest e4m3 value, ties to even,
-// saturating at +-448 (cvt.rn.satfinite).  An all-zero block gets scale 0.
+// Quantisers (OCP MX v1.0): the 32 consecutive k of one row share an e8m0
+// scale 2^X.  MXFP8 E4M3: X = floor(log2(amax)) - 8, elements x * 2^-X
+// rounded to the nearest e4m3 value, ties to even, saturating at +-448
+// (cvt.rn.satfinite); the two-term split uses X = floor(log2(amax)) - 7 for
+// hi and for the exact residual lo (one binade of headroom: nothing
+// saturates).  MXFP4: X = floor(log2(amax)) - 2, e2m1 saturating at +-6.  An
+// all-zero block gets scale byte 0.
 //
 // GEMM design (B200):
 //  * D^T[n, r] = W_e[n, :] . A[r, :]: the 128 weight rows of a tile are the
 //    MMA's M, the rows (tokens) of the group its N, as in the bf16 path.
 //  * Both operands go straight from global memory into 128B-swizzled shared
-//    memory by TMA.  The packed e2m1 weights are expanded by the TMA unit
-//    itself into the layout the MMA reads (16 codes in 8 bytes followed by 8
-//    bytes of padding, so 128 codes fill one 128-byte row); the e4m3
-//    activations are plain bytes.  The SM decodes nothing: no lookup table
-//    and no bf16 copy of a weight exist anywhere.
-//  * Block scales: per 128-k stage a loader warp copies the e8m0 scales of
-//    the tile's 128 weight rows and of the group's rows into shared memory
-//    in the layout tcgen05.cp reads (row m at byte 16*(m%32) + 4*(m/32), one
-//    byte per 32-k block), moves both to the stage's own TMEM columns with
+//    memory by TMA.  For kind::mxf8f6f4 the packed e2m1 weights are expanded
+//    by the TMA unit itself into the layout the MMA reads (16 codes in 8
+//    bytes followed by 8 bytes of padding, so 128 codes fill one 128-byte
+//    row); kind::mxf4 reads them packed (256 codes per row).  The SM decodes
+//    nothing: no lookup table and no bf16 copy of a weight exist anywhere.
+//  * Block scales: per stage a loader warp copies the e8m0 scales of the
+//    tile's 128 weight rows and of the group's rows into shared memory in the
+//    layout tcgen05.cp reads (row m at byte 16*(m%32) + 4*(m/32), one byte
+//    per 32-k block), moves them to the stage's own TMEM columns with
 //    tcgen05.cp.32x128b.warpx4 and commits the copies to the stage's full
-//    barrier; the four K=32 MMAs of the stage select the byte of their block
-//    with their scale-factor ids.  The MMA thread only waits, issues four
-//    MMAs and commits: it is the one serial thread of the pipeline.
-//  * K % 128 == 64 (e.g. 2880): the last stage reads [K-128, K) and issues
-//    only its upper two K=32 steps, so no box reads past the end of a row.
+//    barrier; the MMAs of the stage select their scale bytes with their
+//    scale-factor ids.  The MMA thread only waits, issues four MMAs and
+//    commits: it is the one serial thread of the pipeline.
+//  * K not a multiple of the stage's k: the last stage reads [K - kBK, K)
+//    and skips the MMAs already covered, so no box reads past a row.
 //  * Warp roles (13 warps): 0 and 12 = TMA producers (alternate stages: one
 //    issuing thread alone caps the stream), 1 = TMEM owner + MMA issuer,
 //    4..7 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31, i.e. weight
-//    rows), 2, 3 and 8..11 = scale loaders, one per ring slot, so the global
-//    loads of six stages are in flight at once.  Two TMEM accumulators let
-//    the epilogue of one unit overlap the main loop of the next.
+//    rows), 2, 3 and 8.. = scale loaders, one per ring slot, so the global
+//    loads of every stage in the ring are in flight at once.  Two TMEM
+//    accumulators let the epilogue of one unit overlap the next.
+//  * A block-scaled M=128 MMA occupies the SM's tensor pipe for about 160
+//    cycles whatever N is (measured), so small groups stream weights at a
+//    fixed rate per MMA: K = 64 per MMA (W4A4) streams twice as fast, and
+//    the two-term form's second term rides in the same MMAs.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
