@@ -8,16 +8,29 @@
 //  * the dY tile [128 rows r][64 n] bf16 arrives by TMA in the 128B-swizzled
 //    K-major layout (the MMA's A operand);
 //  * the packed weight block [64 n][64 bytes = 128 k] arrives by TMA;
-//  * the four warps decode it through the pair table and write it TRANSPOSED
-//    as [128 k][64 n] bf16 in the same 128B-swizzled K-major layout (the MMA's
-//    B operand), so both operands use the plain K-major descriptor.
+//  * the eight decode warps decode it through the pair table in its natural
+//    order, weight row n with k contiguous, as two 128B-swizzled halves
+//    [64 n][64 k] bf16.  The MMA reads this tile as an MN-major B operand
+//    (MN = k, the output width; K = n, the contraction), so no transpose
+//    happens anywhere: a quarter warp stores one 128-byte row with eight
+//    conflict-free 16-byte stores, and a warp reads 128 contiguous packed bytes.
 // D[r, k] accumulates in TMEM (lane = row r, column = k).  Work unit = (expert
 // e, chunk of <= 128 of its rows, 128-wide k tile); a persistent grid strides
-// over the units.  Warp roles: 8 decode warps, a TMA producer, an MMA issuer
-// and 4 epilogue warps.  Packed weights and dY tiles stream through a 4-deep
-// TMA ring, block scales are staged in shared memory by the decode warps two
-// stages ahead, four decoded W^T tiles are in flight and two accumulators,
-// so copies, MMAs, decode and the epilogue of the previous unit overlap.
+// over the units.  Warp roles: 8 decode warps, a dY producer, a weight
+// producer, an MMA issuer and 4 epilogue warps.
+//
+// Every stage waits on memory twice, for the packed weights and block scales
+// (mostly DRAM: the stacks are larger than L2) and for the dY tile (mostly L2:
+// the k tiles of one row chunk run side by side).  Each source has its own
+// queue, deep enough to cover its latency:
+//  * dY tiles: a 4-deep TMA ring, released by the MMAs' commit;
+//  * packed weight blocks: a 12-deep TMA ring of 4 KB slots, released by the
+//    decode warps once they have read a block;
+//  * block scales: each decode thread keeps the raw scales of the next 8
+//    stages in registers (a plain load per stage, issued 8 stages before it is
+//    needed), and stores one stage ahead into a double-buffered table.
+// Four decoded W^T tiles are in flight and two accumulators, so copies, MMAs,
+// decode and the epilogue of the previous unit overlap.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -29,9 +42,11 @@ namespace {
 
 constexpr int kDecWarps = 8;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kProdWarp = 8, kMmaWarp = 9, kEpiWarp0 = 10;
-constexpr int kThreads = (kEpiWarp0 + 4) * 32;  // 448
-constexpr int kRing = 4;                       // dY / packed-weight stages in flight
+constexpr int kProdWarp = 8, kWProdWarp = 9, kMmaWarp = 10, kEpiWarp0 = 11;
+constexpr int kThreads = (kEpiWarp0 + 4) * 32;  // 480
+constexpr int kRing = 4;                       // dY stages in flight
+constexpr int kWRing = 12;                     // packed-weight stages in flight
+constexpr int kSQ = 8;                         // stages of block scales queued in registers
 constexpr int kTBuf = 4;                       // decoded W^T tiles in flight
 static_assert(kTBuf <= kRing, "a decoded tile is released through the ring's MMA-done barriers");
 constexpr int kBR = 128;                   // rows per unit (MMA M)
@@ -39,19 +54,20 @@ constexpr int kBKt = 128;                  // k per unit (MMA N)
 constexpr int kBN = 64;                    // n per stage (four k-steps of 16)
 constexpr int kYBytes = kBR * kBN * 2;     // 16 KB
 constexpr int kTBytes = kBKt * kBN * 2;    // 16 KB
+constexpr int kTHalf = kBN * 128;          // one 64-k half of the decoded tile: 64 rows of 128 bytes
 constexpr int kWBytes = kBN * kBKt / 2;    // 4 KB
 constexpr int kTmemCols = 2 * kBKt;  // two accumulators
 
 struct DSmem {
   uint8_t y[kRing][kYBytes];  // dY tiles (1024-aligned for the 128-byte swizzle)
-  uint8_t t[kTBuf][kTBytes];  // decoded W^T tiles
-  uint8_t w[kRing][kWBytes];  // packed weight blocks
-  uint32_t lut[kLut256Words];
+  uint8_t t[kTBuf][kTBytes];  // decoded W tiles, two 64-k halves each
+  uint8_t w[kWRing][kWBytes];  // packed weight blocks
+  uint32_t lut[kLutWords];    // pair table, 128-byte entries (32 lanes)
   uint32_t sc[2][kBN][4];     // raw block scales of a stage: 64 rows x (2 NF4 | 4 MXFP4) blocks of the k tile
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
-  uint64_t full[kRing], mdone[kRing], decoded[kTBuf], accf[2], acce[2], drain;
+  uint64_t full[kRing], mdone[kRing], wfull[kWRing], wempty[kWRing], decoded[kTBuf], accf[2], acce[2], drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -84,19 +100,34 @@ __device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
-// Byte offset of the 16-byte chunk c (8 bf16 of n) of row k in a 128B-swizzled
-// K-major tile with 128-byte rows (8-row atoms of 1 KB).
-__device__ __forceinline__ uint32_t sw128_chunk(int k, int c) {
-  return (uint32_t)((k >> 3) * 1024 + (k & 7) * 128 + ((c ^ (k & 7)) << 4));
+// Shared-memory descriptor of an MN-major operand in the 128-byte swizzle:
+// 64 consecutive MN elements (bf16) fill a 128-byte row, eight rows of
+// consecutive K form a 1 KB atom; lbo = bytes to the next 64 MN elements,
+// sbo = bytes to the next 8 K rows.
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
+  d |= (uint64_t)(lbo >> 4) << 16;           // leading byte offset: next 64 MN elements
+  d |= (uint64_t)(sbo >> 4) << 32;           // stride byte offset: next 8 K rows
+  d |= (uint64_t)1u << 46;                   // descriptor version for tcgen05
+  d |= (uint64_t)2u << 61;                   // 128-byte swizzle
+  return d;
 }
 
 __device__ __forceinline__ void sts_u128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
+// a read of the pair table, which is constant once built: free to schedule
+__device__ __forceinline__ uint32_t lds_lut(uint32_t addr) {
   uint32_t v;
-  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
   return v;
 }
 
@@ -113,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int N = p.N, K = p.K;
 
   griddep_launch_dependents();
-  build_pair_lut256<FMT>(s.lut, tid, kThreads);
+  build_pair_lut<FMT>(s.lut, tid, kThreads);
   griddep_wait();
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, err)) return;
   const int nkt = (K + kBKt - 1) / kBKt;
@@ -126,6 +157,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.mdone[i], 1);
+    }
+    for (int i = 0; i < kWRing; ++i) {
+      mbar_init(&s.wfull[i], 1);
+      mbar_init(&s.wempty[i], 1);
     }
     for (int i = 0; i < kTBuf; ++i) mbar_init(&s.decoded[i], kDecThreads);
     for (int i = 0; i < 2; ++i) {
@@ -162,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp == kProdWarp) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ dY producer
     if (lane == 0) {
       int g = 0, xu = -1;
       DUnit x{};
@@ -173,17 +208,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           x = dunit_of(s, p.E, nkt, q.u);
           xu = q.u;
         }
-        mbar_arrive_expect_tx(&s.full[b], kYBytes + kWBytes);
+        mbar_arrive_expect_tx(&s.full[b], kYBytes);
         tma_load_2d(s.y[b], &tm_y, &s.full[b], q.sb * kBN, x.row0);
-        tma_load_3d(s.w[b], &tm_w, &s.full[b], x.kt * (kBKt / 2), q.sb * kBN, x.e);
       }
       if (*abort)  // let the last copies land before shared memory goes away
         for (int i = max(0, g - kRing); i < g; ++i) mbar_drain(&s.full[i % kRing], (uint32_t)(i / kRing) & 1u);
     }
+  } else if (warp == kWProdWarp) {
+    // ------------------------------------------------------------ weight producer
+    if (lane == 0) {
+      int g = 0, xu = -1;
+      DUnit x{};
+      for (Pos q{(int)blockIdx.x, 0}; q.u < U && !*abort; q = next(q), ++g) {
+        const int b = g % kWRing;
+        if (g >= kWRing && !mbar_wait(&s.wempty[b], (uint32_t)((g - kWRing) / kWRing) & 1u, err, abort)) break;
+        if (q.u != xu) {
+          x = dunit_of(s, p.E, nkt, q.u);
+          xu = q.u;
+        }
+        mbar_arrive_expect_tx(&s.wfull[b], kWBytes);
+        tma_load_3d(s.w[b], &tm_w, &s.wfull[b], x.kt * (kBKt / 2), q.sb * kBN, x.e);
+      }
+      if (*abort)
+        for (int i = max(0, g - kWRing); i < g; ++i) mbar_drain(&s.wfull[i % kWRing], (uint32_t)(i / kWRing) & 1u);
+    }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_m128((uint32_t)kBKt);
+      const uint32_t idesc = idesc_bf16_m128((uint32_t)kBKt) | (1u << 16);  // B (the decoded W tile) MN-major
       int g = 0, uc = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
@@ -199,7 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ya = smem_u32(s.y[b]), ta = smem_u32(s.t[tb]);
 #pragma unroll
           for (int q = 0; q < kBN / 16; ++q)
-            tc_mma_ss(d_tmem, sdesc_k_sw128(ya + q * 32), sdesc_k_sw128(ta + q * 32), idesc, (sb | q) != 0);
+            tc_mma_ss(d_tmem, sdesc_k_sw128(ya + q * 32), sdesc_mn_sw128(ta + q * 16 * 128, kTHalf, 1024), idesc,
+                      (sb | q) != 0);
           tc_commit(&s.mdone[b]);
         }
         if (!ok) break;
@@ -212,8 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kDecWarps) {
     // ------------------------------------------------------------ decode
-    const uint32_t lut = smem_u32(s.lut);
-    const uint32_t lane4 = (uint32_t)lane * 4u;
+    const uint32_t lut_lane = smem_u32(s.lut) + (uint32_t)lane * 4u;  // this lane's column of the pair table
     // one raw block scale of the stage at position q per thread (rows past N:
     // none); the unit's view is recomputed only when q moves to another unit
     int xs_u = -1;
@@ -249,54 +301,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t raw = scale_raw(sp, v);
       scale_store(0, raw, v);
     }
-    // block scales travel two stages ahead: loaded during stage g for stage g+2,
-    // stored at the end of stage g+1
-    sp = next(sp);
-    bool sv_a;
-    uint32_t sraw_a = scale_raw(sp, sv_a);
-    sp = next(sp);
+    // Raw block scales of stages g+1 .. g+kSQ wait in registers, stage j in
+    // slot j % kSQ: a load is issued kSQ stages before its value is stored.
+    uint32_t rq[kSQ];
+    bool vq[kSQ];
+#pragma unroll
+    for (int j = 1; j <= kSQ; ++j) {
+      sp = next(sp);
+      bool v;
+      rq[j % kSQ] = scale_raw(sp, v);
+      vq[j % kSQ] = v;
+    }
+    sp = next(sp);  // stage kSQ + 1
     dec_barrier();
-    // After an abort the loop still runs to its end (no waits, garbage
-    // results), so every decode warp reaches every named barrier.
-    int g = 0;
-    for (int u = blockIdx.x; u < U; u += gridDim.x) {
-      for (int sb = 0; sb < ns; ++sb, ++g) {
-        const int b = g % kRing, tb = g % kTBuf, sb2 = g & 1;  // sb2: scale buffer of this stage
-        bool sv_b;
-        const uint32_t sraw_b = scale_raw(sp, sv_b);
-        sp = next(sp);
-        // this stage's packed weights have landed, and the MMAs of stage g-kTBuf no longer read t[tb]
-        if (!*abort) mbar_wait(&s.full[b], (uint32_t)(g / kRing) & 1u, err, abort);
-        if (g >= kTBuf && !*abort)
-          mbar_wait(&s.mdone[(g - kTBuf) % kRing], (uint32_t)((g - kTBuf) / kRing) & 1u, err, abort);
-        // item (kp, nb) = k pair kp (k = 2kp, 2kp+1 of the tile), n rows nb*8 .. nb*8+7
-        const uint32_t wbase = smem_u32(s.w[b]);
-        const uint32_t tbase = smem_u32(s.t[tb]);
+    // The CTA's stages, flattened and unrolled by kSQ so that every queue slot
+    // index is a compile-time constant.  After an abort the loop still runs to
+    // its end (no waits, garbage results), so every decode warp reaches every
+    // named barrier.
+    const int G = ((U - 1 - (int)blockIdx.x) / (int)gridDim.x + 1) * ns;
+    for (int g0 = 0; g0 < G; g0 += kSQ) {
 #pragma unroll
-        for (int j = 0; j < (kBKt / 2) * (kBN / 8) / kDecThreads; ++j) {
-          const int item = tid + kDecThreads * j;
-          const int kp = item & 63, nb = item >> 6;
-          const int bb = FMT == 0 ? (2 * kp) / 64 : (2 * kp) / 32;
-          uint32_t pr[8];
+      for (int d = 0; d < kSQ; ++d) {
+        const int g = g0 + d;
+        if (g < G) {  // uniform over the decode warps
+          const int wb = g % kWRing, tb = g % kTBuf, sb2 = g & 1;  // sb2: scale table of this stage
+          // this stage's packed weights have landed, and the MMAs of stage g-kTBuf no longer read t[tb]
+          if (!*abort) mbar_wait(&s.wfull[wb], (uint32_t)(g / kWRing) & 1u, err, abort);
+          if (g >= kTBuf && !*abort)
+            mbar_wait(&s.mdone[(g - kTBuf) % kRing], (uint32_t)((g - kTBuf) / kRing) & 1u, err, abort);
+          // item (n, c): packed bytes 4c .. 4c+3 of weight row n, i.e. k = 8c .. 8c+7
+          // of the tile, decoded into the 16-byte chunk c % 8 of row n in half c / 8
+          const uint32_t wbase = smem_u32(s.w[wb]);
+          const uint32_t tbase = smem_u32(s.t[tb]);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t byte = lds_u8(wbase + (uint32_t)((nb * 8 + i) * (kBKt / 2) + kp));
-            pr[i] = bf16x2_mul(lut256_get(lut, byte, lane4, 0u), s.sc[sb2][nb * 8 + i][bb]);
+          for (int j = 0; j < kBN * (kBKt / 8) / kDecThreads; ++j) {
+            const int item = tid + kDecThreads * j;
+            const int c = item & 15, n = item >> 4;
+            const uint32_t word = lds_u32(wbase + (uint32_t)(n * (kBKt / 2) + 4 * c));
+            const uint32_t sc = s.sc[sb2][n][FMT == 0 ? (c >> 3) : (c >> 2)];
+            // byte i holds k = 8c+2i (low half of its pair) and 8c+2i+1
+            const uint32_t p0 = bf16x2_mul(lds_lut(lut_lane + ((word << 7) & 0x7F80u)), sc);
+            const uint32_t p1 = bf16x2_mul(lds_lut(lut_lane + ((word >> 1) & 0x7F80u)), sc);
+            const uint32_t p2 = bf16x2_mul(lds_lut(lut_lane + ((word >> 9) & 0x7F80u)), sc);
+            const uint32_t p3 = bf16x2_mul(lds_lut(lut_lane + ((word >> 17) & 0x7F80u)), sc);
+            sts_u128(tbase + (uint32_t)((c >> 3) * kTHalf + n * 128 + (((c & 7) ^ (n & 7)) << 4)), p0, p1, p2, p3);
           }
-          // row 2kp of W^T takes the low halves (even k), row 2kp+1 the high halves
-          sts_u128(tbase + sw128_chunk(2 * kp, nb), prmt_b32(pr[0], pr[1], 0x5410u),
-                   prmt_b32(pr[2], pr[3], 0x5410u), prmt_b32(pr[4], pr[5], 0x5410u),
-                   prmt_b32(pr[6], pr[7], 0x5410u));
-          sts_u128(tbase + sw128_chunk(2 * kp + 1, nb), prmt_b32(pr[0], pr[1], 0x7632u),
-                   prmt_b32(pr[2], pr[3], 0x7632u), prmt_b32(pr[4], pr[5], 0x7632u),
-                   prmt_b32(pr[6], pr[7], 0x7632u));
+          fence_proxy_async_smem();  // generic-proxy writes of t[tb] before the MMA reads them
+          mbar_arrive(&s.decoded[tb]);
+          const int q1 = (d + 1) % kSQ;    // slot of stage g+1, refilled with stage g+1+kSQ
+          scale_store(sb2 ^ 1, rq[q1], vq[q1]);
+          bool v;
+          rq[q1] = scale_raw(sp, v);
+          vq[q1] = v;
+          sp = next(sp);
+          dec_barrier();  // sc[sb2 ^ 1] written, sc[sb2] and w[wb] no longer read
+          if (tid == 0) mbar_arrive(&s.wempty[wb]);
         }
-        fence_proxy_async_smem();  // generic-proxy writes of t[tb] before the MMA reads them
-        mbar_arrive(&s.decoded[tb]);
-        scale_store(sb2 ^ 1, sraw_a, sv_a);  // stage g+1
-        sraw_a = sraw_b;
-        sv_a = sv_b;
-        dec_barrier();  // sc[sb2 ^ 1] written, sc[sb2] no longer read
       }
     }
   } else {
