@@ -8,7 +8,7 @@
 //  * the dY tile [128 rows r][64 n] bf16 arrives by TMA in the 128B-swizzled
 //    K-major layout (the MMA's A operand);
 //  * the packed weight block [64 n][64 bytes = 128 k] arrives by TMA;
-//  * the eight decode warps decode it through the pair table in its natural
+//  * a decode group of eight warps decodes it through the pair table in its natural
 //    order, weight row n with k contiguous, as two 128B-swizzled halves
 //    [64 n][64 k] bf16.  The MMA reads this tile as an MN-major B operand
 //    (MN = k, the output width; K = n, the contraction), so no transpose
@@ -16,8 +16,10 @@
 //    conflict-free 16-byte stores, and a warp reads 128 contiguous packed bytes.
 // D[r, k] accumulates in TMEM (lane = row r, column = k).  Work unit = (expert
 // e, chunk of <= 128 of its rows, 128-wide k tile); a persistent grid strides
-// over the units.  Warp roles: 8 decode warps, a dY producer, a weight
-// producer, an MMA issuer and 4 epilogue warps.
+// over the units.  Warp roles: two decode groups of 8 warps that take the
+// stages in turn (one group's waits, fences and barrier overlap the other's
+// decode), a dY producer, a weight producer, an MMA issuer and 4 epilogue
+// warps.
 //
 // Every stage waits on memory twice, for the packed weights and block scales
 // (mostly DRAM: the stacks are larger than L2) and for the dY tile (mostly L2:
@@ -26,10 +28,11 @@
 //  * dY tiles: a 4-deep TMA ring, released by the MMAs' commit;
 //  * packed weight blocks: a 12-deep TMA ring of 4 KB slots, released by the
 //    decode warps once they have read a block;
-//  * block scales: each decode thread keeps the raw scales of the next 8
-//    stages in registers (a plain load per stage, issued 8 stages before it is
-//    needed), and stores one stage ahead into a double-buffered table.
-// Four decoded W^T tiles are in flight and two accumulators, so copies, MMAs,
+//  * block scales: each decode thread keeps the raw scales of its group's
+//    next 8 stages in registers (a plain load per stage, issued 8 of the
+//    group's stages before it is needed), and stores one stage ahead into the
+//    group's double-buffered table.
+// Four decoded weight tiles are in flight and two accumulators, so copies, MMAs,
 // decode and the epilogue of the previous unit overlap.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -40,15 +43,21 @@
 namespace gnf4 {
 namespace {
 
-constexpr int kDecWarps = 8;
+constexpr int kDecWarps = 8;                    // warps of one decode group
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kProdWarp = 8, kWProdWarp = 9, kMmaWarp = 10, kEpiWarp0 = 11;
-constexpr int kThreads = (kEpiWarp0 + 4) * 32;  // 480
+constexpr int kDecGroups = 2;                   // groups take stages in turn
+constexpr int kProdWarp = kDecGroups * kDecWarps, kWProdWarp = kProdWarp + 1, kMmaWarp = kProdWarp + 2;
+constexpr int kEpiWarp0 = kProdWarp + 3;
+constexpr int kThreads = (kEpiWarp0 + 4) * 32;  // 736
 constexpr int kRing = 4;                       // dY stages in flight
 constexpr int kWRing = 12;                     // packed-weight stages in flight
 constexpr int kSQ = 8;                         // stages of block scales queued in registers
 constexpr int kTBuf = 4;                       // decoded W^T tiles in flight
 static_assert(kTBuf <= kRing, "a decoded tile is released through the ring's MMA-done barriers");
+// A group waits on a ring slot's phase P only after it has itself waited on
+// phase P-1 (a parity wait cannot tell the two apart): the stage that used
+// the slot one lap earlier must belong to the same group.
+static_assert(kRing % kDecGroups == 0 && kWRing % kDecGroups == 0, "ring depths must be multiples of the group count");
 constexpr int kBR = 128;                   // rows per unit (MMA M)
 constexpr int kBKt = 128;                  // k per unit (MMA N)
 constexpr int kBN = 64;                    // n per stage (four k-steps of 16)
@@ -63,7 +72,7 @@ struct DSmem {
   uint8_t t[kTBuf][kTBytes];  // decoded W tiles, two 64-k halves each
   uint8_t w[kWRing][kWBytes];  // packed weight blocks
   uint32_t lut[kLutWords];    // pair table, 128-byte entries (32 lanes)
-  uint32_t sc[2][kBN][4];     // raw block scales of a stage: 64 rows x (2 NF4 | 4 MXFP4) blocks of the k tile
+  uint32_t sc[kDecGroups][2][kBN][4];  // per decode group, two stages of block scales (bf16x2): 64 rows x (2 NF4 | 4 MXFP4) blocks of the k tile
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
@@ -263,8 +272,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_drain(&s.drain, 0);
       }
     }
-  } else if (warp < kDecWarps) {
+  } else if (warp < kProdWarp) {
     // ------------------------------------------------------------ decode
+    // group grp takes the stages g = grp (mod kDecGroups); gtid = thread of the group
+    const int grp = warp / kDecWarps, gtid = tid - grp * kDecThreads;
     const uint32_t lut_lane = smem_u32(s.lut) + (uint32_t)lane * 4u;  // this lane's column of the pair table
     // one raw block scale of the stage at position q per thread (rows past N:
     // none); the unit's view is recomputed only when q moves to another unit
@@ -272,13 +283,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     DUnit xs{};
     auto scale_raw = [&](Pos q, bool& valid) -> uint32_t {
       valid = false;
-      if (q.u >= U || tid >= kBN * spk) return 0u;
+      if (q.u >= U || gtid >= kBN * spk) return 0u;
       if (q.u != xs_u) {
         xs = dunit_of(s, p.E, nkt, q.u);
         xs_u = q.u;
       }
       const DUnit& x = xs;
-      const int rr = tid / spk, bb = tid - rr * spk;
+      const int rr = gtid / spk, bb = gtid - rr * spk;
       const int n = q.sb * kBN + rr;
       if (n >= N) return 0u;
       const int blk = min(x.kt * spk + bb, nsc - 1);  // past K: any valid scale, never stored
@@ -287,44 +298,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       return FMT == 0 ? __float_as_uint(__ldg(reinterpret_cast<const float*>(p.scales) + idx))
                       : (uint32_t)__ldg(reinterpret_cast<const uint8_t*>(p.scales) + idx);
     };
-    // bf16x2 scale pair (0 for rows past N) into sc[buf]
+    // bf16x2 scale pair (0 for rows past N) into the group's sc[buf]
     auto scale_store = [&](int buf, uint32_t raw, bool valid) {
-      if (tid >= kBN * spk) return;
-      const int rr = tid / spk, bb = tid - rr * spk;
-      s.sc[buf][rr][bb] = !valid ? 0u : (FMT == 0 ? f32_to_bf16x2_rn(__uint_as_float(raw)) : e8m0_to_bf16x2(raw));
+      if (gtid >= kBN * spk) return;
+      const int rr = gtid / spk, bb = gtid - rr * spk;
+      s.sc[grp][buf][rr][bb] = !valid ? 0u : (FMT == 0 ? f32_to_bf16x2_rn(__uint_as_float(raw)) : e8m0_to_bf16x2(raw));
     };
-    auto dec_barrier = [&]() { asm volatile("bar.sync 1, %0;" ::"r"(kDecThreads) : "memory"); };
+    auto dec_barrier = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(kDecThreads) : "memory"); };
+    auto next_own = [&](Pos q) {  // this group's next stage
+#pragma unroll
+      for (int i = 0; i < kDecGroups; ++i) q = next(q);
+      return q;
+    };
 
     Pos sp{(int)blockIdx.x, 0};
+    for (int i = 0; i < grp; ++i) sp = next(sp);  // the group's first stage
     {
       bool v;
       const uint32_t raw = scale_raw(sp, v);
       scale_store(0, raw, v);
     }
-    // Raw block scales of stages g+1 .. g+kSQ wait in registers, stage j in
-    // slot j % kSQ: a load is issued kSQ stages before its value is stored.
+    // Raw block scales of the group's next kSQ stages wait in registers (its
+    // i-th stage in slot i % kSQ): a load is issued kSQ of the group's stages
+    // before its value is stored.
     uint32_t rq[kSQ];
     bool vq[kSQ];
 #pragma unroll
     for (int j = 1; j <= kSQ; ++j) {
-      sp = next(sp);
+      sp = next_own(sp);
       bool v;
       rq[j % kSQ] = scale_raw(sp, v);
       vq[j % kSQ] = v;
     }
-    sp = next(sp);  // stage kSQ + 1
+    sp = next_own(sp);  // the group's stage kSQ + 1
     dec_barrier();
-    // The CTA's stages, flattened and unrolled by kSQ so that every queue slot
-    // index is a compile-time constant.  After an abort the loop still runs to
-    // its end (no waits, garbage results), so every decode warp reaches every
-    // named barrier.
-    const int G = ((U - 1 - (int)blockIdx.x) / (int)gridDim.x + 1) * ns;
-    for (int g0 = 0; g0 < G; g0 += kSQ) {
+    // The group's stages, flattened and unrolled by kSQ so that every queue
+    // slot index is a compile-time constant.  After an abort the loop still
+    // runs to its end (no waits, garbage results), so every decode warp
+    // reaches every named barrier.
+    const int G = ((U - 1 - (int)blockIdx.x) / (int)gridDim.x + 1) * ns;  // the CTA's stages
+    const int Gi = (G - grp + kDecGroups - 1) / kDecGroups;               // this group's
+    for (int i0 = 0; i0 < Gi; i0 += kSQ) {
 #pragma unroll
       for (int d = 0; d < kSQ; ++d) {
-        const int g = g0 + d;
-        if (g < G) {  // uniform over the decode warps
-          const int wb = g % kWRing, tb = g % kTBuf, sb2 = g & 1;  // sb2: scale table of this stage
+        const int i = i0 + d, g = grp + kDecGroups * i;
+        if (i < Gi) {  // uniform over the group
+          const int wb = g % kWRing, tb = g % kTBuf, sb2 = i & 1;  // sb2: scale table of this stage
           // this stage's packed weights have landed, and the MMAs of stage g-kTBuf no longer read t[tb]
           if (!*abort) mbar_wait(&s.wfull[wb], (uint32_t)(g / kWRing) & 1u, err, abort);
           if (g >= kTBuf && !*abort)
@@ -335,10 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t tbase = smem_u32(s.t[tb]);
 #pragma unroll
           for (int j = 0; j < kBN * (kBKt / 8) / kDecThreads; ++j) {
-            const int item = tid + kDecThreads * j;
+            const int item = gtid + kDecThreads * j;
             const int c = item & 15, n = item >> 4;
             const uint32_t word = lds_u32(wbase + (uint32_t)(n * (kBKt / 2) + 4 * c));
-            const uint32_t sc = s.sc[sb2][n][FMT == 0 ? (c >> 3) : (c >> 2)];
+            const uint32_t sc = s.sc[grp][sb2][n][FMT == 0 ? (c >> 3) : (c >> 2)];
             // byte i holds k = 8c+2i (low half of its pair) and 8c+2i+1
             const uint32_t p0 = bf16x2_mul(lds_lut(lut_lane + ((word << 7) & 0x7F80u)), sc);
             const uint32_t p1 = bf16x2_mul(lds_lut(lut_lane + ((word >> 1) & 0x7F80u)), sc);
@@ -348,14 +367,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();  // generic-proxy writes of t[tb] before the MMA reads them
           mbar_arrive(&s.decoded[tb]);
-          const int q1 = (d + 1) % kSQ;    // slot of stage g+1, refilled with stage g+1+kSQ
+          const int q1 = (d + 1) % kSQ;  // slot of the group's stage i+1, refilled with its stage i+1+kSQ
           scale_store(sb2 ^ 1, rq[q1], vq[q1]);
           bool v;
           rq[q1] = scale_raw(sp, v);
           vq[q1] = v;
-          sp = next(sp);
+          sp = next_own(sp);
           dec_barrier();  // sc[sb2 ^ 1] written, sc[sb2] and w[wb] no longer read
-          if (tid == 0) mbar_arrive(&s.wempty[wb]);
+          if (gtid == 0) mbar_arrive(&s.wempty[wb]);
         }
       }
     }
