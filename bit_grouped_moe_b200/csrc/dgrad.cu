@@ -8,7 +8,7 @@
 //  * the dY tile [128 rows r][64 n] bf16 arrives by TMA in the 128B-swizzled
 //    K-major layout (the MMA's A operand);
 //  * the packed weight block [64 n][64 bytes = 128 k] arrives by TMA;
-//  * a decode group of eight warps decodes it through the pair table in its natural
+//  * a decode group of four warps decodes it through the pair table in its natural
 //    order, weight row n with k contiguous, as two 128B-swizzled halves
 //    [64 n][64 k] bf16.  The MMA reads this tile as an MN-major B operand
 //    (MN = k, the output width; K = n, the contraction), so no transpose
@@ -16,24 +16,25 @@
 //    conflict-free 16-byte stores, and a warp reads 128 contiguous packed bytes.
 // D[r, k] accumulates in TMEM (lane = row r, column = k).  Work unit = (expert
 // e, chunk of <= 128 of its rows, 128-wide k tile); a persistent grid strides
-// over the units.  Warp roles: two decode groups of 8 warps that take the
-// stages in turn (one group's waits, fences and barrier overlap the other's
-// decode), a dY producer, a weight producer, an MMA issuer and 4 epilogue
-// warps.
+// over the units.  Warp roles: four decode groups of 4 warps that take the
+// stages in turn (one group's waits, proxy fence and barrier overlap the
+// others' decode), a dY producer, a weight producer, an MMA issuer and 4
+// epilogue warps.
 //
 // Every stage waits on memory twice, for the packed weights and block scales
 // (mostly DRAM: the stacks are larger than L2) and for the dY tile (mostly L2:
 // the k tiles of one row chunk run side by side).  Each source has its own
 // queue, deep enough to cover its latency:
 //  * dY tiles: a 4-deep TMA ring, released by the MMAs' commit;
-//  * packed weight blocks: a 12-deep TMA ring of 4 KB slots, released by the
-//    decode warps once they have read a block;
+//  * packed weight blocks: an 8-deep TMA ring of 4 KB slots, released by the
+//    decode group once it has read a block;
 //  * block scales: each decode thread keeps the raw scales of its group's
-//    next 8 stages in registers (a plain load per stage, issued 8 of the
-//    group's stages before it is needed), and stores one stage ahead into the
-//    group's double-buffered table.
-// Four decoded weight tiles are in flight and two accumulators, so copies, MMAs,
-// decode and the epilogue of the previous unit overlap.
+//    next 4 stages (16 stages of the CTA) in registers, a plain load issued
+//    that far ahead, and stores one stage ahead into the group's
+//    double-buffered table.
+// Four decoded weight tiles are in flight (one per group) and two
+// accumulators, so copies, MMAs, decode and the epilogue of the previous unit
+// overlap.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -43,16 +44,16 @@
 namespace gnf4 {
 namespace {
 
-constexpr int kDecWarps = 8;                    // warps of one decode group
+constexpr int kDecWarps = 4;                    // warps of one decode group
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecGroups = 2;                   // groups take stages in turn
+constexpr int kDecGroups = 4;                   // groups take stages in turn
 constexpr int kProdWarp = kDecGroups * kDecWarps, kWProdWarp = kProdWarp + 1, kMmaWarp = kProdWarp + 2;
 constexpr int kEpiWarp0 = kProdWarp + 3;
 constexpr int kThreads = (kEpiWarp0 + 4) * 32;  // 736
 constexpr int kRing = 4;                       // dY stages in flight
-constexpr int kWRing = 12;                     // packed-weight stages in flight
-constexpr int kSQ = 8;                         // stages of block scales queued in registers
-constexpr int kTBuf = 4;                       // decoded W^T tiles in flight
+constexpr int kWRing = 8;                      // packed-weight stages in flight
+constexpr int kSQ = 4;                         // stages of block scales queued in registers
+constexpr int kTBuf = 4;                       // decoded weight tiles in flight
 static_assert(kTBuf <= kRing, "a decoded tile is released through the ring's MMA-done barriers");
 // A group waits on a ring slot's phase P only after it has itself waited on
 // phase P-1 (a parity wait cannot tell the two apart): the stage that used
@@ -191,7 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   const int nsc = FMT == 0 ? K / 64 : K / 32;        // scales per weight row
-  const int spk = FMT == 0 ? kBKt / 64 : kBKt / 32;  // scale blocks of a row in one k tile
+  constexpr int spk = FMT == 0 ? kBKt / 64 : kBKt / 32;                  // scale blocks of a row in one k tile
+  constexpr int kSpt = (kBN * spk + kDecThreads - 1) / kDecThreads;  // block scales per decode thread per stage
+  constexpr int kItems = kBN * (kBKt / 8) / kDecThreads;             // 16-byte chunks per decode thread per stage
 
   // The CTA's stage stream: stage g = (unit u, n block sb), units strided by the grid.
   struct Pos {
@@ -277,32 +280,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     // group grp takes the stages g = grp (mod kDecGroups); gtid = thread of the group
     const int grp = warp / kDecWarps, gtid = tid - grp * kDecThreads;
     const uint32_t lut_lane = smem_u32(s.lut) + (uint32_t)lane * 4u;  // this lane's column of the pair table
-    // one raw block scale of the stage at position q per thread (rows past N:
-    // none); the unit's view is recomputed only when q moves to another unit
+    // Raw block scale j (of kSpt) of this thread for the stage at position q;
+    // the unit's view is recomputed only when q moves to another unit.  A row
+    // past N has no scale and reads as 0, which stores as a zero factor: NF4
+    // keeps the fp32 bits (+0 converts to the bf16 zero), MXFP4 marks a real
+    // e8m0 byte with bit 8.
     int xs_u = -1;
     DUnit xs{};
-    auto scale_raw = [&](Pos q, bool& valid) -> uint32_t {
-      valid = false;
-      if (q.u >= U || gtid >= kBN * spk) return 0u;
+    auto scale_raw = [&](Pos q, int j) -> uint32_t {
+      const int vi = gtid + kDecThreads * j;
+      if (q.u >= U || vi >= kBN * spk) return 0u;
       if (q.u != xs_u) {
         xs = dunit_of(s, p.E, nkt, q.u);
         xs_u = q.u;
       }
       const DUnit& x = xs;
-      const int rr = gtid / spk, bb = gtid - rr * spk;
+      const int rr = vi / spk, bb = vi - rr * spk;
       const int n = q.sb * kBN + rr;
       if (n >= N) return 0u;
       const int blk = min(x.kt * spk + bb, nsc - 1);  // past K: any valid scale, never stored
       const size_t idx = ((size_t)x.e * N + (size_t)n) * (size_t)nsc + (size_t)blk;
-      valid = true;
       return FMT == 0 ? __float_as_uint(__ldg(reinterpret_cast<const float*>(p.scales) + idx))
-                      : (uint32_t)__ldg(reinterpret_cast<const uint8_t*>(p.scales) + idx);
+                      : 0x100u | (uint32_t)__ldg(reinterpret_cast<const uint8_t*>(p.scales) + idx);
     };
-    // bf16x2 scale pair (0 for rows past N) into the group's sc[buf]
-    auto scale_store = [&](int buf, uint32_t raw, bool valid) {
-      if (gtid >= kBN * spk) return;
-      const int rr = gtid / spk, bb = gtid - rr * spk;
-      s.sc[grp][buf][rr][bb] = !valid ? 0u : (FMT == 0 ? f32_to_bf16x2_rn(__uint_as_float(raw)) : e8m0_to_bf16x2(raw));
+    // bf16x2 scale pair into the group's sc[buf]
+    auto scale_store = [&](int buf, int j, uint32_t raw) {
+      const int vi = gtid + kDecThreads * j;
+      if (vi >= kBN * spk) return;
+      const int rr = vi / spk, bb = vi - rr * spk;
+      s.sc[grp][buf][rr][bb] = FMT == 0 ? f32_to_bf16x2_rn(__uint_as_float(raw))
+                                        : ((raw & 0x100u) ? e8m0_to_bf16x2(raw & 0xFFu) : 0u);
     };
     auto dec_barrier = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(kDecThreads) : "memory"); };
     auto next_own = [&](Pos q) {  // this group's next stage
@@ -313,22 +320,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     Pos sp{(int)blockIdx.x, 0};
     for (int i = 0; i < grp; ++i) sp = next(sp);  // the group's first stage
-    {
-      bool v;
-      const uint32_t raw = scale_raw(sp, v);
-      scale_store(0, raw, v);
-    }
+#pragma unroll
+    for (int j = 0; j < kSpt; ++j) scale_store(0, j, scale_raw(sp, j));
     // Raw block scales of the group's next kSQ stages wait in registers (its
     // i-th stage in slot i % kSQ): a load is issued kSQ of the group's stages
     // before its value is stored.
-    uint32_t rq[kSQ];
-    bool vq[kSQ];
+    uint32_t rq[kSQ][kSpt];
 #pragma unroll
-    for (int j = 1; j <= kSQ; ++j) {
+    for (int i = 1; i <= kSQ; ++i) {
       sp = next_own(sp);
-      bool v;
-      rq[j % kSQ] = scale_raw(sp, v);
-      vq[j % kSQ] = v;
+#pragma unroll
+      for (int j = 0; j < kSpt; ++j) rq[i % kSQ][j] = scale_raw(sp, j);
     }
     sp = next_own(sp);  // the group's stage kSQ + 1
     dec_barrier();
@@ -352,8 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // of the tile, decoded into the 16-byte chunk c % 8 of row n in half c / 8
           const uint32_t wbase = smem_u32(s.w[wb]);
           const uint32_t tbase = smem_u32(s.t[tb]);
+          // item (n, c): packed bytes 4c .. 4c+3 of weight row n, i.e. k = 8c .. 8c+7
+          // of the tile, decoded into the 16-byte chunk c % 8 of row n in half c / 8
 #pragma unroll
-          for (int j = 0; j < kBN * (kBKt / 8) / kDecThreads; ++j) {
+          for (int j = 0; j < kItems; ++j) {
             const int item = gtid + kDecThreads * j;
             const int c = item & 15, n = item >> 4;
             const uint32_t word = lds_u32(wbase + (uint32_t)(n * (kBKt / 2) + 4 * c));
@@ -368,10 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();  // generic-proxy writes of t[tb] before the MMA reads them
           mbar_arrive(&s.decoded[tb]);
           const int q1 = (d + 1) % kSQ;  // slot of the group's stage i+1, refilled with its stage i+1+kSQ
-          scale_store(sb2 ^ 1, rq[q1], vq[q1]);
-          bool v;
-          rq[q1] = scale_raw(sp, v);
-          vq[q1] = v;
+#pragma unroll
+          for (int j = 0; j < kSpt; ++j) {
+            scale_store(sb2 ^ 1, j, rq[q1][j]);
+            rq[q1][j] = scale_raw(sp, j);
+          }
           sp = next_own(sp);
           dec_barrier();  // sc[sb2 ^ 1] written, sc[sb2] and w[wb] no longer read
           if (gtid == 0) mbar_arrive(&s.wempty[wb]);
