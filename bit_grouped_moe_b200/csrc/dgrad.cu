@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.wfull[i], 1);
       mbar_init(&s.wempty[i], 1);
     }
-    for (int i = 0; i < kTBuf; ++i) mbar_init(&s.decoded[i], kDecThreads);
+    for (int i = 0; i < kTBuf; ++i) mbar_init(&s.decoded[i], kDecWarps);  // one arrival per warp of a group
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.accf[i], 1);
       mbar_init(&s.acce[i], 128);
@@ -369,8 +369,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t p3 = bf16x2_mul(lds_lut(lut_lane + ((word >> 17) & 0x7F80u)), sc);
             sts_u128(tbase + (uint32_t)((c >> 3) * kTHalf + n * 128 + (((c & 7) ^ (n & 7)) << 4)), p0, p1, p2, p3);
           }
-          fence_proxy_async_smem();  // generic-proxy writes of t[tb] before the MMA reads them
-          mbar_arrive(&s.decoded[tb]);
+          // every thread orders its generic-proxy writes of t[tb] before the
+          // MMA's reads; one lane per warp then signals (32 arrivals on one
+          // word would serialise)
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.decoded[tb]);
           const int q1 = (d + 1) % kSQ;  // slot of the group's stage i+1, refilled with its stage i+1+kSQ
 #pragma unroll
           for (int j = 0; j < kSpt; ++j) {
@@ -417,7 +421,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               reinterpret_cast<uint4*>(dst)[qq] = o;
             }
           } else {
-            for (int i = 0; i < 32 && kc + i < K; ++i) dst[i] = __float2bfloat16_rn(__uint_as_float(v[i]));
+#pragma unroll
+            for (int i = 0; i < 32; ++i)  // static indices keep v in registers
+              if (kc + i < K) dst[i] = __float2bfloat16_rn(__uint_as_float(v[i]));
           }
         }
       }
