@@ -423,8 +423,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           __nv_bfloat16* hcol = p.y + (size_t)x.row0 * I + col;
 #pragma unroll
           for (int m = 0; m < 16; ++m) {
-            const float keep = __uint_as_float(v[2 * m + (up_lane ? 1 : 0)]);
-            const float send = __uint_as_float(v[2 * m + (up_lane ? 0 : 1)]);
+            // select between two static indices so v stays in registers
+            const float even = __uint_as_float(v[2 * m]), odd = __uint_as_float(v[2 * m + 1]);
+            const float keep = up_lane ? odd : even;
+            const float send = up_lane ? even : odd;
             const float got = __shfl_xor_sync(0xffffffffu, send, 16);
             const int i = 2 * m + (up_lane ? 1 : 0);
             // low lane: gate = keep (row 2m), up = got; high lane: up = keep (row 2m+1), gate = got
