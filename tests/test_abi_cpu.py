@@ -159,3 +159,48 @@ def test_fused_combine_gemv_refusals(g):
 def test_selftest_limit_refusal(g):
     assert g._lib.gnf4_selftest_bounded_wait(0, None) == g.ERR_INVALID_ARG
     assert g._lib.gnf4_selftest_bounded_wait((1 << 32) + 1, None) == g.ERR_INVALID_ARG
+
+
+DGRAD = ["gnf4_grouped_dgrad_nf4", "gnf4_grouped_dgrad_mxfp4"]
+
+
+@pytest.mark.parametrize("name", DGRAD)
+@pytest.mark.parametrize("E,N,K", [(0, 64, 64), (1025, 64, 64), (4, 60, 64), (4, 64, 0), (4, 64, 16)])
+def test_dgrad_shape_refusals(g, name, E, N, K):
+    """The data gradient takes the grouped GEMM's shape rules (N = the
+    contracted weight rows, K = the output width) before any pointer."""
+    st = getattr(g._lib, name)(None, None, None, ctypes.c_void_p(16), None, E, N, K, 8, None, None)
+    assert st == g.ERR_UNSUPPORTED_SHAPE, g.last_error()
+
+
+@pytest.mark.parametrize("name", DGRAD)
+def test_dgrad_group_description_and_empty_call(g, name):
+    f = getattr(g._lib, name)
+    off = ctypes.c_void_p(16)
+    assert f(None, None, None, None, None, 4, 64, 64, 8, None, None) == g.ERR_INVALID_ARG
+    assert f(None, None, None, off, off, 4, 64, 64, 8, None, None) == g.ERR_INVALID_ARG
+    assert f(None, None, None, off, None, 4, 64, 64, 0, None, None) == g.OK  # M == 0 launches nothing
+
+
+def test_dgrad_host_pointers_refused(g):
+    """A CPU buffer is never computed on: the call refuses it (no CPU fallback)."""
+    dy = np.zeros((8, 64), np.uint16)
+    w = np.zeros((4, 64, 32), np.uint8)
+    am = np.ones((4, 64, 1), np.float32)
+    off = np.array([0, 2, 4, 6, 8], np.int32)
+    dx = np.zeros((8, 64), np.uint16)
+    p = lambda x: x.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    st = g._lib.gnf4_grouped_dgrad_nf4(p(dy), p(w), p(am), p(off), None, 4, 64, 64, 8, p(dx), None)
+    assert st in (g.ERR_INVALID_ARG, g.ERR_CUDA)
+
+
+@pytest.mark.parametrize("name", ["gnf4_grouped_gemm_nf4_swiglu", "gnf4_grouped_gemm_mxfp4_swiglu",
+                                  "gnf4_grouped_gemv_nf4_swiglu", "gnf4_grouped_gemv_mxfp4_swiglu"])
+def test_swiglu_width_refusals_and_empty_call(g, name):
+    """The output width I must be a positive multiple of 64 (a gate_up stack
+    of 2I rows, 64 gate + 64 up rows per weight tile)."""
+    f = getattr(g._lib, name)
+    off = ctypes.c_void_p(16)
+    for width in (0, 32, 96, -64):
+        assert f(None, None, None, off, None, 4, width, 64, 8, None, None) == g.ERR_UNSUPPORTED_SHAPE, width
+    assert f(None, None, None, off, None, 4, 64, 64, 0, None, None) == g.OK  # M == 0 launches nothing
