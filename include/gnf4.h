@@ -340,8 +340,8 @@ gnf4_status gnf4_quantize_mxfp8(const void *x, int M, int K, uint8_t *codes, uin
 
 /* Two-term form (the activations as hi + lo, two MXFP8 tensors), which
  * keeps the bf16-activation accuracy of the MXFP4 GEMM on the native path
- * (SURVEY reading of the block-scaled MXFP4 operand; the pages give no
- * rule).  Per block of 32 consecutive k of one row:
+ * (a reading: no page gives a rule for splitting the activation operand of
+ * the block-scaled MXFP4 GEMM).  Per block of 32 consecutive k of one row:
  *     hi = MXFP8 of x, lo = MXFP8 of the exact residual r = x - hi,
  *     both with X = floor(log2(max |value|)) - 7 (one binade of headroom,
  *     so no element saturates), e4m3 round to nearest even;

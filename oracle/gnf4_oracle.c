@@ -43,8 +43,8 @@
  *   [OCP-MX]   OCP Microscaling Formats (MX) v1.0: e2m1 element, e8m0 scale,
  *              shared exponent floor(log2(amax)) - emax_elem (reading C8).
  *
- * Readings of points the pages leave open are listed in the design doc under
- * "Readings"; each function below names the ones it depends on.
+ * Points the pages leave open are taken as numbered readings (C1, C2, ...);
+ * each function below names the ones it depends on.
  */
 #include <math.h>
 #include <stdint.h>
