@@ -34,12 +34,15 @@ if ROOT not in sys.path:
 from bit_grouped_moe_b200 import inputs  # noqa: E402
 
 METRIC = "grouped 4-bit GEMM TFLOP/s (prefill) & weight GB/s (decode) vs B200 roofline"
-DEFAULT_WORKLOAD = "olmoe-decode-t8"
+DEFAULT_WORKLOAD = "kimi-prefill"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-N_WEIGHT_COPIES = 4  # default; --weight-copies changes it (profiling uses 1)
+N_WEIGHT_COPIES = 4  # rotating copies when one weight stack fits in L2 (--weight-copies overrides)
+L2_BYTES = 126 * 2**20
 N_BATCHES = 8
 GRAPH_STEPS = 20  # steps captured per CUDA graph (decode timing only)
-EVENT_EVERY = 7  # the dominant kernel is event-timed on every 7th timed step (7 is coprime with the batch and copy rotations)
+DOMINANT_REPS = 60  # launches of the dominant kernel timed one by one (median, p10, p90)
+# Nominal dense peaks of one B200 (context beside the measured ones): TFLOP/s per MMA kind, HBM3e GB/s.
+NOMINAL = {"bf16": 2250.0, "fp8": 4500.0, "fp4": 9000.0, "hbm_gbs": 7700.0}
 
 
 # ------------------------------------------------------------------ helpers
@@ -347,6 +350,26 @@ class Workload:
         else:
             self.fn(a2, w2, s2, self.y2, offsets=self.off)
 
+    def dominant(self, i):
+        """Launches the dominant kernel alone (the first projection, or dX of
+        it for the backward step) on weight copy i, with the routing of the
+        last step: the kernel the roofline is reported for."""
+        (w1, s1), _ = self.stacks[i % N_WEIGHT_COPIES]
+        g = self.g
+        if self.dgrad:
+            self.dfn(self.dy1, w1, s1, self.dx1, offsets=self.off)
+        elif self.w4a8:
+            if self.a4:
+                g.grouped_gemm_w4a4(self.qa1, self.sa1, w1, s1, self.y1, offsets=self.off)
+            elif self.split:
+                g.grouped_gemm_w4a8x2(self.qa1, self.sa1, self.la1, self.ls1, w1, s1, self.y1, offsets=self.off)
+            else:
+                g.grouped_gemm_w4a8(self.qa1, self.sa1, w1, s1, self.y1, offsets=self.off)
+        elif self.swiglu:
+            self.fn1(self.xs, w1, s1, self.hs, offsets=self.off)
+        else:
+            self.fn(self.xs, w1, s1, self.y1, offsets=self.off)
+
     def launches_per_step(self):
         # route (one launch for at most 256 pairs, else hist + scan + scatter + gather) + 2 projections + combine
         route = 1 if 0 < self.M <= 256 else 4
@@ -432,11 +455,12 @@ def oracle_step(wl_obj, batch_i, n_slice=None):
     return int(wbytes), 2 * wl_obj.M * (n1 * wl_obj.p1.K + n2 * wl_obj.p2.K)
 
 
-def cpu_baseline(wl_obj, budget_s=15.0):
-    """Oracle timed on the host cores on a bounded sample of the workload."""
+def cpu_baseline(wl_obj, budget_s=15.0, threads=None):
+    """Oracle timed on the host cores (all of them, or `threads`) on a bounded
+    sample of the workload."""
     import oracle
 
-    cores = os.cpu_count() or 1
+    cores = threads or os.cpu_count() or 1
     oracle.set_threads(cores)
     # calibrate the weight-row slice so that one step costs ~budget/6
     t0 = time.perf_counter()
@@ -455,6 +479,79 @@ def cpu_baseline(wl_obj, budget_s=15.0):
     return {"bytes": tot_b, "flops": tot_f, "seconds": dt, "cores": cores, "steps": steps, "n_slice": n_slice}
 
 
+def roofline(wl, args, peaks, peak_src, dom_ms, hit, dom_stats, traffic):
+    """Roofline of the dominant kernel (median of its own timed loop).
+
+    F = 2*M*N*K useful flops; B = algorithmic bytes (weights + scales of the
+    experts hit, activations read once, output written once).  The bound is
+    the combined one, t = max(F / tensor peak, B / HBM peak), with the tensor
+    peak of the MMA kind the kernel executes expressed in useful flops (the
+    two-term form issues two fp8-rate MMAs per useful one).  `frac` = t /
+    measured time against the measured peaks; the same against the nominal
+    dense peaks is `frac_nominal`.  The measured tensor peak is the burst
+    figure, or the sustained one when the kernel's own loop ran power-capped
+    (sw_power_cap active or the median SM clock below 90% of max)."""
+    p = wl.p1
+    M, N, K = wl.M, p.N, p.K
+    F = 2.0 * M * N * K
+    wbytes = wl.weight_bytes(p, hit)
+    if wl.dgrad:
+        io = 2 * M * N + 2 * M * K  # dY read, dX written
+        kind, per = "bf16", 1.0
+    elif wl.w4a8:
+        if wl.a4:
+            abytes, kind, per = M * K // 2 + M * K // 32, "fp4", 1.0
+        elif wl.split:
+            abytes, kind, per = 2 * (M * K + M * K // 32), "fp8", 0.5
+        else:
+            abytes, kind, per = M * K + M * K // 32, "fp8", 1.0
+        io = abytes + 2 * M * N
+    else:
+        n_out = N // 2 if wl.swiglu else N
+        io = 2 * M * K + 2 * M * n_out
+        kind, per = "bf16", 1.0
+    B = float(wbytes + io)
+    ratio = {"bf16": 1.0, "fp8": 2.0, "fp4": 4.0}[kind]
+    dc = dom_stats.get("clocks") or {}
+    capped = ("sw_power_cap" in (dc.get("reasons") or [])) or (
+        dc.get("sm_mhz") is not None and dc.get("sm_max_mhz") and dc["sm_mhz"] < 0.9 * dc["sm_max_mhz"])
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * ratio * per
+    sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * ratio * per
+    tpk = sust if capped else burst
+    nominal_t = NOMINAL[kind] * per
+    hbm = peaks["hbm_gbs"]
+    t = dom_ms / 1e3
+    t_tensor, t_hbm = F / (tpk * 1e12), B / (hbm * 1e9)
+    bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    t_nom = max(F / (nominal_t * 1e12), B / (NOMINAL["hbm_gbs"] * 1e9))
+    achieved = F / t / 1e12 if bound == "tensor" else B / t / 1e9
+    kname = (f"dgrad_tc_kernel<{wl.wl.fmt}> (dX of {p.name}, K={K}, N={N})" if wl.dgrad else
+             f"gemm_mx_kernel<W4A4> ({p.name}, K={K}, N={N})" if wl.a4 else
+             f"gemm_mx_kernel<two-term> ({p.name}, K={K}, N={N})" if wl.split else
+             f"gemm_mx_kernel<W4A8> ({p.name}, K={K}, N={N})" if wl.w4a8 else
+             f"gemv_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({p.name}, K={K}, N={N})" if wl.decode else
+             f"gemm_tc_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({p.name}, K={K}, N={N})")
+    return {
+        "bound": bound, "achieved": round(achieved, 1), "peak": round(tpk if bound == "tensor" else hbm, 1),
+        "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": round(max(t_tensor, t_hbm) / t, 4),
+        "traffic": traffic, "kernel": kname,
+        "algorithmic_flops_per_launch": int(F), "algorithmic_bytes_per_launch": int(B),
+        "experts_hit": int(hit), "launch_us": dom_stats,
+        "tensor": {"achieved_tflops": round(F / t / 1e12, 1), "mma_kind": kind,
+                   "peak_measured": round(tpk, 1), "frac_measured": round(F / t / 1e12 / tpk, 4),
+                   "peak_nominal": round(nominal_t, 1), "frac_nominal": round(F / t / 1e12 / nominal_t, 4),
+                   "peak_burst": round(burst, 1), "peak_sustained": round(sust, 1),
+                   "peak_choice": "sustained (loop ran power-capped)" if capped else "burst"},
+        "hbm": {"achieved_gbs": round(B / t / 1e9, 1), "peak_measured": hbm,
+                "frac_measured": round(B / t / 1e9 / hbm, 4), "peak_nominal": NOMINAL["hbm_gbs"],
+                "frac_nominal": round(B / t / 1e9 / NOMINAL["hbm_gbs"], 4)},
+        "combined_bound_us": round(max(t_tensor, t_hbm) * 1e6, 3), "frac_nominal": round(t_nom / t, 4),
+        "peak_source": f"{peak_src} (MEASURED_PEAKS.json: bf16_tflops / bf16_tflops_sustained x the nominal "
+                       f"{kind}/bf16 ratio {ratio:g}{', halved for the two-term form' if per != 1 else ''}; hbm_gbs)",
+    }
+
+
+
 # ------------------------------------------------------------------ main
 
 
@@ -468,8 +565,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dgrad", action="store_true",
                     help="time the backward step instead: route + the dgrad of both projections (TFLOP/s)")
-    ap.add_argument("--graph", action="store_true",
-                    help=f"decode: also time the steps replayed from one CUDA graph of {20} steps")
+    ap.add_argument("--no-graph", action="store_true",
+                    help=f"decode: skip timing the steps replayed from one CUDA graph of {GRAPH_STEPS} steps")
     ap.add_argument("--w4a8", action="store_true",
                     help="MXFP4 workloads: native W4A8 mode (MXFP8 activations, block-scaled tcgen05 GEMM)")
     ap.add_argument("--w4a8x2", action="store_true",
@@ -482,9 +579,15 @@ def main():
                          "(measured slower on B200: the epilogue's round trips extend every unit)")
     ap.add_argument("--swiglu", action="store_true",
                     help="first projection = fused gate_up + SwiGLU (gate rows first); the second reads its output")
-    ap.add_argument("--weight-copies", type=int, default=N_WEIGHT_COPIES,
+    ap.add_argument("--weight-copies", type=int, default=None,
                     help="rotating copies of every weight stack (4 keeps the rotation larger than L2)")
     args = ap.parse_args()
+    wl0 = inputs.WORKLOADS[args.workload]
+    if args.weight_copies is None:
+        # one stack of the first projection larger than 3x L2 needs no rotation
+        per = 0.5 + (4 / 64 if wl0.fmt == "nf4" else 1 / 32)
+        one = wl0.E * wl0.projections[0].N * wl0.projections[0].K * per
+        args.weight_copies = 1 if one > 3 * L2_BYTES else N_WEIGHT_COPIES
     globals()["N_WEIGHT_COPIES"] = max(1, args.weight_copies)
 
     wl_def = inputs.WORKLOADS[args.workload]
@@ -515,7 +618,8 @@ def _config(wl_obj_or_def, world):
         "experts": wl.E, "top_k": wl.k, "tokens_per_step": wl.T,
         "projections": [{"name": p.name, "K": p.K, "N": p.N} for p in wl.projections],
         "format": wl.fmt,
-        "l2": f"{N_WEIGHT_COPIES} rotating copies of every weight stack (inputs larger than L2), {N_BATCHES} token batches",
+        "l2": (f"{N_WEIGHT_COPIES} rotating copies of every weight stack (inputs larger than L2)" if N_WEIGHT_COPIES > 1
+               else "one copy of every weight stack: a stack alone is larger than L2") + f", {N_BATCHES} token batches",
         "parallelism": f"{world} independent replica(s)",
     }
 
@@ -537,11 +641,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     torch.cuda.synchronize()
     assert wl.g.device_errors() == 0, "device error word set during warm-up"
 
-    # timed region (inputs resident): K steps, events around the dominant kernel
-    # The dominant kernel is timed with events on every EVENT_EVERY-th step: an
-    # event between two launches ends the programmatic overlap of the pair.
-    sampled = [i for i in range(steps) if i % EVENT_EVERY == 0]
-    ev_pairs = {i: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for i in sampled}
+    # timed region (inputs resident): K whole steps, no event inside it, so
+    # consecutive launches keep their programmatic overlap
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     sampler.start()
@@ -551,7 +652,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     t_wall0 = time.time()
     start.record(stream)
     for i in range(steps):
-        wl.step(i, ev_pairs.get(i))
+        wl.step(i)
     stop.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
@@ -561,7 +662,36 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     clocks = sampler.summary(t_wall0, t_wall1)
     ms_local = start.elapsed_time(stop)
     ms = max_over_ranks(ms_local, world)
-    dom_ms = sum(a.elapsed_time(b) for a, b in ev_pairs.values()) / len(ev_pairs)
+
+    # the dominant kernel in a loop of its own: DOMINANT_REPS launches, each
+    # bracketed by events on the launching stream, weight copies rotating (the
+    # rotation is larger than L2 for the decode shapes; a prefill stack alone
+    # is), routing of batch 0
+    wl.step(0)
+    torch.cuda.synchronize()
+    dsampler = ClockSampler(local)
+    dsampler.start()
+    time.sleep(0.3)
+    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(DOMINANT_REPS)]
+    torch.cuda.synchronize()
+    d_wall0 = time.time()
+    for r, (a, b) in enumerate(dev_ev):
+        a.record(stream)
+        wl.dominant(r)
+        b.record(stream)
+    torch.cuda.synchronize()
+    d_wall1 = time.time()
+    time.sleep(0.2)
+    dsampler.stop()
+    dclocks = dsampler.summary(d_wall0, d_wall1)
+    dom = sorted(a.elapsed_time(b) for a, b in dev_ev)
+    dom_ms = statistics.median(dom)
+    dom_stats = {"reps": len(dom), "median_us": round(dom_ms * 1e3, 3),
+                 "p10_us": round(dom[int(0.1 * (len(dom) - 1))] * 1e3, 3),
+                 "p90_us": round(dom[int(0.9 * (len(dom) - 1))] * 1e3, 3),
+                 "mean_us": round(statistics.fmean(dom) * 1e3, 3), "clocks": dclocks}
+    dom_hit = wl.hit[0]
     assert wl.g.device_errors() == 0, "device error word set during the timed steps"
 
     # e2e through the public API with host buffers (pinned), copies in the timed region.
@@ -618,7 +748,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
 
     # decode: the same steps replayed from one CUDA graph of GRAPH_STEPS steps
     graph = None
-    if decode and args.graph:
+    if decode and not args.no_graph:
         gs = torch.cuda.Stream()
         gs.wait_stream(stream)
         cg = torch.cuda.CUDAGraph()
@@ -663,43 +793,20 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
                                                                   ("gemm_w4a8" if wl.w4a8 else "gemm_tc"))))
     kern_key = f"{kern_base}_{wl.wl.fmt}{'_swiglu' if wl.swiglu else ''}:{args.workload}:{wl.p1.name}"
     sha = kernel_source_sha([kern_file, "common.cuh"])
-    if decode:
-        mean_hit = sum(wl.hit[i % N_BATCHES] for i in sampled) / len(sampled)
-        alg = wl.proj_bytes(wl.p1, mean_hit)
-        achieved = alg / (dom_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": committed_traffic(kern_key, sha),
-                "kernel": f"gemv_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})",
-                "algorithmic_bytes_per_launch": int(alg), "avg_launch_us": round(dom_ms * 1e3, 3),
-                "peak_source": f"hbm_gbs of {peak_src}"}
-    else:
-        flops = 2 * wl.M * wl.p1.N * wl.p1.K
-        achieved = flops / (dom_ms / 1e3) / 1e12
-        pk = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-        pk_src = f"bf16_tflops_sustained of {peak_src} (kind::f16 MMA on decoded bf16 tiles)"
-        if wl.a4:  # fp4-rate MMA: the measured bf16 peak x the nominal dense fp4 / bf16 ratio (9 / 2.25)
-            pk = round(4 * pk, 1)
-            pk_src = f"4 x bf16_tflops_sustained of {peak_src} (kind::mxf4 runs at the fp4 rate)"
-        elif wl.w4a8:  # 8-bit-rate MMA: the measured bf16 peak x the nominal dense fp8 / bf16 ratio (4.5 / 2.25)
-            pk = round(2 * pk, 1)
-            pk_src = f"2 x bf16_tflops_sustained of {peak_src} (kind::mxf8f6f4 runs at the fp8 rate)"
-        kname = (f"dgrad_tc_kernel<{wl.wl.fmt}> (dX of {wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.dgrad else
-                 f"gemm_mx_kernel<W4A4> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.a4 else
-                 f"gemm_mx_kernel<two-term> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.split else
-                 f"gemm_mx_kernel<W4A8> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})" if wl.w4a8 else
-                 f"gemm_tc_kernel<{wl.wl.fmt}{', swiglu' if wl.swiglu else ''}> ({wl.p1.name}, K={wl.p1.K}, N={wl.p1.N})")
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk, "unit": "TFLOP/s",
-                "frac": round(achieved / pk, 4), "traffic": committed_traffic(kern_key, sha), "kernel": kname,
-                "algorithmic_flops_per_launch": int(flops), "avg_launch_us": round(dom_ms * 1e3, 3),
-                "peak_source": pk_src}
+    roof = roofline(wl, args, peaks, peak_src, dom_ms, dom_hit, dom_stats, committed_traffic(kern_key, sha))
 
-    cpu = None
+    cpu = cpu1 = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl)
         v = cb["bytes"] / cb["seconds"] / 1e9 if decode else cb["flops"] / cb["seconds"] / 1e12
         cpu = {"value": round(v, 6), "unit": unit, "cores": cb["cores"], "kind": "oracle",
                "sample": f"{cb['steps']} steps of the same workload on the first {cb['n_slice']} weight rows of "
                          f"each projection (route + fp64 grouped GEMM x2 + combine), {cb['seconds']:.1f} s"}
+        c1 = cpu_baseline(wl, budget_s=8.0, threads=1)
+        v1 = c1["bytes"] / c1["seconds"] / 1e9 if decode else c1["flops"] / c1["seconds"] / 1e12
+        cpu1 = {"value": round(v1, 6), "unit": unit, "cores": 1, "kind": "oracle",
+                "sample": f"{c1['steps']} steps on the first {c1['n_slice']} weight rows of each projection, "
+                          f"{c1['seconds']:.1f} s"}
 
     if rank == 0:
         line = {
@@ -716,7 +823,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
                               {"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if wl.w4a8 else {}),
                            **({"combine": "in the second GEMV's epilogue"} if wl.fused_combine else {}),
                            **({"step": "backward: route + dgrad of both projections"} if wl.dgrad else {})),
-            "roofline": roof, "cpu_baseline": cpu,
+            "roofline": roof, "cpu_baseline": cpu, **({"cpu_baseline_1core": cpu1} if cpu1 else {}),
             "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
             "gpu_launches": steps * wl.launches_per_step(), "clocks": clocks, "impl": "libgnf4",

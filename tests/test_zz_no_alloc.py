@@ -24,7 +24,10 @@ def _alloc(T, k, E, K):
 def test_static_route_matches_workspace_route_on_two_calls():
     from bit_grouped_moe_b200 import gnf4
 
-    cases = [(4096, 8, 384, 7168, "zipf"), (37, 4, 128, 64, "uniform")]  # two calls in a row, different shapes
+    # two calls in a row, both above 256 pairs (the multi-kernel routing that
+    # uses the shared array), with different E and chunk counts, so the second
+    # call must overwrite the first call's per-chunk histograms
+    cases = [(4096, 8, 384, 7168, "zipf"), (300, 4, 128, 64, "uniform")]
     for n, (T, k, E, K, kind) in enumerate(cases):
         rng = inputs.rng(900 + n)
         if kind == "zipf":
