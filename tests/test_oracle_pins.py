@@ -84,6 +84,33 @@ def test_byte_examples_pin_nibble_order():
         assert out[0, 0] == ex["values"][0] and out[0, 1] == ex["values"][1]
 
 
+def test_mxfp4_decode_matches_compressed_tensors():
+    """Reading C5 (element 2i in the low nibble), C6 (e2m1 code map) and C7
+    (e8m0 rule) against an independent library: compressed-tensors' FP4
+    unpacking and MX scale decompression, the decode the pages report their
+    MXFP4 reference as bit-identical to (grouped-nf4-gemm index.json,
+    problems_solved: MXFP4 reference decode vs compressed-tensors).  Every
+    byte value, scales over the bf16-exact range of the configs and beyond."""
+    helpers = pytest.importorskip("compressed_tensors.compressors.nvfp4.helpers")
+    mx = pytest.importorskip("compressed_tensors.compressors.mx_utils")
+    import torch
+
+    g = inputs.rng(5)
+    rows, K = 24, 512
+    blocks = g.integers(0, 256, size=(rows, K // 2), dtype=np.uint8)
+    blocks[0, :] = np.arange(256, dtype=np.uint8)  # every byte value once
+    scales = g.integers(100, 160, size=(rows, K // 32), dtype=np.uint8)
+    ours = oracle.dequant_mxfp4(blocks, scales)
+    vals = helpers.unpack_fp4_from_uint8(torch.from_numpy(blocks), rows, K, dtype=torch.float32)
+    sc = mx.decompress_mx_scale(torch.from_numpy(scales)).to(torch.float32).repeat_interleave(32, dim=1)
+    theirs = (vals * sc).numpy()
+    # bit patterns, except that the library multiplies a zero by a signed scale
+    # to +0 while the oracle keeps the code's sign (code 8 is -0, reading C6)
+    assert np.array_equal(ours, theirs)
+    nz = theirs != 0
+    assert np.array_equal(ours.view(np.uint32)[nz], theirs.view(np.uint32)[nz])
+
+
 def _codes_from_values(vals, table):
     """Map decoded values back to code indices by exact match (bit pattern)."""
     tb = table.view(np.uint32)
