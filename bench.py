@@ -692,6 +692,15 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
                  "p90_us": round(dom[int(0.9 * (len(dom) - 1))] * 1e3, 3),
                  "mean_us": round(statistics.fmean(dom) * 1e3, 3), "clocks": dclocks}
     dom_hit = wl.hit[0]
+    # host cost of one call (argument checks, tensor-map encodes, launch) through
+    # the Python binding: enqueue time of the same launches, no events, no sync
+    torch.cuda.synchronize()
+    h0 = time.perf_counter()
+    for r in range(DOMINANT_REPS):
+        wl.dominant(r)
+    h1 = time.perf_counter()
+    torch.cuda.synchronize()
+    dom_stats["host_enqueue_us_per_call"] = round((h1 - h0) / DOMINANT_REPS * 1e6, 2)
     assert wl.g.device_errors() == 0, "device error word set during the timed steps"
 
     # e2e through the public API with host buffers (pinned), copies in the timed region.

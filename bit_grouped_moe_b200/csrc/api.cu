@@ -199,8 +199,8 @@ gnf4_status grouped_gemm(int fmt, bool swiglu, const void* a, const uint8_t* w, 
   DeviceState* d = nullptr;
   GNF4_TRY(device_state(&d));
   CUtensorMap tm_a, tm_a_big, tm_w;
-  GNF4_TRY(encode_act_map(&tm_a, a, M, K, 32));
-  GNF4_TRY(encode_act_map(&tm_a_big, a, M, K, 128));
+  GNF4_TRY(encode_act_map(&tm_a, a, M, K, gemm_tc_small_box_rows()));
+  GNF4_TRY(encode_act_map(&tm_a_big, a, M, K, gemm_tc_big_box_rows()));
   const int wrows = gemm_tc_weight_rows_per_unit();
   if (swiglu)
     GNF4_TRY(encode_swiglu_weight_map(&tm_w, w, E, N / 2, K));
@@ -234,6 +234,8 @@ gnf4_status grouped_gemv(int fmt, bool swiglu, const void* a, const uint8_t* w, 
                                : (N + gemv_rows_per_block() - 1) / gemv_rows_per_block();
   const int grid = gemv_grid(hit * per, d->num_sms);
   cudaError_t e = launch_gemv(fmt, swiglu, p, grid, as_stream(stream));
+  if (e == cudaErrorInvalidConfiguration)
+    return fail(GNF4_ERR_CUDA, "grouped GEMV: the decode table does not fit above the kernel's shared data");
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMV launch");
   return GNF4_OK;
 }
@@ -265,6 +267,8 @@ gnf4_status grouped_gemv_combine(int fmt, const void* a, const uint8_t* w, const
   // at least one CTA, so tokens without a valid pair still get their zero row
   const int grid = M > 0 ? gemv_grid(hit * per, d->num_sms) : 1;
   cudaError_t e = launch_gemv(fmt, false, p, grid, as_stream(stream), &c);
+  if (e == cudaErrorInvalidConfiguration)
+    return fail(GNF4_ERR_CUDA, "grouped GEMV + combine: the decode table does not fit above the kernel's shared data");
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMV + combine launch");
   return GNF4_OK;
 }

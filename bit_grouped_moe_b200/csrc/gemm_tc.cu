@@ -8,30 +8,38 @@
 // Design (B200):
 //  * The MMA is computed transposed: D^T[n, r] = W_e[n, :] . A[r, :].  The
 //    decoded weight tile (128 weight rows x 64 k, bf16) is the MMA's A
-//    operand and lives in TMEM; the activation rows of the group are the B
-//    operand, loaded by TMA into 128B-swizzled shared memory.  The token
-//    dimension is the MMA's N, so a group of r rows costs an MMA with
-//    N = round_up(r, 16) instead of a padded 128-row tile.
-//  * Work unit = (expert e, 128-row weight tile j, chunk of <= 128 of the
-//    expert's rows).  Units are listed expert-major, then weight tile, then
-//    chunk, so CTAs running at the same time share weight tiles in L2.  The
-//    list is derived on the device from the group offsets (no host sync, no
-//    tile list in global memory); a persistent grid strides over it.
-//  * Decoupled rings keep enough bytes in flight: packed weights (10
-//    stages x 4 KB, its own TMA thread), activation tiles (5 stages x 16 KB,
-//    its own TMA thread) and decoded weights in TMEM (8 stages x 32 columns),
-//    plus two TMEM accumulators so the epilogue of one unit overlaps the
-//    main loop of the next.
-//  * Warp roles (22 warps): 0 and 20 = weight TMA (alternate stages), 1 =
-//    TMEM owner + MMA issuer, 2 and 21 = activation TMA (alternate stages; a
-//    group of more than 32 rows comes as one 128-row box), 3 = scale loader (raw block scales copied into a
-//    shared-memory ring with cp.async, 8 k-stages per chunk, 3 chunks ahead,
-//    so decode never waits on a global load), 4..15 = decode (three groups of
-//    four taking k-stages in turn; warp w owns TMEM lanes 32*(w%4)..+31, i.e.
-//    weight rows), 16..19 = epilogue.
+//    operand and lives in TMEM; up to 256 activation rows of the group are
+//    the B operand, loaded by TMA into 128B-swizzled shared memory.  The
+//    token dimension is the MMA's N (the group's rows rounded up to 16, at
+//    most 256), so small groups are not padded to a full tile.
+//  * Why 256 rows per unit: the thread that issues the MMAs must test a
+//    barrier once per 64-k stage, and on B200 that test costs it about
+//    200-250 cycles whenever MMAs are in flight (measured), whatever the
+//    barrier's state.  At N = 256 a stage is 4 x 128 cycles of tensor work,
+//    which hides the test; at N = 128 the test bounds the stage at about half
+//    of the tensor rate.  For the same reason the MMA thread tests a single
+//    barrier per stage: the decode warps wait for the stage's activation tile
+//    before they report the decoded weights, so their report covers both.
+//  * Work unit = (expert e, 128-row weight tile j, chunk of <= 256 of the
+//    expert's rows), derived on the device from the group offsets (no host
+//    sync, no tile list in global memory).  Experts are taken largest first
+//    (a stable rank sort of the row counts in shared memory), then weight
+//    tile, then chunk, so under a skewed routing the long experts start
+//    first and the small ones fill the tail of the persistent grid.
+//  * Rings: packed weights (8 stages x 4 KB, two TMA threads taking stages in
+//    turn), activation tiles (4 stages x 32 KB, one TMA thread; 32-row boxes
+//    for groups of at most 32 rows, else 64-row boxes), decoded weights in
+//    TMEM (8 stages x 32 columns).  The accumulator (256 columns) is single:
+//    the next unit's MMAs wait for the epilogue to drain it.
+//  * Warp roles (25 warps): 0 and 24 = weight TMA, 1 = TMEM owner + MMA
+//    issuer, 2 = activation TMA, 3 = scale loader (raw block scales copied
+//    into a shared-memory ring with cp.async, 8 k-stages per chunk, 3 chunks
+//    ahead), 4..19 = decode (four groups of four; group g takes the stages
+//    it = g mod 4, so every activation slot and every TMEM slot is waited on
+//    by one group only), 20..23 = epilogue.
 //  * Decode: a thread owns one weight row; per 64-k stage it reads its 32
 //    packed bytes from shared memory, and for every byte builds the address
-//    of a lane-private pair-table entry with one PRMT, loads the two bf16
+//    of a lane-private pair-table entry (PRMT + shift), loads the two bf16
 //    codes, multiplies them by the block scale in bf16x2 and finally stores
 //    32 columns to TMEM with tcgen05.st.
 #include <cuda.h>
@@ -43,43 +51,44 @@
 namespace gnf4 {
 namespace {
 
-constexpr int kBT = 128;   // activation rows (tokens) per unit = max MMA N
+constexpr int kBT = 256;   // activation rows (tokens) per unit = max MMA N
 constexpr int kBW = 128;   // weight rows per unit = MMA M
 constexpr int kBK = 64;    // k per stage
-constexpr int kWStages = 10;
-constexpr int kAStages = 5;
+constexpr int kWStages = 8;
+constexpr int kAStages = 4;
 constexpr int kTStages = 8;
 constexpr int kSChunk = 8;       // k-stages per scale chunk
 constexpr int kSStages = 3;      // scale chunks in flight
 constexpr int kSRowWords = 9;    // raw scale words per row per chunk (NF4 8, MXFP4 5), padded
-constexpr int kDecGroups = 3;
+constexpr int kDecGroups = 4;
 constexpr int kDecWarp0 = 4;
-constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;  // 16
-constexpr int kWProd2 = kEpiWarp0 + 4;                 // 20: second weight producer
-constexpr int kAProd2 = kWProd2 + 1;                   // 21: second activation producer
-constexpr int kThreads = (kAProd2 + 1) * 32;           // 704
-constexpr int kBigBox = 128;                           // activation rows per TMA box for large groups
-constexpr int kAccCols = 2 * kBT;                      // two fp32 accumulators
-constexpr int kACol0 = kAccCols;                       // decoded-weight ring
+constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;  // 20
+constexpr int kWProd2 = kEpiWarp0 + 4;                 // 24: second weight producer
+constexpr int kThreads = (kWProd2 + 1) * 32;           // 800
+constexpr int kSmallBox = 32;                          // activation rows per box, groups of <= 32 rows
+constexpr int kBigBox = 64;                            // activation rows per box otherwise
+constexpr int kACol0 = kBT;                            // decoded-weight ring after the accumulator
 constexpr int kTmemCols = 512;
-constexpr int kActStageBytes = kBT * kBK * 2;          // 16 KB
+constexpr int kActStageBytes = kBT * kBK * 2;          // 32 KB
 constexpr int kWStageBytes = kBW * kBK / 2;            // 4 KB
-constexpr int kActBox = 32;                            // activation rows per TMA box
 static_assert(kACol0 + kTStages * (kBK / 2) <= kTmemCols, "TMEM budget");
+static_assert(kAStages % kDecGroups == 0 && kTStages % kDecGroups == 0,
+              "each activation / TMEM slot must belong to one decode group");
 
 struct Smem {
   uint8_t act[kAStages][kActStageBytes];  // 1024-aligned (offset 0)
-  uint32_t lut[kLut256Words];             // 64 KB
+  uint32_t lut[kLutWords];                // 32 KB pair table, entry b of lane l at word 32 b + l
   uint8_t wq[kWStages][kWStageBytes];
   uint32_t sring[kSStages][kBW][kSRowWords];  // raw block scales of kSChunk k-stages per row
   int off[kMaxExperts + 1];
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
+  int order[kMaxExperts];  // experts by descending row count (stable)
   uint64_t wfull[kWStages], wempty[kWStages];
   uint64_t afull[kAStages], aempty[kAStages];
   uint64_t tfull[kTStages], tempty[kTStages];
   uint64_t sfull[kSStages], sempty[kSStages];
-  uint64_t accf[2], acce[2];
+  uint64_t accf, acce;
   uint64_t mdone;  // abort path only: every issued MMA has retired
   uint32_t tmem_base;
   int abort;
@@ -89,10 +98,6 @@ static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
 struct Unit {
   int e, j, row0, rows;
 };
-
-// Partial accumulators per unit: groups of at most 32 (64) rows split the
-// 128 accumulator columns into 4 (2) independent sums of 32 (64) columns.
-__device__ __forceinline__ int acc_split(int rows) { return rows <= 32 ? 4 : (rows <= 64 ? 2 : 1); }
 
 // Weight row (within the expert) held by TMEM lane nl of weight tile j.
 // SwiGLU tiles take 64 gate rows and the matching 64 up rows of a gate_up
@@ -114,10 +119,13 @@ __device__ __forceinline__ int stage_row(int nl) {
   return (x < 16 ? 0 : 64) + 16 * q + (x & 15);
 }
 
+// Unit u: position p of the largest-first expert order, then weight tile,
+// then chunk of kBT rows.
 __device__ __forceinline__ Unit unit_of(const Smem& s, int E, int u) {
   Unit x;
-  x.e = find_group(s.upre, E, u);
-  const int local = u - s.upre[x.e];
+  const int p = find_group(s.upre, E, u);
+  x.e = s.order[p];
+  const int local = u - s.upre[p];
   const int rows_e = s.off[x.e + 1] - s.off[x.e];
   const int nch = (rows_e + kBT - 1) / kBT;
   x.j = local / nch;
@@ -125,6 +133,16 @@ __device__ __forceinline__ Unit unit_of(const Smem& s, int E, int u) {
   x.row0 = s.off[x.e] + c * kBT;
   x.rows = min(kBT, s.off[x.e + 1] - x.row0);
   return x;
+}
+
+// Two bf16 codes of byte j of `word` (pair table, 128-byte stride per entry).
+// lane8 = 8 * lane: the PRMT puts the byte in bits 8..15, 8 * lane in bits
+// 0..7 and zeros above, and the shift turns that into 128 * byte + 4 * lane.
+__device__ __forceinline__ uint32_t lut_get(uint32_t lut, uint32_t word, uint32_t lane8, uint32_t j) {
+  uint32_t v;
+  const uint32_t off = prmt_b32(word, lane8, 0x5504u | (j << 4)) >> 1;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(lut + off));
+  return v;
 }
 
 template <int FMT, bool SWI>
@@ -140,15 +158,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_launch_dependents();
   griddep_wait();
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, err)) return;
+  // largest-first expert order: rank = experts with more rows, ties by index
+  for (int e = tid; e < p.E; e += kThreads) {
+    const int re = s.off[e + 1] - s.off[e];
+    int rank = 0;
+    for (int f = 0; f < p.E; ++f) {
+      const int rf = s.off[f + 1] - s.off[f];
+      rank += (rf > re || (rf == re && f < e)) ? 1 : 0;
+    }
+    s.scratch[rank] = e;
+  }
+  __syncthreads();
+  for (int i = tid; i < p.E; i += kThreads) s.order[i] = s.scratch[i];
+  __syncthreads();
   const int I = p.N / 2;  // SwiGLU: output columns
   const int nwt = SWI ? I / (kBW / 2) : (p.N + kBW - 1) / kBW;
-  block_exclusive_scan(p.E, s.upre, s.scratch,
-                       [&](int e) { return ((s.off[e + 1] - s.off[e] + kBT - 1) / kBT) * nwt; });
+  block_exclusive_scan(p.E, s.upre, s.scratch, [&](int q) {
+    const int e = s.order[q];
+    return ((s.off[e + 1] - s.off[e] + kBT - 1) / kBT) * nwt;
+  });
   const int U = s.upre[p.E];
   if ((int)blockIdx.x >= U) return;  // uniform over the block
   const int nk = (p.K + kBK - 1) / kBK;
 
-  build_pair_lut256<FMT>(s.lut, tid, kThreads);
+  build_pair_lut<FMT>(s.lut, tid, kThreads);
   if (tid == 0) {
     for (int i = 0; i < kWStages; ++i) {
       mbar_init(&s.wfull[i], 1);
@@ -166,10 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.sfull[i], 32);
       mbar_init(&s.sempty[i], 4 * kDecGroups);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.accf[i], 1);
-      mbar_init(&s.acce[i], 4);
-    }
+    mbar_init(&s.accf, 1);
+    mbar_init(&s.acce, 4);
     mbar_init(&s.mdone, 1);
     s.abort = 0;
     fence_mbar_init();
@@ -215,33 +246,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = max(0, it - kWStages); i < it; ++i)
           if ((i & 1) == pi) mbar_drain(&s.wfull[i % kWStages], (i / kWStages) & 1);
     }
-  } else if (warp == 2 || warp == kAProd2) {
+  } else if (warp == 2) {
     // ------------------------------------------------------------ activation TMA
-    // Two producer threads alternate stages; a group of more than 32 rows is
-    // loaded as one 128-row box, a smaller one as one 32-row box.
-    const int pi = warp == 2 ? 0 : 1;
+    // A group of at most 32 rows comes as one 32-row box, a larger one as
+    // ceil(rows / 64) boxes of 64 rows (rows past M read as zero).
     if (lane == 0) {
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const Unit x = unit_of(s, p.E, u);
-        const bool big = x.rows > kActBox;
+        const bool big = x.rows > kSmallBox;
+        const int nb = big ? (x.rows + kBigBox - 1) / kBigBox : 1;
         for (int kt = 0; kt < nk; ++kt, ++it) {
-          if ((it & 1) != pi) continue;
           const int st = it % kAStages, use = it / kAStages;
           if (it >= kAStages && !(ok = mbar_wait(&s.aempty[st], (use - 1) & 1, err, abort))) break;
           if (big) {
-            mbar_arrive_expect_tx(&s.afull[st], kBigBox * 128);
-            tma_load_2d(s.act[st], &tm_a_big, &s.afull[st], kt * kBK, x.row0);
+            mbar_arrive_expect_tx(&s.afull[st], nb * kBigBox * 128);
+            for (int b = 0; b < nb; ++b)
+              tma_load_2d(s.act[st] + b * kBigBox * 128, &tm_a_big, &s.afull[st], kt * kBK, x.row0 + b * kBigBox);
           } else {
-            mbar_arrive_expect_tx(&s.afull[st], kActBox * 128);
+            mbar_arrive_expect_tx(&s.afull[st], kSmallBox * 128);
             tma_load_2d(s.act[st], &tm_a, &s.afull[st], kt * kBK, x.row0);
           }
         }
       }
       if (!ok)
-        for (int i = max(0, it - kAStages); i < it; ++i)
-          if ((i & 1) == pi) mbar_drain(&s.afull[i % kAStages], (i / kAStages) & 1);
+        for (int i = max(0, it - kAStages); i < it; ++i) mbar_drain(&s.afull[i % kAStages], (i / kAStages) & 1);
     }
   } else if (warp == 3) {
     // ------------------------------------------------------------ scale loader
@@ -270,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q = 0; q < cnt; ++q) cp_async_4(&s.sring[slot][r][q], src + q);
           } else {
             const uint8_t* base = reinterpret_cast<const uint8_t*>(p.scales);
-            const size_t b0 = rowsc + 2 * (size_t)kt0;               // first scale byte of the chunk
+            const size_t b0 = rowsc + 2 * (size_t)kt0;                     // first scale byte of the chunk
             const size_t b1 = min(rowsc + (size_t)nsc, b0 + 2 * kSChunk);  // one past the last
             const size_t w0 = b0 & ~(size_t)3;
             for (size_t wq = w0, q = 0; wq < b1; wq += 4, ++q) cp_async_4(&s.sring[slot][r][q], base + wq);
@@ -286,36 +316,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
         const Unit x = unit_of(s, p.E, u);
-        const int ab = uc & 1;
-        if (uc >= 2 && !(ok = mbar_wait(&s.acce[ab], ((uc >> 1) - 1) & 1, err, abort))) break;
+        if (uc >= 1 && !(ok = mbar_wait(&s.acce, (uc - 1) & 1, err, abort))) break;
         tc_fence_after();
         const uint32_t idesc = idesc_bf16_m128((uint32_t)((x.rows + 15) & ~15));
-        const uint32_t d_tmem = tmem + (uint32_t)(ab * kBT);
-        // Small groups: the k-steps of a stage go to independent partial
-        // accumulators, so consecutive MMAs do not wait for each other.
-        const int nsplit = acc_split(x.rows);
-        const uint32_t sub_w = (uint32_t)(kBT / nsplit);
         for (int kt = 0; kt < nk; ++kt, ++it) {
           const int sa = it % kAStages, sT = it % kTStages;
-          // poll both barriers before looking at either result
-          const bool ra = mbar_try_wait(&s.afull[sa], (it / kAStages) & 1);
-          const bool rt = mbar_try_wait(&s.tfull[sT], (it / kTStages) & 1);
-          if (!(ra && rt)) {
-            if (!(ok = mbar_wait(&s.afull[sa], (it / kAStages) & 1, err, abort))) break;
-            if (!(ok = mbar_wait(&s.tfull[sT], (it / kTStages) & 1, err, abort))) break;
-          }
+          // one barrier per stage: the decode warps report a stage only after
+          // its activation tile has landed
+          if (!(ok = mbar_wait(&s.tfull[sT], (it / kTStages) & 1, err, abort))) break;
           tc_fence_after();
           const uint32_t a_col = tmem + (uint32_t)(kACol0 + sT * (kBK / 2));
           const uint32_t b_addr = smem_u32(s.act[sa]);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            tc_mma_ts(d_tmem + (uint32_t)(kk % nsplit) * sub_w, a_col + kk * 8, sdesc_k_sw128(b_addr + kk * 32), idesc,
-                      kt != 0 || kk >= nsplit);
+            tc_mma_ts(tmem, a_col + kk * 8, sdesc_k_sw128(b_addr + kk * 32), idesc, (kt | kk) != 0);
           tc_commit(&s.aempty[sa]);
           tc_commit(&s.tempty[sT]);
         }
         if (!ok) break;
-        tc_commit(&s.accf[ab]);
+        tc_commit(&s.accf);
       }
       if (!ok) {
         // abort: let every MMA already issued retire before TMEM is released
@@ -328,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grp = (warp - kDecWarp0) >> 2, q = warp & 3;
     const int nl = q * 32 + lane;
     const uint32_t lut = smem_u32(s.lut);
-    const uint32_t lane4 = (uint32_t)lane * 4u;
+    const uint32_t lane8 = (uint32_t)lane * 8u;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     int it = 0, ci = 0;
     bool ok = true;
@@ -338,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q8 = kt % kSChunk, slot = ci % kSStages;
         if (q8 == 0 && !(ok = mbar_wait(&s.sfull[slot], (ci / kSStages) & 1, err, abort))) break;
         if (it % kDecGroups == grp) {
-          const int sw = it % kWStages, sT = it % kTStages;
+          const int sw = it % kWStages, sT = it % kTStages, sa = it % kAStages;
           if (!(ok = mbar_wait(&s.wfull[sw], (it / kWStages) & 1, err, abort))) break;
           if (it >= kTStages && !(ok = mbar_wait(&s.tempty[sT], ((it / kTStages) - 1) & 1, err, abort))) break;
           uint32_t sc0, sc1;
@@ -367,17 +386,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive(&s.wempty[sw]);  // packed bytes are in registers now
           uint32_t v[32];
           {
-            uint32_t h0[16], h1[16];
-            decode16_lut256(lut, lane4, c0, sc0, h0);
-            decode16_lut256(lut, lane4, c1, sc1, h1);
+            const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              v[i] = h0[i];
-              v[16 + i] = h1[i];
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t sc = i < 4 ? sc0 : sc1;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) v[4 * i + j] = bf16x2_mul(lut_get(lut, w[i], lane8, (uint32_t)j), sc);
             }
           }
           tmem_st_32x32b_x32(t_lane + (uint32_t)(kACol0 + sT * (kBK / 2)), v);
           tmem_wait_st();
+          // the MMA thread tests only this barrier: report the stage once its
+          // activation tile has landed as well
+          if (!(ok = mbar_wait(&s.afull[sa], (it / kAStages) & 1, err, abort))) break;
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s.tfull[sT]);
@@ -389,30 +410,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp >= kEpiWarp0) {
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
     int uc = 0;
     for (int u = blockIdx.x; u < U; u += gridDim.x, ++uc) {
       const Unit x = unit_of(s, p.E, u);
-      const int ab = uc & 1;
-      if (!mbar_wait(&s.accf[ab], (uc >> 1) & 1, err, abort)) break;
+      if (!mbar_wait(&s.accf, uc & 1, err, abort)) break;
       tc_fence_after();
       const int n = x.j * kBW + q * 32 + lane;
       __nv_bfloat16* ycol = p.y + (size_t)x.row0 * p.N + n;
-      const int nsplit = acc_split(x.rows);
       for (int c = 0; c * 32 < x.rows; ++c) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBT + c * 32), v);
+        tmem_ld_32x32b_x32(t_lane + (uint32_t)(c * 32), v);
         tmem_wait_ld();
-        for (int j = 1; j < nsplit; ++j) {  // partial accumulators, summed in a fixed order
-          uint32_t w2[32];
-          tmem_ld_32x32b_x32(t_lane + (uint32_t)(ab * kBT + j * (kBT / nsplit) + c * 32), w2);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w2[i]));
-        }
         const int lim = min(32, x.rows - c * 32);
         if (SWI) {
           // lane x < 16 holds gate(col), lane x + 16 up(col).  Per pair of rows
@@ -441,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.acce[ab]);
+      if (lane == 0) mbar_arrive(&s.acce);
     }
   }
 
@@ -480,5 +492,7 @@ cudaError_t launch_gemm_tc(int fmt, bool swiglu, const CUtensorMap& tm_a, const 
 
 int gemm_tc_rows_per_unit() { return kBT; }
 int gemm_tc_weight_rows_per_unit() { return kBW; }
+int gemm_tc_small_box_rows() { return kSmallBox; }
+int gemm_tc_big_box_rows() { return kBigBox; }
 
 }  // namespace gnf4

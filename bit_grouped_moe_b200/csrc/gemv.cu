@@ -12,11 +12,10 @@
 // computes the partial sums of all 64 rows (four m16 tiles) for the group's
 // <= 8 rows (the MMA's 8 columns); a fixed-order shared-memory reduction over
 // the 8 warps finishes the unit.  Per item a lane holds 16 bytes (32 codes)
-// of each of its 8 weight rows, decodes every byte with one PRMT, which
+// of each of its 8 weight rows and decodes every byte with one PRMT, which
 // builds the shared-memory address of a lane-private pair-table entry, and
-// one shared load, multiplies the bf16 pair by the row's block scale, and
-// feeds the pairs to m16n8k16 warp MMAs.  The MMA does the k reduction that
-// a CUDA-core GEMV would do with shuffles.
+// one shared load; the bf16 pairs feed m16n8k16 warp MMAs.  The MMA does the
+// k reduction that a CUDA-core GEMV would do with shuffles.
 //
 // Fused combine (CMB): after a half has stored its unit's rows, each row
 // counts its (token, 64-column block) in; the half that completes a token's
@@ -32,17 +31,23 @@
 // decoded), so every warp always has about one item (4 KB) in flight without
 // a second register set.
 //
-// The pair table sits at shared-window address 0x10000 (one copy per SM, 64
-// KB): the PRMT that extracts a byte also inserts the table's base, so a
-// lookup is exactly one PRMT and one shared load.
+// The pair table (one copy per SM, 64 KB) starts at the first 64 KB boundary
+// of the shared window above the kernel's other shared data (0x10000 unless
+// static shared memory grows past the budget checked on the host): the PRMT
+// that extracts a byte also inserts the table's base, so a lookup is exactly
+// one PRMT and one shared load.
 //
-// Lane (g, t) = (lane / 4, lane % 4) owns rows g and g+8 of every tile and,
-// in every item, the 32 consecutive k in [32t, 32t+32) (one NF4 half-block,
-// one MXFP4 block).  The MMA's k index is a permutation of these physical k;
-// the activation fragment uses the same permutation.
-//   * MXFP4: e2m1 x 2^(e-127) is exact in bf16.
-//   * NF4: the code is rounded to bf16, then multiplied by bf16(absmax) and
-//     rounded again (relative error <= ~3 * 2^-9 per weight); sums are fp32.
+// Lane (g, t) = (lane / 4, lane % 4) owns rows g and g+8 of every tile.  The
+// MMA's k index is a permutation of the physical k, and the activation
+// fragment uses the same permutation:
+//   * MXFP4: the lane takes the 32 consecutive k [32t, 32t+32) of an item (one
+//     block); each decoded pair is multiplied by the row's block scale in
+//     bf16, which is exact (e2m1 x 2^(e-127) is a bf16 value).
+//   * NF4: the lane takes k [16t, 16t+16) of each 64-k block, so the four MMA
+//     steps of a block stay inside it.  The MMAs multiply the bf16-rounded
+//     codes into a fresh fp32 partial sum per block, which is multiplied by
+//     the rows' fp32 absmax and added to the accumulator: one bf16 rounding
+//     per weight (the code's, <= 2^-9 relative), no bf16 product.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -57,10 +62,9 @@ constexpr int kSplit = 8;                 // warps per half = K-splits of a unit
 constexpr int kRows = 64;                 // weight rows per unit (4 m16 tiles)
 constexpr int kMaxTokens = 8;             // rows of a group = MMA columns
 constexpr int kDK = 128;                  // k per item
-constexpr uint32_t kLutWindow = 0x10000u;  // shared-window address of the pair table
-constexpr int kSmemBytes = 0x20000;        // dynamic shared memory per CTA
+constexpr int kSmemBytes = 0x20000;  // dynamic shared memory per CTA
 
-// Everything but the pair table; lives below kLutWindow.
+// Everything but the pair table; lives below it.
 struct GemvLow {
   float red[2][kSplit][4][32][4];  // 32 KB: partial sums per half and K-split
   int done[2][kMaxTokens];         // fused combine: tokens a half's unit completed (-1: none)
@@ -69,15 +73,8 @@ struct GemvLow {
   int scratch[kMaxExperts];
 };
 
-// f32 -> bf16 (round to nearest even, NaN kept quiet), duplicated in both halves.
-__device__ __forceinline__ uint32_t cvt_bf16x2_dup(float f) {
-  uint32_t d;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(d) : "f"(f));
-  return d;
-}
-
 // One pair-table lookup: byte j of `word` selects the entry; `lanesel` holds
-// 4*lane in byte 0 and the table base's byte 2 (0x01) in byte 2.
+// 4*lane in byte 0 and byte 2 of the table's 64 KB-aligned base in byte 2.
 __device__ __forceinline__ uint32_t lut_lookup(uint32_t word, uint32_t lanesel, uint32_t j) {
   uint32_t v;
   asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(prmt_b32(word, lanesel, 0x7604u | (j << 4))));
@@ -92,7 +89,7 @@ __device__ __forceinline__ void half_barrier(int h) {
 struct UnitView {
   const uint8_t* w;            // weight row n0 (q = 0), byte 0
   const uint8_t* sc;           // first scale of row n0 (bytes)
-  const __nv_bfloat16* x;      // activation row of token g (row 0 if g >= rows), k = 32t
+  const __nv_bfloat16* x;      // activation row of token g (row 0 if g >= rows), at the lane's first k
   int qv;                      // rows n0 + 8q < N  <=>  q < qv
   bool tv;                     // token g exists
 };
@@ -116,7 +113,8 @@ __device__ __forceinline__ UnitView unit_view(const GemvLow& s, const GroupedArg
   v.w = p.w + row * (size_t)(p.K / 2);
   v.sc = reinterpret_cast<const uint8_t*>(p.scales) + row * (size_t)nsc * (FMT == 0 ? 4u : 1u);
   v.tv = g < rows;
-  v.x = p.a + (size_t)(r0 + (v.tv ? g : 0)) * p.K + 32 * t;
+  // NF4: lane t takes k [16t, 16t+16) of every 64-k block; MXFP4: k [32t, 32t+32) of every item
+  v.x = p.a + (size_t)(r0 + (v.tv ? g : 0)) * p.K + (FMT == 0 ? 16 : 32) * t;
   v.qv = (p.N - n0 + 7) / 8;
   return v;
 }
@@ -124,34 +122,61 @@ __device__ __forceinline__ UnitView unit_view(const GemvLow& s, const GroupedArg
 // Loads of one item for tile i (rows q = 2i, 2i+1): packed weights and raw scales.
 // `rb` = packed bytes per weight row, `nsr` = scales per weight row, `gap` =
 // I - 32 (kModeSwiglu: rows from the unit's last gate row block to its up rows).
+//   NF4 (block-aligned): wq[q] = the lane's 8 bytes of 64-k blocks 2d (x, y) and
+//   2d+1 (z, w); sr[2q + b] = the raw fp32 absmax of block 2d + b (0 past K).
+//   MXFP4: wq[q] = the lane's 16 bytes of the item; sr[q] = the e8m0 byte of its block.
 template <int FMT, int MODE>
 __device__ __forceinline__ void load_tile(const UnitView& v, int d, int t, int K, size_t rb, size_t nsr, int gap,
-                                          int i, uint4 (&wq)[8], uint32_t (&sr)[8]) {
-  const bool inK = d * kDK + 32 * t < K;
-  const size_t kb = inK ? (size_t)(d * (kDK / 2) + 16 * t) : 0;  // outside K: any valid address
-  const size_t si = inK ? (size_t)(FMT == 0 ? 2 * d + (t >> 1) : 4 * d + t) : 0;
+                                          int i, uint4 (&wq)[8], uint32_t (&sr)[16]) {
 #pragma unroll
   for (int hq = 0; hq < 2; ++hq) {
     const int q = 2 * i + hq;
     const int roff = MODE == kModeClamp ? 8 * min(q, v.qv - 1) : (MODE == kModeSwiglu && q >= 4 ? 8 * q + gap : 8 * q);
-    wq[q] = ldg_nc_u128(v.w + (size_t)roff * rb + kb);
-    if (FMT == 0)
-      sr[q] = __ldg(reinterpret_cast<const unsigned int*>(v.sc + ((size_t)roff * nsr + si) * 4u));
-    else
-      sr[q] = __ldg(v.sc + (size_t)roff * nsr + si);
+    const uint8_t* wrow = v.w + (size_t)roff * rb;
+    if (FMT == 0) {
+      const int nb = K / 64;
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const int blk = 2 * d + b;
+        const bool in = blk < nb;
+        const uint2 w8 = ldg_nc_u64(wrow + (in ? (size_t)(32 * blk + 8 * t) : 0));  // outside K: any valid address
+        if (b == 0) {
+          wq[q].x = w8.x;
+          wq[q].y = w8.y;
+        } else {
+          wq[q].z = w8.x;
+          wq[q].w = w8.y;
+        }
+        sr[2 * q + b] = in ? __ldg(reinterpret_cast<const unsigned int*>(v.sc) + (size_t)roff * nsr + blk) : 0u;
+      }
+    } else {
+      const bool inK = d * kDK + 32 * t < K;
+      const size_t kb = inK ? (size_t)(d * (kDK / 2) + 16 * t) : 0;  // outside K: any valid address
+      wq[q] = ldg_nc_u128(wrow + kb);
+      sr[q] = __ldg(v.sc + (size_t)roff * nsr + (inK ? (size_t)(4 * d + t) : 0));
+    }
   }
 }
 
+// Activations of token g for one item.  NF4: xa[2b], xa[2b+1] = k [16t, 16t+16)
+// of block 2d + b; MXFP4: xa[c] = k [32t + 8c, 32t + 8c + 8) of the item.
+template <int FMT>
 __device__ __forceinline__ void load_acts(const UnitView& v, int d, int t, int K, uint4 (&xa)[4]) {
-  const bool ok = v.tv && (d * kDK + 32 * t < K);
+  if (FMT == 0) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) xa[c] = ok ? ldg_u128(v.x + d * kDK + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+    for (int b = 0; b < 2; ++b) {
+      const bool ok = v.tv && ((2 * d + b) * 64 < K);
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        xa[2 * b + c] = ok ? ldg_u128(v.x + d * kDK + 64 * b + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  } else {
+    const bool ok = v.tv && (d * kDK + 32 * t < K);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) xa[c] = ok ? ldg_u128(v.x + d * kDK + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+  }
 }
 
-template <int FMT>
-__device__ __forceinline__ uint32_t scale_pair(uint32_t raw) {
-  return FMT == 0 ? cvt_bf16x2_dup(__uint_as_float(raw)) : e8m0_to_bf16x2(raw);
-}
 
 // Sum over the valid pairs of token t (sorted row inside [0, nvalid)).
 __device__ __forceinline__ int valid_pairs(const CombineArgs& c, int t, int nvalid) {
@@ -171,18 +196,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p, Combin
   const int g = lane >> 2, t = lane & 3;
   const int h = warp / kSplit, ks = warp % kSplit;
 
-  // The table must occupy [kLutWindow, kLutWindow + 64 KB) of this CTA's
-  // shared window, with GemvLow below it.
+  // The table takes the first 64 KB boundary above GemvLow; the host refuses
+  // to launch when the window cannot hold it (gemv_static_smem_ok), so this
+  // check only guards against a window placed differently than the host saw.
   const uint32_t base = smem_u32(smem_raw);
-  if (base + (uint32_t)sizeof(GemvLow) > kLutWindow ||
-      base + (uint32_t)kSmemBytes < kLutWindow + (uint32_t)kLut256Bytes) {
+  const uint32_t lut_at = (base + (uint32_t)sizeof(GemvLow) + 0xFFFFu) & ~0xFFFFu;
+  if (lut_at + (uint32_t)kLut256Bytes > base + (uint32_t)kSmemBytes) {
     if (tid == 0) atomicOr(p.err, GNF4_DEVERR_INTERNAL);
     return;
   }
   griddep_launch_dependents();
   // the pair table depends on nothing earlier in the stream: build it while
   // the previous kernel finishes (made visible by the barriers below)
-  build_pair_lut256<FMT>(reinterpret_cast<uint32_t*>(smem_raw + (kLutWindow - base)), tid, kThreads);
+  build_pair_lut256<FMT>(reinterpret_cast<uint32_t*>(smem_raw + (lut_at - base)), tid, kThreads);
   griddep_wait();
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, p.err)) return;
   const int nblk = MODE == kModeSwiglu ? (p.N / 2) / (kRows / 2) : (p.N + kRows - 1) / kRows;
@@ -207,19 +233,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p, Combin
 
   // first item of this warp's stream
   uint4 wq[8], xa[4];
-  uint32_t sr[8];
+  uint32_t sr[16];
   UnitView cur{};
   if (u < U) {
     cur = unit_view<FMT, MODE>(s, p, u, g, t);
     if (d_lo < d_hi) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) load_tile<FMT, MODE>(cur, d_lo, t, K, rb, nsr, gap, i, wq, sr);
-      load_acts(cur, d_lo, t, K, xa);
+      load_acts<FMT>(cur, d_lo, t, K, xa);
     }
   }
   __syncthreads();
 
-  const uint32_t lanesel = (uint32_t)lane * 4u | (kLutWindow & 0x00FF0000u);
+  const uint32_t lanesel = (uint32_t)lane * 4u | (lut_at & 0x00FF0000u);
 
   for (; u < U; u += ustride) {  // uniform over the half
     float acc[4][4];
@@ -235,24 +261,48 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p, Combin
       const bool has_next = !last || u + ustride < U;
       if (last && has_next) cur = unit_view<FMT, MODE>(s, p, u + ustride, g, t);
       uint4 xn[4];
-      if (has_next) load_acts(cur, dn, t, K, xn);
+      if (has_next) load_acts<FMT>(cur, dn, t, K, xn);
 
       const uint32_t xp[16] = {xa[0].x, xa[0].y, xa[0].z, xa[0].w, xa[1].x, xa[1].y, xa[1].z, xa[1].w,
                                xa[2].x, xa[2].y, xa[2].z, xa[2].w, xa[3].x, xa[3].y, xa[3].z, xa[3].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t s0 = scale_pair<FMT>(sr[2 * i]), s1 = scale_pair<FMT>(sr[2 * i + 1]);
         const uint32_t w0[4] = {wq[2 * i].x, wq[2 * i].y, wq[2 * i].z, wq[2 * i].w};
         const uint32_t w1[4] = {wq[2 * i + 1].x, wq[2 * i + 1].y, wq[2 * i + 1].z, wq[2 * i + 1].w};
-        // MMA step j takes bytes 2j, 2j+1 of both rows (word j/2, bytes 2(j%2) and 2(j%2)+1)
+        if (FMT == 0) {
+          // Block-aligned: the four MMA steps of 64-k block b take the quad's
+          // k [16t + 4j, 16t + 4j + 4) (bytes 2j, 2j+1 of the lane's 8), so a
+          // step never leaves its block; the fp32 partial sum of the block is
+          // then scaled once by the rows' absmax.
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t b0 = 2u * (uint32_t)(j & 1);
-          const uint32_t a0 = bf16x2_mul(lut_lookup(w0[j >> 1], lanesel, b0), s0);
-          const uint32_t a1 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0), s1);
-          const uint32_t a2 = bf16x2_mul(lut_lookup(w0[j >> 1], lanesel, b0 + 1u), s0);
-          const uint32_t a3 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0 + 1u), s1);
-          mma_bf16_16816(acc[i], a0, a1, a2, a3, xp[2 * j], xp[2 * j + 1]);
+          for (int b = 0; b < 2; ++b) {
+            float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t bs = 2u * (uint32_t)(j & 1);
+              const uint32_t ww0 = w0[2 * b + (j >> 1)], ww1 = w1[2 * b + (j >> 1)];
+              mma_bf16_16816(part, lut_lookup(ww0, lanesel, bs), lut_lookup(ww1, lanesel, bs),
+                             lut_lookup(ww0, lanesel, bs + 1u), lut_lookup(ww1, lanesel, bs + 1u), xp[8 * b + 2 * j],
+                             xp[8 * b + 2 * j + 1]);
+            }
+            const float s0 = __uint_as_float(sr[4 * i + b]), s1 = __uint_as_float(sr[4 * i + 2 + b]);
+            acc[i][0] = fmaf(s0, part[0], acc[i][0]);
+            acc[i][1] = fmaf(s0, part[1], acc[i][1]);
+            acc[i][2] = fmaf(s1, part[2], acc[i][2]);
+            acc[i][3] = fmaf(s1, part[3], acc[i][3]);
+          }
+        } else {
+          const uint32_t s0 = e8m0_to_bf16x2(sr[2 * i]), s1 = e8m0_to_bf16x2(sr[2 * i + 1]);
+          // MMA step j takes bytes 2j, 2j+1 of both rows (word j/2, bytes 2(j%2) and 2(j%2)+1)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t b0 = 2u * (uint32_t)(j & 1);
+            const uint32_t a0 = bf16x2_mul(lut_lookup(w0[j >> 1], lanesel, b0), s0);
+            const uint32_t a1 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0), s1);
+            const uint32_t a2 = bf16x2_mul(lut_lookup(w0[j >> 1], lanesel, b0 + 1u), s0);
+            const uint32_t a3 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0 + 1u), s1);
+            mma_bf16_16816(acc[i], a0, a1, a2, a3, xp[2 * j], xp[2 * j + 1]);
+          }
         }
         if (has_next) load_tile<FMT, MODE>(cur, dn, t, K, rb, nsr, gap, i, wq, sr);
       }
@@ -361,10 +411,38 @@ int gemv_grid(long long units, int num_sms) {
   return (int)(ctas < num_sms ? ctas : num_sms);
 }
 
+// Host side of the pair-table placement: the dynamic window starts after the
+// device's reserved and the kernel's static shared memory (at most 1 KB of
+// alignment more), and the table needs GemvLow below the 64 KB boundary.
+// Checked once per device; a launch the table cannot fit is refused with
+// cudaErrorInvalidConfiguration before anything is enqueued.
+template <typename Kernel>
+static cudaError_t table_fits_once(Kernel kernel, std::atomic<int> (&state)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool tracked = dev >= 0 && dev < 64;
+  if (tracked) {
+    const int st = state[dev].load(std::memory_order_acquire);
+    if (st != 0) return st > 0 ? cudaSuccess : cudaErrorInvalidConfiguration;
+  }
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return e;
+  int reserved = 0;
+  if ((e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
+  const size_t start = ((size_t)reserved + fa.sharedSizeBytes + 1023) & ~(size_t)1023;
+  const bool fits = start + sizeof(GemvLow) <= 0x10000u;
+  if (tracked) state[dev].store(fits ? 1 : -1, std::memory_order_release);
+  return fits ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
 template <int FMT, int MODE, bool CMB>
 static cudaError_t launch_gemv_t(const GroupedArgs& p, const CombineArgs& c, int grid, cudaStream_t stream) {
   static std::atomic<bool> configured[64];
-  const cudaError_t e = set_smem_limit_once(gemv_kernel<FMT, MODE, CMB>, kSmemBytes, configured);
+  static std::atomic<int> placed[64];
+  cudaError_t e = table_fits_once(gemv_kernel<FMT, MODE, CMB>, placed);
+  if (e != cudaSuccess) return e;
+  e = set_smem_limit_once(gemv_kernel<FMT, MODE, CMB>, kSmemBytes, configured);
   if (e != cudaSuccess) return e;
   return launch_pdl(gemv_kernel<FMT, MODE, CMB>, dim3(grid), dim3(kThreads), (size_t)kSmemBytes, stream, p, c);
 }

@@ -64,6 +64,8 @@ struct GroupedArgs {
 size_t gemm_tc_smem_bytes();
 int gemm_tc_rows_per_unit();
 int gemm_tc_weight_rows_per_unit();
+int gemm_tc_small_box_rows();  // activation rows per box for groups of at most this many rows (tm_a)
+int gemm_tc_big_box_rows();    // activation rows per box otherwise (tm_a_big)
 // swiglu: p.w is a gate_up stack [E, N = 2I, K/2] (tm_w its 5-D gate/up view) and p.y the [M, I] output h.
 cudaError_t launch_gemm_tc(int fmt, bool swiglu, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big,
                            const CUtensorMap& tm_w, const GroupedArgs& p, int grid, cudaStream_t stream);

@@ -141,6 +141,12 @@ WORKLOADS = {
     "kimi-prefill": Workload("kimi-prefill", "mxfp4", E=384, k=8, T=4096,
                              projections=(Projection("gate_up", 7168, 4096), Projection("down", 2048, 7168)),
                              routing="zipf", zipf_s=1.2),
+    # The same shapes scaled to 48 experts and 512 tokens (the same mean of 85
+    # rows per expert, Zipf(1.2) skew): a device footprint of about 1 GB, for
+    # profiler captures of the Kimi-class kernels.
+    "kimi-prefill-e48": Workload("kimi-prefill-e48", "mxfp4", E=48, k=8, T=512,
+                                 projections=(Projection("gate_up", 7168, 4096), Projection("down", 2048, 7168)),
+                                 routing="zipf", zipf_s=1.2),
 }
 
 
