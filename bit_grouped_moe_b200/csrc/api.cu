@@ -134,6 +134,20 @@ gnf4_status encode_act_map(CUtensorMap* m, const void* a, int M, int K, int box_
   return GNF4_OK;
 }
 
+// Y [M, cols] bf16 row-major, written by TMA stores of box_cols x box_rows (no swizzle).
+gnf4_status encode_out_map(CUtensorMap* m, void* y, int M, int cols, int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(GNF4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)M};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GNF4_ERR_CUDA, "output tensor map encode failed (CUresult %d)", (int)r);
+  return GNF4_OK;
+}
+
 // W [E, N, K/2] u8: box_bytes x box_rows x 1 boxes, no swizzle, zero fill.
 gnf4_status encode_weight_map(CUtensorMap* m, const void* w, int E, int N, int K, int box_bytes, int box_rows) {
   auto fn = encode_fn();
@@ -198,14 +212,16 @@ gnf4_status grouped_gemm(int fmt, bool swiglu, const void* a, const uint8_t* w, 
   if (M == 0) return GNF4_OK;
   DeviceState* d = nullptr;
   GNF4_TRY(device_state(&d));
-  CUtensorMap tm_a, tm_a_big, tm_w;
+  CUtensorMap tm_a, tm_a_big, tm_w, tm_y;
   GNF4_TRY(encode_act_map(&tm_a, a, M, K, gemm_tc_small_box_rows()));
+  GNF4_TRY(encode_out_map(&tm_y, y, M, swiglu ? N / 2 : N, swiglu ? gemm_tc_weight_box_rows() / 2 : gemm_tc_weight_box_rows(),
+                          gemm_tc_out_box_rows()));
   GNF4_TRY(encode_act_map(&tm_a_big, a, M, K, gemm_tc_big_box_rows()));
   const int wrows = gemm_tc_weight_rows_per_unit();
   if (swiglu)
     GNF4_TRY(encode_swiglu_weight_map(&tm_w, w, E, N / 2, K));
   else
-    GNF4_TRY(encode_weight_map(&tm_w, w, E, N, K, 32, wrows));
+    GNF4_TRY(encode_weight_map(&tm_w, w, E, N, K, 32, gemm_tc_weight_box_rows()));
   GroupedArgs p{static_cast<const __nv_bfloat16*>(a), w, scales, offsets, counts,
                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
   // upper bound on work units: every group adds at most one partial chunk
@@ -214,8 +230,8 @@ gnf4_status grouped_gemm(int fmt, bool swiglu, const void* a, const uint8_t* w, 
   const long long chunks = (M + rpu - 1) / rpu + (E < M ? E : M);
   const long long units = chunks * nwt;
   if (units >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d, N=%d give too many work units", M, N);
-  const int grid = (int)(units < d->num_sms ? units : d->num_sms);
-  cudaError_t e = launch_gemm_tc(fmt, swiglu, tm_a, tm_a_big, tm_w, p, grid, as_stream(stream));
+  const int grid = gemm_tc_grid(units, d->num_sms);
+  cudaError_t e = launch_gemm_tc(fmt, swiglu, tm_a, tm_a_big, tm_w, tm_y, p, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMM launch");
   return GNF4_OK;
 }

@@ -62,13 +62,18 @@ struct GroupedArgs {
 
 // gemm_tc.cu
 size_t gemm_tc_smem_bytes();
-int gemm_tc_rows_per_unit();
-int gemm_tc_weight_rows_per_unit();
+int gemm_tc_rows_per_unit();         // token rows per unit
+int gemm_tc_weight_rows_per_unit();  // weight rows per unit (a CTA pair)
+int gemm_tc_weight_box_rows();       // weight rows per CTA (tm_w box)
+int gemm_tc_grid(long long units, int num_sms);  // CTAs (whole pairs) for `units` units
+int gemm_tc_out_box_rows();          // tokens per output store (tm_y box rows)
 int gemm_tc_small_box_rows();  // activation rows per box for groups of at most this many rows (tm_a)
 int gemm_tc_big_box_rows();    // activation rows per box otherwise (tm_a_big)
 // swiglu: p.w is a gate_up stack [E, N = 2I, K/2] (tm_w its 5-D gate/up view) and p.y the [M, I] output h.
+// tm_y: the output [M, N] (SwiGLU: [M, I]) bf16 in boxes of 128 (SwiGLU: 64) columns x gemm_tc_out_box_rows() rows.
 cudaError_t launch_gemm_tc(int fmt, bool swiglu, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big,
-                           const CUtensorMap& tm_w, const GroupedArgs& p, int grid, cudaStream_t stream);
+                           const CUtensorMap& tm_w, const CUtensorMap& tm_y, const GroupedArgs& p, int grid,
+                           cudaStream_t stream);
 
 // Fused top-k combine in the GEMV epilogue (device pointers).
 struct CombineArgs {
