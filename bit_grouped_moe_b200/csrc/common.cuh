@@ -381,6 +381,16 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// Acquire / release accesses of a shared-memory counter (CTA scope).
+__device__ __forceinline__ uint32_t ld_acquire_shared(const void* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_shared(void* p, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
 // ---------------------------------------------------------------- CTA pairs
 // Two CTAs of a cluster share one MMA (cta_group::2): the even CTA issues it,
 // both hold half of each operand and their own half of the accumulator.

@@ -45,8 +45,10 @@
 //  * Epilogue: TMEM -> registers -> bf16 tile in shared memory -> one TMA
 //    store per 32 tokens (double-buffered); a ragged last chunk is stored
 //    element by element.
-//  * Warp roles per CTA (25 warps): 0 and 24 = weight TMA, 1 = TMEM owner
-//    (both CTAs) + MMA issuer (even CTA), 2 = activation TMA, 3 = scale loader
+//  * Warp roles per CTA (26 warps): 0 and 24 = weight TMA, 1 = TMEM owner
+//    (both CTAs) + MMA issuer (even CTA), 25 = stage poller (even CTA: tests
+//    the stage barriers and publishes a ready count the MMA thread reads with
+//    a load-acquire), 2 = activation TMA, 3 = scale loader
 //    (raw block scales copied into a shared-memory ring with cp.async, 8
 //    k-stages per chunk, 3 chunks ahead), 4..19 = decode (four groups of
 //    four; group g takes the stages it = g mod 4, so every ring slot is
@@ -79,7 +81,8 @@ constexpr int kDecGroups = 4;
 constexpr int kDecWarp0 = 4;
 constexpr int kEpiWarp0 = kDecWarp0 + 4 * kDecGroups;  // 20
 constexpr int kWProd2 = kEpiWarp0 + 4;                 // 24: second weight producer
-constexpr int kThreads = (kWProd2 + 1) * 32;           // 800
+constexpr int kPoller = kWProd2 + 1;                   // 25: tests the stage barriers for the MMA thread
+constexpr int kThreads = (kPoller + 1) * 32;           // 832
 constexpr int kSmallBox = 16;                          // activation rows per box, half-tiles of <= 16 rows
 constexpr int kBigBox = 64;                            // activation rows per box otherwise
 constexpr int kACol0 = kBT;                            // decoded-weight ring after the accumulator
@@ -110,6 +113,7 @@ struct Smem {
   uint64_t accf, acce;  // acce: even CTA only, 8 arrivals (both CTAs' epilogue warps)
   uint64_t mdone;       // abort path only: every issued MMA has retired
   uint32_t tmem_base;
+  uint32_t tready;  // even CTA: stages whose report is complete (the poller counts, the MMA thread reads)
   int abort;
 };
 static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
@@ -228,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&s.accf, 1);
     mbar_init(&s.acce, 8);
     mbar_init(&s.mdone, 1);
+    s.tready = 0;
     s.abort = 0;
     fence_mbar_init();
   }
@@ -348,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && cta == 0) {
       int it = 0, uc = 0;
+      uint32_t ready = 0;  // stages the poller had counted complete at the last read
       bool ok = true;
       for (int u = pair; u < U && ok; u += npairs, ++uc) {
         const Unit x = unit_of(s, p.E, u);
@@ -356,9 +362,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t idesc = idesc_bf16_m256((uint32_t)x.n);
         for (int kt = 0; kt < nk; ++kt, ++it) {
           const int sa = it % kAStages, sT = it % kTStages;
-          // one barrier per stage: both CTAs' decode warps report a stage only
-          // after their CTA's activation half-tile has landed
-          if (!(ok = mbar_wait_cl(&s.tfull[sT], (it / kTStages) & 1, err, abort))) break;
+          // Both CTAs report a stage only after its activation half-tiles have
+          // landed.  The poller warp tests those barriers and counts the
+          // complete stages; this thread re-reads the count only when it has
+          // used up the last one it read.  Any shared-memory access here waits
+          // ~220 cycles behind the decode warps' table lookups (measured), long
+          // enough to let the tensor pipe run dry if paid every stage; the
+          // poller runs several stages ahead, so one read covers several.
+          if ((int)ready <= it) ready = ld_acquire_shared(&s.tready);
+          if ((int)ready <= it) {
+            const long long t0 = clock64();
+            while ((int)(ready = ld_acquire_shared(&s.tready)) <= it) {
+              if (*abort) {
+                ok = false;
+                break;
+              }
+              if (clock64() - t0 > kSpinLimitCycles) {
+                atomicOr(err, GNF4_DEVERR_TIMEOUT);
+                *abort = 1;
+                ok = false;
+                break;
+              }
+            }
+            if (!ok) break;
+          }
           tc_fence_after();
           const uint32_t a_col = tmem + (uint32_t)(kACol0 + sT * (kBK / 2));
           const uint32_t b_addr = smem_u32(s.act[sa]);
@@ -376,6 +403,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit_pair(&s.mdone);
         mbar_drain(&s.mdone, 0);
       }
+    }
+  } else if (warp == kPoller) {
+    // ------------------------------------------------------------ stage poller (even CTA)
+    if (lane == 0 && cta == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int u = pair; u < U && ok; u += npairs)
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          if (!(ok = mbar_wait_cl(&s.tfull[it % kTStages], (it / kTStages) & 1, err, abort))) break;
+          st_release_shared(&s.tready, (uint32_t)(it + 1));
+        }
     }
   } else if (warp >= kDecWarp0 && warp < kEpiWarp0) {
     // ------------------------------------------------------------ decode
