@@ -12,10 +12,11 @@
 // computes the partial sums of all 64 rows (four m16 tiles) for the group's
 // <= 8 rows (the MMA's 8 columns); a fixed-order shared-memory reduction over
 // the 8 warps finishes the unit.  Per item a lane holds 16 bytes (32 codes)
-// of each of its 8 weight rows and decodes every byte with one PRMT, which
+// of each of its 8 weight rows, decodes every byte with one PRMT, which
 // builds the shared-memory address of a lane-private pair-table entry, and
-// one shared load; the bf16 pairs feed m16n8k16 warp MMAs.  The MMA does the
-// k reduction that a CUDA-core GEMV would do with shuffles.
+// one shared load, multiplies the bf16 pair by the row's block scale, and
+// feeds the pairs to m16n8k16 warp MMAs.  The MMA does the k reduction that
+// a CUDA-core GEMV would do with shuffles.
 //
 // Fused combine (CMB): after a half has stored its unit's rows, each row
 // counts its (token, 64-column block) in; the half that completes a token's
@@ -37,17 +38,13 @@
 // that extracts a byte also inserts the table's base, so a lookup is exactly
 // one PRMT and one shared load.
 //
-// Lane (g, t) = (lane / 4, lane % 4) owns rows g and g+8 of every tile.  The
-// MMA's k index is a permutation of the physical k, and the activation
-// fragment uses the same permutation:
-//   * MXFP4: the lane takes the 32 consecutive k [32t, 32t+32) of an item (one
-//     block); each decoded pair is multiplied by the row's block scale in
-//     bf16, which is exact (e2m1 x 2^(e-127) is a bf16 value).
-//   * NF4: the lane takes k [16t, 16t+16) of each 64-k block, so the four MMA
-//     steps of a block stay inside it.  The MMAs multiply the bf16-rounded
-//     codes into a fresh fp32 partial sum per block, which is multiplied by
-//     the rows' fp32 absmax and added to the accumulator: one bf16 rounding
-//     per weight (the code's, <= 2^-9 relative), no bf16 product.
+// Lane (g, t) = (lane / 4, lane % 4) owns rows g and g+8 of every tile and,
+// in every item, the 32 consecutive k in [32t, 32t+32) (one NF4 half-block,
+// one MXFP4 block).  The MMA's k index is a permutation of these physical k;
+// the activation fragment uses the same permutation.
+//   * MXFP4: e2m1 x 2^(e-127) is exact in bf16.
+//   * NF4: the code is rounded to bf16, then multiplied by bf16(absmax) and
+//     rounded again (relative error <= ~3 * 2^-9 per weight); sums are fp32.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -73,6 +70,13 @@ struct GemvLow {
   int scratch[kMaxExperts];
 };
 
+// f32 -> bf16 (round to nearest even, NaN kept quiet), duplicated in both halves.
+__device__ __forceinline__ uint32_t cvt_bf16x2_dup(float f) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(d) : "f"(f));
+  return d;
+}
+
 // One pair-table lookup: byte j of `word` selects the entry; `lanesel` holds
 // 4*lane in byte 0 and byte 2 of the table's 64 KB-aligned base in byte 2.
 __device__ __forceinline__ uint32_t lut_lookup(uint32_t word, uint32_t lanesel, uint32_t j) {
@@ -89,7 +93,7 @@ __device__ __forceinline__ void half_barrier(int h) {
 struct UnitView {
   const uint8_t* w;            // weight row n0 (q = 0), byte 0
   const uint8_t* sc;           // first scale of row n0 (bytes)
-  const __nv_bfloat16* x;      // activation row of token g (row 0 if g >= rows), at the lane's first k
+  const __nv_bfloat16* x;      // activation row of token g (row 0 if g >= rows), k = 32t
   int qv;                      // rows n0 + 8q < N  <=>  q < qv
   bool tv;                     // token g exists
 };
@@ -113,8 +117,7 @@ __device__ __forceinline__ UnitView unit_view(const GemvLow& s, const GroupedArg
   v.w = p.w + row * (size_t)(p.K / 2);
   v.sc = reinterpret_cast<const uint8_t*>(p.scales) + row * (size_t)nsc * (FMT == 0 ? 4u : 1u);
   v.tv = g < rows;
-  // NF4: lane t takes k [16t, 16t+16) of every 64-k block; MXFP4: k [32t, 32t+32) of every item
-  v.x = p.a + (size_t)(r0 + (v.tv ? g : 0)) * p.K + (FMT == 0 ? 16 : 32) * t;
+  v.x = p.a + (size_t)(r0 + (v.tv ? g : 0)) * p.K + 32 * t;
   v.qv = (p.N - n0 + 7) / 8;
   return v;
 }
@@ -122,61 +125,34 @@ __device__ __forceinline__ UnitView unit_view(const GemvLow& s, const GroupedArg
 // Loads of one item for tile i (rows q = 2i, 2i+1): packed weights and raw scales.
 // `rb` = packed bytes per weight row, `nsr` = scales per weight row, `gap` =
 // I - 32 (kModeSwiglu: rows from the unit's last gate row block to its up rows).
-//   NF4 (block-aligned): wq[q] = the lane's 8 bytes of 64-k blocks 2d (x, y) and
-//   2d+1 (z, w); sr[2q + b] = the raw fp32 absmax of block 2d + b (0 past K).
-//   MXFP4: wq[q] = the lane's 16 bytes of the item; sr[q] = the e8m0 byte of its block.
 template <int FMT, int MODE>
 __device__ __forceinline__ void load_tile(const UnitView& v, int d, int t, int K, size_t rb, size_t nsr, int gap,
-                                          int i, uint4 (&wq)[8], uint32_t (&sr)[16]) {
+                                          int i, uint4 (&wq)[8], uint32_t (&sr)[8]) {
+  const bool inK = d * kDK + 32 * t < K;
+  const size_t kb = inK ? (size_t)(d * (kDK / 2) + 16 * t) : 0;  // outside K: any valid address
+  const size_t si = inK ? (size_t)(FMT == 0 ? 2 * d + (t >> 1) : 4 * d + t) : 0;
 #pragma unroll
   for (int hq = 0; hq < 2; ++hq) {
     const int q = 2 * i + hq;
     const int roff = MODE == kModeClamp ? 8 * min(q, v.qv - 1) : (MODE == kModeSwiglu && q >= 4 ? 8 * q + gap : 8 * q);
-    const uint8_t* wrow = v.w + (size_t)roff * rb;
-    if (FMT == 0) {
-      const int nb = K / 64;
-#pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        const int blk = 2 * d + b;
-        const bool in = blk < nb;
-        const uint2 w8 = ldg_nc_u64(wrow + (in ? (size_t)(32 * blk + 8 * t) : 0));  // outside K: any valid address
-        if (b == 0) {
-          wq[q].x = w8.x;
-          wq[q].y = w8.y;
-        } else {
-          wq[q].z = w8.x;
-          wq[q].w = w8.y;
-        }
-        sr[2 * q + b] = in ? __ldg(reinterpret_cast<const unsigned int*>(v.sc) + (size_t)roff * nsr + blk) : 0u;
-      }
-    } else {
-      const bool inK = d * kDK + 32 * t < K;
-      const size_t kb = inK ? (size_t)(d * (kDK / 2) + 16 * t) : 0;  // outside K: any valid address
-      wq[q] = ldg_nc_u128(wrow + kb);
-      sr[q] = __ldg(v.sc + (size_t)roff * nsr + (inK ? (size_t)(4 * d + t) : 0));
-    }
+    wq[q] = ldg_nc_u128(v.w + (size_t)roff * rb + kb);
+    if (FMT == 0)
+      sr[q] = __ldg(reinterpret_cast<const unsigned int*>(v.sc + ((size_t)roff * nsr + si) * 4u));
+    else
+      sr[q] = __ldg(v.sc + (size_t)roff * nsr + si);
   }
 }
 
-// Activations of token g for one item.  NF4: xa[2b], xa[2b+1] = k [16t, 16t+16)
-// of block 2d + b; MXFP4: xa[c] = k [32t + 8c, 32t + 8c + 8) of the item.
-template <int FMT>
 __device__ __forceinline__ void load_acts(const UnitView& v, int d, int t, int K, uint4 (&xa)[4]) {
-  if (FMT == 0) {
+  const bool ok = v.tv && (d * kDK + 32 * t < K);
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const bool ok = v.tv && ((2 * d + b) * 64 < K);
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-        xa[2 * b + c] = ok ? ldg_u128(v.x + d * kDK + 64 * b + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
-    }
-  } else {
-    const bool ok = v.tv && (d * kDK + 32 * t < K);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) xa[c] = ok ? ldg_u128(v.x + d * kDK + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
-  }
+  for (int c = 0; c < 4; ++c) xa[c] = ok ? ldg_u128(v.x + d * kDK + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
 }
 
+template <int FMT>
+__device__ __forceinline__ uint32_t scale_pair(uint32_t raw) {
+  return FMT == 0 ? cvt_bf16x2_dup(__uint_as_float(raw)) : e8m0_to_bf16x2(raw);
+}
 
 // Sum over the valid pairs of token t (sorted row inside [0, nvalid)).
 __device__ __forceinline__ int valid_pairs(const CombineArgs& c, int t, int nvalid) {
@@ -197,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p, Combin
   const int h = warp / kSplit, ks = warp % kSplit;
 
   // The table takes the first 64 KB boundary above GemvLow; the host refuses
-  // to launch when the window cannot hold it (gemv_static_smem_ok), so this
+  // to launch when the window cannot hold it (table_fits_once), so this
   // check only guards against a window placed differently than the host saw.
   const uint32_t base = smem_u32(smem_raw);
   const uint32_t lut_at = (base + (uint32_t)sizeof(GemvLow) + 0xFFFFu) & ~0xFFFFu;
@@ -233,14 +209,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p, Combin
 
   // first item of this warp's stream
   uint4 wq[8], xa[4];
-  uint32_t sr[16];
+  uint32_t sr[8];
   UnitView cur{};
   if (u < U) {
     cur = unit_view<FMT, MODE>(s, p, u, g, t);
     if (d_lo < d_hi) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) load_tile<FMT, MODE>(cur, d_lo, t, K, rb, nsr, gap, i, wq, sr);
-      load_acts<FMT>(cur, d_lo, t, K, xa);
+      load_acts(cur, d_lo, t, K, xa);
     }
   }
   __syncthreads();
@@ -261,48 +237,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GroupedArgs p, Combin
       const bool has_next = !last || u + ustride < U;
       if (last && has_next) cur = unit_view<FMT, MODE>(s, p, u + ustride, g, t);
       uint4 xn[4];
-      if (has_next) load_acts<FMT>(cur, dn, t, K, xn);
+      if (has_next) load_acts(cur, dn, t, K, xn);
 
       const uint32_t xp[16] = {xa[0].x, xa[0].y, xa[0].z, xa[0].w, xa[1].x, xa[1].y, xa[1].z, xa[1].w,
                                xa[2].x, xa[2].y, xa[2].z, xa[2].w, xa[3].x, xa[3].y, xa[3].z, xa[3].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
+        const uint32_t s0 = scale_pair<FMT>(sr[2 * i]), s1 = scale_pair<FMT>(sr[2 * i + 1]);
         const uint32_t w0[4] = {wq[2 * i].x, wq[2 * i].y, wq[2 * i].z, wq[2 * i].w};
         const uint32_t w1[4] = {wq[2 * i + 1].x, wq[2 * i + 1].y, wq[2 * i + 1].z, wq[2 * i + 1].w};
-        if (FMT == 0) {
-          // Block-aligned: the four MMA steps of 64-k block b take the quad's
-          // k [16t + 4j, 16t + 4j + 4) (bytes 2j, 2j+1 of the lane's 8), so a
-          // step never leaves its block; the fp32 partial sum of the block is
-          // then scaled once by the rows' absmax.
+        // MMA step j takes bytes 2j, 2j+1 of both rows (word j/2, bytes 2(j%2) and 2(j%2)+1)
 #pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t bs = 2u * (uint32_t)(j & 1);
-              const uint32_t ww0 = w0[2 * b + (j >> 1)], ww1 = w1[2 * b + (j >> 1)];
-              mma_bf16_16816(part, lut_lookup(ww0, lanesel, bs), lut_lookup(ww1, lanesel, bs),
-                             lut_lookup(ww0, lanesel, bs + 1u), lut_lookup(ww1, lanesel, bs + 1u), xp[8 * b + 2 * j],
-                             xp[8 * b + 2 * j + 1]);
-            }
-            const float s0 = __uint_as_float(sr[4 * i + b]), s1 = __uint_as_float(sr[4 * i + 2 + b]);
-            acc[i][0] = fmaf(s0, part[0], acc[i][0]);
-            acc[i][1] = fmaf(s0, part[1], acc[i][1]);
-            acc[i][2] = fmaf(s1, part[2], acc[i][2]);
-            acc[i][3] = fmaf(s1, part[3], acc[i][3]);
-          }
-        } else {
-          const uint32_t s0 = e8m0_to_bf16x2(sr[2 * i]), s1 = e8m0_to_bf16x2(sr[2 * i + 1]);
-          // MMA step j takes bytes 2j, 2j+1 of both rows (word j/2, bytes 2(j%2) and 2(j%2)+1)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t b0 = 2u * (uint32_t)(j & 1);
-            const uint32_t a0 = bf16x2_mul(lut_lookup(w0[j >> 1], lanesel, b0), s0);
-            const uint32_t a1 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0), s1);
-            const uint32_t a2 = bf16x2_mul(lut_lookup(w0[j >> 1], lanesel, b0 + 1u), s0);
-            const uint32_t a3 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0 + 1u), s1);
-            mma_bf16_16816(acc[i], a0, a1, a2, a3, xp[2 * j], xp[2 * j + 1]);
-          }
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t b0 = 2u * (uint32_t)(j & 1);
+          const uint32_t a0 = bf16x2_mul(lut_lookup(w0[j >> 1], lanesel, b0), s0);
+          const uint32_t a1 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0), s1);
+          const uint32_t a2 = bf16x2_mul(lut_lookup(w0[j >> 1], lanesel, b0 + 1u), s0);
+          const uint32_t a3 = bf16x2_mul(lut_lookup(w1[j >> 1], lanesel, b0 + 1u), s1);
+          mma_bf16_16816(acc[i], a0, a1, a2, a3, xp[2 * j], xp[2 * j + 1]);
         }
         if (has_next) load_tile<FMT, MODE>(cur, dn, t, K, rb, nsr, gap, i, wq, sr);
       }

@@ -37,8 +37,10 @@
 //    commits: it is the one serial thread of the pipeline.
 //  * K not a multiple of the stage's k: the last stage reads [K - kBK, K)
 //    and skips the MMAs already covered, so no box reads past a row.
-//  * Warp roles (13 warps): 0 and 12 = TMA producers (alternate stages: one
+//  * Warp roles (14 warps): 0 and 12 = TMA producers (alternate stages: one
 //    issuing thread alone caps the stream), 1 = TMEM owner + MMA issuer,
+//    13 = stage poller (tests the full barriers and publishes a count of
+//    complete stages that the MMA thread reads with a load-acquire),
 //    4..7 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31, i.e. weight
 //    rows), 2, 3 and 8.. = scale loaders, one per ring slot, so the global
 //    loads of every stage in the ring are in flight at once.  Two TMEM
@@ -241,7 +243,8 @@ constexpr int kBW = 128;  // weight rows per unit = MMA M
 constexpr int kBox = 32;  // activation rows per small TMA box
 constexpr int kEpiWarp0 = 4;
 constexpr int kProd2 = 12;  // second TMA producer warp
-constexpr int kThreads = 13 * 32;
+constexpr int kPoller = 13;  // tests the stage barriers for the MMA thread
+constexpr int kThreads = 14 * 32;
 constexpr int kWStageBytes = kBW * 128;  // one 128-byte row per weight row and stage
 constexpr int kTmemCols = 512;
 
@@ -270,6 +273,7 @@ struct MxSmem {
   uint64_t accf[2], acce[2];
   uint64_t mdone;  // abort path only: every issued MMA has retired
   uint32_t tmem_base;
+  uint32_t sready;  // stages whose operands and scales are complete (the poller counts, the MMA thread reads)
   int abort;
 };
 #define GNF4_MX_CHECK(M)                                                                               \
@@ -416,6 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.acce[i], 4);
     }
     mbar_init(&s.mdone, 1);
+    s.sready = 0;
     s.abort = 0;
     fence_mbar_init();
   }
@@ -541,11 +546,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(&s.ldone[li]);
       mbar_drain(&s.ldone[li], 0);
     }
+  } else if (warp == kPoller) {
+    // ------------------------------------------------------------ stage poller
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < U && ok; u += gridDim.x)
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          if (!(ok = mbar_wait(&s.full[it % kStages], (uint32_t)(it / kStages) & 1u, err, abort))) break;
+          st_release_shared(&s.sready, (uint32_t)(it + 1));
+        }
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int it = 0, uc = 0;
-      bool ok = true, ready = false;  // ready: the full barrier of stage `it` was seen complete in advance
+      uint32_t ready = 0;  // stages the poller had counted complete at the last read
+      bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
         const Unit x = unit_of<MODE>(s, p.E, u);
         const int ab = uc & 1;
@@ -559,10 +576,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < nk; ++kt, ++it) {
           const int st = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-          if (!ready && !(ok = mbar_wait(&s.full[st], ph, err, abort))) break;
+          (void)ph;
+          // The poller warp tests the stage barriers and counts complete
+          // stages; this thread re-reads the count only after using up the
+          // last value.  An mbarrier test here costs ~220 cycles while MMAs
+          // are in flight (measured), enough to let the tensor pipe run dry.
+          if ((int)ready <= it) ready = ld_acquire_shared(&s.sready);
+          if ((int)ready <= it) {
+            const long long t0 = clock64();
+            while ((int)(ready = ld_acquire_shared(&s.sready)) <= it) {
+              if (*abort) {
+                ok = false;
+                break;
+              }
+              if (clock64() - t0 > kSpinLimitCycles) {
+                atomicOr(err, GNF4_DEVERR_TIMEOUT);
+                *abort = 1;
+                ok = false;
+                break;
+              }
+            }
+            if (!ok) break;
+          }
           tc_fence_after();
-          // test the next stage's barrier now: its latency overlaps this stage's issue
-          ready = mbar_try_wait(&s.full[(it + 1) % kStages], (uint32_t)((it + 1) / kStages) & 1u);
           const uint32_t t_sfw = tmem + (uint32_t)(sf_col0 + G::kSfCols * st);
           const uint32_t t_sfa = t_sfw + 4u * (uint32_t)(G::kSfwWords / 128);
           const uint32_t w_addr = smem_u32(s.w[st]), a_addr = smem_u32(s.a[st]);
