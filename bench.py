@@ -149,7 +149,7 @@ class Workload:
     than L2, a set of token batches, and the step's output buffers."""
 
     def __init__(self, name, device, seed, build_host_copy, swiglu=False, dgrad=False, w4a8=False,
-                 fused_combine=False, w4a8x2=False, w4a4=False):
+                 fused_combine=False, w4a8x2=False, w4a4=False, native=True):
         import torch
 
         from bit_grouped_moe_b200 import gnf4
@@ -244,6 +244,19 @@ class Workload:
                         ("mxfp4", True): f.grouped_gemv_mxfp4_swiglu, ("mxfp4", False): f.grouped_gemm_mxfp4_swiglu}[
                 (wl.fmt, self.decode)]
             self.hs = torch.empty(M, self.p1.N // 2, dtype=torch.bfloat16, device=device)
+        # MXFP4 prefill: groups of at most 96 rows on the native two-term path (the
+        # GEMM call with a workspace), larger groups on the decode path
+        ws_n = [gnf4.mxfp4_workspace_bytes(M, p.K) for p in (self.p1, self.p2)]
+        self.native = (native and wl.fmt == "mxfp4" and not self.decode and not dgrad and not self.w4a8
+                       and not swiglu and min(ws_n) > 0)
+        if self.native:
+            self.mws = torch.empty(max(ws_n), dtype=torch.uint8, device=device)  # the projections run in turn
+            self.fn = lambda a, w, s, y, offsets: gnf4.grouped_gemm_mxfp4_ws(a, w, s, y, self.mws, offsets=offsets)
+        lim = gnf4.mxfp4_native_max_rows()
+        self.native_rows = []  # rows in groups the native path takes, per batch
+        for b in self.batches:
+            sizes = np.bincount(b[0].reshape(-1), minlength=E)
+            self.native_rows.append(int(sizes[sizes <= lim].sum()) if self.native else 0)
 
     def _stack(self, fmt, p, seed, keep_host):
         torch = self.torch
@@ -374,7 +387,9 @@ class Workload:
         # route (one launch for at most 256 pairs, else hist + scan + scatter + gather) + 2 projections + combine
         route = 1 if 0 < self.M <= 256 else 4
         combine = 0 if (self.dgrad or self.fused_combine) else 1
-        return route + 2 + combine + (2 if self.w4a8 else 0)
+        # the native MXFP4 call: split quantiser + native GEMM + decode GEMM per projection (M > 96)
+        native = 4 if self.native else 0
+        return route + 2 + combine + (2 if self.w4a8 else 0) + native
 
 
 # ------------------------------------------------------------------ distributed
@@ -510,6 +525,10 @@ def roofline(wl, args, peaks, peak_src, dom_ms, hit, dom_stats, traffic):
         n_out = N // 2 if wl.swiglu else N
         io = 2 * M * K + 2 * M * n_out
         kind, per = "bf16", 1.0
+        if wl.native:
+            # the native path's rows: two e4m3 terms + scales written by the quantiser and read by the GEMM; its
+            # MMAs run at the fp8 rate, two per useful product, so its useful-flop peak is the bf16 one
+            io += 2 * 2 * wl.native_rows[0] * (K + K // 32)
     B = float(wbytes + io)
     ratio = {"bf16": 1.0, "fp8": 2.0, "fp4": 4.0}[kind]
     dc = dom_stats.get("clocks") or {}
@@ -525,7 +544,10 @@ def roofline(wl, args, peaks, peak_src, dom_ms, hit, dom_stats, traffic):
     bound = "tensor" if t_tensor >= t_hbm else "hbm"
     t_nom = max(F / (nominal_t * 1e12), B / (NOMINAL["hbm_gbs"] * 1e9))
     achieved = F / t / 1e12 if bound == "tensor" else B / t / 1e9
-    kname = (f"dgrad_tc_kernel<{wl.wl.fmt}> (dX of {p.name}, K={K}, N={N})" if wl.dgrad else
+    kname = (f"gnf4_grouped_gemm_mxfp4_ws ({p.name}, K={K}, N={N}): quant_mxfp8_rows_kernel + "
+             f"gemm_mx_kernel<two-term> on the {wl.native_rows[0]} rows of groups <= 96 rows, "
+             f"gemm_tc_kernel<mxfp4> on the rest (3 launches)" if wl.native else
+             f"dgrad_tc_kernel<{wl.wl.fmt}> (dX of {p.name}, K={K}, N={N})" if wl.dgrad else
              f"gemm_mx_kernel<W4A4> ({p.name}, K={K}, N={N})" if wl.a4 else
              f"gemm_mx_kernel<two-term> ({p.name}, K={K}, N={N})" if wl.split else
              f"gemm_mx_kernel<W4A8> ({p.name}, K={K}, N={N})" if wl.w4a8 else
@@ -548,6 +570,8 @@ def roofline(wl, args, peaks, peak_src, dom_ms, hit, dom_stats, traffic):
         "combined_bound_us": round(max(t_tensor, t_hbm) * 1e6, 3), "frac_nominal": round(t_nom / t, 4),
         "peak_source": f"{peak_src} (MEASURED_PEAKS.json: bf16_tflops / bf16_tflops_sustained x the nominal "
                        f"{kind}/bf16 ratio {ratio:g}{', halved for the two-term form' if per != 1 else ''}; hbm_gbs)",
+        **({"tensor_note": "native rows run kind::mxf8f6f4 at 2x the bf16 rate with two MMAs per useful product, "
+                           "the rest kind::f16: both at the bf16 useful-flop peak"} if wl.native else {}),
     }
 
 
@@ -577,6 +601,8 @@ def main():
     ap.add_argument("--fused-combine", action="store_true",
                     help="decode: run the top-k combine in the second GEMV's epilogue instead of as its own launch "
                          "(measured slower on B200: the epilogue's round trips extend every unit)")
+    ap.add_argument("--no-native", action="store_true",
+                    help="MXFP4 prefill: every group on the decode path (gnf4_grouped_gemm_mxfp4 without a workspace)")
     ap.add_argument("--swiglu", action="store_true",
                     help="first projection = fused gate_up + SwiGLU (gate rows first); the second reads its output")
     ap.add_argument("--weight-copies", type=int, default=None,
@@ -630,7 +656,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     dev = f"cuda:{local}"
     torch.cuda.set_device(local)
     wl = Workload(args.workload, dev, seed=1234 + rank, build_host_copy=(rank == 0 and world == 1),
-                  swiglu=args.swiglu, dgrad=args.dgrad, w4a8=args.w4a8, fused_combine=args.fused_combine, w4a8x2=args.w4a8x2, w4a4=args.w4a4)
+                  swiglu=args.swiglu, dgrad=args.dgrad, w4a8=args.w4a8, fused_combine=args.fused_combine,
+                  w4a8x2=args.w4a8x2, w4a4=args.w4a4, native=not args.no_native)
     decode = wl.decode
     wl.h_host = wl.h.cpu().view(torch.int16).numpy().view(np.uint16)
     stream = torch.cuda.current_stream()
@@ -797,11 +824,11 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
 
     peaks, peak_src = load_peaks()
     kern_file = "gemv.cu" if decode else ("dgrad.cu" if wl.dgrad else ("mx.cu" if wl.w4a8 else "gemm_tc.cu"))
-    kern_base = "gemv" if decode else ("dgrad_tc" if wl.dgrad else
+    kern_base = "gemm_mxfp4_ws" if wl.native else "gemv" if decode else ("dgrad_tc" if wl.dgrad else
                                        ("gemm_w4a4" if wl.a4 else ("gemm_w4a8x2" if wl.split else
                                                                   ("gemm_w4a8" if wl.w4a8 else "gemm_tc"))))
     kern_key = f"{kern_base}_{wl.wl.fmt}{'_swiglu' if wl.swiglu else ''}:{args.workload}:{wl.p1.name}"
-    sha = kernel_source_sha([kern_file, "common.cuh"])
+    sha = kernel_source_sha(["mx.cu", "gemm_tc.cu", "common.cuh"] if wl.native else [kern_file, "common.cuh"])
     roof = roofline(wl, args, peaks, peak_src, dom_ms, dom_hit, dom_stats, committed_traffic(kern_key, sha))
 
     cpu = cpu1 = None
@@ -831,6 +858,9 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
                               if wl.split else
                               {"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if wl.w4a8 else {}),
                            **({"combine": "in the second GEMV's epilogue"} if wl.fused_combine else {}),
+                           **({"mxfp4_path": "groups <= 96 rows: native two-term MXFP8 x e2m1 (kind::mxf8f6f4, "
+                                             "bf16-activation accuracy); larger groups: decode to bf16 (kind::f16)"}
+                              if wl.native else {}),
                            **({"step": "backward: route + dgrad of both projections"} if wl.dgrad else {})),
             "roofline": roof, "cpu_baseline": cpu, **({"cpu_baseline_1core": cpu1} if cpu1 else {}),
             "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

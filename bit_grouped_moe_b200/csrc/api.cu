@@ -205,9 +205,10 @@ gnf4_status check_grouped(int fmt, const void* a, const uint8_t* w, const void* 
 }
 
 // swiglu: w is a gate_up stack [E, N = 2I, K/2] and y the [M, I] output h.
+// min_rows > 0: groups of fewer rows are skipped (their rows of y are left to another kernel).
 gnf4_status grouped_gemm(int fmt, bool swiglu, const void* a, const uint8_t* w, const void* scales,
                          const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M, void* y,
-                         void* stream) {
+                         void* stream, int min_rows = 0) {
   GNF4_TRY(check_grouped(fmt, a, w, scales, offsets, counts, E, N, K, M, y));
   if (M == 0) return GNF4_OK;
   DeviceState* d = nullptr;
@@ -224,6 +225,7 @@ gnf4_status grouped_gemm(int fmt, bool swiglu, const void* a, const uint8_t* w, 
     GNF4_TRY(encode_weight_map(&tm_w, w, E, N, K, 32, gemm_tc_weight_box_rows()));
   GroupedArgs p{static_cast<const __nv_bfloat16*>(a), w, scales, offsets, counts,
                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M};
+  p.min_rows = min_rows;
   // upper bound on work units: every group adds at most one partial chunk
   const long long nwt = (N + wrows - 1) / wrows;  // SwiGLU: (2I / 128) tiles of 64 gate + 64 up rows
   const long long rpu = gemm_tc_rows_per_unit();
@@ -317,7 +319,7 @@ gnf4_status grouped_dgrad(int fmt, const void* dy, const uint8_t* w, const void*
 gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* lo_codes,
                               const uint8_t* lo_scales, const uint8_t* w, const uint8_t* w_scales,
                               const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M, void* y,
-                              void* stream) {
+                              void* stream, int max_rows = 1 << 30) {
   const bool split = lo_codes != nullptr || lo_scales != nullptr;
   if (E < 1 || E > kMaxExperts) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "E=%d outside [1, %d]", E, kMaxExperts);
   if (N < 1 || N % 8 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N=%d must be a positive multiple of 8", N);
@@ -389,7 +391,8 @@ gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, c
   const int grid = (int)(units < d->num_sms ? units : d->num_sms);
   cudaError_t e = launch_gemm_mx(split ? 1 : 0, tm_a, tm_a_big, tm_w, tm_w_tail, a_scales,
                                  split ? lo_scales : nullptr, w_scales, offsets, counts,
-                                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M, grid, as_stream(stream));
+                                 static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M, grid, as_stream(stream),
+                                 max_rows);
   if (e != cudaSuccess) return cuda_fail(e, "W4A8 grouped GEMM launch");
   return GNF4_OK;
 }
@@ -449,6 +452,51 @@ gnf4_status grouped_gemm_w4a4(const uint8_t* a_blocks, const uint8_t* a_scales, 
   cudaError_t e = launch_gemm_mx(2, tm_a, tm_a_big, tm_w, tm_w, a_scales, nullptr, w_scales, offsets, counts,
                                  static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "W4A4 grouped GEMM launch");
+  return GNF4_OK;
+}
+
+// Workspace of the MXFP4 GEMM's native path: the two-term MXFP8 split of the
+// activations as hi codes [M, K], lo codes [M, K], hi scales [M, K/32] and lo
+// scales [M, K/32], each part 16-byte aligned.
+struct SplitWorkspace {
+  size_t hi, lo, hi_scales, lo_scales, total;
+};
+SplitWorkspace split_workspace(int M, int K) {
+  const size_t codes = (size_t)M * (size_t)K;  // a multiple of 64: K % 64 == 0
+  const size_t sc = ((size_t)M * (size_t)(K / 32) + 15) & ~size_t(15);
+  return {0, codes, 2 * codes, 2 * codes + sc, 2 * codes + 2 * sc};
+}
+
+// Shapes on which the native path runs (the two-term GEMM's rules).
+bool native_mxfp4_applies(int E, int N, int K) { return K >= 128 && K % 64 == 0 && (long long)E * N < (1LL << 31); }
+
+// Groups of at most gemm_mx_rows_per_unit(two-term) rows on the native
+// two-term path (one unit per weight tile), larger groups on the decode path.
+gnf4_status grouped_gemm_mxfp4_ws(const void* a, const uint8_t* w, const uint8_t* scales, const int32_t* offsets,
+                                  const int32_t* counts, int E, int N, int K, int M, void* y, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  GNF4_TRY(check_grouped(1, a, w, scales, offsets, counts, E, N, K, M, y));
+  if (M == 0) return GNF4_OK;
+  if (workspace == nullptr || !native_mxfp4_applies(E, N, K))
+    return grouped_gemm(1, false, a, w, scales, offsets, counts, E, N, K, M, y, stream);
+  const SplitWorkspace L = split_workspace(M, K);
+  if (workspace_bytes < L.total)
+    return fail(GNF4_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu bytes needed", workspace_bytes,
+                L.total);
+  GNF4_TRY(check_ptr(workspace, "workspace", 16));
+  GNF4_TRY(check_ptr(w, "w (native path: 32-byte alignment)", 32));
+  DeviceState* d = nullptr;
+  GNF4_TRY(device_state(&d));
+  const int thr = gemm_mx_rows_per_unit(1);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaError_t e = launch_quant_mxfp8_split_rows(static_cast<const __nv_bfloat16*>(a), K, offsets, counts, E, M, thr,
+                                                d->err, ws + L.hi, ws + L.hi_scales, ws + L.lo, ws + L.lo_scales,
+                                                d->num_sms, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "MXFP8 split quantiser (small groups) launch");
+  GNF4_TRY(grouped_gemm_w4a8(ws + L.hi, ws + L.hi_scales, ws + L.lo, ws + L.lo_scales, w, scales, offsets, counts, E,
+                             N, K, M, y, stream, thr));
+  if (M > thr)  // some group may hold more rows
+    GNF4_TRY(grouped_gemm(1, false, a, w, scales, offsets, counts, E, N, K, M, y, stream, thr + 1));
   return GNF4_OK;
 }
 
@@ -583,6 +631,19 @@ gnf4_status gnf4_grouped_gemm_nf4(const void* a, const uint8_t* w, const float* 
 gnf4_status gnf4_grouped_gemm_mxfp4(const void* a, const uint8_t* w, const uint8_t* scales, const int32_t* offsets,
                                     const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
   return grouped_gemm(1, false, a, w, scales, offsets, counts, E, N, K, M, y, stream);
+}
+
+size_t gnf4_grouped_gemm_mxfp4_workspace_bytes(int M, int K) {
+  if (M < 1 || K < 128 || K % 64 != 0 || K > 65536) return 0;
+  return split_workspace(M, K).total;
+}
+
+int gnf4_grouped_gemm_mxfp4_native_max_rows(void) { return gemm_mx_rows_per_unit(1); }
+
+gnf4_status gnf4_grouped_gemm_mxfp4_ws(const void* a, const uint8_t* w, const uint8_t* scales,
+                                       const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M,
+                                       void* y, void* workspace, size_t workspace_bytes, void* stream) {
+  return grouped_gemm_mxfp4_ws(a, w, scales, offsets, counts, E, N, K, M, y, workspace, workspace_bytes, stream);
 }
 
 gnf4_status gnf4_grouped_gemv_nf4(const void* a, const uint8_t* w, const float* absmax, const int32_t* offsets,

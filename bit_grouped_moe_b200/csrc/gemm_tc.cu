@@ -205,7 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nwt = SWI ? ((I / (kBW / 2)) + 1) / 2 : (p.N + 2 * kBW - 1) / (2 * kBW);
   block_exclusive_scan(p.E, s.upre, s.scratch, [&](int q) {
     const int e = s.order[q];
-    return ((s.off[e + 1] - s.off[e] + kBT - 1) / kBT) * nwt;
+    const int r = s.off[e + 1] - s.off[e];
+    return r >= p.min_rows ? ((r + kBT - 1) / kBT) * nwt : 0;
   });
   const int U = s.upre[p.E];
   if (pair >= U) return;  // uniform over the pair

@@ -58,6 +58,7 @@ struct GroupedArgs {
   __nv_bfloat16* y;        // [M, N]
   unsigned* err;           // device error word
   int E, N, K, M;
+  int min_rows = 0;  // tcgen05 GEMM: groups with fewer rows are left to another kernel (rows of y not written)
 };
 
 // gemm_tc.cu
@@ -119,7 +120,14 @@ cudaError_t launch_quant_mxfp4_act(const __nv_bfloat16* x, long long elems, uint
 cudaError_t launch_gemm_mx(int mode, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
                            const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* lo_scales,
                            const uint8_t* w_scales, const int* offsets, const int* counts, __nv_bfloat16* y,
-                           unsigned* err, int E, int N, int K, int M, int grid, cudaStream_t stream);
+                           unsigned* err, int E, int N, int K, int M, int grid, cudaStream_t stream,
+                           int max_rows = 1 << 30);  // groups of more rows are skipped (rows of y not written)
+// The two-term split of the rows of the groups with at most max_rows rows only (other rows not written);
+// offsets / counts as the grouped GEMM.  Persistent grid of num_sms * 8 CTAs.
+cudaError_t launch_quant_mxfp8_split_rows(const __nv_bfloat16* x, int K, const int* offsets, const int* counts,
+                                          int E, int M, int max_rows, unsigned* err, uint8_t* hi_codes,
+                                          uint8_t* hi_scales, uint8_t* lo_codes, uint8_t* lo_scales, int num_sms,
+                                          cudaStream_t stream);
 size_t gemm_mx_smem_bytes(int mode);
 int gemm_mx_rows_per_unit(int mode);
 int gemm_mx_k_per_stage(int mode);

@@ -85,22 +85,17 @@ __device__ __forceinline__ int ilog2_f32(uint32_t b) {
   return (b >> 23) != 0 ? (int)(b >> 23) - 127 : (31 - __clz((int)b)) - 149;
 }
 
-// One thread quantises 8 consecutive k (16 bytes of bf16); the 4 threads of
-// a 32-k block agree on its amax with two shuffles.  TOP = 8: the OCP rule
-// (exponent floor(log2 amax) - 8).  SPLIT: the two-term split with one
-// binade of headroom (exponent floor(log2 amax) - 7 for both terms): hi of
-// x, then lo of the exact residual x - hi.
+// One thread quantises octet o (8 consecutive k, 16 bytes of bf16); the 4
+// lanes of a 32-k block (lanes 4i..4i+3 of the warp, all 32 lanes calling)
+// agree on its amax with two shuffles.  TOP = 8: the OCP rule (exponent
+// floor(log2 amax) - 8).  SPLIT: the two-term split with one binade of
+// headroom (exponent floor(log2 amax) - 7 for both terms): hi of x, then lo
+// of the exact residual x - hi.  ok = false: the lane joins the shuffles only.
 template <bool SPLIT>
-__global__ void __launch_bounds__(kQThreads) quant_mxfp8_kernel(const __nv_bfloat16* __restrict__ x,
-                                                                long long octets, uint8_t* __restrict__ codes,
-                                                                uint8_t* __restrict__ scales,
-                                                                uint8_t* __restrict__ lo_codes,
-                                                                uint8_t* __restrict__ lo_scales) {
+__device__ __forceinline__ void quant_octet(const __nv_bfloat16* __restrict__ x, long long o, bool ok, int lane,
+                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                            uint8_t* __restrict__ lo_codes, uint8_t* __restrict__ lo_scales) {
   constexpr int kTop = SPLIT ? 7 : 8;
-  griddep_launch_dependents();
-  griddep_wait();
-  const long long o = (long long)blockIdx.x * kQThreads + threadIdx.x;
-  const bool ok = o < octets;
   const uint4 v = ok ? ldg_nc_u128(x + o * 8) : make_uint4(0u, 0u, 0u, 0u);
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   // |bf16| compares like its bit pattern with the sign cleared
@@ -131,7 +126,7 @@ __global__ void __launch_bounds__(kQThreads) quant_mxfp8_kernel(const __nv_bfloa
   }
   if (ok) {
     *reinterpret_cast<uint2*>(codes + o * 8) = make_uint2(out[0], out[1]);
-    if ((threadIdx.x & 3) == 0) scales[o >> 2] = (uint8_t)(X + 127);
+    if ((lane & 3) == 0) scales[o >> 2] = (uint8_t)(X + 127);
   }
   if (SPLIT) {
     // residual in the scaled domain: exact in fp32 (x has 8 significant bits,
@@ -165,8 +160,52 @@ __global__ void __launch_bounds__(kQThreads) quant_mxfp8_kernel(const __nv_bfloa
     }
     if (ok) {
       *reinterpret_cast<uint2*>(lo_codes + o * 8) = make_uint2(lo[0], lo[1]);
-      if ((threadIdx.x & 3) == 0) lo_scales[o >> 2] = (uint8_t)(XL + 127);
+      if ((lane & 3) == 0) lo_scales[o >> 2] = (uint8_t)(XL + 127);
     }
+  }
+}
+
+template <bool SPLIT>
+__global__ void __launch_bounds__(kQThreads) quant_mxfp8_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                long long octets, uint8_t* __restrict__ codes,
+                                                                uint8_t* __restrict__ scales,
+                                                                uint8_t* __restrict__ lo_codes,
+                                                                uint8_t* __restrict__ lo_scales) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const long long o = (long long)blockIdx.x * kQThreads + threadIdx.x;
+  quant_octet<SPLIT>(x, o, o < octets, (int)(threadIdx.x & 31), codes, scales, lo_codes, lo_scales);
+}
+
+// The same quantiser over the rows of the groups with at most max_rows rows
+// only (the rows the native two-term GEMM reads when it takes the small
+// groups); other rows are not written.  Persistent grid: one warp per row at
+// a time, the rows of the selected groups enumerated through an exclusive
+// scan of their sizes.
+template <bool SPLIT>
+__global__ void __launch_bounds__(kQThreads) quant_mxfp8_rows_kernel(const __nv_bfloat16* __restrict__ x, int K,
+                                                                     const int* offsets, const int* counts, int E,
+                                                                     int M, int max_rows, unsigned* err,
+                                                                     uint8_t* __restrict__ codes,
+                                                                     uint8_t* __restrict__ scales,
+                                                                     uint8_t* __restrict__ lo_codes,
+                                                                     uint8_t* __restrict__ lo_scales) {
+  __shared__ int off[kMaxExperts + 1], pre[kMaxExperts + 1], scratch[kMaxExperts];
+  griddep_launch_dependents();
+  griddep_wait();
+  if (!load_groups(offsets, counts, E, M, off, scratch, err)) return;
+  block_exclusive_scan(E, pre, scratch, [&](int e) {
+    const int r = off[e + 1] - off[e];
+    return r <= max_rows ? r : 0;
+  });
+  const int R = pre[E];
+  const int lane = threadIdx.x & 31, wpb = kQThreads / 32;
+  const int per_row = K / 8;  // octets; a multiple of 4 (K % 32 == 0), so blocks never straddle rows
+  for (int c = blockIdx.x * wpb + (threadIdx.x >> 5); c < R; c += gridDim.x * wpb) {
+    const int g = find_group(pre, E, c);
+    const long long row = off[g] + (c - pre[g]);
+    for (int b = 0; b < per_row; b += 32)
+      quant_octet<SPLIT>(x, row * per_row + b + lane, b + lane < per_row, lane, codes, scales, lo_codes, lo_scales);
   }
 }
 
@@ -294,6 +333,7 @@ struct MxArgs {
   __nv_bfloat16* y;    // [M, N]
   unsigned* err;
   int E, N, K, M;
+  int max_rows;  // groups with more rows are left to another kernel (their rows of y are not written)
 };
 
 struct Unit {
@@ -400,8 +440,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_wait();
   if (!load_groups(p.offsets, p.counts, p.E, p.M, s.off, s.scratch, err)) return;
   const int nwt = (p.N + kBW - 1) / kBW;
-  block_exclusive_scan(p.E, s.upre, s.scratch,
-                       [&](int e) { return ((s.off[e + 1] - s.off[e] + G::kBT - 1) / G::kBT) * nwt; });
+  block_exclusive_scan(p.E, s.upre, s.scratch, [&](int e) {
+    const int r = s.off[e + 1] - s.off[e];
+    return r <= p.max_rows ? ((r + G::kBT - 1) / G::kBT) * nwt : 0;
+  });
   const int U = s.upre[p.E];
   if ((int)blockIdx.x >= U) return;  // uniform over the block
   const int K = p.K;
@@ -695,6 +737,15 @@ cudaError_t launch_quant_mxfp8(const __nv_bfloat16* x, long long elems, uint8_t*
                     scales, lo_codes, lo_scales);
 }
 
+cudaError_t launch_quant_mxfp8_split_rows(const __nv_bfloat16* x, int K, const int* offsets, const int* counts,
+                                          int E, int M, int max_rows, unsigned* err, uint8_t* hi_codes,
+                                          uint8_t* hi_scales, uint8_t* lo_codes, uint8_t* lo_scales, int num_sms,
+                                          cudaStream_t stream) {
+  const int grid = num_sms * (2048 / kQThreads);
+  return launch_pdl(quant_mxfp8_rows_kernel<true>, dim3((unsigned)grid), dim3(kQThreads), 0, stream, x, K, offsets,
+                    counts, E, M, max_rows, err, hi_codes, hi_scales, lo_codes, lo_scales);
+}
+
 cudaError_t launch_quant_mxfp4_act(const __nv_bfloat16* x, long long elems, uint8_t* blocks, uint8_t* scales,
                                    cudaStream_t stream) {
   const long long octets = elems / 8;
@@ -729,8 +780,9 @@ static cudaError_t launch_gemm_mx_t(const CUtensorMap& tm_a, const CUtensorMap& 
 cudaError_t launch_gemm_mx(int mode, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
                            const CUtensorMap& tm_w_tail, const uint8_t* a_scales, const uint8_t* lo_scales,
                            const uint8_t* w_scales, const int* offsets, const int* counts, __nv_bfloat16* y,
-                           unsigned* err, int E, int N, int K, int M, int grid, cudaStream_t stream) {
-  MxArgs p{a_scales, lo_scales, w_scales, offsets, counts, y, err, E, N, K, M};
+                           unsigned* err, int E, int N, int K, int M, int grid, cudaStream_t stream,
+                           int max_rows) {
+  MxArgs p{a_scales, lo_scales, w_scales, offsets, counts, y, err, E, N, K, M, max_rows};
   if (mode == kW4A4) return launch_gemm_mx_t<kW4A4>(tm_a, tm_a_big, tm_w, tm_w_tail, p, grid, stream);
   if (mode == kSplit) return launch_gemm_mx_t<kSplit>(tm_a, tm_a_big, tm_w, tm_w_tail, p, grid, stream);
   return launch_gemm_mx_t<kW4A8>(tm_a, tm_a_big, tm_w, tm_w_tail, p, grid, stream);

@@ -59,6 +59,11 @@ _lib.gnf4_quantize_mxfp4_act.argtypes = [_P, _I, _I, _P, _P, _P]
 _lib.gnf4_grouped_gemm_w4a4.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_grouped_gemm_w4a8x2.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
+_lib.gnf4_grouped_gemm_mxfp4_workspace_bytes.argtypes = [_I, _I]
+_lib.gnf4_grouped_gemm_mxfp4_workspace_bytes.restype = _SZ
+_lib.gnf4_grouped_gemm_mxfp4_native_max_rows.argtypes = []
+_lib.gnf4_grouped_gemm_mxfp4_native_max_rows.restype = _I
+_lib.gnf4_grouped_gemm_mxfp4_ws.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]
 _lib.gnf4_dequant_nf4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 _lib.gnf4_dequant_mxfp4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", "gnf4_route_topk_permute",
@@ -66,7 +71,7 @@ for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_st
               "gnf4_quantize_mxfp8_split", "gnf4_grouped_gemm_w4a8x2",
               "gnf4_quantize_mxfp4_act", "gnf4_grouped_gemm_w4a4", "gnf4_selftest_bounded_wait",
               "gnf4_grouped_gemv_nf4_combine", "gnf4_grouped_gemv_mxfp4_combine",
-              "gnf4_dequant_nf4_f32", "gnf4_dequant_mxfp4_f32"):
+              "gnf4_dequant_nf4_f32", "gnf4_dequant_mxfp4_f32", "gnf4_grouped_gemm_mxfp4_ws"):
     getattr(_lib, _name).restype = _I
 
 
@@ -171,6 +176,26 @@ def grouped_gemm_nf4(a, w, absmax, y, offsets=None, counts=None, stream=None):
 
 def grouped_gemm_mxfp4(a, w, scales, y, offsets=None, counts=None, stream=None):
     _grouped(_lib.gnf4_grouped_gemm_mxfp4, a, w, scales, y, offsets, counts, stream)
+
+
+def mxfp4_workspace_bytes(M: int, K: int) -> int:
+    """Workspace that lets grouped_gemm_mxfp4_ws run small groups natively (0: the native path does not apply)."""
+    return int(_lib.gnf4_grouped_gemm_mxfp4_workspace_bytes(M, K))
+
+
+def mxfp4_native_max_rows() -> int:
+    """Largest group grouped_gemm_mxfp4_ws runs on the native block-scaled path."""
+    return int(_lib.gnf4_grouped_gemm_mxfp4_native_max_rows())
+
+
+def grouped_gemm_mxfp4_ws(a, w, scales, y, workspace, offsets=None, counts=None, stream=None):
+    """MXFP4 grouped GEMM, small groups on the native two-term path (workspace: a uint8 device tensor of at least
+    mxfp4_workspace_bytes(M, K) bytes, or None for the decode path throughout)."""
+    E, N, K2 = w.shape
+    M = a.shape[0]
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.gnf4_grouped_gemm_mxfp4_ws(_ptr(a), _ptr(w), _ptr(scales), _ptr(offsets), _ptr(counts), E, N, 2 * K2,
+                                           M, _ptr(y), _ptr(workspace), nbytes, _stream(stream)))
 
 
 def grouped_gemv_nf4(a, w, absmax, y, offsets=None, counts=None, stream=None):

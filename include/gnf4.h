@@ -202,6 +202,35 @@ gnf4_status gnf4_grouped_gemm_nf4(const void *a, const uint8_t *w, const float *
 gnf4_status gnf4_grouped_gemm_mxfp4(const void *a, const uint8_t *w, const uint8_t *scales, const int32_t *offsets,
                                     const int32_t *counts, int E, int N, int K, int M, void *y, void *stream);
 
+/* The same MXFP4 grouped GEMM with the native block-scaled path for small
+ * groups (grouped-nf4-gemm releases, v0.2.0 "the MXFP4 native-byte lane";
+ * bw24 v0.9.0, Documentation "prefill arc design": the e2m1 stack read as it
+ * is by a block-scaled MMA).  Same arguments, rules and result tolerance as
+ * gnf4_grouped_gemm_mxfp4, plus a caller-owned device workspace:
+ *   - groups of at most gnf4_grouped_gemm_mxfp4_native_max_rows() (96) rows:
+ *     their activation rows are split into two MXFP8 terms in the workspace
+ *     (the rule of gnf4_quantize_mxfp8_split) and multiplied on tcgen05
+ *     kind::mxf8f6f4 against the stack unchanged, nothing decoded on the SM;
+ *   - larger groups: the decode path of gnf4_grouped_gemm_mxfp4.
+ * On B200 the native path takes about half the time of the decode path per
+ * group of up to 96 rows; a larger group needs one native unit per 96 rows
+ * per weight tile, which the decode path covers with one per 256.
+ *
+ * workspace: NULL (every group takes the decode path, nothing else is
+ * needed), or device memory of at least
+ * gnf4_grouped_gemm_mxfp4_workspace_bytes(M, K) bytes, 16-byte aligned; a
+ * smaller non-NULL workspace is refused with GNF4_ERR_INVALID_ARG.  Its
+ * contents are scratch: written and read within the call's stream order.
+ * When K % 64 != 0 or K < 128 the native path does not apply: the workspace
+ * size is 0 and every group takes the decode path.  With a workspace, w must
+ * be 32-byte aligned.  Up to three launches (split quantiser, native GEMM,
+ * decode GEMM; the last is skipped when M <= 96), no host synchronisation. */
+size_t gnf4_grouped_gemm_mxfp4_workspace_bytes(int M, int K);
+int gnf4_grouped_gemm_mxfp4_native_max_rows(void);
+gnf4_status gnf4_grouped_gemm_mxfp4_ws(const void *a, const uint8_t *w, const uint8_t *scales,
+                                       const int32_t *offsets, const int32_t *counts, int E, int N, int K, int M,
+                                       void *y, void *workspace, size_t workspace_bytes, void *stream);
+
 /* ------------------------------------------------------------------ */
 /* Grouped GEMV (decode: at most 8 rows per group)                     */
 /* ------------------------------------------------------------------ */

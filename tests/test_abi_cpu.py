@@ -50,6 +50,26 @@ def test_route_workspace_size(g):
     assert g.route_workspace_bytes(4, 0, 8) == 0
 
 
+def test_mxfp4_workspace_size(g):
+    """hi and lo e4m3 codes [M, K] plus hi and lo e8m0 scales [M, K/32], each part 16-byte aligned; 0 where the
+    native path does not apply (K % 64 != 0 or K < 128)."""
+    for M, K in [(1, 128), (33, 2880), (32768, 7168), (7, 192)]:
+        sc = (M * (K // 32) + 15) // 16 * 16
+        assert g.mxfp4_workspace_bytes(M, K) == 2 * M * K + 2 * sc
+    for M, K in [(0, 256), (8, 96), (8, 64), (8, 160), (-1, 256)]:
+        assert g.mxfp4_workspace_bytes(M, K) == 0
+    assert g.mxfp4_native_max_rows() == 96
+
+
+def test_mxfp4_ws_refusals(g):
+    f = g._lib.gnf4_grouped_gemm_mxfp4_ws
+    one = ctypes.c_void_p(16)
+    # the shape rules of the MXFP4 GEMM, before any pointer
+    assert f(None, None, None, one, None, 4, 60, 256, 8, None, None, 0, None) == g.ERR_UNSUPPORTED_SHAPE
+    assert f(None, None, None, None, None, 4, 64, 256, 8, None, None, 0, None) == g.ERR_INVALID_ARG
+    assert f(None, None, None, one, None, 4, 64, 256, 0, None, None, 0, None) == 0  # M == 0: nothing to do
+
+
 def _raw(g, name, *args):
     return getattr(g._lib, name)(*args)
 

@@ -1,4 +1,5 @@
-"""Full-size parity of the dgrad and the native block-scaled MXFP4 modes at the
+"""Full-size parity of the dgrad, the native block-scaled MXFP4 modes and the
+MXFP4 GEMM with a workspace (small groups native, large groups decoded) at the
 Kimi-class shapes (384 experts, 4096 tokens top-8 with Zipf(1.2) skew; gate_up
 K=7168 N=4096, down K=2048 N=7168), on sampled rows.
 
@@ -74,7 +75,7 @@ def _own_bound(got, ref, what):
                            + ", ".join(f"{tuple(i)} gpu={got[tuple(i)]:.6g} ref={ref[tuple(i)]:.6g}" for i in bad[:5]))
 
 
-@pytest.mark.parametrize("mode", ["w4a8", "w4a8x2", "w4a4", "dgrad"])
+@pytest.mark.parametrize("mode", ["w4a8", "w4a8x2", "w4a4", "dgrad", "ws"])
 @pytest.mark.parametrize("proj", [0, 1])
 def test_kimi_native_modes_and_dgrad_sampled(g, routing, mode, proj):
     wl, off = routing
@@ -100,6 +101,16 @@ def test_kimi_native_modes_and_dgrad_sampled(g, routing, mode, proj):
     a_d = to_dev_bf16(a)
     y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
     sub_a = np.concatenate([a[int(off[e]):int(off[e + 1])] for e in experts])
+    if mode == "ws":  # small groups native two-term, large groups decode path: the path's own tolerance
+        ws = torch.empty(g.mxfp4_workspace_bytes(M, K), dtype=torch.uint8, device="cuda")
+        g.grouped_gemm_mxfp4_ws(a_d, w_d, sc_d, y, ws, offsets=off_d)
+        torch.cuda.synchronize()
+        assert g.device_errors() == 0
+        sizes = np.diff(off)[experts]
+        assert (sizes <= 96).any() and (sizes > 96).any(), "the sample should hold groups of both paths"
+        ref16 = oracle.grouped_gemm_mxfp4(sub_a, w_small, s_small, sub_off, rows=sub_rows)
+        assert_within_tolerance(bf16_to_f64(y)[rows], ref16, f"kimi mxfp4 ws {p.name}")
+        return
     if mode == "w4a4":
         qa = torch.empty(M, K // 2, dtype=torch.uint8, device="cuda")
         sa = torch.empty(M, K // 32, dtype=torch.uint8, device="cuda")
