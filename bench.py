@@ -230,10 +230,11 @@ class Workload:
                 self.ls1 = torch.empty_like(self.sa1)
                 self.la2 = torch.empty_like(self.qa2)
                 self.ls2 = torch.empty_like(self.sa2)
-        # decode: the second projection's GEMV carries the top-k combine in its epilogue
-        self.fused_combine = fused_combine and self.decode and not dgrad and not w4a8
+        # the second projection's GEMV (decode) or GEMM (prefill, every group decoded) carries the top-k combine
+        self.fused_combine = fused_combine and not dgrad and not self.w4a8
         if self.fused_combine:
-            self.fn2c = f.grouped_gemv_nf4_combine if wl.fmt == "nf4" else f.grouped_gemv_mxfp4_combine
+            self.fn2c = ({"nf4": f.grouped_gemv_nf4_combine, "mxfp4": f.grouped_gemv_mxfp4_combine} if self.decode else
+                         {"nf4": f.grouped_gemm_nf4_combine, "mxfp4": f.grouped_gemm_mxfp4_combine})[wl.fmt]
             self.cnt = torch.zeros(max(f.combine_counters_bytes(self.T, self.p2.N) // 4, 1), dtype=torch.int32,
                                    device=device)
         # optional fused gate_up + SwiGLU first projection: h [M, N1/2] feeds the second
@@ -387,8 +388,9 @@ class Workload:
         # route (one launch for at most 256 pairs, else hist + scan + scatter + gather) + 2 projections + combine
         route = 1 if 0 < self.M <= 256 else 4
         combine = 0 if (self.dgrad or self.fused_combine) else 1
-        # the native MXFP4 call: split quantiser + native GEMM + decode GEMM per projection (M > 96)
-        native = 4 if self.native else 0
+        # the native MXFP4 call: split quantiser + native GEMM + decode GEMM per projection (M > 96); the
+        # fused-combine second projection is one launch
+        native = (2 if self.fused_combine else 4) if self.native else 0
         return route + 2 + combine + (2 if self.w4a8 else 0) + native
 
 
@@ -599,8 +601,8 @@ def main():
     ap.add_argument("--w4a4", action="store_true",
                     help="MXFP4 workloads: native W4A4 mode (MXFP4 activations, kind::mxf4 block-scaled GEMM)")
     ap.add_argument("--fused-combine", action="store_true",
-                    help="decode: run the top-k combine in the second GEMV's epilogue instead of as its own launch "
-                         "(measured slower on B200: the epilogue's round trips extend every unit)")
+                    help="run the top-k combine inside the second projection's launch (decode: the GEMV epilogue; "
+                         "prefill: after each GEMM unit, every group on the decode path) instead of as its own launch")
     ap.add_argument("--no-native", action="store_true",
                     help="MXFP4 prefill: every group on the decode path (gnf4_grouped_gemm_mxfp4 without a workspace)")
     ap.add_argument("--swiglu", action="store_true",
@@ -857,7 +859,9 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
                               {"activations": "two-term MXFP8 hi + lo (quantised every step; bf16-activation accuracy)"}
                               if wl.split else
                               {"activations": "MXFP8 (native W4A8 mode: quantised every step)"} if wl.w4a8 else {}),
-                           **({"combine": "in the second GEMV's epilogue"} if wl.fused_combine else {}),
+                           **({"combine": "in the second GEMV's epilogue" if wl.decode else
+                                          "after each unit of the second GEMM (decode path for every group)"}
+                              if wl.fused_combine else {}),
                            **({"mxfp4_path": "groups <= 96 rows: native two-term MXFP8 x e2m1 (kind::mxf8f6f4, "
                                              "bf16-activation accuracy); larger groups: decode to bf16 (kind::f16)"}
                               if wl.native else {}),

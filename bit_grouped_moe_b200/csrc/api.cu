@@ -206,9 +206,10 @@ gnf4_status check_grouped(int fmt, const void* a, const uint8_t* w, const void* 
 
 // swiglu: w is a gate_up stack [E, N = 2I, K/2] and y the [M, I] output h.
 // min_rows > 0: groups of fewer rows are skipped (their rows of y are left to another kernel).
+// combine: the top-k combine after each unit (all groups, not with swiglu).
 gnf4_status grouped_gemm(int fmt, bool swiglu, const void* a, const uint8_t* w, const void* scales,
                          const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M, void* y,
-                         void* stream, int min_rows = 0) {
+                         void* stream, int min_rows = 0, const CombineArgs* combine = nullptr) {
   GNF4_TRY(check_grouped(fmt, a, w, scales, offsets, counts, E, N, K, M, y));
   if (M == 0) return GNF4_OK;
   DeviceState* d = nullptr;
@@ -233,7 +234,7 @@ gnf4_status grouped_gemm(int fmt, bool swiglu, const void* a, const uint8_t* w, 
   const long long units = chunks * nwt;
   if (units >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d, N=%d give too many work units", M, N);
   const int grid = gemm_tc_grid(units, d->num_sms);
-  cudaError_t e = launch_gemm_tc(fmt, swiglu, tm_a, tm_a_big, tm_w, tm_y, p, grid, as_stream(stream));
+  cudaError_t e = launch_gemm_tc(fmt, swiglu, tm_a, tm_a_big, tm_w, tm_y, p, grid, as_stream(stream), combine);
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMM launch");
   return GNF4_OK;
 }
@@ -289,6 +290,29 @@ gnf4_status grouped_gemv_combine(int fmt, const void* a, const uint8_t* w, const
     return fail(GNF4_ERR_CUDA, "grouped GEMV + combine: the decode table does not fit above the kernel's shared data");
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMV + combine launch");
   return GNF4_OK;
+}
+
+// GEMM with the top-k combine after each unit's epilogue.
+gnf4_status grouped_gemm_combine(int fmt, const void* a, const uint8_t* w, const void* scales,
+                                 const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M, void* y,
+                                 const int32_t* sorted_to_flat, const int32_t* flat_to_sorted, const float* weights,
+                                 int T, int k, void* out, int32_t* counters, void* stream) {
+  if (T < 0 || k < 1) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T=%d / k=%d invalid", T, k);
+  if ((long long)T * k >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T*k too large");
+  GNF4_TRY(check_grouped(fmt, a, w, scales, offsets, counts, E, N, K, M, y));
+  if (T == 0) return GNF4_OK;
+  GNF4_TRY(check_ptr(flat_to_sorted, "flat_to_sorted", 4));
+  GNF4_TRY(check_ptr(weights, "weights", 4));
+  GNF4_TRY(check_ptr(out, "out", 16));
+  if (M == 0) {  // no routed row, so no valid pair: every output row is zero
+    cudaError_t e = cudaMemsetAsync(out, 0, (size_t)T * (size_t)N * 2, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "zeroing out");
+    return GNF4_OK;
+  }
+  GNF4_TRY(check_ptr(sorted_to_flat, "sorted_to_flat", 4));
+  GNF4_TRY(check_ptr(counters, "counters", 4));
+  CombineArgs c{sorted_to_flat, flat_to_sorted, weights, static_cast<__nv_bfloat16*>(out), counters, T, k};
+  return grouped_gemm(fmt, false, a, w, scales, offsets, counts, E, N, K, M, y, stream, 0, &c);
 }
 
 // dY [M, N] bf16 and the [E, N, K/2] stack -> dX [M, K] bf16.
@@ -741,6 +765,24 @@ gnf4_status gnf4_grouped_gemv_mxfp4_combine(const void* a, const uint8_t* w, con
                                             const float* weights, int T, int k, void* out, int32_t* counters,
                                             void* stream) {
   return grouped_gemv_combine(1, a, w, scales, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
+                              weights, T, k, out, counters, stream);
+}
+
+gnf4_status gnf4_grouped_gemm_nf4_combine(const void* a, const uint8_t* w, const float* absmax,
+                                          const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M,
+                                          void* y, const int32_t* sorted_to_flat, const int32_t* flat_to_sorted,
+                                          const float* weights, int T, int k, void* out, int32_t* counters,
+                                          void* stream) {
+  return grouped_gemm_combine(0, a, w, absmax, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
+                              weights, T, k, out, counters, stream);
+}
+
+gnf4_status gnf4_grouped_gemm_mxfp4_combine(const void* a, const uint8_t* w, const uint8_t* scales,
+                                            const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M,
+                                            void* y, const int32_t* sorted_to_flat, const int32_t* flat_to_sorted,
+                                            const float* weights, int T, int k, void* out, int32_t* counters,
+                                            void* stream) {
+  return grouped_gemm_combine(1, a, w, scales, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
                               weights, T, k, out, counters, stream);
 }
 

@@ -45,6 +45,15 @@
 //  * Epilogue: TMEM -> registers -> bf16 tile in shared memory -> one TMA
 //    store per 32 tokens (double-buffered); a ragged last chunk is stored
 //    element by element.
+//  * Fused combine (CMB, the second projection): once a unit's accumulator
+//    is drained and released (the next unit's MMAs already run), its stores
+//    are waited for and published, and each of its rows counts its (token,
+//    128-column tile) in with an atomic; the thread that completes a token's
+//    last valid pair queues it, and the epilogue warps then compute the
+//    queued tokens' 128 output columns with the same fp32 fmaf sequence as
+//    the separate combine (pairs in slot order), reading the rows through L2,
+//    so the fused output equals GEMM + combine bit for bit.  The work
+//    overlaps the next unit's mainloop instead of holding the accumulator.
 //  * Warp roles per CTA (26 warps): 0 and 24 = weight TMA, 1 = TMEM owner
 //    (both CTAs) + MMA issuer (even CTA), 25 = stage poller (even CTA: tests
 //    the stage barriers and publishes a ready count the MMA thread reads with
@@ -106,6 +115,8 @@ struct Smem {
   int upre[kMaxExperts + 1];
   int scratch[kMaxExperts];
   int order[kMaxExperts];  // experts by descending row count (stable)
+  int done[kBT];           // fused combine: tokens this unit's rows completed
+  int ndone;
   uint64_t wfull[kWStages], wempty[kWStages];
   uint64_t afull[kAStages], aempty[kAStages];
   uint64_t tfull[kTStages], tempty[kTStages];  // tfull: even CTA only, one arrival per CTA
@@ -121,6 +132,54 @@ static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
 struct Unit {
   int e, j, row0, rows, n;  // n: MMA N (rows rounded up to 32)
 };
+
+// Fused combine: pairs of token t whose sorted row lies in [0, nvalid).
+__device__ __forceinline__ int cmb_valid_pairs(const CombineArgs& c, int t, int nvalid) {
+  int need = 0;
+  for (int j = 0; j < c.k; ++j) {
+    const int r = __ldg(c.f2s + (size_t)t * c.k + j);
+    need += (r >= 0 && r < nvalid) ? 1 : 0;
+  }
+  return need;
+}
+
+// out[t, n0 .. n0+8) = bf16(sum_j w[t, j] * y[f2s[t*k + j], n0 ..]) over the
+// valid pairs in slot order, fp32 fmaf from 0 (the separate combine's
+// sequence); rows read through L2.  Loads of 8 slots are issued together.
+__device__ __forceinline__ void cmb_token_cols8(const CombineArgs& c, const __nv_bfloat16* y, int N, int t, int n0,
+                                                int nvalid) {
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int j0 = 0; j0 < c.k; j0 += 8) {
+    uint4 yv[8];
+    float wv[8];
+    bool ok[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = j0 + jj;
+      const int r = j < c.k ? __ldg(c.f2s + (size_t)t * c.k + j) : -1;
+      ok[jj] = r >= 0 && r < nvalid;
+      yv[jj] = ok[jj] ? __ldcg(reinterpret_cast<const uint4*>(y + (size_t)r * N + n0)) : make_uint4(0u, 0u, 0u, 0u);
+      wv[jj] = ok[jj] ? __ldg(c.w + (size_t)t * c.k + j) : 0.f;
+    }
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      if (!ok[jj]) continue;
+      const uint32_t qq[4] = {yv[jj].x, yv[jj].y, yv[jj].z, yv[jj].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        acc[2 * h] = fmaf(wv[jj], __uint_as_float(qq[h] << 16), acc[2 * h]);
+        acc[2 * h + 1] = fmaf(wv[jj], __uint_as_float(qq[h] & 0xFFFF0000u), acc[2 * h + 1]);
+      }
+    }
+  }
+  uint32_t o[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * h], acc[2 * h + 1]);
+    o[h] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  *reinterpret_cast<uint4*>(c.out + (size_t)t * N + n0) = make_uint4(o[0], o[1], o[2], o[3]);
+}
 
 // Weight row (within the expert) held by TMEM lane nl of this CTA in pair
 // tile j (cta = 0 or 1).  SwiGLU: single tile jj = 2j + cta takes 64 gate
@@ -170,10 +229,12 @@ __device__ __forceinline__ uint32_t lut_get(uint32_t lut, uint32_t word, uint32_
   return v;
 }
 
-template <int FMT, bool SWI>
+template <int FMT, bool SWI, bool CMB>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_big,
-                   const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_y, GroupedArgs p) {
+                   const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_y, GroupedArgs p,
+                   CombineArgs cmb) {
+  static_assert(!(SWI && CMB), "the combine follows the second projection, not the fused gate_up");
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -209,6 +270,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     return r >= p.min_rows ? ((r + kBT - 1) / kBT) * nwt : 0;
   });
   const int U = s.upre[p.E];
+  if (CMB) {
+    if (tid == 0) s.ndone = 0;
+    if (blockIdx.x == 0) {  // tokens without a valid pair get a zero row (no unit ever completes them)
+      const int nvalid = s.off[p.E];
+      for (int t = tid; t < cmb.T; t += kThreads)
+        if (cmb_valid_pairs(cmb, t, nvalid) == 0)
+          for (int n = 0; n < p.N; n += 8)
+            *reinterpret_cast<uint4*>(cmb.out + (size_t)t * p.N + n) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
   if (pair >= U) return;  // uniform over the pair
   const int nk = (p.K + kBK - 1) / kBK;
 
@@ -582,6 +653,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       // the accumulator's TMEM loads have completed (tcgen05.wait::ld): relaxed
       if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&s.acce), 0));
+      if (CMB) {
+        // The unit's rows of y are published before they are counted: the
+        // TMA stores have completed (not only read their source), the proxy
+        // fence orders them before the issuer's generic accesses, the
+        // barrier before every epilogue thread's, and each counting thread's
+        // fence (cumulative) before its count.
+        if (issuer) {
+          bulk_wait_all();
+          fence_proxy_async_all();
+        }
+        named_bar(kBarEpi, 128);
+        const int et = q * 32 + lane;
+        const int nvalid = s.off[p.E];
+        const int ntile = (p.N + kBW - 1) / kBW;
+        for (int rr = et; rr < x.rows; rr += 128) {
+          const int f = __ldg(cmb.s2f + x.row0 + rr);
+          if (f < 0 || f >= cmb.T * cmb.k) continue;
+          const int t = f / cmb.k;
+          int* ctr = cmb.cnt + (size_t)t * ntile + jj;
+          __threadfence();
+          if (atomicAdd(ctr, 1) == cmb_valid_pairs(cmb, t, nvalid) - 1) {
+            __threadfence();  // the other units' rows of t are visible to this thread from here on
+            *ctr = 0;         // every pair of this tile is in: ready for the next call
+            s.done[atomicAdd(&s.ndone, 1)] = t;
+          }
+        }
+        named_bar(kBarEpi, 128);
+        const int nd = s.ndone;
+        if (nd > 0) __threadfence();  // the completing threads' acquisitions, for every reader
+        // 16 threads per token (8 columns each), 8 tokens at a time
+        for (int o = et; o < nd * 16; o += 128) {
+          const int n0 = col0 + (o & 15) * 8;
+          if (n0 < p.N) cmb_token_cols8(cmb, p.y, p.N, s.done[o >> 4], n0, nvalid);
+        }
+        named_bar(kBarEpi, 128);
+        if (et == 0) s.ndone = 0;
+      }
     }
     if (issuer) bulk_wait_all();  // every store has completed before the CTA ends
   }
@@ -624,23 +732,31 @@ static cudaError_t launch_pair(void (*kernel)(KArgs...), int grid, size_t smem, 
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int FMT, bool SWI>
+template <int FMT, bool SWI, bool CMB>
 cudaError_t launch_gemm_tc_t(const CUtensorMap& tm_a, const CUtensorMap& tm_a_big, const CUtensorMap& tm_w,
-                             const CUtensorMap& tm_y, const GroupedArgs& p, int grid, cudaStream_t stream) {
+                             const CUtensorMap& tm_y, const GroupedArgs& p, const CombineArgs& c, int grid,
+                             cudaStream_t stream) {
   static std::atomic<bool> configured[64];
-  const cudaError_t e = set_smem_limit_once(gemm_tc_kernel<FMT, SWI>, (int)gemm_tc_smem_bytes(), configured);
+  const cudaError_t e = set_smem_limit_once(gemm_tc_kernel<FMT, SWI, CMB>, (int)gemm_tc_smem_bytes(), configured);
   if (e != cudaSuccess) return e;
-  return launch_pair(gemm_tc_kernel<FMT, SWI>, grid, gemm_tc_smem_bytes(), stream, tm_a, tm_a_big, tm_w, tm_y, p);
+  return launch_pair(gemm_tc_kernel<FMT, SWI, CMB>, grid, gemm_tc_smem_bytes(), stream, tm_a, tm_a_big, tm_w, tm_y,
+                     p, c);
 }
 
 cudaError_t launch_gemm_tc(int fmt, bool swiglu, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big,
                            const CUtensorMap& tm_w, const CUtensorMap& tm_y, const GroupedArgs& p, int grid,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, const CombineArgs* combine) {
+  const CombineArgs none{};
+  if (combine != nullptr) {
+    if (swiglu) return cudaErrorInvalidValue;
+    return fmt == 0 ? launch_gemm_tc_t<0, false, true>(tm_a, tm_a_big, tm_w, tm_y, p, *combine, grid, stream)
+                    : launch_gemm_tc_t<1, false, true>(tm_a, tm_a_big, tm_w, tm_y, p, *combine, grid, stream);
+  }
   if (fmt == 0)
-    return swiglu ? launch_gemm_tc_t<0, true>(tm_a, tm_a_big, tm_w, tm_y, p, grid, stream)
-                  : launch_gemm_tc_t<0, false>(tm_a, tm_a_big, tm_w, tm_y, p, grid, stream);
-  return swiglu ? launch_gemm_tc_t<1, true>(tm_a, tm_a_big, tm_w, tm_y, p, grid, stream)
-                : launch_gemm_tc_t<1, false>(tm_a, tm_a_big, tm_w, tm_y, p, grid, stream);
+    return swiglu ? launch_gemm_tc_t<0, true, false>(tm_a, tm_a_big, tm_w, tm_y, p, none, grid, stream)
+                  : launch_gemm_tc_t<0, false, false>(tm_a, tm_a_big, tm_w, tm_y, p, none, grid, stream);
+  return swiglu ? launch_gemm_tc_t<1, true, false>(tm_a, tm_a_big, tm_w, tm_y, p, none, grid, stream)
+                : launch_gemm_tc_t<1, false, false>(tm_a, tm_a_big, tm_w, tm_y, p, none, grid, stream);
 }
 
 int gemm_tc_rows_per_unit() { return kBT; }
@@ -669,8 +785,8 @@ int gemm_tc_grid(long long units, int num_sms) {
     cfg.numAttrs = 1;
     static std::atomic<bool> configured[64];
     int n = 0;
-    if (set_smem_limit_once(gemm_tc_kernel<0, false>, (int)gemm_tc_smem_bytes(), configured) == cudaSuccess &&
-        cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<0, false>, &cfg) == cudaSuccess && n > 0)
+    if (set_smem_limit_once(gemm_tc_kernel<0, false, false>, (int)gemm_tc_smem_bytes(), configured) == cudaSuccess &&
+        cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<0, false, false>, &cfg) == cudaSuccess && n > 0)
       mc = n;
     else
       mc = num_sms / 2;

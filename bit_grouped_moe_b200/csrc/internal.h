@@ -72,17 +72,19 @@ int gemm_tc_small_box_rows();  // activation rows per box for groups of at most 
 int gemm_tc_big_box_rows();    // activation rows per box otherwise (tm_a_big)
 // swiglu: p.w is a gate_up stack [E, N = 2I, K/2] (tm_w its 5-D gate/up view) and p.y the [M, I] output h.
 // tm_y: the output [M, N] (SwiGLU: [M, I]) bf16 in boxes of 128 (SwiGLU: 64) columns x gemm_tc_out_box_rows() rows.
+struct CombineArgs;
+// combine (not with swiglu): also out[t] = sum_j w[t,j] y[f2s[t*k+j]] after each unit (counters per 128 columns).
 cudaError_t launch_gemm_tc(int fmt, bool swiglu, const CUtensorMap& tm_a, const CUtensorMap& tm_a_big,
                            const CUtensorMap& tm_w, const CUtensorMap& tm_y, const GroupedArgs& p, int grid,
-                           cudaStream_t stream);
+                           cudaStream_t stream, const CombineArgs* combine = nullptr);
 
-// Fused top-k combine in the GEMV epilogue (device pointers).
+// Fused top-k combine in the GEMV / GEMM epilogue (device pointers).
 struct CombineArgs {
   const int* s2f;     // sorted_to_flat [M]
   const int* f2s;     // flat_to_sorted [T*k]
   const float* w;     // weights [T, k]
   __nv_bfloat16* out; // [T, N]
-  int* cnt;           // [T, ceil(N/64)] counters, zero before the call and after it
+  int* cnt;           // [T, ceil(N/64)] counters (the GEMM uses [T, ceil(N/128)]), zero before and after a call
   int T, k;
 };
 

@@ -49,7 +49,8 @@ for _name in _GROUPED:
     getattr(_lib, _name).argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.gnf4_combine_counters_bytes.argtypes = [_I, _I]
 _lib.gnf4_combine_counters_bytes.restype = _SZ
-for _name in ("gnf4_grouped_gemv_nf4_combine", "gnf4_grouped_gemv_mxfp4_combine"):
+for _name in ("gnf4_grouped_gemv_nf4_combine", "gnf4_grouped_gemv_mxfp4_combine", "gnf4_grouped_gemm_nf4_combine",
+              "gnf4_grouped_gemm_mxfp4_combine"):
     getattr(_lib, _name).argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P]
 _lib.gnf4_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, _P]
 _lib.gnf4_quantize_mxfp8.argtypes = [_P, _I, _I, _P, _P, _P]
@@ -70,7 +71,8 @@ for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_st
               *_GROUPED, "gnf4_combine", "gnf4_quantize_mxfp8", "gnf4_grouped_gemm_w4a8",
               "gnf4_quantize_mxfp8_split", "gnf4_grouped_gemm_w4a8x2",
               "gnf4_quantize_mxfp4_act", "gnf4_grouped_gemm_w4a4", "gnf4_selftest_bounded_wait",
-              "gnf4_grouped_gemv_nf4_combine", "gnf4_grouped_gemv_mxfp4_combine",
+              "gnf4_grouped_gemv_nf4_combine", "gnf4_grouped_gemv_mxfp4_combine", "gnf4_grouped_gemm_nf4_combine",
+              "gnf4_grouped_gemm_mxfp4_combine",
               "gnf4_dequant_nf4_f32", "gnf4_dequant_mxfp4_f32", "gnf4_grouped_gemm_mxfp4_ws"):
     getattr(_lib, _name).restype = _I
 
@@ -341,6 +343,20 @@ def grouped_gemv_nf4_combine(a, w, absmax, y, sorted_to_flat, flat_to_sorted, we
 def grouped_gemv_mxfp4_combine(a, w, scales, y, sorted_to_flat, flat_to_sorted, weights, out, counters,
                                offsets=None, counts=None, stream=None):
     _gemv_combine(_lib.gnf4_grouped_gemv_mxfp4_combine, a, w, scales, y, sorted_to_flat, flat_to_sorted, weights,
+                  out, counters, offsets, counts, stream)
+
+
+def grouped_gemm_nf4_combine(a, w, absmax, y, sorted_to_flat, flat_to_sorted, weights, out, counters,
+                             offsets=None, counts=None, stream=None):
+    """Grouped GEMM (y) with the top-k combine of y into out [T, N] after each work unit, in the same launch.
+    counters: zeroed int32 device buffer of combine_counters_bytes(T, N) bytes (left zero)."""
+    _gemv_combine(_lib.gnf4_grouped_gemm_nf4_combine, a, w, absmax, y, sorted_to_flat, flat_to_sorted, weights,
+                  out, counters, offsets, counts, stream)
+
+
+def grouped_gemm_mxfp4_combine(a, w, scales, y, sorted_to_flat, flat_to_sorted, weights, out, counters,
+                               offsets=None, counts=None, stream=None):
+    _gemv_combine(_lib.gnf4_grouped_gemm_mxfp4_combine, a, w, scales, y, sorted_to_flat, flat_to_sorted, weights,
                   out, counters, offsets, counts, stream)
 
 

@@ -334,6 +334,28 @@ gnf4_status gnf4_grouped_gemv_mxfp4_combine(const void *a, const uint8_t *w, con
                                             const int32_t *flat_to_sorted, const float *weights, int T, int k,
                                             void *out, int32_t *counters, void *stream);
 
+/* The grouped GEMM of the second projection (prefill: any number of rows
+ * per group) with the same top-k combine after each work unit's epilogue
+ * (grouped-nf4-gemm releases, v0.2.5 "arena -> kernel": moe_layer_forward
+ * runs gate -> GLU -> down, then the weighted unsort).  Results, arguments
+ * and counter rules exactly as gnf4_grouped_gemv_*_combine, with the shape
+ * rules of gnf4_grouped_gemm_*: out equals gnf4_grouped_gemm_* followed by
+ * gnf4_combine bit for bit.  y is still written (the combine reads the
+ * token's other rows from it through L2).  Each unit's combine runs after
+ * its accumulator is released, so it overlaps the next unit's MMAs.  M == 0
+ * zeroes out (no pair is valid).  One launch; every group takes the decode
+ * path (there is no native-path variant of this call). */
+gnf4_status gnf4_grouped_gemm_nf4_combine(const void *a, const uint8_t *w, const float *absmax,
+                                          const int32_t *offsets, const int32_t *counts, int E, int N, int K, int M,
+                                          void *y, const int32_t *sorted_to_flat, const int32_t *flat_to_sorted,
+                                          const float *weights, int T, int k, void *out, int32_t *counters,
+                                          void *stream);
+gnf4_status gnf4_grouped_gemm_mxfp4_combine(const void *a, const uint8_t *w, const uint8_t *scales,
+                                            const int32_t *offsets, const int32_t *counts, int E, int N, int K,
+                                            int M, void *y, const int32_t *sorted_to_flat,
+                                            const int32_t *flat_to_sorted, const float *weights, int T, int k,
+                                            void *out, int32_t *counters, void *stream);
+
 /* ------------------------------------------------------------------ */
 /* Native W4A8 mode: MXFP8 activations x MXFP4 weights                 */
 /* ------------------------------------------------------------------ */
