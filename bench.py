@@ -705,6 +705,10 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
               for _ in range(DOMINANT_REPS)]
     torch.cuda.synchronize()
     d_wall0 = time.time()
+    # a head start for the GPU (torch's spin kernel, ~2.5 ms): every launch of the
+    # loop is queued before it runs, so the event pairs time the device only and
+    # not the host's enqueue of a short kernel
+    torch.cuda._sleep(5_000_000)
     for r, (a, b) in enumerate(dev_ev):
         a.record(stream)
         wl.dominant(r)

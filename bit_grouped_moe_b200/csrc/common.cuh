@@ -549,61 +549,86 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 }
 
 // ---------------------------------------------------------------- groups
+// Warp 0 does the group bookkeeping (E <= kMaxExperts): lane l owns the
+// contiguous run of groups [l*per, l*per + per), per = ceil(E/32), so an
+// exclusive scan is one pass over the run, five shuffles and a second pass.
+// A block-wide Hillis-Steele scan took ~5k cycles for 64 groups (14 block
+// barriers); this takes about one global-load latency.
+
+// Exclusive scan of the lanes' partial sums (warp 0).
+__device__ __forceinline__ int warp_exclusive_sum(int v, int lane, int* total) {
+  int incl = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  *total = __shfl_sync(0xffffffffu, incl, 31);
+  return incl - v;
+}
+
 // Loads the group description into shared memory as row offsets off[0..E]
 // (from `offsets`, or as the exclusive scan of `counts`) and checks it.
 // Returns false (and flags GNF4_DEVERR_BAD_OFFSETS) if it is malformed.  All
 // threads of the block must call it; it ends with __syncthreads().
 __device__ __forceinline__ bool load_groups(const int* offsets, const int* counts, int E, int M, int* off,
                                             int* scratch, unsigned* err) {
+  (void)scratch;
   __shared__ int s_bad;
-  const int tid = threadIdx.x, nt = blockDim.x;
-  if (tid == 0) s_bad = 0;
-  if (offsets != nullptr) {
-    for (int i = tid; i <= E; i += nt) off[i] = offsets[i];
-    __syncthreads();
-  } else {
-    // Hillis-Steele inclusive scan of counts into scratch, then shift.
-    for (int i = tid; i < E; i += nt) scratch[i] = counts[i];
-    __syncthreads();
-    for (int d = 1; d < E; d <<= 1) {
-      int v[kMaxExperts / 128 + 1];
-      int c = 0;
-      for (int i = tid; i < E; i += nt) v[c++] = (i >= d) ? scratch[i - d] : 0;
-      __syncthreads();
-      c = 0;
-      for (int i = tid; i < E; i += nt) scratch[i] += v[c++];
-      __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = (E + 31) >> 5;
+    const int b = min(lane * per, E), e_end = min(b + per, E);
+    bool bad = false;
+    if (offsets != nullptr) {
+      for (int i = lane; i <= E; i += 32) off[i] = offsets[i];
+      __syncwarp();
+      for (int i = b; i < e_end; ++i) bad |= off[i + 1] < off[i];
+    } else {
+      int sum = 0;
+      for (int i = b; i < e_end; ++i) {
+        const int c = __ldg(counts + i);
+        bad |= c < 0;
+        sum += c;
+      }
+      int total = 0;
+      int run = warp_exclusive_sum(sum, lane, &total);
+      for (int i = b; i < e_end; ++i) {
+        off[i] = run;
+        run += __ldg(counts + i);
+      }
+      if (lane == 0) off[E] = total;
+      __syncwarp();
     }
-    for (int i = tid; i <= E; i += nt) off[i] = (i == 0) ? 0 : scratch[i - 1];
-    for (int i = tid; i < E; i += nt)
-      if (counts[i] < 0) s_bad = 1;
-    __syncthreads();
+    if (lane == 0) bad |= off[0] != 0 || off[E] > M;
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) s_bad = bad ? 1 : 0;
   }
-  for (int i = tid; i < E; i += nt)
-    if (off[i + 1] < off[i]) s_bad = 1;
-  if (tid == 0 && (off[0] != 0 || off[E] > M)) s_bad = 1;
   __syncthreads();
   const bool bad = s_bad != 0;
-  if (bad && tid == 0 && blockIdx.x == 0) atomicOr(err, GNF4_DEVERR_BAD_OFFSETS);
+  if (bad && threadIdx.x == 0 && blockIdx.x == 0) atomicOr(err, GNF4_DEVERR_BAD_OFFSETS);
   return !bad;
 }
 
-// Exclusive scan over e of val(e), written to pre[0..E]; all threads call.
+// Exclusive scan over e of val(e), written to pre[0..E]; all threads call
+// (warp 0 computes; val is evaluated twice per e and must be pure).
 template <class F>
 __device__ __forceinline__ void block_exclusive_scan(int E, int* pre, int* scratch, F val) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  for (int i = tid; i < E; i += nt) scratch[i] = val(i);
-  __syncthreads();
-  for (int d = 1; d < E; d <<= 1) {
-    int v[kMaxExperts / 128 + 1];
-    int c = 0;
-    for (int i = tid; i < E; i += nt) v[c++] = (i >= d) ? scratch[i - d] : 0;
-    __syncthreads();
-    c = 0;
-    for (int i = tid; i < E; i += nt) scratch[i] += v[c++];
-    __syncthreads();
+  (void)scratch;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = (E + 31) >> 5;
+    const int b = min(lane * per, E), e_end = min(b + per, E);
+    int sum = 0;
+    for (int i = b; i < e_end; ++i) sum += val(i);
+    int total = 0;
+    int run = warp_exclusive_sum(sum, lane, &total);
+    for (int i = b; i < e_end; ++i) {
+      pre[i] = run;
+      run += val(i);
+    }
+    if (lane == 0) pre[E] = total;
   }
-  for (int i = tid; i <= E; i += nt) pre[i] = (i == 0) ? 0 : scratch[i - 1];
   __syncthreads();
 }
 

@@ -103,14 +103,24 @@ def _check(status: int) -> None:
         raise Gnf4Error(status, last_error())
 
 
+# Pointers and streams go to ctypes as plain ints (every entry point has its
+# argtypes set, so each is passed as a full-width pointer).  Building
+# c_void_p objects and torch.cuda.current_stream() per call cost ~10 us of
+# host time per launch, more than a single-token decode kernel takes.
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
+
+
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+_cur_device = getattr(torch._C, "_cuda_getDevice", None)
 
 
 def _stream(stream):
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None and _cur_device is not None:
+        return _raw_stream(_cur_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def device_errors(clear: bool = True) -> int:

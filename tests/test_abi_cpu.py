@@ -50,6 +50,18 @@ def test_route_workspace_size(g):
     assert g.route_workspace_bytes(4, 0, 8) == 0
 
 
+def test_binding_sets_argtypes_for_every_call(g):
+    """The binding passes pointers as plain ints: each entry point it calls
+    must declare its argument types, or a pointer would be cut to a C int."""
+    import re
+    src = open(g.__file__).read()
+    called = set(re.findall(r"_lib\.(gnf4_\w+)", src)) | set(re.findall(r"\"(gnf4_\w+)\"", src))
+    assert called
+    missing = [n for n in sorted(called) if getattr(g._lib, n).argtypes is None and n not in ("gnf4_last_error",
+                                                                                               "gnf4_version")]
+    assert not missing, missing
+
+
 def test_mxfp4_workspace_size(g):
     """hi and lo e4m3 codes [M, K] plus hi and lo e8m0 scales [M, K/32], each part 16-byte aligned; 0 where the
     native path does not apply (K % 64 != 0 or K < 128)."""
