@@ -101,6 +101,7 @@ constexpr int kWStageBytes = kBW * kBK / 2;            // 4 KB
 static_assert(kACol0 + kTStages * (kBK / 2) <= kTmemCols, "TMEM budget");
 static_assert(kAStages % kDecGroups == 0 && kTStages % kDecGroups == 0 && kWStages % kDecGroups == 0,
               "each ring slot must belong to one decode group");
+static_assert(kAStages == kTStages, "one commit per stage releases the activation and decoded-weight slots");
 constexpr int kOutRows = 32;                           // tokens per epilogue store
 constexpr int kOutBytes = kOutRows * kBW * 2;          // 8 KB: 32 tokens x 128 weight rows, bf16
 constexpr int kBarEpi = 1 + kDecGroups;                // named barrier of the epilogue warps (decode groups: 1..4)
@@ -118,8 +119,9 @@ struct Smem {
   int done[kBT];           // fused combine: tokens this unit's rows completed
   int ndone;
   uint64_t wfull[kWStages], wempty[kWStages];
-  uint64_t afull[kAStages], aempty[kAStages];
-  uint64_t tfull[kTStages], tempty[kTStages];  // tfull: even CTA only, one arrival per CTA
+  uint64_t afull[kAStages];
+  uint64_t sdone[kAStages];  // a stage's MMAs completed: frees its activation slot and its decoded-weight slot
+  uint64_t tfull[kTStages];  // even CTA only, one arrival per CTA
   uint64_t sfull[kSStages], sempty[kSStages];
   uint64_t accf, acce;  // acce: even CTA only, 8 arrivals (both CTAs' epilogue warps)
   uint64_t mdone;       // abort path only: every issued MMA has retired
@@ -291,12 +293,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kAStages; ++i) {
       mbar_init(&s.afull[i], 1);
-      mbar_init(&s.aempty[i], 1);
+      mbar_init(&s.sdone[i], 1);
     }
-    for (int i = 0; i < kTStages; ++i) {
-      mbar_init(&s.tfull[i], 2);
-      mbar_init(&s.tempty[i], 1);
-    }
+    for (int i = 0; i < kTStages; ++i) mbar_init(&s.tfull[i], 2);
     for (int i = 0; i < kSStages; ++i) {
       mbar_init(&s.sfull[i], 32);
       mbar_init(&s.sempty[i], 4 * kDecGroups);
@@ -370,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nb = big ? (h + kBigBox - 1) / kBigBox : 1;
         for (int kt = 0; kt < nk; ++kt, ++it) {
           const int st = it % kAStages, use = it / kAStages;
-          if (it >= kAStages && !(ok = mbar_wait_cl(&s.aempty[st], (use - 1) & 1, err, abort))) break;
+          if (it >= kAStages && !(ok = mbar_wait_cl(&s.sdone[st], (use - 1) & 1, err, abort))) break;
           if (big) {
             mbar_arrive_expect_tx(&s.afull[st], nb * kBigBox * 128);
             for (int b = 0; b < nb; ++b)
@@ -441,31 +440,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           // ~220 cycles behind the decode warps' table lookups (measured), long
           // enough to let the tensor pipe run dry if paid every stage; the
           // poller runs several stages ahead, so one read covers several.
-          if ((int)ready <= it) ready = ld_acquire_shared(&s.tready);
+          // One fence after each fresh read orders the MMAs of every stage
+          // that read covers after the decode warps' TMEM stores (measured in
+          // isolation: a fence and an acquire per stage add ~110 cycles to the
+          // ~200 of four small-N pair MMAs).
           if ((int)ready <= it) {
-            const long long t0 = clock64();
-            while ((int)(ready = ld_acquire_shared(&s.tready)) <= it) {
-              if (*abort) {
-                ok = false;
-                break;
+            ready = ld_acquire_shared(&s.tready);
+            if ((int)ready <= it) {
+              const long long t0 = clock64();
+              while ((int)(ready = ld_acquire_shared(&s.tready)) <= it) {
+                if (*abort) {
+                  ok = false;
+                  break;
+                }
+                if (clock64() - t0 > kSpinLimitCycles) {
+                  atomicOr(err, GNF4_DEVERR_TIMEOUT);
+                  *abort = 1;
+                  ok = false;
+                  break;
+                }
               }
-              if (clock64() - t0 > kSpinLimitCycles) {
-                atomicOr(err, GNF4_DEVERR_TIMEOUT);
-                *abort = 1;
-                ok = false;
-                break;
-              }
+              if (!ok) break;
             }
-            if (!ok) break;
+            tc_fence_after();
           }
-          tc_fence_after();
           const uint32_t a_col = tmem + (uint32_t)(kACol0 + sT * (kBK / 2));
           const uint32_t b_addr = smem_u32(s.act[sa]);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
             tc_mma_ts_pair(tmem, a_col + kk * 8, sdesc_k_sw128(b_addr + kk * 32), idesc, (kt | kk) != 0);
-          tc_commit_pair(&s.aempty[sa]);
-          tc_commit_pair(&s.tempty[sT]);
+          tc_commit_pair(&s.sdone[sa]);  // sa == sT: one commit frees both slots
         }
         if (!ok) break;
         tc_commit_pair(&s.accf);
@@ -509,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it % kDecGroups == grp) {
           const int sw = it % kWStages, sT = it % kTStages, sa = it % kAStages;
           if (live) live = mbar_wait(&s.wfull[sw], (it / kWStages) & 1, err, abort);
-          if (live && it >= kTStages) live = mbar_wait_cl(&s.tempty[sT], ((it / kTStages) - 1) & 1, err, abort);
+          if (live && it >= kTStages) live = mbar_wait_cl(&s.sdone[sT], ((it / kTStages) - 1) & 1, err, abort);
           live = __all_sync(0xffffffffu, live);
           if (live) {
             uint32_t sc0, sc1;
