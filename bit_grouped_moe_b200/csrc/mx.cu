@@ -179,9 +179,9 @@ __global__ void __launch_bounds__(kQThreads) quant_mxfp8_kernel(const __nv_bfloa
 
 // The same quantiser over the rows of the groups with at most max_rows rows
 // only (the rows the native two-term GEMM reads when it takes the small
-// groups); other rows are not written.  Persistent grid: one warp per row at
-// a time, the rows of the selected groups enumerated through an exclusive
-// scan of their sizes.
+// groups); other rows are not written.  Persistent grid: one warp per
+// 32-octet chunk of a row at a time, the rows of the selected groups
+// enumerated through an exclusive scan of their sizes.
 template <bool SPLIT>
 __global__ void __launch_bounds__(kQThreads) quant_mxfp8_rows_kernel(const __nv_bfloat16* __restrict__ x, int K,
                                                                      const int* offsets, const int* counts, int E,
@@ -201,11 +201,15 @@ __global__ void __launch_bounds__(kQThreads) quant_mxfp8_rows_kernel(const __nv_
   const int R = pre[E];
   const int lane = threadIdx.x & 31, wpb = kQThreads / 32;
   const int per_row = K / 8;  // octets; a multiple of 4 (K % 32 == 0), so blocks never straddle rows
-  for (int c = blockIdx.x * wpb + (threadIdx.x >> 5); c < R; c += gridDim.x * wpb) {
-    const int g = find_group(pre, E, c);
-    const long long row = off[g] + (c - pre[g]);
-    for (int b = 0; b < per_row; b += 32)
-      quant_octet<SPLIT>(x, row * per_row + b + lane, b + lane < per_row, lane, codes, scales, lo_codes, lo_scales);
+  const int cpr = (per_row + 31) / 32;  // 32-octet chunks per row
+  // one warp per (row, chunk): a row is spread over warps, so no warp walks
+  // a long row's chunks one load latency after another
+  const long long items = (long long)R * cpr;
+  for (long long c = (long long)blockIdx.x * wpb + (threadIdx.x >> 5); c < items; c += (long long)gridDim.x * wpb) {
+    const int rr = (int)(c / cpr), b = (int)(c - (long long)rr * cpr) * 32;
+    const int g = find_group(pre, E, rr);
+    const long long row = off[g] + (rr - pre[g]);
+    quant_octet<SPLIT>(x, row * per_row + b + lane, b + lane < per_row, lane, codes, scales, lo_codes, lo_scales);
   }
 }
 
