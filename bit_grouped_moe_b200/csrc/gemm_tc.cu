@@ -626,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int i = 2 * m + (up_lane ? 1 : 0);
             // low lane: gate = keep (row 2m), up = got; high lane: up = keep (row 2m+1), gate = got
             const float g = up_lane ? got : keep, uu = up_lane ? keep : got;
-            const __nv_bfloat16 hv = __float2bfloat16_rn(silu_mul(g, uu));
+            const __nv_bfloat16 hv = __float2bfloat16_rn(silu_mul_tanh(g, uu));
             if (staged)
               reinterpret_cast<__nv_bfloat16*>(st)[i * kCols + cl] = hv;
             else if (i < lim && col < I)
