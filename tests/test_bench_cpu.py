@@ -1,0 +1,53 @@
+"""The bench's roofline arithmetic on CPU: the reported fraction is the
+combined bound max(F / tensor peak, B / HBM peak) over the measured time,
+with the sustained tensor peak when the kernel's own loop ran power-capped,
+and the native MXFP4 path's quantised activations counted in B."""
+import types
+
+import pytest
+
+import bench
+
+PEAKS = {"bf16_tflops": 1656.8, "bf16_tflops_sustained": 1388.7, "hbm_gbs": 6520.2}
+
+
+def _wl(native=False, M=32768, N=4096, K=7168, native_rows=1413):
+    p = types.SimpleNamespace(N=N, K=K, name="gate_up")
+    wl = types.SimpleNamespace(p1=p, M=M, dgrad=False, w4a8=False, a4=False, split=False, swiglu=False, decode=False,
+                               native=native, native_rows=[native_rows], wl=types.SimpleNamespace(fmt="mxfp4"))
+    wl.weight_bytes = lambda pp, hit: int(hit * pp.N * (pp.K // 2 + pp.K / 32))
+    return wl
+
+
+def _stats(capped):
+    return {"clocks": {"sm_mhz": 1792.0 if capped else 1965.0, "sm_max_mhz": 1965.0,
+                       "reasons": ["sw_power_cap"] if capped else []}}
+
+
+@pytest.mark.parametrize("capped", [False, True])
+@pytest.mark.parametrize("native", [False, True])
+def test_roofline_is_the_combined_bound(capped, native):
+    wl = _wl(native=native)
+    M, N, K, hit, ms = wl.M, wl.p1.N, wl.p1.K, 133, 2.36
+    r = bench.roofline(wl, None, PEAKS, "measured", ms, hit, _stats(capped), None)
+    F = 2.0 * M * N * K
+    B = hit * N * (K // 2 + K / 32) + 2 * M * K + 2 * M * N + (4 * 1413 * (K + K // 32) if native else 0)
+    peak = PEAKS["bf16_tflops_sustained" if capped else "bf16_tflops"]
+    t = ms / 1e3
+    assert r["algorithmic_flops_per_launch"] == int(F)
+    assert r["algorithmic_bytes_per_launch"] == int(B)
+    assert r["frac"] == pytest.approx(max(F / (peak * 1e12), B / (PEAKS["hbm_gbs"] * 1e9)) / t, abs=1e-4)
+    assert r["tensor"]["peak_measured"] == pytest.approx(peak, abs=0.05)
+    assert r["bound"] == "tensor"  # this shape sits on the tensor side of the ridge
+    nominal = max(F / (bench.NOMINAL["bf16"] * 1e12), B / (bench.NOMINAL["hbm_gbs"] * 1e9)) / t
+    assert r["frac_nominal"] == pytest.approx(nominal, abs=1e-4)
+    assert r["combined_bound_us"] == pytest.approx(max(F / (peak * 1e12), B / (PEAKS["hbm_gbs"] * 1e9)) * 1e6,
+                                                   abs=1e-2)
+
+
+def test_roofline_small_groups_are_hbm_bound():
+    wl = _wl(M=2048, N=5760, K=2880, native_rows=2048, native=True)
+    r = bench.roofline(wl, None, PEAKS, "measured", 0.423, 128, _stats(False), None)
+    assert r["bound"] == "hbm"
+    assert r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(r["algorithmic_bytes_per_launch"] / 0.423e-3 / 1e9, rel=1e-3)
