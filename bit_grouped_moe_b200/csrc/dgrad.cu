@@ -18,8 +18,10 @@
 // e, chunk of <= 128 of its rows, 128-wide k tile); a persistent grid strides
 // over the units.  Warp roles: four decode groups of 4 warps that take the
 // stages in turn (one group's waits, proxy fence and barrier overlap the
-// others' decode), a dY producer, a weight producer, an MMA issuer and 4
-// epilogue warps.
+// others' decode), a dY producer, a weight producer, an MMA issuer, 4
+// epilogue warps and a stage poller (it tests the dY and decoded-tile
+// barriers and publishes a count of complete stages that the MMA thread
+// reads with a load-acquire).
 //
 // Every stage waits on memory twice, for the packed weights and block scales
 // (mostly DRAM: the stacks are larger than L2) and for the dY tile (mostly L2:
@@ -49,7 +51,8 @@ constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kDecGroups = 4;                   // groups take stages in turn
 constexpr int kProdWarp = kDecGroups * kDecWarps, kWProdWarp = kProdWarp + 1, kMmaWarp = kProdWarp + 2;
 constexpr int kEpiWarp0 = kProdWarp + 3;
-constexpr int kThreads = (kEpiWarp0 + 4) * 32;  // 736
+constexpr int kPollWarp = kEpiWarp0 + 4;        // tests the stage barriers for the MMA thread
+constexpr int kThreads = (kPollWarp + 1) * 32;  // 768
 constexpr int kRing = 4;                       // dY stages in flight
 constexpr int kWRing = 8;                      // packed-weight stages in flight
 constexpr int kSQ = 4;                         // stages of block scales queued in registers
@@ -79,6 +82,7 @@ struct DSmem {
   int scratch[kMaxExperts];
   uint64_t full[kRing], mdone[kRing], wfull[kWRing], wempty[kWRing], decoded[kTBuf], accf[2], acce[2], drain;
   uint32_t tmem_base;
+  uint32_t sready;  // stages whose dY tile and decoded tile are complete (the poller counts, the MMA thread reads)
   int abort;
 };
 
@@ -179,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&s.drain, 1);
     s.abort = 0;
+    s.sready = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_y);
     prefetch_tmap(&tm_w);
@@ -249,6 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_m128((uint32_t)kBKt) | (1u << 16);  // B (the decoded W tile) MN-major
       int g = 0, uc = 0;
+      uint32_t ready = 0;  // stages the poller had counted complete at the last read
       bool ok = true;
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ++uc) {
         const int ab = uc & 1;
@@ -257,9 +263,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem + (uint32_t)(ab * kBKt);
         for (int sb = 0; sb < ns; ++sb, ++g) {
           const int b = g % kRing, tb = g % kTBuf;
-          if (!(ok = mbar_wait(&s.full[b], (uint32_t)(g / kRing) & 1u, err, abort))) break;
-          if (!(ok = mbar_wait(&s.decoded[tb], (uint32_t)(g / kTBuf) & 1u, err, abort))) break;
-          tc_fence_after();
+          // The poller warp tests the dY and decoded-tile barriers and counts
+          // the complete stages; this thread re-reads the count only when it
+          // has used up the last one it read (an mbarrier test here costs
+          // ~220 cycles while MMAs are in flight, measured in the forward
+          // GEMM), and one fence after each fresh read covers every stage it
+          // counted.
+          if ((int)ready <= g) {
+            ready = ld_acquire_shared(&s.sready);
+            if ((int)ready <= g) {
+              const long long t0 = clock64();
+              while ((int)(ready = ld_acquire_shared(&s.sready)) <= g) {
+                if (*abort) {
+                  ok = false;
+                  break;
+                }
+                if (clock64() - t0 > kSpinLimitCycles) {
+                  atomicOr(err, GNF4_DEVERR_TIMEOUT);
+                  *abort = 1;
+                  ok = false;
+                  break;
+                }
+              }
+              if (!ok) break;
+            }
+            tc_fence_after();
+          }
           const uint32_t ya = smem_u32(s.y[b]), ta = smem_u32(s.t[tb]);
 #pragma unroll
           for (int q = 0; q < kBN / 16; ++q)
@@ -274,6 +303,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(&s.drain);
         mbar_drain(&s.drain, 0);
       }
+    }
+  } else if (warp == kPollWarp) {
+    // ------------------------------------------------------------ stage poller
+    if (lane == 0) {
+      int g = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < U && ok; u += gridDim.x)
+        for (int sb = 0; sb < ns; ++sb, ++g) {
+          if (!(ok = mbar_wait(&s.full[g % kRing], (uint32_t)(g / kRing) & 1u, err, abort))) break;
+          if (!(ok = mbar_wait(&s.decoded[g % kTBuf], (uint32_t)(g / kTBuf) & 1u, err, abort))) break;
+          st_release_shared(&s.sready, (uint32_t)(g + 1));
+        }
     }
   } else if (warp < kProdWarp) {
     // ------------------------------------------------------------ decode
