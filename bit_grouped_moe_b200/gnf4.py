@@ -190,14 +190,18 @@ def grouped_gemm_mxfp4(a, w, scales, y, offsets=None, counts=None, stream=None):
     _grouped(_lib.gnf4_grouped_gemm_mxfp4, a, w, scales, y, offsets, counts, stream)
 
 
-def mxfp4_workspace_bytes(M: int, K: int) -> int:
+def grouped_gemm_mxfp4_workspace_bytes(M: int, K: int) -> int:
     """Workspace that lets grouped_gemm_mxfp4_ws run small groups natively (0: the native path does not apply)."""
     return int(_lib.gnf4_grouped_gemm_mxfp4_workspace_bytes(M, K))
 
 
-def mxfp4_native_max_rows() -> int:
+def grouped_gemm_mxfp4_native_max_rows() -> int:
     """Largest group grouped_gemm_mxfp4_ws runs on the native block-scaled path."""
     return int(_lib.gnf4_grouped_gemm_mxfp4_native_max_rows())
+
+
+mxfp4_workspace_bytes = grouped_gemm_mxfp4_workspace_bytes
+mxfp4_native_max_rows = grouped_gemm_mxfp4_native_max_rows
 
 
 def grouped_gemm_mxfp4_ws(a, w, scales, y, workspace, offsets=None, counts=None, stream=None):

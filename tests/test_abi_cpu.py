@@ -62,6 +62,16 @@ def test_binding_sets_argtypes_for_every_call(g):
     assert not missing, missing
 
 
+def test_every_entry_point_has_a_same_name_binding(g):
+    """The binding exposes each C entry point under its name without the gnf4_ prefix."""
+    import re
+    hdr = open(g.HEADER_PATH).read()
+    names = sorted(set(re.findall(r"\b(gnf4_\w+)\s*\(", hdr)))
+    assert len(names) > 20
+    missing = [n for n in names if not hasattr(g, n[len("gnf4_"):])]
+    assert not missing, missing
+
+
 def test_mxfp4_workspace_size(g):
     """hi and lo e4m3 codes [M, K] plus hi and lo e8m0 scales [M, K/32], each part 16-byte aligned; 0 where the
     native path does not apply (K % 64 != 0 or K < 128)."""
