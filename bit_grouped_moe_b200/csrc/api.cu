@@ -236,6 +236,7 @@ gnf4_status grouped_gemm(int fmt, bool swiglu, const void* a, const uint8_t* w, 
   const int grid = gemm_tc_grid(units, d->num_sms);
   cudaError_t e = launch_gemm_tc(fmt, swiglu, tm_a, tm_a_big, tm_w, tm_y, p, grid, as_stream(stream), combine);
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMM launch");
+  note_launch(kPathDecode);
   return GNF4_OK;
 }
 
@@ -256,6 +257,7 @@ gnf4_status grouped_gemv(int fmt, bool swiglu, const void* a, const uint8_t* w, 
   if (e == cudaErrorInvalidConfiguration)
     return fail(GNF4_ERR_CUDA, "grouped GEMV: the decode table does not fit above the kernel's shared data");
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMV launch");
+  note_launch(kPathGemv);
   return GNF4_OK;
 }
 
@@ -289,6 +291,7 @@ gnf4_status grouped_gemv_combine(int fmt, const void* a, const uint8_t* w, const
   if (e == cudaErrorInvalidConfiguration)
     return fail(GNF4_ERR_CUDA, "grouped GEMV + combine: the decode table does not fit above the kernel's shared data");
   if (e != cudaSuccess) return cuda_fail(e, "grouped GEMV + combine launch");
+  note_launch(kPathGemv);
   return GNF4_OK;
 }
 
@@ -307,6 +310,7 @@ gnf4_status grouped_gemm_combine(int fmt, const void* a, const uint8_t* w, const
   if (M == 0) {  // no routed row, so no valid pair: every output row is zero
     cudaError_t e = cudaMemsetAsync(out, 0, (size_t)T * (size_t)N * 2, as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(e, "zeroing out");
+    note_launch(kPathOther);
     return GNF4_OK;
   }
   GNF4_TRY(check_ptr(sorted_to_flat, "sorted_to_flat", 4));
@@ -333,6 +337,7 @@ gnf4_status grouped_dgrad(int fmt, const void* dy, const uint8_t* w, const void*
   const int grid = (int)(units < d->num_sms ? units : d->num_sms);
   cudaError_t e = launch_dgrad_tc(fmt, tm_y, tm_w, p, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "grouped dgrad launch");
+  note_launch(kPathDecode);
   return GNF4_OK;
 }
 
@@ -418,6 +423,7 @@ gnf4_status grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, c
                                  static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M, grid, as_stream(stream),
                                  max_rows);
   if (e != cudaSuccess) return cuda_fail(e, "W4A8 grouped GEMM launch");
+  note_launch(kPathNative);
   return GNF4_OK;
 }
 
@@ -476,6 +482,7 @@ gnf4_status grouped_gemm_w4a4(const uint8_t* a_blocks, const uint8_t* a_scales, 
   cudaError_t e = launch_gemm_mx(2, tm_a, tm_a_big, tm_w, tm_w, a_scales, nullptr, w_scales, offsets, counts,
                                  static_cast<__nv_bfloat16*>(y), d->err, E, N, K, M, grid, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "W4A4 grouped GEMM launch");
+  note_launch(kPathNative);
   return GNF4_OK;
 }
 
@@ -517,6 +524,7 @@ gnf4_status grouped_gemm_mxfp4_ws(const void* a, const uint8_t* w, const uint8_t
                                                 d->err, ws + L.hi, ws + L.hi_scales, ws + L.lo, ws + L.lo_scales,
                                                 d->num_sms, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "MXFP8 split quantiser (small groups) launch");
+  note_launch(kPathOther);
   GNF4_TRY(grouped_gemm_w4a8(ws + L.hi, ws + L.hi_scales, ws + L.lo, ws + L.lo_scales, w, scales, offsets, counts, E,
                              N, K, M, y, stream, thr));
   if (M > thr)  // some group may hold more rows
@@ -531,9 +539,63 @@ gnf4_status check_swiglu_width(int I) {
   return GNF4_OK;
 }
 
+// Fused gate_up + SwiGLU: the [E, 2I, K/2] gate_up stack -> h [M, I].
+gnf4_status grouped_swiglu(bool gemv, int fmt, const void* a, const uint8_t* w_gate_up, const void* scales,
+                           const int32_t* offsets, const int32_t* counts, int E, int I, int K, int M, void* h,
+                           void* stream) {
+  GNF4_TRY(check_swiglu_width(I));
+  return gemv ? grouped_gemv(fmt, true, a, w_gate_up, scales, offsets, counts, E, 2 * I, K, M, h, stream)
+              : grouped_gemm(fmt, true, a, w_gate_up, scales, offsets, counts, E, 2 * I, K, M, h, stream);
+}
+
 }  // namespace
 
 void set_last_error(const char* msg) { snprintf(t_last_error, sizeof(t_last_error), "%s", msg); }
+
+// ------------------------------------------------------------- engagement
+namespace {
+
+struct EntryCounters {
+  std::atomic<uint64_t> calls{0}, refused{0}, engaged{0}, rows{0}, decode{0}, native{0}, gemv{0};
+};
+
+constexpr int kEntries = static_cast<int>(Entry::count);
+EntryCounters g_counters[kEntries];
+const char* const kEntryNames[kEntries] = {
+#define GNF4_ENTRY_NAME(n) "gnf4_" #n,
+    GNF4_COUNTED_ENTRIES(GNF4_ENTRY_NAME)
+#undef GNF4_ENTRY_NAME
+};
+
+thread_local int t_call_depth = 0;
+thread_local unsigned t_call_paths = 0;  // families the current outermost call enqueued
+
+void add(std::atomic<uint64_t>& c, uint64_t v) { c.fetch_add(v, std::memory_order_relaxed); }
+
+}  // namespace
+
+CallScope::CallScope(Entry e, long long rows) : entry_(e), rows_(rows), outer_(t_call_depth++ == 0) {
+  if (outer_) t_call_paths = 0;
+}
+
+CallScope::~CallScope() { --t_call_depth; }
+
+gnf4_status CallScope::operator()(gnf4_status s) {
+  if (!outer_) return s;
+  EntryCounters& c = g_counters[static_cast<int>(entry_)];
+  add(c.calls, 1);
+  if (s != GNF4_OK) add(c.refused, 1);
+  if (t_call_paths != 0) {
+    add(c.engaged, 1);
+    add(c.rows, rows_ > 0 ? (uint64_t)rows_ : 0);
+    if (t_call_paths & kPathDecode) add(c.decode, 1);
+    if (t_call_paths & kPathNative) add(c.native, 1);
+    if (t_call_paths & kPathGemv) add(c.gemv, 1);
+  }
+  return s;
+}
+
+void note_launch(unsigned path) { t_call_paths |= path; }
 
 }  // namespace gnf4
 
@@ -544,6 +606,34 @@ extern "C" {
 const char* gnf4_last_error(void) { return t_last_error; }
 
 const char* gnf4_version(void) { return "libgnf4 0.1.0 (sm_100a)"; }
+
+gnf4_status gnf4_call_stats_get(const char* entry, gnf4_call_stats* out, int reset) {
+  if (out == nullptr) return fail(GNF4_ERR_INVALID_ARG, "out is NULL");
+  int first = 0, last = kEntries;
+  if (entry != nullptr) {
+    while (first < kEntries && strcmp(kEntryNames[first], entry) != 0) ++first;
+    if (first == kEntries) return fail(GNF4_ERR_INVALID_ARG, "'%s' is not a counted entry point", entry);
+    last = first + 1;
+  }
+  gnf4_call_stats sum = {};
+  for (int i = first; i < last; ++i) {
+    EntryCounters& c = g_counters[i];
+    auto take = [reset](std::atomic<uint64_t>& v) {
+      return reset ? v.exchange(0, std::memory_order_relaxed) : v.load(std::memory_order_relaxed);
+    };
+    sum.calls += take(c.calls);
+    sum.refused += take(c.refused);
+    sum.engaged += take(c.engaged);
+    sum.rows += take(c.rows);
+    sum.decode_path += take(c.decode);
+    sum.native_path += take(c.native);
+    sum.gemv_path += take(c.gemv);
+  }
+  *out = sum;
+  return GNF4_OK;
+}
+
+const char* gnf4_call_stats_name(int i) { return i >= 0 && i < kEntries ? kEntryNames[i] : nullptr; }
 
 gnf4_status gnf4_device_errors(uint32_t* flags, int clear) {
   if (flags == nullptr) return fail(GNF4_ERR_INVALID_ARG, "flags is NULL");
@@ -576,9 +666,10 @@ size_t gnf4_route_workspace_bytes(int T, int k, int E) {
   return route_workspace_bytes(T, k, E);
 }
 
-gnf4_status gnf4_route_permute(const int32_t* topk_ids, const void* x, int T, int k, int E, int K,
-                               int32_t* offsets, int32_t* sorted_to_flat, int32_t* flat_to_sorted, void* x_sorted,
-                               void* workspace, size_t workspace_bytes, int32_t* bad_id_count, void* stream) {
+static gnf4_status route_permute_impl(const int32_t* topk_ids, const void* x, int T, int k, int E, int K,
+                                      int32_t* offsets, int32_t* sorted_to_flat, int32_t* flat_to_sorted,
+                                      void* x_sorted, void* workspace, size_t workspace_bytes, int32_t* bad_id_count,
+                                      void* stream) {
   if (T < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T=%d is negative", T);
   if (E < 1 || E > 4096) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "E=%d outside [1, 4096]", E);
   if (k < 1 || k > E) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, E=%d]", k, E);
@@ -606,13 +697,23 @@ gnf4_status gnf4_route_permute(const int32_t* topk_ids, const void* x, int T, in
                                sorted_to_flat, flat_to_sorted, static_cast<__nv_bfloat16*>(x_sorted), workspace,
                                bad_id_count, d->num_sms, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "route_permute launch");
+  note_launch(kPathOther);
   return GNF4_OK;
 }
 
-gnf4_status gnf4_route_topk_permute(const float* logits, const float* bias, int T, int E, int k, const void* x, int K,
-                                    int32_t* topk_ids, float* topk_weights, int32_t* offsets,
-                                    int32_t* sorted_to_flat, int32_t* flat_to_sorted, void* x_sorted,
-                                    void* workspace, size_t workspace_bytes, void* stream) {
+gnf4_status gnf4_route_permute(const int32_t* topk_ids, const void* x, int T, int k, int E, int K,
+                               int32_t* offsets, int32_t* sorted_to_flat, int32_t* flat_to_sorted, void* x_sorted,
+                               void* workspace, size_t workspace_bytes, int32_t* bad_id_count, void* stream) {
+  CallScope call(Entry::route_permute, (long long)T * k);
+  return call(route_permute_impl(topk_ids, x, T, k, E, K, offsets, sorted_to_flat, flat_to_sorted, x_sorted, workspace,
+                                 workspace_bytes, bad_id_count, stream));
+}
+
+static gnf4_status route_topk_permute_impl(const float* logits, const float* bias, int T, int E, int k,
+                                           const void* x, int K, int32_t* topk_ids, float* topk_weights,
+                                           int32_t* offsets,
+                                           int32_t* sorted_to_flat, int32_t* flat_to_sorted, void* x_sorted,
+                                           void* workspace, size_t workspace_bytes, void* stream) {
   if (T < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T=%d is negative", T);
   if (E < 1 || E > 4096) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "E=%d outside [1, 4096]", E);
   if (k < 1 || k > E || k > kMaxRouterTopK)
@@ -644,17 +745,29 @@ gnf4_status gnf4_route_topk_permute(const float* logits, const float* bias, int 
                                     static_cast<__nv_bfloat16*>(x_sorted), workspace, d->num_sms,
                                     as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "route_topk_permute launch");
+  note_launch(kPathOther);
   return GNF4_OK;
+}
+
+gnf4_status gnf4_route_topk_permute(const float* logits, const float* bias, int T, int E, int k, const void* x, int K,
+                                    int32_t* topk_ids, float* topk_weights, int32_t* offsets,
+                                    int32_t* sorted_to_flat, int32_t* flat_to_sorted, void* x_sorted,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  CallScope call(Entry::route_topk_permute, (long long)T * k);
+  return call(route_topk_permute_impl(logits, bias, T, E, k, x, K, topk_ids, topk_weights, offsets, sorted_to_flat,
+                                      flat_to_sorted, x_sorted, workspace, workspace_bytes, stream));
 }
 
 gnf4_status gnf4_grouped_gemm_nf4(const void* a, const uint8_t* w, const float* absmax, const int32_t* offsets,
                                   const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
-  return grouped_gemm(0, false, a, w, absmax, offsets, counts, E, N, K, M, y, stream);
+  CallScope call(Entry::grouped_gemm_nf4, (long long)M);
+  return call(grouped_gemm(0, false, a, w, absmax, offsets, counts, E, N, K, M, y, stream));
 }
 
 gnf4_status gnf4_grouped_gemm_mxfp4(const void* a, const uint8_t* w, const uint8_t* scales, const int32_t* offsets,
                                     const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
-  return grouped_gemm(1, false, a, w, scales, offsets, counts, E, N, K, M, y, stream);
+  CallScope call(Entry::grouped_gemm_mxfp4, (long long)M);
+  return call(grouped_gemm(1, false, a, w, scales, offsets, counts, E, N, K, M, y, stream));
 }
 
 size_t gnf4_grouped_gemm_mxfp4_workspace_bytes(int M, int K) {
@@ -667,21 +780,24 @@ int gnf4_grouped_gemm_mxfp4_native_max_rows(void) { return gemm_mx_rows_per_unit
 gnf4_status gnf4_grouped_gemm_mxfp4_ws(const void* a, const uint8_t* w, const uint8_t* scales,
                                        const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M,
                                        void* y, void* workspace, size_t workspace_bytes, void* stream) {
-  return grouped_gemm_mxfp4_ws(a, w, scales, offsets, counts, E, N, K, M, y, workspace, workspace_bytes, stream);
+  CallScope call(Entry::grouped_gemm_mxfp4_ws, (long long)M);
+  return call(grouped_gemm_mxfp4_ws(a, w, scales, offsets, counts, E, N, K, M, y, workspace, workspace_bytes, stream));
 }
 
 gnf4_status gnf4_grouped_gemv_nf4(const void* a, const uint8_t* w, const float* absmax, const int32_t* offsets,
                                   const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
-  return grouped_gemv(0, false, a, w, absmax, offsets, counts, E, N, K, M, y, stream);
+  CallScope call(Entry::grouped_gemv_nf4, (long long)M);
+  return call(grouped_gemv(0, false, a, w, absmax, offsets, counts, E, N, K, M, y, stream));
 }
 
 gnf4_status gnf4_grouped_gemv_mxfp4(const void* a, const uint8_t* w, const uint8_t* scales, const int32_t* offsets,
                                     const int32_t* counts, int E, int N, int K, int M, void* y, void* stream) {
-  return grouped_gemv(1, false, a, w, scales, offsets, counts, E, N, K, M, y, stream);
+  CallScope call(Entry::grouped_gemv_mxfp4, (long long)M);
+  return call(grouped_gemv(1, false, a, w, scales, offsets, counts, E, N, K, M, y, stream));
 }
 
-gnf4_status gnf4_combine(const void* y, const int32_t* flat_to_sorted, const float* weights, int T, int k, int N,
-                         void* out, void* stream) {
+static gnf4_status combine_impl(const void* y, const int32_t* flat_to_sorted, const float* weights, int T, int k, int N,
+                                void* out, void* stream) {
   if (T < 0 || k < 1) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T=%d / k=%d invalid", T, k);
   if (N < 8 || N % 8 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N=%d must be a positive multiple of 8", N);
   if (T == 0) return GNF4_OK;
@@ -694,7 +810,14 @@ gnf4_status gnf4_combine(const void* y, const int32_t* flat_to_sorted, const flo
   cudaError_t e = launch_combine(static_cast<const __nv_bfloat16*>(y), flat_to_sorted, weights, T, k, N,
                                  static_cast<__nv_bfloat16*>(out), d->num_sms, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  note_launch(kPathOther);
   return GNF4_OK;
+}
+
+gnf4_status gnf4_combine(const void* y, const int32_t* flat_to_sorted, const float* weights, int T, int k, int N,
+                         void* out, void* stream) {
+  CallScope call(Entry::combine, (long long)T * k);
+  return call(combine_impl(y, flat_to_sorted, weights, T, k, N, out, stream));
 }
 
 static gnf4_status dequant(int fmt, const uint8_t* w, const void* scales, int64_t rows, int K, float* out,
@@ -711,17 +834,20 @@ static gnf4_status dequant(int fmt, const uint8_t* w, const void* scales, int64_
   GNF4_TRY(device_state(&d));
   cudaError_t e = launch_dequant(fmt, w, scales, rows, K, out, d->num_sms, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
+  note_launch(kPathOther);
   return GNF4_OK;
 }
 
 gnf4_status gnf4_dequant_nf4_f32(const uint8_t* w, const float* absmax, int64_t rows, int K, float* out,
                                  void* stream) {
-  return dequant(0, w, absmax, rows, K, out, stream);
+  CallScope call(Entry::dequant_nf4_f32, (long long)rows);
+  return call(dequant(0, w, absmax, rows, K, out, stream));
 }
 
 gnf4_status gnf4_dequant_mxfp4_f32(const uint8_t* w, const uint8_t* scales, int64_t rows, int K, float* out,
                                    void* stream) {
-  return dequant(1, w, scales, rows, K, out, stream);
+  CallScope call(Entry::dequant_mxfp4_f32, (long long)rows);
+  return call(dequant(1, w, scales, rows, K, out, stream));
 }
 
 }  // extern "C"
@@ -730,19 +856,22 @@ extern "C" {
 
 gnf4_status gnf4_grouped_dgrad_nf4(const void* dy, const uint8_t* w, const float* absmax, const int32_t* offsets,
                                    const int32_t* counts, int E, int N, int K, int M, void* dx, void* stream) {
-  return grouped_dgrad(0, dy, w, absmax, offsets, counts, E, N, K, M, dx, stream);
+  CallScope call(Entry::grouped_dgrad_nf4, (long long)M);
+  return call(grouped_dgrad(0, dy, w, absmax, offsets, counts, E, N, K, M, dx, stream));
 }
 
 gnf4_status gnf4_grouped_dgrad_mxfp4(const void* dy, const uint8_t* w, const uint8_t* scales, const int32_t* offsets,
                                      const int32_t* counts, int E, int N, int K, int M, void* dx, void* stream) {
-  return grouped_dgrad(1, dy, w, scales, offsets, counts, E, N, K, M, dx, stream);
+  CallScope call(Entry::grouped_dgrad_mxfp4, (long long)M);
+  return call(grouped_dgrad(1, dy, w, scales, offsets, counts, E, N, K, M, dx, stream));
 }
 
 gnf4_status gnf4_grouped_gemm_nf4_swiglu(const void* a, const uint8_t* w_gate_up, const float* absmax,
                                          const int32_t* offsets, const int32_t* counts, int E, int I, int K, int M,
                                          void* h, void* stream) {
-  GNF4_TRY(check_swiglu_width(I));
-  return grouped_gemm(0, true, a, w_gate_up, absmax, offsets, counts, E, 2 * I, K, M, h, stream);
+  CallScope call(Entry::grouped_gemm_nf4_swiglu, (long long)M);
+  return call(grouped_swiglu(false, 0, a, w_gate_up, absmax, offsets, counts, E, I, K, M, h,
+                             stream));
 }
 
 size_t gnf4_combine_counters_bytes(int T, int N) {
@@ -755,8 +884,9 @@ gnf4_status gnf4_grouped_gemv_nf4_combine(const void* a, const uint8_t* w, const
                                           void* y, const int32_t* sorted_to_flat, const int32_t* flat_to_sorted,
                                           const float* weights, int T, int k, void* out, int32_t* counters,
                                           void* stream) {
-  return grouped_gemv_combine(0, a, w, absmax, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
-                              weights, T, k, out, counters, stream);
+  CallScope call(Entry::grouped_gemv_nf4_combine, (long long)M);
+  return call(grouped_gemv_combine(0, a, w, absmax, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
+                                   weights, T, k, out, counters, stream));
 }
 
 gnf4_status gnf4_grouped_gemv_mxfp4_combine(const void* a, const uint8_t* w, const uint8_t* scales,
@@ -764,8 +894,9 @@ gnf4_status gnf4_grouped_gemv_mxfp4_combine(const void* a, const uint8_t* w, con
                                             void* y, const int32_t* sorted_to_flat, const int32_t* flat_to_sorted,
                                             const float* weights, int T, int k, void* out, int32_t* counters,
                                             void* stream) {
-  return grouped_gemv_combine(1, a, w, scales, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
-                              weights, T, k, out, counters, stream);
+  CallScope call(Entry::grouped_gemv_mxfp4_combine, (long long)M);
+  return call(grouped_gemv_combine(1, a, w, scales, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
+                                   weights, T, k, out, counters, stream));
 }
 
 gnf4_status gnf4_grouped_gemm_nf4_combine(const void* a, const uint8_t* w, const float* absmax,
@@ -773,8 +904,9 @@ gnf4_status gnf4_grouped_gemm_nf4_combine(const void* a, const uint8_t* w, const
                                           void* y, const int32_t* sorted_to_flat, const int32_t* flat_to_sorted,
                                           const float* weights, int T, int k, void* out, int32_t* counters,
                                           void* stream) {
-  return grouped_gemm_combine(0, a, w, absmax, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
-                              weights, T, k, out, counters, stream);
+  CallScope call(Entry::grouped_gemm_nf4_combine, (long long)M);
+  return call(grouped_gemm_combine(0, a, w, absmax, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
+                                   weights, T, k, out, counters, stream));
 }
 
 gnf4_status gnf4_grouped_gemm_mxfp4_combine(const void* a, const uint8_t* w, const uint8_t* scales,
@@ -782,11 +914,12 @@ gnf4_status gnf4_grouped_gemm_mxfp4_combine(const void* a, const uint8_t* w, con
                                             void* y, const int32_t* sorted_to_flat, const int32_t* flat_to_sorted,
                                             const float* weights, int T, int k, void* out, int32_t* counters,
                                             void* stream) {
-  return grouped_gemm_combine(1, a, w, scales, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
-                              weights, T, k, out, counters, stream);
+  CallScope call(Entry::grouped_gemm_mxfp4_combine, (long long)M);
+  return call(grouped_gemm_combine(1, a, w, scales, offsets, counts, E, N, K, M, y, sorted_to_flat, flat_to_sorted,
+                                   weights, T, k, out, counters, stream));
 }
 
-gnf4_status gnf4_quantize_mxfp8(const void* x, int M, int K, uint8_t* codes, uint8_t* scales, void* stream) {
+static gnf4_status quantize_mxfp8_impl(const void* x, int M, int K, uint8_t* codes, uint8_t* scales, void* stream) {
   if (M < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d is negative", M);
   if (K < 32 || K % 32 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K=%d must be a positive multiple of 32", K);
   if (M == 0) return GNF4_OK;
@@ -798,16 +931,25 @@ gnf4_status gnf4_quantize_mxfp8(const void* x, int M, int K, uint8_t* codes, uin
   cudaError_t e = launch_quant_mxfp8(static_cast<const __nv_bfloat16*>(x), (long long)M * K, codes, scales, nullptr,
                                      nullptr, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "MXFP8 quantiser launch");
+  note_launch(kPathOther);
   return GNF4_OK;
+}
+
+gnf4_status gnf4_quantize_mxfp8(const void* x, int M, int K, uint8_t* codes, uint8_t* scales, void* stream) {
+  CallScope call(Entry::quantize_mxfp8, (long long)M);
+  return call(quantize_mxfp8_impl(x, M, K, codes, scales, stream));
 }
 
 gnf4_status gnf4_grouped_gemm_w4a8(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w,
                                    const uint8_t* w_scales, const int32_t* offsets, const int32_t* counts, int E,
                                    int N, int K, int M, void* y, void* stream) {
-  return grouped_gemm_w4a8(a_codes, a_scales, nullptr, nullptr, w, w_scales, offsets, counts, E, N, K, M, y, stream);
+  CallScope call(Entry::grouped_gemm_w4a8, (long long)M);
+  return call(
+      grouped_gemm_w4a8(a_codes, a_scales, nullptr, nullptr, w, w_scales, offsets, counts, E, N, K, M, y, stream));
 }
 
-gnf4_status gnf4_quantize_mxfp4_act(const void* x, int M, int K, uint8_t* blocks, uint8_t* scales, void* stream) {
+static gnf4_status quantize_mxfp4_act_impl(const void* x, int M, int K, uint8_t* blocks, uint8_t* scales,
+                                           void* stream) {
   if (M < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d is negative", M);
   if (K < 32 || K % 32 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K=%d must be a positive multiple of 32", K);
   if (M == 0) return GNF4_OK;
@@ -819,17 +961,24 @@ gnf4_status gnf4_quantize_mxfp4_act(const void* x, int M, int K, uint8_t* blocks
   cudaError_t e = launch_quant_mxfp4_act(static_cast<const __nv_bfloat16*>(x), (long long)M * K, blocks, scales,
                                          as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "MXFP4 activation quantiser launch");
+  note_launch(kPathOther);
   return GNF4_OK;
+}
+
+gnf4_status gnf4_quantize_mxfp4_act(const void* x, int M, int K, uint8_t* blocks, uint8_t* scales, void* stream) {
+  CallScope call(Entry::quantize_mxfp4_act, (long long)M);
+  return call(quantize_mxfp4_act_impl(x, M, K, blocks, scales, stream));
 }
 
 gnf4_status gnf4_grouped_gemm_w4a4(const uint8_t* a_blocks, const uint8_t* a_scales, const uint8_t* w,
                                    const uint8_t* w_scales, const int32_t* offsets, const int32_t* counts, int E,
                                    int N, int K, int M, void* y, void* stream) {
-  return grouped_gemm_w4a4(a_blocks, a_scales, w, w_scales, offsets, counts, E, N, K, M, y, stream);
+  CallScope call(Entry::grouped_gemm_w4a4, (long long)M);
+  return call(grouped_gemm_w4a4(a_blocks, a_scales, w, w_scales, offsets, counts, E, N, K, M, y, stream));
 }
 
-gnf4_status gnf4_quantize_mxfp8_split(const void* x, int M, int K, uint8_t* hi_codes, uint8_t* hi_scales,
-                                      uint8_t* lo_codes, uint8_t* lo_scales, void* stream) {
+static gnf4_status quantize_mxfp8_split_impl(const void* x, int M, int K, uint8_t* hi_codes, uint8_t* hi_scales,
+                                             uint8_t* lo_codes, uint8_t* lo_scales, void* stream) {
   if (M < 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "M=%d is negative", M);
   if (K < 32 || K % 32 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K=%d must be a positive multiple of 32", K);
   if (M == 0) return GNF4_OK;
@@ -843,37 +992,56 @@ gnf4_status gnf4_quantize_mxfp8_split(const void* x, int M, int K, uint8_t* hi_c
   cudaError_t e = launch_quant_mxfp8(static_cast<const __nv_bfloat16*>(x), (long long)M * K, hi_codes, hi_scales,
                                      lo_codes, lo_scales, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "MXFP8 split quantiser launch");
+  note_launch(kPathOther);
   return GNF4_OK;
+}
+
+gnf4_status gnf4_quantize_mxfp8_split(const void* x, int M, int K, uint8_t* hi_codes, uint8_t* hi_scales,
+                                      uint8_t* lo_codes, uint8_t* lo_scales, void* stream) {
+  CallScope call(Entry::quantize_mxfp8_split, (long long)M);
+  return call(quantize_mxfp8_split_impl(x, M, K, hi_codes, hi_scales, lo_codes, lo_scales, stream));
+}
+
+static gnf4_status grouped_gemm_w4a8x2_impl(const uint8_t* hi_codes, const uint8_t* hi_scales, const uint8_t* lo_codes,
+                                            const uint8_t* lo_scales, const uint8_t* w, const uint8_t* w_scales,
+                                            const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M,
+                                            void* y, void* stream) {
+  if (lo_codes == nullptr || lo_scales == nullptr) return fail(GNF4_ERR_INVALID_ARG, "lo_codes / lo_scales is NULL");
+  return grouped_gemm_w4a8(hi_codes, hi_scales, lo_codes, lo_scales, w, w_scales, offsets, counts, E, N, K, M, y,
+                           stream);
 }
 
 gnf4_status gnf4_grouped_gemm_w4a8x2(const uint8_t* hi_codes, const uint8_t* hi_scales, const uint8_t* lo_codes,
                                      const uint8_t* lo_scales, const uint8_t* w, const uint8_t* w_scales,
                                      const int32_t* offsets, const int32_t* counts, int E, int N, int K, int M,
                                      void* y, void* stream) {
-  if (lo_codes == nullptr || lo_scales == nullptr) return fail(GNF4_ERR_INVALID_ARG, "lo_codes / lo_scales is NULL");
-  return grouped_gemm_w4a8(hi_codes, hi_scales, lo_codes, lo_scales, w, w_scales, offsets, counts, E, N, K, M, y,
-                           stream);
+  CallScope call(Entry::grouped_gemm_w4a8x2, (long long)M);
+  return call(grouped_gemm_w4a8x2_impl(hi_codes, hi_scales, lo_codes, lo_scales, w, w_scales, offsets, counts, E, N, K,
+                                       M, y, stream));
 }
 
 gnf4_status gnf4_grouped_gemm_mxfp4_swiglu(const void* a, const uint8_t* w_gate_up, const uint8_t* scales,
                                            const int32_t* offsets, const int32_t* counts, int E, int I, int K, int M,
                                            void* h, void* stream) {
-  GNF4_TRY(check_swiglu_width(I));
-  return grouped_gemm(1, true, a, w_gate_up, scales, offsets, counts, E, 2 * I, K, M, h, stream);
+  CallScope call(Entry::grouped_gemm_mxfp4_swiglu, (long long)M);
+  return call(grouped_swiglu(false, 1, a, w_gate_up, scales, offsets, counts, E, I, K, M, h,
+                             stream));
 }
 
 gnf4_status gnf4_grouped_gemv_nf4_swiglu(const void* a, const uint8_t* w_gate_up, const float* absmax,
                                          const int32_t* offsets, const int32_t* counts, int E, int I, int K, int M,
                                          void* h, void* stream) {
-  GNF4_TRY(check_swiglu_width(I));
-  return grouped_gemv(0, true, a, w_gate_up, absmax, offsets, counts, E, 2 * I, K, M, h, stream);
+  CallScope call(Entry::grouped_gemv_nf4_swiglu, (long long)M);
+  return call(grouped_swiglu(true, 0, a, w_gate_up, absmax, offsets, counts, E, I, K, M, h,
+                             stream));
 }
 
 gnf4_status gnf4_grouped_gemv_mxfp4_swiglu(const void* a, const uint8_t* w_gate_up, const uint8_t* scales,
                                            const int32_t* offsets, const int32_t* counts, int E, int I, int K, int M,
                                            void* h, void* stream) {
-  GNF4_TRY(check_swiglu_width(I));
-  return grouped_gemv(1, true, a, w_gate_up, scales, offsets, counts, E, 2 * I, K, M, h, stream);
+  CallScope call(Entry::grouped_gemv_mxfp4_swiglu, (long long)M);
+  return call(grouped_swiglu(true, 1, a, w_gate_up, scales, offsets, counts, E, I, K, M, h,
+                             stream));
 }
 
 }  // extern "C"

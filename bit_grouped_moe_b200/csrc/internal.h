@@ -11,6 +11,8 @@
 #include <atomic>
 #include <utility>
 
+#include "gnf4.h"
+
 namespace gnf4 {
 
 // Launch with programmatic stream serialization: the kernel may be scheduled
@@ -159,6 +161,46 @@ cudaError_t launch_bounded_wait_probe(unsigned* err, long long limit_cycles, cud
 
 // api.cu: sets the text gnf4_last_error() returns on this thread
 void set_last_error(const char* msg);
+
+// api.cu: engagement counters, one record per entry point that enqueues work.
+#define GNF4_COUNTED_ENTRIES(X)                                                                              \
+  X(route_permute) X(route_permute_static) X(route_topk_permute) X(grouped_gemm_nf4) X(grouped_gemm_mxfp4) \
+  X(grouped_gemm_mxfp4_ws) X(grouped_gemv_nf4) X(grouped_gemv_mxfp4) X(grouped_dgrad_nf4)                \
+  X(grouped_dgrad_mxfp4) X(grouped_gemm_nf4_swiglu) X(grouped_gemm_mxfp4_swiglu)                          \
+  X(grouped_gemv_nf4_swiglu) X(grouped_gemv_mxfp4_swiglu) X(grouped_gemv_nf4_combine)                     \
+  X(grouped_gemv_mxfp4_combine) X(grouped_gemm_nf4_combine) X(grouped_gemm_mxfp4_combine)                 \
+  X(quantize_mxfp8) X(quantize_mxfp8_split) X(quantize_mxfp4_act) X(grouped_gemm_w4a8)                    \
+  X(grouped_gemm_w4a8x2) X(grouped_gemm_w4a4) X(combine) X(dequant_nf4_f32) X(dequant_mxfp4_f32)
+
+enum class Entry : int {
+#define GNF4_ENTRY_ENUM(n) n,
+  GNF4_COUNTED_ENTRIES(GNF4_ENTRY_ENUM)
+#undef GNF4_ENTRY_ENUM
+      count
+};
+
+// Kernel families a call can launch (the counters' *_path fields).
+enum : unsigned { kPathDecode = 1u, kPathNative = 2u, kPathGemv = 4u, kPathOther = 8u };
+
+// One counted call: the outermost scope on a thread records it when the
+// status passes through operator(); nested scopes (an entry point called by
+// another) record nothing of their own.
+class CallScope {
+ public:
+  CallScope(Entry e, long long rows);
+  ~CallScope();
+  gnf4_status operator()(gnf4_status s);
+  CallScope(const CallScope&) = delete;
+  CallScope& operator=(const CallScope&) = delete;
+
+ private:
+  Entry entry_;
+  long long rows_;
+  bool outer_;
+};
+
+// Marks that the current call enqueued work of the given family.
+void note_launch(unsigned path);
 
 // dequant.cu
 cudaError_t launch_dequant(int fmt, const uint8_t* w, const void* scales, int64_t rows, int K, float* out,

@@ -37,10 +37,10 @@ std::mutex g_scratch_mu;
 }  // namespace
 }  // namespace gnf4
 
-extern "C" gnf4_status gnf4_route_permute_static(const int32_t* topk_ids, const void* x, int T, int k, int E,
-                                                 int K, int32_t* offsets, int32_t* sorted_to_flat,
-                                                 int32_t* flat_to_sorted, void* x_sorted, int32_t* bad_id_count,
-                                                 void* stream) {
+static gnf4_status route_permute_static_impl(const int32_t* topk_ids, const void* x, int T, int k, int E,
+                                             int K, int32_t* offsets, int32_t* sorted_to_flat,
+                                             int32_t* flat_to_sorted, void* x_sorted, int32_t* bad_id_count,
+                                             void* stream) {
   using namespace gnf4;
   // the size check needs no device
   if (T >= 0 && k >= 1 && E >= 1) {
@@ -85,4 +85,13 @@ extern "C" gnf4_status gnf4_route_permute_static(const int32_t* topk_ids, const 
   // every word they later read.
   return gnf4_route_permute(topk_ids, x, T, k, E, K, offsets, sorted_to_flat, flat_to_sorted, x_sorted, scratch,
                             kStaticRouteScratchBytes, bad_id_count, stream);
+}
+
+extern "C" gnf4_status gnf4_route_permute_static(const int32_t* topk_ids, const void* x, int T, int k, int E,
+                                                 int K, int32_t* offsets, int32_t* sorted_to_flat,
+                                                 int32_t* flat_to_sorted, void* x_sorted, int32_t* bad_id_count,
+                                                 void* stream) {
+  gnf4::CallScope call(gnf4::Entry::route_permute_static, (long long)T * k);
+  return call(route_permute_static_impl(topk_ids, x, T, k, E, K, offsets, sorted_to_flat, flat_to_sorted, x_sorted,
+                                        bad_id_count, stream));
 }

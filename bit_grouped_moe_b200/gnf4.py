@@ -67,6 +67,10 @@ _lib.gnf4_grouped_gemm_mxfp4_native_max_rows.restype = _I
 _lib.gnf4_grouped_gemm_mxfp4_ws.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]
 _lib.gnf4_dequant_nf4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
 _lib.gnf4_dequant_mxfp4_f32.argtypes = [_P, _P, _I64, _I, _P, _P]
+_lib.gnf4_call_stats_get.argtypes = [ctypes.c_char_p, _P, _I]
+_lib.gnf4_call_stats_get.restype = _I
+_lib.gnf4_call_stats_name.argtypes = [_I]
+_lib.gnf4_call_stats_name.restype = ctypes.c_char_p
 for _name in ("gnf4_device_errors", "gnf4_route_permute", "gnf4_route_permute_static", "gnf4_route_topk_permute",
               *_GROUPED, "gnf4_combine", "gnf4_quantize_mxfp8", "gnf4_grouped_gemm_w4a8",
               "gnf4_quantize_mxfp8_split", "gnf4_grouped_gemm_w4a8x2",
@@ -128,6 +132,36 @@ def device_errors(clear: bool = True) -> int:
     v = ctypes.c_uint32(0)
     _check(_lib.gnf4_device_errors(ctypes.cast(ctypes.pointer(v), ctypes.c_void_p), int(clear)))
     return int(v.value)
+
+
+class CallStats(ctypes.Structure):
+    """gnf4_call_stats: one entry point's engagement counters."""
+    _fields_ = [(n, ctypes.c_uint64) for n in
+                ("calls", "refused", "engaged", "rows", "decode_path", "native_path", "gemv_path")]
+
+
+def call_stats_get(entry: str | None = None, reset: bool = False) -> dict:
+    """Engagement counters of the entry point `entry` (its C name, e.g.
+    "gnf4_grouped_gemm_mxfp4_ws"), or their sums over every counted entry
+    point when `entry` is None; `reset` zeroes what was read.  Host-side,
+    no device access."""
+    s = CallStats()
+    _check(_lib.gnf4_call_stats_get(None if entry is None else entry.encode(), ctypes.addressof(s), int(reset)))
+    return {n: int(getattr(s, n)) for n, _ in CallStats._fields_}
+
+
+def call_stats_name(i: int) -> str | None:
+    """C name of the i-th counted entry point, None past the last."""
+    n = _lib.gnf4_call_stats_name(i)
+    return None if n is None else n.decode()
+
+
+def call_stats_names() -> list[str]:
+    names, i = [], 0
+    while (n := call_stats_name(i)) is not None:
+        names.append(n)
+        i += 1
+    return names
 
 
 def route_workspace_bytes(T: int, k: int, E: int) -> int:

@@ -93,6 +93,50 @@ gnf4_status gnf4_device_errors(uint32_t *flags, int clear);
 gnf4_status gnf4_selftest_bounded_wait(unsigned long long limit_cycles, void *stream);
 
 /* ------------------------------------------------------------------ */
+/* Engagement counters                                                  */
+/* ------------------------------------------------------------------ */
+
+/* A returned status says that a call was accepted; these counters say
+ * whether it reached a kernel, and which kernel family ran (grouped-nf4-gemm
+ * releases, v0.2.6 "Honest instrumentation": a patch count is not a call
+ * count; status page, "What is open": a silent fallback made countable).
+ * One record per entry point that enqueues work, kept on the host,
+ * process-wide (all devices, all threads), updated with relaxed atomics;
+ * counting needs no device and no synchronisation.  A call that another
+ * entry point makes on the caller's behalf (gnf4_route_permute_static runs
+ * gnf4_route_permute) counts under the outer entry point only.
+ *
+ * Which kernels a call launches is decided on the host; which groups a
+ * launched kernel then finds work in is decided on the device from the
+ * offsets (gnf4_grouped_gemm_mxfp4_ws launches the native kernel for groups
+ * of at most gnf4_grouped_gemm_mxfp4_native_max_rows() rows and, when
+ * M exceeds that, the decode-path kernel for the larger ones). */
+typedef struct {
+    uint64_t calls;       /* times the entry point was called */
+    uint64_t refused;     /* calls that returned a status other than GNF4_OK */
+    uint64_t engaged;     /* calls that enqueued work (a kernel, or a memset) */
+    uint64_t rows;        /* summed over engaged calls: M for the grouped
+                             and quantiser calls, T*k for routing and the
+                             separate combine, weight rows for dequant */
+    uint64_t decode_path; /* engaged calls that launched a tensor-core kernel
+                             on decoded weights (kind::f16: GEMM, SwiGLU
+                             GEMM, fused-combine GEMM, dgrad) */
+    uint64_t native_path; /* engaged calls that launched the native
+                             block-scaled kernel (W4A8, two-term, W4A4) */
+    uint64_t gemv_path;   /* engaged calls that launched the decode GEMV */
+} gnf4_call_stats;
+
+/* Copies the counters of the entry point named `entry` (its C name, e.g.
+ * "gnf4_grouped_gemm_mxfp4_ws") into *out, or their sums over every entry
+ * point when `entry` is NULL; with `reset` != 0 those counters are then set
+ * to zero.  GNF4_ERR_INVALID_ARG for a NULL `out` or a name that is not
+ * counted (nothing is reset then). */
+gnf4_status gnf4_call_stats_get(const char *entry, gnf4_call_stats *out, int reset);
+
+/* Name of the i-th counted entry point (0-based), or NULL past the last. */
+const char *gnf4_call_stats_name(int i);
+
+/* ------------------------------------------------------------------ */
 /* Routing: sort (token, slot) pairs into per-expert row groups         */
 /* ------------------------------------------------------------------ */
 
