@@ -412,6 +412,19 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
+def engagement(g) -> dict:
+    """libgnf4's engagement counters for the entry points called since the
+    last reset: calls, calls that enqueued work, and how many reached each
+    kernel family (decode-path tcgen05, native block-scaled, GEMV).  Host-side
+    counters; reading them touches no device."""
+    out = {}
+    for name in g.call_stats_names():
+        st = g.call_stats_get(name)
+        if st["calls"]:
+            out[name[len("gnf4_"):]] = {k: v for k, v in st.items() if v or k == "calls"}
+    return out
+
+
 def max_over_ranks(value: float, world: int) -> float:
     if world <= 1:
         return value
@@ -678,6 +691,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
+    wl.g.call_stats_get(None, reset=True)  # count the timed steps' calls only
     t_wall0 = time.time()
     start.record(stream)
     for i in range(steps):
@@ -685,6 +699,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     stop.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
+    engaged = engagement(wl.g)
     barrier(world)
     time.sleep(0.2)
     sampler.stop()
@@ -933,8 +948,8 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
                     "steps": e2e_steps,
                     "copies": "overlapped with the neighbouring steps' kernels (copy streams, double buffers)"
                               if pipelined else "in stream order with the step's kernels"},
-            "gpu_launches": steps * wl.launches_per_step(), "clocks": clocks, "impl": "libgnf4",
-            **({"cuda_graph": graph} if graph is not None else {}),
+            "gpu_launches": steps * wl.launches_per_step(), "engagement": engaged, "clocks": clocks,
+            "impl": "libgnf4", **({"cuda_graph": graph} if graph is not None else {}),
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -51,3 +51,20 @@ def test_roofline_small_groups_are_hbm_bound():
     assert r["bound"] == "hbm"
     assert r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(r["algorithmic_bytes_per_launch"] / 0.423e-3 / 1e9, rel=1e-3)
+
+
+def test_engagement_lists_the_called_entry_points_only():
+    """The bench line's engagement object: one record per entry point called in the timed steps, zero fields
+    dropped except `calls`, read from the library's own host-side counters."""
+    import ctypes
+
+    from bit_grouped_moe_b200 import build
+    build.build()
+    from bit_grouped_moe_b200 import gnf4 as g
+    g.call_stats_get(None, reset=True)
+    assert bench.engagement(g) == {}
+    f = g._lib.gnf4_grouped_gemm_nf4
+    f(None, None, None, ctypes.c_void_p(16), None, 0, 64, 64, 8, None, None)  # refused: E = 0
+    f(None, None, None, ctypes.c_void_p(16), None, 4, 64, 64, 0, None, None)  # accepted, nothing to enqueue
+    assert bench.engagement(g) == {"grouped_gemm_nf4": {"calls": 2, "refused": 1}}
+    g.call_stats_get(None, reset=True)
