@@ -799,6 +799,7 @@ gnf4_status gnf4_grouped_gemv_mxfp4(const void* a, const uint8_t* w, const uint8
 static gnf4_status combine_impl(const void* y, const int32_t* flat_to_sorted, const float* weights, int T, int k, int N,
                                 void* out, void* stream) {
   if (T < 0 || k < 1) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T=%d / k=%d invalid", T, k);
+  if ((long long)T * k >= (1LL << 31)) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T*k too large");
   if (N < 8 || N % 8 != 0) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N=%d must be a positive multiple of 8", N);
   if (T == 0) return GNF4_OK;
   GNF4_TRY(check_ptr(y, "y", 16));

@@ -161,8 +161,8 @@ size_t gnf4_route_workspace_bytes(int T, int k, int E);
  *                  (grouped-nf4-gemm releases, v0.3.0 "Also": model-global
  *                  expert ids read out of bounds silently).
  * Within an expert, pairs keep ascending flat index (a stable sort).
- * Rules: T >= 0, 1 <= k <= E <= 4096, K % 8 == 0, x and x_sorted 16-byte
- * aligned.  T == 0 writes offsets only. */
+ * Rules: T >= 0, 1 <= k <= E <= 4096, T*k <= 2^30, K >= 8 and K % 8 == 0,
+ * x and x_sorted 16-byte aligned.  T == 0 writes offsets only. */
 gnf4_status gnf4_route_permute(const int32_t *topk_ids, const void *x, int T, int k, int E, int K,
                                int32_t *offsets, int32_t *sorted_to_flat, int32_t *flat_to_sorted,
                                void *x_sorted, void *workspace, size_t workspace_bytes,
@@ -212,8 +212,9 @@ gnf4_status gnf4_route_permute_static(const int32_t *topk_ids, const void *x, in
  *
  * logits: device fp32 [T, E] (4-byte aligned); bias: device fp32 [E] or
  * NULL; x: bf16 [T, K]; outputs as gnf4_route_permute plus topk_ids int32
- * [T, k] and topk_weights fp32 [T, k].  1 <= k <= min(E, 32), E <= 4096;
- * workspace as gnf4_route_workspace_bytes(T, k, E).  T*k <= 256 runs as one
+ * [T, k] and topk_weights fp32 [T, k].  1 <= k <= min(E, 32), E <= 4096,
+ * other shape rules as gnf4_route_permute; workspace as
+ * gnf4_route_workspace_bytes(T, k, E).  T*k <= 256 runs as one
  * launch.  The pages fix no tie rule or weight convention: this is a
  * reading. */
 gnf4_status gnf4_route_topk_permute(const float *logits, const float *bias, int T, int E, int k, const void *x, int K,
@@ -266,7 +267,8 @@ gnf4_status gnf4_grouped_gemm_mxfp4(const void *a, const uint8_t *w, const uint8
  * smaller non-NULL workspace is refused with GNF4_ERR_INVALID_ARG.  Its
  * contents are scratch: written and read within the call's stream order.
  * When K % 64 != 0 or K < 128 the native path does not apply: the workspace
- * size is 0 and every group takes the decode path.  With a workspace, w must
+ * size is 0 and every group takes the decode path; so does every group when
+ * E*N >= 2^31.  With a workspace, w must
  * be 32-byte aligned.  Up to three launches (split quantiser, native GEMM,
  * decode GEMM; the last is skipped when M <= 96), no host synchronisation. */
 size_t gnf4_grouped_gemm_mxfp4_workspace_bytes(int M, int K);
@@ -326,7 +328,7 @@ gnf4_status gnf4_grouped_dgrad_mxfp4(const void *dy, const uint8_t *w, const uin
  * [M, 2I] projection output never reaches global memory.
  *
  * Arguments as the grouped GEMM / GEMV calls, with I (the output width) in
- * place of N: I must be a positive multiple of 64.  The GEMV forms keep the
+ * place of N: I must be a positive multiple of 64, at most 2^29.  The GEMV forms keep the
  * rule of at most 8 rows per group (larger groups are skipped and flagged
  * with GNF4_DEVERR_GEMV_ROWS). */
 gnf4_status gnf4_grouped_gemm_nf4_swiglu(const void *a, const uint8_t *w_gate_up, const float *absmax,
@@ -382,7 +384,8 @@ gnf4_status gnf4_grouped_gemv_mxfp4_combine(const void *a, const uint8_t *w, con
  * per group) with the same top-k combine after each work unit's epilogue
  * (grouped-nf4-gemm releases, v0.2.5 "arena -> kernel": moe_layer_forward
  * runs gate -> GLU -> down, then the weighted unsort).  Results, arguments
- * and counter rules exactly as gnf4_grouped_gemv_*_combine, with the shape
+ * and counter rules exactly as gnf4_grouped_gemv_*_combine (T >= 0, k >= 1,
+ * T*k < 2^31 for both), with the shape
  * rules of gnf4_grouped_gemm_*: out equals gnf4_grouped_gemm_* followed by
  * gnf4_combine bit for bit.  y is still written (the combine reads the
  * token's other rows from it through L2).  Each unit's combine runs after
@@ -419,8 +422,8 @@ gnf4_status gnf4_grouped_gemm_mxfp4_combine(const void *a, const uint8_t *w, con
  *            saturating at +-448, sign kept on zero results
  * (OCP MX v1.0 MXFP8; the pages give no rule, this is the reading used).
  * Bit-exact: the same inputs give the same bytes on every run.  K must be a
- * positive multiple of 32; inputs must be finite.  x, codes: 16-byte
- * aligned device memory; scales: device memory.
+ * positive multiple of 32 and M >= 0 (M == 0 does nothing); inputs must be
+ * finite.  x, codes: 16-byte aligned device memory; scales: device memory.
  *
  * gnf4_grouped_gemm_w4a8: for every sorted row r of expert e
  *     y[r, n] = sum_k A[r, k] * W_e[n, k],
@@ -429,8 +432,8 @@ gnf4_status gnf4_grouped_gemm_mxfp4_combine(const void *a, const uint8_t *w, con
  * products exact, fp32 accumulation, bf16 output y [M, N].  w, w_scales,
  * offsets, counts, E, N and M as the MXFP4 grouped GEMM; a_codes / a_scales
  * as written by gnf4_quantize_mxfp8 for the group-sorted rows.  K must be a
- * multiple of 64 in [128, 65536].  Alignment: a_codes 16 bytes, w 32 bytes,
- * y 16 bytes.  Rows past offsets[E] are not written. */
+ * multiple of 64 in [128, 65536], and E*N < 2^31.  Alignment: a_codes
+ * 16 bytes, w 32 bytes, y 16 bytes.  Rows past offsets[E] are not written. */
 gnf4_status gnf4_quantize_mxfp8(const void *x, int M, int K, uint8_t *codes, uint8_t *scales, void *stream);
 
 /* Two-term form (the activations as hi + lo, two MXFP8 tensors), which
@@ -491,7 +494,8 @@ gnf4_status gnf4_grouped_gemm_w4a4(const uint8_t *a_blocks, const uint8_t *a_sca
  * flat_to_sorted is -1 (or not below T*k) contribute nothing.
  *   y bf16 [T*k, N] (group-sorted expert outputs); flat_to_sorted int32 [T*k];
  *   weights fp32 [T, k]; out bf16 [T, N] OUT.
- * Rules: T >= 0, k >= 1, N % 8 == 0, y and out 16-byte aligned. */
+ * Rules: T >= 0, k >= 1, T*k < 2^31, N >= 8 and N % 8 == 0, y and out
+ * 16-byte aligned. */
 gnf4_status gnf4_combine(const void *y, const int32_t *flat_to_sorted, const float *weights, int T, int k, int N,
                          void *out, void *stream);
 
@@ -502,12 +506,13 @@ gnf4_status gnf4_combine(const void *y, const int32_t *flat_to_sorted, const flo
 /* fp32 decode of `rows` packed rows of K elements: out[r, k] = NF4[code] *
  * absmax[r, k/64] (one fp32 multiply, round to nearest, no flush to zero).
  * This is the reference decode the pages call dequant_ref (grouped-nf4-gemm
- * 0.33.1 on PyPI, example 1).  Rules: K % 64 == 0, rows >= 0. */
+ * 0.33.1 on PyPI, example 1).  Rules: K >= 64 and K % 64 == 0, rows >= 0. */
 gnf4_status gnf4_dequant_nf4_f32(const uint8_t *w, const float *absmax, int64_t rows, int K, float *out,
                                  void *stream);
 
 /* fp32 decode of MXFP4 rows: out[r, k] = e2m1[code] * 2^(scale-127), with
- * scale 255 decoding to NaN (same page, example 2).  Rules: K % 32 == 0. */
+ * scale 255 decoding to NaN (same page, example 2).  Rules: K >= 32 and
+ * K % 32 == 0, rows >= 0. */
 gnf4_status gnf4_dequant_mxfp4_f32(const uint8_t *w, const uint8_t *scales, int64_t rows, int K, float *out,
                                    void *stream);
 
