@@ -88,16 +88,34 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, uuid: str | None = None):
         self.index = index
+        self.uuid = uuid
         self.samples = []
         self.proc = None
         self.thread = None
+        self.ident = None
+
+    def gpu_id(self) -> str:
+        """The GPU for nvidia-smi: by UUID, which names the device this process
+        computes on whatever CUDA_VISIBLE_DEVICES remaps; by index when
+        nvidia-smi does not know that UUID."""
+        if self.uuid:
+            ident = self.uuid if self.uuid.startswith("GPU-") else "GPU-" + self.uuid
+            try:
+                r = subprocess.run(["nvidia-smi", "-i", ident, "--query-gpu=uuid", "--format=csv,noheader"],
+                                   capture_output=True, text=True, timeout=20)
+                if r.returncode == 0 and r.stdout.strip():
+                    return ident
+            except (OSError, subprocess.TimeoutExpired):
+                pass
+        return str(self.index)
 
     def start(self):
+        self.ident = self.gpu_id()
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", "-i", self.ident, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -138,7 +156,18 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(mhz)}
+                "reasons": sorted(reasons), "samples": len(mhz), "gpu": self.ident}
+
+
+def gpu_uuid(local: int) -> str | None:
+    """UUID of the CUDA device `local` as torch sees it (None if unavailable)."""
+    try:
+        import torch
+
+        u = getattr(torch.cuda.get_device_properties(local), "uuid", None)
+        return str(u) if u else None
+    except Exception:  # noqa: BLE001 -- clocks then fall back to the index
+        return None
 
 
 # ------------------------------------------------------------------ workload
@@ -686,7 +715,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     # timed region (inputs resident): K whole steps, no event inside it, so
     # consecutive launches keep their programmatic overlap
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(local, gpu_uuid(local))
     sampler.start()
     time.sleep(0.3)
     barrier(world)
@@ -713,7 +742,7 @@ def run_gpu(args, steps, warmup, world, rank, local, decode):
     # is), routing of batch 0
     wl.step(0)
     torch.cuda.synchronize()
-    dsampler = ClockSampler(local)
+    dsampler = ClockSampler(local, gpu_uuid(local))
     dsampler.start()
     time.sleep(0.3)
     dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

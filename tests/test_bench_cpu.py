@@ -68,3 +68,31 @@ def test_engagement_lists_the_called_entry_points_only():
     f(None, None, None, ctypes.c_void_p(16), None, 4, 64, 64, 0, None, None)  # accepted, nothing to enqueue
     assert bench.engagement(g) == {"grouped_gemm_nf4": {"calls": 2, "refused": 1}}
     g.call_stats_get(None, reset=True)
+
+
+def test_clock_sampler_names_the_gpu_by_uuid_and_falls_back_to_the_index(monkeypatch):
+    """nvidia-smi numbers GPUs physically, CUDA after CUDA_VISIBLE_DEVICES: the sampler asks for the device's
+    UUID, and takes the index only when nvidia-smi does not know that UUID (or is missing)."""
+    import subprocess
+    import types as _t
+
+    seen = []
+
+    def fake_run(cmd, **kw):
+        seen.append(cmd)
+        ok = cmd[2] == "GPU-1234-abcd"
+        return _t.SimpleNamespace(returncode=0 if ok else 6, stdout="GPU-1234-abcd\n" if ok else "")
+
+    monkeypatch.setattr(subprocess, "run", fake_run)
+    assert bench.ClockSampler(3, "1234-abcd").gpu_id() == "GPU-1234-abcd"
+    assert bench.ClockSampler(3, "GPU-1234-abcd").gpu_id() == "GPU-1234-abcd"
+    assert bench.ClockSampler(3, "ffff").gpu_id() == "3"
+    assert bench.ClockSampler(5, None).gpu_id() == "5"
+
+    def missing(cmd, **kw):
+        raise FileNotFoundError("nvidia-smi")
+
+    monkeypatch.setattr(subprocess, "run", missing)
+    assert bench.ClockSampler(2, "1234-abcd").gpu_id() == "2"
+    s = bench.ClockSampler(0)
+    assert s.summary(0.0, 1.0) == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "gpu": None}
