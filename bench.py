@@ -297,10 +297,9 @@ class Workload:
                 w, s = inputs.nf4_direct(rng, E, p.N, p.K)
             else:
                 w, s = inputs.mxfp4_random(rng, E, p.N, p.K)
-            if keep_host:
-                if self.host_stacks is None:
-                    self.host_stacks = []
-                self.host_stacks.append((w, s))
+            if self.host_stacks is None:
+                self.host_stacks = []
+            self.host_stacks.append((w, s))
             return torch.from_numpy(w).to(self.dev), torch.from_numpy(s).to(self.dev)
         w = inputs.device_random_bytes(seed, (E, p.N, p.K // 2), device=self.dev)
         if fmt == "nf4":
