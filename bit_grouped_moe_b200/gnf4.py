@@ -307,44 +307,7 @@ def dequant_mxfp4_f32(w, scales, out, stream=None):
     _check(_lib.gnf4_dequant_mxfp4_f32(_ptr(w), _ptr(scales), rows, K, _ptr(out), _stream(stream)))
 
 
-# ---------------------------------------------------------------- convenience
-
-
-def moe_step(fmt, x, topk_ids, weights, w1, s1, w2, s2, h=None, ws=None, stream=None, decode=None):
-    """One pass of the path: route -> GEMM (proj 1) -> GEMM (proj 2) -> combine.
-
-    The activation between the two projections is not part of the path (no
-    GLU here): ``h`` [T*k, K2] bf16 is the second projection's input; if None,
-    the first projection's output columns [:K2] are used.  ``decode`` forces
-    the GEMV (True) or the tiled GEMM (False); by default the GEMV is used when
-    T <= 8 (at most 8 rows per group, host-known with no sync).
-    Returns (out [T, N2] bf16, offsets).
-    """
-    T, k = topk_ids.shape
-    E = w1.shape[0]
-    K1 = x.shape[1]
-    M = T * k
-    dev = x.device
-    N1 = w1.shape[1]
-    N2, K2 = w2.shape[1], w2.shape[2] * 2
-    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    s2f = torch.empty(M, dtype=torch.int32, device=dev)
-    f2s = torch.empty(M, dtype=torch.int32, device=dev)
-    xs = torch.empty(M, K1, dtype=torch.bfloat16, device=dev)
-    if ws is None:
-        ws = torch.empty(max(route_workspace_bytes(T, k, E), 16), dtype=torch.uint8, device=dev)
-    route_permute(topk_ids, x, E, offsets, s2f, f2s, xs, ws, stream=stream)
-    use_gemv = (T <= MAX_GEMV_ROWS) if decode is None else decode
-    y1 = torch.empty(M, N1, dtype=torch.bfloat16, device=dev)
-    fn1 = {("nf4", True): grouped_gemv_nf4, ("nf4", False): grouped_gemm_nf4,
-           ("mxfp4", True): grouped_gemv_mxfp4, ("mxfp4", False): grouped_gemm_mxfp4}[(fmt, use_gemv)]
-    fn1(xs, w1, s1, y1, offsets=offsets, stream=stream)
-    a2 = h if h is not None else y1[:, :K2].contiguous()
-    y2 = torch.empty(M, N2, dtype=torch.bfloat16, device=dev)
-    fn1(a2, w2, s2, y2, offsets=offsets, stream=stream)
-    out = torch.empty(T, N2, dtype=torch.bfloat16, device=dev)
-    combine(y2, f2s, weights, out, stream=stream)
-    return out, offsets
+# ---------------------------------------------------------------- native MX modes
 
 
 def quantize_mxfp8(x, codes, scales, stream=None):
