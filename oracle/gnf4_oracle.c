@@ -45,6 +45,13 @@
  *
  * Points the pages leave open are taken as numbered readings (C1, C2, ...);
  * each function below names the ones it depends on.
+ *
+ * PARITY UNPINNED: the NF4 nibble order (reading C2: element 2i in the high
+ * nibble, the bitsandbytes convention) has no pin outside this project.  The
+ * pages print no packed NF4 bytes and no library that packs NF4 is installed,
+ * so only the hand-worked byte examples of the test suite fix the reading.
+ * Every other function here has an external pin (closed forms, library
+ * routines, brute force or the pages' printed figures).
  */
 #include <math.h>
 #include <stdint.h>
