@@ -1,7 +1,8 @@
 """CPU oracle for the grouped 4-bit MoE expert GEMM -- TEST INFRASTRUCTURE.
 
-Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may import this package.  The product path (the CUDA library and
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU legs of
+``bench.py`` (its CPU baseline and its ``--impl reference`` arm) may import
+this package.  The product path (the CUDA library and
 its Python binding) never imports it and shares no code with it.
 
 The arithmetic lives in ``gnf4_oracle.c`` (plain C, fp64 sums, fp32 decode).

@@ -3,8 +3,9 @@
  *
  * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, obviously
  * correct statement of what the GPU library computes.  Only the test suite,
- * the smoke check and the benchmark's CPU-baseline leg may load it.  It
- * shares no code, header, table or constant generator with the CUDA path.
+ * the smoke check and the benchmark's CPU legs (its CPU baseline and its
+ * reference arm) may load it.  It shares no code, header, table or constant
+ * generator with the CUDA path.
  *
  * Precision: quantise / dequantise in fp32 exactly as the formats define
  * them; every sum (GEMM, combine) is accumulated in fp64.
