@@ -17,12 +17,15 @@ from bit_grouped_moe_b200 import build
 ONE = ctypes.c_void_p(16)  # a non-NULL group description; never dereferenced on the host
 SHAPE = 2
 SETTINGS = settings(max_examples=150, deadline=None, derandomize=True)
+_G = None  # the binding, set by the fixture (refused() reads its last_error)
 
 
 @pytest.fixture(scope="module")
 def g():
+    global _G
     build.build()
     from bit_grouped_moe_b200 import gnf4
+    _G = gnf4
     return gnf4
 
 
@@ -44,6 +47,11 @@ def grouped_ok(kq, E, N, K, M):
 
 
 def refused(status):
+    """True for GNF4_ERR_UNSUPPORTED_SHAPE, which must come with a message naming what was wrong."""
+    if status == SHAPE and _G is not None:
+        msg = _G.last_error()
+        assert msg and any(w in msg for w in ("E=", "N=", "K=", "M=", "I=", "T=", "k=", "rows=", "too large", "T*k",
+                                              "E*N")), msg
     return status == SHAPE
 
 
