@@ -6,6 +6,13 @@ NF4 weights for parity tests are made by passing ``normal_weights`` through
 the oracle's quantiser; the bench draws NF4 codes and block absmax values
 directly (``nf4_direct``) so that the product path never runs oracle code.
 
+The synthetic routing (``route_topk``) draws router logits and keeps each
+token's k largest, which defines the workloads' expert-load distribution
+(N(0,1) logits, optionally with a Zipf rank bias).  Its ids and weights are
+inputs to the routing and combine steps on both sides alike.  The library's
+router epilogue is never compared against it: its parity tests draw logits
+here and compare the kernel with the oracle's own top-k.
+
 Workload shapes follow the pages' models (OLMoE-1B-7B, Qwen3-30B-A3B,
 gpt-oss-120b, a Kimi-class MoE); see ``WORKLOADS``.
 """
