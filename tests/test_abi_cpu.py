@@ -246,3 +246,14 @@ def test_swiglu_width_refusals_and_empty_call(g, name):
     for width in (0, 32, 96, -64):
         assert f(None, None, None, off, None, 4, width, 64, 8, None, None) == g.ERR_UNSUPPORTED_SHAPE, width
     assert f(None, None, None, off, None, 4, 64, 64, 0, None, None) == g.OK  # M == 0 launches nothing
+
+
+def test_library_needs_no_torch_or_python(lib_path):
+    """The boundary is plain C over a self-contained library: libgnf4.so links the C/C++ runtime only (the CUDA
+    runtime is static), never torch, c10 or libpython."""
+    out = subprocess.run(["readelf", "-d", lib_path], capture_output=True, text=True).stdout
+    needed = re.findall(r"\(NEEDED\)\s+Shared library: \[([^\]]+)\]", out)
+    assert needed
+    allowed = ("libstdc++", "libgcc_s", "libc.", "libm.", "ld-linux", "libdl", "librt", "libpthread")
+    extra = [n for n in needed if not n.startswith(allowed)]
+    assert not extra, extra
